@@ -1,0 +1,294 @@
+"""CPU oracle for the packed-INT4 ConvRot quantized linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+module.  The product library never imports, links or calls it, and it never
+imports the product: the two share no code.
+
+The arithmetic lives in ``tint4_oracle.c`` (plain C, OpenMP over rows); this
+module only compiles it on first use and marshals numpy arrays through ctypes.
+Every function states which page passage it restates; the C file's header
+lists the readings taken where the pages are silent.
+
+Parity status: every function here is pinned by a ``-m "not gpu"`` test to
+something other than itself (closed forms, invariants, brute force, worked
+examples derived by hand in ``tests/golden/``).  None is pinned to a number
+printed by the pages, because the pages print no tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "tint4_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle into ``oracle/liboracle.so`` (gcc, OpenMP)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+           "-ffp-contract=off", "-fno-fast-math", "-Wall", "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        L = ctypes.c_long
+        sig = {
+            "oracle_hadamard": [I, P],
+            "oracle_fwht_f32": [P, I],
+            "oracle_rotate_rows_f32": [P, L, I, I],
+            "oracle_pack_int4": [P, L, I, P],
+            "oracle_unpack_int4": [P, L, I, P],
+            "oracle_pack_weights": [P, I, I, I, P, P, P],
+            "oracle_quantize_act": [P, I, I, I, I, P, P, P],
+            "oracle_gemm_i32": [P, P, I, I, I, P],
+            "oracle_gemm_i32_sampled": [P, P, I, P, L, P],
+            "oracle_epilogue": [P, P, P, P, I, I, P],
+            "oracle_epilogue_sampled": [P, P, P, P, P, L, P],
+            "oracle_convrot_linear": [P, P, P, P, I, I, I, I, I, P],
+            "oracle_w4a16": [P, P, P, P, I, I, I, I, P],
+            "oracle_num_threads": [],
+        }
+        for name, args in sig.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = I
+        lib.oracle_double_to_bf16.argtypes = [ctypes.c_double]
+        lib.oracle_double_to_bf16.restype = ctypes.c_uint16
+        _lib = lib
+        return lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _check(rc, name):
+    if rc != 0:
+        raise ValueError(f"{name}: oracle rejected its arguments (rc={rc})")
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle uses."""
+    return int(_load().oracle_num_threads())
+
+
+# --------------------------------------------------------------------------
+# bf16 helpers (the oracle's own; inputs arrive as raw bf16 bits, uint16)
+# --------------------------------------------------------------------------
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> float32 values, exactly."""
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def double_to_bf16_bits(v: float) -> int:
+    """Round one double to the nearest bf16 (ties to even), return its bits."""
+    return int(_load().oracle_double_to_bf16(float(v)))
+
+
+# --------------------------------------------------------------------------
+# Rotation
+# --------------------------------------------------------------------------
+
+def hadamard(g: int) -> np.ndarray:
+    """Orthonormal Sylvester Hadamard matrix H_g (fp64, g x g), natural order.
+
+    The matrix behind the rotation the pages call Hadamard / QuaRot / ConvRot
+    ("ComfyUI-INT-Crush", "Inference > INT4 > CUDA backend"; "TINT4 v1.2",
+    "参数选择指南" enable_quarot)."""
+    H = np.empty((g, g), dtype=np.float64)
+    _check(_load().oracle_hadamard(g, _ptr(H)), "hadamard")
+    return H
+
+
+def fwht_f32(v: np.ndarray) -> np.ndarray:
+    """Orthonormal fast Walsh-Hadamard transform of one fp32 block (copy)."""
+    out = _c(v, np.float32).copy()
+    _check(_load().oracle_fwht_f32(_ptr(out), out.size), "fwht_f32")
+    return out
+
+
+def rotate_rows_f32(rows: np.ndarray, g: int) -> np.ndarray:
+    """Rotate every length-g block along the last axis (fp32, copy).
+
+    "ComfyUI-INT-Crush", "Forward Pass" step 2 (rotate activations with the
+    layer's rot_size); the same block rotation is applied to W offline."""
+    out = _c(rows, np.float32).copy()
+    K = out.shape[-1]
+    n = out.size // K
+    _check(_load().oracle_rotate_rows_f32(_ptr(out), n, K, g), "rotate_rows_f32")
+    return out
+
+
+# --------------------------------------------------------------------------
+# Packing
+# --------------------------------------------------------------------------
+
+def pack_int4(codes: np.ndarray) -> np.ndarray:
+    """int8 codes [R, K] -> uint8 [R, K/2], code 2j in the low nibble of byte j.
+
+    "ComfyUI-INT-Crush", "Weight Format" (uint8, 2 per byte)."""
+    q = _c(codes, np.int8)
+    R, K = q.shape
+    out = np.empty((R, K // 2), dtype=np.uint8)
+    _check(_load().oracle_pack_int4(_ptr(q), R, K, _ptr(out)), "pack_int4")
+    return out
+
+
+def unpack_int4(packed: np.ndarray) -> np.ndarray:
+    """uint8 [R, K/2] -> int8 codes [R, K] (two's complement nibbles)."""
+    p = _c(packed, np.uint8)
+    R, Kh = p.shape
+    out = np.empty((R, 2 * Kh), dtype=np.int8)
+    _check(_load().oracle_unpack_int4(_ptr(p), R, 2 * Kh, _ptr(out)), "unpack_int4")
+    return out
+
+
+# --------------------------------------------------------------------------
+# Quantization
+# --------------------------------------------------------------------------
+
+def pack_weights(W: np.ndarray, g: int):
+    """Twin of ``tint4_pack_weights``: rotate W along K, per-row symmetric int4.
+
+    Returns (packed uint8 [N, K/2], row_scale fp32 [N], codes int8 [N, K]).
+    "ComfyUI-INT-Crush", "Weight Format"; "feat: packed int4 convrot model
+    loading and dispatch", "Summary" (packed nibbles + row scales)."""
+    Wc = _c(W, np.float32)
+    N, K = Wc.shape
+    packed = np.empty((N, K // 2), dtype=np.uint8)
+    scale = np.empty(N, dtype=np.float32)
+    codes = np.empty((N, K), dtype=np.int8)
+    _check(_load().oracle_pack_weights(_ptr(Wc), N, K, g, _ptr(packed), _ptr(scale),
+                                       _ptr(codes)), "pack_weights")
+    return packed, scale, codes
+
+
+def quantize_act(x_bits: np.ndarray, g: int, bits: int):
+    """Twin of ``convrot_quantize_act``: rotate x then per-token symmetric codes.
+
+    x_bits: bf16 bit patterns uint16 [M, K].  Returns (codes int8 [M, K],
+    tok_scale fp32 [M], packed uint8 [M, K/2] or None for bits == 8).
+    "ComfyUI-INT-Crush", "Inference > INT4 > Triton backend" (dynamic
+    activation quantization) and "Forward Pass" steps 2 and 5."""
+    x = _c(x_bits, np.uint16)
+    M, K = x.shape
+    codes = np.empty((M, K), dtype=np.int8)
+    scale = np.empty(M, dtype=np.float32)
+    packed = np.empty((M, K // 2), dtype=np.uint8) if bits == 4 else None
+    _check(_load().oracle_quantize_act(_ptr(x), M, K, g, bits, _ptr(codes), _ptr(scale),
+                                       _ptr(packed)), "quantize_act")
+    return codes, scale, packed
+
+
+# --------------------------------------------------------------------------
+# GEMM, epilogue, whole layer
+# --------------------------------------------------------------------------
+
+def gemm_i32(a: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """acc[m, n] = sum_k a[m, k] w[n, k] (exact int32).
+
+    "ComfyUI-INT-Crush", "Inference > INT4 > CUDA backend" (INT8 GEMM)."""
+    ac, wc = _c(a, np.int8), _c(w, np.int8)
+    M, K = ac.shape
+    N = wc.shape[0]
+    out = np.empty((M, N), dtype=np.int32)
+    _check(_load().oracle_gemm_i32(_ptr(ac), _ptr(wc), M, N, K, _ptr(out)), "gemm_i32")
+    return out
+
+
+def gemm_i32_sampled(a: np.ndarray, w: np.ndarray, pairs: np.ndarray) -> np.ndarray:
+    """The same sums for selected (m, n) pairs only (pairs int64 [P, 2])."""
+    ac, wc = _c(a, np.int8), _c(w, np.int8)
+    pr = _c(pairs, np.int64)
+    out = np.empty(pr.shape[0], dtype=np.int32)
+    _check(_load().oracle_gemm_i32_sampled(_ptr(ac), _ptr(wc), ac.shape[1], _ptr(pr),
+                                           pr.shape[0], _ptr(out)), "gemm_i32_sampled")
+    return out
+
+
+def epilogue(acc, tok_scale, row_scale, bias_bits=None) -> np.ndarray:
+    """y = bf16(acc * s_tok * s_row (+ bias)) in fp64; returns bf16 bits.
+
+    "ComfyUI-INT-Crush", "Inference > INT4 > CUDA backend" (fused dequant)."""
+    A = _c(acc, np.int32)
+    M, N = A.shape
+    st, sr = _c(tok_scale, np.float32), _c(row_scale, np.float32)
+    b = None if bias_bits is None else _c(bias_bits, np.uint16)
+    y = np.empty((M, N), dtype=np.uint16)
+    _check(_load().oracle_epilogue(_ptr(A), _ptr(st), _ptr(sr), _ptr(b), M, N, _ptr(y)),
+           "epilogue")
+    return y
+
+
+def epilogue_sampled(acc, tok_scale, row_scale, pairs, bias_bits=None) -> np.ndarray:
+    """Epilogue for selected (m, n) pairs; acc holds their sums in pair order."""
+    A = _c(acc, np.int32)
+    st, sr = _c(tok_scale, np.float32), _c(row_scale, np.float32)
+    pr = _c(pairs, np.int64)
+    b = None if bias_bits is None else _c(bias_bits, np.uint16)
+    y = np.empty(pr.shape[0], dtype=np.uint16)
+    _check(_load().oracle_epilogue_sampled(_ptr(A), _ptr(st), _ptr(sr), _ptr(b), _ptr(pr),
+                                           pr.shape[0], _ptr(y)), "epilogue_sampled")
+    return y
+
+
+def convrot_linear(x_bits, w_packed, row_scale, g, act_bits, bias_bits=None) -> np.ndarray:
+    """Twin of ``convrot_w4a8_linear`` (act_bits 8) / ``convrot_w4a4_linear`` (4).
+
+    Rotate + quantize x, unpack W, int32 GEMM, fused dequant; bf16 bits out.
+    "ComfyUI-INT-Crush", "Inference > INT4 > CUDA backend" (fused ConvRot path)."""
+    x = _c(x_bits, np.uint16)
+    wp = _c(w_packed, np.uint8)
+    sr = _c(row_scale, np.float32)
+    b = None if bias_bits is None else _c(bias_bits, np.uint16)
+    M, K = x.shape
+    N = wp.shape[0]
+    y = np.empty((M, N), dtype=np.uint16)
+    _check(_load().oracle_convrot_linear(_ptr(x), _ptr(wp), _ptr(sr), _ptr(b), M, N, K, g,
+                                         act_bits, _ptr(y)), "convrot_linear")
+    return y
+
+
+def w4a16(x_bits, q_packed, scale_bits, zero, group) -> np.ndarray:
+    """Twin of ``w4a16_gemv_gemm``: y = x . ((q - z) * s)^T, fp64 accumulation.
+
+    "TINT4 v1.2", "v1.1 新特性 > 5" (_qdata/_scale/_zp) and "参数选择指南"
+    (group_size 128 standard); "ComfyUI-INT-Crush", "Inference > INT4 >
+    Triton backend" (W4A16 when rot_size == 0)."""
+    x = _c(x_bits, np.uint16)
+    q = _c(q_packed, np.uint8)
+    s = _c(scale_bits, np.uint16)
+    z = _c(zero, np.uint8)
+    M, K = x.shape
+    N = q.shape[0]
+    y = np.empty((M, N), dtype=np.uint16)
+    _check(_load().oracle_w4a16(_ptr(x), _ptr(q), _ptr(s), _ptr(z), M, N, K, group, _ptr(y)),
+           "w4a16")
+    return y

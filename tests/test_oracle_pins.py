@@ -1,0 +1,395 @@
+"""Pins of the CPU oracle to things other than itself (CPU only).
+
+Each test ties one oracle function to a closed form, an invariant, a brute
+force computation or a worked example derived by hand (tests/golden/), so that
+a plausible mistake in the oracle -- a dropped term, a wrong sign or index, a
+transposed operand, a wrong nibble order or rounding mode -- fails here before
+the oracle is trusted as the reference of the CUDA path.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+from int4_weight_quantized_block_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+GROUPS = (16, 64, 256)
+
+
+def golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def bits(x):
+    return inputs.f32_to_bf16_bits(np.asarray(x, dtype=np.float32))
+
+
+# ---------------------------------------------------------------- Hadamard
+
+@pytest.mark.parametrize("g", GROUPS + (4, 1024))
+def test_hadamard_orthonormal_exact(g):
+    """H H^T = I exactly: entries are +-2^-k, so every product sum is exact."""
+    H = oracle.hadamard(g)
+    assert np.array_equal(H @ H.T, np.eye(g))
+    assert np.array_equal(H, H.T)
+
+
+@pytest.mark.parametrize("g", GROUPS)
+def test_hadamard_walsh_closed_form(g):
+    """Sylvester order: H[i, j] = (-1)^popcount(i & j) / sqrt(g)."""
+    H = oracle.hadamard(g)
+    i = np.arange(g)[:, None]
+    j = np.arange(g)[None, :]
+    par = np.vectorize(lambda v: bin(v).count("1") & 1)(i & j)
+    closed = np.where(par == 1, -1.0, 1.0) / math.sqrt(g)
+    assert np.array_equal(H, closed)
+
+
+@pytest.mark.parametrize("g", GROUPS)
+def test_fwht_unit_vectors_are_hadamard_columns(g):
+    """FWHT(e_j) is column j of H, exactly (sums of +-1 then a power-of-two scale)."""
+    H = oracle.hadamard(g)
+    for j in (0, 1, g // 2 - 1, g - 1):
+        e = np.zeros(g, np.float32)
+        e[j] = 1.0
+        assert np.array_equal(oracle.fwht_f32(e).astype(np.float64), H[:, j])
+
+
+@pytest.mark.parametrize("g", GROUPS)
+def test_fwht_matches_dense_fp64(g):
+    """The fp32 FWHT equals the dense fp64 product H v up to fp32 rounding."""
+    r = np.random.default_rng(1)
+    H = oracle.hadamard(g)
+    for _ in range(20):
+        v = r.standard_normal(g).astype(np.float32) * np.float32(r.uniform(0.1, 100))
+        ref = H @ v.astype(np.float64)
+        got = oracle.fwht_f32(v).astype(np.float64)
+        tol = 1e-6 * math.log2(g) * np.abs(v).max()
+        assert np.abs(got - ref).max() <= tol
+
+
+@pytest.mark.parametrize("g", GROUPS)
+def test_rotation_is_an_involution(g):
+    """H is symmetric and orthogonal, so rotating twice gives back the input."""
+    r = np.random.default_rng(2)
+    x = r.standard_normal((3, 4 * g)).astype(np.float32)
+    back = oracle.rotate_rows_f32(oracle.rotate_rows_f32(x, g), g)
+    assert np.allclose(back, x, rtol=0, atol=1e-5 * np.abs(x).max())
+
+
+@pytest.mark.parametrize("g", GROUPS)
+def test_rotation_leaves_product_unchanged(g):
+    """(x R)(W R)^T = x W^T: rotating both operands by the same block rotation
+    leaves the product unchanged (to 1e-5 relative in fp32)."""
+    r = np.random.default_rng(3)
+    K = 4 * g
+    x = r.standard_normal((7, K)).astype(np.float32)
+    x[:, 3] *= 50
+    W = (r.standard_normal((9, K)) * 0.02).astype(np.float32)
+    xr = oracle.rotate_rows_f32(x, g).astype(np.float64)
+    Wr = oracle.rotate_rows_f32(W, g).astype(np.float64)
+    ref = x.astype(np.float64) @ W.astype(np.float64).T
+    got = xr @ Wr.T
+    scale = np.abs(x).max() * np.abs(W).max() * math.sqrt(K)
+    assert np.abs(got - ref).max() <= 1e-5 * scale
+
+
+def test_rotation_acts_blockwise():
+    """Each g-block is rotated on its own: a one-hot in block b touches only block b."""
+    g, K = 16, 64
+    x = np.zeros((1, K), np.float32)
+    x[0, 2 * g + 5] = 3.0
+    v = oracle.rotate_rows_f32(x, g)[0]
+    H = oracle.hadamard(g)
+    assert np.all(v[: 2 * g] == 0) and np.all(v[3 * g:] == 0)
+    assert np.array_equal(v[2 * g: 3 * g].astype(np.float64), 3.0 * H[:, 5])
+
+
+# ---------------------------------------------------------------- packing
+
+def test_pack_order_golden():
+    d = golden("pack_order.json")
+    codes = np.array([d["codes"]], np.int8)
+    assert oracle.pack_int4(codes).tolist() == [d["packed"]]
+    assert oracle.unpack_int4(np.array([d["packed"]], np.uint8)).tolist() == [d["codes"]]
+
+
+def test_pack_roundtrip_all_codes():
+    allc = np.array([[a, b] for a in range(-8, 8) for b in range(-8, 8)], np.int8).reshape(1, -1)
+    p = oracle.pack_int4(allc)
+    assert len(set(p[0].tolist())) == 256          # every byte value occurs once
+    assert np.array_equal(oracle.unpack_int4(p), allc)
+
+
+def test_unpack_pack_roundtrip_random_bytes():
+    b = inputs.random_bytes(33, 48)
+    assert np.array_equal(oracle.pack_int4(oracle.unpack_int4(b)), b)
+
+
+# ---------------------------------------------------------------- quantization
+
+def test_rounding_ties_golden():
+    d = golden("rounding_ties.json")
+    W = np.array([d["w_row"]], np.float32)
+    packed, s, codes = oracle.pack_weights(W, 0)
+    assert s[0] == np.float32(d["w_scale"])
+    assert codes[0].tolist() == d["w_codes"]
+    x = bits([d["x_row"]])
+    c8, s8, _ = oracle.quantize_act(x, 0, 8)
+    assert c8[0].tolist() == d["x_codes_int8"] and s8[0] == 1.0
+    c4, s4, p4 = oracle.quantize_act(x, 0, 4)
+    assert c4[0].tolist() == d["x_codes_int4"]
+    assert np.array_equal(oracle.unpack_int4(p4), c4)
+
+
+@pytest.mark.parametrize("bits_", (8, 4))
+@pytest.mark.parametrize("g", GROUPS)
+def test_act_quant_error_bound(g, bits_):
+    """|v - q s| <= s/2 per element, where v = H x is computed independently in
+    fp64; the largest |v| maps to +-Q; codes stay in [-Q, Q]."""
+    Q = 127 if bits_ == 8 else 7
+    x = inputs.activations(8, 2 * g, seed=11)
+    codes, s, _ = oracle.quantize_act(x, g, bits_)
+    H = oracle.hadamard(g)
+    xf = oracle.bf16_bits_to_f32(x).astype(np.float64)
+    v = (xf.reshape(8, -1, g) @ H.T).reshape(8, -1)
+    for m in range(8):
+        assert np.all(np.abs(codes[m]) <= Q)
+        err = np.abs(v[m] - codes[m].astype(np.float64) * s[m])
+        # s/2 from rounding, plus the fp32 rounding of v and s
+        assert err.max() <= 0.5 * s[m] * (1 + 1e-5) + 1e-6 * np.abs(v[m]).max()
+        assert abs(int(codes[m][np.argmax(np.abs(v[m]))])) == Q
+        assert abs(s[m] - np.abs(v[m]).max() / Q) <= 1e-6 * s[m]
+
+
+@pytest.mark.parametrize("g", GROUPS)
+def test_weight_quant_error_bound(g):
+    W = inputs.weights(6, 2 * g, seed=12)
+    packed, s, codes = oracle.pack_weights(W, g)
+    H = oracle.hadamard(g)
+    v = (W.astype(np.float64).reshape(6, -1, g) @ H.T).reshape(6, -1)
+    for n in range(6):
+        err = np.abs(v[n] - codes[n] * np.float64(s[n]))
+        assert err.max() <= 0.5 * s[n] * (1 + 1e-5) + 1e-6 * np.abs(v[n]).max()
+        assert np.abs(codes[n]).max() == 7
+    assert np.array_equal(oracle.unpack_int4(packed), codes)
+
+
+def test_zero_rows():
+    """A zero row has scale 0 and codes 0 (no division by zero)."""
+    x = np.zeros((2, 64), np.uint16)
+    c, s, _ = oracle.quantize_act(x, 16, 8)
+    assert np.all(c == 0) and np.all(s == 0)
+    p, sw, cw = oracle.pack_weights(np.zeros((2, 64), np.float32), 64)
+    assert np.all(p == 0) and np.all(sw == 0)
+
+
+def test_onehot_worked_example():
+    d = golden("onehot_g16.json")
+    g = d["g"]
+    x = bits([d["x"]])
+    c8, s8, _ = oracle.quantize_act(x, g, 8)
+    assert c8[0].tolist() == d["act_codes_int8"]
+    c4, s4, _ = oracle.quantize_act(x, g, 4)
+    assert c4[0].tolist() == d["act_codes_int4"]
+    W = np.array(d["W"], np.float32)
+    packed, sw, cw = oracle.pack_weights(W, g)
+    assert cw.tolist() == d["w_codes"]
+    assert packed.tolist() == d["w_packed"]
+    assert np.allclose(sw, d["w_row_scale_exact"], rtol=1e-7)
+    acc8 = oracle.gemm_i32(c8, cw)
+    assert acc8[0].tolist() == d["acc_int8"]
+    acc4 = oracle.gemm_i32(c4, cw)
+    assert acc4[0].tolist() == d["acc_int4"]
+    y = oracle.bf16_bits_to_f32(oracle.epilogue(acc8, s8, sw))
+    assert y[0].tolist() == d["y"]
+    y2 = oracle.bf16_bits_to_f32(oracle.convrot_linear(x, packed, sw, g, 8))
+    assert y2[0].tolist() == d["y"]
+    y3 = oracle.bf16_bits_to_f32(oracle.convrot_linear(x, packed, sw, g, 4))
+    assert y3[0].tolist() == d["y"]
+
+
+# ---------------------------------------------------------------- GEMM
+
+@pytest.mark.parametrize("shape", [(1, 1, 1), (3, 5, 7), (17, 9, 64), (8, 33, 130)])
+def test_gemm_brute_force(shape):
+    """int32 GEMM == exact integer matmul (numpy int64) on tiny shapes."""
+    M, N, K = shape
+    a = inputs.random_codes(M, K, -127, 127, seed=5)
+    w = inputs.random_codes(N, K, -8, 7, seed=6)
+    ref = a.astype(np.int64) @ w.astype(np.int64).T
+    assert np.array_equal(oracle.gemm_i32(a, w), ref)
+
+
+def test_gemm_operand_orientation():
+    """acc[m, n] pairs row m of a with row n of w (not a transposed operand)."""
+    a = np.zeros((2, 4), np.int8)
+    w = np.zeros((3, 4), np.int8)
+    a[1, 2] = 5
+    w[2, 2] = -3
+    acc = oracle.gemm_i32(a, w)
+    expect = np.zeros((2, 3), np.int64)
+    expect[1, 2] = -15
+    assert np.array_equal(acc, expect)
+
+
+def test_gemm_sampled_matches_full():
+    a = inputs.random_codes(20, 96, -127, 127, seed=7)
+    w = inputs.random_codes(30, 96, -7, 7, seed=8)
+    full = oracle.gemm_i32(a, w)
+    pairs = np.array([[0, 0], [19, 29], [5, 17], [11, 3]], np.int64)
+    assert np.array_equal(oracle.gemm_i32_sampled(a, w, pairs), full[pairs[:, 0], pairs[:, 1]])
+
+
+def test_gemm_rejects_int32_overflow():
+    a = np.full((1, 140000), 127, np.int8)
+    w = np.full((1, 140000), 127, np.int8)
+    with pytest.raises(ValueError):
+        oracle.gemm_i32(a, w)
+
+
+# ---------------------------------------------------------------- bf16 rounding / epilogue
+
+def _bf16_nearest_even(v: float) -> float:
+    """Brute force: the bf16 value nearest to v, ties to an even mantissa."""
+    fv = Fraction(v)
+    if v == 0:
+        return 0.0
+    best = None
+    sign = 1 if v > 0 else -1
+    e = math.frexp(abs(v))[1]
+    cands = []
+    for ee in (e - 1, e, e + 1):
+        for m in range(128, 256):
+            cands.append(Fraction(m) * Fraction(2) ** (ee - 8))
+    for c in cands:
+        c = c * sign
+        d = abs(c - fv)
+        key = (d, 0 if (int(abs(c) / Fraction(2) ** (math.frexp(float(abs(c)))[1] - 8)) % 2 == 0) else 1)
+        if best is None or key < best[0]:
+            best = (key, c)
+    return float(best[1])
+
+
+def test_double_to_bf16_brute_force():
+    r = np.random.default_rng(4)
+    vals = list(r.standard_normal(300) * 10.0 ** r.integers(-5, 6, 300))
+    # exact ties between neighbouring bf16 values (odd mantissa + half ulp)
+    vals += [1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(2.0 + 2.0 ** -7), 3.0 + 2.0 ** -7]
+    for v in vals:
+        b = oracle.double_to_bf16_bits(v)
+        got = float(oracle.bf16_bits_to_f32(np.array([b], np.uint16))[0])
+        assert got == _bf16_nearest_even(float(v)), v
+
+
+def test_epilogue_closed_form():
+    r = np.random.default_rng(5)
+    acc = r.integers(-10 ** 6, 10 ** 6, size=(6, 5)).astype(np.int32)
+    st = inputs.positive_scales(6, seed=3)
+    sr = inputs.positive_scales(5, seed=4)
+    bias = bits(r.standard_normal(5))
+    y = oracle.bf16_bits_to_f32(oracle.epilogue(acc, st, sr, bias))
+    ref = (acc.astype(np.float64) * st.astype(np.float64)[:, None] * sr.astype(np.float64)[None, :]
+           + oracle.bf16_bits_to_f32(bias).astype(np.float64)[None, :])
+    for m in range(6):
+        for n in range(5):
+            assert y[m, n] == _bf16_nearest_even(float(ref[m, n]))
+    pairs = np.array([[0, 0], [5, 4], [2, 3]], np.int64)
+    ys = oracle.epilogue_sampled(acc[pairs[:, 0], pairs[:, 1]], st, sr, pairs, bias)
+    assert np.array_equal(ys, oracle.epilogue(acc, st, sr, bias)[pairs[:, 0], pairs[:, 1]])
+
+
+# ---------------------------------------------------------------- whole layer
+
+@pytest.mark.parametrize("act_bits,rel", [(8, 0.2), (4, 0.3)])
+def test_linear_approximates_float_product(act_bits, rel):
+    """The quantized layer approximates the plain float product x W^T: the
+    error is the quantization noise, far below the signal (a transposed operand,
+    a wrong scale or a wrong sign would give an O(1) relative error)."""
+    g = 64
+    x = inputs.activations(32, 256, seed=21)
+    W = inputs.weights(48, 256, seed=22)
+    packed, sr, _ = oracle.pack_weights(W, g)
+    y = oracle.bf16_bits_to_f32(oracle.convrot_linear(x, packed, sr, g, act_bits)).astype(np.float64)
+    ref = oracle.bf16_bits_to_f32(x).astype(np.float64) @ W.astype(np.float64).T
+    err = np.sqrt(np.mean((y - ref) ** 2)) / np.sqrt(np.mean(ref ** 2))
+    assert err < rel
+
+
+def test_rotation_reduces_quant_error_with_outliers():
+    """With outlier channels, rotating before quantization lowers the activation
+    quantization error (the reason the pages rotate): rebuild x from its codes
+    (inverse rotation = the same rotation) and compare with and without it."""
+    x = inputs.activations(32, 256, seed=23)
+    xf = oracle.bf16_bits_to_f32(x).astype(np.float64)
+    for act_bits, gain in ((8, 4.0), (4, 1.8)):
+        errs = {}
+        for g in (0, 256):
+            c, s, _ = oracle.quantize_act(x, g, act_bits)
+            deq = c.astype(np.float64) * s[:, None].astype(np.float64)
+            if g:
+                deq = oracle.rotate_rows_f32(deq.astype(np.float32), g).astype(np.float64)
+            errs[g] = np.sqrt(np.mean((deq - xf) ** 2))
+        assert errs[0] > gain * errs[256]
+
+
+def test_linear_is_composition():
+    g = 16
+    x = inputs.activations(5, 64, seed=25)
+    W = inputs.weights(7, 64, seed=26)
+    packed, sr, cw = oracle.pack_weights(W, g)
+    c, st, _ = oracle.quantize_act(x, g, 8)
+    y = oracle.epilogue(oracle.gemm_i32(c, oracle.unpack_int4(packed)), st, sr)
+    assert np.array_equal(oracle.convrot_linear(x, packed, sr, g, 8), y)
+
+
+# ---------------------------------------------------------------- W4A16
+
+def test_w4a16_golden():
+    d = golden("w4a16_groups.json")
+    K, G = d["K"], d["group"]
+    q = np.array([[b] * (K // 2) for b in d["row_byte"]], np.uint8)
+    z = np.array(d["zero"], np.uint8)
+    s = bits(d["scale"])
+    x = bits(np.ones((1, K)))
+    y = oracle.bf16_bits_to_f32(oracle.w4a16(x, q, s, z, G))
+    assert y[0].tolist() == d["y"]
+
+
+def test_w4a16_reduces_to_plain_matmul():
+    """z = 8, s = 1: the layer is x . (q - 8)^T, exactly an integer-weight matmul."""
+    M, N, K, G = 3, 10, 256, 128
+    op = inputs.w4a16_operands(M, N, K, G, seed=31)
+    z = np.full((N, K // G), 8, np.uint8)
+    s = bits(np.ones((N, K // G)))
+    y = oracle.bf16_bits_to_f32(oracle.w4a16(op.x, op.q, s, z, G)).astype(np.float64)
+    lo = (op.q & 0xF).astype(np.int64)
+    hi = (op.q >> 4).astype(np.int64)
+    qk = np.empty((N, K), np.int64)
+    qk[:, 0::2] = lo
+    qk[:, 1::2] = hi
+    ref = oracle.bf16_bits_to_f32(op.x).astype(np.float64) @ (qk - 8).T.astype(np.float64)
+    for m in range(M):
+        for n in range(N):
+            assert y[m, n] == _bf16_nearest_even(float(ref[m, n]))
+
+
+def test_w4a16_general_dequant():
+    M, N, K, G = 2, 12, 384, 128
+    op = inputs.w4a16_operands(M, N, K, G, seed=32)
+    y = oracle.bf16_bits_to_f32(oracle.w4a16(op.x, op.q, op.scale, op.zero, G)).astype(np.float64)
+    qk = np.empty((N, K), np.float64)
+    qk[:, 0::2] = op.q & 0xF
+    qk[:, 1::2] = op.q >> 4
+    zk = np.repeat(op.zero.astype(np.float64), G, axis=1)
+    sk = np.repeat(oracle.bf16_bits_to_f32(op.scale).astype(np.float64), G, axis=1)
+    ref = oracle.bf16_bits_to_f32(op.x).astype(np.float64) @ ((qk - zk) * sk).T
+    for m in range(M):
+        for n in range(N):
+            assert y[m, n] == _bf16_nearest_even(float(ref[m, n]))
