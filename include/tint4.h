@@ -1,0 +1,191 @@
+/*
+ * tint4.h -- C ABI of the packed-INT4 ConvRot quantized linear layer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (page titles and sections it restates):
+ *   "ComfyUI-INT-Crush", "Forward Pass": rotate the activations (Hadamard,
+ *   rot_size), quantize weights and activations, run the GEMM;
+ *   "Inference > INT4 > CUDA backend": INT4 -> INT8 unpack, INT8 GEMM with
+ *   fused dequant, and for rot_size 256 a fused rotate + quantize + GEMM;
+ *   "Inference > INT4 > Triton backend": dynamic activation quantization
+ *   (W4A8) and the W4A16 path for rot_size 0; "Weight Format": INT4 weights
+ *   are uint8 with two values per byte.
+ *   "feat: packed int4 convrot model loading and dispatch" (stable-diffusion.cpp
+ *   #2010), "Summary": packed nibbles stream to the backend unconverted with
+ *   row scales beside them; the activation rotate+quantize is shared by every
+ *   linear that reads the same input (convrot_w4a4 and W4A8 kinds).
+ *   "TINT4 v1.2 -- torchao INT4 for ComfyUI", "v1.1 新特性 > 5": the W4A16
+ *   layer keeps _qdata/_scale/_zp.
+ *
+ * Formats (readings of the pages, which do not fix them):
+ *   bf16          raw bfloat16 bits (uint16_t), round-to-nearest-even.
+ *   rotation      block Hadamard along K: each length-g block v of a row is
+ *                 replaced by H_g v, H_g the Sylvester (natural-order)
+ *                 Hadamard matrix / sqrt(g); g in {16, 64, 256}; 0 = none.
+ *   packed int4   uint8 [rows, K/2] row-major; byte j of a row holds element
+ *                 2j in its low nibble and 2j+1 in its high nibble, each a
+ *                 4-bit two's complement code.  Symmetric codes use [-7, 7].
+ *   scales        fp32, one per row of W (row_scale [N]) and one per token
+ *                 (tok_scale [M]); scale = absmax / 7 (int4) or / 127 (int8),
+ *                 code = clamp(round_half_even(v / scale)); an all-zero row
+ *                 has scale 0 and codes 0.
+ *   output        y[m, n] = bf16( acc[m, n] * tok_scale[m] * row_scale[n]
+ *                 (+ bias[n]) ), acc the exact int32 sum of code products.
+ *
+ * Conventions for every call:
+ *   - Pointers are DEVICE pointers of the current CUDA device unless stated.
+ *     The caller owns and allocates every buffer; the library never allocates
+ *     device memory and keeps no pointer after the call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; outputs are valid once the
+ *     stream reaches that point.
+ *   - Argument and shape errors are returned synchronously, before anything
+ *     is launched.  Nothing throws across the ABI.  Calls on different
+ *     streams do not share mutable state except the device error word.
+ *   - Shape rules: M >= 0, N >= 16 and N % 16 == 0, K >= 32 and K % 32 == 0,
+ *     K % g == 0; K <= 16384 for the rotate/quantize calls.  Pointers must
+ *     be 16-byte aligned.  Padding K up to the weight's width is the
+ *     caller's job ("ComfyUI-INT-Crush", "Forward Pass" step 3).
+ *   - Device-side waits are bounded (default 4 s, see
+ *     tint4_set_wait_limit_ns); a wait that gives up records a code in the
+ *     device error word, read by tint4_get_device_error.
+ */
+#ifndef TINT4_H
+#define TINT4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TINT4_OK = 0,
+    TINT4_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum value */
+    TINT4_ERR_UNSUPPORTED_SHAPE = 2, /* a shape rule above is broken */
+    TINT4_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned */
+    TINT4_ERR_CUDA = 4,              /* a CUDA runtime / driver call failed */
+    TINT4_ERR_TIMEOUT = 5,           /* a bounded device-side wait gave up */
+    TINT4_ERR_WORKSPACE = 6,         /* workspace missing or too small */
+    TINT4_ERR_NO_DEVICE = 7          /* the current device is not sm_100 */
+} tint4_status;
+
+typedef uint16_t tint4_bf16;
+
+/* ABI version, bumped on any signature change. */
+int tint4_abi_version(void);
+
+/* Static description of a status code (never NULL). */
+const char* tint4_status_string(tint4_status status);
+
+/*
+ * Offline weight preparation ("ComfyUI-INT-Crush", "Workflow" converter with
+ * --rot-size / --int-bits 4 and "Weight Format"; TINT4, "量化方案" step 2).
+ * W fp32 [N, K] -> each g-block along K rotated -> per-row symmetric int4
+ * codes in [-7, 7], row_scale[n] = absmax_n / 7 -> w_packed uint8 [N, K/2].
+ * group: 0 (no rotation), 16, 64 or 256.  Rotating W with the same block
+ * rotation as the activations leaves x W^T unchanged.
+ */
+tint4_status tint4_pack_weights(const float* W, int N, int K, int group, uint8_t* w_packed,
+                                float* row_scale, void* stream);
+
+/*
+ * Dynamic per-token activation rotate + quantize ("ComfyUI-INT-Crush",
+ * "Forward Pass" steps 2 and 5; "Inference > INT4 > Triton backend").
+ * x bf16 [M, K] -> rotate each g-block (fp32) -> tok_scale[m] = absmax_m / Q
+ * -> codes.  bits 8: codes is int8 [M, K], Q = 127 (W4A8).  bits 4: codes is
+ * packed uint8 [M, K/2], Q = 7 (W4A4).  One call can feed every linear that
+ * reads the same input and group ("feat: packed int4 convrot ...", "Summary").
+ */
+tint4_status convrot_quantize_act(const tint4_bf16* x, int M, int K, int group, int bits,
+                                  void* codes, float* tok_scale, void* stream);
+
+/*
+ * W4A8 GEMM with fused dequant ("ComfyUI-INT-Crush", "Inference > INT4 >
+ * CUDA backend").  a int8 [M, K] activation codes, tok_scale fp32 [M],
+ * w_packed uint8 [N, K/2], row_scale fp32 [N], bias bf16 [N] or NULL,
+ * y bf16 [M, N].  int32 accumulation on the tensor cores.
+ */
+tint4_status w4a8_gemm(const int8_t* a, const float* tok_scale, const uint8_t* w_packed,
+                       const float* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
+                       int N, int K, void* stream);
+
+/*
+ * W4A4 GEMM ("Load Diffusion Model INT4 (W4A4)", enable_convrot; stable-
+ * diffusion.cpp "feat: packed int4 convrot ...", convrot_w4a4).  a_packed
+ * uint8 [M, K/2] packed int4 activation codes; otherwise as w4a8_gemm.
+ */
+tint4_status w4a4_gemm(const uint8_t* a_packed, const float* tok_scale, const uint8_t* w_packed,
+                       const float* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
+                       int N, int K, void* stream);
+
+/* Bytes of workspace convrot_w4a8_linear (bits 8) / convrot_w4a4_linear
+ * (bits 4) need: the activation codes plus the token scales, 256-aligned. */
+size_t convrot_linear_workspace_size(int M, int K, int bits);
+
+/*
+ * Fused ConvRot linear ("ComfyUI-INT-Crush", "Inference > INT4 > CUDA
+ * backend": Hadamard rotation + activation quantization + INT8 GEMM as one
+ * call; "Forward Pass" last note).  x bf16 [M, K] -> y bf16 [M, N].  The
+ * rotate+quantize grid and the GEMM grid run back to back on `stream` with
+ * programmatic dependent launch; the codes pass through `workspace`
+ * (device memory of at least convrot_linear_workspace_size(M, K, 8) bytes,
+ * 256-byte aligned, owned by the caller; its contents are scratch).
+ */
+tint4_status convrot_w4a8_linear(const tint4_bf16* x, const uint8_t* w_packed,
+                                 const float* row_scale, const tint4_bf16* bias, tint4_bf16* y,
+                                 int M, int N, int K, int group, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/* As convrot_w4a8_linear with int4 activation codes (W4A4). */
+tint4_status convrot_w4a4_linear(const tint4_bf16* x, const uint8_t* w_packed,
+                                 const float* row_scale, const tint4_bf16* bias, tint4_bf16* y,
+                                 int M, int N, int K, int group, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/*
+ * W4A16 group-wise asymmetric linear for small M ("TINT4 v1.2", "v1.1 新特性
+ * > 5" _qdata/_scale/_zp, "参数选择指南" group 128; "ComfyUI-INT-Crush",
+ * "Inference > INT4 > Triton backend" W4A16).  x bf16 [M, K]; w_q uint8
+ * [N, K/2] unsigned codes 0..15 packed low nibble first; scale bf16
+ * [N, K/group]; zero uint8 [N, K/group] holding 0..15; y bf16 [M, N] with
+ * y[m, n] = sum_k x[m, k] * (q[n, k] - zero[n, k/group]) * scale[n, k/group]
+ * accumulated in fp32.  group must be 128; 1 <= M <= 64; K % 128 == 0.
+ */
+tint4_status w4a16_gemv_gemm(const tint4_bf16* x, const uint8_t* w_q, const tint4_bf16* scale,
+                             const uint8_t* zero, int group, tint4_bf16* y, int M, int N, int K,
+                             void* stream);
+
+/*
+ * Test entry: the raw int32 accumulators acc[m, n] = sum_k qa[m, k] qw[n, k]
+ * of the same tensor-core GEMM (act_bits 8: a is int8 [M, K]; act_bits 4: a
+ * is packed uint8 [M, K/2]).  acc int32 [M, N].
+ */
+tint4_status tint4_debug_int32_gemm(const void* a, int act_bits, const uint8_t* w_packed,
+                                    int32_t* acc, int M, int N, int K, void* stream);
+
+/*
+ * Test entry for the bounded waits: launches one CTA that waits on a barrier
+ * nobody arrives at, for at most limit_ns nanoseconds, then records
+ * TINT4_ERR_TIMEOUT in the device error word and returns.  The context stays
+ * usable.  limit_ns must be in [1e3, 1e10].
+ */
+tint4_status tint4_debug_bounded_wait(uint64_t limit_ns, void* stream);
+
+/*
+ * Synchronizes `stream`, then reads and clears the device error word of the
+ * current device.  Returns TINT4_OK, TINT4_ERR_TIMEOUT (a bounded wait gave
+ * up since the last read) or TINT4_ERR_CUDA.
+ */
+tint4_status tint4_get_device_error(void* stream);
+
+/* Limit of every device-side wait for later launches, in nanoseconds
+ * (default 4e9).  Values outside [1e3, 6e10] return TINT4_ERR_INVALID_ARG. */
+tint4_status tint4_set_wait_limit_ns(uint64_t limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TINT4_H */

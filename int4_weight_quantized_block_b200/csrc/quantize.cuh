@@ -1,0 +1,175 @@
+// quantize.cuh -- block Hadamard rotation + per-row symmetric quantization.
+//
+// One kernel serves two entry points:
+//  * convrot_quantize_act: bf16 activations [M, K] -> int8 codes [M, K] (W4A8)
+//    or packed int4 codes [M, K/2] (W4A4), plus one fp32 scale per token
+//    ("ComfyUI-INT-Crush", "Forward Pass" step 2 rotate and step 5 quantize;
+//    "Inference > INT4 > Triton backend": dynamic per-token activation quant).
+//  * tint4_pack_weights: fp32 weights [N, K] -> packed int4 [N, K/2] + fp32
+//    row scales (offline; "ComfyUI-INT-Crush", "Weight Format"; stable-
+//    diffusion.cpp "feat: packed int4 convrot model loading and dispatch",
+//    "Summary": packed nibbles with row scales).
+//
+// Layout of the work: one CTA per row, 8 warps.  The row is cut into chunks
+// of 256 values; a warp owns chunks w, w+8, w+16, ... and each lane holds 8
+// consecutive values of a chunk in registers (16-byte bf16 loads, fully
+// coalesced).  A rotation block of g values (g = 16, 64 or 256) spans g/8
+// lanes, so the fast Walsh-Hadamard transform runs as three in-register
+// butterfly stages (spans 1, 2, 4) followed by log2(g/8) shuffle stages (spans
+// 8 .. g/2), in that order; every butterfly forms (a + b, a - b) with a the
+// value at the lower index, so the rotated fp32 values do not depend on which
+// thread computes them.  Then the CTA reduces |v| to the row maximum, forms
+// scale = absmax / Q with an IEEE division, and writes the codes
+// clamp(rne(v / scale), -Q, Q) straight from registers.  HBM traffic is one
+// read of the input and one write of the codes: the kernel is bandwidth
+// bound.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace tint4 {
+
+constexpr int kQuantWarps = 8;
+constexpr int kQuantThreads = kQuantWarps * 32;
+constexpr int kQuantChunk = 256;       // values per warp chunk (32 lanes x 8)
+constexpr int kQuantMaxChunksPerWarp = 8;
+constexpr int kQuantMaxK = kQuantWarps * kQuantMaxChunksPerWarp * kQuantChunk;  // 16384
+
+__device__ __forceinline__ void load8_as_f32(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+__device__ __forceinline__ void load8_as_f32(const float* p, float (&v)[8]) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// Orthonormal FWHT over blocks of G values spread as 8 per lane.
+template <int G>
+__device__ __forceinline__ void fwht_lane8(float (&v)[8], int lane) {
+    // in-register stages, spans 1, 2, 4
+#pragma unroll
+    for (int h = 1; h < 8; h *= 2) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if ((j & h) == 0) {
+                const float a = v[j], b = v[j + h];
+                v[j] = a + b;
+                v[j + h] = a - b;
+            }
+        }
+    }
+    // cross-lane stages, spans 8 .. G/2 (lane distance 1 .. G/16)
+#pragma unroll
+    for (int d = 1; d < G / 8; d *= 2) {
+        const bool upper = (lane & d) != 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float other = __shfl_xor_sync(0xFFFFFFFFu, v[j], d);
+            // lower index holds a, upper holds b: lower -> a + b, upper -> a - b
+            v[j] = upper ? (other - v[j]) : (v[j] + other);
+        }
+    }
+    // 1/sqrt(G): a power of two for G = 4^k, so this is exact
+    constexpr float s = (G == 16) ? 0.25f : (G == 64) ? 0.125f : (G == 256) ? 0.0625f : 1.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] *= s;
+}
+
+// CH = chunks per warp held in registers (K <= 8 warps * CH * 256).
+template <typename InT, int G, int BITS, int CH>
+__global__ void __launch_bounds__(kQuantThreads)
+rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K,
+                            void* __restrict__ codes, float* __restrict__ scales) {
+    constexpr int Q = (BITS == 8) ? 127 : 7;
+    const int row = blockIdx.x;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    __shared__ float red[kQuantWarps];
+
+    // Under programmatic dependent launch, let the consumer grid start its
+    // prologue while this grid runs; it waits for our completion before
+    // reading the codes.
+    grid_launch_dependents();
+
+    const InT* src = in + static_cast<size_t>(row) * K;
+    const int nchunks = (K + kQuantChunk - 1) / kQuantChunk;
+
+    float v[CH][8];
+    float amax = 0.0f;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+        const int chunk = warp + c * kQuantWarps;
+        const int base = chunk * kQuantChunk + lane * 8;
+        if (chunk < nchunks && base < K) {
+            load8_as_f32(src + base, v[c]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[c][j] = 0.0f;
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+        const int chunk = warp + c * kQuantWarps;
+        if (chunk < nchunks) {  // warp-uniform
+            if (G > 0) fwht_lane8<(G > 0 ? G : 16)>(v[c], lane);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[c][j]));
+        }
+    }
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, d));
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    amax = red[0];
+#pragma unroll
+    for (int w = 1; w < kQuantWarps; ++w) amax = fmaxf(amax, red[w]);
+
+    const float scale = __fdiv_rn(amax, static_cast<float>(Q));
+    if (threadIdx.x == 0) scales[row] = scale;
+
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+        const int chunk = warp + c * kQuantWarps;
+        const int base = chunk * kQuantChunk + lane * 8;
+        if (chunk < nchunks && base < K) {
+            int q[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float t = 0.0f;
+                if (scale > 0.0f) {
+                    t = rintf(__fdiv_rn(v[c][j], scale));
+                    t = fminf(fmaxf(t, static_cast<float>(-Q)), static_cast<float>(Q));
+                }
+                q[j] = static_cast<int>(t);
+            }
+            if (BITS == 8) {
+                uint2 out;
+                out.x = (q[0] & 0xFF) | ((q[1] & 0xFF) << 8) | ((q[2] & 0xFF) << 16) |
+                        (static_cast<uint32_t>(q[3] & 0xFF) << 24);
+                out.y = (q[4] & 0xFF) | ((q[5] & 0xFF) << 8) | ((q[6] & 0xFF) << 16) |
+                        (static_cast<uint32_t>(q[7] & 0xFF) << 24);
+                int8_t* dst = static_cast<int8_t*>(codes) + static_cast<size_t>(row) * K + base;
+                *reinterpret_cast<uint2*>(dst) = out;
+            } else {
+                // low nibble = even index, high nibble = odd index
+                uint32_t out = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) out |= static_cast<uint32_t>(q[j] & 0xF) << (4 * j);
+                uint8_t* dst =
+                    static_cast<uint8_t*>(codes) + static_cast<size_t>(row) * (K / 2) + base / 2;
+                *reinterpret_cast<uint32_t*>(dst) = out;
+            }
+        }
+    }
+}
+
+}  // namespace tint4

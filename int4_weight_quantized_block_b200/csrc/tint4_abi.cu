@@ -1,0 +1,440 @@
+// tint4_abi.cu -- the C ABI of include/tint4.h: argument checks, tensor maps,
+// launch configuration.  Every operation runs in the kernels of quantize.cuh,
+// gemm.cuh and w4a16.cuh; nothing here touches tensor data.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/tint4.h"
+#include "gemm.cuh"
+#include "ptx.cuh"
+#include "quantize.cuh"
+#include "w4a16.cuh"
+
+namespace {
+
+using namespace tint4;
+
+constexpr int kAbiVersion = 1;
+constexpr int kMaxDevices = 64;
+constexpr int kGemmBN = 256;
+constexpr int kGemmStages = 3;
+
+std::atomic<uint64_t> g_wait_limit_ns{4000000000ull};
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ------------------------------------------------------------------ device check
+
+tint4_status check_device(int* dev_out = nullptr) {
+    static std::atomic<int> cache[kMaxDevices];  // 0 unknown, 1 ok, 2 unsupported
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return TINT4_ERR_NO_DEVICE;
+    }
+    if (dev_out) *dev_out = dev;
+    if (dev < 0 || dev >= kMaxDevices) return TINT4_ERR_NO_DEVICE;
+    int c = cache[dev].load(std::memory_order_relaxed);
+    if (c == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return TINT4_ERR_NO_DEVICE;
+        }
+        c = (major == 10 && minor == 0) ? 1 : 2;
+        cache[dev].store(c, std::memory_order_relaxed);
+    }
+    return c == 1 ? TINT4_OK : TINT4_ERR_NO_DEVICE;
+}
+
+tint4_status last_launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? TINT4_OK : TINT4_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// 2-D uint8 tensor [outer, inner] with row pitch `pitch` bytes; box
+// [box_outer, box_inner]; out-of-range elements read as zero.
+bool make_map_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                 uint64_t pitch, uint32_t box_inner, uint32_t box_outer,
+                 CUtensorMapSwizzle swizzle) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {pitch};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ shape rules
+
+tint4_status check_mnk(int M, int N, int K) {
+    if (M < 0 || N < 0 || K < 0) return TINT4_ERR_INVALID_ARG;
+    if (N < 16 || N % 16 != 0) return TINT4_ERR_UNSUPPORTED_SHAPE;
+    if (K < 32 || K % 32 != 0 || K > 65536) return TINT4_ERR_UNSUPPORTED_SHAPE;
+    if (M > 65535 * kGemmBM) return TINT4_ERR_UNSUPPORTED_SHAPE;
+    return TINT4_OK;
+}
+
+bool valid_group(int g) { return g == 0 || g == 16 || g == 64 || g == 256; }
+
+// ------------------------------------------------------------------ rotate + quantize
+
+template <typename InT, int G, int BITS, int CH>
+void launch_rq(const InT* in, int rows, int K, void* codes, float* scales, cudaStream_t st) {
+    rotate_quantize_rows_kernel<InT, G, BITS, CH><<<rows, kQuantThreads, 0, st>>>(in, rows, K,
+                                                                                   codes, scales);
+}
+
+template <typename InT, int G, int BITS>
+void launch_rq_ch(const InT* in, int rows, int K, void* codes, float* scales, cudaStream_t st) {
+    const int nchunks = (K + kQuantChunk - 1) / kQuantChunk;
+    const int per_warp = (nchunks + kQuantWarps - 1) / kQuantWarps;
+    if (per_warp <= 1) launch_rq<InT, G, BITS, 1>(in, rows, K, codes, scales, st);
+    else if (per_warp <= 2) launch_rq<InT, G, BITS, 2>(in, rows, K, codes, scales, st);
+    else if (per_warp <= 4) launch_rq<InT, G, BITS, 4>(in, rows, K, codes, scales, st);
+    else launch_rq<InT, G, BITS, 8>(in, rows, K, codes, scales, st);
+}
+
+template <typename InT, int BITS>
+void launch_rq_g(const InT* in, int rows, int K, int g, void* codes, float* scales,
+                 cudaStream_t st) {
+    switch (g) {
+        case 0: launch_rq_ch<InT, 0, BITS>(in, rows, K, codes, scales, st); break;
+        case 16: launch_rq_ch<InT, 16, BITS>(in, rows, K, codes, scales, st); break;
+        case 64: launch_rq_ch<InT, 64, BITS>(in, rows, K, codes, scales, st); break;
+        default: launch_rq_ch<InT, 256, BITS>(in, rows, K, codes, scales, st); break;
+    }
+}
+
+tint4_status check_rq_shape(int rows, int K, int g) {
+    if (rows < 0 || K < 0) return TINT4_ERR_INVALID_ARG;
+    if (!valid_group(g)) return TINT4_ERR_INVALID_ARG;
+    if (K < 32 || K % 32 != 0 || K > kQuantMaxK) return TINT4_ERR_UNSUPPORTED_SHAPE;
+    if (g != 0 && K % g != 0) return TINT4_ERR_UNSUPPORTED_SHAPE;
+    return TINT4_OK;
+}
+
+// ------------------------------------------------------------------ GEMM
+
+template <bool A_INT4, bool OUT_I32>
+tint4_status launch_gemm(const void* a, const uint8_t* w, const float* st, const float* sr,
+                         const __nv_bfloat16* bias, void* out, int M, int N, int K,
+                         cudaStream_t stream, bool pdl) {
+    using L = GemmLayout<A_INT4, kGemmBN, kGemmStages>;
+    auto kern = w4_gemm_kernel<A_INT4, kGemmBN, kGemmStages, OUT_I32>;
+    CUtensorMap ta, tw;
+    bool ok;
+    if (A_INT4)
+        ok = make_map_u8(&ta, a, K / 2, M, K / 2, 64, kGemmBM, CU_TENSOR_MAP_SWIZZLE_NONE);
+    else
+        ok = make_map_u8(&ta, a, K, M, K, kGemmBK, kGemmBM, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && make_map_u8(&tw, w, K / 2, N, K / 2, 64, kGemmBN, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!ok) return TINT4_ERR_CUDA;
+
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static std::atomic<bool> attr_done[kMaxDevices];
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 L::kSmemBytes) != cudaSuccess) {
+            cudaGetLastError();
+            return TINT4_ERR_CUDA;
+        }
+        attr_done[dev].store(true, std::memory_order_release);
+    }
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((N + kGemmBN - 1) / kGemmBN, (M + kGemmBM - 1) / kGemmBM, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = L::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (pdl) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    const uint64_t wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tw, st, sr, bias, out, M, N, K, wait_ns) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return TINT4_ERR_CUDA;
+    }
+    return TINT4_OK;
+}
+
+tint4_status gemm_entry(bool a_int4, const void* a, const float* tok_scale, const uint8_t* w,
+                        const float* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
+                        int N, int K, void* stream) {
+    tint4_status s = check_mnk(M, N, K);
+    if (s != TINT4_OK) return s;
+    if (M > 0 && (!a || !tok_scale || !w || !row_scale || !y)) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(tok_scale) || !aligned16(w) || !aligned16(row_scale) ||
+        !aligned16(y) || !aligned16(bias))
+        return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (M == 0) return TINT4_OK;
+    const auto* b = reinterpret_cast<const __nv_bfloat16*>(bias);
+    return a_int4 ? launch_gemm<true, false>(a, w, tok_scale, row_scale, b, y, M, N, K,
+                                             as_stream(stream), false)
+                  : launch_gemm<false, false>(a, w, tok_scale, row_scale, b, y, M, N, K,
+                                              as_stream(stream), false);
+}
+
+tint4_status linear_entry(int bits, const tint4_bf16* x, const uint8_t* w_packed,
+                          const float* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
+                          int N, int K, int group, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+    tint4_status s = check_mnk(M, N, K);
+    if (s != TINT4_OK) return s;
+    if ((s = check_rq_shape(M, K, group)) != TINT4_OK) return s;
+    if (M > 0 && (!x || !w_packed || !row_scale || !y)) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_packed) || !aligned16(row_scale) || !aligned16(y) ||
+        !aligned16(bias))
+        return TINT4_ERR_MISALIGNED;
+    if (M > 0 && (!workspace || workspace_bytes < convrot_linear_workspace_size(M, K, bits)))
+        return TINT4_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (M == 0) return TINT4_OK;
+    const size_t code_bytes = static_cast<size_t>(M) * K / (bits == 8 ? 1 : 2);
+    uint8_t* codes = static_cast<uint8_t*>(workspace);
+    float* tok_scale = reinterpret_cast<float*>(codes + align_up(code_bytes, 256));
+    cudaStream_t st = as_stream(stream);
+    const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    const auto* b = reinterpret_cast<const __nv_bfloat16*>(bias);
+    if (bits == 8) launch_rq_g<__nv_bfloat16, 8>(xb, M, K, group, codes, tok_scale, st);
+    else launch_rq_g<__nv_bfloat16, 4>(xb, M, K, group, codes, tok_scale, st);
+    if ((s = last_launch_status()) != TINT4_OK) return s;
+    return bits == 8
+               ? launch_gemm<false, false>(codes, w_packed, tok_scale, row_scale, b, y, M, N, K,
+                                           st, true)
+               : launch_gemm<true, false>(codes, w_packed, tok_scale, row_scale, b, y, M, N, K,
+                                          st, true);
+}
+
+// ------------------------------------------------------------------ W4A16
+
+template <int NB>
+void launch_w4a16(const __nv_bfloat16* x, const uint8_t* q, const __nv_bfloat16* s,
+                  const uint8_t* z, __nv_bfloat16* y, int M, int N, int K, cudaStream_t st) {
+    const int grid = (N + kW16Rows - 1) / kW16Rows;
+    w4a16_mma_kernel<NB><<<grid, kW16Threads, 0, st>>>(x, q, s, z, y, M, N, K);
+}
+
+// ------------------------------------------------------------------ bounded-wait test
+
+__global__ void bounded_wait_test_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ uint32_t abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0u;
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // nobody arrives on `bar`: the wait must run out and report
+        mbar_wait_bounded(&bar, 0, &abort_flag, limit_ns, kDevErrTimeoutTest);
+    }
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+int tint4_abi_version(void) { return kAbiVersion; }
+
+const char* tint4_status_string(tint4_status status) {
+    switch (status) {
+        case TINT4_OK: return "ok";
+        case TINT4_ERR_INVALID_ARG: return "invalid argument";
+        case TINT4_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case TINT4_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case TINT4_ERR_CUDA: return "CUDA error";
+        case TINT4_ERR_TIMEOUT: return "device-side wait timed out";
+        case TINT4_ERR_WORKSPACE: return "workspace missing or too small";
+        case TINT4_ERR_NO_DEVICE: return "current device is not an sm_100 GPU";
+    }
+    return "unknown status";
+}
+
+tint4_status tint4_pack_weights(const float* W, int N, int K, int group, uint8_t* w_packed,
+                                float* row_scale, void* stream) {
+    tint4_status s = check_rq_shape(N, K, group);
+    if (s != TINT4_OK) return s;
+    if (N > 0 && (!W || !w_packed || !row_scale)) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(w_packed) || !aligned16(row_scale)) return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (N == 0) return TINT4_OK;
+    launch_rq_g<float, 4>(W, N, K, group, w_packed, row_scale, as_stream(stream));
+    return last_launch_status();
+}
+
+tint4_status convrot_quantize_act(const tint4_bf16* x, int M, int K, int group, int bits,
+                                  void* codes, float* tok_scale, void* stream) {
+    if (bits != 8 && bits != 4) return TINT4_ERR_INVALID_ARG;
+    tint4_status s = check_rq_shape(M, K, group);
+    if (s != TINT4_OK) return s;
+    if (M > 0 && (!x || !codes || !tok_scale)) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(tok_scale)) return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (M == 0) return TINT4_OK;
+    const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    if (bits == 8) launch_rq_g<__nv_bfloat16, 8>(xb, M, K, group, codes, tok_scale, as_stream(stream));
+    else launch_rq_g<__nv_bfloat16, 4>(xb, M, K, group, codes, tok_scale, as_stream(stream));
+    return last_launch_status();
+}
+
+tint4_status w4a8_gemm(const int8_t* a, const float* tok_scale, const uint8_t* w_packed,
+                       const float* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
+                       int N, int K, void* stream) {
+    return gemm_entry(false, a, tok_scale, w_packed, row_scale, bias, y, M, N, K, stream);
+}
+
+tint4_status w4a4_gemm(const uint8_t* a_packed, const float* tok_scale, const uint8_t* w_packed,
+                       const float* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
+                       int N, int K, void* stream) {
+    return gemm_entry(true, a_packed, tok_scale, w_packed, row_scale, bias, y, M, N, K, stream);
+}
+
+size_t convrot_linear_workspace_size(int M, int K, int bits) {
+    if (M < 0 || K < 0 || (bits != 8 && bits != 4)) return 0;
+    const size_t code_bytes = static_cast<size_t>(M) * K / (bits == 8 ? 1 : 2);
+    return align_up(code_bytes, 256) + align_up(static_cast<size_t>(M) * sizeof(float), 256);
+}
+
+tint4_status convrot_w4a8_linear(const tint4_bf16* x, const uint8_t* w_packed,
+                                 const float* row_scale, const tint4_bf16* bias, tint4_bf16* y,
+                                 int M, int N, int K, int group, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    return linear_entry(8, x, w_packed, row_scale, bias, y, M, N, K, group, workspace,
+                        workspace_bytes, stream);
+}
+
+tint4_status convrot_w4a4_linear(const tint4_bf16* x, const uint8_t* w_packed,
+                                 const float* row_scale, const tint4_bf16* bias, tint4_bf16* y,
+                                 int M, int N, int K, int group, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    return linear_entry(4, x, w_packed, row_scale, bias, y, M, N, K, group, workspace,
+                        workspace_bytes, stream);
+}
+
+tint4_status w4a16_gemv_gemm(const tint4_bf16* x, const uint8_t* w_q, const tint4_bf16* scale,
+                             const uint8_t* zero, int group, tint4_bf16* y, int M, int N, int K,
+                             void* stream) {
+    if (M < 0 || N < 0 || K < 0) return TINT4_ERR_INVALID_ARG;
+    if (group != kW16Group) return TINT4_ERR_UNSUPPORTED_SHAPE;
+    if (M < 1 || M > 64 || N < 16 || N % 16 != 0 || K < kW16Group || K % kW16Group != 0)
+        return TINT4_ERR_UNSUPPORTED_SHAPE;
+    if (!x || !w_q || !scale || !zero || !y) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_q) || !aligned16(scale) || !aligned16(zero) ||
+        !aligned16(y))
+        return TINT4_ERR_MISALIGNED;
+    tint4_status s = check_device();
+    if (s != TINT4_OK) return s;
+    const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    const auto* sb = reinterpret_cast<const __nv_bfloat16*>(scale);
+    auto* yb = reinterpret_cast<__nv_bfloat16*>(y);
+    cudaStream_t st = as_stream(stream);
+    const int nb = (M + 7) / 8;
+    if (nb <= 1) launch_w4a16<1>(xb, w_q, sb, zero, yb, M, N, K, st);
+    else if (nb <= 2) launch_w4a16<2>(xb, w_q, sb, zero, yb, M, N, K, st);
+    else if (nb <= 4) launch_w4a16<4>(xb, w_q, sb, zero, yb, M, N, K, st);
+    else launch_w4a16<8>(xb, w_q, sb, zero, yb, M, N, K, st);
+    return last_launch_status();
+}
+
+tint4_status tint4_debug_int32_gemm(const void* a, int act_bits, const uint8_t* w_packed,
+                                    int32_t* acc, int M, int N, int K, void* stream) {
+    if (act_bits != 8 && act_bits != 4) return TINT4_ERR_INVALID_ARG;
+    tint4_status s = check_mnk(M, N, K);
+    if (s != TINT4_OK) return s;
+    if (M > 0 && (!a || !w_packed || !acc)) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(w_packed) || !aligned16(acc)) return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (M == 0) return TINT4_OK;
+    return act_bits == 4 ? launch_gemm<true, true>(a, w_packed, nullptr, nullptr, nullptr, acc, M,
+                                                   N, K, as_stream(stream), false)
+                         : launch_gemm<false, true>(a, w_packed, nullptr, nullptr, nullptr, acc,
+                                                    M, N, K, as_stream(stream), false);
+}
+
+tint4_status tint4_debug_bounded_wait(uint64_t limit_ns, void* stream) {
+    if (limit_ns < 1000ull || limit_ns > 10000000000ull) return TINT4_ERR_INVALID_ARG;
+    tint4_status s = check_device();
+    if (s != TINT4_OK) return s;
+    bounded_wait_test_kernel<<<1, 32, 0, as_stream(stream)>>>(limit_ns);
+    return last_launch_status();
+}
+
+tint4_status tint4_get_device_error(void* stream) {
+    tint4_status s = check_device();
+    if (s != TINT4_OK) return s;
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return TINT4_ERR_CUDA;
+    }
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) {
+        cudaGetLastError();
+        return TINT4_ERR_CUDA;
+    }
+    if (v != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) {
+            cudaGetLastError();
+            return TINT4_ERR_CUDA;
+        }
+        return TINT4_ERR_TIMEOUT;
+    }
+    return TINT4_OK;
+}
+
+tint4_status tint4_set_wait_limit_ns(uint64_t limit_ns) {
+    if (limit_ns < 1000ull || limit_ns > 60000000000ull) return TINT4_ERR_INVALID_ARG;
+    g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+    return TINT4_OK;
+}
+
+}  // extern "C"

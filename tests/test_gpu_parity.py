@@ -1,0 +1,249 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Every test feeds the same seeded inputs to both sides.  Bars:
+  * packed weight bytes and int32 accumulators: bit-exact;
+  * activation codes: equal except at rounding ties (<= 1e-4 of elements,
+    each off by at most 1) -- both sides decide them in fp32;
+  * bf16 outputs: max |gpu - oracle| / rms(oracle) <= 1e-2.
+Small cases span several tiles and ragged tails in M, N and K; the full-size
+workloads are checked on sampled outputs the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import int4_weight_quantized_block_b200 as t4
+from int4_weight_quantized_block_b200 import inputs
+from gpu_util import (CODE_MISMATCH_FRAC, Y_TOL, bf16_from_gpu, bf16_to_gpu, code_mismatch,
+                      dev, rel_err, to_gpu)
+
+pytestmark = pytest.mark.gpu
+
+
+# ------------------------------------------------------------------ weights
+
+@pytest.mark.parametrize("N,K,g", [(16, 32, 0), (48, 352, 16), (272, 320, 64), (33 * 16, 768, 256),
+                                   (256, 256, 256), (64, 16384, 16)])
+def test_pack_weights_bit_exact(N, K, g):
+    W = inputs.weights(N, K, seed=100 + K)
+    W[3, :] = 0.0                                   # an all-zero row
+    p_ref, s_ref, _ = oracle.pack_weights(W, g)
+    p, s = t4.tint4_pack_weights(to_gpu(W), g)
+    torch.cuda.synchronize()
+    assert np.array_equal(p.cpu().numpy(), p_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+# ------------------------------------------------------------------ activations
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("M,K,g", [(1, 32, 0), (7, 352, 16), (130, 320, 64), (64, 256, 256),
+                                   (33, 3072, 256), (5, 12288, 64), (3, 16384, 256)])
+def test_quantize_act(M, K, g, bits):
+    x = inputs.activations(M, K, seed=200 + K)
+    if M > 2:
+        x[2, :] = 0                                  # an all-zero token
+    c_ref, s_ref, p_ref = oracle.quantize_act(x, g, bits)
+    codes, s = t4.convrot_quantize_act(bf16_to_gpu(x), g, bits)
+    torch.cuda.synchronize()
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    if bits == 8:
+        frac, dmax = code_mismatch(codes.cpu().numpy(), c_ref)
+    else:
+        frac, dmax = code_mismatch(oracle.unpack_int4(codes.cpu().numpy()), c_ref)
+    assert frac <= CODE_MISMATCH_FRAC and dmax <= 1
+
+
+# ------------------------------------------------------------------ int32 GEMM
+
+GEMM_SHAPES = [
+    (1, 16, 32),        # minimum
+    (64, 256, 256),     # the tiny layer
+    (200, 272, 352),    # 2 M tiles (ragged), 2 N tiles (ragged 16), 3 K stages (ragged 96)
+    (129, 512, 1024),
+    (300, 768, 3072),
+]
+
+
+@pytest.mark.parametrize("act_bits", [8, 4])
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_int32_accumulators_bit_exact(M, N, K, act_bits):
+    Q = 127 if act_bits == 8 else 7
+    qa = inputs.random_codes(M, K, -Q, Q, seed=300 + M)
+    qw = inputs.random_codes(N, K, -7, 7, seed=301 + N)
+    # extreme rows: all +Q against all +7 / -7
+    qa[0, :] = Q
+    qw[0, :] = 7
+    qw[1 % N, :] = -7
+    wp = oracle.pack_int4(qw)
+    acc_ref = oracle.gemm_i32(qa, qw)
+    a = to_gpu(qa) if act_bits == 8 else to_gpu(oracle.pack_int4(qa))
+    acc = t4.tint4_debug_int32_gemm(a, act_bits, to_gpu(wp))
+    torch.cuda.synchronize()
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+
+
+@pytest.mark.parametrize("act_bits", [8, 4])
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES[1:4])
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_gemm_bf16_epilogue(M, N, K, act_bits, with_bias):
+    Q = 127 if act_bits == 8 else 7
+    qa = inputs.random_codes(M, K, -Q, Q, seed=400 + M)
+    qw = inputs.random_codes(N, K, -7, 7, seed=401 + N)
+    st = inputs.positive_scales(M, seed=402)
+    sr = inputs.positive_scales(N, seed=403)
+    bias = inputs.f32_to_bf16_bits(np.linspace(-3, 3, N)) if with_bias else None
+    y_ref = oracle.epilogue(oracle.gemm_i32(qa, qw), st, sr, bias)
+    wp = oracle.pack_int4(qw)
+    b = bf16_to_gpu(bias) if with_bias else None
+    if act_bits == 8:
+        y = t4.w4a8_gemm(to_gpu(qa), to_gpu(st), to_gpu(wp), to_gpu(sr), b)
+    else:
+        y = t4.w4a4_gemm(to_gpu(oracle.pack_int4(qa)), to_gpu(st), to_gpu(wp), to_gpu(sr), b)
+    torch.cuda.synchronize()
+    assert rel_err(bf16_from_gpu(y), y_ref) <= Y_TOL
+
+
+# ------------------------------------------------------------------ fused linear
+
+@pytest.mark.parametrize("act_bits", [8, 4])
+@pytest.mark.parametrize("M,N,K,g", [(64, 256, 256, 256), (200, 272, 320, 64),
+                                     (33, 512, 768, 16), (129, 256, 1024, 256)])
+def test_convrot_linear_small(M, N, K, g, act_bits):
+    x = inputs.activations(M, K, seed=500 + K)
+    W = inputs.weights(N, K, seed=501 + N)
+    wp, sr, _ = oracle.pack_weights(W, g)
+    y_ref = oracle.convrot_linear(x, wp, sr, g, act_bits)
+    fn = t4.convrot_w4a8_linear if act_bits == 8 else t4.convrot_w4a4_linear
+    y = fn(bf16_to_gpu(x), to_gpu(wp), to_gpu(sr), g)
+    torch.cuda.synchronize()
+    assert rel_err(bf16_from_gpu(y), y_ref) <= Y_TOL
+
+
+def test_quantized_linear_module_end_to_end():
+    """Weights packed on the GPU, layer run on the GPU, both against the oracle."""
+    M, N, K, g = 96, 320, 512, 64
+    x = inputs.activations(M, K, seed=77)
+    W = inputs.weights(N, K, seed=78)
+    lin = t4.QuantizedLinear.from_float(to_gpu(W), g, act_bits=8)
+    y = lin(bf16_to_gpu(x))
+    wp, sr, _ = oracle.pack_weights(W, g)
+    torch.cuda.synchronize()
+    assert np.array_equal(lin.w_packed.cpu().numpy(), wp)
+    assert rel_err(bf16_from_gpu(y), oracle.convrot_linear(x, wp, sr, g, 8)) <= Y_TOL
+
+
+def _sample_pairs(M, N, n, seed):
+    r = np.random.default_rng(seed)
+    pairs = np.stack([r.integers(0, M, n), r.integers(0, N, n)], axis=1)
+    corners = np.array([[0, 0], [M - 1, N - 1], [0, N - 1], [M - 1, 0],
+                        [M // 2, N // 2], [127, 255], [128, 256]])
+    corners = corners[(corners[:, 0] < M) & (corners[:, 1] < N)]
+    return np.concatenate([pairs, corners]).astype(np.int64)
+
+
+@pytest.mark.parametrize("name", ["dit_qkv_w4a8", "dit_qkv_w4a4", "dit_mlp_up_w4a8",
+                                  "dit_mlp_down_w4a8"])
+def test_full_size_workloads_sampled(name):
+    """The full-size layers: weights packed on the GPU (bit-exact against the
+    oracle, all of them), activation codes (all of them), and the layer output
+    on sampled (m, n) pairs that the oracle computes one by one."""
+    w = inputs.WORKLOADS[name]
+    M, N, K, g, bits = w["M"], w["N"], w["K"], w["group"], w["act_bits"]
+    x, W = inputs.layer_inputs(name)
+    wp_ref, sr_ref, qw_ref = oracle.pack_weights(W, g)
+    wp, sr = t4.tint4_pack_weights(to_gpu(W), g)
+    codes, st = t4.convrot_quantize_act(bf16_to_gpu(x), g, bits)
+    fn = t4.convrot_w4a8_linear if bits == 8 else t4.convrot_w4a4_linear
+    y = fn(bf16_to_gpu(x), wp, sr, g)
+    torch.cuda.synchronize()
+    assert np.array_equal(wp.cpu().numpy(), wp_ref)
+    assert np.array_equal(sr.cpu().numpy().view(np.uint32), sr_ref.view(np.uint32))
+    qa_ref, st_ref, _ = oracle.quantize_act(x, g, bits)
+    qa_gpu = codes.cpu().numpy() if bits == 8 else oracle.unpack_int4(codes.cpu().numpy())
+    frac, dmax = code_mismatch(qa_gpu, qa_ref)
+    assert frac <= CODE_MISMATCH_FRAC and dmax <= 1
+    assert np.array_equal(st.cpu().numpy().view(np.uint32), st_ref.view(np.uint32))
+    pairs = _sample_pairs(M, N, 4096, seed=9)
+    acc = oracle.gemm_i32_sampled(qa_ref, qw_ref, pairs)
+    y_ref = oracle.epilogue_sampled(acc, st_ref, sr_ref, pairs)
+    y_gpu = bf16_from_gpu(y)[pairs[:, 0], pairs[:, 1]]
+    assert rel_err(y_gpu, y_ref) <= Y_TOL
+    # int32 accumulators of the same codes, bit-exact on the samples
+    a = to_gpu(qa_ref) if bits == 8 else to_gpu(oracle.pack_int4(qa_ref))
+    acc_gpu = t4.tint4_debug_int32_gemm(a, bits, to_gpu(wp_ref))
+    torch.cuda.synchronize()
+    assert np.array_equal(acc_gpu.cpu().numpy()[pairs[:, 0], pairs[:, 1]], acc)
+
+
+# ------------------------------------------------------------------ W4A16
+
+@pytest.mark.parametrize("M,N,K", [(1, 16, 128), (4, 272, 384), (16, 512, 1024),
+                                   (9, 128, 4096), (64, 64, 256), (33, 96, 512)])
+def test_w4a16(M, N, K):
+    op = inputs.w4a16_operands(M, N, K, 128, seed=600 + M)
+    y_ref = oracle.w4a16(op.x, op.q, op.scale, op.zero, 128)
+    y = t4.w4a16_gemv_gemm(bf16_to_gpu(op.x), to_gpu(op.q), bf16_to_gpu(op.scale),
+                           to_gpu(op.zero), 128)
+    torch.cuda.synchronize()
+    assert rel_err(bf16_from_gpu(y), y_ref) <= Y_TOL
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_w4a16_full_size(M):
+    w = inputs.WORKLOADS["te_decode_w4a16"]
+    op = inputs.w4a16_operands(M, w["N"], w["K"], w["group"])
+    y_ref = oracle.w4a16(op.x, op.q, op.scale, op.zero, w["group"])
+    y = t4.w4a16_gemv_gemm(bf16_to_gpu(op.x), to_gpu(op.q), bf16_to_gpu(op.scale),
+                           to_gpu(op.zero), w["group"])
+    torch.cuda.synchronize()
+    assert rel_err(bf16_from_gpu(y), y_ref) <= Y_TOL
+
+
+# ------------------------------------------------------------------ edge cases
+
+def test_empty_m_is_a_no_op():
+    wp = to_gpu(np.zeros((256, 128), np.uint8))
+    sr = to_gpu(np.ones(256, np.float32))
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device=dev())
+    y = t4.convrot_w4a8_linear(x, wp, sr, 256)
+    assert y.shape == (0, 256)
+    a = torch.empty((0, 256), dtype=torch.int8, device=dev())
+    st = torch.empty((0,), dtype=torch.float32, device=dev())
+    assert t4.w4a8_gemm(a, st, wp, sr).shape == (0, 256)
+
+
+def test_zero_input_gives_zero_output():
+    x = torch.zeros((64, 256), dtype=torch.bfloat16, device=dev())
+    W = inputs.weights(256, 256, seed=5)
+    wp, sr = t4.tint4_pack_weights(to_gpu(W), 256)
+    y = t4.convrot_w4a8_linear(x, wp, sr, 256)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(y).item() == 0
+
+
+def test_misaligned_pointer_is_rejected():
+    buf = torch.zeros(64 * 256 + 16, dtype=torch.int8, device=dev())
+    a = buf[8:8 + 64 * 256].view(64, 256)
+    st = torch.ones(64, dtype=torch.float32, device=dev())
+    wp = torch.zeros((256, 128), dtype=torch.uint8, device=dev())
+    sr = torch.ones(256, dtype=torch.float32, device=dev())
+    with pytest.raises(t4.Tint4Error) as e:
+        t4.w4a8_gemm(a, st, wp, sr)
+    assert e.value.name == "TINT4_ERR_MISALIGNED"
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A device-side wait that nobody releases gives up after its limit and
+    reports TINT4_ERR_TIMEOUT; the context stays usable afterwards."""
+    assert t4.tint4_get_device_error() == 0
+    t4.tint4_debug_bounded_wait(2_000_000)       # 2 ms
+    assert t4.tint4_get_device_error() == 5
+    assert t4.tint4_get_device_error() == 0     # the read cleared it
+    qa = inputs.random_codes(64, 256, -127, 127, seed=1)
+    qw = inputs.random_codes(256, 256, -7, 7, seed=2)
+    acc = t4.tint4_debug_int32_gemm(to_gpu(qa), 8, to_gpu(oracle.pack_int4(qw)))
+    torch.cuda.synchronize()
+    assert np.array_equal(acc.cpu().numpy(), oracle.gemm_i32(qa, qw))
+    assert t4.tint4_get_device_error() == 0
