@@ -1,0 +1,476 @@
+#!/usr/bin/env python3
+"""Benchmark of the packed-INT4 ConvRot quantized linear on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one ConvRot W4A8 linear of the fused-QKV attention projection of a
+diffusion transformer (M = 4608 tokens = 64x64 latent patches + 512 text
+tokens, K = 3072, N = 9216, Hadamard group 256): rotate + quantize the bf16
+activations, stream the packed int4 weights through the tcgen05 int8 GEMM,
+fused dequant to bf16 -- the call a user makes, ``convrot_w4a8_linear``.
+Inputs are seeded synthetic tensors of that shape (x ~ N(0, 1) with 1% of the
+channels x50, W ~ N(0, 0.02) packed offline); L2 is flushed (256 MiB write)
+between timed steps, outside the timed events.
+
+Metric: effective TOPS = 2 M N K / t.  Rank 0 prints one JSON line with the
+roofline of the dominant kernel (the GEMM, int8 tensor-core bound), the CPU
+oracle's throughput on a bounded sample (cpu_baseline), an end-to-end number
+through the same call with pinned host buffers (copies inside the timed
+region) and, under "rows", the other workloads' kernels: the tiny layer, the
+W4A4 variant, the MLP pair (group 64), the small-M W4A16 decode GEMM, and the
+rotate+quantize kernel alone.
+
+Multi-GPU (torchrun): every rank runs the same per-GPU workload on its own
+tokens (independent batches, no exchange: weak scaling); the step time is the
+max over ranks.  ``--impl reference`` times the CPU oracle on the host cores
+instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "ConvRot W4A8/W4A4 linear TOPS & GB/s, % of INT8 TC / HBM roofline, 1xB200"
+MAIN = "dit_qkv_w4a8"
+L2_FLUSH_BYTES = 256 << 20
+INT8_OVER_BF16 = 2.0   # nominal dense int8 : bf16 tensor-core ratio on B200 (4.5 : 2.25 POPS)
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def peaks():
+    """Measured peaks of this machine (driver-written), else the recipe's fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sus=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "int4_weight_quantized_block_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes from a committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(kernel, {}).get(workload)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def bf16_gpu(bits, dev):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+def event_pair():
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+def time_steps(fn, steps, flush=None, dev=None):
+    """Per-step CUDA-event times (ms) of fn() on the current stream, with
+    flush() (untimed) before each step."""
+    times = []
+    for _ in range(steps):
+        if flush is not None:
+            flush()
+        a, b = event_pair()
+        a.record()
+        fn()
+        b.record()
+        times.append((a, b))
+    torch.cuda.synchronize(dev)
+    return [a.elapsed_time(b) for a, b in times]
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, dev):
+    import int4_weight_quantized_block_b200 as t4
+    from int4_weight_quantized_block_b200 import inputs, build as _build
+
+    _build.build()
+    pk = peaks()
+    int8_peak = INT8_OVER_BF16 * pk["bf16"]            # burst: kernels timed one launch at a time
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.zero_()
+
+    w = inputs.WORKLOADS[MAIN]
+    M, N, K, g = w["M"], w["N"], w["K"], w["group"]
+    x_np, W_np = inputs.layer_inputs(MAIN, seed=inputs.SEED + rank)
+    x = bf16_gpu(x_np, dev)
+    wp, sr = t4.tint4_pack_weights(torch.from_numpy(W_np).to(dev), g)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(t4.convrot_linear_workspace_size(M, K, 8), dtype=torch.uint8, device=dev)
+    ops = 2.0 * M * N * K
+
+    def step():
+        t4.convrot_w4a8_linear(x, wp, sr, g, None, y, ws)
+
+    for _ in range(args.warmup):
+        flush()
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        times = time_steps(step, args.steps, flush, dev)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    ms_local = sum(times) / len(times)
+    ms = ms_local
+    if world > 1:
+        t = torch.tensor([ms_local], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * ops / (ms * 1e-3) / 1e12
+
+    # components of the step, timed kernel by kernel (same kernels, two calls)
+    codes = torch.empty((M, K), dtype=torch.int8, device=dev)
+    st = torch.empty((M,), dtype=torch.float32, device=dev)
+    t4.convrot_quantize_act(x, g, 8, codes, st)
+    q_ms = statistics.median(time_steps(lambda: t4.convrot_quantize_act(x, g, 8, codes, st),
+                                        args.steps, flush, dev))
+    gemm_ms = statistics.median(time_steps(lambda: t4.w4a8_gemm(codes, st, wp, sr, None, y),
+                                           args.steps, flush, dev))
+    gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
+
+    # end to end through the same call, pinned host buffers, copies timed
+    x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        t4.convrot_w4a8_linear(x_dev, wp, sr, g, None, y, ws)
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    e2e_ms = statistics.mean(time_steps(e2e_step, max(3, args.steps // 4), flush, dev))
+    e2e_ms_max = e2e_ms
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms_max = float(t.item())
+
+    rows = {}
+    if rank == 0 and not args.no_rows:
+        rows = bench_rows(args, t4, inputs, dev, flush, pk, int8_peak)
+        rows["rotate_quantize_qkv"] = {
+            "kernel": "rotate_quantize_rows_kernel", "us": q_ms * 1e3,
+            "GBps": (M * K * 2 + M * K + M * 4) / (q_ms * 1e-3) / 1e9,
+            "frac_hbm": (M * K * 2 + M * K + M * 4) / (q_ms * 1e-3) / 1e9 / pk["hbm"]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(w, target_s=args.cpu_seconds)
+
+    clocks = clk.summary()
+    traffic = ncu_traffic("w4_gemm_kernel", MAIN)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8",
+        "data": "synthetic (seeded; x ~ N(0,1) with 1% channels x50, W ~ N(0,0.02) packed offline)",
+        "config": {"workload": f"{MAIN}: ConvRot W4A8 fused-QKV projection, M={M} tokens "
+                               f"(64x64 latent + 512 text), K={K}, N={N}, Hadamard group {g}",
+                   "M": M, "N": N, "K": K, "group": g, "act_bits": 8,
+                   "per_gpu_tokens": M, "parallelism": f"independent batches x{world}",
+                   "l2": "flushed (256 MiB write) before every timed step, outside the events"},
+        "roofline": {"bound": "tensor", "kernel": "w4_gemm_kernel (tcgen05 kind::i8)",
+                     "achieved": round(gemm_tops, 2), "peak": round(int8_peak, 1),
+                     "unit": "TOPS", "frac": round(gemm_tops / int8_peak, 4),
+                     "traffic": traffic,
+                     "peak_source": f"{pk['source']}: 2 x bf16 cuBLAS burst "
+                                    f"{pk['bf16']} TFLOP/s (nominal int8:bf16 = 2)",
+                     "kernel_us": round(gemm_ms * 1e3, 2)},
+        "e2e": {"value": round(world * ops / (e2e_ms_max * 1e-3) / 1e12, 3), "unit": "TOPS",
+                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
+                "ms_per_step": round(e2e_ms_max, 4)},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rows:
+        line["rows"] = rows
+    return line
+
+
+def bench_rows(args, t4, inputs, dev, flush, pk, int8_peak):
+    """The other workloads, kernel by kernel (median of CUDA-event times)."""
+    rows = {}
+    reps = max(5, args.steps)
+
+    def gemm_layer(name):
+        w = inputs.WORKLOADS[name]
+        M, N, K, g, bits = w["M"], w["N"], w["K"], w["group"], w["act_bits"]
+        x_np, W_np = inputs.layer_inputs(name)
+        x = bf16_gpu(x_np, dev)
+        wp, sr = t4.tint4_pack_weights(torch.from_numpy(W_np).to(dev), g)
+        codes, st = t4.convrot_quantize_act(x, g, bits)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(t4.convrot_linear_workspace_size(M, K, bits), dtype=torch.uint8, device=dev)
+        gemm = t4.w4a8_gemm if bits == 8 else t4.w4a4_gemm
+        lin = t4.convrot_w4a8_linear if bits == 8 else t4.convrot_w4a4_linear
+        gemm(codes, st, wp, sr, None, y)
+        lin(x, wp, sr, g, None, y, ws)
+        torch.cuda.synchronize(dev)
+        g_ms = statistics.median(time_steps(lambda: gemm(codes, st, wp, sr, None, y), reps, flush, dev))
+        l_ms = statistics.median(time_steps(lambda: lin(x, wp, sr, g, None, y, ws), reps, flush, dev))
+        ops = 2.0 * M * N * K
+        return {"M": M, "N": N, "K": K, "group": g, "act_bits": bits,
+                "gemm_us": round(g_ms * 1e3, 2), "gemm_TOPS": round(ops / g_ms / 1e9, 2),
+                "gemm_frac_int8": round(ops / g_ms / 1e9 / int8_peak, 4),
+                "linear_us": round(l_ms * 1e3, 2), "linear_TOPS": round(ops / l_ms / 1e9, 2)}
+
+    rows["tiny_w4a8"] = gemm_layer("tiny_w4a8")
+    rows["dit_qkv_w4a4"] = gemm_layer("dit_qkv_w4a4")
+    rows["dit_mlp_up_w4a8"] = gemm_layer("dit_mlp_up_w4a8")
+    rows["dit_mlp_down_w4a8"] = gemm_layer("dit_mlp_down_w4a8")
+
+    # W4A16 decode: rotate over 8 weight copies (> L2) so bytes come from HBM
+    w = inputs.WORKLOADS["te_decode_w4a16"]
+    N, K, G = w["N"], w["K"], w["group"]
+    copies = []
+    for c in range(8):
+        op = inputs.w4a16_operands(1, N, K, G, seed=inputs.SEED + 100 + c)
+        copies.append((torch.from_numpy(op.q).to(dev), bf16_gpu(op.scale, dev),
+                       torch.from_numpy(op.zero).to(dev)))
+    for M in w["Ms"]:
+        op = inputs.w4a16_operands(M, N, K, G)
+        x = bf16_gpu(op.x, dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        it = [0]
+
+        def call():
+            q, s, z = copies[it[0] % len(copies)]
+            it[0] += 1
+            t4.w4a16_gemv_gemm(x, q, s, z, G, y)
+
+        for _ in range(8):
+            call()
+        ms = statistics.median(time_steps(call, max(40, reps), None, dev))
+        byts = N * K // 2 + N * (K // G) * 3 + M * K * 2 + M * N * 2
+        rows[f"te_decode_w4a16_M{M}"] = {
+            "kernel": "w4a16_mma_kernel", "M": M, "N": N, "K": K, "group": G,
+            "us": round(ms * 1e3, 2), "GBps": round(byts / ms / 1e6, 1),
+            "frac_hbm": round(byts / ms / 1e6 / pk["hbm"], 4),
+            "l2": "8 weight copies rotated (211 MB > L2)"}
+    return rows
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline / reference arm)
+# ---------------------------------------------------------------------------
+
+def cpu_baseline(w, target_s=15.0, M_sample=None):
+    """Time the oracle (as it stands) on a bounded sample of the workload:
+    the first M_sample tokens against all N weight rows (rotate + quantize,
+    unpack, int32 GEMM, epilogue).  Returns the cpu_baseline object."""
+    import oracle
+    from int4_weight_quantized_block_b200 import inputs
+    oracle.build()
+    M, N, K, g = w["M"], w["N"], w["K"], w["group"]
+    bits = w.get("act_bits", 8)
+    x_np, W_np = inputs.layer_inputs(MAIN, M=M)
+    wp, sr, _ = oracle.pack_weights(W_np, g)
+    if M_sample is None:
+        # calibrate on 8 tokens, then size the sample for ~target_s seconds
+        t0 = time.perf_counter()
+        oracle.convrot_linear(x_np[:8], wp, sr, g, bits)
+        dt = time.perf_counter() - t0
+        M_sample = int(max(8, min(M, 8 * target_s / max(dt, 1e-3))))
+    t0 = time.perf_counter()
+    oracle.convrot_linear(x_np[:M_sample], wp, sr, g, bits)
+    dt = time.perf_counter() - t0
+    ops = 2.0 * M_sample * N * K
+    return {"value": round(ops / dt / 1e12, 6), "unit": "TOPS", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"first {M_sample} of {M} tokens x all {N} rows, K={K} "
+                      f"({dt:.1f} s; C oracle, OpenMP)"}
+
+
+def run_reference(args):
+    from int4_weight_quantized_block_b200 import inputs
+    w = inputs.WORKLOADS[MAIN]
+    M, N, K = w["M"], w["N"], w["K"]
+    per_step_s = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    cal = cpu_baseline(w, target_s=per_step_s)
+    Ms = int(cal["sample"].split()[1])
+    import oracle
+    x_np, W_np = inputs.layer_inputs(MAIN)
+    wp, sr, _ = oracle.pack_weights(W_np, w["group"])
+    for _ in range(args.warmup):
+        oracle.convrot_linear(x_np[:Ms], wp, sr, w["group"], 8)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.convrot_linear(x_np[:Ms], wp, sr, w["group"], 8)
+        times.append(time.perf_counter() - t0)
+    s = sum(times) / len(times)
+    ops = 2.0 * Ms * N * K
+    value = ops / s / 1e12
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(s * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic (seeded)",
+        "config": {"workload": f"{MAIN}: ConvRot W4A8 fused-QKV projection, M={M}, K={K}, "
+                               f"N={N}, group {w['group']}",
+                   "M": M, "N": N, "K": K, "group": w["group"], "act_bits": 8,
+                   "sample_tokens_per_step": Ms},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "kind": "oracle",
+                         "cores": oracle.num_threads(),
+                         "sample": f"first {Ms} of {M} tokens x all {N} rows per step"},
+        "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-rows", action="store_true", help="skip the per-workload rows")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}), flush=True)
+        sys.exit(1)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", device_id=dev,
+                                             timeout=datetime.timedelta(seconds=120))
+    try:
+        line = run_ours(args, rank, world, dev)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -65,9 +65,14 @@ def _load():
             "oracle_gemm_i32": [P, P, I, I, I, P],
             "oracle_gemm_i32_sampled": [P, P, I, P, L, P],
             "oracle_epilogue": [P, P, P, P, I, I, P],
+            "oracle_epilogue_f64": [P, P, P, P, I, I, P],
             "oracle_epilogue_sampled": [P, P, P, P, P, L, P],
+            "oracle_epilogue_sampled_f64": [P, P, P, P, P, L, P],
             "oracle_convrot_linear": [P, P, P, P, I, I, I, I, I, P],
+            "oracle_convrot_linear_f64": [P, P, P, P, I, I, I, I, I, P],
             "oracle_w4a16": [P, P, P, P, I, I, I, I, P],
+            "oracle_w4a16_f64": [P, P, P, P, I, I, I, I, P],
+            "oracle_round_bf16": [P, L, P],
             "oracle_num_threads": [],
         }
         for name, args in sig.items():
@@ -110,6 +115,14 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
 def double_to_bf16_bits(v: float) -> int:
     """Round one double to the nearest bf16 (ties to even), return its bits."""
     return int(_load().oracle_double_to_bf16(float(v)))
+
+
+def round_bf16(v: np.ndarray) -> np.ndarray:
+    """Round an fp64 array to bf16 bits (nearest, ties to even), same shape."""
+    a = _c(v, np.float64)
+    out = np.empty(a.shape, dtype=np.uint16)
+    _check(_load().oracle_round_bf16(_ptr(a), a.size, _ptr(out)), "round_bf16")
+    return out
 
 
 # --------------------------------------------------------------------------
@@ -247,6 +260,30 @@ def epilogue(acc, tok_scale, row_scale, bias_bits=None) -> np.ndarray:
     return y
 
 
+def epilogue_f64(acc, tok_scale, row_scale, bias_bits=None) -> np.ndarray:
+    """The epilogue's value before the bf16 rounding (fp64)."""
+    A = _c(acc, np.int32)
+    M, N = A.shape
+    st, sr = _c(tok_scale, np.float32), _c(row_scale, np.float32)
+    b = None if bias_bits is None else _c(bias_bits, np.uint16)
+    y = np.empty((M, N), dtype=np.float64)
+    _check(_load().oracle_epilogue_f64(_ptr(A), _ptr(st), _ptr(sr), _ptr(b), M, N, _ptr(y)),
+           "epilogue_f64")
+    return y
+
+
+def epilogue_sampled_f64(acc, tok_scale, row_scale, pairs, bias_bits=None) -> np.ndarray:
+    """Unrounded epilogue for selected (m, n) pairs (fp64)."""
+    A = _c(acc, np.int32)
+    st, sr = _c(tok_scale, np.float32), _c(row_scale, np.float32)
+    pr = _c(pairs, np.int64)
+    b = None if bias_bits is None else _c(bias_bits, np.uint16)
+    y = np.empty(pr.shape[0], dtype=np.float64)
+    _check(_load().oracle_epilogue_sampled_f64(_ptr(A), _ptr(st), _ptr(sr), _ptr(b), _ptr(pr),
+                                               pr.shape[0], _ptr(y)), "epilogue_sampled_f64")
+    return y
+
+
 def epilogue_sampled(acc, tok_scale, row_scale, pairs, bias_bits=None) -> np.ndarray:
     """Epilogue for selected (m, n) pairs; acc holds their sums in pair order."""
     A = _c(acc, np.int32)
@@ -273,6 +310,34 @@ def convrot_linear(x_bits, w_packed, row_scale, g, act_bits, bias_bits=None) -> 
     y = np.empty((M, N), dtype=np.uint16)
     _check(_load().oracle_convrot_linear(_ptr(x), _ptr(wp), _ptr(sr), _ptr(b), M, N, K, g,
                                          act_bits, _ptr(y)), "convrot_linear")
+    return y
+
+
+def convrot_linear_f64(x_bits, w_packed, row_scale, g, act_bits, bias_bits=None) -> np.ndarray:
+    """The fused linear's value before the bf16 rounding (fp64)."""
+    x = _c(x_bits, np.uint16)
+    wp = _c(w_packed, np.uint8)
+    sr = _c(row_scale, np.float32)
+    b = None if bias_bits is None else _c(bias_bits, np.uint16)
+    M, K = x.shape
+    N = wp.shape[0]
+    y = np.empty((M, N), dtype=np.float64)
+    _check(_load().oracle_convrot_linear_f64(_ptr(x), _ptr(wp), _ptr(sr), _ptr(b), M, N, K, g,
+                                             act_bits, _ptr(y)), "convrot_linear_f64")
+    return y
+
+
+def w4a16_f64(x_bits, q_packed, scale_bits, zero, group) -> np.ndarray:
+    """The W4A16 layer's value before the bf16 rounding (fp64 accumulation)."""
+    x = _c(x_bits, np.uint16)
+    q = _c(q_packed, np.uint8)
+    s = _c(scale_bits, np.uint16)
+    z = _c(zero, np.uint8)
+    M, K = x.shape
+    N = q.shape[0]
+    y = np.empty((M, N), dtype=np.float64)
+    _check(_load().oracle_w4a16_f64(_ptr(x), _ptr(q), _ptr(s), _ptr(z), M, N, K, group,
+                                    _ptr(y)), "w4a16_f64")
     return y
 
 

@@ -325,44 +325,71 @@ int oracle_gemm_i32_sampled(const int8_t* a, const int8_t* w, int K, const int64
     return ORACLE_OK;
 }
 
-/* Fused dequant: y[m, n] = bf16( acc * s_tok[m] * s_row[n] (+ bias[n]) ),
- * evaluated in fp64 and rounded once.  bias may be NULL. */
-int oracle_epilogue(const int32_t* acc, const float* s_tok, const float* s_row,
-                    const uint16_t* bias, int M, int N, uint16_t* y) {
+/* Fused dequant, unrounded: y[m, n] = acc * s_tok[m] * s_row[n] (+ bias[n]),
+ * evaluated in fp64.  bias may be NULL. */
+int oracle_epilogue_f64(const int32_t* acc, const float* s_tok, const float* s_row,
+                        const uint16_t* bias, int M, int N, double* y) {
     if (!acc || !s_tok || !s_row || !y || M < 0 || N < 0) return ORACLE_BAD_ARG;
 #pragma omp parallel for schedule(static)
     for (int m = 0; m < M; ++m)
         for (int n = 0; n < N; ++n) {
             double v = (double)acc[(long)m * N + n] * (double)s_tok[m] * (double)s_row[n];
             if (bias) v += (double)bf16_bits_to_float(bias[n]);
-            y[(long)m * N + n] = double_to_bf16_bits(v);
+            y[(long)m * N + n] = v;
         }
     return ORACLE_OK;
 }
 
-/* Epilogue for a list of (m, n) pairs with their accumulators. */
-int oracle_epilogue_sampled(const int32_t* acc, const float* s_tok, const float* s_row,
-                            const uint16_t* bias, const int64_t* pairs, long npairs,
-                            uint16_t* y) {
+/* Fused dequant to the layer's bf16 output: the fp64 value above, rounded
+ * once to bf16 (nearest, ties to even). */
+int oracle_epilogue(const int32_t* acc, const float* s_tok, const float* s_row,
+                    const uint16_t* bias, int M, int N, uint16_t* y) {
+    if (!acc || !s_tok || !s_row || !y || M < 0 || N < 0) return ORACLE_BAD_ARG;
+    double* t = (double*)malloc(sizeof(double) * ((size_t)M * N + 1));
+    if (!t) return ORACLE_BAD_ARG;
+    int rc = oracle_epilogue_f64(acc, s_tok, s_row, bias, M, N, t);
+    for (long i = 0; rc == ORACLE_OK && i < (long)M * N; ++i) y[i] = double_to_bf16_bits(t[i]);
+    free(t);
+    return rc;
+}
+
+/* Epilogue for a list of (m, n) pairs with their accumulators, unrounded. */
+int oracle_epilogue_sampled_f64(const int32_t* acc, const float* s_tok, const float* s_row,
+                                const uint16_t* bias, const int64_t* pairs, long npairs,
+                                double* y) {
     if (!acc || !s_tok || !s_row || !pairs || !y || npairs < 0) return ORACLE_BAD_ARG;
     for (long i = 0; i < npairs; ++i) {
         long m = pairs[2 * i], n = pairs[2 * i + 1];
         double v = (double)acc[i] * (double)s_tok[m] * (double)s_row[n];
         if (bias) v += (double)bf16_bits_to_float(bias[n]);
-        y[i] = double_to_bf16_bits(v);
+        y[i] = v;
     }
     return ORACLE_OK;
+}
+
+/* ... and rounded to bf16. */
+int oracle_epilogue_sampled(const int32_t* acc, const float* s_tok, const float* s_row,
+                            const uint16_t* bias, const int64_t* pairs, long npairs,
+                            uint16_t* y) {
+    if (!y || npairs < 0) return ORACLE_BAD_ARG;
+    double* t = (double*)malloc(sizeof(double) * ((size_t)npairs + 1));
+    if (!t) return ORACLE_BAD_ARG;
+    int rc = oracle_epilogue_sampled_f64(acc, s_tok, s_row, bias, pairs, npairs, t);
+    for (long i = 0; rc == ORACLE_OK && i < npairs; ++i) y[i] = double_to_bf16_bits(t[i]);
+    free(t);
+    return rc;
 }
 
 /* ------------------------------------------------------------------------ */
 /* Whole W4A8 / W4A4 linear (twin of convrot_w4a8_linear / ..._w4a4_...)    */
 /* ------------------------------------------------------------------------ */
 
-/* y = bf16( (Q_act(rot(x)) . unpack(w_packed)^T) * s_tok * s_row (+ bias) ).
- * act_bits 8 or 4; g the rotation group (0: none).  Scratch is allocated here. */
-int oracle_convrot_linear(const uint16_t* x, const uint8_t* w_packed, const float* row_scale,
-                          const uint16_t* bias, int M, int N, int K, int g, int act_bits,
-                          uint16_t* y) {
+/* y = (Q_act(rot(x)) . unpack(w_packed)^T) * s_tok * s_row (+ bias), unrounded
+ * (fp64).  act_bits 8 or 4; g the rotation group (0: none).  Scratch is
+ * allocated here. */
+int oracle_convrot_linear_f64(const uint16_t* x, const uint8_t* w_packed, const float* row_scale,
+                              const uint16_t* bias, int M, int N, int K, int g, int act_bits,
+                              double* y) {
     if (!x || !w_packed || !row_scale || !y || M < 0 || N <= 0 || K <= 0) return ORACLE_BAD_ARG;
     int8_t* qa = (int8_t*)malloc((size_t)M * K + 1);
     int8_t* qw = (int8_t*)malloc((size_t)N * K + 1);
@@ -373,7 +400,7 @@ int oracle_convrot_linear(const uint16_t* x, const uint8_t* w_packed, const floa
         rc = oracle_quantize_act(x, M, K, g, act_bits, qa, st, NULL);
         if (rc == ORACLE_OK) rc = oracle_unpack_int4(w_packed, N, K, qw);
         if (rc == ORACLE_OK) rc = oracle_gemm_i32(qa, qw, M, N, K, acc);
-        if (rc == ORACLE_OK) rc = oracle_epilogue(acc, st, row_scale, bias, M, N, y);
+        if (rc == ORACLE_OK) rc = oracle_epilogue_f64(acc, st, row_scale, bias, M, N, y);
     }
     free(qa);
     free(qw);
@@ -382,15 +409,28 @@ int oracle_convrot_linear(const uint16_t* x, const uint8_t* w_packed, const floa
     return rc;
 }
 
+/* The layer's bf16 output: the value above rounded once to bf16. */
+int oracle_convrot_linear(const uint16_t* x, const uint8_t* w_packed, const float* row_scale,
+                          const uint16_t* bias, int M, int N, int K, int g, int act_bits,
+                          uint16_t* y) {
+    if (!y || M < 0 || N <= 0) return ORACLE_BAD_ARG;
+    double* t = (double*)malloc(sizeof(double) * ((size_t)M * N + 1));
+    if (!t) return ORACLE_BAD_ARG;
+    int rc = oracle_convrot_linear_f64(x, w_packed, row_scale, bias, M, N, K, g, act_bits, t);
+    for (long i = 0; rc == ORACLE_OK && i < (long)M * N; ++i) y[i] = double_to_bf16_bits(t[i]);
+    free(t);
+    return rc;
+}
+
 /* ------------------------------------------------------------------------ */
 /* W4A16 group-wise asymmetric linear (twin of w4a16_gemv_gemm)             */
 /* ------------------------------------------------------------------------ */
 
-/* y[m, n] = bf16( sum_k x[m, k] * (q[n, k] - z[n, k/G]) * s[n, k/G] ) with
+/* y[m, n] = sum_k x[m, k] * (q[n, k] - z[n, k/G]) * s[n, k/G], unrounded, with
  * q uint4 packed low-first in uint8 [N, K/2], s bf16 [N, K/G], z uint8
  * [N, K/G] holding 0..15.  fp64 accumulation. */
-int oracle_w4a16(const uint16_t* x, const uint8_t* q, const uint16_t* s, const uint8_t* z,
-                 int M, int N, int K, int G, uint16_t* y) {
+int oracle_w4a16_f64(const uint16_t* x, const uint8_t* q, const uint16_t* s, const uint8_t* z,
+                     int M, int N, int K, int G, double* y) {
     if (!x || !q || !s || !z || !y || M < 0 || N < 0 || K <= 0 || G <= 0 || K % G || K % 2)
         return ORACLE_BAD_ARG;
     int ng = K / G;
@@ -405,8 +445,27 @@ int oracle_w4a16(const uint16_t* x, const uint8_t* q, const uint16_t* s, const u
                            (double)bf16_bits_to_float(s[(long)n * ng + k / G]);
                 acc += (double)bf16_bits_to_float(x[(long)m * K + k]) * w;
             }
-            y[(long)m * N + n] = double_to_bf16_bits(acc);
+            y[(long)m * N + n] = acc;
         }
+    return ORACLE_OK;
+}
+
+/* The same, rounded once to bf16: the layer's output. */
+int oracle_w4a16(const uint16_t* x, const uint8_t* q, const uint16_t* s, const uint8_t* z,
+                 int M, int N, int K, int G, uint16_t* y) {
+    if (!y || M < 0 || N < 0) return ORACLE_BAD_ARG;
+    double* t = (double*)malloc(sizeof(double) * ((size_t)M * N + 1));
+    if (!t) return ORACLE_BAD_ARG;
+    int rc = oracle_w4a16_f64(x, q, s, z, M, N, K, G, t);
+    for (long i = 0; rc == ORACLE_OK && i < (long)M * N; ++i) y[i] = double_to_bf16_bits(t[i]);
+    free(t);
+    return rc;
+}
+
+/* Round an array of doubles to bf16 bits (nearest, ties to even). */
+int oracle_round_bf16(const double* v, long n, uint16_t* out) {
+    if (!v || !out || n < 0) return ORACLE_BAD_ARG;
+    for (long i = 0; i < n; ++i) out[i] = double_to_bf16_bits(v[i]);
     return ORACLE_OK;
 }
 

@@ -4,7 +4,10 @@ Every test feeds the same seeded inputs to both sides.  Bars:
   * packed weight bytes and int32 accumulators: bit-exact;
   * activation codes: equal except at rounding ties (<= 1e-4 of elements,
     each off by at most 1) -- both sides decide them in fp32;
-  * bf16 outputs: max |gpu - oracle| / rms(oracle) <= 1e-2.
+  * bf16 outputs: max |gpu - oracle| / rms(oracle) <= 1e-2, where a one-ulp
+    difference counts as a rounding tie (not an error) when the oracle's fp64
+    value lies within the kernel's fp32 evaluation error of the bf16 rounding
+    midpoint; ties must stay below 1e-3 of the outputs (oracle/compare.py).
 Small cases span several tiles and ragged tails in M, N and K; the full-size
 workloads are checked on sampled outputs the oracle computes one by one.
 """
@@ -15,8 +18,15 @@ import torch
 import oracle
 import int4_weight_quantized_block_b200 as t4
 from int4_weight_quantized_block_b200 import inputs
-from gpu_util import (CODE_MISMATCH_FRAC, Y_TOL, bf16_from_gpu, bf16_to_gpu, code_mismatch,
-                      dev, rel_err, to_gpu)
+from oracle.compare import accumulation_error, check_bf16, gemm_eval_error
+from gpu_util import CODE_MISMATCH_FRAC, bf16_from_gpu, bf16_to_gpu, code_mismatch, dev, to_gpu
+
+
+def assert_gemm_output(y_gpu_bits, ref64, bias_bits=None):
+    b64 = None if bias_bits is None else oracle.bf16_bits_to_f32(bias_bits).astype(np.float64)
+    c = check_bf16(y_gpu_bits, ref64, gemm_eval_error(ref64, b64))
+    assert c.ok, str(c)
+
 
 pytestmark = pytest.mark.gpu
 
@@ -94,7 +104,7 @@ def test_gemm_bf16_epilogue(M, N, K, act_bits, with_bias):
     st = inputs.positive_scales(M, seed=402)
     sr = inputs.positive_scales(N, seed=403)
     bias = inputs.f32_to_bf16_bits(np.linspace(-3, 3, N)) if with_bias else None
-    y_ref = oracle.epilogue(oracle.gemm_i32(qa, qw), st, sr, bias)
+    y_ref = oracle.epilogue_f64(oracle.gemm_i32(qa, qw), st, sr, bias)
     wp = oracle.pack_int4(qw)
     b = bf16_to_gpu(bias) if with_bias else None
     if act_bits == 8:
@@ -102,7 +112,7 @@ def test_gemm_bf16_epilogue(M, N, K, act_bits, with_bias):
     else:
         y = t4.w4a4_gemm(to_gpu(oracle.pack_int4(qa)), to_gpu(st), to_gpu(wp), to_gpu(sr), b)
     torch.cuda.synchronize()
-    assert rel_err(bf16_from_gpu(y), y_ref) <= Y_TOL
+    assert_gemm_output(bf16_from_gpu(y), y_ref, np.broadcast_to(bias, (M, N)) if with_bias else None)
 
 
 # ------------------------------------------------------------------ fused linear
@@ -114,11 +124,11 @@ def test_convrot_linear_small(M, N, K, g, act_bits):
     x = inputs.activations(M, K, seed=500 + K)
     W = inputs.weights(N, K, seed=501 + N)
     wp, sr, _ = oracle.pack_weights(W, g)
-    y_ref = oracle.convrot_linear(x, wp, sr, g, act_bits)
+    y_ref = oracle.convrot_linear_f64(x, wp, sr, g, act_bits)
     fn = t4.convrot_w4a8_linear if act_bits == 8 else t4.convrot_w4a4_linear
     y = fn(bf16_to_gpu(x), to_gpu(wp), to_gpu(sr), g)
     torch.cuda.synchronize()
-    assert rel_err(bf16_from_gpu(y), y_ref) <= Y_TOL
+    assert_gemm_output(bf16_from_gpu(y), y_ref)
 
 
 def test_quantized_linear_module_end_to_end():
@@ -131,7 +141,7 @@ def test_quantized_linear_module_end_to_end():
     wp, sr, _ = oracle.pack_weights(W, g)
     torch.cuda.synchronize()
     assert np.array_equal(lin.w_packed.cpu().numpy(), wp)
-    assert rel_err(bf16_from_gpu(y), oracle.convrot_linear(x, wp, sr, g, 8)) <= Y_TOL
+    assert_gemm_output(bf16_from_gpu(y), oracle.convrot_linear_f64(x, wp, sr, g, 8))
 
 
 def _sample_pairs(M, N, n, seed):
@@ -167,9 +177,9 @@ def test_full_size_workloads_sampled(name):
     assert np.array_equal(st.cpu().numpy().view(np.uint32), st_ref.view(np.uint32))
     pairs = _sample_pairs(M, N, 4096, seed=9)
     acc = oracle.gemm_i32_sampled(qa_ref, qw_ref, pairs)
-    y_ref = oracle.epilogue_sampled(acc, st_ref, sr_ref, pairs)
+    y_ref = oracle.epilogue_sampled_f64(acc, st_ref, sr_ref, pairs)
     y_gpu = bf16_from_gpu(y)[pairs[:, 0], pairs[:, 1]]
-    assert rel_err(y_gpu, y_ref) <= Y_TOL
+    assert_gemm_output(y_gpu, y_ref)
     # int32 accumulators of the same codes, bit-exact on the samples
     a = to_gpu(qa_ref) if bits == 8 else to_gpu(oracle.pack_int4(qa_ref))
     acc_gpu = t4.tint4_debug_int32_gemm(a, bits, to_gpu(wp_ref))
@@ -183,22 +193,24 @@ def test_full_size_workloads_sampled(name):
                                    (9, 128, 4096), (64, 64, 256), (33, 96, 512)])
 def test_w4a16(M, N, K):
     op = inputs.w4a16_operands(M, N, K, 128, seed=600 + M)
-    y_ref = oracle.w4a16(op.x, op.q, op.scale, op.zero, 128)
+    y_ref = oracle.w4a16_f64(op.x, op.q, op.scale, op.zero, 128)
     y = t4.w4a16_gemv_gemm(bf16_to_gpu(op.x), to_gpu(op.q), bf16_to_gpu(op.scale),
                            to_gpu(op.zero), 128)
     torch.cuda.synchronize()
-    assert rel_err(bf16_from_gpu(y), y_ref) <= Y_TOL
+    c = check_bf16(bf16_from_gpu(y), y_ref, accumulation_error(y_ref))
+    assert c.ok, str(c)
 
 
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_w4a16_full_size(M):
     w = inputs.WORKLOADS["te_decode_w4a16"]
     op = inputs.w4a16_operands(M, w["N"], w["K"], w["group"])
-    y_ref = oracle.w4a16(op.x, op.q, op.scale, op.zero, w["group"])
+    y_ref = oracle.w4a16_f64(op.x, op.q, op.scale, op.zero, w["group"])
     y = t4.w4a16_gemv_gemm(bf16_to_gpu(op.x), to_gpu(op.q), bf16_to_gpu(op.scale),
                            to_gpu(op.zero), w["group"])
     torch.cuda.synchronize()
-    assert rel_err(bf16_from_gpu(y), y_ref) <= Y_TOL
+    c = check_bf16(bf16_from_gpu(y), y_ref, accumulation_error(y_ref))
+    assert c.ok, str(c)
 
 
 # ------------------------------------------------------------------ edge cases

@@ -393,3 +393,49 @@ def test_w4a16_general_dequant():
     for m in range(M):
         for n in range(N):
             assert y[m, n] == _bf16_nearest_even(float(ref[m, n]))
+
+
+# ---------------------------------------------------------------- fp64 outputs and the comparison
+
+def test_unrounded_outputs_round_to_the_bf16_outputs():
+    """The bf16 outputs are exactly the fp64 values rounded once."""
+    g = 64
+    x = inputs.activations(6, 128, seed=41)
+    W = inputs.weights(32, 128, seed=42)
+    wp, sr, _ = oracle.pack_weights(W, g)
+    y64 = oracle.convrot_linear_f64(x, wp, sr, g, 8)
+    assert np.array_equal(oracle.round_bf16(y64), oracle.convrot_linear(x, wp, sr, g, 8))
+    op = inputs.w4a16_operands(3, 32, 256, 128, seed=43)
+    w64 = oracle.w4a16_f64(op.x, op.q, op.scale, op.zero, 128)
+    assert np.array_equal(oracle.round_bf16(w64), oracle.w4a16(op.x, op.q, op.scale, op.zero, 128))
+    for v in w64.ravel()[:50]:
+        assert oracle.double_to_bf16_bits(v) == oracle.round_bf16(np.array([v]))[0]
+
+
+def test_compare_flags_errors_and_accepts_ties():
+    from oracle.compare import check_bf16
+    ref = np.array([1.0, 2.0, -3.0, 0.5], np.float64)
+    exact = oracle.round_bf16(ref)
+    c = check_bf16(exact, ref, 1e-9)
+    assert c.ok and c.max_rel == 0 and c.ties == 0
+    # a one-ulp difference far from any midpoint is an error, not a tie
+    off = exact.copy()
+    off[1] += 1
+    c = check_bf16(off, ref, 1e-9)
+    assert c.ties == 0 and c.max_rel == pytest.approx(2.0 ** -6 / np.sqrt(np.mean(ref ** 2)))
+    off[1] += 1                                  # two ulps at 2.0: over the tolerance
+    c = check_bf16(off, ref, 1e-9)
+    assert c.ties == 0 and c.max_rel > 1e-2 and not c.ok
+    # a value sitting on a rounding midpoint: either neighbour is a tie
+    mid = 1.0 + 2.0 ** -8                       # halfway between 1 and 1 + 2^-7
+    ref2 = np.full(2000, 1.0)
+    ref2[0] = mid
+    g = oracle.round_bf16(ref2)
+    g[0] = oracle.double_to_bf16_bits(1.0 + 2.0 ** -7)   # the other neighbour
+    c = check_bf16(g, ref2, 1e-6)
+    assert c.ties == 1 and c.max_rel == 0 and c.ok
+    # too many ties fail
+    ref3 = np.full(100, mid)
+    g3 = np.full(100, oracle.double_to_bf16_bits(1.0 + 2.0 ** -7), np.uint16)
+    c = check_bf16(g3, ref3, 1e-6)
+    assert c.ties == 100 and not c.ok
