@@ -57,12 +57,13 @@ def check_bf16(gpu_bits: np.ndarray, ref_f64: np.ndarray, err_abs) -> Bf16Check:
 
     err_abs: bound (scalar or per element) on the fp32 evaluation error of
     the value before its bf16 rounding."""
+    ref_arr = np.asarray(ref_f64, np.float64)
     g_bits = np.asarray(gpu_bits, np.uint16).ravel()
-    ref = np.asarray(ref_f64, np.float64).ravel()
+    ref = ref_arr.ravel()
     o_bits = round_bf16(ref)
     g = bits_to_f64(g_bits)
     o = bits_to_f64(o_bits)
-    err = np.broadcast_to(np.asarray(err_abs, np.float64), ref.shape).ravel()
+    err = np.broadcast_to(np.asarray(err_abs, np.float64), ref_arr.shape).ravel()
     differ = g_bits != o_bits
     adjacent = np.abs(_order_key(g_bits) - _order_key(o_bits)) == 1
     tie = differ & adjacent & (np.abs(ref - 0.5 * (g + o)) <= err)

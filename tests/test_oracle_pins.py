@@ -439,3 +439,20 @@ def test_compare_flags_errors_and_accepts_ties():
     g3 = np.full(100, oracle.double_to_bf16_bits(1.0 + 2.0 ** -7), np.uint16)
     c = check_bf16(g3, ref3, 1e-6)
     assert c.ties == 100 and not c.ok
+
+
+def test_compare_accepts_2d_inputs_and_error_arrays():
+    from oracle.compare import check_bf16, gemm_eval_error, accumulation_error
+    g = 16
+    x = inputs.activations(8, 64, seed=44)
+    W = inputs.weights(32, 64, seed=45)
+    wp, sr, _ = oracle.pack_weights(W, g)
+    y64 = oracle.convrot_linear_f64(x, wp, sr, g, 8)
+    y = oracle.convrot_linear(x, wp, sr, g, 8)
+    c = check_bf16(y, y64, gemm_eval_error(y64))
+    assert c.ok and c.ties == 0 and c.max_rel == 0
+    c = check_bf16(y, y64, accumulation_error(y64))
+    assert c.ok
+    bias = np.broadcast_to(inputs.f32_to_bf16_bits(np.ones(32)), (8, 32))
+    c = check_bf16(y, y64, gemm_eval_error(y64, oracle.bf16_bits_to_f32(bias)))
+    assert c.ok
