@@ -9,19 +9,18 @@
 //
 // The cost is streaming the packed weights from HBM (0.5 byte per weight plus
 // 3 bytes of scale and zero point per 128 weights).  Per group the sum is
-// split as
-//   s * ( sum_k x_k * (128 + q_k)  -  (128 + z) * sum_k x_k )
-// so the weights enter the multiply as the exact bf16 values 128 + q, which
-// one AND/OR per two nibbles makes from the packed bytes (0x4300 | q is
-// bf16(128 + q)); the per-token group sums of x cost one shuffle reduction
-// per group.  The products run on the warp-level bf16 tensor-core MMA
-// (m16n8k16, fp32 accumulation): at M = 16 the 805 M multiply-adds of the
-// 4096 x 12288 layer would take several times the HBM time on the fp32 CUDA
-// cores.  Weights form the MMA's A operand straight from registers (16 rows x
-// 128 K per warp step, one 16-byte load per lane and row), tokens the B
-// operand (n = 8 per block).  The K order inside an MMA is permuted so that
-// each lane's 32 packed nibbles map onto its own fragment slots; x is
-// gathered in the same order, which leaves each dot product unchanged.
+//   s * sum_k x_k * (q_k - z)
+// with q_k - z formed exactly in bf16: 0x4300 | q is bf16(128 + q), one
+// AND/OR per two nibbles from the packed bytes, and subtracting bf16(128 + z)
+// leaves the small integer q - z, exact.  The products run on the warp-level
+// bf16 tensor-core MMA (m16n8k16, fp32 accumulation): at M = 16 the 805 M
+// multiply-adds of the 4096 x 12288 layer would take several times the HBM
+// time on the fp32 CUDA cores.  Weights form the MMA's A operand straight
+// from registers (16 rows x 128 K per warp step, one 16-byte load per lane
+// and row), tokens the B operand (n = 8 per block).  The K order inside an
+// MMA is permuted so that each lane's 32 packed nibbles map onto its own
+// fragment slots; x is gathered in the same order, which leaves each dot
+// product unchanged.
 //
 // CTA = 4 warps on the same 16 weight rows; warp w takes the K groups w,
 // w + 4, ...; the 4 partial results meet in shared memory.
@@ -51,8 +50,12 @@ __device__ __forceinline__ uint32_t nib_pair_bf16(uint32_t w, int i) {
     return ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
 }
 
-__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+// elementwise a - b of two bf16 pairs (exact here: small integers)
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
 
 // NB = number of 8-token blocks (M <= 8 * NB).
 template <int NB>
@@ -99,16 +102,27 @@ w4a16_mma_kernel(const __nv_bfloat16* __restrict__ x, const uint8_t* __restrict_
             if (G >= ngroups) break;  // warp-uniform
             const float sA = __bfloat162float(wscale[static_cast<size_t>(rowA) * ngroups + G]);
             const float sB = __bfloat162float(wscale[static_cast<size_t>(rowB) * ngroups + G]);
-            const float zA = 128.0f + static_cast<float>(wzero[static_cast<size_t>(rowA) * ngroups + G]);
-            const float zB = 128.0f + static_cast<float>(wzero[static_cast<size_t>(rowB) * ngroups + G]);
+            // bf16x2 (128 + z, 128 + z): subtracting it from (128 + q) leaves q - z exactly
+            const uint32_t zA = 0x43004300u | (0x00010001u * wzero[static_cast<size_t>(rowA) * ngroups + G]);
+            const uint32_t zB = 0x43004300u | (0x00010001u * wzero[static_cast<size_t>(rowB) * ngroups + G]);
             const uint32_t wa[4] = {pa[u].x, pa[u].y, pa[u].z, pa[u].w};
             const uint32_t wb[4] = {pb[u].x, pb[u].y, pb[u].z, pb[u].w};
+            // dequantized A fragments (q - z in bf16), shared by every token block
+            uint32_t afr[8][4];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int w = j >> 1;          // packed word of this lane's 16 bytes
+                const int i0 = 2 * (j & 1);    // nibble pairs (i0, i0+4) and (i0+1, i0+5)
+                afr[j][0] = bf16x2_sub(nib_pair_bf16(wa[w], i0), zA);      // row g,   k 2t, 2t+1
+                afr[j][1] = bf16x2_sub(nib_pair_bf16(wb[w], i0), zB);      // row g+8, k 2t, 2t+1
+                afr[j][2] = bf16x2_sub(nib_pair_bf16(wa[w], i0 + 1), zA);  // row g,   k 2t+8, 2t+9
+                afr[j][3] = bf16x2_sub(nib_pair_bf16(wb[w], i0 + 1), zB);  // row g+8, k 2t+8, 2t+9
+            }
 #pragma unroll
             for (int b = 0; b < NB; ++b) {
                 // x[token 8b + g][G*128 + 32t .. +31]
                 const int tok = 8 * b + g;
                 uint32_t xw[16];
-                float xs = 0.0f;
                 if (tok < M) {
                     const uint4* xp = reinterpret_cast<const uint4*>(
                         x + static_cast<size_t>(tok) * K + G * kW16Group + 32 * t);
@@ -117,42 +131,28 @@ w4a16_mma_kernel(const __nv_bfloat16* __restrict__ x, const uint8_t* __restrict_
                         const uint4 q = __ldg(xp + v);
                         xw[4 * v] = q.x; xw[4 * v + 1] = q.y; xw[4 * v + 2] = q.z; xw[4 * v + 3] = q.w;
                     }
-#pragma unroll
-                    for (int v = 0; v < 16; ++v) xs += bf16lo(xw[v]) + bf16hi(xw[v]);
                 } else {
 #pragma unroll
                     for (int v = 0; v < 16; ++v) xw[v] = 0u;
                 }
-                // group sum of x for token 8b + g, then fetch the sums of the
-                // two token columns this lane accumulates (8b + 2t, 8b + 2t + 1)
-                xs += __shfl_xor_sync(0xFFFFFFFFu, xs, 1);
-                xs += __shfl_xor_sync(0xFFFFFFFFu, xs, 2);
-                const float xs0 = __shfl_sync(0xFFFFFFFFu, xs, (2 * t) * 4);
-                const float xs1 = __shfl_sync(0xFFFFFFFFu, xs, (2 * t + 1) * 4);
-
                 float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    const int w = j >> 1;          // packed word of this lane's 16 bytes
-                    const int i0 = 2 * (j & 1);    // nibble pair (i0, i0+4) and (i0+1, i0+5)
-                    uint32_t a[4];
-                    a[0] = nib_pair_bf16(wa[w], i0);       // row g,   virtual k 2t, 2t+1
-                    a[1] = nib_pair_bf16(wb[w], i0);       // row g+8, virtual k 2t, 2t+1
-                    a[2] = nib_pair_bf16(wa[w], i0 + 1);   // row g,   virtual k 2t+8, 2t+9
-                    a[3] = nib_pair_bf16(wb[w], i0 + 1);   // row g+8, virtual k 2t+8, 2t+9
-                    // x values 8w + (0..7) of this lane's slice, paired the same way
+                    const int w = j >> 1;
+                    const int i0 = 2 * (j & 1);
+                    // x values 8w + (0..7) of this lane's slice, paired like the nibbles
                     const uint32_t X0 = xw[4 * w + (i0 >> 1)];       // x[8w+i0],   x[8w+i0+1]
                     const uint32_t X2 = xw[4 * w + 2 + (i0 >> 1)];   // x[8w+i0+4], x[8w+i0+5]
                     const uint32_t b0 = __byte_perm(X0, X2, 0x5410);  // (x[i0],   x[i0+4])
                     const uint32_t b1 = __byte_perm(X0, X2, 0x7632);  // (x[i0+1], x[i0+5])
-                    mma_bf16_16816(acc, a, b0, b1);
+                    mma_bf16_16816(acc, afr[j], b0, b1);
                 }
                 // acc: [0] row g / token 8b+2t, [1] row g / 8b+2t+1,
                 //      [2] row g+8 / 8b+2t,     [3] row g+8 / 8b+2t+1
-                total[b][0] += sA * (acc[0] - zA * xs0);
-                total[b][1] += sA * (acc[1] - zA * xs1);
-                total[b][2] += sB * (acc[2] - zB * xs0);
-                total[b][3] += sB * (acc[3] - zB * xs1);
+                total[b][0] = fmaf(sA, acc[0], total[b][0]);
+                total[b][1] = fmaf(sA, acc[1], total[b][1]);
+                total[b][2] = fmaf(sB, acc[2], total[b][2]);
+                total[b][3] = fmaf(sB, acc[3], total[b][3]);
             }
         }
     }

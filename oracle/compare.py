@@ -18,7 +18,14 @@ import numpy as np
 from . import round_bf16
 
 Y_TOL = 1e-2          # max |gpu - oracle| / rms(oracle) outside ties
-TIE_FRAC = 1e-3       # at most this fraction of outputs may be rounding ties
+# At most this fraction of outputs may be rounding ties.  An fp32 evaluation
+# with relative error e disagrees with the exact rounding on about
+# 2 e / 2^-8 of the outputs: e ~ 2^-23 for the integer GEMM's epilogue (two
+# or three fp32 roundings of an exact int32 sum) gives ~6e-5, bounded here by
+# 1e-3; e ~ 1e-5 for fp32 dot products of K = 4096 summed on the tensor cores
+# gives ~5e-3, the bound the W4A16 tests pass explicitly.
+TIE_FRAC = 1e-3
+TIE_FRAC_ACCUMULATED = 5e-3
 
 
 def bits_to_f64(b: np.ndarray) -> np.ndarray:
@@ -38,6 +45,7 @@ class Bf16Check:
     ties: int             # one-ulp differences at rounding midpoints
     n: int
     worst_index: int
+    tie_limit: float = TIE_FRAC
 
     @property
     def tie_frac(self) -> float:
@@ -45,14 +53,15 @@ class Bf16Check:
 
     @property
     def ok(self) -> bool:
-        return self.max_rel <= Y_TOL and self.tie_frac <= TIE_FRAC
+        return self.max_rel <= Y_TOL and self.tie_frac <= self.tie_limit
 
     def __str__(self):
         return (f"max|diff|/rms={self.max_rel:.3e} (tol {Y_TOL}), ties={self.ties}/{self.n} "
-                f"(<= {TIE_FRAC:g}), worst at {self.worst_index}")
+                f"(<= {self.tie_limit:g}), worst at {self.worst_index}")
 
 
-def check_bf16(gpu_bits: np.ndarray, ref_f64: np.ndarray, err_abs) -> Bf16Check:
+def check_bf16(gpu_bits: np.ndarray, ref_f64: np.ndarray, err_abs,
+               tie_limit: float = TIE_FRAC) -> Bf16Check:
     """Compare bf16 results (bits) with the oracle's unrounded fp64 values.
 
     err_abs: bound (scalar or per element) on the fp32 evaluation error of
@@ -72,7 +81,8 @@ def check_bf16(gpu_bits: np.ndarray, ref_f64: np.ndarray, err_abs) -> Bf16Check:
     worst = int(np.argmax(d)) if d.size else -1
     dmax = float(d.max()) if d.size else 0.0
     max_rel = dmax / rms if rms > 0 else dmax
-    return Bf16Check(max_rel=max_rel, ties=int(tie.sum()), n=int(ref.size), worst_index=worst)
+    return Bf16Check(max_rel=max_rel, ties=int(tie.sum()), n=int(ref.size), worst_index=worst,
+                     tie_limit=tie_limit)
 
 
 def gemm_eval_error(ref_f64: np.ndarray, bias_f64=None) -> np.ndarray:
