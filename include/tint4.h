@@ -145,6 +145,32 @@ tint4_status convrot_w4a4_linear(const tint4_bf16* x, const uint8_t* w_packed,
                                  size_t workspace_bytes, void* stream);
 
 /*
+ * convrot_w4a8_linear without a caller-provided workspace, for callers that
+ * cannot allocate device memory at the point of the call: code that runs
+ * inside a fixed memory budget, a host program without a device allocator
+ * of its own, or a plug-in whose host application owns every allocation.
+ * (The pages have no counterpart: it is a packaging of the same layer.)
+ * The activation codes and token scales go to one fixed 16 MiB device array
+ * inside this library, which every GPU that loads the library holds until
+ * the process exits.  Inputs and outputs are as convrot_w4a8_linear; the
+ * caller still owns x, w_packed, row_scale, bias and y.
+ *   - Sizes: M * K + 4 * M bytes (each rounded up to 256) must fit in
+ *     16 MiB, else TINT4_ERR_WORKSPACE is returned and nothing is launched.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - No allocation: the call makes no cudaMalloc / cudaFree and calls no
+ *     allocating routine.
+ *   - Every call on a device shares the one array, and it keeps whatever the
+ *     last call left in it (nothing in it needs to start at zero).  Calls
+ *     whose work overlaps on the GPU (two streams, or two host threads)
+ *     race on it and corrupt each other's results: serialize them.
+ */
+tint4_status convrot_w4a8_linear_noalloc(const tint4_bf16* x, const uint8_t* w_packed,
+                                         const float* row_scale, const tint4_bf16* bias,
+                                         tint4_bf16* y, int M, int N, int K, int group,
+                                         void* stream);
+
+/*
  * W4A16 group-wise asymmetric linear for small M ("TINT4 v1.2", "v1.1 新特性
  * > 5" _qdata/_scale/_zp, "参数选择指南" group 128; "ComfyUI-INT-Crush",
  * "Inference > INT4 > Triton backend" W4A16).  x bf16 [M, K]; w_q uint8

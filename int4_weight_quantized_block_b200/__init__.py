@@ -25,6 +25,7 @@ __all__ = [
     "convrot_linear_workspace_size",
     "convrot_w4a8_linear",
     "convrot_w4a4_linear",
+    "convrot_w4a8_linear_noalloc",
     "w4a16_gemv_gemm",
     "tint4_debug_int32_gemm",
     "tint4_debug_bounded_wait",
@@ -162,6 +163,25 @@ def convrot_w4a8_linear(x, w_packed, row_scale, group, bias=None, y=None, worksp
 def convrot_w4a4_linear(x, w_packed, row_scale, group, bias=None, y=None, workspace=None):
     """Fused rotate + int4 quantize + W4A4 GEMM: bf16 x [M, K] -> bf16 y [M, N]."""
     return _linear("convrot_w4a4_linear", 4, x, w_packed, row_scale, group, bias, y, workspace)
+
+
+def convrot_w4a8_linear_noalloc(x, w_packed, row_scale, group, bias=None, y=None):
+    """convrot_w4a8_linear whose scratch is the library's fixed 16 MiB device
+    array instead of a caller workspace (for callers that cannot allocate
+    device memory).  Calls that overlap on the GPU race on that array."""
+    _need(x, "x", torch.bfloat16)
+    M, K = x.shape
+    N = w_packed.shape[0]
+    _need(w_packed, "w_packed", torch.uint8, (N, K // 2))
+    _need(row_scale, "row_scale", torch.float32, (N,))
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, (N,))
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(y, "y", torch.bfloat16, (M, N))
+    _native.call("convrot_w4a8_linear_noalloc", _ptr(x), _ptr(w_packed), _ptr(row_scale),
+                 _ptr(bias), _ptr(y), M, N, K, group, _stream(x.device))
+    return y
 
 
 def w4a16_gemv_gemm(x, w_q, scale, zero, group: int = 128, y=None) -> torch.Tensor:

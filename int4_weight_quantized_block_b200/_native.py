@@ -39,6 +39,7 @@ SIGNATURES = {
     "convrot_linear_workspace_size": (SZ, [I, I, I]),
     "convrot_w4a8_linear": (I, [P, P, P, P, P, I, I, I, I, P, SZ, P]),
     "convrot_w4a4_linear": (I, [P, P, P, P, P, I, I, I, I, P, SZ, P]),
+    "convrot_w4a8_linear_noalloc": (I, [P, P, P, P, P, I, I, I, I, P]),
     "w4a16_gemv_gemm": (I, [P, P, P, P, I, P, I, I, I, P]),
     "tint4_debug_int32_gemm": (I, [P, I, P, P, I, I, I, P]),
     "tint4_debug_bounded_wait": (I, [U64, P]),

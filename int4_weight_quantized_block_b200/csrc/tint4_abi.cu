@@ -277,6 +277,36 @@ __global__ void bounded_wait_test_kernel(uint64_t limit_ns) {
     }
 }
 
+// ------------------------------------------------------------------ allocation-free fused linear
+//
+// For callers that cannot allocate device memory: the scratch of the fused
+// W4A8 linear (activation codes + token scales) lives in one fixed device
+// array that every device holds from the moment it loads this library until
+// the process exits.  Host code must not hand the array's name to a kernel
+// (on the host it is only a stand-in for the symbol); its device address is
+// looked up once per device with cudaGetSymbolAddress.
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;   // 16 MiB
+static __device__ __align__(256) uint8_t g_static_linear_scratch[kStaticScratchBytes];
+
+std::mutex g_static_scratch_mu;
+void* g_static_scratch_ptr[kMaxDevices];
+
+// Device address of the scratch array on `dev` (the current device); the
+// first call on a device resolves it.  nullptr on failure.
+void* static_scratch_address(int dev) {
+    std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+    if (g_static_scratch_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_linear_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        g_static_scratch_ptr[dev] = p;
+    }
+    return g_static_scratch_ptr[dev];
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -358,6 +388,34 @@ tint4_status convrot_w4a4_linear(const tint4_bf16* x, const uint8_t* w_packed,
                                  size_t workspace_bytes, void* stream) {
     return linear_entry(4, x, w_packed, row_scale, bias, y, M, N, K, group, workspace,
                         workspace_bytes, stream);
+}
+
+tint4_status convrot_w4a8_linear_noalloc(const tint4_bf16* x, const uint8_t* w_packed,
+                                         const float* row_scale, const tint4_bf16* bias,
+                                         tint4_bf16* y, int M, int N, int K, int group,
+                                         void* stream) {
+    tint4_status s = check_mnk(M, N, K);
+    if (s != TINT4_OK) return s;
+    if ((s = check_rq_shape(M, K, group)) != TINT4_OK) return s;
+    if (M > 0 && (!x || !w_packed || !row_scale || !y)) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_packed) || !aligned16(row_scale) || !aligned16(y) ||
+        !aligned16(bias))
+        return TINT4_ERR_MISALIGNED;
+    if (convrot_linear_workspace_size(M, K, 8) > kStaticScratchBytes) return TINT4_ERR_WORKSPACE;
+    int dev = 0;
+    if ((s = check_device(&dev)) != TINT4_OK) return s;
+    if (M == 0) return TINT4_OK;
+    uint8_t* codes = static_cast<uint8_t*>(static_scratch_address(dev));
+    if (codes == nullptr) return TINT4_ERR_CUDA;
+    float* tok_scale =
+        reinterpret_cast<float*>(codes + align_up(static_cast<size_t>(M) * K, 256));
+    cudaStream_t st = as_stream(stream);
+    launch_rq_g<__nv_bfloat16, 8>(reinterpret_cast<const __nv_bfloat16*>(x), M, K, group, codes,
+                                  tok_scale, st);
+    if ((s = last_launch_status()) != TINT4_OK) return s;
+    return launch_gemm<false, false>(codes, w_packed, tok_scale, row_scale,
+                                     reinterpret_cast<const __nv_bfloat16*>(bias), y, M, N, K,
+                                     st, true);
 }
 
 tint4_status w4a16_gemv_gemm(const tint4_bf16* x, const uint8_t* w_q, const tint4_bf16* scale,
