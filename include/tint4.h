@@ -121,7 +121,8 @@ tint4_status w4a4_gemm(const uint8_t* a_packed, const float* tok_scale, const ui
                        int N, int K, void* stream);
 
 /* Bytes of workspace convrot_w4a8_linear (bits 8) / convrot_w4a4_linear
- * (bits 4) need: the activation codes plus the token scales, 256-aligned. */
+ * (bits 4) need: the activation codes, one byte per code for both widths
+ * (M * K), plus the token scales (4 * M), each rounded up to 256. */
 size_t convrot_linear_workspace_size(int M, int K, int bits);
 
 /*
@@ -138,7 +139,11 @@ tint4_status convrot_w4a8_linear(const tint4_bf16* x, const uint8_t* w_packed,
                                  int M, int N, int K, int group, void* workspace,
                                  size_t workspace_bytes, void* stream);
 
-/* As convrot_w4a8_linear with int4 activation codes (W4A4). */
+/* As convrot_w4a8_linear with int4 activation codes (W4A4): codes in
+ * [-7, 7], scale absmax / 7.  Inside the call the codes are kept one per byte
+ * and run through the W4A8 tensor-core kernel, whose int32 sums are the same
+ * integers; the packed int4 format is the one convrot_quantize_act(bits 4)
+ * and w4a4_gemm exchange. */
 tint4_status convrot_w4a4_linear(const tint4_bf16* x, const uint8_t* w_packed,
                                  const float* row_scale, const tint4_bf16* bias, tint4_bf16* y,
                                  int M, int N, int K, int group, void* workspace,

@@ -95,20 +95,6 @@ __device__ __forceinline__ void unpack32_permuted(const uint4 p, uint4& lo, uint
     hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-__device__ __forceinline__ uint4 lds128(const uint8_t* p) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(smem_u32(p)));
-    return v;
-}
-
-__device__ __forceinline__ void sts128(uint8_t* p, const uint4 v) {
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "r"(v.x),
-                 "r"(v.y), "r"(v.z), "r"(v.w)
-                 : "memory");
-}
-
 // Unpack `rows` rows of 64 packed bytes (one K stage) from `src` into the
 // 128-byte swizzled K-major int8 layout at `dst`.  Thread t of the 128 unpack
 // threads handles 16-byte pieces t, t + 128, ...; a piece is 32 K values of
@@ -234,7 +220,10 @@ w4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             // every MMA issued so far lands before acc_full flips (also on abort,
             // so that the TMEM is quiet before it is freed)
             umma_commit(acc_full);
+            uint32_t never = 0u;
+            (void)mbar_wait_bounded(acc_full, 0, &never, wait_ns, 0u);
         }
+        __syncwarp();   // lanes 1-31 park here instead of polling a barrier
     } else {
         const int t = threadIdx.x - 64;  // 0..127
         for (int kt = 0; kt < KT; ++kt) {
@@ -326,12 +315,8 @@ w4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
     }
 
-    // ---- teardown: the accumulator must be quiet before TMEM is released
-    if (warp == 1) {
-        // wait for the final commit even on abort (bounded, ignores the flag)
-        uint32_t never = 0u;
-        mbar_wait_bounded(acc_full, 0, &never, wait_ns, 0u);
-    }
+    // ---- teardown: the accumulator is quiet (warp 1 waited on acc_full,
+    // also on abort) before TMEM is released
     tcgen05_fence_before();
     __syncthreads();
     if (warp == 1) {

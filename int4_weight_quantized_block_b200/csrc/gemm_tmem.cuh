@@ -1,0 +1,347 @@
+// gemm_tmem.cuh -- persistent W4A8 GEMM with the unpacked weights in tensor
+// memory.
+//
+//   acc[m, n] = sum_k qa[m, k] * qw[n, k]            (int32, exact)
+//   y[m, n]   = bf16( acc * s_tok[m] * s_row[n] (+ bias[n]) )
+//
+// "ComfyUI-INT-Crush", "Inference > INT4 > CUDA backend": INT4 weights are
+// unpacked to INT8 and run through an INT8 GEMM with fused dequant;
+// stable-diffusion.cpp "feat: packed int4 convrot model loading and
+// dispatch", "Summary": the packed nibbles stay packed in memory (about half a
+// byte per weight).
+//
+// Shape of the product on the tensor core: the weights are the MMA's M side
+// (128 rows = the 128 TMEM lanes) and the tokens its N side (192 per tile).
+// Per 128-wide K step the TMA brings one activation tile (192 tokens x 128
+// int8 codes, 128-byte swizzle: the MMA's B operand) and one packed weight
+// tile (128 rows x 64 bytes, 64-byte swizzle) into shared memory.  Each of
+// 128 unpack threads owns one weight row: it reads its 64 packed bytes
+// (bank-conflict-free thanks to the swizzle), widens every nibble to an int8
+// (x16, see below) and writes the 128 K values with one tcgen05.st into a
+// TMEM A-operand stage.  The widened weights never go back to shared memory.
+//
+// The CTA is persistent (one per SM) and walks a static list of 128 x 192
+// tiles.  Warp roles (18 warps):
+//   warp 0      TMA producer (4-deep ring of 24 KB activation + 8 KB weight
+//               stages)
+//   warp 1      TMEM owner; one thread issues tcgen05.mma.cta_group::1.kind::i8
+//               (A from TMEM, B from shared memory, M 128, N 192, K 32)
+//   warps 2-9   weight unpack into the 4 TMEM A stages (32 columns each);
+//               warps 2-5 take the even K steps and warps 6-9 the odd ones,
+//               so two unpack chains run side by side on every SM
+//               sub-partition (each warp may only reach its quarter of the
+//               TMEM lanes, warp % 4)
+//   warps 10-17 epilogue: tcgen05.ld of one accumulator buffer while the MMAs
+//               fill the other (two 192-column int32 buffers); two warps per
+//               TMEM lane quarter, each on half of the tokens.  A thread holds
+//               one weight row (= one output column), so it scales its values,
+//               rounds them to bf16 and writes them with 2-byte shared-memory
+//               stores into a [192 tokens][128 columns] staging tile, which one
+//               TMA tensor store then writes to y (row-major [M, N]) and clips
+//               at the M and N edges.
+// TMEM columns: accumulators at 0 and 192, A stages at 384 + 32 s.
+//
+// A nibble moved into the high half of its byte, low half cleared, is the
+// int8 value 16 * code; the accumulators hold 16 * acc and the epilogue
+// shifts back exactly (|16 acc| < 2^31 for K <= 65536).
+#pragma once
+
+#include "ptx.cuh"
+
+namespace tint4 {
+
+constexpr int kTmBM = 128;       // weight rows per tile (UMMA M, TMEM lanes)
+constexpr int kTmBN = 192;       // tokens per tile (UMMA N)
+constexpr int kTmBK = 128;       // K values per stage
+constexpr int kTmStages = 4;     // activation smem stages = TMEM A stages
+constexpr int kTmThreads = 576;  // 18 warps
+constexpr int kTmActBytes = kTmBN * kTmBK;            // 24 KB per stage
+constexpr int kTmWBytes = kTmBM * kTmBK / 2;          // 8 KB packed weights per stage
+constexpr int kTmOutBytes = kTmBN * kTmBM * 2;        // 48 KB bf16 staging tile
+constexpr int kTmSmemBytes = kTmStages * (kTmActBytes + kTmWBytes) + kTmOutBytes + 256 + 1024;
+constexpr uint32_t kTmColD = 0;                       // accumulator buffer b at b * kTmBN
+constexpr uint32_t kTmColA = 2 * kTmBN;               // A stage s at kTmColA + 32 s
+static_assert(kTmColA + 32 * kTmStages <= 512, "TMEM budget");
+static_assert(kTmActBytes % 1024 == 0 && kTmWBytes % 1024 == 0, "swizzled stage alignment");
+
+__device__ __forceinline__ void umma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Bounded wait by lane 0 of the warp, result broadcast: the warp leaves
+// together (tcgen05.st / tcgen05.ld are warp-collective).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
+                                          uint64_t limit_ns, unsigned err) {
+    const int lane = threadIdx.x & 31;
+    int ok = 0;
+    if (lane == 0) ok = mbar_wait_bounded(bar, parity, abort, limit_ns, err) ? 1 : 0;
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    return ok != 0;
+}
+
+template <bool OUT_I32>
+__global__ void __launch_bounds__(kTmThreads, 1)
+w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
+                      const __grid_constant__ CUtensorMap tmap_w,
+                      const __grid_constant__ CUtensorMap tmap_y, const float* __restrict__ tok_scale,
+                      const float* __restrict__ row_scale, const __nv_bfloat16* __restrict__ bias,
+                      void* __restrict__ out, int M, int N, int K, uint64_t wait_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* sAct = smem;
+    uint8_t* sW = smem + kTmStages * kTmActBytes;
+    uint8_t* sOut = sW + kTmStages * kTmWBytes;
+    uint64_t* act_full = reinterpret_cast<uint64_t*>(sOut + kTmOutBytes);
+    uint64_t* a_full = act_full + kTmStages;       // TMEM A stage written (128 arrivals)
+    uint64_t* empty = a_full + kTmStages;          // stage consumed by the MMAs (commit)
+    uint64_t* acc_full = empty + kTmStages;        // [2] accumulator ready (commit)
+    uint64_t* acc_empty = acc_full + 2;            // [2] accumulator drained (8 warp arrivals)
+    uint64_t* final_bar = acc_empty + 2;           // all MMAs done (teardown)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
+    volatile uint32_t* abort_flag = tmem_slot + 1;
+    volatile uint32_t* epi_go = tmem_slot + 2;     // epilogue: proceed with this tile
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int m_tiles = (M + kTmBN - 1) / kTmBN;
+    const int n_tiles = (N + kTmBM - 1) / kTmBM;
+    const int n_work = m_tiles * n_tiles;
+    const int KT = (K + kTmBK - 1) / kTmBK;
+    const int my_tiles = (blockIdx.x < n_work) ? (n_work - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kTmStages; ++s) {
+            mbar_init(&act_full[s], 1);
+            mbar_init(&a_full[s], 128);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 8);
+        }
+        mbar_init(final_bar, 1);
+        *abort_flag = 0u;
+        fence_mbarrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmap_act);
+        prefetch_tensormap(&tmap_w);
+        if (!OUT_I32) prefetch_tensormap(&tmap_y);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tcgen05_fence_before();
+    __syncthreads();
+    tcgen05_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    // the codes and token scales may come from the grid launched just before
+    grid_dependency_wait();
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t c = 0;
+            int issued = 0;
+            for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
+                const int tile = blockIdx.x + i * gridDim.x;
+                const int m0 = (tile % m_tiles) * kTmBN;
+                const int n0 = (tile / m_tiles) * kTmBM;
+                for (int kt = 0; kt < KT; ++kt, ++c) {
+                    const int s = c % kTmStages;
+                    const uint32_t ph = (c / kTmStages) & 1;
+                    if (!mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, wait_ns,
+                                           kDevErrTimeoutProducer))
+                        break;
+                    mbar_arrive_expect_tx(&act_full[s], kTmActBytes + kTmWBytes);
+                    tma_load_2d(&tmap_act, &act_full[s], sAct + s * kTmActBytes, kt * kTmBK, m0);
+                    tma_load_2d(&tmap_w, &act_full[s], sW + s * kTmWBytes, kt * (kTmBK / 2), n0);
+                    ++issued;
+                }
+            }
+            if (*abort_flag) {
+                uint32_t never = 0u;
+                const int first = issued > kTmStages ? issued - kTmStages : 0;
+                for (int j = first; j < issued; ++j)
+                    (void)mbar_wait_bounded(&act_full[j % kTmStages], (j / kTmStages) & 1, &never,
+                                            wait_ns, 0u);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_i8(kTmBM, kTmBN);
+            uint32_t c = 0;
+            bool ok = true;
+            for (int i = 0; i < my_tiles && ok; ++i) {
+                const int buf = i & 1;
+                const uint32_t aph = (i >> 1) & 1;
+                if (!mbar_wait_bounded(&acc_empty[buf], aph ^ 1, abort_flag, wait_ns,
+                                       kDevErrTimeoutConsumer)) {
+                    ok = false;
+                    break;
+                }
+                tcgen05_fence_after();
+                const uint32_t d_tmem = tmem_base + kTmColD + buf * kTmBN;
+                for (int kt = 0; kt < KT; ++kt, ++c) {
+                    const int s = c % kTmStages;
+                    const uint32_t ph = (c / kTmStages) & 1;
+                    if (!mbar_wait_bounded(&act_full[s], ph, abort_flag, wait_ns,
+                                           kDevErrTimeoutConsumer) ||
+                        !mbar_wait_bounded(&a_full[s], ph, abort_flag, wait_ns,
+                                           kDevErrTimeoutConsumer)) {
+                        ok = false;
+                        break;
+                    }
+                    tcgen05_fence_after();
+                    const uint32_t a_tmem = tmem_base + kTmColA + 32 * s;
+                    const uint32_t b_addr = smem_u32(sAct + s * kTmActBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kTmBK / 32; ++kk)
+                        umma_i8_ts(d_tmem, a_tmem + 8 * kk, umma_desc_sw128(b_addr + 32 * kk),
+                                   idesc, (kt | kk) != 0);
+                    umma_commit(&empty[s]);
+                }
+                if (ok) umma_commit(&acc_full[buf]);
+            }
+            // everything issued lands before TMEM is released
+            umma_commit(final_bar);
+            uint32_t never = 0u;
+            (void)mbar_wait_bounded(final_bar, 0, &never, wait_ns, 0u);
+        }
+        __syncwarp();   // lanes 1-31 park here instead of polling a barrier
+    } else if (warp < 10) {
+        // ------------------------------------------------ weight unpack -> TMEM (warps 2-9)
+        const int q = warp & 3;                 // TMEM lane quarter
+        const int r = q * 32 + lane;            // weight row within the tile
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        const int total = my_tiles * KT;        // K steps this CTA runs
+        // 64-byte swizzle of the TMA tile: chunk v of row r sits at chunk
+        // v ^ ((r >> 1) & 3); 8 consecutive rows then hit 8 distinct bank groups
+        const int sw = (r >> 1) & 3;
+        for (int j = (warp < 6 ? 0 : 1); j < total; j += 2) {
+            const int s = j % kTmStages;
+            const uint32_t ph = (j / kTmStages) & 1;
+            if (!warp_wait(&act_full[s], ph, abort_flag, wait_ns, kDevErrTimeoutConsumer)) break;
+            const uint8_t* row = sW + s * kTmWBytes + r * 64;
+            uint32_t a[32];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const uint4 p = lds128(row + 16 * (v ^ sw));
+                const uint32_t w4[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) unpack8_natural(w4[u], a[8 * v + 2 * u], a[8 * v + 2 * u + 1]);
+            }
+            // the TMEM A stage is free: its previous MMAs completed before
+            // the producer refilled this stage (empty[s] -> act_full[s])
+            tcgen05_fence_after();
+            tmem_st_32x32b_x32(tmem_base + lane_base + kTmColA + 32 * s, a);
+            tmem_st_wait();
+            tcgen05_fence_before();
+            mbar_arrive(&a_full[s]);
+        }
+    } else if (warp < 18) {
+        // ------------------------------------------------ epilogue (warps 10-17)
+        const int e = warp - 10;                // 0..7
+        const int q = warp & 3;                 // TMEM lane quarter
+        const int half = e >> 2;                // tokens [96 half, 96 half + 96)
+        const int r = q * 32 + lane;            // weight row in the tile = output column
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        const bool leader = (e == 0 && lane == 0);
+        for (int i = 0; i < my_tiles; ++i) {
+            const int tile = blockIdx.x + i * gridDim.x;
+            const int m0 = (tile % m_tiles) * kTmBN;
+            const int n0 = (tile / m_tiles) * kTmBM;
+            const int n = n0 + r;
+            const int buf = i & 1;
+            // one thread waits for the accumulator and for the previous tile's
+            // store to have read the staging tile; the named barrier hands the
+            // decision to all 8 warps at once
+            if (leader) {
+                const bool ok = mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1, abort_flag,
+                                                  wait_ns, kDevErrTimeoutEpilogue);
+                if (!OUT_I32) bulk_wait_group_read0();
+                *epi_go = ok ? 1u : 0u;
+            }
+            named_barrier_sync(1, 256);
+            if (*epi_go == 0u) break;
+            tcgen05_fence_after();
+            const bool row_ok = n < N;
+            // (16 acc) * s_tok * (s_row / 16) equals acc * s_tok * s_row in fp32:
+            // scaling by a power of two commutes with the rounding
+            const float sr16 = (row_ok && !OUT_I32) ? __ldg(row_scale + n) * 0.0625f : 0.0f;
+            const float b = (row_ok && !OUT_I32 && bias != nullptr) ? __bfloat162float(bias[n]) : 0.0f;
+#pragma unroll 1
+            for (int c0 = half * (kTmBN / 2); c0 < (half + 1) * (kTmBN / 2); c0 += 32) {
+                if (m0 + c0 >= M) break;   // warp-uniform
+                uint32_t acc[32];
+                tmem_ld_32x32b_x32(tmem_base + lane_base + kTmColD + buf * kTmBN + c0, acc);
+                tmem_ld_wait();
+                const int mb = m0 + c0;
+                const int mcount = min(32, M - mb);
+                if (OUT_I32) {
+                    if (!row_ok) continue;
+                    int32_t* o = static_cast<int32_t*>(out) + static_cast<size_t>(mb) * N + n;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (j < mcount) o[static_cast<size_t>(j) * N] = static_cast<int32_t>(acc[j]) >> 4;
+                } else {
+                    float st[32];
+                    if (mcount == 32) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const float4 v = __ldg(reinterpret_cast<const float4*>(tok_scale + mb + j));
+                            st[j] = v.x; st[j + 1] = v.y; st[j + 2] = v.z; st[j + 3] = v.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) st[j] = (j < mcount) ? __ldg(tok_scale + mb + j) : 0.0f;
+                    }
+                    // staging tile row = token (256 bytes), column = this thread's row
+                    uint8_t* dst = sOut + c0 * (kTmBM * 2) + r * 2;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float v =
+                            static_cast<float>(static_cast<int32_t>(acc[j])) * st[j] * sr16 + b;
+                        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+                        asm volatile("st.shared.b16 [%0], %1;" ::"r"(smem_u32(dst + j * (kTmBM * 2))),
+                                     "h"(*reinterpret_cast<const unsigned short*>(&h))
+                                     : "memory");
+                    }
+                }
+            }
+            // the accumulator buffer is drained: the MMAs may refill it
+            tcgen05_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            if (!OUT_I32) {
+                fence_proxy_async_smem();          // staging writes -> TMA engine
+                named_barrier_sync(1, 256);
+                if (leader) {
+                    tma_store_2d(&tmap_y, sOut, n0, m0);
+                    bulk_commit_group();
+                }
+            }
+        }
+        if (leader && !OUT_I32) bulk_wait_group0();
+    }
+
+    // ---- teardown: every MMA has landed (warp 1 waited on final_bar)
+    tcgen05_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tcgen05_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+}  // namespace tint4

@@ -84,12 +84,13 @@ __device__ __forceinline__ void fwht_lane8(float (&v)[8], int lane) {
     for (int j = 0; j < 8; ++j) v[j] *= s;
 }
 
-// CH = chunks per warp held in registers (K <= 8 warps * CH * 256).
-template <typename InT, int G, int BITS, int CH>
+// Q = 127 (int8 codes) or 7 (int4 codes); PACKED: int4 codes two per byte,
+// else one code per int8.  CH = chunks per warp held in registers
+// (K <= 8 warps * CH * 256).
+template <typename InT, int G, int Q, bool PACKED, int CH>
 __global__ void __launch_bounds__(kQuantThreads)
 rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K,
                             void* __restrict__ codes, float* __restrict__ scales) {
-    constexpr int Q = (BITS == 8) ? 127 : 7;
     const int row = blockIdx.x;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -151,7 +152,7 @@ rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K,
                 }
                 q[j] = static_cast<int>(t);
             }
-            if (BITS == 8) {
+            if (!PACKED) {
                 uint2 out;
                 out.x = (q[0] & 0xFF) | ((q[1] & 0xFF) << 8) | ((q[2] & 0xFF) << 16) |
                         (static_cast<uint32_t>(q[3] & 0xFF) << 24);

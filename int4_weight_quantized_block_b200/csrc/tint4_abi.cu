@@ -7,10 +7,12 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "../../include/tint4.h"
 #include "gemm.cuh"
+#include "gemm_tmem.cuh"
 #include "ptx.cuh"
 #include "quantize.cuh"
 #include "w4a16.cuh"
@@ -85,10 +87,11 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D uint8 tensor [outer, inner] with row pitch `pitch` bytes; box
-// [box_outer, box_inner]; out-of-range elements read as zero.
-bool make_map_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                 uint64_t pitch, uint32_t box_inner, uint32_t box_outer,
+// 2-D tensor [outer, inner] of `dtype` with row pitch `pitch` bytes; box
+// [box_outer, box_inner]; out-of-range elements read as zero and are not
+// written by stores.
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                 uint64_t outer, uint64_t pitch, uint32_t box_inner, uint32_t box_outer,
                  CUtensorMapSwizzle swizzle) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
@@ -96,11 +99,18 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ou
     const cuuint64_t strides[1] = {pitch};
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
-                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+    const CUresult r = enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+bool make_map_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                 uint64_t pitch, uint32_t box_inner, uint32_t box_outer,
+                 CUtensorMapSwizzle swizzle) {
+    return make_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, inner, outer, pitch, box_inner,
+                       box_outer, swizzle);
 }
 
 // ------------------------------------------------------------------ shape rules
@@ -117,30 +127,31 @@ bool valid_group(int g) { return g == 0 || g == 16 || g == 64 || g == 256; }
 
 // ------------------------------------------------------------------ rotate + quantize
 
-template <typename InT, int G, int BITS, int CH>
+// Q = 127 or 7; PACKED: int4 codes two per byte, else one code per int8
+template <typename InT, int G, int Q, bool PACKED, int CH>
 void launch_rq(const InT* in, int rows, int K, void* codes, float* scales, cudaStream_t st) {
-    rotate_quantize_rows_kernel<InT, G, BITS, CH><<<rows, kQuantThreads, 0, st>>>(in, rows, K,
-                                                                                   codes, scales);
+    rotate_quantize_rows_kernel<InT, G, Q, PACKED, CH>
+        <<<rows, kQuantThreads, 0, st>>>(in, rows, K, codes, scales);
 }
 
-template <typename InT, int G, int BITS>
+template <typename InT, int G, int Q, bool PACKED>
 void launch_rq_ch(const InT* in, int rows, int K, void* codes, float* scales, cudaStream_t st) {
     const int nchunks = (K + kQuantChunk - 1) / kQuantChunk;
     const int per_warp = (nchunks + kQuantWarps - 1) / kQuantWarps;
-    if (per_warp <= 1) launch_rq<InT, G, BITS, 1>(in, rows, K, codes, scales, st);
-    else if (per_warp <= 2) launch_rq<InT, G, BITS, 2>(in, rows, K, codes, scales, st);
-    else if (per_warp <= 4) launch_rq<InT, G, BITS, 4>(in, rows, K, codes, scales, st);
-    else launch_rq<InT, G, BITS, 8>(in, rows, K, codes, scales, st);
+    if (per_warp <= 1) launch_rq<InT, G, Q, PACKED, 1>(in, rows, K, codes, scales, st);
+    else if (per_warp <= 2) launch_rq<InT, G, Q, PACKED, 2>(in, rows, K, codes, scales, st);
+    else if (per_warp <= 4) launch_rq<InT, G, Q, PACKED, 4>(in, rows, K, codes, scales, st);
+    else launch_rq<InT, G, Q, PACKED, 8>(in, rows, K, codes, scales, st);
 }
 
-template <typename InT, int BITS>
+template <typename InT, int Q, bool PACKED>
 void launch_rq_g(const InT* in, int rows, int K, int g, void* codes, float* scales,
                  cudaStream_t st) {
     switch (g) {
-        case 0: launch_rq_ch<InT, 0, BITS>(in, rows, K, codes, scales, st); break;
-        case 16: launch_rq_ch<InT, 16, BITS>(in, rows, K, codes, scales, st); break;
-        case 64: launch_rq_ch<InT, 64, BITS>(in, rows, K, codes, scales, st); break;
-        default: launch_rq_ch<InT, 256, BITS>(in, rows, K, codes, scales, st); break;
+        case 0: launch_rq_ch<InT, 0, Q, PACKED>(in, rows, K, codes, scales, st); break;
+        case 16: launch_rq_ch<InT, 16, Q, PACKED>(in, rows, K, codes, scales, st); break;
+        case 64: launch_rq_ch<InT, 64, Q, PACKED>(in, rows, K, codes, scales, st); break;
+        default: launch_rq_ch<InT, 256, Q, PACKED>(in, rows, K, codes, scales, st); break;
     }
 }
 
@@ -154,21 +165,84 @@ tint4_status check_rq_shape(int rows, int K, int g) {
 
 // ------------------------------------------------------------------ GEMM
 
-template <bool A_INT4, bool OUT_I32>
-tint4_status launch_gemm(const void* a, const uint8_t* w, const float* st, const float* sr,
-                         const __nv_bfloat16* bias, void* out, int M, int N, int K,
-                         cudaStream_t stream, bool pdl) {
-    using L = GemmLayout<A_INT4, kGemmBN, kGemmStages>;
-    auto kern = w4_gemm_kernel<A_INT4, kGemmBN, kGemmStages, OUT_I32>;
+int num_sms(int dev) {
+    static std::atomic<int> cache[kMaxDevices];
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v == 0) {
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            v = 148;
+        }
+        cache[dev].store(v, std::memory_order_relaxed);
+    }
+    return v;
+}
+
+cudaLaunchAttribute pdl_attr() {
+    cudaLaunchAttribute a;
+    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a.val.programmaticStreamSerializationAllowed = 1;
+    return a;
+}
+
+// W4A8: int8 activation codes, weights widened into TMEM (gemm_tmem.cuh).
+template <bool OUT_I32>
+tint4_status launch_gemm_tmem(const void* a, const uint8_t* w, const float* st, const float* sr,
+                              const __nv_bfloat16* bias, void* out, int M, int N, int K,
+                              cudaStream_t stream, bool pdl) {
+    auto kern = w4a8_tmem_gemm_kernel<OUT_I32>;
+    CUtensorMap ta, tw, ty;
+    std::memset(&ty, 0, sizeof(ty));
+    bool ok = make_map_u8(&ta, a, K, M, K, kTmBK, kTmBN, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && make_map_u8(&tw, w, K / 2, N, K / 2, kTmBK / 2, kTmBM, CU_TENSOR_MAP_SWIZZLE_64B);
+    if (!OUT_I32)   // y bf16 [M, N]: the epilogue's staging tile goes out as one box
+        ok = ok && make_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, N, M,
+                               static_cast<uint64_t>(N) * 2, kTmBM, kTmBN,
+                               CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!ok) return TINT4_ERR_CUDA;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static std::atomic<bool> attr_done[kMaxDevices];
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kTmSmemBytes) != cudaSuccess) {
+            cudaGetLastError();
+            return TINT4_ERR_CUDA;
+        }
+        attr_done[dev].store(true, std::memory_order_release);
+    }
+    const int tiles = ((M + kTmBN - 1) / kTmBN) * ((N + kTmBM - 1) / kTmBM);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(std::min(tiles, num_sms(dev)), 1, 1);
+    cfg.blockDim = dim3(kTmThreads, 1, 1);
+    cfg.dynamicSmemBytes = kTmSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    if (pdl) {
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    const uint64_t wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tw, ty, st, sr, bias, out, M, N, K, wait_ns) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return TINT4_ERR_CUDA;
+    }
+    return TINT4_OK;
+}
+
+// W4A4 with packed int4 activation codes: both operands unpacked in shared
+// memory (gemm.cuh).
+template <bool OUT_I32>
+tint4_status launch_gemm_smem_w4a4(const void* a, const uint8_t* w, const float* st,
+                                   const float* sr, const __nv_bfloat16* bias, void* out, int M,
+                                   int N, int K, cudaStream_t stream, bool pdl) {
+    using L = GemmLayout<true, kGemmBN, kGemmStages>;
+    auto kern = w4_gemm_kernel<true, kGemmBN, kGemmStages, OUT_I32>;
     CUtensorMap ta, tw;
-    bool ok;
-    if (A_INT4)
-        ok = make_map_u8(&ta, a, K / 2, M, K / 2, 64, kGemmBM, CU_TENSOR_MAP_SWIZZLE_NONE);
-    else
-        ok = make_map_u8(&ta, a, K, M, K, kGemmBK, kGemmBM, CU_TENSOR_MAP_SWIZZLE_128B);
+    bool ok = make_map_u8(&ta, a, K / 2, M, K / 2, 64, kGemmBM, CU_TENSOR_MAP_SWIZZLE_NONE);
     ok = ok && make_map_u8(&tw, w, K / 2, N, K / 2, 64, kGemmBN, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return TINT4_ERR_CUDA;
-
     int dev = 0;
     cudaGetDevice(&dev);
     static std::atomic<bool> attr_done[kMaxDevices];
@@ -185,10 +259,8 @@ tint4_status launch_gemm(const void* a, const uint8_t* w, const float* st, const
     cfg.blockDim = dim3(kGemmThreads, 1, 1);
     cfg.dynamicSmemBytes = L::kSmemBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
     if (pdl) {
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
@@ -199,6 +271,16 @@ tint4_status launch_gemm(const void* a, const uint8_t* w, const float* st, const
         return TINT4_ERR_CUDA;
     }
     return TINT4_OK;
+}
+
+// A_INT4: activation codes packed two per byte (else int8, one per byte).
+template <bool A_INT4, bool OUT_I32>
+tint4_status launch_gemm(const void* a, const uint8_t* w, const float* st, const float* sr,
+                         const __nv_bfloat16* bias, void* out, int M, int N, int K,
+                         cudaStream_t stream, bool pdl) {
+    if (A_INT4)
+        return launch_gemm_smem_w4a4<OUT_I32>(a, w, st, sr, bias, out, M, N, K, stream, pdl);
+    return launch_gemm_tmem<OUT_I32>(a, w, st, sr, bias, out, M, N, K, stream, pdl);
 }
 
 tint4_status gemm_entry(bool a_int4, const void* a, const float* tok_scale, const uint8_t* w,
@@ -235,20 +317,20 @@ tint4_status linear_entry(int bits, const tint4_bf16* x, const uint8_t* w_packed
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TINT4_ERR_MISALIGNED;
     if ((s = check_device()) != TINT4_OK) return s;
     if (M == 0) return TINT4_OK;
-    const size_t code_bytes = static_cast<size_t>(M) * K / (bits == 8 ? 1 : 2);
+    // one int8 per code for both widths: the W4A4 codes (in [-7, 7]) are kept
+    // one per byte in the workspace and run through the W4A8 kernel, whose
+    // int32 sums are the same numbers
+    const size_t code_bytes = static_cast<size_t>(M) * K;
     uint8_t* codes = static_cast<uint8_t*>(workspace);
     float* tok_scale = reinterpret_cast<float*>(codes + align_up(code_bytes, 256));
     cudaStream_t st = as_stream(stream);
     const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
     const auto* b = reinterpret_cast<const __nv_bfloat16*>(bias);
-    if (bits == 8) launch_rq_g<__nv_bfloat16, 8>(xb, M, K, group, codes, tok_scale, st);
-    else launch_rq_g<__nv_bfloat16, 4>(xb, M, K, group, codes, tok_scale, st);
+    if (bits == 8) launch_rq_g<__nv_bfloat16, 127, false>(xb, M, K, group, codes, tok_scale, st);
+    else launch_rq_g<__nv_bfloat16, 7, false>(xb, M, K, group, codes, tok_scale, st);
     if ((s = last_launch_status()) != TINT4_OK) return s;
-    return bits == 8
-               ? launch_gemm<false, false>(codes, w_packed, tok_scale, row_scale, b, y, M, N, K,
-                                           st, true)
-               : launch_gemm<true, false>(codes, w_packed, tok_scale, row_scale, b, y, M, N, K,
-                                          st, true);
+    return launch_gemm<false, false>(codes, w_packed, tok_scale, row_scale, b, y, M, N, K, st,
+                                     true);
 }
 
 // ------------------------------------------------------------------ W4A16
@@ -337,7 +419,7 @@ tint4_status tint4_pack_weights(const float* W, int N, int K, int group, uint8_t
     if (!aligned16(W) || !aligned16(w_packed) || !aligned16(row_scale)) return TINT4_ERR_MISALIGNED;
     if ((s = check_device()) != TINT4_OK) return s;
     if (N == 0) return TINT4_OK;
-    launch_rq_g<float, 4>(W, N, K, group, w_packed, row_scale, as_stream(stream));
+    launch_rq_g<float, 7, true>(W, N, K, group, w_packed, row_scale, as_stream(stream));
     return last_launch_status();
 }
 
@@ -351,8 +433,10 @@ tint4_status convrot_quantize_act(const tint4_bf16* x, int M, int K, int group, 
     if ((s = check_device()) != TINT4_OK) return s;
     if (M == 0) return TINT4_OK;
     const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
-    if (bits == 8) launch_rq_g<__nv_bfloat16, 8>(xb, M, K, group, codes, tok_scale, as_stream(stream));
-    else launch_rq_g<__nv_bfloat16, 4>(xb, M, K, group, codes, tok_scale, as_stream(stream));
+    if (bits == 8)
+        launch_rq_g<__nv_bfloat16, 127, false>(xb, M, K, group, codes, tok_scale, as_stream(stream));
+    else
+        launch_rq_g<__nv_bfloat16, 7, true>(xb, M, K, group, codes, tok_scale, as_stream(stream));
     return last_launch_status();
 }
 
@@ -370,7 +454,7 @@ tint4_status w4a4_gemm(const uint8_t* a_packed, const float* tok_scale, const ui
 
 size_t convrot_linear_workspace_size(int M, int K, int bits) {
     if (M < 0 || K < 0 || (bits != 8 && bits != 4)) return 0;
-    const size_t code_bytes = static_cast<size_t>(M) * K / (bits == 8 ? 1 : 2);
+    const size_t code_bytes = static_cast<size_t>(M) * K;   // one byte per code, both widths
     return align_up(code_bytes, 256) + align_up(static_cast<size_t>(M) * sizeof(float), 256);
 }
 
@@ -410,8 +494,8 @@ tint4_status convrot_w4a8_linear_noalloc(const tint4_bf16* x, const uint8_t* w_p
     float* tok_scale =
         reinterpret_cast<float*>(codes + align_up(static_cast<size_t>(M) * K, 256));
     cudaStream_t st = as_stream(stream);
-    launch_rq_g<__nv_bfloat16, 8>(reinterpret_cast<const __nv_bfloat16*>(x), M, K, group, codes,
-                                  tok_scale, st);
+    launch_rq_g<__nv_bfloat16, 127, false>(reinterpret_cast<const __nv_bfloat16*>(x), M, K, group,
+                                           codes, tok_scale, st);
     if ((s = last_launch_status()) != TINT4_OK) return s;
     return launch_gemm<false, false>(codes, w_packed, tok_scale, row_scale,
                                      reinterpret_cast<const __nv_bfloat16*>(bias), y, M, N, K,

@@ -63,7 +63,7 @@ def test_version_and_status_strings(lib):
 
 def test_workspace_size(lib):
     assert lib.convrot_linear_workspace_size(4608, 3072, 8) == 4608 * 3072 + 4608 * 4 + 0
-    assert lib.convrot_linear_workspace_size(4608, 3072, 4) == 4608 * 1536 + 4608 * 4
+    assert lib.convrot_linear_workspace_size(4608, 3072, 4) == 4608 * 3072 + 4608 * 4
     assert lib.convrot_linear_workspace_size(3, 64, 8) == 256 + 256
     assert lib.convrot_linear_workspace_size(3, 64, 5) == 0
     assert lib.convrot_linear_workspace_size(-1, 64, 8) == 0
