@@ -156,12 +156,52 @@ class ClockSampler:
                 "samples": len(self.samples), "source": "nvml"}
 
 
+def max_over_ranks(value: float, dev) -> float:
+    """The max of a per-rank float over all ranks (the job's step time is its
+    slowest rank's).  One all-reduce of one number, outside the data path."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own tokens (independent batches)."""
+    from int4_weight_quantized_block_b200 import inputs
+    return inputs.SEED + rank
+
+
 def bf16_gpu(bits, dev):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
 
 
 def event_pair():
     return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+def graph_time(calls, reps, dev):
+    """Mean device time (ms) of one call when `reps` calls run back to back
+    from one CUDA graph replay: for kernels shorter than the host's launch
+    path, per-call events would time the host, not the GPU.  `calls(i)`
+    issues the i-th call (inputs rotated by the caller)."""
+    calls(0)
+    torch.cuda.synchronize(dev)
+    side = torch.cuda.Stream(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            for i in range(reps):
+                calls(i)
+    torch.cuda.synchronize(dev)
+    g.replay()                      # warm
+    torch.cuda.synchronize(dev)
+    a, b = event_pair()
+    a.record()
+    g.replay()
+    b.record()
+    torch.cuda.synchronize(dev)
+    return a.elapsed_time(b) / reps
 
 
 def time_steps(fn, steps, flush=None, dev=None):
@@ -198,7 +238,7 @@ def run_ours(args, rank, world, dev):
 
     w = inputs.WORKLOADS[MAIN]
     M, N, K, g = w["M"], w["N"], w["K"], w["group"]
-    x_np, W_np = inputs.layer_inputs(MAIN, seed=inputs.SEED + rank)
+    x_np, W_np = inputs.layer_inputs(MAIN, seed=rank_seed(rank))
     x = bf16_gpu(x_np, dev)
     wp, sr = t4.tint4_pack_weights(torch.from_numpy(W_np).to(dev), g)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
@@ -220,20 +260,17 @@ def run_ours(args, rank, world, dev):
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
-    ms_local = sum(times) / len(times)
-    ms = ms_local
-    if world > 1:
-        t = torch.tensor([ms_local], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(sum(times) / len(times), dev)
     value = world * ops / (ms * 1e-3) / 1e12
 
-    # components of the step, timed kernel by kernel (same kernels, two calls)
+    # components of the step, timed kernel by kernel (same kernels, two calls);
+    # the rotate+quantize kernel is short: 32 calls in one graph, 8 copies of x
     codes = torch.empty((M, K), dtype=torch.int8, device=dev)
     st = torch.empty((M,), dtype=torch.float32, device=dev)
     t4.convrot_quantize_act(x, g, 8, codes, st)
-    q_ms = statistics.median(time_steps(lambda: t4.convrot_quantize_act(x, g, 8, codes, st),
-                                        args.steps, flush, dev))
+    xs = [x] + [x.clone() for _ in range(7)]
+    q_ms = graph_time(lambda i: t4.convrot_quantize_act(xs[i % 8], g, 8, codes, st), 32, dev)
+    del xs
     gemm_ms = statistics.median(time_steps(lambda: t4.w4a8_gemm(codes, st, wp, sr, None, y),
                                            args.steps, flush, dev))
     gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
@@ -250,12 +287,8 @@ def run_ours(args, rank, world, dev):
 
     for _ in range(2):
         e2e_step()
-    e2e_ms = statistics.mean(time_steps(e2e_step, max(3, args.steps // 4), flush, dev))
-    e2e_ms_max = e2e_ms
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms_max = float(t.item())
+    e2e_ms_max = max_over_ranks(statistics.mean(time_steps(e2e_step, max(3, args.steps // 4),
+                                                           flush, dev)), dev)
 
     rows = {}
     if rank == 0 and not args.no_rows:
@@ -353,22 +386,18 @@ def bench_rows(args, t4, inputs, dev, flush, pk, int8_peak):
         op = inputs.w4a16_operands(M, N, K, G)
         x = bf16_gpu(op.x, dev)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        it = [0]
 
-        def call():
-            q, s, z = copies[it[0] % len(copies)]
-            it[0] += 1
+        def call(i):
+            q, s, z = copies[i % len(copies)]
             t4.w4a16_gemv_gemm(x, q, s, z, G, y)
 
-        for _ in range(8):
-            call()
-        ms = statistics.median(time_steps(call, max(40, reps), None, dev))
+        ms = graph_time(call, 64, dev)
         byts = N * K // 2 + N * (K // G) * 3 + M * K * 2 + M * N * 2
         rows[f"te_decode_w4a16_M{M}"] = {
             "kernel": "w4a16_mma_kernel", "M": M, "N": N, "K": K, "group": G,
             "us": round(ms * 1e3, 2), "GBps": round(byts / ms / 1e6, 1),
             "frac_hbm": round(byts / ms / 1e6 / pk["hbm"], 4),
-            "l2": "8 weight copies rotated (211 MB > L2)"}
+            "timing": "64 calls in one CUDA graph, 8 weight copies rotated (211 MB > L2)"}
     return rows
 
 
@@ -411,7 +440,7 @@ def run_reference(args):
     from int4_weight_quantized_block_b200 import inputs
     w = inputs.WORKLOADS[MAIN]
     M, N, K = w["M"], w["N"], w["K"]
-    per_step_s = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    per_step_s = max(0.1, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
     cal = cpu_baseline(w, target_s=per_step_s)
     Ms = int(cal["sample"].split()[1])
     import oracle

@@ -182,7 +182,8 @@ tint4_status convrot_w4a8_linear_noalloc(const tint4_bf16* x, const uint8_t* w_p
  * [N, K/2] unsigned codes 0..15 packed low nibble first; scale bf16
  * [N, K/group]; zero uint8 [N, K/group] holding 0..15; y bf16 [M, N] with
  * y[m, n] = sum_k x[m, k] * (q[n, k] - zero[n, k/group]) * scale[n, k/group]
- * accumulated in fp32.  group must be 128; 1 <= M <= 64; K % 128 == 0.
+ * accumulated in fp32.  group must be 128; 1 <= M <= 32; K % 128 == 0,
+ * K <= 16384.
  */
 tint4_status w4a16_gemv_gemm(const tint4_bf16* x, const uint8_t* w_q, const tint4_bf16* scale,
                              const uint8_t* zero, int group, tint4_bf16* y, int M, int N, int K,

@@ -10,17 +10,18 @@
 //    diffusion.cpp "feat: packed int4 convrot model loading and dispatch",
 //    "Summary": packed nibbles with row scales).
 //
-// Layout of the work: one CTA per row, 8 warps.  The row is cut into chunks
-// of 256 values; a warp owns chunks w, w+8, w+16, ... and each lane holds 8
-// consecutive values of a chunk in registers (16-byte bf16 loads, fully
-// coalesced).  A rotation block of g values (g = 16, 64 or 256) spans g/8
+// Layout of the work: one CTA per row, one warp per 256-value chunk (two
+// chunks per warp above 32 chunks); each lane holds 8 consecutive values of
+// a chunk in registers (16-byte bf16 loads, fully coalesced), so registers
+// stay few and many rows are in flight per SM.  A rotation block of g values (g = 16, 64 or 256) spans g/8
 // lanes, so the fast Walsh-Hadamard transform runs as three in-register
 // butterfly stages (spans 1, 2, 4) followed by log2(g/8) shuffle stages (spans
 // 8 .. g/2), in that order; every butterfly forms (a + b, a - b) with a the
 // value at the lower index, so the rotated fp32 values do not depend on which
 // thread computes them.  Then the CTA reduces |v| to the row maximum, forms
 // scale = absmax / Q with an IEEE division, and writes the codes
-// clamp(rne(v / scale), -Q, Q) straight from registers.  HBM traffic is one
+// clamp(rne(v / scale), -Q, Q) straight from registers (quant8: the same
+// codes without a division per value).  HBM traffic is one
 // read of the input and one write of the codes: the kernel is bandwidth
 // bound.
 #pragma once
@@ -29,11 +30,10 @@
 
 namespace tint4 {
 
-constexpr int kQuantWarps = 8;
-constexpr int kQuantThreads = kQuantWarps * 32;
+constexpr int kQuantMaxWarps = 32;
 constexpr int kQuantChunk = 256;       // values per warp chunk (32 lanes x 8)
-constexpr int kQuantMaxChunksPerWarp = 8;
-constexpr int kQuantMaxK = kQuantWarps * kQuantMaxChunksPerWarp * kQuantChunk;  // 16384
+constexpr int kQuantMaxChunksPerWarp = 2;
+constexpr int kQuantMaxK = kQuantMaxWarps * kQuantMaxChunksPerWarp * kQuantChunk;  // 16384
 
 __device__ __forceinline__ void load8_as_f32(const __nv_bfloat16* p, float (&v)[8]) {
     const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
@@ -70,12 +70,13 @@ __device__ __forceinline__ void fwht_lane8(float (&v)[8], int lane) {
     // cross-lane stages, spans 8 .. G/2 (lane distance 1 .. G/16)
 #pragma unroll
     for (int d = 1; d < G / 8; d *= 2) {
-        const bool upper = (lane & d) != 0;
+        // lower index holds a, upper holds b: lower -> a + b, upper -> a - b;
+        // fma(+-1, own, other) is that sum or difference, rounded once
+        const float sgn = (lane & d) ? -1.0f : 1.0f;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const float other = __shfl_xor_sync(0xFFFFFFFFu, v[j], d);
-            // lower index holds a, upper holds b: lower -> a + b, upper -> a - b
-            v[j] = upper ? (other - v[j]) : (v[j] + other);
+            v[j] = fmaf(sgn, v[j], other);
         }
     }
     // 1/sqrt(G): a power of two for G = 4^k, so this is exact
@@ -84,17 +85,44 @@ __device__ __forceinline__ void fwht_lane8(float (&v)[8], int lane) {
     for (int j = 0; j < 8; ++j) v[j] *= s;
 }
 
+// Codes clamp(rint(v_j / s), -Q, Q) of 8 values, with v_j / s the IEEE fp32
+// quotient, from the products t_j = v_j * fl(1/s).  |t - fl(v/s)| <= 3 *
+// 2^-24 * |v/s| <= 2.3e-5 here (|v/s| <= Q + tiny), so whenever every t_j of
+// the warp lies at least 2^-15 away from a half-integer, t and fl(v/s) round
+// to the same integers; otherwise (rare, warp-uniform branch) the codes are
+// recomputed with the IEEE division itself.  Same codes as a division per
+// value, a fraction of the instructions.  scale == 0 gives rs == 0 and codes 0.
+template <int Q>
+__device__ __forceinline__ void quant8(const float (&v)[8], float scale, float rs, int (&q)[8]) {
+    float k[8];
+    bool near = false;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float t = v[j] * rs;
+        k[j] = rintf(t);
+        near |= fabsf(fabsf(t - k[j]) - 0.5f) < 3.0517578125e-5f;
+    }
+    if (__any_sync(0xFFFFFFFFu, near) && scale > 0.0f) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) k[j] = rintf(__fdiv_rn(v[j], scale));
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        q[j] = static_cast<int>(fminf(fmaxf(k[j], static_cast<float>(-Q)), static_cast<float>(Q)));
+}
+
 // Q = 127 (int8 codes) or 7 (int4 codes); PACKED: int4 codes two per byte,
-// else one code per int8.  CH = chunks per warp held in registers
-// (K <= 8 warps * CH * 256).
+// else one code per int8.  CH = chunks per warp held in registers; the CTA
+// has blockDim.x / 32 warps (K <= warps * CH * 256).
 template <typename InT, int G, int Q, bool PACKED, int CH>
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantMaxWarps * 32)
 rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K,
                             void* __restrict__ codes, float* __restrict__ scales) {
     const int row = blockIdx.x;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    __shared__ float red[kQuantWarps];
+    const int nwarps = blockDim.x >> 5;
+    __shared__ float red[kQuantMaxWarps];
 
     // Under programmatic dependent launch, let the consumer grid start its
     // prologue while this grid runs; it waits for our completion before
@@ -108,7 +136,7 @@ rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K,
     float amax = 0.0f;
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
-        const int chunk = warp + c * kQuantWarps;
+        const int chunk = warp + c * nwarps;
         const int base = chunk * kQuantChunk + lane * 8;
         if (chunk < nchunks && base < K) {
             load8_as_f32(src + base, v[c]);
@@ -119,7 +147,7 @@ rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K,
     }
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
-        const int chunk = warp + c * kQuantWarps;
+        const int chunk = warp + c * nwarps;
         if (chunk < nchunks) {  // warp-uniform
             if (G > 0) fwht_lane8<(G > 0 ? G : 16)>(v[c], lane);
 #pragma unroll
@@ -131,27 +159,20 @@ rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K,
     if (lane == 0) red[warp] = amax;
     __syncthreads();
     amax = red[0];
-#pragma unroll
-    for (int w = 1; w < kQuantWarps; ++w) amax = fmaxf(amax, red[w]);
+    for (int w = 1; w < nwarps; ++w) amax = fmaxf(amax, red[w]);
 
     const float scale = __fdiv_rn(amax, static_cast<float>(Q));
+    const float rscale = scale > 0.0f ? __frcp_rn(scale) : 0.0f;
     if (threadIdx.x == 0) scales[row] = scale;
 
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
-        const int chunk = warp + c * kQuantWarps;
+        const int chunk = warp + c * nwarps;
         const int base = chunk * kQuantChunk + lane * 8;
-        if (chunk < nchunks && base < K) {
+        if (chunk < nchunks) {   // warp-uniform (quant8 votes across the warp)
             int q[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                float t = 0.0f;
-                if (scale > 0.0f) {
-                    t = rintf(__fdiv_rn(v[c][j], scale));
-                    t = fminf(fmaxf(t, static_cast<float>(-Q)), static_cast<float>(Q));
-                }
-                q[j] = static_cast<int>(t);
-            }
+            quant8<Q>(v[c], scale, rscale, q);
+            if (base >= K) continue;
             if (!PACKED) {
                 uint2 out;
                 out.x = (q[0] & 0xFF) | ((q[1] & 0xFF) << 8) | ((q[2] & 0xFF) << 16) |

@@ -127,21 +127,18 @@ bool valid_group(int g) { return g == 0 || g == 16 || g == 64 || g == 256; }
 
 // ------------------------------------------------------------------ rotate + quantize
 
-// Q = 127 or 7; PACKED: int4 codes two per byte, else one code per int8
-template <typename InT, int G, int Q, bool PACKED, int CH>
-void launch_rq(const InT* in, int rows, int K, void* codes, float* scales, cudaStream_t st) {
-    rotate_quantize_rows_kernel<InT, G, Q, PACKED, CH>
-        <<<rows, kQuantThreads, 0, st>>>(in, rows, K, codes, scales);
-}
-
+// Q = 127 or 7; PACKED: int4 codes two per byte, else one code per int8.
+// One CTA per row, one warp per 256-value chunk (two per warp above 32).
 template <typename InT, int G, int Q, bool PACKED>
 void launch_rq_ch(const InT* in, int rows, int K, void* codes, float* scales, cudaStream_t st) {
     const int nchunks = (K + kQuantChunk - 1) / kQuantChunk;
-    const int per_warp = (nchunks + kQuantWarps - 1) / kQuantWarps;
-    if (per_warp <= 1) launch_rq<InT, G, Q, PACKED, 1>(in, rows, K, codes, scales, st);
-    else if (per_warp <= 2) launch_rq<InT, G, Q, PACKED, 2>(in, rows, K, codes, scales, st);
-    else if (per_warp <= 4) launch_rq<InT, G, Q, PACKED, 4>(in, rows, K, codes, scales, st);
-    else launch_rq<InT, G, Q, PACKED, 8>(in, rows, K, codes, scales, st);
+    if (nchunks <= kQuantMaxWarps) {
+        rotate_quantize_rows_kernel<InT, G, Q, PACKED, 1>
+            <<<rows, nchunks * 32, 0, st>>>(in, rows, K, codes, scales);
+    } else {
+        rotate_quantize_rows_kernel<InT, G, Q, PACKED, 2>
+            <<<rows, ((nchunks + 1) / 2) * 32, 0, st>>>(in, rows, K, codes, scales);
+    }
 }
 
 template <typename InT, int Q, bool PACKED>
@@ -335,11 +332,35 @@ tint4_status linear_entry(int bits, const tint4_bf16* x, const uint8_t* w_packed
 
 // ------------------------------------------------------------------ W4A16
 
-template <int NB>
-void launch_w4a16(const __nv_bfloat16* x, const uint8_t* q, const __nv_bfloat16* s,
-                  const uint8_t* z, __nv_bfloat16* y, int M, int N, int K, cudaStream_t st) {
-    const int grid = (N + kW16Rows - 1) / kW16Rows;
-    w4a16_mma_kernel<NB><<<grid, kW16Threads, 0, st>>>(x, q, s, z, y, M, N, K);
+template <int NB, int MB>
+tint4_status launch_w4a16(const __nv_bfloat16* x, const uint8_t* q, const __nv_bfloat16* s,
+                          const uint8_t* z, __nv_bfloat16* y, int M, int N, int K,
+                          cudaStream_t st) {
+    using L = W16Layout<NB, MB>;
+    auto kern = w4a16_mma_kernel<NB, MB>;
+    CUtensorMap tw, tx;
+    bool ok = make_map_u8(&tw, q, K / 2, N, K / 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
+    ok = ok && make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M,
+                           static_cast<uint64_t>(K) * 2, kW16Group, 8 * NB,
+                           CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!ok) return TINT4_ERR_CUDA;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static std::atomic<bool> attr_done[kMaxDevices];
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 L::smem(kW16MaxK / kW16Group)) != cudaSuccess) {
+            cudaGetLastError();
+            return TINT4_ERR_CUDA;
+        }
+        attr_done[dev].store(true, std::memory_order_release);
+    }
+    const int nblk = (N + 15) / 16;
+    // persistent: one CTA per SM unless that would give a CTA more than MB blocks
+    const int grid = std::max(std::min(num_sms(dev), nblk), (nblk + MB - 1) / MB);
+    kern<<<grid, kW16Threads9, L::smem(K / kW16Group), st>>>(
+        tw, tx, s, z, y, M, N, K, g_wait_limit_ns.load(std::memory_order_relaxed));
+    return last_launch_status();
 }
 
 // ------------------------------------------------------------------ bounded-wait test
@@ -507,7 +528,8 @@ tint4_status w4a16_gemv_gemm(const tint4_bf16* x, const uint8_t* w_q, const tint
                              void* stream) {
     if (M < 0 || N < 0 || K < 0) return TINT4_ERR_INVALID_ARG;
     if (group != kW16Group) return TINT4_ERR_UNSUPPORTED_SHAPE;
-    if (M < 1 || M > 64 || N < 16 || N % 16 != 0 || K < kW16Group || K % kW16Group != 0)
+    if (M < 1 || M > 32 || N < 16 || N % 16 != 0 || K < kW16Group || K % kW16Group != 0 ||
+        K > kW16MaxK)
         return TINT4_ERR_UNSUPPORTED_SHAPE;
     if (!x || !w_q || !scale || !zero || !y) return TINT4_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_q) || !aligned16(scale) || !aligned16(zero) ||
@@ -520,11 +542,9 @@ tint4_status w4a16_gemv_gemm(const tint4_bf16* x, const uint8_t* w_q, const tint
     auto* yb = reinterpret_cast<__nv_bfloat16*>(y);
     cudaStream_t st = as_stream(stream);
     const int nb = (M + 7) / 8;
-    if (nb <= 1) launch_w4a16<1>(xb, w_q, sb, zero, yb, M, N, K, st);
-    else if (nb <= 2) launch_w4a16<2>(xb, w_q, sb, zero, yb, M, N, K, st);
-    else if (nb <= 4) launch_w4a16<4>(xb, w_q, sb, zero, yb, M, N, K, st);
-    else launch_w4a16<8>(xb, w_q, sb, zero, yb, M, N, K, st);
-    return last_launch_status();
+    if (nb <= 1) return launch_w4a16<1, 6>(xb, w_q, sb, zero, yb, M, N, K, st);
+    if (nb <= 2) return launch_w4a16<2, 6>(xb, w_q, sb, zero, yb, M, N, K, st);
+    return launch_w4a16<4, 3>(xb, w_q, sb, zero, yb, M, N, K, st);
 }
 
 tint4_status tint4_debug_int32_gemm(const void* a, int act_bits, const uint8_t* w_packed,

@@ -114,7 +114,7 @@ def test_linear_workspace_rules(lib):
 
 def test_w4a16_rules(lib):
     assert lib.w4a16_gemv_gemm(16, 16, 16, 16, 64, 16, 1, 256, 256, NULL) == 2   # group
-    assert lib.w4a16_gemv_gemm(16, 16, 16, 16, 128, 16, 65, 256, 256, NULL) == 2  # M > 64
+    assert lib.w4a16_gemv_gemm(16, 16, 16, 16, 128, 16, 33, 256, 256, NULL) == 2  # M > 32
     assert lib.w4a16_gemv_gemm(16, 16, 16, 16, 128, 16, 1, 256, 192, NULL) == 2  # K % 128
     assert lib.w4a16_gemv_gemm(NULL, 16, 16, 16, 128, 16, 1, 256, 256, NULL) == 1
     assert lib.w4a16_gemv_gemm(16, 24, 16, 16, 128, 16, 1, 256, 256, NULL) == 3

@@ -190,7 +190,8 @@ def test_full_size_workloads_sampled(name):
 # ------------------------------------------------------------------ W4A16
 
 @pytest.mark.parametrize("M,N,K", [(1, 16, 128), (4, 272, 384), (16, 512, 1024),
-                                   (9, 128, 4096), (64, 64, 256), (33, 96, 512)])
+                                   (9, 128, 4096), (32, 64, 256), (17, 96, 512),
+                                   (16, 2400, 1024), (3, 12288, 256)])
 def test_w4a16(M, N, K):
     op = inputs.w4a16_operands(M, N, K, 128, seed=600 + M)
     y_ref = oracle.w4a16_f64(op.x, op.q, op.scale, op.zero, 128)
@@ -259,3 +260,25 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     torch.cuda.synchronize()
     assert np.array_equal(acc.cpu().numpy(), oracle.gemm_i32(qa, qw))
     assert t4.tint4_get_device_error() == 0
+
+
+def test_quantize_exact_ties():
+    """Values that sit exactly on rounding midpoints (scale exactly 1 or 1/127):
+    the kernel's codes must equal the oracle's round-half-to-even codes."""
+    ties = np.arange(-126.5, 127.0, 1.0)                      # 254 exact ties
+    row = np.concatenate([[127.0, -127.0], ties]).astype(np.float32)
+    x = inputs.f32_to_bf16_bits(np.stack([row, row[::-1], row * 0.5]))
+    for bits in (8, 4):
+        c_ref, s_ref, _ = oracle.quantize_act(x, 0, bits)
+        codes, s = t4.convrot_quantize_act(bf16_to_gpu(x), 0, bits)
+        torch.cuda.synchronize()
+        got = codes.cpu().numpy() if bits == 8 else oracle.unpack_int4(codes.cpu().numpy())
+        assert np.array_equal(got, c_ref)
+        assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    wt = np.concatenate([[7.0, -7.0], np.arange(-6.5, 7.0, 1.0), np.arange(-6.5, 7.0, 1.0)[::-1],
+                         [0.5, -0.5]]).astype(np.float32)
+    W = np.stack([wt, -wt])
+    p_ref, s_ref, _ = oracle.pack_weights(W, 0)
+    p, s = t4.tint4_pack_weights(to_gpu(W), 0)
+    torch.cuda.synchronize()
+    assert np.array_equal(p.cpu().numpy(), p_ref)
