@@ -332,16 +332,16 @@ tint4_status linear_entry(int bits, const tint4_bf16* x, const uint8_t* w_packed
 
 // ------------------------------------------------------------------ W4A16
 
-template <int NB, int MB>
+template <int NB, int MB, int PER_SM>
 tint4_status launch_w4a16(const __nv_bfloat16* x, const uint8_t* q, const __nv_bfloat16* s,
                           const uint8_t* z, __nv_bfloat16* y, int M, int N, int K,
                           cudaStream_t st) {
     using L = W16Layout<NB, MB>;
     auto kern = w4a16_mma_kernel<NB, MB>;
     CUtensorMap tw, tx;
-    bool ok = make_map_u8(&tw, q, K / 2, N, K / 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
+    bool ok = make_map_u8(&tw, q, K / 2, N, K / 2, 128, 16, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M,
-                           static_cast<uint64_t>(K) * 2, kW16Group, 8 * NB,
+                           static_cast<uint64_t>(K) * 2, kW16GPS * kW16Group, 8 * NB,
                            CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return TINT4_ERR_CUDA;
     int dev = 0;
@@ -356,8 +356,8 @@ tint4_status launch_w4a16(const __nv_bfloat16* x, const uint8_t* q, const __nv_b
         attr_done[dev].store(true, std::memory_order_release);
     }
     const int nblk = (N + 15) / 16;
-    // persistent: one CTA per SM unless that would give a CTA more than MB blocks
-    const int grid = std::max(std::min(num_sms(dev), nblk), (nblk + MB - 1) / MB);
+    // persistent: PER_SM CTAs per SM unless that would give a CTA more than MB blocks
+    const int grid = std::max(std::min(PER_SM * num_sms(dev), nblk), (nblk + MB - 1) / MB);
     kern<<<grid, kW16Threads9, L::smem(K / kW16Group), st>>>(
         tw, tx, s, z, y, M, N, K, g_wait_limit_ns.load(std::memory_order_relaxed));
     return last_launch_status();
@@ -542,9 +542,9 @@ tint4_status w4a16_gemv_gemm(const tint4_bf16* x, const uint8_t* w_q, const tint
     auto* yb = reinterpret_cast<__nv_bfloat16*>(y);
     cudaStream_t st = as_stream(stream);
     const int nb = (M + 7) / 8;
-    if (nb <= 1) return launch_w4a16<1, 6>(xb, w_q, sb, zero, yb, M, N, K, st);
-    if (nb <= 2) return launch_w4a16<2, 6>(xb, w_q, sb, zero, yb, M, N, K, st);
-    return launch_w4a16<4, 3>(xb, w_q, sb, zero, yb, M, N, K, st);
+    if (nb <= 1) return launch_w4a16<1, 4, 2>(xb, w_q, sb, zero, yb, M, N, K, st);
+    if (nb <= 2) return launch_w4a16<2, 6, 1>(xb, w_q, sb, zero, yb, M, N, K, st);
+    return launch_w4a16<4, 2, 1>(xb, w_q, sb, zero, yb, M, N, K, st);
 }
 
 tint4_status tint4_debug_int32_gemm(const void* a, int act_bits, const uint8_t* w_packed,

@@ -23,15 +23,20 @@
 // slots; x is gathered in the same order, which leaves each dot product
 // unchanged.
 //
-// Work split: a persistent grid of one CTA per SM; CTA c owns a contiguous
-// run of 16-row blocks (at most MB).  A producer warp streams, for every K
-// group, the packed weights of those rows (one 16-row TMA box per block) and
-// the matching x tile (all tokens) into an 8-deep shared-memory ring; consumer
-// warp w takes groups w, w + 8, ... (ring slot w), reads its x fragments once
-// and uses them for all of the CTA's row blocks.  The TMA keeps up to 8
-// groups of weights in flight per SM whatever the warps are doing, which is
-// what an HBM-bound stream needs.  The 8 partial sums of each output meet in
-// shared memory at the end.
+// Work split: a persistent grid of one (M <= 8: two) CTAs per SM; CTA c owns
+// a contiguous run of 16-row blocks (at most MB).  A producer warp streams,
+// two K groups at a time, the packed weights of those rows (one 16-row x
+// 128-byte TMA box per block: whole 128-byte lines of every row, which DRAM
+// serves best) and the matching x tile into an 8-deep shared-memory ring;
+// consumer warp w takes stages w, w + 8, ... (ring slot w), reads its x
+// fragments once per group and uses them for all of the CTA's row blocks, two
+// blocks at a time so that independent MMA chains overlap.  The 8 partial
+// sums of each output meet in shared memory at the end.
+//
+// The weight boxes use the 128-byte swizzle (16-byte chunk c of smem row r at
+// c ^ (r & 7)).  The two rows an 8-lane phase reads would hit the same banks,
+// so MMA row m holds weight row pi(m) = 4 (m & 1) + (m >> 1) (m < 8; +8 above),
+// which puts them 4 rows apart and onto disjoint chunk sets: conflict-free.
 #pragma once
 
 #include "ptx.cuh"
@@ -63,22 +68,42 @@ __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
     return d;
 }
 
+// x values 8w .. 8w + 7 of a lane's slice (one 16-byte word q, bf16) to the
+// B fragments of k steps 2w (f0) and 2w + 1 (f1): k step 2w + h takes the
+// values (2h, 2h + 4) and (2h + 1, 2h + 5), matching the nibble pairing of
+// the weights
+__device__ __forceinline__ void x_frag(const uint4& q, uint32_t (&f0)[2], uint32_t (&f1)[2]) {
+    f0[0] = __byte_perm(q.x, q.z, 0x5410);
+    f0[1] = __byte_perm(q.x, q.z, 0x7632);
+    f1[0] = __byte_perm(q.y, q.w, 0x5410);
+    f1[1] = __byte_perm(q.y, q.w, 0x7632);
+}
+
 constexpr int kW16Stages = 8;        // = consumer warps: warp w owns ring slot w
 constexpr int kW16Threads9 = (kW16Warps + 1) * 32;   // + the TMA producer warp
+constexpr int kW16GPS = 2;           // K groups per stage (128 packed bytes per row)
+constexpr int kW16MaxK = 16384;      // scales / zero points of a CTA's rows stay in shared memory
 
-constexpr int kW16MaxK = 16384;   // scales / zero points of a CTA's rows stay in shared memory
+// MMA row m (0..15) of a block holds weight row w16_perm(m) of the block
+__host__ __device__ constexpr int w16_perm(int m) {
+    return (m & 8) | ((m & 1) << 2) | ((m >> 1) & 3);
+}
 
 template <int NB, int MB>
 struct W16Layout {
-    static constexpr int kWBytes = MB * 16 * 64;           // packed weights of one group
-    static constexpr int kXBytes = 8 * NB * kW16Group * 2;  // x tile of one group (bf16)
+    static constexpr int kBoxBytes = 16 * 128;                          // one block, two groups
+    static constexpr int kWBytes = MB * kBoxBytes;
+    static constexpr int kXBytes = 8 * NB * kW16GPS * kW16Group * 2;     // x tile, two groups
     static constexpr int kStage = kWBytes + kXBytes;
     static constexpr int kRedBytes = kW16Warps * MB * NB * 32 * 16;
     static constexpr int kBarOff = kW16Stages * kStage > kRedBytes ? kW16Stages * kStage : kRedBytes;
     static constexpr int kSzOff = kBarOff + (2 * kW16Stages + 1) * 8 + 120;
     // the CTA's rows of scale (bf16) and zero point (uint8), all groups, as
     // they lie in global memory
-    __host__ __device__ static constexpr int smem(int ngroups) { return kSzOff + MB * 16 * ngroups * 3 + 16; }
+    __host__ __device__ static constexpr int smem(int ngroups) {
+        return kSzOff + MB * 16 * ngroups * 3 + 16 + 1024;   // + 1024: base alignment
+    }
+    static_assert(kStage % 1024 == 0, "swizzled boxes need 1 KB alignment");
 };
 
 // NB = number of 8-token blocks (M <= 8 * NB); MB = 16-row blocks per CTA at most.
@@ -88,7 +113,9 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
                  const __nv_bfloat16* __restrict__ wscale, const uint8_t* __restrict__ wzero,
                  __nv_bfloat16* __restrict__ y, int M, int N, int K, uint64_t wait_ns) {
     using L = W16Layout<NB, MB>;
-    extern __shared__ __align__(128) uint8_t w16_smem[];
+    extern __shared__ uint8_t w16_smem_raw[];
+    uint8_t* w16_smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(w16_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(w16_smem + L::kBarOff);
     uint64_t* empty = full + kW16Stages;
     uint64_t* sz_full = empty + kW16Stages;        // scales + zero points landed
@@ -97,14 +124,17 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int g = lane >> 2;   // MMA group id: weight row g / g + 8, token column g
+    const int g = lane >> 2;   // MMA group id: MMA rows g / g + 8, token column g
     const int t = lane & 3;    // thread in group: which 32-value slice of a K group
     const int ngroups = K / kW16Group;
+    const int nstages = (ngroups + kW16GPS - 1) / kW16GPS;
     const int nblk = (N + 15) / 16;
     // contiguous run of row blocks of this CTA
     const int b0 = static_cast<int>((static_cast<long long>(blockIdx.x) * nblk) / gridDim.x);
     const int b1 = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * nblk) / gridDim.x);
     const int nb_here = b1 - b0;   // 1..MB (the host sizes the grid)
+    const int rA = w16_perm(g), rB = w16_perm(g + 8);   // weight rows of MMA rows g, g + 8
+    const int swz = rA & 7;                              // = rB & 7
 
     const __nv_bfloat16* sScale = reinterpret_cast<const __nv_bfloat16*>(w16_smem + L::kSzOff);
     const uint8_t* sZero = w16_smem + L::kSzOff + MB * 16 * ngroups * 2;
@@ -141,26 +171,26 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
                          sbytes, sz_full);
             bulk_load_1d(w16_smem + L::kSzOff + MB * 16 * ngroups * 2,
                          wzero + static_cast<size_t>(b0) * 16 * ngroups, zbytes, sz_full);
-            const uint32_t bytes = nb_here * 1024 + L::kXBytes;
+            const uint32_t bytes = nb_here * L::kBoxBytes + L::kXBytes;
             int issued = 0;
-            for (int G = 0; G < ngroups; ++G) {
-                const int s = G % kW16Stages;
-                const uint32_t ph = (G / kW16Stages) & 1;
+            for (int j = 0; j < nstages; ++j) {
+                const int s = j % kW16Stages;
+                const uint32_t ph = (j / kW16Stages) & 1;
                 if (!mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, wait_ns, kDevErrTimeoutProducer))
                     break;
                 uint8_t* st = w16_smem + s * L::kStage;
                 mbar_arrive_expect_tx(&full[s], bytes);
                 for (int rb = 0; rb < nb_here; ++rb)
-                    tma_load_2d(&tmap_w, &full[s], st + rb * 1024, G * 64, (b0 + rb) * 16);
-                tma_load_2d(&tmap_x, &full[s], st + L::kWBytes, G * kW16Group, 0);
+                    tma_load_2d(&tmap_w, &full[s], st + rb * L::kBoxBytes, j * 128, (b0 + rb) * 16);
+                tma_load_2d(&tmap_x, &full[s], st + L::kWBytes, j * kW16GPS * kW16Group, 0);
                 ++issued;
             }
+            uint32_t never = 0u;
             if (*abort_flag) {
                 // let the copies in flight land before the ring is reused or freed
-                uint32_t never = 0u;
                 (void)mbar_wait_bounded(sz_full, 0, &never, wait_ns, 0u);
-                for (int G = (issued > kW16Stages ? issued - kW16Stages : 0); G < issued; ++G)
-                    (void)mbar_wait_bounded(&full[G % kW16Stages], (G / kW16Stages) & 1, &never,
+                for (int j = (issued > kW16Stages ? issued - kW16Stages : 0); j < issued; ++j)
+                    (void)mbar_wait_bounded(&full[j % kW16Stages], (j / kW16Stages) & 1, &never,
                                             wait_ns, 0u);
             }
         }
@@ -169,72 +199,109 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
         int szok = 0;
         if (lane == 0) szok = mbar_wait_bounded(sz_full, 0, abort_flag, wait_ns, kDevErrTimeoutConsumer);
         if (__shfl_sync(0xFFFFFFFFu, szok, 0) == 0) goto consumers_done;
-        for (int G = warp; G < ngroups; G += kW16Warps) {
-            const int s = G % kW16Stages;
-            const uint32_t ph = (G / kW16Stages) & 1;
+        for (int j = warp; j < nstages; j += kW16Warps) {
+            const int s = j % kW16Stages;
+            const uint32_t ph = (j / kW16Stages) & 1;
             int ok = 0;
             if (lane == 0) ok = mbar_wait_bounded(&full[s], ph, abort_flag, wait_ns, kDevErrTimeoutConsumer);
             if (__shfl_sync(0xFFFFFFFFu, ok, 0) == 0) break;
             const uint8_t* st = w16_smem + s * L::kStage;
-            // x fragments: token 8b + g, values 32t .. 32t + 31 of the group,
-            // regrouped into the MMA's B layout
-            uint32_t bfr[NB][8][2];
+#pragma unroll 1
+            for (int gi = 0; gi < kW16GPS; ++gi) {
+                const int G = j * kW16GPS + gi;
+                if (G >= ngroups) break;   // warp-uniform
+                // x fragments: token 8b + g, values 32t .. 32t + 31 of group G,
+                // regrouped into the MMA's B layout
+                // (with 4 token blocks the fragments of all 8 k steps would not
+                // fit next to the sums: then they are re-read per row pair)
+                constexpr bool kXReload = NB >= 4;
+                const uint8_t* xg = st + L::kWBytes + g * (kW16GPS * kW16Group * 2) + gi * (kW16Group * 2) + 64 * t;
+                uint32_t bfr[kXReload ? 1 : NB][kXReload ? 1 : 8][2];
+                if constexpr (!kXReload) {
 #pragma unroll
-            for (int b = 0; b < NB; ++b) {
-                const uint8_t* xr = st + L::kWBytes + (8 * b + g) * (kW16Group * 2) + 64 * t;
-                uint32_t xw[16];
+                    for (int b = 0; b < NB; ++b) {
+                        const uint8_t* xr = xg + 8 * b * (kW16GPS * kW16Group * 2);
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const uint4 q = lds128(xr + 16 * v);
-                    xw[4 * v] = q.x; xw[4 * v + 1] = q.y; xw[4 * v + 2] = q.z; xw[4 * v + 3] = q.w;
+                        for (int w = 0; w < 4; ++w) {
+                            const uint4 q = lds128(xr + 16 * w);
+                            x_frag(q, bfr[b][2 * w], bfr[b][2 * w + 1]);
+                        }
+                    }
                 }
+                // this lane's 16-byte chunk of group G in rows rA / rB (swizzled)
+                const int chunk_off = ((4 * gi + t) ^ swz) << 4;
+                // row blocks in pairs: two independent dequant + MMA chains per
+                // k step keep the tensor pipe and the ALUs busy together
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int w = j >> 1;
-                    const int i0 = 2 * (j & 1);
-                    const uint32_t X0 = xw[4 * w + (i0 >> 1)];       // x[8w+i0],   x[8w+i0+1]
-                    const uint32_t X2 = xw[4 * w + 2 + (i0 >> 1)];   // x[8w+i0+4], x[8w+i0+5]
-                    bfr[b][j][0] = __byte_perm(X0, X2, 0x5410);      // (x[i0],   x[i0+4])
-                    bfr[b][j][1] = __byte_perm(X0, X2, 0x7632);      // (x[i0+1], x[i0+5])
-                }
-            }
+                for (int rp = 0; rp < MB; rp += 2) {
+                    if (rp >= nb_here) break;   // CTA-uniform
+                    uint32_t wa[2][4], wb[2][4], zA[2], zB[2];
+                    float sA[2], sB[2];
 #pragma unroll
-            for (int rb = 0; rb < MB; ++rb) {
-                if (rb >= nb_here) break;   // CTA-uniform
-                const float sA = __bfloat162float(sScale[(rb * 16 + g) * ngroups + G]);
-                const float sB = __bfloat162float(sScale[(rb * 16 + g + 8) * ngroups + G]);
-                // bf16x2 (128 + z, 128 + z): subtracting it from (128 + q) leaves q - z exactly
-                const uint32_t zA = 0x43004300u | (0x00010001u * sZero[(rb * 16 + g) * ngroups + G]);
-                const uint32_t zB = 0x43004300u | (0x00010001u * sZero[(rb * 16 + g + 8) * ngroups + G]);
-                const uint4 pa = lds128(st + rb * 1024 + g * 64 + t * 16);
-                const uint4 pb = lds128(st + rb * 1024 + (g + 8) * 64 + t * 16);
-                const uint32_t wa[4] = {pa.x, pa.y, pa.z, pa.w};
-                const uint32_t wb[4] = {pb.x, pb.y, pb.z, pb.w};
-                float acc[NB][4];
+                    for (int p = 0; p < 2; ++p) {
+                        // a missing second block (odd count) reads a stale box;
+                        // its sums are dropped below
+                        const int rb = min(rp + p, MB - 1);
+                        const uint8_t* box = st + rb * L::kBoxBytes;
+                        const uint4 pa = lds128(box + rA * 128 + chunk_off);
+                        const uint4 pb = lds128(box + rB * 128 + chunk_off);
+                        wa[p][0] = pa.x; wa[p][1] = pa.y; wa[p][2] = pa.z; wa[p][3] = pa.w;
+                        wb[p][0] = pb.x; wb[p][1] = pb.y; wb[p][2] = pb.z; wb[p][3] = pb.w;
+                        sA[p] = __bfloat162float(sScale[(rb * 16 + rA) * ngroups + G]);
+                        sB[p] = __bfloat162float(sScale[(rb * 16 + rB) * ngroups + G]);
+                        // bf16x2 (128 + z, 128 + z): subtracting it from (128 + q) leaves q - z exactly
+                        zA[p] = 0x43004300u | (0x00010001u * sZero[(rb * 16 + rA) * ngroups + G]);
+                        zB[p] = 0x43004300u | (0x00010001u * sZero[(rb * 16 + rB) * ngroups + G]);
+                    }
+                    float acc[2][NB][4];
 #pragma unroll
-                for (int b = 0; b < NB; ++b)
+                    for (int p = 0; p < 2; ++p)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) acc[b][j] = 0.0f;
+                        for (int b = 0; b < NB; ++b)
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int w = j >> 1;          // packed word of this lane's 16 bytes
-                    const int i0 = 2 * (j & 1);    // nibble pairs (i0, i0+4) and (i0+1, i0+5)
-                    uint32_t a[4];
-                    a[0] = bf16x2_sub(nib_pair_bf16(wa[w], i0), zA);       // row g,   k 2t, 2t+1
-                    a[1] = bf16x2_sub(nib_pair_bf16(wb[w], i0), zB);       // row g+8, k 2t, 2t+1
-                    a[2] = bf16x2_sub(nib_pair_bf16(wa[w], i0 + 1), zA);   // row g,   k 2t+8, 2t+9
-                    a[3] = bf16x2_sub(nib_pair_bf16(wb[w], i0 + 1), zB);   // row g+8, k 2t+8, 2t+9
+                            for (int q = 0; q < 4; ++q) acc[p][b][q] = 0.0f;
 #pragma unroll
-                    for (int b = 0; b < NB; ++b) mma_bf16_16816(acc[b], a, bfr[b][j][0], bfr[b][j][1]);
-                }
-                // acc: [0] row g / token 8b+2t, [1] row g / 8b+2t+1,
-                //      [2] row g+8 / 8b+2t,     [3] row g+8 / 8b+2t+1
+                    for (int k = 0; k < 8; ++k) {
+                        const int w = k >> 1;          // packed word of this lane's 16 bytes
+                        const int i0 = 2 * (k & 1);    // nibble pairs (i0, i0+4) and (i0+1, i0+5)
+                        uint32_t bk[NB][2];
+                        if constexpr (kXReload) {
+                            uint32_t unused[2];
 #pragma unroll
-                for (int b = 0; b < NB; ++b) {
-                    total[rb][b][0] = fmaf(sA, acc[b][0], total[rb][b][0]);
-                    total[rb][b][1] = fmaf(sA, acc[b][1], total[rb][b][1]);
-                    total[rb][b][2] = fmaf(sB, acc[b][2], total[rb][b][2]);
-                    total[rb][b][3] = fmaf(sB, acc[b][3], total[rb][b][3]);
+                            for (int b = 0; b < NB; ++b) {
+                                const uint4 q = lds128(xg + 8 * b * (kW16GPS * kW16Group * 2) + 16 * w);
+                                if (k & 1) x_frag(q, unused, bk[b]);
+                                else x_frag(q, bk[b], unused);
+                            }
+                        } else {
+#pragma unroll
+                            for (int b = 0; b < NB; ++b) { bk[b][0] = bfr[b][k][0]; bk[b][1] = bfr[b][k][1]; }
+                        }
+#pragma unroll
+                        for (int p = 0; p < 2; ++p) {
+                            uint32_t a[4];
+                            a[0] = bf16x2_sub(nib_pair_bf16(wa[p][w], i0), zA[p]);       // MMA row g,   k 2t, 2t+1
+                            a[1] = bf16x2_sub(nib_pair_bf16(wb[p][w], i0), zB[p]);       // MMA row g+8, k 2t, 2t+1
+                            a[2] = bf16x2_sub(nib_pair_bf16(wa[p][w], i0 + 1), zA[p]);   // MMA row g,   k 2t+8, 2t+9
+                            a[3] = bf16x2_sub(nib_pair_bf16(wb[p][w], i0 + 1), zB[p]);   // MMA row g+8, k 2t+8, 2t+9
+#pragma unroll
+                            for (int b = 0; b < NB; ++b)
+                                mma_bf16_16816(acc[p][b], a, bk[b][0], bk[b][1]);
+                        }
+                    }
+                    // acc: [0] MMA row g / token 8b+2t, [1] row g / 8b+2t+1,
+                    //      [2] MMA row g+8 / 8b+2t,     [3] row g+8 / 8b+2t+1
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        if (rp + p >= MB || rp + p >= nb_here) break;
+#pragma unroll
+                        for (int b = 0; b < NB; ++b) {
+                            total[rp + p][b][0] = fmaf(sA[p], acc[p][b][0], total[rp + p][b][0]);
+                            total[rp + p][b][1] = fmaf(sA[p], acc[p][b][1], total[rp + p][b][1]);
+                            total[rp + p][b][2] = fmaf(sB[p], acc[p][b][2], total[rp + p][b][2]);
+                            total[rp + p][b][3] = fmaf(sB[p], acc[p][b][3], total[rp + p][b][3]);
+                        }
+                    }
                 }
             }
             __syncwarp();
@@ -267,7 +334,7 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
         }
         const int gg = ln >> 2, tt = ln & 3;
         const int tok0 = 8 * b + 2 * tt;
-        const int r0 = (b0 + rb) * 16 + gg, r1 = r0 + 8;
+        const int r0 = (b0 + rb) * 16 + w16_perm(gg), r1 = (b0 + rb) * 16 + w16_perm(gg + 8);
         if (tok0 < M) {
             if (r0 < N) y[static_cast<size_t>(tok0) * N + r0] = __float2bfloat16_rn(v[0]);
             if (r1 < N) y[static_cast<size_t>(tok0) * N + r1] = __float2bfloat16_rn(v[2]);
