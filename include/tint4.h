@@ -182,8 +182,12 @@ tint4_status convrot_w4a8_linear_noalloc(const tint4_bf16* x, const uint8_t* w_p
  * [N, K/2] unsigned codes 0..15 packed low nibble first; scale bf16
  * [N, K/group]; zero uint8 [N, K/group] holding 0..15; y bf16 [M, N] with
  * y[m, n] = sum_k x[m, k] * (q[n, k] - zero[n, k/group]) * scale[n, k/group]
- * accumulated in fp32.  group must be 128; 1 <= M <= 32; K % 128 == 0,
- * K <= 16384.
+ * accumulated in fp32.  group must be 128; 1 <= M <= 32; N % 16 == 0;
+ * K % 128 == 0, K <= 16384; all pointers 16-byte aligned.  One kernel launch
+ * per 16 tokens: a batch of 17..32 tokens reads the weights twice.  Errors:
+ * TINT4_ERR_UNSUPPORTED_SHAPE for sizes outside these limits,
+ * TINT4_ERR_MISALIGNED, TINT4_ERR_INVALID_ARG for null pointers; nothing is
+ * launched then.
  */
 tint4_status w4a16_gemv_gemm(const tint4_bf16* x, const uint8_t* w_q, const tint4_bf16* scale,
                              const uint8_t* zero, int group, tint4_bf16* y, int M, int N, int K,

@@ -332,34 +332,44 @@ tint4_status linear_entry(int bits, const tint4_bf16* x, const uint8_t* w_packed
 
 // ------------------------------------------------------------------ W4A16
 
-template <int NB, int MB, int PER_SM>
+template <int NB>
 tint4_status launch_w4a16(const __nv_bfloat16* x, const uint8_t* q, const __nv_bfloat16* s,
                           const uint8_t* z, __nv_bfloat16* y, int M, int N, int K,
                           cudaStream_t st) {
-    using L = W16Layout<NB, MB>;
-    auto kern = w4a16_mma_kernel<NB, MB>;
-    CUtensorMap tw, tx;
-    bool ok = make_map_u8(&tw, q, K / 2, N, K / 2, 128, 16, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M,
-                           static_cast<uint64_t>(K) * 2, kW16GPS * kW16Group, 8 * NB,
-                           CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (!ok) return TINT4_ERR_CUDA;
+    using C = W16Cfg<NB>;
+    auto kern = w4a16_mma_kernel<NB>;
+    CUtensorMap tw;
+    if (!make_map_u8(&tw, q, K / 2, N, K / 2, 128, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+        return TINT4_ERR_CUDA;
     int dev = 0;
     cudaGetDevice(&dev);
     static std::atomic<bool> attr_done[kMaxDevices];
     if (!attr_done[dev].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 L::smem(kW16MaxK / kW16Group)) != cudaSuccess) {
+                                 C::kSmemMax) != cudaSuccess) {
             cudaGetLastError();
             return TINT4_ERR_CUDA;
         }
         attr_done[dev].store(true, std::memory_order_release);
     }
-    const int nblk = (N + 15) / 16;
-    // persistent: PER_SM CTAs per SM unless that would give a CTA more than MB blocks
-    const int grid = std::max(std::min(PER_SM * num_sms(dev), nblk), (nblk + MB - 1) / MB);
-    kern<<<grid, kW16Threads9, L::smem(K / kW16Group), st>>>(
-        tw, tx, s, z, y, M, N, K, g_wait_limit_ns.load(std::memory_order_relaxed));
+    const int nblk = N / 16;
+    // one CTA per SM unless that would give a CTA more than kW16MB blocks
+    const int sms = num_sms(dev);
+    const int grid = nblk <= kW16MB * sms ? std::min(sms, nblk) : (nblk + kW16MB - 1) / kW16MB;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(C::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::smem(K / kW16Group);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const W16Consts kc{0x000F000Fu, 0x43004300u};
+    if (cudaLaunchKernelEx(&cfg, kern, tw, x, s, z, y, M, N, K, kc,
+                           g_wait_limit_ns.load(std::memory_order_relaxed)) != cudaSuccess) {
+        cudaGetLastError();
+        return TINT4_ERR_CUDA;
+    }
     return last_launch_status();
 }
 
@@ -541,10 +551,16 @@ tint4_status w4a16_gemv_gemm(const tint4_bf16* x, const uint8_t* w_q, const tint
     const auto* sb = reinterpret_cast<const __nv_bfloat16*>(scale);
     auto* yb = reinterpret_cast<__nv_bfloat16*>(y);
     cudaStream_t st = as_stream(stream);
-    const int nb = (M + 7) / 8;
-    if (nb <= 1) return launch_w4a16<1, 4, 2>(xb, w_q, sb, zero, yb, M, N, K, st);
-    if (nb <= 2) return launch_w4a16<2, 6, 1>(xb, w_q, sb, zero, yb, M, N, K, st);
-    return launch_w4a16<4, 2, 1>(xb, w_q, sb, zero, yb, M, N, K, st);
+    // 16 tokens per launch: a 17..32-token batch streams the weights twice
+    for (int m0 = 0; m0 < M; m0 += kW16MaxM) {
+        const int mc = std::min(kW16MaxM, M - m0);
+        const __nv_bfloat16* xs = xb + static_cast<size_t>(m0) * K;
+        __nv_bfloat16* ys = yb + static_cast<size_t>(m0) * N;
+        s = mc <= 8 ? launch_w4a16<1>(xs, w_q, sb, zero, ys, mc, N, K, st)
+                    : launch_w4a16<2>(xs, w_q, sb, zero, ys, mc, N, K, st);
+        if (s != TINT4_OK) return s;
+    }
+    return TINT4_OK;
 }
 
 tint4_status tint4_debug_int32_gemm(const void* a, int act_bits, const uint8_t* w_packed,

@@ -9,63 +9,90 @@
 //
 // The cost is streaming the packed weights from HBM (0.5 byte per weight plus
 // 3 bytes of scale and zero point per 128 weights); every weight is used by
-// at most 32 tokens.  Per group the sum is
-//   s * sum_k x_k * (q_k - z)
-// with q_k - z formed exactly in bf16: 0x4300 | q is bf16(128 + q), one
-// shift + AND/OR per two nibbles from the packed bytes, and subtracting
-// bf16(128 + z) leaves the small integer q - z.  The products run on the
+// at most 16 tokens of one launch.  Per group the sum is written
+//   s * (sum_k x_k * (128 + q_k)  -  (128 + z) * sum_k x_k)
+// which is the same number: 128 + q_k is exact in bf16 (OR a nibble into the
+// mantissa of bf16 128), so the dequantization is one bit operation per two
+// weights plus a shift, and the zero point leaves the inner loop.  The sums
+// of x per group come from the same MMA with an all-ones weight tile.  The products run on the
 // warp-level bf16 MMA (m16n8k16, fp32 accumulation): at M = 16 the 805 M
 // multiply-adds of the 4096 x 12288 layer would take several times the HBM
 // time on the fp32 CUDA cores.  Weights are the MMA's A operand straight from
-// registers (16 rows x 128 K per warp step, one 16-byte load per lane and
-// row), tokens the B operand (n = 8 per block).  The K order inside an MMA is
-// permuted so that each lane's 32 packed nibbles map onto its own fragment
-// slots; x is gathered in the same order, which leaves each dot product
-// unchanged.
+// registers (16 rows x 16 K per MMA, one 16-byte load per lane and row and
+// group), tokens the B operand (n = 8 per token block).  The K order inside
+// an MMA is permuted so that each lane's 32 packed nibbles of a group map onto
+// its own fragment slots; x is gathered in the same order, which leaves each
+// dot product unchanged.
 //
-// Work split: a persistent grid of one (M <= 8: two) CTAs per SM; CTA c owns
-// a contiguous run of 16-row blocks (at most MB).  A producer warp streams,
-// two K groups at a time, the packed weights of those rows (one 16-row x
-// 128-byte TMA box per block: whole 128-byte lines of every row, which DRAM
-// serves best) and the matching x tile into an 8-deep shared-memory ring;
-// consumer warp w takes stages w, w + 8, ... (ring slot w), reads its x
-// fragments once per group and uses them for all of the CTA's row blocks, two
-// blocks at a time so that independent MMA chains overlap.  The 8 partial
-// sums of each output meet in shared memory at the end.
+// Work split: one CTA per SM owns a contiguous run of 16-row blocks (at most
+// kW16MB).  A unit of work is one K group pair x one block pair: a 32-row x
+// 128-byte TMA box (4 KB; smaller boxes leave the copy engine, not DRAM, as
+// the limit).  The run's units, in pair-major order, are split into equal
+// contiguous ranges, one per warp, so a warp mostly stays on one group pair.  Every warp is
+// its own producer: its lane 0 keeps the warp's next units in flight in a
+// private ring, so no warp waits for another until the end.  A warp keeps the
+// x fragments of its current group pair in registers for all blocks of the
+// run, and its running sums in registers; the partial sums of the warps meet
+// in shared memory once at the end.  Scales and zero points of the run's rows
+// are copied to shared memory once, transposed to [group][row] so that the 8
+// rows an MMA fragment touches are adjacent (conflict-free reads).
 //
 // The weight boxes use the 128-byte swizzle (16-byte chunk c of smem row r at
-// c ^ (r & 7)).  The two rows an 8-lane phase reads would hit the same banks,
-// so MMA row m holds weight row pi(m) = 4 (m & 1) + (m >> 1) (m < 8; +8 above),
-// which puts them 4 rows apart and onto disjoint chunk sets: conflict-free.
+// c ^ (r & 7)).  The two rows an 8-lane phase reads would share banks, so MMA
+// row m holds weight row pi(m) = 4 (m & 1) + (m >> 1) (m < 8; +8 above), which
+// puts them 4 rows apart and onto disjoint chunk sets: conflict-free.
+//
+// Launched with programmatic dependent launch: the CTA sets up its barriers
+// while the previous kernel of the stream drains, and waits for it before
+// the first read of any input.
 #pragma once
 
 #include "ptx.cuh"
 
 namespace tint4 {
 
-constexpr int kW16Warps = 8;
-constexpr int kW16Threads = kW16Warps * 32;
-constexpr int kW16Group = 128;       // K values per quantization group
+constexpr int kW16Group = 128;      // K values per quantization group
+constexpr int kW16Box = 32 * 128;   // one unit: 2 row blocks x 2 groups of packed bytes
+constexpr int kW16Ring = 128 * 1024;  // all warps' rings
+constexpr int kW16MB = 8;           // 16-row blocks per CTA at most
+constexpr int kW16Rows = kW16MB * 16;
+constexpr int kW16MaxK = 16384;
+constexpr int kW16MaxM = 16;        // tokens per launch (the host splits larger batches)
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
                                                const uint32_t b0, const uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
         "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// nibbles (i, i + 4) of a packed word -> bf16x2 (128 + q_i, 128 + q_{i+4})
-__device__ __forceinline__ uint32_t nib_pair_bf16(uint32_t w, int i) {
-    return ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+// Constants of the nibble unpack, passed as a kernel parameter: the compiler
+// then takes them as constant-bank operands instead of rebuilding them in
+// registers around every use (two bit operations per pair instead of one).
+struct W16Consts {
+    uint32_t mask;    // 0x000F000F: the low nibble of each 16-bit half
+    uint32_t base;    // 0x43004300: bf16x2 (128, 128)
+};
+
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t m, uint32_t o) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(m), "r"(o));   // (a & m) | o
+    return d;
 }
 
-// elementwise a - b of two bf16 pairs (exact here: small integers)
-__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
+// One packed word (nibbles q0..q7, q_i at bits 4i) to the four bf16x2 pairs
+// (128 + q0, 128 + q4), (128 + q1, 128 + q5), (128 + q2, 128 + q6),
+// (128 + q3, 128 + q7), all exact: a nibble OR-ed into the low mantissa bits
+// of bf16 128 (0x4300) adds its value (the 7-bit mantissa has room for 4 bits
+// only at the bottom, so the upper nibbles are shifted down first).  Seven
+// ALU instructions per 8 weights: this is what bounds the kernel's math.
+__device__ __forceinline__ void unpack_word(uint32_t w, const W16Consts& c, uint32_t (&p)[4]) {
+    p[0] = and_or(w, c.mask, c.base);
+    p[1] = and_or(w >> 4, c.mask, c.base);
+    p[2] = and_or(w >> 8, c.mask, c.base);
+    p[3] = and_or(w >> 12, c.mask, c.base);
 }
 
 // x values 8w .. 8w + 7 of a lane's slice (one 16-byte word q, bf16) to the
@@ -79,269 +106,327 @@ __device__ __forceinline__ void x_frag(const uint4& q, uint32_t (&f0)[2], uint32
     f1[1] = __byte_perm(q.y, q.w, 0x7632);
 }
 
-constexpr int kW16Stages = 8;        // = consumer warps: warp w owns ring slot w
-constexpr int kW16Threads9 = (kW16Warps + 1) * 32;   // + the TMA producer warp
-constexpr int kW16GPS = 2;           // K groups per stage (128 packed bytes per row)
-constexpr int kW16MaxK = 16384;      // scales / zero points of a CTA's rows stay in shared memory
-
 // MMA row m (0..15) of a block holds weight row w16_perm(m) of the block
 __host__ __device__ constexpr int w16_perm(int m) {
     return (m & 8) | ((m & 1) << 2) | ((m >> 1) & 3);
 }
 
-template <int NB, int MB>
-struct W16Layout {
-    static constexpr int kBoxBytes = 16 * 128;                          // one block, two groups
-    static constexpr int kWBytes = MB * kBoxBytes;
-    static constexpr int kXBytes = 8 * NB * kW16GPS * kW16Group * 2;     // x tile, two groups
-    static constexpr int kStage = kWBytes + kXBytes;
-    static constexpr int kRedBytes = kW16Warps * MB * NB * 32 * 16;
-    static constexpr int kBarOff = kW16Stages * kStage > kRedBytes ? kW16Stages * kStage : kRedBytes;
-    static constexpr int kSzOff = kBarOff + (2 * kW16Stages + 1) * 8 + 120;
-    // the CTA's rows of scale (bf16) and zero point (uint8), all groups, as
-    // they lie in global memory
-    __host__ __device__ static constexpr int smem(int ngroups) {
-        return kSzOff + MB * 16 * ngroups * 3 + 16 + 1024;   // + 1024: base alignment
+// NB 8-token blocks with WARPS warps: the running sums (kW16MB blocks x NB x 4
+// floats) and the x fragments of a group pair (NB x 32 words) stay in
+// registers, so NB = 2 runs 8 warps (255 registers each), NB = 1 16 warps.
+// The ring takes what shared memory the scales and zero points leave: every
+// warp's units are in flight at once for the decode shapes.
+template <int NB>
+struct W16Cfg {
+    static constexpr int WARPS = NB == 1 ? 12 : 8;
+    static constexpr int THREADS = WARPS * 32;
+    static constexpr int kMaxSlots = 8;
+    static constexpr int kBarBytes = WARPS * kMaxSlots * 8 + 16;   // + abort flag
+    static constexpr int kRedBytes = WARPS * kW16MB * NB * 32 * 16;   // reuses the ring
+    static constexpr int kSmemMax = 227 * 1024;
+    // boxes in flight per warp for a K of ngroups groups
+    __host__ __device__ static constexpr int slots(int ngroups) {
+        return (kSmemMax - 1024 - kBarBytes - ngroups * kW16Rows * 4) / (WARPS * kW16Box) < kMaxSlots
+                   ? (kSmemMax - 1024 - kBarBytes - ngroups * kW16Rows * 4) / (WARPS * kW16Box)
+                   : kMaxSlots;
     }
-    static_assert(kStage % 1024 == 0, "swizzled boxes need 1 KB alignment");
+    __host__ __device__ static constexpr int ring_bytes(int ngroups) {
+        return slots(ngroups) * WARPS * kW16Box;
+    }
+    // ring | barriers | transposed scales and -(128 + zero point) (bf16 each) of kW16Rows rows
+    __host__ __device__ static constexpr int smem(int ngroups) {
+        return ring_bytes(ngroups) + kBarBytes + ngroups * kW16Rows * 4 + 1024;   // + 1024: alignment
+    }
+    static_assert(kRedBytes <= 2 * WARPS * kW16Box, "the reduction reuses the ring");
+    static_assert((kSmemMax - 1024 - kBarBytes - (kW16MaxK / kW16Group) * kW16Rows * 4) /
+                          (WARPS * kW16Box) >= 2,
+                  "double buffering at least, at the largest K");
 };
 
-// NB = number of 8-token blocks (M <= 8 * NB); MB = 16-row blocks per CTA at most.
-template <int NB, int MB>
-__global__ void __launch_bounds__(kW16Threads9, 1)
-w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+// NB = number of 8-token blocks (M <= 8 * NB <= 16).
+template <int NB>
+__global__ void __launch_bounds__(W16Cfg<NB>::THREADS, 1)
+w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16* __restrict__ x,
                  const __nv_bfloat16* __restrict__ wscale, const uint8_t* __restrict__ wzero,
-                 __nv_bfloat16* __restrict__ y, int M, int N, int K, uint64_t wait_ns) {
-    using L = W16Layout<NB, MB>;
+                 __nv_bfloat16* __restrict__ y, int M, int N, int K, const W16Consts kc,
+                 uint64_t wait_ns) {
+    using C = W16Cfg<NB>;
+    constexpr int WARPS = C::WARPS;
     extern __shared__ uint8_t w16_smem_raw[];
-    uint8_t* w16_smem = reinterpret_cast<uint8_t*>(
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(w16_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(w16_smem + L::kBarOff);
-    uint64_t* empty = full + kW16Stages;
-    uint64_t* sz_full = empty + kW16Stages;        // scales + zero points landed
-    volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sz_full + 1);
-    float* red = reinterpret_cast<float*>(w16_smem);   // reused after the main loop
+    const int ngroups = K / kW16Group;
+    const int SLOTS = C::slots(ngroups);
+    const int ring_bytes = SLOTS * WARPS * kW16Box;
+    uint64_t* full_all = reinterpret_cast<uint64_t*>(sm + ring_bytes);
+    volatile uint32_t* abort_flag =
+        reinterpret_cast<volatile uint32_t*>(full_all + WARPS * C::kMaxSlots);
+    float* red = reinterpret_cast<float*>(sm);   // reused after the main loop
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int g = lane >> 2;   // MMA group id: MMA rows g / g + 8, token column g
-    const int t = lane & 3;    // thread in group: which 32-value slice of a K group
-    const int ngroups = K / kW16Group;
-    const int nstages = (ngroups + kW16GPS - 1) / kW16GPS;
-    const int nblk = (N + 15) / 16;
-    // contiguous run of row blocks of this CTA
+    const int t = lane & 3;    // which 32-value slice of a group
+    const int npairs = (ngroups + 1) / 2;
+    const int nblk = N / 16;
     const int b0 = static_cast<int>((static_cast<long long>(blockIdx.x) * nblk) / gridDim.x);
     const int b1 = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * nblk) / gridDim.x);
-    const int nb_here = b1 - b0;   // 1..MB (the host sizes the grid)
+    const int nb = b1 - b0;             // 1..kW16MB (the host sizes the grid)
+    const int nbp = (nb + 1) / 2;       // block pairs (an odd run's last box reads 16 rows it skips)
     const int rA = w16_perm(g), rB = w16_perm(g + 8);   // weight rows of MMA rows g, g + 8
     const int swz = rA & 7;                              // = rB & 7
 
-    const __nv_bfloat16* sScale = reinterpret_cast<const __nv_bfloat16*>(w16_smem + L::kSzOff);
-    const uint8_t* sZero = w16_smem + L::kSzOff + MB * 16 * ngroups * 2;
+    uint16_t* sScale = reinterpret_cast<uint16_t*>(sm + ring_bytes + C::kBarBytes);  // bf16 bits, [group][row]
+    // -(128 + z) as bf16, [group][row]
+    uint16_t* sNegC = reinterpret_cast<uint16_t*>(sm + ring_bytes + C::kBarBytes + ngroups * kW16Rows * 2);
 
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < kW16Stages; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1);
-        }
-        mbar_init(sz_full, 1);
-        *abort_flag = 0u;
+    // the run's units in pair-major order, u = P * nbp + bp; this warp takes
+    // the contiguous, balanced range [u0, u1)
+    const int ntot = npairs * nbp;
+    const int u0 = static_cast<int>((static_cast<long long>(warp) * ntot) / WARPS);
+    const int u1 = static_cast<int>((static_cast<long long>(warp + 1) * ntot) / WARPS);
+    const int nunits = u1 - u0;
+    uint64_t* full = full_all + warp * SLOTS;
+    uint8_t* ring = sm + warp * SLOTS * kW16Box;
+
+    if (lane == 0) {
+        for (int i = 0; i < SLOTS; ++i) mbar_init(&full[i], 1);
+        if (warp == 0) *abort_flag = 0u;
         fence_mbarrier_init();
+        prefetch_tensormap(&tmap_w);
+    }
+    __syncthreads();
+    // inputs may come from the previous kernel of the stream
+    grid_dependency_wait();
+    grid_launch_dependents();
+
+    int issued = 0;
+    auto issue = [&](int i) {
+        const int slot = i % SLOTS;
+        const int P = (u0 + i) / nbp;
+        const int bp = (u0 + i) % nbp;
+        mbar_arrive_expect_tx(&full[slot], kW16Box);
+        tma_load_2d(&tmap_w, &full[slot], ring + slot * kW16Box, P * 128, (b0 + 2 * bp) * 16);
+    };
+    if (lane == 0)
+        for (; issued < SLOTS && issued < nunits; ++issued) issue(issued);
+
+    // scales and zero points of the run's rows (contiguous, [row][group] in
+    // global memory), transposed to [group][row] (the zero point as bf16
+    // -(128 + z), exact): 16-byte loads, all of a thread's issued before the
+    // first is used
+    {
+        const int nel = nb * 16 * ngroups;
+        const size_t base = static_cast<size_t>(b0) * 16 * ngroups;   // 16-byte aligned offsets
+        const uint4* sv = reinterpret_cast<const uint4*>(wscale + base);
+        const uint4* zv = reinterpret_cast<const uint4*>(wzero + base);
+        constexpr int kSV = (kW16Rows * (kW16MaxK / kW16Group) / 8 + C::THREADS - 1) / C::THREADS;
+        constexpr int kZV = (kW16Rows * (kW16MaxK / kW16Group) / 16 + C::THREADS - 1) / C::THREADS;
+        uint4 sreg[kSV], zreg[kZV];
+#pragma unroll
+        for (int i = 0; i < kSV; ++i) {
+            const int v = threadIdx.x + i * C::THREADS;
+            if (v * 8 < nel) sreg[i] = __ldg(sv + v);
+        }
+#pragma unroll
+        for (int i = 0; i < kZV; ++i) {
+            const int v = threadIdx.x + i * C::THREADS;
+            if (v * 16 < nel) zreg[i] = __ldg(zv + v);
+        }
+#pragma unroll
+        for (int i = 0; i < kSV; ++i) {
+            const int v = threadIdx.x + i * C::THREADS;
+            if (v * 8 < nel) {
+                const uint32_t wv[4] = {sreg[i].x, sreg[i].y, sreg[i].z, sreg[i].w};
+                int r = (v * 8) / ngroups, G = v * 8 - r * ngroups;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const uint16_t h = static_cast<uint16_t>(wv[e >> 1] >> (16 * (e & 1)));
+                    sScale[G * kW16Rows + r] = h;
+                    if (++G == ngroups) { G = 0; ++r; }
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kZV; ++i) {
+            const int v = threadIdx.x + i * C::THREADS;
+            if (v * 16 < nel) {
+                const uint32_t wv[4] = {zreg[i].x, zreg[i].y, zreg[i].z, zreg[i].w};
+                int r = (v * 16) / ngroups, G = v * 16 - r * ngroups;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    sNegC[G * kW16Rows + r] = static_cast<uint16_t>(0xC300u + ((wv[e >> 2] >> (8 * (e & 3))) & 0xFFu));
+                    if (++G == ngroups) { G = 0; ++r; }
+                }
+            }
+        }
     }
     __syncthreads();
 
-    float total[MB][NB][4];
+    float total[kW16MB][NB][4];
 #pragma unroll
-    for (int rb = 0; rb < MB; ++rb)
+    for (int j = 0; j < kW16MB; ++j)
 #pragma unroll
         for (int b = 0; b < NB; ++b)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) total[rb][b][j] = 0.0f;
+            for (int q = 0; q < 4; ++q) total[j][b][q] = 0.0f;
 
-    if (warp == kW16Warps) {
-        // ------------------------------------------------ TMA producer
-        if (lane == 0) {
-            prefetch_tensormap(&tmap_w);
-            prefetch_tensormap(&tmap_x);
-            // this CTA's rows of scales and zero points are one contiguous,
-            // 16-byte aligned range each (row starts are multiples of 16)
-            const uint32_t sbytes = nb_here * 16 * ngroups * 2, zbytes = nb_here * 16 * ngroups;
-            mbar_arrive_expect_tx(sz_full, sbytes + zbytes);
-            bulk_load_1d(w16_smem + L::kSzOff, wscale + static_cast<size_t>(b0) * 16 * ngroups,
-                         sbytes, sz_full);
-            bulk_load_1d(w16_smem + L::kSzOff + MB * 16 * ngroups * 2,
-                         wzero + static_cast<size_t>(b0) * 16 * ngroups, zbytes, sz_full);
-            const uint32_t bytes = nb_here * L::kBoxBytes + L::kXBytes;
-            int issued = 0;
-            for (int j = 0; j < nstages; ++j) {
-                const int s = j % kW16Stages;
-                const uint32_t ph = (j / kW16Stages) & 1;
-                if (!mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, wait_ns, kDevErrTimeoutProducer))
-                    break;
-                uint8_t* st = w16_smem + s * L::kStage;
-                mbar_arrive_expect_tx(&full[s], bytes);
-                for (int rb = 0; rb < nb_here; ++rb)
-                    tma_load_2d(&tmap_w, &full[s], st + rb * L::kBoxBytes, j * 128, (b0 + rb) * 16);
-                tma_load_2d(&tmap_x, &full[s], st + L::kWBytes, j * kW16GPS * kW16Group, 0);
-                ++issued;
-            }
-            uint32_t never = 0u;
-            if (*abort_flag) {
-                // let the copies in flight land before the ring is reused or freed
-                (void)mbar_wait_bounded(sz_full, 0, &never, wait_ns, 0u);
-                for (int j = (issued > kW16Stages ? issued - kW16Stages : 0); j < issued; ++j)
-                    (void)mbar_wait_bounded(&full[j % kW16Stages], (j / kW16Stages) & 1, &never,
-                                            wait_ns, 0u);
-            }
-        }
-    } else {
-        // ------------------------------------------------ consumers
-        int szok = 0;
-        if (lane == 0) szok = mbar_wait_bounded(sz_full, 0, abort_flag, wait_ns, kDevErrTimeoutConsumer);
-        if (__shfl_sync(0xFFFFFFFFu, szok, 0) == 0) goto consumers_done;
-        for (int j = warp; j < nstages; j += kW16Warps) {
-            const int s = j % kW16Stages;
-            const uint32_t ph = (j / kW16Stages) & 1;
-            int ok = 0;
-            if (lane == 0) ok = mbar_wait_bounded(&full[s], ph, abort_flag, wait_ns, kDevErrTimeoutConsumer);
-            if (__shfl_sync(0xFFFFFFFFu, ok, 0) == 0) break;
-            const uint8_t* st = w16_smem + s * L::kStage;
-#pragma unroll 1
-            for (int gi = 0; gi < kW16GPS; ++gi) {
-                const int G = j * kW16GPS + gi;
-                if (G >= ngroups) break;   // warp-uniform
-                // x fragments: token 8b + g, values 32t .. 32t + 31 of group G,
-                // regrouped into the MMA's B layout
-                // (with 4 token blocks the fragments of all 8 k steps would not
-                // fit next to the sums: then they are re-read per row pair)
-                constexpr bool kXReload = NB >= 4;
-                const uint8_t* xg = st + L::kWBytes + g * (kW16GPS * kW16Group * 2) + gi * (kW16Group * 2) + 64 * t;
-                uint32_t bfr[kXReload ? 1 : NB][kXReload ? 1 : 8][2];
-                if constexpr (!kXReload) {
+    int consumed = 0, cslot = 0;
+    uint32_t cphase = 0u;
+    bool aborted = false;
+    const int P0 = u0 / nbp, P1 = nunits > 0 ? (u1 - 1) / nbp : P0 - 1;
+    for (int P = P0; P <= P1 && !aborted; ++P) {
+        const int bp_lo = P == P0 ? u0 % nbp : 0;                 // this warp's block pairs of pair P
+        const int bp_hi = P == P1 ? (u1 - 1) % nbp + 1 : nbp;
+        const bool two = 2 * P + 1 < ngroups;   // an odd group count's last pair has one
+        // (a missing second group gets x = 0: its sums vanish, whatever its box holds)
+        // x fragments of groups 2P, 2P + 1: token 8b + g, values 32t .. 32t + 31,
+        // in the MMA's B layout (zeros for tokens >= M and for a missing group)
+        uint32_t bfr[2][NB][8][2];
 #pragma unroll
-                    for (int b = 0; b < NB; ++b) {
-                        const uint8_t* xr = xg + 8 * b * (kW16GPS * kW16Group * 2);
+        for (int gi = 0; gi < 2; ++gi)
 #pragma unroll
-                        for (int w = 0; w < 4; ++w) {
-                            const uint4 q = lds128(xr + 16 * w);
-                            x_frag(q, bfr[b][2 * w], bfr[b][2 * w + 1]);
-                        }
+            for (int b = 0; b < NB; ++b) {
+                const int tok = 8 * b + g;
+                if (tok < M && (gi == 0 || two)) {
+                    const uint4* xr = reinterpret_cast<const uint4*>(
+                        x + static_cast<size_t>(tok) * K + (2 * P + gi) * kW16Group + 32 * t);
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const uint4 q = __ldg(xr + w);
+                        x_frag(q, bfr[gi][b][2 * w], bfr[gi][b][2 * w + 1]);
                     }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) bfr[gi][b][k][0] = bfr[gi][b][k][1] = 0u;
                 }
-                // this lane's 16-byte chunk of group G in rows rA / rB (swizzled)
-                const int chunk_off = ((4 * gi + t) ^ swz) << 4;
-                // row blocks in pairs: two independent dequant + MMA chains per
-                // k step keep the tensor pipe and the ALUs busy together
+            }
+        // per-group sums of x (tokens 8b + 2t, 8b + 2t + 1 in [0], [1]: the MMA's
+        // accumulator layout) from an all-ones weight tile
+        float xs[2][NB][4];
+        {
+            const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};
 #pragma unroll
-                for (int rp = 0; rp < MB; rp += 2) {
-                    if (rp >= nb_here) break;   // CTA-uniform
-                    uint32_t wa[2][4], wb[2][4], zA[2], zB[2];
-                    float sA[2], sB[2];
+            for (int gi = 0; gi < 2; ++gi)
 #pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        // a missing second block (odd count) reads a stale box;
-                        // its sums are dropped below
-                        const int rb = min(rp + p, MB - 1);
-                        const uint8_t* box = st + rb * L::kBoxBytes;
-                        const uint4 pa = lds128(box + rA * 128 + chunk_off);
-                        const uint4 pb = lds128(box + rB * 128 + chunk_off);
-                        wa[p][0] = pa.x; wa[p][1] = pa.y; wa[p][2] = pa.z; wa[p][3] = pa.w;
-                        wb[p][0] = pb.x; wb[p][1] = pb.y; wb[p][2] = pb.z; wb[p][3] = pb.w;
-                        sA[p] = __bfloat162float(sScale[(rb * 16 + rA) * ngroups + G]);
-                        sB[p] = __bfloat162float(sScale[(rb * 16 + rB) * ngroups + G]);
-                        // bf16x2 (128 + z, 128 + z): subtracting it from (128 + q) leaves q - z exactly
-                        zA[p] = 0x43004300u | (0x00010001u * sZero[(rb * 16 + rA) * ngroups + G]);
-                        zB[p] = 0x43004300u | (0x00010001u * sZero[(rb * 16 + rB) * ngroups + G]);
-                    }
-                    float acc[2][NB][4];
+                for (int b = 0; b < NB; ++b) {
 #pragma unroll
-                    for (int p = 0; p < 2; ++p)
+                    for (int q = 0; q < 4; ++q) xs[gi][b][q] = 0.0f;
 #pragma unroll
-                        for (int b = 0; b < NB; ++b)
+                    for (int k = 0; k < 8; ++k)
+                        mma_bf16_16816(xs[gi][b], ones, bfr[gi][b][k][0], bfr[gi][b][k][1]);
+                }
+        }
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) acc[p][b][q] = 0.0f;
+        for (int bp = 0; bp < kW16MB / 2; ++bp) {
+            if (bp >= bp_hi) break;   // warp-uniform
+            if (bp < bp_lo) continue;
+            const int slot = cslot;
+            int ok = 0;
+            if (lane == 0)
+                ok = mbar_wait_bounded(&full[slot], cphase, abort_flag, wait_ns, kDevErrTimeoutConsumer);
+            if (__shfl_sync(0xFFFFFFFFu, ok, 0) == 0) { aborted = true; break; }
+            const uint8_t* box = ring + slot * kW16Box;
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const int w = k >> 1;          // packed word of this lane's 16 bytes
-                        const int i0 = 2 * (k & 1);    // nibble pairs (i0, i0+4) and (i0+1, i0+5)
-                        uint32_t bk[NB][2];
-                        if constexpr (kXReload) {
-                            uint32_t unused[2];
+            for (int hb = 0; hb < 2; ++hb) {
+                const int j = 2 * bp + hb;         // block of the run
+                if (j >= nb) break;                // CTA-uniform
+                const uint8_t* bbox = box + hb * 16 * 128;
 #pragma unroll
-                            for (int b = 0; b < NB; ++b) {
-                                const uint4 q = lds128(xg + 8 * b * (kW16GPS * kW16Group * 2) + 16 * w);
-                                if (k & 1) x_frag(q, unused, bk[b]);
-                                else x_frag(q, bk[b], unused);
-                            }
-                        } else {
+                for (int gi = 0; gi < 2; ++gi) {
+                    // this lane's 16-byte chunk of group 2P + gi in rows rA / rB (swizzled)
+                    const int coff = ((4 * gi + t) ^ swz) << 4;
+                    const uint4 pa = *reinterpret_cast<const uint4*>(bbox + rA * 128 + coff);
+                    const uint4 pb = *reinterpret_cast<const uint4*>(bbox + rB * 128 + coff);
+                    const int G = min(2 * P + gi, ngroups - 1);   // a missing group has x = 0
+                    const int r = j * 16;
+                    const float sA = __uint_as_float(static_cast<uint32_t>(sScale[G * kW16Rows + r + rA]) << 16);
+                    const float sB = __uint_as_float(static_cast<uint32_t>(sScale[G * kW16Rows + r + rB]) << 16);
+                    const float cA = __uint_as_float(static_cast<uint32_t>(sNegC[G * kW16Rows + r + rA]) << 16);
+                    const float cB = __uint_as_float(static_cast<uint32_t>(sNegC[G * kW16Rows + r + rB]) << 16);
+                    const uint32_t wa[4] = {pa.x, pa.y, pa.z, pa.w};
+                    const uint32_t wb[4] = {pb.x, pb.y, pb.z, pb.w};
+                    float acc[NB][4];
 #pragma unroll
-                            for (int b = 0; b < NB; ++b) { bk[b][0] = bfr[b][k][0]; bk[b][1] = bfr[b][k][1]; }
-                        }
+                    for (int b = 0; b < NB; ++b)
 #pragma unroll
-                        for (int p = 0; p < 2; ++p) {
-                            uint32_t a[4];
-                            a[0] = bf16x2_sub(nib_pair_bf16(wa[p][w], i0), zA[p]);       // MMA row g,   k 2t, 2t+1
-                            a[1] = bf16x2_sub(nib_pair_bf16(wb[p][w], i0), zB[p]);       // MMA row g+8, k 2t, 2t+1
-                            a[2] = bf16x2_sub(nib_pair_bf16(wa[p][w], i0 + 1), zA[p]);   // MMA row g,   k 2t+8, 2t+9
-                            a[3] = bf16x2_sub(nib_pair_bf16(wb[p][w], i0 + 1), zB[p]);   // MMA row g+8, k 2t+8, 2t+9
+                        for (int q = 0; q < 4; ++q) acc[b][q] = 0.0f;
 #pragma unroll
-                            for (int b = 0; b < NB; ++b)
-                                mma_bf16_16816(acc[p][b], a, bk[b][0], bk[b][1]);
+                    for (int w = 0; w < 4; ++w) {
+                        // packed word w of rows rA / rB: k steps 2w (pairs (0,4), (1,5))
+                        // and 2w + 1 (pairs (2,6), (3,7))
+                        uint32_t da[4], db[4];
+                        unpack_word(wa[w], kc, da);
+                        unpack_word(wb[w], kc, db);
+                        const uint32_t a0[4] = {da[0], db[0], da[1], db[1]};   // rows g, g+8 x k 2t.., 2t+8..
+                        const uint32_t a1[4] = {da[2], db[2], da[3], db[3]};
+#pragma unroll
+                        for (int b = 0; b < NB; ++b) {
+                            mma_bf16_16816(acc[b], a0, bfr[gi][b][2 * w][0], bfr[gi][b][2 * w][1]);
+                            mma_bf16_16816(acc[b], a1, bfr[gi][b][2 * w + 1][0], bfr[gi][b][2 * w + 1][1]);
                         }
                     }
                     // acc: [0] MMA row g / token 8b+2t, [1] row g / 8b+2t+1,
                     //      [2] MMA row g+8 / 8b+2t,     [3] row g+8 / 8b+2t+1
 #pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        if (rp + p >= MB || rp + p >= nb_here) break;
-#pragma unroll
-                        for (int b = 0; b < NB; ++b) {
-                            total[rp + p][b][0] = fmaf(sA[p], acc[p][b][0], total[rp + p][b][0]);
-                            total[rp + p][b][1] = fmaf(sA[p], acc[p][b][1], total[rp + p][b][1]);
-                            total[rp + p][b][2] = fmaf(sB[p], acc[p][b][2], total[rp + p][b][2]);
-                            total[rp + p][b][3] = fmaf(sB[p], acc[p][b][3], total[rp + p][b][3]);
-                        }
+                    for (int b = 0; b < NB; ++b) {
+                        total[j][b][0] = fmaf(sA, fmaf(cA, xs[gi][b][0], acc[b][0]), total[j][b][0]);
+                        total[j][b][1] = fmaf(sA, fmaf(cA, xs[gi][b][1], acc[b][1]), total[j][b][1]);
+                        total[j][b][2] = fmaf(sB, fmaf(cB, xs[gi][b][0], acc[b][2]), total[j][b][2]);
+                        total[j][b][3] = fmaf(sB, fmaf(cB, xs[gi][b][1], acc[b][3]), total[j][b][3]);
                     }
                 }
             }
+            ++consumed;
+            if (++cslot == SLOTS) { cslot = 0; cphase ^= 1u; }
+            // the slot is free again: refill it with this warp's unit SLOTS ahead
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
+            if (lane == 0 && issued < nunits) {
+                fence_proxy_async_smem();
+                issue(issued);
+                ++issued;
+            }
         }
-    consumers_done:;
+    }
+    if (aborted && lane == 0) {
+        // let this warp's copies in flight land before the ring is reused
+        uint32_t never = 0u;
+        for (int i = consumed; i < issued; ++i)
+            (void)mbar_wait_bounded(&full[i % SLOTS], (i / SLOTS) & 1, &never, wait_ns, 0u);
     }
 
-    // ---- the 8 consumer warps' partial sums meet in shared memory (the ring
-    // is idle once every warp is here: each stage was released after use)
+    // ---- the warps' partial sums meet in shared memory
     __syncthreads();
-    if (warp < kW16Warps) {
 #pragma unroll
-        for (int rb = 0; rb < MB; ++rb)
+    for (int j = 0; j < kW16MB; ++j) {
+        if (j >= nb) break;
 #pragma unroll
-            for (int b = 0; b < NB; ++b)
-                *reinterpret_cast<float4*>(red + (((warp * MB + rb) * NB + b) * 32 + lane) * 4) =
-                    make_float4(total[rb][b][0], total[rb][b][1], total[rb][b][2], total[rb][b][3]);
+        for (int b = 0; b < NB; ++b)
+            *reinterpret_cast<float4*>(red + (((warp * kW16MB + j) * NB + b) * 32 + lane) * 4) =
+                make_float4(total[j][b][0], total[j][b][1], total[j][b][2], total[j][b][3]);
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < nb_here * NB * 32; e += kW16Threads9) {
+    if (*abort_flag) return;   // the device error word says why; y is left as it was
+    for (int e = threadIdx.x; e < nb * NB * 32; e += C::THREADS) {
         const int ln = e & 31;
         const int b = (e >> 5) % NB;
-        const int rb = (e >> 5) / NB;
+        const int j = (e >> 5) / NB;
         float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-        for (int w = 0; w < kW16Warps; ++w) {
-            const float4 p = *reinterpret_cast<const float4*>(red + (((w * MB + rb) * NB + b) * 32 + ln) * 4);
+        for (int w = 0; w < WARPS; ++w) {
+            const float4 p = *reinterpret_cast<const float4*>(red + (((w * kW16MB + j) * NB + b) * 32 + ln) * 4);
             v[0] += p.x; v[1] += p.y; v[2] += p.z; v[3] += p.w;
         }
         const int gg = ln >> 2, tt = ln & 3;
         const int tok0 = 8 * b + 2 * tt;
-        const int r0 = (b0 + rb) * 16 + w16_perm(gg), r1 = (b0 + rb) * 16 + w16_perm(gg + 8);
+        const int r0 = (b0 + j) * 16 + w16_perm(gg), r1 = (b0 + j) * 16 + w16_perm(gg + 8);
         if (tok0 < M) {
-            if (r0 < N) y[static_cast<size_t>(tok0) * N + r0] = __float2bfloat16_rn(v[0]);
-            if (r1 < N) y[static_cast<size_t>(tok0) * N + r1] = __float2bfloat16_rn(v[2]);
+            y[static_cast<size_t>(tok0) * N + r0] = __float2bfloat16_rn(v[0]);
+            y[static_cast<size_t>(tok0) * N + r1] = __float2bfloat16_rn(v[2]);
         }
         if (tok0 + 1 < M) {
-            if (r0 < N) y[static_cast<size_t>(tok0 + 1) * N + r0] = __float2bfloat16_rn(v[1]);
-            if (r1 < N) y[static_cast<size_t>(tok0 + 1) * N + r1] = __float2bfloat16_rn(v[3]);
+            y[static_cast<size_t>(tok0 + 1) * N + r0] = __float2bfloat16_rn(v[1]);
+            y[static_cast<size_t>(tok0 + 1) * N + r1] = __float2bfloat16_rn(v[3]);
         }
     }
 }
