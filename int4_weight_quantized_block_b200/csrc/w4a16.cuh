@@ -34,8 +34,8 @@
 // x fragments of its current group pair in registers for all blocks of the
 // run, and its running sums in registers; the partial sums of the warps meet
 // in shared memory once at the end.  Scales and zero points of the run's rows
-// are copied to shared memory once, transposed to [group][row] so that the 8
-// rows an MMA fragment touches are adjacent (conflict-free reads).
+// are copied to shared memory once, by two bulk copies issued ahead of the
+// weight boxes.
 //
 // The weight boxes use the 128-byte swizzle (16-byte chunk c of smem row r at
 // c ^ (r & 7)).  The two rows an 8-lane phase reads would share banks, so MMA
@@ -121,24 +121,24 @@ struct W16Cfg {
     static constexpr int WARPS = NB == 1 ? 12 : 8;
     static constexpr int THREADS = WARPS * 32;
     static constexpr int kMaxSlots = 8;
-    static constexpr int kBarBytes = WARPS * kMaxSlots * 8 + 16;   // + abort flag
+    static constexpr int kBarBytes = WARPS * kMaxSlots * 8 + 16;   // + scale/zero barrier, abort flag
     static constexpr int kRedBytes = WARPS * kW16MB * NB * 32 * 16;   // reuses the ring
     static constexpr int kSmemMax = 227 * 1024;
     // boxes in flight per warp for a K of ngroups groups
     __host__ __device__ static constexpr int slots(int ngroups) {
-        return (kSmemMax - 1024 - kBarBytes - ngroups * kW16Rows * 4) / (WARPS * kW16Box) < kMaxSlots
-                   ? (kSmemMax - 1024 - kBarBytes - ngroups * kW16Rows * 4) / (WARPS * kW16Box)
+        return (kSmemMax - 1024 - kBarBytes - ngroups * kW16Rows * 3) / (WARPS * kW16Box) < kMaxSlots
+                   ? (kSmemMax - 1024 - kBarBytes - ngroups * kW16Rows * 3) / (WARPS * kW16Box)
                    : kMaxSlots;
     }
     __host__ __device__ static constexpr int ring_bytes(int ngroups) {
         return slots(ngroups) * WARPS * kW16Box;
     }
-    // ring | barriers | transposed scales and -(128 + zero point) (bf16 each) of kW16Rows rows
+    // ring | barriers | scales (bf16) and zero points (uint8) of up to kW16Rows rows, as in global memory
     __host__ __device__ static constexpr int smem(int ngroups) {
-        return ring_bytes(ngroups) + kBarBytes + ngroups * kW16Rows * 4 + 1024;   // + 1024: alignment
+        return ring_bytes(ngroups) + kBarBytes + ngroups * kW16Rows * 3 + 1024;   // + 1024: alignment
     }
     static_assert(kRedBytes <= 2 * WARPS * kW16Box, "the reduction reuses the ring");
-    static_assert((kSmemMax - 1024 - kBarBytes - (kW16MaxK / kW16Group) * kW16Rows * 4) /
+    static_assert((kSmemMax - 1024 - kBarBytes - (kW16MaxK / kW16Group) * kW16Rows * 3) /
                           (WARPS * kW16Box) >= 2,
                   "double buffering at least, at the largest K");
 };
@@ -159,8 +159,8 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
     const int SLOTS = C::slots(ngroups);
     const int ring_bytes = SLOTS * WARPS * kW16Box;
     uint64_t* full_all = reinterpret_cast<uint64_t*>(sm + ring_bytes);
-    volatile uint32_t* abort_flag =
-        reinterpret_cast<volatile uint32_t*>(full_all + WARPS * C::kMaxSlots);
+    uint64_t* sz_full = full_all + WARPS * C::kMaxSlots;   // scales + zero points landed
+    volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sz_full + 1);
     float* red = reinterpret_cast<float*>(sm);   // reused after the main loop
 
     const int warp = threadIdx.x >> 5;
@@ -176,9 +176,9 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
     const int rA = w16_perm(g), rB = w16_perm(g + 8);   // weight rows of MMA rows g, g + 8
     const int swz = rA & 7;                              // = rB & 7
 
-    uint16_t* sScale = reinterpret_cast<uint16_t*>(sm + ring_bytes + C::kBarBytes);  // bf16 bits, [group][row]
-    // -(128 + z) as bf16, [group][row]
-    uint16_t* sNegC = reinterpret_cast<uint16_t*>(sm + ring_bytes + C::kBarBytes + ngroups * kW16Rows * 2);
+    // the run's rows of scale (bf16 bits) and zero point, [row][group] as in global memory
+    const uint16_t* sScale = reinterpret_cast<const uint16_t*>(sm + ring_bytes + C::kBarBytes);
+    const uint8_t* sZero = sm + ring_bytes + C::kBarBytes + ngroups * kW16Rows * 2;
 
     // the run's units in pair-major order, u = P * nbp + bp; this warp takes
     // the contiguous, balanced range [u0, u1)
@@ -191,7 +191,10 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
 
     if (lane == 0) {
         for (int i = 0; i < SLOTS; ++i) mbar_init(&full[i], 1);
-        if (warp == 0) *abort_flag = 0u;
+        if (warp == 0) {
+            *abort_flag = 0u;
+            mbar_init(sz_full, 1);
+        }
         fence_mbarrier_init();
         prefetch_tensormap(&tmap_w);
     }
@@ -201,6 +204,7 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
     grid_launch_dependents();
 
     int issued = 0;
+    bool nunits_ok = true;
     auto issue = [&](int i) {
         const int slot = i % SLOTS;
         const int P = (u0 + i) / nbp;
@@ -208,60 +212,24 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
         mbar_arrive_expect_tx(&full[slot], kW16Box);
         tma_load_2d(&tmap_w, &full[slot], ring + slot * kW16Box, P * 128, (b0 + 2 * bp) * 16);
     };
+    // The run's scales and zero points (two contiguous, 16-byte aligned
+    // ranges) go out first, as two bulk copies: behind tens of MB of weight
+    // boxes they would hold up every warp's first unit.
+    if (threadIdx.x == 0) {
+        const uint32_t sbytes = nb * 16 * ngroups * 2, zbytes = nb * 16 * ngroups;
+        const size_t base = static_cast<size_t>(b0) * 16 * ngroups;
+        mbar_arrive_expect_tx(sz_full, sbytes + zbytes);
+        bulk_load_1d(sm + ring_bytes + C::kBarBytes, wscale + base, sbytes, sz_full);
+        bulk_load_1d(sm + ring_bytes + C::kBarBytes + ngroups * kW16Rows * 2, wzero + base, zbytes, sz_full);
+    }
+    __syncwarp();
     if (lane == 0)
         for (; issued < SLOTS && issued < nunits; ++issued) issue(issued);
-
-    // scales and zero points of the run's rows (contiguous, [row][group] in
-    // global memory), transposed to [group][row] (the zero point as bf16
-    // -(128 + z), exact): 16-byte loads, all of a thread's issued before the
-    // first is used
     {
-        const int nel = nb * 16 * ngroups;
-        const size_t base = static_cast<size_t>(b0) * 16 * ngroups;   // 16-byte aligned offsets
-        const uint4* sv = reinterpret_cast<const uint4*>(wscale + base);
-        const uint4* zv = reinterpret_cast<const uint4*>(wzero + base);
-        constexpr int kSV = (kW16Rows * (kW16MaxK / kW16Group) / 8 + C::THREADS - 1) / C::THREADS;
-        constexpr int kZV = (kW16Rows * (kW16MaxK / kW16Group) / 16 + C::THREADS - 1) / C::THREADS;
-        uint4 sreg[kSV], zreg[kZV];
-#pragma unroll
-        for (int i = 0; i < kSV; ++i) {
-            const int v = threadIdx.x + i * C::THREADS;
-            if (v * 8 < nel) sreg[i] = __ldg(sv + v);
-        }
-#pragma unroll
-        for (int i = 0; i < kZV; ++i) {
-            const int v = threadIdx.x + i * C::THREADS;
-            if (v * 16 < nel) zreg[i] = __ldg(zv + v);
-        }
-#pragma unroll
-        for (int i = 0; i < kSV; ++i) {
-            const int v = threadIdx.x + i * C::THREADS;
-            if (v * 8 < nel) {
-                const uint32_t wv[4] = {sreg[i].x, sreg[i].y, sreg[i].z, sreg[i].w};
-                int r = (v * 8) / ngroups, G = v * 8 - r * ngroups;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const uint16_t h = static_cast<uint16_t>(wv[e >> 1] >> (16 * (e & 1)));
-                    sScale[G * kW16Rows + r] = h;
-                    if (++G == ngroups) { G = 0; ++r; }
-                }
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < kZV; ++i) {
-            const int v = threadIdx.x + i * C::THREADS;
-            if (v * 16 < nel) {
-                const uint32_t wv[4] = {zreg[i].x, zreg[i].y, zreg[i].z, zreg[i].w};
-                int r = (v * 16) / ngroups, G = v * 16 - r * ngroups;
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    sNegC[G * kW16Rows + r] = static_cast<uint16_t>(0xC300u + ((wv[e >> 2] >> (8 * (e & 3))) & 0xFFu));
-                    if (++G == ngroups) { G = 0; ++r; }
-                }
-            }
-        }
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait_bounded(sz_full, 0, abort_flag, wait_ns, kDevErrTimeoutConsumer);
+        if (__shfl_sync(0xFFFFFFFFu, ok, 0) == 0) nunits_ok = false;
     }
-    __syncthreads();
 
     float total[kW16MB][NB][4];
 #pragma unroll
@@ -273,7 +241,7 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
 
     int consumed = 0, cslot = 0;
     uint32_t cphase = 0u;
-    bool aborted = false;
+    bool aborted = !nunits_ok;
     const int P0 = u0 / nbp, P1 = nunits > 0 ? (u1 - 1) / nbp : P0 - 1;
     for (int P = P0; P <= P1 && !aborted; ++P) {
         const int bp_lo = P == P0 ? u0 % nbp : 0;                 // this warp's block pairs of pair P
@@ -340,10 +308,11 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
                     const uint4 pb = *reinterpret_cast<const uint4*>(bbox + rB * 128 + coff);
                     const int G = min(2 * P + gi, ngroups - 1);   // a missing group has x = 0
                     const int r = j * 16;
-                    const float sA = __uint_as_float(static_cast<uint32_t>(sScale[G * kW16Rows + r + rA]) << 16);
-                    const float sB = __uint_as_float(static_cast<uint32_t>(sScale[G * kW16Rows + r + rB]) << 16);
-                    const float cA = __uint_as_float(static_cast<uint32_t>(sNegC[G * kW16Rows + r + rA]) << 16);
-                    const float cB = __uint_as_float(static_cast<uint32_t>(sNegC[G * kW16Rows + r + rB]) << 16);
+                    const float sA = __uint_as_float(static_cast<uint32_t>(sScale[(r + rA) * ngroups + G]) << 16);
+                    const float sB = __uint_as_float(static_cast<uint32_t>(sScale[(r + rB) * ngroups + G]) << 16);
+                    // -(128 + z) exactly: (2^23 - 128) - (2^23 + z)
+                    const float cA = 8388480.0f - __uint_as_float(0x4B000000u | sZero[(r + rA) * ngroups + G]);
+                    const float cB = 8388480.0f - __uint_as_float(0x4B000000u | sZero[(r + rB) * ngroups + G]);
                     const uint32_t wa[4] = {pa.x, pa.y, pa.z, pa.w};
                     const uint32_t wb[4] = {pb.x, pb.y, pb.z, pb.w};
                     float acc[NB][4];
@@ -391,6 +360,7 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
     if (aborted && lane == 0) {
         // let this warp's copies in flight land before the ring is reused
         uint32_t never = 0u;
+        if (warp == 0) (void)mbar_wait_bounded(sz_full, 0, &never, wait_ns, 0u);
         for (int i = consumed; i < issued; ++i)
             (void)mbar_wait_bounded(&full[i % SLOTS], (i / SLOTS) & 1, &never, wait_ns, 0u);
     }
