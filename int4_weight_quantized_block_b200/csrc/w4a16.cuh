@@ -120,7 +120,7 @@ template <int NB>
 struct W16Cfg {
     static constexpr int WARPS = NB == 1 ? 12 : 8;
     static constexpr int THREADS = WARPS * 32;
-    static constexpr int kMaxSlots = 8;
+    static constexpr int kMaxSlots = 2;
     static constexpr int kBarBytes = WARPS * kMaxSlots * 8 + 16;   // + scale/zero barrier, abort flag
     static constexpr int kRedBytes = WARPS * kW16MB * NB * 32 * 16;   // reuses the ring
     static constexpr int kSmemMax = 227 * 1024;
