@@ -398,6 +398,42 @@ def bench_rows(args, t4, inputs, dev, flush, pk, int8_peak):
             "us": round(ms * 1e3, 2), "GBps": round(byts / ms / 1e6, 1),
             "frac_hbm": round(byts / ms / 1e6 / pk["hbm"], 4),
             "timing": "64 calls in one CUDA graph, 8 weight copies rotated (211 MB > L2)"}
+
+    # W4A8 decode (same shape, ConvRot group 256): the fused linear and the GEMM
+    # alone, 8 copies of the packed weights rotated
+    w = inputs.WORKLOADS["te_decode_w4a8"]
+    N, K, g = w["N"], w["K"], w["group"]
+    _, W_np = inputs.layer_inputs("te_decode_w4a8", M=1)
+    wp0, sr0 = t4.tint4_pack_weights(torch.from_numpy(W_np).to(dev), g)
+    del W_np
+    wcopies = [(wp0.clone(), sr0.clone()) for _ in range(8)]
+    for M in w["Ms"]:
+        x_np = inputs.activations(M, K, inputs.SEED)
+        x = bf16_gpu(x_np, dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(t4.convrot_linear_workspace_size(M, K, 8), dtype=torch.uint8, device=dev)
+        codes, st = t4.convrot_quantize_act(x, g, 8)
+
+        def lin(i):
+            wp, sr = wcopies[i % len(wcopies)]
+            t4.convrot_w4a8_linear(x, wp, sr, g, None, y, ws)
+
+        def gem(i):
+            wp, sr = wcopies[i % len(wcopies)]
+            t4.w4a8_gemm(codes, st, wp, sr, None, y)
+
+        l_ms = graph_time(lin, 64, dev)
+        g_ms = graph_time(gem, 64, dev)
+        wbytes = N * K // 2 + N * 4
+        l_bytes = wbytes + M * K * 2 + M * N * 2
+        g_bytes = wbytes + M * K + M * 4 + M * N * 2
+        rows[f"te_decode_w4a8_M{M}"] = {
+            "M": M, "N": N, "K": K, "group": g,
+            "linear_us": round(l_ms * 1e3, 2), "linear_GBps": round(l_bytes / l_ms / 1e6, 1),
+            "linear_frac_hbm": round(l_bytes / l_ms / 1e6 / pk["hbm"], 4),
+            "gemm_us": round(g_ms * 1e3, 2), "gemm_GBps": round(g_bytes / g_ms / 1e6, 1),
+            "gemm_frac_hbm": round(g_bytes / g_ms / 1e6 / pk["hbm"], 4),
+            "timing": "64 calls in one CUDA graph, 8 weight copies rotated (201 MB > L2)"}
     return rows
 
 

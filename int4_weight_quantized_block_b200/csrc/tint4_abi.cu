@@ -16,6 +16,7 @@
 #include "ptx.cuh"
 #include "quantize.cuh"
 #include "w4a16.cuh"
+#include "w4a8_small.cuh"
 
 namespace {
 
@@ -270,11 +271,59 @@ tint4_status launch_gemm_smem_w4a4(const void* a, const uint8_t* w, const float*
     return TINT4_OK;
 }
 
+// Small M (<= kS8MaxM tokens): the warp-MMA kernel that streams the packed
+// weights once (w4a8_small.cuh).
+template <int NB, bool A_INT4, bool OUT_I32>
+tint4_status launch_gemm_small(const void* a, const uint8_t* w, const float* st, const float* sr,
+                               const __nv_bfloat16* bias, void* out, int M, int N, int K,
+                               cudaStream_t stream, bool pdl) {
+    auto kern = w4a8_small_kernel<NB, A_INT4, OUT_I32>;
+    CUtensorMap tw;
+    if (!make_map_u8(&tw, w, K / 2, N, K / 2, 128, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+        return TINT4_ERR_CUDA;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static std::atomic<bool> attr_done[kMaxDevices];
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 S8Cfg<NB>::SMEM) != cudaSuccess) {
+            cudaGetLastError();
+            return TINT4_ERR_CUDA;
+        }
+        attr_done[dev].store(true, std::memory_order_release);
+    }
+    const int nblk = N / 16;
+    // one CTA per SM unless that would give a CTA more than kS8MB blocks
+    const int sms = num_sms(dev);
+    const int grid = nblk <= kS8MB * sms ? std::min(sms, nblk) : (nblk + kS8MB - 1) / kS8MB;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(S8Cfg<NB>::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = S8Cfg<NB>::SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    if (pdl) {
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    if (cudaLaunchKernelEx(&cfg, kern, tw, static_cast<const uint8_t*>(a), st, sr, bias, out, M,
+                           N, K, 0xF0F0F0F0u,
+                           g_wait_limit_ns.load(std::memory_order_relaxed)) != cudaSuccess) {
+        cudaGetLastError();
+        return TINT4_ERR_CUDA;
+    }
+    return last_launch_status();
+}
+
 // A_INT4: activation codes packed two per byte (else int8, one per byte).
 template <bool A_INT4, bool OUT_I32>
 tint4_status launch_gemm(const void* a, const uint8_t* w, const float* st, const float* sr,
                          const __nv_bfloat16* bias, void* out, int M, int N, int K,
                          cudaStream_t stream, bool pdl) {
+    if (M <= 8)
+        return launch_gemm_small<1, A_INT4, OUT_I32>(a, w, st, sr, bias, out, M, N, K, stream, pdl);
+    if (M <= kS8MaxM)
+        return launch_gemm_small<2, A_INT4, OUT_I32>(a, w, st, sr, bias, out, M, N, K, stream, pdl);
     if (A_INT4)
         return launch_gemm_smem_w4a4<OUT_I32>(a, w, st, sr, bias, out, M, N, K, stream, pdl);
     return launch_gemm_tmem<OUT_I32>(a, w, st, sr, bias, out, M, N, K, stream, pdl);

@@ -1,0 +1,282 @@
+// w4a8_small.cuh -- the W4A8 / W4A4 ConvRot GEMM for small M (decode).
+//
+//   acc[m, n] = sum_k qa[m, k] * qw[n, k]            (int32, exact)
+//   y[m, n]   = bf16(float(acc) * s_tok[m] * s_row[n] (+ bias[n]))
+//
+// "ComfyUI-INT-Crush", "Inference > INT4": packed signed int4 weights with a
+// per-row scale, streamed raw and unpacked next to the integer MMA; the
+// activation codes come from the rotate + quantize step (int8 for W4A8, int4
+// packed two per byte for W4A4).
+//
+// With at most 16 tokens every weight is used at most 16 times: the cost is
+// streaming the packed weights (0.5 byte each) from HBM.  The big GEMM's
+// 192-token tiles would waste almost all of their tensor-core work here, so
+// this kernel runs the warp-level int8 MMA (m16n8k32) with the weights as
+// the A operand straight from registers and the tokens as B (n = 8 per
+// block).  A nibble moves into the top half of its byte by one AND (high
+// nibbles) or one shift + AND (low nibbles), which gives the int8 value
+// 16 q exactly; the factor 16 (256 with int4 activations) leaves the int32
+// sums by a shift.  The K order inside an MMA is permuted: each lane takes 8
+// consecutive weights of a row from one packed word, even positions in its
+// first k slot and odd positions in its second, and gathers the activation
+// codes in the same order, which leaves each dot product unchanged.
+//
+// Work split (as the W4A16 kernel): one CTA per SM owns a contiguous run of
+// 16-row blocks (at most kS8MB); a unit is 256 K x one block pair, a 32-row x
+// 128-byte TMA box (4 KB, 128-byte swizzle; MMA row m holds weight row
+// pi(m) = 4 (m & 1) + (m >> 1) (m < 8, +8 above) so that the 8 lanes of a
+// load phase hit disjoint banks).  The run's units, K-chunk-major, are split
+// into equal contiguous ranges, one per warp; every warp is its own TMA
+// producer with a private ring of boxes.  A warp keeps its activation
+// fragments for the current K chunk and its int32 sums for every block of
+// the run in registers; the warps' sums meet in shared memory at the end
+// (integer adds: any order gives the same bits).
+#pragma once
+
+#include "ptx.cuh"
+
+namespace tint4 {
+
+constexpr int kS8Box = 32 * 128;    // one unit: 2 row blocks x 256 K of packed weights
+constexpr int kS8MB = 8;            // 16-row blocks per CTA at most
+constexpr int kS8MaxM = 16;         // tokens per launch
+constexpr int kS8Ring = 128 * 1024;
+
+// The int32 sums of every block of the run (kS8MB x NB x 4) and a K chunk's
+// activation fragments (NB x 16 words) stay in registers: 16 warps of at most
+// 128 registers for one token block, 8 warps of up to 255 for two.
+template <int NB>
+struct S8Cfg {
+    static constexpr int WARPS = NB == 1 ? 16 : 8;
+    static constexpr int THREADS = WARPS * 32;
+    static constexpr int SLOTS = kS8Ring / (WARPS * kS8Box);   // boxes in flight per warp
+    static constexpr int SMEM = kS8Ring + WARPS * SLOTS * 8 + 16 + 1024;   // + barriers, abort flag, alignment
+    static_assert(WARPS * kS8MB * NB * 32 * 16 <= kS8Ring, "the reduction reuses the ring");
+};
+
+// MMA row m (0..15) of a block holds weight row s8_perm(m) of the block
+__host__ __device__ constexpr int s8_perm(int m) {
+    return (m & 8) | ((m & 1) << 2) | ((m >> 1) & 3);
+}
+
+__device__ __forceinline__ void mma_s8_16832(int32_t (&d)[4], const uint32_t (&a)[4],
+                                             uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// NB 8-token blocks (M <= 8 NB <= 16); A_INT4: activation codes packed two
+// per byte; OUT_I32: write the exact int32 sums instead of bf16 (test entry).
+template <int NB, bool A_INT4, bool OUT_I32>
+__global__ void __launch_bounds__(S8Cfg<NB>::THREADS, 1)
+w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __restrict__ act,
+                  const float* __restrict__ tok_scale, const float* __restrict__ row_scale,
+                  const __nv_bfloat16* __restrict__ bias, void* __restrict__ out, int M, int N,
+                  int K, uint32_t hi_mask, uint64_t wait_ns) {
+    using C = S8Cfg<NB>;
+    constexpr int kS8Warps = C::WARPS, kS8Slots = C::SLOTS, kS8Threads = C::THREADS;
+    extern __shared__ uint8_t s8_smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(s8_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* full_all = reinterpret_cast<uint64_t*>(sm + kS8Ring);
+    volatile uint32_t* abort_flag =
+        reinterpret_cast<volatile uint32_t*>(full_all + kS8Warps * kS8Slots);
+    int32_t* red = reinterpret_cast<int32_t*>(sm);   // reused after the main loop
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2;   // MMA group id: MMA rows g / g + 8, token column g
+    const int t = lane & 3;    // which 32-value slice of a 128-K half chunk
+    const int nchunks = (K + 255) / 256;
+    const int nblk = N / 16;
+    const int b0 = static_cast<int>((static_cast<long long>(blockIdx.x) * nblk) / gridDim.x);
+    const int b1 = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * nblk) / gridDim.x);
+    const int nb = b1 - b0;             // 1..kS8MB (the host sizes the grid)
+    const int nbp = (nb + 1) / 2;       // block pairs (an odd run's last box reads 16 rows it skips)
+    const int rA = s8_perm(g), rB = s8_perm(g + 8);
+    const int swz = rA & 7;             // = rB & 7
+
+    // the run's units in chunk-major order, u = P * nbp + bp; this warp's range
+    const int ntot = nchunks * nbp;
+    const int u0 = static_cast<int>((static_cast<long long>(warp) * ntot) / kS8Warps);
+    const int u1 = static_cast<int>((static_cast<long long>(warp + 1) * ntot) / kS8Warps);
+    const int nunits = u1 - u0;
+    uint64_t* full = full_all + warp * kS8Slots;
+    uint8_t* ring = sm + warp * kS8Slots * kS8Box;
+
+    if (lane == 0) {
+        for (int i = 0; i < kS8Slots; ++i) mbar_init(&full[i], 1);
+        if (warp == 0) *abort_flag = 0u;
+        fence_mbarrier_init();
+        prefetch_tensormap(&tmap_w);
+    }
+    __syncthreads();
+    // inputs may come from the previous kernel of the stream
+    grid_dependency_wait();
+    grid_launch_dependents();
+
+    int issued = 0;
+    auto issue = [&](int i) {
+        const int slot = i % kS8Slots;
+        const int P = (u0 + i) / nbp;
+        const int bp = (u0 + i) % nbp;
+        mbar_arrive_expect_tx(&full[slot], kS8Box);
+        tma_load_2d(&tmap_w, &full[slot], ring + slot * kS8Box, P * 128, (b0 + 2 * bp) * 16);
+    };
+    if (lane == 0)
+        for (; issued < kS8Slots && issued < nunits; ++issued) issue(issued);
+
+    int32_t total[kS8MB][NB][4];
+#pragma unroll
+    for (int j = 0; j < kS8MB; ++j)
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) total[j][b][q] = 0;
+
+    int consumed = 0, cslot = 0;
+    uint32_t cphase = 0u;
+    bool aborted = false;
+    const int P0 = u0 / nbp, P1 = nunits > 0 ? (u1 - 1) / nbp : P0 - 1;
+    for (int P = P0; P <= P1 && !aborted; ++P) {
+        const int bp_lo = P == P0 ? u0 % nbp : 0;                 // this warp's block pairs of chunk P
+        const int bp_hi = P == P1 ? (u1 - 1) % nbp + 1 : nbp;
+        // activation fragments of chunk P: token 8b + g, K positions
+        // 256 P + 128 h + 32 t + 8 i + {0, 2, 4, 6} (first slot) and + {1, 3, 5, 7}
+        // (second slot) of MMA i of half h; zeros for tokens >= M and K >= K
+        uint32_t bfr[2][NB][4][2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                const int tok = 8 * b + g;
+                const int kb = 256 * P + 128 * h + 32 * t;   // K % 32 == 0: a slice is all in or all out
+                if (tok < M && kb < K) {
+                    if constexpr (A_INT4) {
+                        const uint4 c = __ldg(reinterpret_cast<const uint4*>(
+                            act + static_cast<size_t>(tok) * (K / 2) + kb / 2));
+                        const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            bfr[h][b][i][0] = (cw[i] << 4) & hi_mask;   // 16 x even positions
+                            bfr[h][b][i][1] = cw[i] & hi_mask;          // 16 x odd positions
+                        }
+                    } else {
+                        const uint4* ar = reinterpret_cast<const uint4*>(act + static_cast<size_t>(tok) * K + kb);
+                        const uint4 c0 = __ldg(ar), c1 = __ldg(ar + 1);
+                        const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            bfr[h][b][i][0] = __byte_perm(cw[2 * i], cw[2 * i + 1], 0x6420);
+                            bfr[h][b][i][1] = __byte_perm(cw[2 * i], cw[2 * i + 1], 0x7531);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) bfr[h][b][i][0] = bfr[h][b][i][1] = 0u;
+                }
+            }
+#pragma unroll
+        for (int bp = 0; bp < kS8MB / 2; ++bp) {
+            if (bp >= bp_hi) break;   // warp-uniform
+            if (bp < bp_lo) continue;
+            const int slot = cslot;
+            int ok = 0;
+            if (lane == 0)
+                ok = mbar_wait_bounded(&full[slot], cphase, abort_flag, wait_ns, kDevErrTimeoutConsumer);
+            if (__shfl_sync(0xFFFFFFFFu, ok, 0) == 0) { aborted = true; break; }
+            const uint8_t* box = ring + slot * kS8Box;
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {
+                const int j = 2 * bp + hb;         // block of the run
+                if (j >= nb) break;                // CTA-uniform
+                const uint8_t* bbox = box + hb * 16 * 128;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    // this lane's 16-byte chunk of half h in rows rA / rB (swizzled)
+                    const int coff = ((4 * h + t) ^ swz) << 4;
+                    const uint4 pa = *reinterpret_cast<const uint4*>(bbox + rA * 128 + coff);
+                    const uint4 pb = *reinterpret_cast<const uint4*>(bbox + rB * 128 + coff);
+                    const uint32_t wa[4] = {pa.x, pa.y, pa.z, pa.w};
+                    const uint32_t wb[4] = {pb.x, pb.y, pb.z, pb.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        // word i: 8 consecutive weights; low nibbles = even positions
+                        uint32_t a[4];
+                        a[0] = (wa[i] << 4) & hi_mask;   // MMA row g,   first slot
+                        a[1] = (wb[i] << 4) & hi_mask;   // MMA row g+8, first slot
+                        a[2] = wa[i] & hi_mask;          // MMA row g,   second slot
+                        a[3] = wb[i] & hi_mask;          // MMA row g+8, second slot
+#pragma unroll
+                        for (int b = 0; b < NB; ++b)
+                            mma_s8_16832(total[j][b], a, bfr[h][b][i][0], bfr[h][b][i][1]);
+                    }
+                }
+            }
+            ++consumed;
+            if (++cslot == kS8Slots) { cslot = 0; cphase ^= 1u; }
+            // the slot is free again: refill it with this warp's unit kS8Slots ahead
+            __syncwarp();
+            if (lane == 0 && issued < nunits) {
+                fence_proxy_async_smem();
+                issue(issued);
+                ++issued;
+            }
+        }
+    }
+    if (aborted && lane == 0) {
+        // let this warp's copies in flight land before the ring is reused
+        uint32_t never = 0u;
+        for (int i = consumed; i < issued; ++i)
+            (void)mbar_wait_bounded(&full[i % kS8Slots], (i / kS8Slots) & 1, &never, wait_ns, 0u);
+    }
+
+    // ---- the warps' partial sums meet in shared memory
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kS8MB; ++j) {
+        if (j >= nb) break;
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+            *reinterpret_cast<int4*>(red + (((warp * kS8MB + j) * NB + b) * 32 + lane) * 4) =
+                make_int4(total[j][b][0], total[j][b][1], total[j][b][2], total[j][b][3]);
+    }
+    __syncthreads();
+    if (*abort_flag) return;   // the device error word says why; the output is left as it was
+    constexpr int kShift = A_INT4 ? 8 : 4;                 // the sums carry 16 (or 256) x
+    constexpr float kUnscale = A_INT4 ? 1.0f / 256.0f : 1.0f / 16.0f;
+    for (int e = threadIdx.x; e < nb * NB * 32; e += kS8Threads) {
+        const int ln = e & 31;
+        const int b = (e >> 5) % NB;
+        const int j = (e >> 5) / NB;
+        int32_t v[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int w = 0; w < kS8Warps; ++w) {
+            const int4 p = *reinterpret_cast<const int4*>(red + (((w * kS8MB + j) * NB + b) * 32 + ln) * 4);
+            v[0] += p.x; v[1] += p.y; v[2] += p.z; v[3] += p.w;
+        }
+        const int gg = ln >> 2, tt = ln & 3;
+        const int tok0 = 8 * b + 2 * tt;
+        const int r0 = (b0 + j) * 16 + s8_perm(gg), r1 = (b0 + j) * 16 + s8_perm(gg + 8);
+        // v: [0] row r0 / token tok0, [1] r0 / tok0 + 1, [2] r1 / tok0, [3] r1 / tok0 + 1
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int tok = tok0 + (q & 1);
+            const int row = (q & 2) ? r1 : r0;
+            if (tok >= M) continue;
+            if constexpr (OUT_I32) {
+                reinterpret_cast<int32_t*>(out)[static_cast<size_t>(tok) * N + row] = v[q] >> kShift;
+            } else {
+                const float bsv = bias ? __bfloat162float(bias[row]) : 0.0f;
+                const float val = static_cast<float>(v[q]) * __ldg(tok_scale + tok) *
+                                  (__ldg(row_scale + row) * kUnscale) + bsv;
+                reinterpret_cast<__nv_bfloat16*>(out)[static_cast<size_t>(tok) * N + row] =
+                    __float2bfloat16_rn(val);
+            }
+        }
+    }
+}
+
+}  // namespace tint4

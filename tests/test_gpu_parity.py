@@ -115,6 +115,64 @@ def test_gemm_bf16_epilogue(M, N, K, act_bits, with_bias):
     assert_gemm_output(bf16_from_gpu(y), y_ref, np.broadcast_to(bias, (M, N)) if with_bias else None)
 
 
+# ------------------------------------------------------------------ small-M GEMM
+# M <= 16 runs the warp-MMA decode kernel (one pass over the packed weights).
+
+SMALL_M_SHAPES = [
+    (1, 16, 32),          # one block, one partial K chunk
+    (3, 48, 288),         # odd block count (a half-used last box), K = 256 + 32
+    (8, 272, 1088),       # one full token block, 17 blocks, ragged K chunk
+    (9, 528, 4096),       # a second token block holding one token
+    (16, 1024, 768),      # two full token blocks
+    (5, 18960, 64),       # more row blocks than one wave of CTAs takes
+    (2, 32, 16384),       # long K: sums of the x16 form near 2^28
+]
+
+
+@pytest.mark.parametrize("act_bits", [8, 4])
+@pytest.mark.parametrize("M,N,K", SMALL_M_SHAPES)
+def test_small_m_int32_bit_exact(M, N, K, act_bits):
+    Q = 127 if act_bits == 8 else 7
+    qa = inputs.random_codes(M, K, -Q, Q, seed=350 + M)
+    qw = inputs.random_codes(N, K, -7, 7, seed=351 + N)
+    qa[0, :] = Q                                  # extreme sums: +Q against all +7 / all -7
+    qw[0, :] = 7
+    qw[1 % N, :] = -7
+    acc_ref = oracle.gemm_i32(qa, qw)
+    a = to_gpu(qa) if act_bits == 8 else to_gpu(oracle.pack_int4(qa))
+    acc = t4.tint4_debug_int32_gemm(a, act_bits, to_gpu(oracle.pack_int4(qw)))
+    torch.cuda.synchronize()
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+
+
+@pytest.mark.parametrize("act_bits", [8, 4])
+@pytest.mark.parametrize("M,N,K", SMALL_M_SHAPES[1:5])
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_small_m_gemm_bf16(M, N, K, act_bits, with_bias):
+    test_gemm_bf16_epilogue(M, N, K, act_bits, with_bias)
+
+
+@pytest.mark.parametrize("act_bits", [8, 4])
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_decode_w4a8_full_size(M, act_bits):
+    """The decode layer (K = 4096, N = 12288, group 256) through the fused
+    linear, every output against the oracle, and the int32 sums bit-exact."""
+    w = inputs.WORKLOADS["te_decode_w4a8"]
+    N, K, g = w["N"], w["K"], w["group"]
+    x = inputs.activations(M, K, seed=inputs.SEED)
+    W = inputs.weights(N, K, seed=inputs.SEED)
+    wp, sr, qw = oracle.pack_weights(W, g)
+    fn = t4.convrot_w4a8_linear if act_bits == 8 else t4.convrot_w4a4_linear
+    y = fn(bf16_to_gpu(x), to_gpu(wp), to_gpu(sr), g)
+    qa, st, _ = oracle.quantize_act(x, g, act_bits)
+    acc_ref = oracle.gemm_i32(qa, qw)
+    a = to_gpu(qa) if act_bits == 8 else to_gpu(oracle.pack_int4(qa))
+    acc = t4.tint4_debug_int32_gemm(a, act_bits, to_gpu(wp))
+    torch.cuda.synchronize()
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    assert_gemm_output(bf16_from_gpu(y), oracle.epilogue_f64(acc_ref, st, sr, None))
+
+
 # ------------------------------------------------------------------ fused linear
 
 @pytest.mark.parametrize("act_bits", [8, 4])
