@@ -66,12 +66,20 @@ def peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
 
 
-def kernel_source_hash() -> str:
+# the sources each profiled kernel is built from (its own file + the PTX helpers)
+KERNEL_SOURCES = {
+    "w4a8_tmem_gemm_kernel": ("gemm_tmem.cuh", "ptx.cuh"),
+    "rotate_quantize_rows_kernel": ("quantize.cuh", "ptx.cuh"),
+    "w4a16_mma_kernel": ("w4a16.cuh", "ptx.cuh"),
+    "w4a8_small_kernel": ("w4a8_small.cuh", "ptx.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "int4_weight_quantized_block_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -83,7 +91,7 @@ def ncu_traffic(kernel: str, workload: str):
         return None
     d = json.load(open(p))
     e = d.get(kernel, {}).get(workload)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -303,7 +311,7 @@ def run_ours(args, rank, world, dev):
         cpu = cpu_baseline(w, target_s=args.cpu_seconds)
 
     clocks = clk.summary()
-    traffic = ncu_traffic("w4_gemm_kernel", MAIN)
+    traffic = ncu_traffic("w4a8_tmem_gemm_kernel", MAIN)
     line = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -322,7 +330,7 @@ def run_ours(args, rank, world, dev):
                    "M": M, "N": N, "K": K, "group": g, "act_bits": 8,
                    "per_gpu_tokens": M, "parallelism": f"independent batches x{world}",
                    "l2": "flushed (256 MiB write) before every timed step, outside the events"},
-        "roofline": {"bound": "tensor", "kernel": "w4_gemm_kernel (tcgen05 kind::i8)",
+        "roofline": {"bound": "tensor", "kernel": "w4a8_tmem_gemm_kernel (tcgen05 kind::i8)",
                      "achieved": round(gemm_tops, 2), "peak": round(int8_peak, 1),
                      "unit": "TOPS", "frac": round(gemm_tops / int8_peak, 4),
                      "traffic": traffic,
@@ -533,6 +541,17 @@ def run_profile_case(case: str, dev):
                 t4.convrot_quantize_act(x, g, bits, codes, st)
             else:
                 gemm(codes, st, wp, sr, None, y)
+    elif case.startswith("decode_w4a8_M"):
+        M = int(case[len("decode_w4a8_M"):])
+        w = inputs.WORKLOADS["te_decode_w4a8"]
+        N, K, g = w["N"], w["K"], w["group"]
+        _, W_np = inputs.layer_inputs("te_decode_w4a8", M=1)
+        wp, sr = t4.tint4_pack_weights(torch.from_numpy(W_np).to(dev), g)
+        x = bf16_gpu(inputs.activations(M, K, inputs.SEED), dev)
+        codes, st = t4.convrot_quantize_act(x, g, 8)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            t4.w4a8_gemm(codes, st, wp, sr, None, y)
     elif case.startswith("w4a16_M"):
         M = int(case[len("w4a16_M"):])
         w = inputs.WORKLOADS["te_decode_w4a16"]
@@ -557,7 +576,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--profile", default=None,
                     help="run only a few launches of one kernel for ncu: qkv_gemm, "
-                         "qkv_gemm_w4a4, qkv_quantize, w4a16_M<m>")
+                         "qkv_gemm_w4a4, qkv_quantize, w4a16_M<m>, decode_w4a8_M<m>")
     args = ap.parse_args()
     if args.profile:
         dev = torch.device("cuda", 0)
