@@ -92,23 +92,29 @@ __device__ __forceinline__ void fwht_lane8(float (&v)[8], int lane) {
 // to the same integers; otherwise (rare, warp-uniform branch) the codes are
 // recomputed with the IEEE division itself.  Same codes as a division per
 // value, a fraction of the instructions.  scale == 0 gives rs == 0 and codes 0.
+//
+// Rounding without the conversion unit: adding 1.5 * 2^23 to a float of
+// magnitude < 2^22 rounds it to an integer (to nearest, ties to even, as
+// rintf) and leaves that integer in the low bits of the sum, two's
+// complement in the low byte.  m[j] are those sums' bit patterns.
 template <int Q>
-__device__ __forceinline__ void quant8(const float (&v)[8], float scale, float rs, int (&q)[8]) {
-    float k[8];
+__device__ __forceinline__ void quant8(const float (&v)[8], float scale, float rs, uint32_t (&m)[8]) {
+    constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
     bool near = false;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        const float t = v[j] * rs;
-        k[j] = rintf(t);
-        near |= fabsf(fabsf(t - k[j]) - 0.5f) < 3.0517578125e-5f;
+        const float t = fminf(fmaxf(v[j] * rs, static_cast<float>(-Q)), static_cast<float>(Q));
+        const float r = t + kMagic;
+        near |= fabsf(t - (r - kMagic)) > 0.5f - 3.0517578125e-5f;
+        m[j] = __float_as_uint(r);
     }
     if (__any_sync(0xFFFFFFFFu, near) && scale > 0.0f) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) k[j] = rintf(__fdiv_rn(v[j], scale));
+        for (int j = 0; j < 8; ++j) {
+            const float t = fminf(fmaxf(__fdiv_rn(v[j], scale), static_cast<float>(-Q)), static_cast<float>(Q));
+            m[j] = __float_as_uint(t + kMagic);
+        }
     }
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-        q[j] = static_cast<int>(fminf(fmaxf(k[j], static_cast<float>(-Q)), static_cast<float>(Q)));
 }
 
 // Q = 127 (int8 codes) or 7 (int4 codes); PACKED: int4 codes two per byte,
@@ -170,22 +176,21 @@ rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K,
         const int chunk = warp + c * nwarps;
         const int base = chunk * kQuantChunk + lane * 8;
         if (chunk < nchunks) {   // warp-uniform (quant8 votes across the warp)
-            int q[8];
-            quant8<Q>(v[c], scale, rscale, q);
+            uint32_t m[8];
+            quant8<Q>(v[c], scale, rscale, m);
             if (base >= K) continue;
+            // the code of value j is the low byte of m[j] (two's complement)
+            const uint32_t lo = __byte_perm(__byte_perm(m[0], m[1], 0x0040), __byte_perm(m[2], m[3], 0x0040), 0x5410);
+            const uint32_t hi = __byte_perm(__byte_perm(m[4], m[5], 0x0040), __byte_perm(m[6], m[7], 0x0040), 0x5410);
             if (!PACKED) {
-                uint2 out;
-                out.x = (q[0] & 0xFF) | ((q[1] & 0xFF) << 8) | ((q[2] & 0xFF) << 16) |
-                        (static_cast<uint32_t>(q[3] & 0xFF) << 24);
-                out.y = (q[4] & 0xFF) | ((q[5] & 0xFF) << 8) | ((q[6] & 0xFF) << 16) |
-                        (static_cast<uint32_t>(q[7] & 0xFF) << 24);
                 int8_t* dst = static_cast<int8_t*>(codes) + static_cast<size_t>(row) * K + base;
-                *reinterpret_cast<uint2*>(dst) = out;
+                *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
             } else {
-                // low nibble = even index, high nibble = odd index
-                uint32_t out = 0;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) out |= static_cast<uint32_t>(q[j] & 0xF) << (4 * j);
+                // low nibble = even index, high nibble = odd index: gather the
+                // even-index codes and the odd-index codes, then interleave nibbles
+                const uint32_t ev = __byte_perm(lo, hi, 0x6420);   // codes 0, 2, 4, 6
+                const uint32_t od = __byte_perm(lo, hi, 0x7531);   // codes 1, 3, 5, 7
+                const uint32_t out = (ev & 0x0F0F0F0Fu) | ((od & 0x0F0F0F0Fu) << 4);
                 uint8_t* dst =
                     static_cast<uint8_t*>(codes) + static_cast<size_t>(row) * (K / 2) + base / 2;
                 *reinterpret_cast<uint32_t*>(dst) = out;

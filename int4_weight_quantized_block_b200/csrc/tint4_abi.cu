@@ -133,7 +133,9 @@ bool valid_group(int g) { return g == 0 || g == 16 || g == 64 || g == 256; }
 template <typename InT, int G, int Q, bool PACKED>
 void launch_rq_ch(const InT* in, int rows, int K, void* codes, float* scales, cudaStream_t st) {
     const int nchunks = (K + kQuantChunk - 1) / kQuantChunk;
-    if (nchunks <= kQuantMaxWarps) {
+    // two chunks per warp once a row has more than 8: the per-row work (the
+    // absmax reduction, the scale's division) then spreads over more values
+    if (nchunks <= 8) {
         rotate_quantize_rows_kernel<InT, G, Q, PACKED, 1>
             <<<rows, nchunks * 32, 0, st>>>(in, rows, K, codes, scales);
     } else {
