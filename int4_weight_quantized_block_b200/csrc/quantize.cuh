@@ -35,22 +35,40 @@ constexpr int kQuantChunk = 256;       // values per warp chunk (32 lanes x 8)
 constexpr int kQuantMaxChunksPerWarp = 2;
 constexpr int kQuantMaxK = kQuantMaxWarps * kQuantMaxChunksPerWarp * kQuantChunk;  // 16384
 
-__device__ __forceinline__ void load8_as_f32(const __nv_bfloat16* p, float (&v)[8]) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        v[2 * i] = __uint_as_float(w[i] << 16);
-        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-}
+// 8 consecutive inputs as loaded (one 16-byte load of bf16, two of fp32),
+// converted to fp32 only when used: a CTA holds the next row's raw chunks
+// while it works on the current one.
+template <typename InT>
+struct RawChunk;
 
-__device__ __forceinline__ void load8_as_f32(const float* p, float (&v)[8]) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
+template <>
+struct RawChunk<__nv_bfloat16> {
+    uint4 u;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint4*>(p)); }
+    __device__ __forceinline__ void zero() { u = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ void to_f32(float (&v)[8]) const {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+};
+
+template <>
+struct RawChunk<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float* p) {
+        a = __ldg(reinterpret_cast<const float4*>(p));
+        b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    }
+    __device__ __forceinline__ void zero() { a = b = make_float4(0.0f, 0.0f, 0.0f, 0.0f); }
+    __device__ __forceinline__ void to_f32(float (&v)[8]) const {
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+};
 
 // Orthonormal FWHT over blocks of G values spread as 8 per lane.
 template <int G>
@@ -119,81 +137,91 @@ __device__ __forceinline__ void quant8(const float (&v)[8], float scale, float r
 
 // Q = 127 (int8 codes) or 7 (int4 codes); PACKED: int4 codes two per byte,
 // else one code per int8.  CH = chunks per warp held in registers; the CTA
-// has blockDim.x / 32 warps (K <= warps * CH * 256).
+// has blockDim.x / 32 warps (K <= warps * CH * 256).  Persistent: CTA b
+// handles rows b, b + gridDim.x, ..., and the loads of its next row are in
+// flight while it rotates and quantizes the current one.
 template <typename InT, int G, int Q, bool PACKED, int CH>
-__global__ void __launch_bounds__(kQuantMaxWarps * 32)
+__global__ void __launch_bounds__(CH == 1 ? 8 * 32 : kQuantMaxWarps * 32)   // one chunk per warp: K <= 2048
 rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K,
                             void* __restrict__ codes, float* __restrict__ scales) {
-    const int row = blockIdx.x;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int nwarps = blockDim.x >> 5;
-    __shared__ float red[kQuantMaxWarps];
+    __shared__ float red[2][kQuantMaxWarps];   // per-warp maxima, alternate rows
 
     // Under programmatic dependent launch, let the consumer grid start its
     // prologue while this grid runs; it waits for our completion before
     // reading the codes.
     grid_launch_dependents();
 
-    const InT* src = in + static_cast<size_t>(row) * K;
     const int nchunks = (K + kQuantChunk - 1) / kQuantChunk;
-
-    float v[CH][8];
-    float amax = 0.0f;
+    RawChunk<InT> raw[CH];
+    auto fetch = [&](int r) {
 #pragma unroll
-    for (int c = 0; c < CH; ++c) {
-        const int chunk = warp + c * nwarps;
-        const int base = chunk * kQuantChunk + lane * 8;
-        if (chunk < nchunks && base < K) {
-            load8_as_f32(src + base, v[c]);
-        } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) v[c][j] = 0.0f;
+        for (int c = 0; c < CH; ++c) {
+            const int chunk = warp + c * nwarps;
+            const int base = chunk * kQuantChunk + lane * 8;
+            if (r < rows && chunk < nchunks && base < K)
+                raw[c].load(in + static_cast<size_t>(r) * K + base);
+            else
+                raw[c].zero();
         }
-    }
+    };
+    fetch(blockIdx.x);
+
+    int it = 0;
+    for (int row = blockIdx.x; row < rows; row += gridDim.x, ++it) {
+        float v[CH][8];
 #pragma unroll
-    for (int c = 0; c < CH; ++c) {
-        const int chunk = warp + c * nwarps;
-        if (chunk < nchunks) {  // warp-uniform
-            if (G > 0) fwht_lane8<(G > 0 ? G : 16)>(v[c], lane);
+        for (int c = 0; c < CH; ++c) raw[c].to_f32(v[c]);
+        fetch(row + gridDim.x);
+
+        float amax = 0.0f;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[c][j]));
+        for (int c = 0; c < CH; ++c) {
+            const int chunk = warp + c * nwarps;
+            if (chunk < nchunks) {  // warp-uniform
+                if (G > 0) fwht_lane8<(G > 0 ? G : 16)>(v[c], lane);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[c][j]));
+            }
         }
-    }
 #pragma unroll
-    for (int d = 16; d >= 1; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, d));
-    if (lane == 0) red[warp] = amax;
-    __syncthreads();
-    amax = red[0];
-    for (int w = 1; w < nwarps; ++w) amax = fmaxf(amax, red[w]);
+        for (int d = 16; d >= 1; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, d));
+        float* rb = red[it & 1];
+        if (lane == 0) rb[warp] = amax;
+        __syncthreads();
+        amax = rb[0];
+        for (int w = 1; w < nwarps; ++w) amax = fmaxf(amax, rb[w]);
 
-    const float scale = __fdiv_rn(amax, static_cast<float>(Q));
-    const float rscale = scale > 0.0f ? __frcp_rn(scale) : 0.0f;
-    if (threadIdx.x == 0) scales[row] = scale;
+        const float scale = __fdiv_rn(amax, static_cast<float>(Q));
+        const float rscale = scale > 0.0f ? __frcp_rn(scale) : 0.0f;
+        if (threadIdx.x == 0) scales[row] = scale;
 
 #pragma unroll
-    for (int c = 0; c < CH; ++c) {
-        const int chunk = warp + c * nwarps;
-        const int base = chunk * kQuantChunk + lane * 8;
-        if (chunk < nchunks) {   // warp-uniform (quant8 votes across the warp)
-            uint32_t m[8];
-            quant8<Q>(v[c], scale, rscale, m);
-            if (base >= K) continue;
-            // the code of value j is the low byte of m[j] (two's complement)
-            const uint32_t lo = __byte_perm(__byte_perm(m[0], m[1], 0x0040), __byte_perm(m[2], m[3], 0x0040), 0x5410);
-            const uint32_t hi = __byte_perm(__byte_perm(m[4], m[5], 0x0040), __byte_perm(m[6], m[7], 0x0040), 0x5410);
-            if (!PACKED) {
-                int8_t* dst = static_cast<int8_t*>(codes) + static_cast<size_t>(row) * K + base;
-                *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
-            } else {
-                // low nibble = even index, high nibble = odd index: gather the
-                // even-index codes and the odd-index codes, then interleave nibbles
-                const uint32_t ev = __byte_perm(lo, hi, 0x6420);   // codes 0, 2, 4, 6
-                const uint32_t od = __byte_perm(lo, hi, 0x7531);   // codes 1, 3, 5, 7
-                const uint32_t out = (ev & 0x0F0F0F0Fu) | ((od & 0x0F0F0F0Fu) << 4);
-                uint8_t* dst =
-                    static_cast<uint8_t*>(codes) + static_cast<size_t>(row) * (K / 2) + base / 2;
-                *reinterpret_cast<uint32_t*>(dst) = out;
+        for (int c = 0; c < CH; ++c) {
+            const int chunk = warp + c * nwarps;
+            const int base = chunk * kQuantChunk + lane * 8;
+            if (chunk < nchunks) {   // warp-uniform (quant8 votes across the warp)
+                uint32_t m[8];
+                quant8<Q>(v[c], scale, rscale, m);
+                if (base >= K) continue;
+                // the code of value j is the low byte of m[j] (two's complement)
+                const uint32_t lo = __byte_perm(__byte_perm(m[0], m[1], 0x0040), __byte_perm(m[2], m[3], 0x0040), 0x5410);
+                const uint32_t hi = __byte_perm(__byte_perm(m[4], m[5], 0x0040), __byte_perm(m[6], m[7], 0x0040), 0x5410);
+                if (!PACKED) {
+                    int8_t* dst = static_cast<int8_t*>(codes) + static_cast<size_t>(row) * K + base;
+                    *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
+                } else {
+                    // low nibble = even index, high nibble = odd index: gather the
+                    // even-index codes and the odd-index codes, then interleave nibbles
+                    const uint32_t ev = __byte_perm(lo, hi, 0x6420);   // codes 0, 2, 4, 6
+                    const uint32_t od = __byte_perm(lo, hi, 0x7531);   // codes 1, 3, 5, 7
+                    const uint32_t out = (ev & 0x0F0F0F0Fu) | ((od & 0x0F0F0F0Fu) << 4);
+                    uint8_t* dst =
+                        static_cast<uint8_t*>(codes) + static_cast<size_t>(row) * (K / 2) + base / 2;
+                    *reinterpret_cast<uint32_t*>(dst) = out;
+                }
             }
         }
     }

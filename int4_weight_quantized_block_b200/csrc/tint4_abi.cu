@@ -130,18 +130,41 @@ bool valid_group(int g) { return g == 0 || g == 16 || g == 64 || g == 256; }
 
 // Q = 127 or 7; PACKED: int4 codes two per byte, else one code per int8.
 // One CTA per row, one warp per 256-value chunk (two per warp above 32).
+int num_sms(int dev);
+
+// persistent grid: as many CTAs as fit on the GPU at once (per block size,
+// looked up once per device), at most one per row
+template <typename InT, int G, int Q, bool PACKED, int CH>
+void launch_rq_persistent(const InT* in, int rows, int K, void* codes, float* scales, int threads,
+                          cudaStream_t st) {
+    auto kern = rotate_quantize_rows_kernel<InT, G, Q, PACKED, CH>;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static std::atomic<int> per_sm[kMaxDevices][kQuantMaxWarps + 1];
+    const int nw = threads / 32;
+    int occ = per_sm[dev][nw].load(std::memory_order_relaxed);
+    if (occ == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, 0) != cudaSuccess ||
+            occ < 1) {
+            cudaGetLastError();
+            occ = 1;
+        }
+        per_sm[dev][nw].store(occ, std::memory_order_relaxed);
+    }
+    const int grid = std::min(rows, occ * num_sms(dev));
+    kern<<<grid, threads, 0, st>>>(in, rows, K, codes, scales);
+}
+
 template <typename InT, int G, int Q, bool PACKED>
 void launch_rq_ch(const InT* in, int rows, int K, void* codes, float* scales, cudaStream_t st) {
     const int nchunks = (K + kQuantChunk - 1) / kQuantChunk;
     // two chunks per warp once a row has more than 8: the per-row work (the
     // absmax reduction, the scale's division) then spreads over more values
-    if (nchunks <= 8) {
-        rotate_quantize_rows_kernel<InT, G, Q, PACKED, 1>
-            <<<rows, nchunks * 32, 0, st>>>(in, rows, K, codes, scales);
-    } else {
-        rotate_quantize_rows_kernel<InT, G, Q, PACKED, 2>
-            <<<rows, ((nchunks + 1) / 2) * 32, 0, st>>>(in, rows, K, codes, scales);
-    }
+    if (nchunks <= 8)
+        launch_rq_persistent<InT, G, Q, PACKED, 1>(in, rows, K, codes, scales, nchunks * 32, st);
+    else
+        launch_rq_persistent<InT, G, Q, PACKED, 2>(in, rows, K, codes, scales,
+                                                   ((nchunks + 1) / 2) * 32, st);
 }
 
 template <typename InT, int Q, bool PACKED>
