@@ -400,12 +400,19 @@ def bench_rows(args, t4, inputs, dev, flush, pk, int8_peak):
             t4.w4a16_gemv_gemm(x, q, s, z, G, y)
 
         ms = graph_time(call, 64, dev)
+        t4.tint4_set_decode_weight_prefetch(True)
+        ms_pf = graph_time(call, 64, dev)
+        t4.tint4_set_decode_weight_prefetch(False)
         byts = N * K // 2 + N * (K // G) * 3 + M * K * 2 + M * N * 2
         rows[f"te_decode_w4a16_M{M}"] = {
             "kernel": "w4a16_mma_kernel", "M": M, "N": N, "K": K, "group": G,
             "us": round(ms * 1e3, 2), "GBps": round(byts / ms / 1e6, 1),
             "frac_hbm": round(byts / ms / 1e6 / pk["hbm"], 4),
-            "timing": "64 calls in one CUDA graph, 8 weight copies rotated (211 MB > L2)"}
+            "us_chained": round(ms_pf * 1e3, 2), "GBps_chained": round(byts / ms_pf / 1e6, 1),
+            "frac_hbm_chained": round(byts / ms_pf / 1e6 / pk["hbm"], 4),
+            "timing": "64 calls in one CUDA graph, 8 weight copies rotated (211 MB > L2); "
+                      "_chained: with tint4_set_decode_weight_prefetch(1), each call's weights "
+                      "stream while the previous call finishes"}
 
     # W4A8 decode (same shape, ConvRot group 256): the fused linear and the GEMM
     # alone, 8 copies of the packed weights rotated
@@ -432,6 +439,10 @@ def bench_rows(args, t4, inputs, dev, flush, pk, int8_peak):
 
         l_ms = graph_time(lin, 64, dev)
         g_ms = graph_time(gem, 64, dev)
+        t4.tint4_set_decode_weight_prefetch(True)
+        l_ms_pf = graph_time(lin, 64, dev)
+        g_ms_pf = graph_time(gem, 64, dev)
+        t4.tint4_set_decode_weight_prefetch(False)
         wbytes = N * K // 2 + N * 4
         l_bytes = wbytes + M * K * 2 + M * N * 2
         g_bytes = wbytes + M * K + M * 4 + M * N * 2
@@ -441,7 +452,12 @@ def bench_rows(args, t4, inputs, dev, flush, pk, int8_peak):
             "linear_frac_hbm": round(l_bytes / l_ms / 1e6 / pk["hbm"], 4),
             "gemm_us": round(g_ms * 1e3, 2), "gemm_GBps": round(g_bytes / g_ms / 1e6, 1),
             "gemm_frac_hbm": round(g_bytes / g_ms / 1e6 / pk["hbm"], 4),
-            "timing": "64 calls in one CUDA graph, 8 weight copies rotated (201 MB > L2)"}
+            "linear_us_chained": round(l_ms_pf * 1e3, 2),
+            "linear_frac_hbm_chained": round(l_bytes / l_ms_pf / 1e6 / pk["hbm"], 4),
+            "gemm_us_chained": round(g_ms_pf * 1e3, 2),
+            "gemm_frac_hbm_chained": round(g_bytes / g_ms_pf / 1e6 / pk["hbm"], 4),
+            "timing": "64 calls in one CUDA graph, 8 weight copies rotated (201 MB > L2); "
+                      "_chained: with tint4_set_decode_weight_prefetch(1)"}
     return rows
 
 

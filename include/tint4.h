@@ -220,6 +220,22 @@ tint4_status tint4_get_device_error(void* stream);
  * (default 4e9).  Values outside [1e3, 6e10] return TINT4_ERR_INVALID_ARG. */
 tint4_status tint4_set_wait_limit_ns(uint64_t limit_ns);
 
+/*
+ * Decode-chain weight streaming (default off).  The small-M kernels
+ * (w4a16_gemv_gemm; w4a8_gemm, w4a4_gemm and the fused linears at M <= 16)
+ * are launched with programmatic dependent launch, so they may start while
+ * the previous kernel of the stream is still running; they always wait for
+ * it before reading the activations, and, with this switch off, before
+ * reading anything.  With enable = 1 they start streaming their weight
+ * operands (w_q / w_packed, scale, zero, row_scale) at once: in a chain of
+ * layers the next layer's weights then flow from HBM while the current layer
+ * finishes.  Turn it on only when no weight buffer of a call is written by
+ * the kernel launched just before that call on the same stream (weights that
+ * are set up once and then only read meet this).  Process-wide, affects later
+ * launches; enable must be 0 or 1, else TINT4_ERR_INVALID_ARG.
+ */
+tint4_status tint4_set_decode_weight_prefetch(int enable);
+
 #ifdef __cplusplus
 }
 #endif

@@ -31,6 +31,7 @@ __all__ = [
     "tint4_debug_bounded_wait",
     "tint4_get_device_error",
     "tint4_set_wait_limit_ns",
+    "tint4_set_decode_weight_prefetch",
     "tint4_abi_version",
     "QuantizedLinear",
 ]
@@ -231,6 +232,13 @@ def tint4_get_device_error(device=None) -> int:
 
 def tint4_set_wait_limit_ns(limit_ns: int) -> None:
     _native.call("tint4_set_wait_limit_ns", int(limit_ns))
+
+
+def tint4_set_decode_weight_prefetch(enable: bool) -> None:
+    """Let the small-M kernels stream their weights before the previous kernel
+    of the stream has finished (see the header: only when that kernel does not
+    write the weights).  Process-wide; off by default."""
+    _native.call("tint4_set_decode_weight_prefetch", 1 if enable else 0)
 
 
 class QuantizedLinear:

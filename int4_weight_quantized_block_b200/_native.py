@@ -45,6 +45,7 @@ SIGNATURES = {
     "tint4_debug_bounded_wait": (I, [U64, P]),
     "tint4_get_device_error": (I, [P]),
     "tint4_set_wait_limit_ns": (I, [U64]),
+    "tint4_set_decode_weight_prefetch": (I, [ctypes.c_int]),
 }
 
 _lock = threading.Lock()

@@ -28,6 +28,7 @@ constexpr int kGemmBN = 256;
 constexpr int kGemmStages = 3;
 
 std::atomic<uint64_t> g_wait_limit_ns{4000000000ull};
+std::atomic<int> g_decode_prefetch{0};   // tint4_set_decode_weight_prefetch
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -326,13 +327,14 @@ tint4_status launch_gemm_small(const void* a, const uint8_t* w, const float* st,
     cfg.blockDim = dim3(S8Cfg<NB>::THREADS, 1, 1);
     cfg.dynamicSmemBytes = S8Cfg<NB>::SMEM;
     cfg.stream = stream;
+    // always programmatic: the kernel waits for the previous grid before it
+    // reads anything that grid may have written
+    (void)pdl;
     cudaLaunchAttribute attr[1] = {pdl_attr()};
-    if (pdl) {
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-    }
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, tw, static_cast<const uint8_t*>(a), st, sr, bias, out, M,
-                           N, K, 0xF0F0F0F0u,
+                           N, K, 0xF0F0F0F0u, g_decode_prefetch.load(std::memory_order_relaxed),
                            g_wait_limit_ns.load(std::memory_order_relaxed)) != cudaSuccess) {
         cudaGetLastError();
         return TINT4_ERR_CUDA;
@@ -440,6 +442,7 @@ tint4_status launch_w4a16(const __nv_bfloat16* x, const uint8_t* q, const __nv_b
     cfg.numAttrs = 1;
     const W16Consts kc{0x000F000Fu, 0x43004300u};
     if (cudaLaunchKernelEx(&cfg, kern, tw, x, s, z, y, M, N, K, kc,
+                           g_decode_prefetch.load(std::memory_order_relaxed),
                            g_wait_limit_ns.load(std::memory_order_relaxed)) != cudaSuccess) {
         cudaGetLastError();
         return TINT4_ERR_CUDA;
@@ -686,6 +689,12 @@ tint4_status tint4_get_device_error(void* stream) {
 tint4_status tint4_set_wait_limit_ns(uint64_t limit_ns) {
     if (limit_ns < 1000ull || limit_ns > 60000000000ull) return TINT4_ERR_INVALID_ARG;
     g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+    return TINT4_OK;
+}
+
+tint4_status tint4_set_decode_weight_prefetch(int enable) {
+    if (enable != 0 && enable != 1) return TINT4_ERR_INVALID_ARG;
+    g_decode_prefetch.store(enable, std::memory_order_relaxed);
     return TINT4_OK;
 }
 

@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(W16Cfg<NB>::THREADS, 1)
 w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16* __restrict__ x,
                  const __nv_bfloat16* __restrict__ wscale, const uint8_t* __restrict__ wzero,
                  __nv_bfloat16* __restrict__ y, int M, int N, int K, const W16Consts kc,
-                 uint64_t wait_ns) {
+                 int early_weights, uint64_t wait_ns) {
     using C = W16Cfg<NB>;
     constexpr int WARPS = C::WARPS;
     extern __shared__ uint8_t w16_smem_raw[];
@@ -199,9 +199,6 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
         prefetch_tensormap(&tmap_w);
     }
     __syncthreads();
-    // inputs may come from the previous kernel of the stream
-    grid_dependency_wait();
-    grid_launch_dependents();
 
     int issued = 0;
     bool nunits_ok = true;
@@ -214,17 +211,26 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
     };
     // The run's scales and zero points (two contiguous, 16-byte aligned
     // ranges) go out first, as two bulk copies: behind tens of MB of weight
-    // boxes they would hold up every warp's first unit.
-    if (threadIdx.x == 0) {
-        const uint32_t sbytes = nb * 16 * ngroups * 2, zbytes = nb * 16 * ngroups;
-        const size_t base = static_cast<size_t>(b0) * 16 * ngroups;
-        mbar_arrive_expect_tx(sz_full, sbytes + zbytes);
-        bulk_load_1d(sm + ring_bytes + C::kBarBytes, wscale + base, sbytes, sz_full);
-        bulk_load_1d(sm + ring_bytes + C::kBarBytes + ngroups * kW16Rows * 2, wzero + base, zbytes, sz_full);
-    }
-    __syncwarp();
-    if (lane == 0)
-        for (; issued < SLOTS && issued < nunits; ++issued) issue(issued);
+    // boxes they would hold up every warp's first unit.  Then the weight
+    // boxes.  All of it may start before the previous kernel of the stream
+    // has finished only when the caller said the weights are not written by
+    // it (tint4_set_decode_weight_prefetch); x is read after the wait.
+    auto issue_weights = [&]() {
+        if (threadIdx.x == 0) {
+            const uint32_t sbytes = nb * 16 * ngroups * 2, zbytes = nb * 16 * ngroups;
+            const size_t base = static_cast<size_t>(b0) * 16 * ngroups;
+            mbar_arrive_expect_tx(sz_full, sbytes + zbytes);
+            bulk_load_1d(sm + ring_bytes + C::kBarBytes, wscale + base, sbytes, sz_full);
+            bulk_load_1d(sm + ring_bytes + C::kBarBytes + ngroups * kW16Rows * 2, wzero + base, zbytes, sz_full);
+        }
+        __syncwarp();
+        if (lane == 0)
+            for (; issued < SLOTS && issued < nunits; ++issued) issue(issued);
+    };
+    if (early_weights) issue_weights();
+    grid_dependency_wait();
+    grid_launch_dependents();
+    if (!early_weights) issue_weights();
     {
         int ok = 1;
         if (lane == 0) ok = mbar_wait_bounded(sz_full, 0, abort_flag, wait_ns, kDevErrTimeoutConsumer);

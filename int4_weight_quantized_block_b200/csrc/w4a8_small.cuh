@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(S8Cfg<NB>::THREADS, 1)
 w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __restrict__ act,
                   const float* __restrict__ tok_scale, const float* __restrict__ row_scale,
                   const __nv_bfloat16* __restrict__ bias, void* __restrict__ out, int M, int N,
-                  int K, uint32_t hi_mask, uint64_t wait_ns) {
+                  int K, uint32_t hi_mask, int early_weights, uint64_t wait_ns) {
     using C = S8Cfg<NB>;
     constexpr int kS8Warps = C::WARPS, kS8Slots = C::SLOTS, kS8Threads = C::THREADS;
     extern __shared__ uint8_t s8_smem_raw[];
@@ -113,9 +113,6 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
         prefetch_tensormap(&tmap_w);
     }
     __syncthreads();
-    // inputs may come from the previous kernel of the stream
-    grid_dependency_wait();
-    grid_launch_dependents();
 
     int issued = 0;
     auto issue = [&](int i) {
@@ -125,6 +122,13 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
         mbar_arrive_expect_tx(&full[slot], kS8Box);
         tma_load_2d(&tmap_w, &full[slot], ring + slot * kS8Box, P * 128, (b0 + 2 * bp) * 16);
     };
+    // The weights may start streaming before the previous kernel of the
+    // stream has finished only when the caller said they are not written by
+    // it (tint4_set_decode_weight_prefetch); everything else waits for it.
+    if (early_weights && lane == 0)
+        for (; issued < kS8Slots && issued < nunits; ++issued) issue(issued);
+    grid_dependency_wait();
+    grid_launch_dependents();
     if (lane == 0)
         for (; issued < kS8Slots && issued < nunits; ++issued) issue(issued);
 

@@ -126,3 +126,10 @@ def test_debug_entries_rules(lib):
     assert lib.tint4_set_wait_limit_ns(10) == 1
     assert lib.tint4_set_wait_limit_ns(10 ** 11) == 1
     assert lib.tint4_set_wait_limit_ns(4 * 10 ** 9) == 0
+
+
+def test_decode_prefetch_switch_rules(lib):
+    assert lib.tint4_set_decode_weight_prefetch(2) == 1
+    assert lib.tint4_set_decode_weight_prefetch(-1) == 1
+    assert lib.tint4_set_decode_weight_prefetch(1) == 0
+    assert lib.tint4_set_decode_weight_prefetch(0) == 0

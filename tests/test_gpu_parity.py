@@ -173,6 +173,40 @@ def test_decode_w4a8_full_size(M, act_bits):
     assert_gemm_output(bf16_from_gpu(y), oracle.epilogue_f64(acc_ref, st, sr, None))
 
 
+@pytest.mark.parametrize("prefetch", [False, True])
+def test_decode_weight_prefetch_switch(prefetch):
+    """With the decode weight streaming switched on, the small-M kernels give
+    the same bits: the activations (written by the kernel just before, the
+    rotate + quantize of the fused linear) are still read after the wait."""
+    M, N, K, g = 4, 2048, 1024, 256
+    x = inputs.activations(M, K, seed=810)
+    W = inputs.weights(N, K, seed=811)
+    wp, sr, qw = oracle.pack_weights(W, g)
+    op = inputs.w4a16_operands(M, N, K, 128, seed=812)
+    xg, wpg, srg = bf16_to_gpu(x), to_gpu(wp), to_gpu(sr)
+    q16, s16, z16, x16 = to_gpu(op.q), bf16_to_gpu(op.scale), to_gpu(op.zero), bf16_to_gpu(op.x)
+    try:
+        t4.tint4_set_decode_weight_prefetch(prefetch)
+        outs = []
+        for _ in range(3):   # back to back on one stream: each call follows a kernel
+            outs.append((t4.convrot_w4a8_linear(xg, wpg, srg, g),
+                         t4.convrot_w4a4_linear(xg, wpg, srg, g),
+                         t4.w4a16_gemv_gemm(x16, q16, s16, z16, 128)))
+        torch.cuda.synchronize()
+    finally:
+        t4.tint4_set_decode_weight_prefetch(False)
+    y8, y4, y16 = (bf16_from_gpu(o) for o in outs[-1])
+    for o in outs[:-1]:
+        assert np.array_equal(bf16_from_gpu(o[0]), y8)
+        assert np.array_equal(bf16_from_gpu(o[2]), y16)
+    assert_gemm_output(y8, oracle.convrot_linear_f64(x, wp, sr, g, 8))
+    assert_gemm_output(y4, oracle.convrot_linear_f64(x, wp, sr, g, 4))
+    c = check_bf16(y16, oracle.w4a16_f64(op.x, op.q, op.scale, op.zero, 128),
+                   accumulation_error(oracle.w4a16_f64(op.x, op.q, op.scale, op.zero, 128)),
+                   TIE_FRAC_ACCUMULATED)
+    assert c.ok, str(c)
+
+
 # ------------------------------------------------------------------ fused linear
 
 @pytest.mark.parametrize("act_bits", [8, 4])
