@@ -44,6 +44,12 @@
 // A nibble moved into the high half of its byte, low half cleared, is the
 // int8 value 16 * code; the accumulators hold 16 * acc and the epilogue
 // shifts back exactly (|16 acc| < 2^31 for K <= 65536).
+//
+// W4A4 with packed activation codes (A_INT4): the TMA brings the packed
+// activation tile (192 tokens x 64 bytes) into a staging area, and the
+// unpack warps also widen it (x16 again, natural K order) into the swizzled
+// int8 B tile before they signal the stage: the accumulators then hold
+// 256 * acc (|256 acc| < 2^31 for K <= 65536 with codes in [-7, 7]).
 #pragma once
 
 #include "ptx.cuh"
@@ -58,7 +64,9 @@ constexpr int kTmThreads = 576;  // 18 warps
 constexpr int kTmActBytes = kTmBN * kTmBK;            // 24 KB per stage
 constexpr int kTmWBytes = kTmBM * kTmBK / 2;          // 8 KB packed weights per stage
 constexpr int kTmOutBytes = kTmBN * kTmBM * 2;        // 48 KB bf16 staging tile
+constexpr int kTmActPBytes = kTmBN * kTmBK / 2;       // 12 KB packed int4 activation codes per stage
 constexpr int kTmSmemBytes = kTmStages * (kTmActBytes + kTmWBytes) + kTmOutBytes + 256 + 1024;
+constexpr int kTmSmemBytesA4 = kTmSmemBytes + kTmStages * kTmActPBytes;
 constexpr uint32_t kTmColD = 0;                       // accumulator buffer b at b * kTmBN
 constexpr uint32_t kTmColA = 2 * kTmBN;               // A stage s at kTmColA + 32 s
 static_assert(kTmColA + 32 * kTmStages <= 512, "TMEM budget");
@@ -85,7 +93,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     return ok != 0;
 }
 
-template <bool OUT_I32>
+template <bool OUT_I32, bool A_INT4>
 __global__ void __launch_bounds__(kTmThreads, 1)
 w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                       const __grid_constant__ CUtensorMap tmap_w,
@@ -97,7 +105,8 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* sAct = smem;
     uint8_t* sW = smem + kTmStages * kTmActBytes;
-    uint8_t* sOut = sW + kTmStages * kTmWBytes;
+    uint8_t* sActP = sW + kTmStages * kTmWBytes;                       // A_INT4 only
+    uint8_t* sOut = sActP + (A_INT4 ? kTmStages * kTmActPBytes : 0);
     uint64_t* act_full = reinterpret_cast<uint64_t*>(sOut + kTmOutBytes);
     uint64_t* a_full = act_full + kTmStages;       // TMEM A stage written (128 arrivals)
     uint64_t* empty = a_full + kTmStages;          // stage consumed by the MMAs (commit)
@@ -162,8 +171,13 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                     if (!mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, wait_ns,
                                            kDevErrTimeoutProducer))
                         break;
-                    mbar_arrive_expect_tx(&act_full[s], kTmActBytes + kTmWBytes);
-                    tma_load_2d(&tmap_act, &act_full[s], sAct + s * kTmActBytes, kt * kTmBK, m0);
+                    if (A_INT4) {
+                        mbar_arrive_expect_tx(&act_full[s], kTmActPBytes + kTmWBytes);
+                        tma_load_2d(&tmap_act, &act_full[s], sActP + s * kTmActPBytes, kt * (kTmBK / 2), m0);
+                    } else {
+                        mbar_arrive_expect_tx(&act_full[s], kTmActBytes + kTmWBytes);
+                        tma_load_2d(&tmap_act, &act_full[s], sAct + s * kTmActBytes, kt * kTmBK, m0);
+                    }
                     tma_load_2d(&tmap_w, &act_full[s], sW + s * kTmWBytes, kt * (kTmBK / 2), n0);
                     ++issued;
                 }
@@ -245,6 +259,27 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             // the producer refilled this stage (empty[s] -> act_full[s])
             tcgen05_fence_after();
             tmem_st_32x32b_x32(tmem_base + lane_base + kTmColA + 32 * s, a);
+            if (A_INT4) {
+                // widen the packed activation codes of this stage into the
+                // swizzled int8 B tile: 192 rows x 8 chunks of 16 codes, 12
+                // chunks per thread of this K-step parity (the B tile's last
+                // readers, the MMAs of 4 stages ago, completed before the
+                // producer refilled the stage)
+                const uint8_t* ap = sActP + s * kTmActPBytes;
+                uint8_t* ab = sAct + s * kTmActBytes;
+                const int tid = q * 32 + lane;
+#pragma unroll 4
+                for (int i = 0; i < kTmBN * 8 / 128; ++i) {
+                    const int c = tid + 128 * i;
+                    const int rr = c >> 3, k = c & 7;
+                    const uint2 pk = *reinterpret_cast<const uint2*>(ap + rr * 64 + 8 * k);
+                    uint4 o;
+                    unpack8_natural(pk.x, o.x, o.y);
+                    unpack8_natural(pk.y, o.z, o.w);
+                    sts128(ab + rr * 128 + ((k ^ (rr & 7)) << 4), o);
+                }
+                fence_proxy_async_smem();   // generic-proxy writes -> tensor-core reads
+            }
             tmem_st_wait();
             tcgen05_fence_before();
             mbar_arrive(&a_full[s]);
@@ -277,8 +312,10 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             tcgen05_fence_after();
             const bool row_ok = n < N;
             // (16 acc) * s_tok * (s_row / 16) equals acc * s_tok * s_row in fp32:
-            // scaling by a power of two commutes with the rounding
-            const float sr16 = (row_ok && !OUT_I32) ? __ldg(row_scale + n) * 0.0625f : 0.0f;
+            // scaling by a power of two commutes with the rounding (256 for A_INT4)
+            constexpr float kUnscale = A_INT4 ? 1.0f / 256.0f : 0.0625f;
+            constexpr int kShift = A_INT4 ? 8 : 4;
+            const float sr16 = (row_ok && !OUT_I32) ? __ldg(row_scale + n) * kUnscale : 0.0f;
             const float b = (row_ok && !OUT_I32 && bias != nullptr) ? __bfloat162float(bias[n]) : 0.0f;
 #pragma unroll 1
             for (int c0 = half * (kTmBN / 2); c0 < (half + 1) * (kTmBN / 2); c0 += 32) {
@@ -293,7 +330,7 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                     int32_t* o = static_cast<int32_t*>(out) + static_cast<size_t>(mb) * N + n;
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        if (j < mcount) o[static_cast<size_t>(j) * N] = static_cast<int32_t>(acc[j]) >> 4;
+                        if (j < mcount) o[static_cast<size_t>(j) * N] = static_cast<int32_t>(acc[j]) >> kShift;
                 } else {
                     float st[32];
                     if (mcount == 32) {

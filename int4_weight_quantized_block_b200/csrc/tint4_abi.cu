@@ -1,6 +1,7 @@
 // tint4_abi.cu -- the C ABI of include/tint4.h: argument checks, tensor maps,
 // launch configuration.  Every operation runs in the kernels of quantize.cuh,
-// gemm.cuh and w4a16.cuh; nothing here touches tensor data.
+// gemm_tmem.cuh, w4a8_small.cuh and w4a16.cuh; nothing here touches tensor
+// data.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -11,7 +12,6 @@
 #include <mutex>
 
 #include "../../include/tint4.h"
-#include "gemm.cuh"
 #include "gemm_tmem.cuh"
 #include "ptx.cuh"
 #include "quantize.cuh"
@@ -24,8 +24,7 @@ using namespace tint4;
 
 constexpr int kAbiVersion = 1;
 constexpr int kMaxDevices = 64;
-constexpr int kGemmBN = 256;
-constexpr int kGemmStages = 3;
+constexpr int kMaxTokens = 65535 * 128;   // M limit of the GEMM entry points
 
 std::atomic<uint64_t> g_wait_limit_ns{4000000000ull};
 std::atomic<int> g_decode_prefetch{0};   // tint4_set_decode_weight_prefetch
@@ -121,7 +120,7 @@ tint4_status check_mnk(int M, int N, int K) {
     if (M < 0 || N < 0 || K < 0) return TINT4_ERR_INVALID_ARG;
     if (N < 16 || N % 16 != 0) return TINT4_ERR_UNSUPPORTED_SHAPE;
     if (K < 32 || K % 32 != 0 || K > 65536) return TINT4_ERR_UNSUPPORTED_SHAPE;
-    if (M > 65535 * kGemmBM) return TINT4_ERR_UNSUPPORTED_SHAPE;
+    if (M > kMaxTokens) return TINT4_ERR_UNSUPPORTED_SHAPE;
     return TINT4_OK;
 }
 
@@ -209,15 +208,18 @@ cudaLaunchAttribute pdl_attr() {
     return a;
 }
 
-// W4A8: int8 activation codes, weights widened into TMEM (gemm_tmem.cuh).
-template <bool OUT_I32>
+// Weights widened into TMEM (gemm_tmem.cuh); activation codes int8, or
+// packed int4 widened in shared memory (A_INT4).
+template <bool OUT_I32, bool A_INT4>
 tint4_status launch_gemm_tmem(const void* a, const uint8_t* w, const float* st, const float* sr,
                               const __nv_bfloat16* bias, void* out, int M, int N, int K,
                               cudaStream_t stream, bool pdl) {
-    auto kern = w4a8_tmem_gemm_kernel<OUT_I32>;
+    auto kern = w4a8_tmem_gemm_kernel<OUT_I32, A_INT4>;
+    constexpr int smem_bytes = A_INT4 ? kTmSmemBytesA4 : kTmSmemBytes;
     CUtensorMap ta, tw, ty;
     std::memset(&ty, 0, sizeof(ty));
-    bool ok = make_map_u8(&ta, a, K, M, K, kTmBK, kTmBN, CU_TENSOR_MAP_SWIZZLE_128B);
+    bool ok = A_INT4 ? make_map_u8(&ta, a, K / 2, M, K / 2, kTmBK / 2, kTmBN, CU_TENSOR_MAP_SWIZZLE_NONE)
+                     : make_map_u8(&ta, a, K, M, K, kTmBK, kTmBN, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && make_map_u8(&tw, w, K / 2, N, K / 2, kTmBK / 2, kTmBM, CU_TENSOR_MAP_SWIZZLE_64B);
     if (!OUT_I32)   // y bf16 [M, N]: the epilogue's staging tile goes out as one box
         ok = ok && make_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, N, M,
@@ -229,7 +231,7 @@ tint4_status launch_gemm_tmem(const void* a, const uint8_t* w, const float* st, 
     static std::atomic<bool> attr_done[kMaxDevices];
     if (!attr_done[dev].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kTmSmemBytes) != cudaSuccess) {
+                                 smem_bytes) != cudaSuccess) {
             cudaGetLastError();
             return TINT4_ERR_CUDA;
         }
@@ -239,7 +241,7 @@ tint4_status launch_gemm_tmem(const void* a, const uint8_t* w, const float* st, 
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(std::min(tiles, num_sms(dev)), 1, 1);
     cfg.blockDim = dim3(kTmThreads, 1, 1);
-    cfg.dynamicSmemBytes = kTmSmemBytes;
+    cfg.dynamicSmemBytes = smem_bytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1] = {pdl_attr()};
     if (pdl) {
@@ -255,47 +257,6 @@ tint4_status launch_gemm_tmem(const void* a, const uint8_t* w, const float* st, 
     return TINT4_OK;
 }
 
-// W4A4 with packed int4 activation codes: both operands unpacked in shared
-// memory (gemm.cuh).
-template <bool OUT_I32>
-tint4_status launch_gemm_smem_w4a4(const void* a, const uint8_t* w, const float* st,
-                                   const float* sr, const __nv_bfloat16* bias, void* out, int M,
-                                   int N, int K, cudaStream_t stream, bool pdl) {
-    using L = GemmLayout<true, kGemmBN, kGemmStages>;
-    auto kern = w4_gemm_kernel<true, kGemmBN, kGemmStages, OUT_I32>;
-    CUtensorMap ta, tw;
-    bool ok = make_map_u8(&ta, a, K / 2, M, K / 2, 64, kGemmBM, CU_TENSOR_MAP_SWIZZLE_NONE);
-    ok = ok && make_map_u8(&tw, w, K / 2, N, K / 2, 64, kGemmBN, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (!ok) return TINT4_ERR_CUDA;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    static std::atomic<bool> attr_done[kMaxDevices];
-    if (!attr_done[dev].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 L::kSmemBytes) != cudaSuccess) {
-            cudaGetLastError();
-            return TINT4_ERR_CUDA;
-        }
-        attr_done[dev].store(true, std::memory_order_release);
-    }
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((N + kGemmBN - 1) / kGemmBN, (M + kGemmBM - 1) / kGemmBM, 1);
-    cfg.blockDim = dim3(kGemmThreads, 1, 1);
-    cfg.dynamicSmemBytes = L::kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1] = {pdl_attr()};
-    if (pdl) {
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-    }
-    const uint64_t wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
-    if (cudaLaunchKernelEx(&cfg, kern, ta, tw, st, sr, bias, out, M, N, K, wait_ns) !=
-        cudaSuccess) {
-        cudaGetLastError();
-        return TINT4_ERR_CUDA;
-    }
-    return TINT4_OK;
-}
 
 // Small M (<= kS8MaxM tokens): the warp-MMA kernel that streams the packed
 // weights once (w4a8_small.cuh).
@@ -351,9 +312,7 @@ tint4_status launch_gemm(const void* a, const uint8_t* w, const float* st, const
         return launch_gemm_small<1, A_INT4, OUT_I32>(a, w, st, sr, bias, out, M, N, K, stream, pdl);
     if (M <= kS8MaxM)
         return launch_gemm_small<2, A_INT4, OUT_I32>(a, w, st, sr, bias, out, M, N, K, stream, pdl);
-    if (A_INT4)
-        return launch_gemm_smem_w4a4<OUT_I32>(a, w, st, sr, bias, out, M, N, K, stream, pdl);
-    return launch_gemm_tmem<OUT_I32>(a, w, st, sr, bias, out, M, N, K, stream, pdl);
+    return launch_gemm_tmem<OUT_I32, A_INT4>(a, w, st, sr, bias, out, M, N, K, stream, pdl);
 }
 
 tint4_status gemm_entry(bool a_int4, const void* a, const float* tok_scale, const uint8_t* w,
