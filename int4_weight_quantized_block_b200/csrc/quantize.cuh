@@ -115,13 +115,19 @@ __device__ __forceinline__ void fwht_lane8(float (&v)[8], int lane) {
 // magnitude < 2^22 rounds it to an integer (to nearest, ties to even, as
 // rintf) and leaves that integer in the low bits of the sum, two's
 // complement in the low byte.  m[j] are those sums' bit patterns.
-template <int Q>
+//
+// CLAMP = false is for scales >= 1e-30 (fl(1/s) finite): then |t| <= Q (1 +
+// 3 * 2^-24) < Q + 1/2 for every |v| <= absmax, so the codes are within
+// [-Q, Q] without a clamp; __fmul_rn keeps the product from fusing with the
+// rounding addition.
+template <int Q, bool CLAMP>
 __device__ __forceinline__ void quant8(const float (&v)[8], float scale, float rs, uint32_t (&m)[8]) {
     constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
     bool near = false;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        const float t = fminf(fmaxf(v[j] * rs, static_cast<float>(-Q)), static_cast<float>(Q));
+        const float t = CLAMP ? fminf(fmaxf(v[j] * rs, static_cast<float>(-Q)), static_cast<float>(Q))
+                              : __fmul_rn(v[j], rs);
         const float r = t + kMagic;
         near |= fabsf(t - (r - kMagic)) > 0.5f - 3.0517578125e-5f;
         m[j] = __float_as_uint(r);
@@ -140,28 +146,26 @@ __device__ __forceinline__ void quant8(const float (&v)[8], float scale, float r
 // has blockDim.x / 32 warps (K <= warps * CH * 256).  Persistent: CTA b
 // handles rows b, b + gridDim.x, ..., and the loads of its next row are in
 // flight while it rotates and quantizes the current one.
-template <typename InT, int G, int Q, bool PACKED, int CH>
-__global__ void __launch_bounds__(CH == 1 ? 8 * 32 : kQuantMaxWarps * 32)   // one chunk per warp: K <= 2048
-rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K,
-                            void* __restrict__ codes, float* __restrict__ scales) {
+// The rows of one CTA.  FULL: the CTA's warps hold exactly K values (every
+// chunk present and complete), so no per-chunk guard is needed.
+template <typename InT, int G, int Q, bool PACKED, int CH, bool FULL>
+__device__ __forceinline__ void rotate_quantize_rows(const InT* __restrict__ in, int rows, int K,
+                                                     void* __restrict__ codes,
+                                                     float* __restrict__ scales,
+                                                     float (&red)[2][kQuantMaxWarps]) {
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int nwarps = blockDim.x >> 5;
-    __shared__ float red[2][kQuantMaxWarps];   // per-warp maxima, alternate rows
-
-    // Under programmatic dependent launch, let the consumer grid start its
-    // prologue while this grid runs; it waits for our completion before
-    // reading the codes.
-    grid_launch_dependents();
-
     const int nchunks = (K + kQuantChunk - 1) / kQuantChunk;
+    auto present = [&](int c) { return FULL || warp + c * nwarps < nchunks; };   // warp-uniform
+    auto base_of = [&](int c) { return (warp + c * nwarps) * kQuantChunk + lane * 8; };
+
     RawChunk<InT> raw[CH];
     auto fetch = [&](int r) {
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
-            const int chunk = warp + c * nwarps;
-            const int base = chunk * kQuantChunk + lane * 8;
-            if (r < rows && chunk < nchunks && base < K)
+            const int base = base_of(c);
+            if (r < rows && present(c) && (FULL || base < K))
                 raw[c].load(in + static_cast<size_t>(r) * K + base);
             else
                 raw[c].zero();
@@ -179,8 +183,7 @@ rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K,
         float amax = 0.0f;
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
-            const int chunk = warp + c * nwarps;
-            if (chunk < nchunks) {  // warp-uniform
+            if (present(c)) {
                 if (G > 0) fwht_lane8<(G > 0 ? G : 16)>(v[c], lane);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[c][j]));
@@ -196,35 +199,54 @@ rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K,
 
         const float scale = __fdiv_rn(amax, static_cast<float>(Q));
         const float rscale = scale > 0.0f ? __frcp_rn(scale) : 0.0f;
+        const bool tiny = scale < 1e-30f;   // row-uniform: take the clamped path
         if (threadIdx.x == 0) scales[row] = scale;
 
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
-            const int chunk = warp + c * nwarps;
-            const int base = chunk * kQuantChunk + lane * 8;
-            if (chunk < nchunks) {   // warp-uniform (quant8 votes across the warp)
-                uint32_t m[8];
-                quant8<Q>(v[c], scale, rscale, m);
-                if (base >= K) continue;
-                // the code of value j is the low byte of m[j] (two's complement)
-                const uint32_t lo = __byte_perm(__byte_perm(m[0], m[1], 0x0040), __byte_perm(m[2], m[3], 0x0040), 0x5410);
-                const uint32_t hi = __byte_perm(__byte_perm(m[4], m[5], 0x0040), __byte_perm(m[6], m[7], 0x0040), 0x5410);
-                if (!PACKED) {
-                    int8_t* dst = static_cast<int8_t*>(codes) + static_cast<size_t>(row) * K + base;
-                    *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
-                } else {
-                    // low nibble = even index, high nibble = odd index: gather the
-                    // even-index codes and the odd-index codes, then interleave nibbles
-                    const uint32_t ev = __byte_perm(lo, hi, 0x6420);   // codes 0, 2, 4, 6
-                    const uint32_t od = __byte_perm(lo, hi, 0x7531);   // codes 1, 3, 5, 7
-                    const uint32_t out = (ev & 0x0F0F0F0Fu) | ((od & 0x0F0F0F0Fu) << 4);
-                    uint8_t* dst =
-                        static_cast<uint8_t*>(codes) + static_cast<size_t>(row) * (K / 2) + base / 2;
-                    *reinterpret_cast<uint32_t*>(dst) = out;
-                }
+            if (!present(c)) continue;   // warp-uniform (quant8 votes across the warp)
+            const int base = base_of(c);
+            uint32_t m[8];
+            if (tiny) quant8<Q, true>(v[c], scale, rscale, m);
+            else quant8<Q, false>(v[c], scale, rscale, m);
+            if (!FULL && base >= K) continue;
+            // the code of value j is the low byte of m[j] (two's complement)
+            const uint32_t lo = __byte_perm(__byte_perm(m[0], m[1], 0x0040), __byte_perm(m[2], m[3], 0x0040), 0x5410);
+            const uint32_t hi = __byte_perm(__byte_perm(m[4], m[5], 0x0040), __byte_perm(m[6], m[7], 0x0040), 0x5410);
+            if (!PACKED) {
+                int8_t* dst = static_cast<int8_t*>(codes) + static_cast<size_t>(row) * K + base;
+                *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
+            } else {
+                // low nibble = even index, high nibble = odd index: gather the
+                // even-index codes and the odd-index codes, then interleave nibbles
+                const uint32_t ev = __byte_perm(lo, hi, 0x6420);   // codes 0, 2, 4, 6
+                const uint32_t od = __byte_perm(lo, hi, 0x7531);   // codes 1, 3, 5, 7
+                const uint32_t out = (ev & 0x0F0F0F0Fu) | ((od & 0x0F0F0F0Fu) << 4);
+                uint8_t* dst = static_cast<uint8_t*>(codes) + static_cast<size_t>(row) * (K / 2) + base / 2;
+                *reinterpret_cast<uint32_t*>(dst) = out;
             }
         }
     }
+}
+
+// Q = 127 (int8 codes) or 7 (int4 codes); PACKED: int4 codes two per byte,
+// else one code per int8.  CH = chunks per warp held in registers; the CTA
+// has blockDim.x / 32 warps (K <= warps * CH * 256).  Persistent: CTA b
+// handles rows b, b + gridDim.x, ..., and the loads of its next row are in
+// flight while it rotates and quantizes the current one.
+template <typename InT, int G, int Q, bool PACKED, int CH>
+__global__ void __launch_bounds__(CH == 1 ? 8 * 32 : kQuantMaxWarps * 32)   // one chunk per warp: K <= 2048
+rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K,
+                            void* __restrict__ codes, float* __restrict__ scales) {
+    __shared__ float red[2][kQuantMaxWarps];   // per-warp maxima, alternate rows
+    // Under programmatic dependent launch, let the consumer grid start its
+    // prologue while this grid runs; it waits for our completion before
+    // reading the codes.
+    grid_launch_dependents();
+    if (K == static_cast<int>(blockDim.x / 32) * CH * kQuantChunk)
+        rotate_quantize_rows<InT, G, Q, PACKED, CH, true>(in, rows, K, codes, scales, red);
+    else
+        rotate_quantize_rows<InT, G, Q, PACKED, CH, false>(in, rows, K, codes, scales, red);
 }
 
 }  // namespace tint4
