@@ -140,31 +140,6 @@ __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_
         : "memory");
 }
 
-// 2-D tiled bulk tensor store shared -> global (bulk-group completion); the
-// parts of the box outside the tensor are not written.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t x,
-                                             int32_t y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-            reinterpret_cast<uint64_t>(map)),
-        "r"(smem_u32(src)), "r"(x), "r"(y)
-        : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit_group() {
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// wait until the shared-memory sources of all committed bulk stores were read
-__device__ __forceinline__ void bulk_wait_group_read0() {
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
-// wait until all committed bulk stores have completed
-__device__ __forceinline__ void bulk_wait_group0() {
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
 // named barrier among `nthreads` threads (a multiple of 32)
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

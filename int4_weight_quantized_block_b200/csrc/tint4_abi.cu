@@ -216,15 +216,10 @@ tint4_status launch_gemm_tmem(const void* a, const uint8_t* w, const float* st, 
                               cudaStream_t stream, bool pdl) {
     auto kern = w4a8_tmem_gemm_kernel<OUT_I32, A_INT4>;
     constexpr int smem_bytes = A_INT4 ? kTmSmemBytesA4 : kTmSmemBytes;
-    CUtensorMap ta, tw, ty;
-    std::memset(&ty, 0, sizeof(ty));
+    CUtensorMap ta, tw;
     bool ok = A_INT4 ? make_map_u8(&ta, a, K / 2, M, K / 2, kTmBK / 2, kTmBN, CU_TENSOR_MAP_SWIZZLE_NONE)
                      : make_map_u8(&ta, a, K, M, K, kTmBK, kTmBN, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && make_map_u8(&tw, w, K / 2, N, K / 2, kTmBK / 2, kTmBM, CU_TENSOR_MAP_SWIZZLE_64B);
-    if (!OUT_I32)   // y bf16 [M, N]: the epilogue's staging tile goes out as one box
-        ok = ok && make_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, N, M,
-                               static_cast<uint64_t>(N) * 2, kTmBM, kTmBN,
-                               CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return TINT4_ERR_CUDA;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -249,7 +244,7 @@ tint4_status launch_gemm_tmem(const void* a, const uint8_t* w, const float* st, 
         cfg.numAttrs = 1;
     }
     const uint64_t wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
-    if (cudaLaunchKernelEx(&cfg, kern, ta, tw, ty, st, sr, bias, out, M, N, K, wait_ns) !=
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tw, st, sr, bias, out, M, N, K, wait_ns) !=
         cudaSuccess) {
         cudaGetLastError();
         return TINT4_ERR_CUDA;
