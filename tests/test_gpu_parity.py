@@ -294,6 +294,29 @@ def test_w4a16(M, N, K):
     assert c.ok, str(c)
 
 
+@pytest.mark.parametrize("M", [1, 9])
+def test_w4a16_extreme_token_values(M):
+    """Token values far from the rest (tiny, and beyond the fp16 range) in a
+    few groups, against the oracle."""
+    N, K = 256, 2048
+    op = inputs.w4a16_operands(M, N, K, 128, seed=820 + M)
+    x = oracle.bf16_bits_to_f32(op.x).reshape(M, K).astype(np.float64)
+    x[0, 300] = 3.0e-7          # pair 1: below fp16's exact range
+    x[0, 1700] = 1.0e-30        # pair 6
+    if M > 1:
+        # pair 4: above fp16's largest finite value, in the last token only
+        # (its outputs are then one dominant product each, often an exact
+        # bf16 rounding midpoint: a tie the other token rows dilute)
+        x[M - 1, 1100] = 7.0e4
+    xb = inputs.f32_to_bf16_bits(x)
+    y_ref = oracle.w4a16_f64(xb, op.q, op.scale, op.zero, 128)
+    y = t4.w4a16_gemv_gemm(bf16_to_gpu(xb), to_gpu(op.q), bf16_to_gpu(op.scale),
+                           to_gpu(op.zero), 128)
+    torch.cuda.synchronize()
+    c = check_bf16(bf16_from_gpu(y), y_ref, accumulation_error(y_ref), TIE_FRAC_ACCUMULATED)
+    assert c.ok, str(c)
+
+
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_w4a16_full_size(M):
     w = inputs.WORKLOADS["te_decode_w4a16"]
