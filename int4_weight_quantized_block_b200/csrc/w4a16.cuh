@@ -224,8 +224,9 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
             bulk_load_1d(sm + ring_bytes + C::kBarBytes + ngroups * kW16Rows * 2, wzero + base, zbytes, sz_full);
         }
         __syncwarp();
-        if (lane == 0)
-            for (; issued < SLOTS && issued < nunits; ++issued) issue(issued);
+        // one box per warp now, the rest once the scales have landed: every
+        // warp's first box then reaches the front of the memory queues
+        if (lane == 0 && issued < nunits) issue(issued++);
     };
     if (early_weights) issue_weights();
     grid_dependency_wait();
@@ -235,6 +236,8 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
         int ok = 1;
         if (lane == 0) ok = mbar_wait_bounded(sz_full, 0, abort_flag, wait_ns, kDevErrTimeoutConsumer);
         if (__shfl_sync(0xFFFFFFFFu, ok, 0) == 0) nunits_ok = false;
+        if (lane == 0)
+            for (; issued < SLOTS && issued < nunits; ++issued) issue(issued);
     }
 
     float total[kW16MB][NB][4];
