@@ -125,12 +125,13 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
     // The weights may start streaming before the previous kernel of the
     // stream has finished only when the caller said they are not written by
     // it (tint4_set_decode_weight_prefetch); everything else waits for it.
-    if (early_weights && lane == 0)
-        for (; issued < kS8Slots && issued < nunits; ++issued) issue(issued);
+    // One box per warp first, the rest once the first activation fragments
+    // are in: every warp's first box then reaches the front of the memory
+    // queues.
+    if (early_weights && lane == 0 && issued < nunits) issue(issued++);
     grid_dependency_wait();
     grid_launch_dependents();
-    if (lane == 0)
-        for (; issued < kS8Slots && issued < nunits; ++issued) issue(issued);
+    if (lane == 0 && issued == 0 && nunits > 0) issue(issued++);
 
     int32_t total[kS8MB][NB][4];
 #pragma unroll
@@ -182,6 +183,8 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
                     for (int i = 0; i < 4; ++i) bfr[h][b][i][0] = bfr[h][b][i][1] = 0u;
                 }
             }
+        if (lane == 0)
+            for (; issued < kS8Slots && issued < nunits; ++issued) issue(issued);
 #pragma unroll
         for (int bp = 0; bp < kS8MB / 2; ++bp) {
             if (bp >= bp_hi) break;   // warp-uniform
