@@ -54,7 +54,7 @@ namespace tint4 {
 constexpr int kW16Group = 128;      // K values per quantization group
 constexpr int kW16Box = 32 * 128;   // one unit: 2 row blocks x 2 groups of packed bytes
 constexpr int kW16Ring = 128 * 1024;  // all warps' rings
-constexpr int kW16MB = 8;           // 16-row blocks per CTA at most
+constexpr int kW16MB = 6;           // 16-row blocks per CTA at most
 constexpr int kW16Rows = kW16MB * 16;
 constexpr int kW16MaxK = 16384;
 constexpr int kW16MaxM = 16;        // tokens per launch (the host splits larger batches)
@@ -118,7 +118,7 @@ __host__ __device__ constexpr int w16_perm(int m) {
 // warp's units are in flight at once for the decode shapes.
 template <int NB>
 struct W16Cfg {
-    static constexpr int WARPS = NB == 1 ? 12 : 8;
+    static constexpr int WARPS = NB == 1 ? 16 : 8;
     static constexpr int THREADS = WARPS * 32;
     static constexpr int kMaxSlots = 2;
     static constexpr int kBarBytes = WARPS * kMaxSlots * 8 + 16;   // + scale/zero barrier, abort flag
