@@ -119,6 +119,10 @@ class ClockSampler:
         self._nvml = None
 
     def __enter__(self):
+        # the timing loop holds the interpreter lock between launches: let the
+        # sampler thread in often enough to see the timed region
+        self._old_switch = sys.getswitchinterval()
+        sys.setswitchinterval(0.0002)
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -149,6 +153,7 @@ class ClockSampler:
         self._stop.set()
         if self._nvml is not None:
             self._t.join(timeout=2)
+        sys.setswitchinterval(self._old_switch)
 
     def summary(self):
         if not self.samples:
@@ -584,7 +589,7 @@ def run_profile_case(case: str, dev):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-rows", action="store_true", help="skip the per-workload rows")
