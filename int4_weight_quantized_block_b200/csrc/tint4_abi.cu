@@ -298,6 +298,62 @@ tint4_status launch_gemm_small(const void* a, const uint8_t* w, const float* st,
     return last_launch_status();
 }
 
+// The fused linear at M <= kFuseMaxRows, K <= kS8FuseMaxK: one launch of the
+// small-M kernel that rotates and quantizes x itself (group G, codes in
+// [-Q, Q]) while its first weight boxes are in flight.
+template <int G, int Q>
+tint4_status launch_linear_small_fused(const __nv_bfloat16* x, const uint8_t* w, const float* sr,
+                                       const __nv_bfloat16* bias, __nv_bfloat16* y, int M, int N,
+                                       int K, cudaStream_t stream) {
+    auto kern = w4a8_small_kernel<1, false, false, G, Q>;
+    constexpr int smem = S8Cfg<1>::SMEM + kS8FuseBytes;
+    CUtensorMap tw;
+    if (!make_map_u8(&tw, w, K / 2, N, K / 2, 128, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+        return TINT4_ERR_CUDA;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static std::atomic<bool> attr_done[kMaxDevices];
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return TINT4_ERR_CUDA;
+        }
+        attr_done[dev].store(true, std::memory_order_release);
+    }
+    const int nblk = N / 16;
+    const int sms = num_sms(dev);
+    const int grid = nblk <= kS8MB * sms ? std::min(sms, nblk) : (nblk + kS8MB - 1) / kS8MB;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(S8Cfg<1>::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tw, reinterpret_cast<const uint8_t*>(x),
+                           static_cast<const float*>(nullptr), sr, bias, static_cast<void*>(y), M,
+                           N, K, 0xF0F0F0F0u, g_decode_prefetch.load(std::memory_order_relaxed),
+                           g_wait_limit_ns.load(std::memory_order_relaxed)) != cudaSuccess) {
+        cudaGetLastError();
+        return TINT4_ERR_CUDA;
+    }
+    return last_launch_status();
+}
+
+template <int Q>
+tint4_status launch_linear_small_fused_g(const __nv_bfloat16* x, const uint8_t* w, const float* sr,
+                                         const __nv_bfloat16* bias, __nv_bfloat16* y, int M, int N,
+                                         int K, int g, cudaStream_t stream) {
+    switch (g) {
+        case 0: return launch_linear_small_fused<0, Q>(x, w, sr, bias, y, M, N, K, stream);
+        case 16: return launch_linear_small_fused<16, Q>(x, w, sr, bias, y, M, N, K, stream);
+        case 64: return launch_linear_small_fused<64, Q>(x, w, sr, bias, y, M, N, K, stream);
+        default: return launch_linear_small_fused<256, Q>(x, w, sr, bias, y, M, N, K, stream);
+    }
+}
+
 // A_INT4: activation codes packed two per byte (else int8, one per byte).
 template <bool A_INT4, bool OUT_I32>
 tint4_status launch_gemm(const void* a, const uint8_t* w, const float* st, const float* sr,
@@ -344,6 +400,16 @@ tint4_status linear_entry(int bits, const tint4_bf16* x, const uint8_t* w_packed
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TINT4_ERR_MISALIGNED;
     if ((s = check_device()) != TINT4_OK) return s;
     if (M == 0) return TINT4_OK;
+    if (M <= kFuseMaxRows && K <= kS8FuseMaxK) {
+        // decode: one launch, the codes never leave the CTA
+        const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+        const auto* b = reinterpret_cast<const __nv_bfloat16*>(bias);
+        auto* yb = reinterpret_cast<__nv_bfloat16*>(y);
+        return bits == 8 ? launch_linear_small_fused_g<127>(xb, w_packed, row_scale, b, yb, M, N, K,
+                                                            group, as_stream(stream))
+                         : launch_linear_small_fused_g<7>(xb, w_packed, row_scale, b, yb, M, N, K,
+                                                          group, as_stream(stream));
+    }
     // one int8 per code for both widths: the W4A4 codes (in [-7, 7]) are kept
     // one per byte in the workspace and run through the W4A8 kernel, whose
     // int32 sums are the same numbers

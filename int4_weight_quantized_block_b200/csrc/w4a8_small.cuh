@@ -34,6 +34,7 @@
 #pragma once
 
 #include "ptx.cuh"
+#include "quantize.cuh"
 
 namespace tint4 {
 
@@ -67,14 +68,25 @@ __device__ __forceinline__ void mma_s8_16832(int32_t (&d)[4], const uint32_t (&a
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Shared memory of the fused linear: the codes of up to kFuseMaxRows tokens
+// (one per byte) and their scales, behind the ring and barriers.
+constexpr int kS8FuseMaxK = 16 * kQuantChunk;   // one chunk per warp of the 16-warp CTA
+constexpr int kS8FuseBytes = kFuseMaxRows * kS8FuseMaxK + 64 + kFuseMaxRows * kQuantMaxWarps * 4;
+
 // NB 8-token blocks (M <= 8 NB <= 16); A_INT4: activation codes packed two
 // per byte; OUT_I32: write the exact int32 sums instead of bf16 (test entry).
-template <int NB, bool A_INT4, bool OUT_I32>
+// FG, FQ (fused linear, NB = 1, M <= kFuseMaxRows, K <= kS8FuseMaxK): `act`
+// is x (bf16) and the CTA rotates (group FG, 0 = none) and quantizes it (to
+// [-FQ, FQ], one code per byte) into shared memory itself, while its first
+// weight boxes are in flight; tok_scale is then unused.  FQ = 0: not fused.
+template <int NB, bool A_INT4, bool OUT_I32, int FG = 0, int FQ = 0>
 __global__ void __launch_bounds__(S8Cfg<NB>::THREADS, 1)
 w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __restrict__ act,
                   const float* __restrict__ tok_scale, const float* __restrict__ row_scale,
                   const __nv_bfloat16* __restrict__ bias, void* __restrict__ out, int M, int N,
                   int K, uint32_t hi_mask, int early_weights, uint64_t wait_ns) {
+    constexpr bool FUSED = FQ != 0;
+    static_assert(!FUSED || (NB == 1 && !A_INT4 && !OUT_I32), "fused: int8 codes, bf16 out, <= 8 tokens");
     using C = S8Cfg<NB>;
     constexpr int kS8Warps = C::WARPS, kS8Slots = C::SLOTS, kS8Threads = C::THREADS;
     extern __shared__ uint8_t s8_smem_raw[];
@@ -133,6 +145,17 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
     grid_launch_dependents();
     if (lane == 0 && issued == 0 && nunits > 0) issue(issued++);
 
+    // fused linear: x -> codes and scales in shared memory, under the first boxes
+    uint8_t* sfuse = sm + kS8Ring + kS8Warps * kS8Slots * 8 + 16;
+    const int8_t* sCodes = reinterpret_cast<const int8_t*>(sfuse);
+    const float* sTokScale = reinterpret_cast<const float*>(sfuse + kFuseMaxRows * kS8FuseMaxK);
+    if constexpr (FUSED) {
+        rotate_quantize_rows_to_smem<FG, FQ>(
+            reinterpret_cast<const __nv_bfloat16*>(act), M, K, reinterpret_cast<int8_t*>(sfuse),
+            reinterpret_cast<float*>(sfuse + kFuseMaxRows * kS8FuseMaxK),
+            *reinterpret_cast<float(*)[kFuseMaxRows][kQuantMaxWarps]>(sfuse + kFuseMaxRows * kS8FuseMaxK + 64));
+    }
+
     int32_t total[kS8MB][NB][4];
 #pragma unroll
     for (int j = 0; j < kS8MB; ++j)
@@ -169,8 +192,15 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
                             bfr[h][b][i][1] = cw[i] & hi_mask;          // 16 x odd positions
                         }
                     } else {
-                        const uint4* ar = reinterpret_cast<const uint4*>(act + static_cast<size_t>(tok) * K + kb);
-                        const uint4 c0 = __ldg(ar), c1 = __ldg(ar + 1);
+                        uint4 c0, c1;
+                        if constexpr (FUSED) {
+                            c0 = lds128(reinterpret_cast<const uint8_t*>(sCodes) + tok * K + kb);
+                            c1 = lds128(reinterpret_cast<const uint8_t*>(sCodes) + tok * K + kb + 16);
+                        } else {
+                            const uint4* ar = reinterpret_cast<const uint4*>(act + static_cast<size_t>(tok) * K + kb);
+                            c0 = __ldg(ar);
+                            c1 = __ldg(ar + 1);
+                        }
                         const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
@@ -277,7 +307,8 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
                 reinterpret_cast<int32_t*>(out)[static_cast<size_t>(tok) * N + row] = v[q] >> kShift;
             } else {
                 const float bsv = bias ? __bfloat162float(bias[row]) : 0.0f;
-                const float val = static_cast<float>(v[q]) * __ldg(tok_scale + tok) *
+                const float st = FUSED ? sTokScale[tok] : __ldg(tok_scale + tok);
+                const float val = static_cast<float>(v[q]) * st *
                                   (__ldg(row_scale + row) * kUnscale) + bsv;
                 reinterpret_cast<__nv_bfloat16*>(out)[static_cast<size_t>(tok) * N + row] =
                     __float2bfloat16_rn(val);

@@ -173,6 +173,26 @@ def test_decode_w4a8_full_size(M, act_bits):
     assert_gemm_output(bf16_from_gpu(y), oracle.epilogue_f64(acc_ref, st, sr, None))
 
 
+@pytest.mark.parametrize("act_bits", [8, 4])
+@pytest.mark.parametrize("M,N,K,g", [(1, 16, 32, 0), (2, 272, 352, 16), (3, 528, 1088, 64),
+                                     (4, 1024, 4096, 256), (1, 12288, 4096, 256), (4, 96, 3840, 64)])
+def test_fused_decode_linear(M, N, K, g, act_bits):
+    """Decode-sized linears: at M = 1, K <= 4096 the GEMM kernel rotates and
+    quantizes x itself (same codes as the separate rotate+quantize), larger M
+    take the two launches; all against the oracle, with a bias."""
+    x = inputs.activations(M, K, seed=830 + K)
+    if M > 1:
+        x[1, :] = 0                                 # an all-zero token
+    W = inputs.weights(N, K, seed=831 + N)
+    wp, sr, _ = oracle.pack_weights(W, g)
+    bias = inputs.f32_to_bf16_bits(np.linspace(-2, 2, N))
+    y_ref = oracle.convrot_linear_f64(x, wp, sr, g, act_bits, bias)
+    fn = t4.convrot_w4a8_linear if act_bits == 8 else t4.convrot_w4a4_linear
+    y = fn(bf16_to_gpu(x), to_gpu(wp), to_gpu(sr), g, bf16_to_gpu(bias))
+    torch.cuda.synchronize()
+    assert_gemm_output(bf16_from_gpu(y), y_ref, np.broadcast_to(bias, (M, N)))
+
+
 @pytest.mark.parametrize("prefetch", [False, True])
 def test_decode_weight_prefetch_switch(prefetch):
     """With the decode weight streaming switched on, the small-M kernels give
