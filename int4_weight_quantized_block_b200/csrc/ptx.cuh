@@ -90,6 +90,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// [lo, hi) of part i when n items are split into p contiguous parts of
+// near-equal size (the first n % p parts one larger); 32-bit arithmetic.
+__device__ __forceinline__ void even_split(unsigned n, unsigned p, unsigned i, int& lo, int& hi) {
+    const unsigned q = n / p, r = n % p;
+    lo = static_cast<int>(i * q + (i < r ? i : r));
+    hi = lo + static_cast<int>(q) + (i < r ? 1 : 0);
+}
+
 // ----------------------------------------------------------------- proxies / fences
 
 // Make generic-proxy writes to shared memory visible to the async proxy

@@ -169,8 +169,8 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
     const int t = lane & 3;    // which 32-value slice of a group
     const int npairs = (ngroups + 1) / 2;
     const int nblk = N / 16;
-    const int b0 = static_cast<int>((static_cast<long long>(blockIdx.x) * nblk) / gridDim.x);
-    const int b1 = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * nblk) / gridDim.x);
+    int b0, b1;   // this CTA's run of blocks (32-bit arithmetic: 64-bit division is a long
+    even_split(nblk, gridDim.x, blockIdx.x, b0, b1);   // software routine on the prologue's path)
     const int nb = b1 - b0;             // 1..kW16MB (the host sizes the grid)
     const int nbp = (nb + 1) / 2;       // block pairs (an odd run's last box reads 16 rows it skips)
     const int rA = w16_perm(g), rB = w16_perm(g + 8);   // weight rows of MMA rows g, g + 8
@@ -183,8 +183,8 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
     // the run's units in pair-major order, u = P * nbp + bp; this warp takes
     // the contiguous, balanced range [u0, u1)
     const int ntot = npairs * nbp;
-    const int u0 = static_cast<int>((static_cast<long long>(warp) * ntot) / WARPS);
-    const int u1 = static_cast<int>((static_cast<long long>(warp + 1) * ntot) / WARPS);
+    int u0, u1;
+    even_split(ntot, WARPS, warp, u0, u1);
     const int nunits = u1 - u0;
     uint64_t* full = full_all + warp * SLOTS;
     uint8_t* ring = sm + warp * SLOTS * kW16Box;

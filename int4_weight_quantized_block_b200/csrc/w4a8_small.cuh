@@ -103,8 +103,8 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
     const int t = lane & 3;    // which 32-value slice of a 128-K half chunk
     const int nchunks = (K + 255) / 256;
     const int nblk = N / 16;
-    const int b0 = static_cast<int>((static_cast<long long>(blockIdx.x) * nblk) / gridDim.x);
-    const int b1 = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * nblk) / gridDim.x);
+    int b0, b1;   // this CTA's run of blocks (32-bit arithmetic: 64-bit division is a long
+    even_split(nblk, gridDim.x, blockIdx.x, b0, b1);   // software routine on the prologue's path)
     const int nb = b1 - b0;             // 1..kS8MB (the host sizes the grid)
     const int nbp = (nb + 1) / 2;       // block pairs (an odd run's last box reads 16 rows it skips)
     const int rA = s8_perm(g), rB = s8_perm(g + 8);
@@ -112,8 +112,8 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
 
     // the run's units in chunk-major order, u = P * nbp + bp; this warp's range
     const int ntot = nchunks * nbp;
-    const int u0 = static_cast<int>((static_cast<long long>(warp) * ntot) / kS8Warps);
-    const int u1 = static_cast<int>((static_cast<long long>(warp + 1) * ntot) / kS8Warps);
+    int u0, u1;
+    even_split(ntot, kS8Warps, warp, u0, u1);
     const int nunits = u1 - u0;
     uint64_t* full = full_all + warp * kS8Slots;
     uint8_t* ring = sm + warp * kS8Slots * kS8Box;
