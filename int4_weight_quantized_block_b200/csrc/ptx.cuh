@@ -102,6 +102,15 @@ __device__ __forceinline__ void even_split(unsigned n, unsigned p, unsigned i, i
 
 // Make generic-proxy writes to shared memory visible to the async proxy
 // (tensor core operand reads, TMA).
+// 4-byte global -> shared copy that holds no register while in flight
+// (completion: cp_async_wait_all by the issuing thread, then a barrier)
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

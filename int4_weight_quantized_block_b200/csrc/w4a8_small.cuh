@@ -51,7 +51,13 @@ struct S8Cfg {
     static constexpr int WARPS = NB == 1 ? 16 : 8;
     static constexpr int THREADS = WARPS * 32;
     static constexpr int SLOTS = kS8Ring / (WARPS * kS8Box);   // boxes in flight per warp
-    static constexpr int SMEM = kS8Ring + WARPS * SLOTS * 8 + 16 + 1024;   // + barriers, abort flag, alignment
+    // ring | barriers, abort flag | epilogue operands (row scales, bias, token
+    // scales of the run) | fused linear's codes | alignment slack
+    static constexpr int EPI_OFF = kS8Ring + WARPS * SLOTS * 8 + 16;
+    static constexpr int EPI_BYTES = kS8MB * 16 * 4 + kS8MB * 16 * 2 + kS8MaxM * 4;
+    static constexpr int FUSE_OFF = EPI_OFF + EPI_BYTES;
+    static constexpr int SMEM = FUSE_OFF + 1024;
+    static_assert(EPI_OFF % 16 == 0 && FUSE_OFF % 16 == 0, "16-byte aligned regions");
     static_assert(WARPS * kS8MB * NB * 32 * 16 <= kS8Ring, "the reduction reuses the ring");
 };
 
@@ -145,8 +151,21 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
     grid_launch_dependents();
     if (lane == 0 && issued == 0 && nunits > 0) issue(issued++);
 
+    // The epilogue's operands of this run go to shared memory now, by
+    // asynchronous copies that land during the main loop: read from global
+    // memory at the end they would add a memory round trip to every launch.
+    float* sRowScale = reinterpret_cast<float*>(sm + C::EPI_OFF);
+    __nv_bfloat16* sBias = reinterpret_cast<__nv_bfloat16*>(sm + C::EPI_OFF + kS8MB * 16 * 4);
+    float* sTok = reinterpret_cast<float*>(sm + C::EPI_OFF + kS8MB * 16 * 6);
+    if constexpr (!OUT_I32) {
+        const int tid = threadIdx.x;
+        if (tid < nb * 16) cp_async4(sRowScale + tid, row_scale + b0 * 16 + tid);
+        if (bias != nullptr && tid < nb * 8) cp_async4(sBias + 2 * tid, bias + b0 * 16 + 2 * tid);
+        if (!FUSED && tid < M) cp_async4(sTok + tid, tok_scale + tid);
+    }
+
     // fused linear: x -> codes and scales in shared memory, under the first boxes
-    uint8_t* sfuse = sm + kS8Ring + kS8Warps * kS8Slots * 8 + 16;
+    uint8_t* sfuse = sm + C::FUSE_OFF;
     const int8_t* sCodes = reinterpret_cast<const int8_t*>(sfuse);
     const float* sTokScale = reinterpret_cast<const float*>(sfuse + kFuseMaxRows * kS8FuseMaxK);
     if constexpr (FUSED) {
@@ -271,6 +290,7 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
     }
 
     // ---- the warps' partial sums meet in shared memory
+    cp_async_wait_all();
     __syncthreads();
 #pragma unroll
     for (int j = 0; j < kS8MB; ++j) {
@@ -296,20 +316,22 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
         }
         const int gg = ln >> 2, tt = ln & 3;
         const int tok0 = 8 * b + 2 * tt;
-        const int r0 = (b0 + j) * 16 + s8_perm(gg), r1 = (b0 + j) * 16 + s8_perm(gg + 8);
+        const int l0 = j * 16 + s8_perm(gg), l1 = j * 16 + s8_perm(gg + 8);   // rows of the run
+        const int r0 = b0 * 16 + l0, r1 = b0 * 16 + l1;
         // v: [0] row r0 / token tok0, [1] r0 / tok0 + 1, [2] r1 / tok0, [3] r1 / tok0 + 1
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const int tok = tok0 + (q & 1);
             const int row = (q & 2) ? r1 : r0;
+            const int lrow = (q & 2) ? l1 : l0;
             if (tok >= M) continue;
             if constexpr (OUT_I32) {
                 reinterpret_cast<int32_t*>(out)[static_cast<size_t>(tok) * N + row] = v[q] >> kShift;
             } else {
-                const float bsv = bias ? __bfloat162float(bias[row]) : 0.0f;
-                const float st = FUSED ? sTokScale[tok] : __ldg(tok_scale + tok);
+                const float bsv = bias ? __bfloat162float(sBias[lrow]) : 0.0f;
+                const float st = FUSED ? sTokScale[tok] : sTok[tok];
                 const float val = static_cast<float>(v[q]) * st *
-                                  (__ldg(row_scale + row) * kUnscale) + bsv;
+                                  (sRowScale[lrow] * kUnscale) + bsv;
                 reinterpret_cast<__nv_bfloat16*>(out)[static_cast<size_t>(tok) * N + row] =
                     __float2bfloat16_rn(val);
             }
