@@ -72,6 +72,7 @@ def _load():
             "oracle_convrot_linear_f64": [P, P, P, P, I, I, I, I, I, P],
             "oracle_w4a16": [P, P, P, P, I, I, I, I, P],
             "oracle_w4a16_f64": [P, P, P, P, I, I, I, I, P],
+            "oracle_w4a16_dequant_f64": [P, P, P, P, I, I, I, I, P],
             "oracle_round_bf16": [P, L, P],
             "oracle_num_threads": [],
         }
@@ -338,6 +339,26 @@ def w4a16_f64(x_bits, q_packed, scale_bits, zero, group) -> np.ndarray:
     y = np.empty((M, N), dtype=np.float64)
     _check(_load().oracle_w4a16_f64(_ptr(x), _ptr(q), _ptr(s), _ptr(z), M, N, K, group,
                                     _ptr(y)), "w4a16_f64")
+    return y
+
+
+def w4a16_dequant_f64(x_bits, q_packed, scale_bits, zero, group) -> np.ndarray:
+    """The W4A16 layer in its 16-bit unpack + 16-bit GEMM form, before the
+    output's bf16 rounding: each weight is first rounded to the bf16 number
+    nearest to (q - z) * s, then y = x . w^T in fp64.
+
+    "ComfyUI-INT-Crush", "Inference > INT4 > Triton backend": with
+    rot_size == 0 the INT4 weights are widened to 16 bits for a 16-bit GEMM;
+    "TINT4 v1.2", "v1.1 新特性 > 5": the torchao layer's _qdata/_scale/_zp."""
+    x = _c(x_bits, np.uint16)
+    q = _c(q_packed, np.uint8)
+    s = _c(scale_bits, np.uint16)
+    z = _c(zero, np.uint8)
+    M, K = x.shape
+    N = q.shape[0]
+    y = np.empty((M, N), dtype=np.float64)
+    _check(_load().oracle_w4a16_dequant_f64(_ptr(x), _ptr(q), _ptr(s), _ptr(z), M, N, K, group,
+                                            _ptr(y)), "w4a16_dequant_f64")
     return y
 
 

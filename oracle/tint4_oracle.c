@@ -450,6 +450,41 @@ int oracle_w4a16_f64(const uint16_t* x, const uint8_t* q, const uint16_t* s, con
     return ORACLE_OK;
 }
 
+/* The 16-bit unpack + 16-bit GEMM form ("ComfyUI-INT-Crush", "Inference >
+ * INT4 > Triton backend": W4A16 widens the INT4 weights to 16 bits and runs a
+ * 16-bit GEMM): every weight is first dequantized to the bf16 number nearest
+ * to (q - z) * s (the product itself is exact in double), then
+ * y[m, n] = sum_k x[m, k] * w[n, k] in fp64, unrounded. */
+int oracle_w4a16_dequant_f64(const uint16_t* x, const uint8_t* q, const uint16_t* s,
+                             const uint8_t* z, int M, int N, int K, int G, double* y) {
+    if (!x || !q || !s || !z || !y || M < 0 || N < 0 || K <= 0 || G <= 0 || K % G || K % 2)
+        return ORACLE_BAD_ARG;
+    int ng = K / G;
+    int bad = 0;
+#pragma omp parallel for schedule(static) reduction(| : bad)
+    for (int n = 0; n < N; ++n) {
+        double* w = (double*)malloc(sizeof(double) * (size_t)K);
+        if (!w) {
+            bad = 1;
+            continue;
+        }
+        for (int k = 0; k < K; ++k) {
+            uint8_t b = q[(long)n * (K / 2) + k / 2];
+            int code = (k % 2 == 0) ? (b & 0xF) : (b >> 4);
+            double exact = ((double)code - (double)z[(long)n * ng + k / G]) *
+                           (double)bf16_bits_to_float(s[(long)n * ng + k / G]);
+            w[k] = (double)bf16_bits_to_float(double_to_bf16_bits(exact));
+        }
+        for (int m = 0; m < M; ++m) {
+            double acc = 0.0;
+            for (int k = 0; k < K; ++k) acc += (double)bf16_bits_to_float(x[(long)m * K + k]) * w[k];
+            y[(long)m * N + n] = acc;
+        }
+        free(w);
+    }
+    return bad ? ORACLE_BAD_ARG : ORACLE_OK;
+}
+
 /* The same, rounded once to bf16: the layer's output. */
 int oracle_w4a16(const uint16_t* x, const uint8_t* q, const uint16_t* s, const uint8_t* z,
                  int M, int N, int K, int G, uint16_t* y) {

@@ -395,6 +395,49 @@ def test_w4a16_general_dequant():
             assert y[m, n] == _bf16_nearest_even(float(ref[m, n]))
 
 
+def test_w4a16_dequant_golden():
+    """Worked example of the 16-bit unpack form: each weight rounded to bf16
+    (ties to even) before the products; the exact form on the same inputs."""
+    d = golden("w4a16_dequant_rounding.json")
+    K, G = d["K"], d["group"]
+    q = np.array([[b] * (K // 2) for b in d["row_byte"]], np.uint8)
+    z = np.array(d["zero"], np.uint8)
+    s = bits(d["scale"])
+    x = bits(np.ones((1, K)))
+    assert oracle.w4a16_dequant_f64(x, q, s, z, G)[0].tolist() == d["y"]
+    assert oracle.w4a16_f64(x, q, s, z, G)[0].tolist() == d["y_unrounded_weights"]
+
+
+def test_w4a16_dequant_equals_exact_form_for_power_of_two_scales():
+    """With every scale a power of two, (q - z) * s has at most 4 significant
+    bits: the bf16 widening is exact and both forms give the same values."""
+    M, N, K, G = 3, 9, 384, 128
+    op = inputs.w4a16_operands(M, N, K, G, seed=33)
+    rng = np.random.default_rng(34)
+    s = bits(np.ldexp(1.0, rng.integers(-12, 4, size=(N, K // G))))
+    a = oracle.w4a16_dequant_f64(op.x, op.q, s, op.zero, G)
+    b = oracle.w4a16_f64(op.x, op.q, s, op.zero, G)
+    assert np.array_equal(a, b)
+
+
+def test_w4a16_dequant_error_within_half_ulp_bound():
+    """Rounding each weight to 8 significant bits moves it by at most 2^-8 of
+    its size, so the two forms differ by at most sum_k |x_k| |w_k| 2^-8; on
+    general scales they do differ."""
+    M, N, K, G = 4, 16, 512, 128
+    op = inputs.w4a16_operands(M, N, K, G, seed=35)
+    a = oracle.w4a16_dequant_f64(op.x, op.q, op.scale, op.zero, G)
+    b = oracle.w4a16_f64(op.x, op.q, op.scale, op.zero, G)
+    qk = np.empty((N, K), np.float64)
+    qk[:, 0::2] = op.q & 0xF
+    qk[:, 1::2] = op.q >> 4
+    w = (qk - np.repeat(op.zero.astype(np.float64), G, axis=1)) * \
+        np.repeat(oracle.bf16_bits_to_f32(op.scale).astype(np.float64), G, axis=1)
+    bound = np.abs(oracle.bf16_bits_to_f32(op.x).astype(np.float64)) @ np.abs(w).T * 2.0 ** -8
+    assert np.all(np.abs(a - b) <= bound * (1 + 1e-9))
+    assert np.any(a != b)
+
+
 # ---------------------------------------------------------------- fp64 outputs and the comparison
 
 def test_unrounded_outputs_round_to_the_bf16_outputs():
