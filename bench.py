@@ -72,6 +72,7 @@ KERNEL_SOURCES = {
     "rotate_quantize_rows_kernel": ("quantize.cuh", "ptx.cuh"),
     "w4a16_mma_kernel": ("w4a16.cuh", "ptx.cuh"),
     "w4a8_small_kernel": ("w4a8_small.cuh", "ptx.cuh"),
+    "w4a16_tmem_gemm_kernel": ("w4a16_gemm.cuh", "ptx.cuh"),
 }
 
 
@@ -419,6 +420,26 @@ def bench_rows(args, t4, inputs, dev, flush, pk, int8_peak):
                       "_chained: with tint4_set_decode_weight_prefetch(1), each call's weights "
                       "stream while the previous call finishes"}
 
+    # W4A16 prefill: the same layer on thousands of tokens, the tensor-core
+    # GEMM with the weights widened to bf16 in TMEM
+    w = inputs.WORKLOADS["te_prefill_w4a16"]
+    M, N, K, G = w["M"], w["N"], w["K"], w["group"]
+    op = inputs.w4a16_operands(M, N, K, G)
+    xg, qg = bf16_gpu(op.x, dev), torch.from_numpy(op.q).to(dev)
+    sg, zg = bf16_gpu(op.scale, dev), torch.from_numpy(op.zero).to(dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    t4.w4a16_gemv_gemm(xg, qg, sg, zg, G, y)
+    torch.cuda.synchronize(dev)
+    ms = statistics.median(time_steps(lambda: t4.w4a16_gemv_gemm(xg, qg, sg, zg, G, y),
+                                      reps, flush, dev))
+    flops = 2.0 * M * N * K
+    rows["te_prefill_w4a16"] = {
+        "kernel": "w4a16_tmem_gemm_kernel", "M": M, "N": N, "K": K, "group": G,
+        "us": round(ms * 1e3, 2), "TFLOPS": round(flops / ms / 1e9, 2),
+        "frac_bf16": round(flops / ms / 1e9 / pk["bf16"], 4),
+        "timing": "median of CUDA-event times per call, L2 flushed between calls"}
+    del xg, qg, sg, zg, y
+
     # W4A8 decode (same shape, ConvRot group 256): the fused linear and the GEMM
     # alone, 8 copies of the packed weights rotated
     w = inputs.WORKLOADS["te_decode_w4a8"]
@@ -575,7 +596,7 @@ def run_profile_case(case: str, dev):
             t4.w4a8_gemm(codes, st, wp, sr, None, y)
     elif case.startswith("w4a16_M"):
         M = int(case[len("w4a16_M"):])
-        w = inputs.WORKLOADS["te_decode_w4a16"]
+        w = inputs.WORKLOADS["te_prefill_w4a16" if M > 32 else "te_decode_w4a16"]
         op = inputs.w4a16_operands(M, w["N"], w["K"], w["group"])
         x, q, s, z = (bf16_gpu(op.x, dev), torch.from_numpy(op.q).to(dev),
                       bf16_gpu(op.scale, dev), torch.from_numpy(op.zero).to(dev))

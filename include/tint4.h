@@ -176,18 +176,23 @@ tint4_status convrot_w4a8_linear_noalloc(const tint4_bf16* x, const uint8_t* w_p
                                          void* stream);
 
 /*
- * W4A16 group-wise asymmetric linear for small M ("TINT4 v1.2", "v1.1 新特性
- * > 5" _qdata/_scale/_zp, "参数选择指南" group 128; "ComfyUI-INT-Crush",
+ * W4A16 group-wise asymmetric linear ("TINT4 v1.2", "v1.1 新特性 > 5"
+ * _qdata/_scale/_zp, "参数选择指南" group 128; "ComfyUI-INT-Crush",
  * "Inference > INT4 > Triton backend" W4A16).  x bf16 [M, K]; w_q uint8
  * [N, K/2] unsigned codes 0..15 packed low nibble first; scale bf16
  * [N, K/group]; zero uint8 [N, K/group] holding 0..15; y bf16 [M, N] with
  * y[m, n] = sum_k x[m, k] * (q[n, k] - zero[n, k/group]) * scale[n, k/group]
- * accumulated in fp32.  group must be 128; 1 <= M <= 32; N % 16 == 0;
- * K % 128 == 0, K <= 16384; all pointers 16-byte aligned.  One kernel launch
- * per 16 tokens: a batch of 17..32 tokens reads the weights twice.  Errors:
- * TINT4_ERR_UNSUPPORTED_SHAPE for sizes outside these limits,
- * TINT4_ERR_MISALIGNED, TINT4_ERR_INVALID_ARG for null pointers; nothing is
- * launched then.
+ * accumulated in fp32.
+ *   - M <= 32 (decode): the weights are streamed once per 16 tokens (a batch
+ *     of 17..32 tokens reads them twice) and each product uses
+ *     (q - z) * s exactly; K <= 16384.
+ *   - M > 32 (prefill): one tensor-core GEMM launch; every weight is first
+ *     rounded to the bf16 number nearest to (q - z) * s (what a bf16
+ *     dequantize-then-matmul uses), products accumulate in fp32; K <= 65536.
+ * group must be 128; 1 <= M <= 65535 * 128; N % 16 == 0; K % 128 == 0; all
+ * pointers 16-byte aligned.  Errors: TINT4_ERR_UNSUPPORTED_SHAPE for sizes
+ * outside these limits, TINT4_ERR_MISALIGNED, TINT4_ERR_INVALID_ARG for null
+ * pointers; nothing is launched then.
  */
 tint4_status w4a16_gemv_gemm(const tint4_bf16* x, const uint8_t* w_q, const tint4_bf16* scale,
                              const uint8_t* zero, int group, tint4_bf16* y, int M, int N, int K,

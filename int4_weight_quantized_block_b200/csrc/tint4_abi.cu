@@ -16,6 +16,7 @@
 #include "ptx.cuh"
 #include "quantize.cuh"
 #include "w4a16.cuh"
+#include "w4a16_gemm.cuh"
 #include "w4a8_small.cuh"
 
 namespace {
@@ -25,6 +26,7 @@ using namespace tint4;
 constexpr int kAbiVersion = 1;
 constexpr int kMaxDevices = 64;
 constexpr int kMaxTokens = 65535 * 128;   // M limit of the GEMM entry points
+constexpr int kW16SmallMaxM = 32;         // W4A16: up to here the streaming kernel, above the GEMM
 
 std::atomic<uint64_t> g_wait_limit_ns{4000000000ull};
 std::atomic<int> g_decode_prefetch{0};   // tint4_set_decode_weight_prefetch
@@ -428,6 +430,45 @@ tint4_status linear_entry(int bits, const tint4_bf16* x, const uint8_t* w_packed
 
 // ------------------------------------------------------------------ W4A16
 
+// Large M: the tcgen05 GEMM with the weights dequantized into TMEM
+// (w4a16_gemm.cuh).
+tint4_status launch_w4a16_gemm(const __nv_bfloat16* x, const uint8_t* q, const __nv_bfloat16* s,
+                               const uint8_t* z, __nv_bfloat16* y, int M, int N, int K,
+                               cudaStream_t st) {
+    auto kern = w4a16_tmem_gemm_kernel;
+    CUtensorMap tx, tq;
+    bool ok = make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M,
+                          static_cast<uint64_t>(K) * 2, kWgBK, kWgBN, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && make_map_u8(&tq, q, K / 2, N, K / 2, kWgBK / 2, kWgBM, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!ok) return TINT4_ERR_CUDA;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static std::atomic<bool> attr_done[kMaxDevices];
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kWgSmemBytes) != cudaSuccess) {
+            cudaGetLastError();
+            return TINT4_ERR_CUDA;
+        }
+        attr_done[dev].store(true, std::memory_order_release);
+    }
+    const int tiles = ((M + kWgBN - 1) / kWgBN) * ((N + kWgBM - 1) / kWgBM);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(std::min(tiles, num_sms(dev)), 1, 1);
+    cfg.blockDim = dim3(kWgThreads, 1, 1);
+    cfg.dynamicSmemBytes = kWgSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tx, tq, s, z, y, M, N, K,
+                           g_wait_limit_ns.load(std::memory_order_relaxed)) != cudaSuccess) {
+        cudaGetLastError();
+        return TINT4_ERR_CUDA;
+    }
+    return last_launch_status();
+}
+
 template <int NB>
 tint4_status launch_w4a16(const __nv_bfloat16* x, const uint8_t* q, const __nv_bfloat16* s,
                           const uint8_t* z, __nv_bfloat16* y, int M, int N, int K,
@@ -635,8 +676,9 @@ tint4_status w4a16_gemv_gemm(const tint4_bf16* x, const uint8_t* w_q, const tint
                              void* stream) {
     if (M < 0 || N < 0 || K < 0) return TINT4_ERR_INVALID_ARG;
     if (group != kW16Group) return TINT4_ERR_UNSUPPORTED_SHAPE;
-    if (M < 1 || M > 32 || N < 16 || N % 16 != 0 || K < kW16Group || K % kW16Group != 0 ||
-        K > kW16MaxK)
+    const bool small = M <= kW16SmallMaxM;
+    if (M < 1 || M > kMaxTokens || N < 16 || N % 16 != 0 || K < kW16Group ||
+        K % kW16Group != 0 || K > (small ? kW16MaxK : 65536))
         return TINT4_ERR_UNSUPPORTED_SHAPE;
     if (!x || !w_q || !scale || !zero || !y) return TINT4_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_q) || !aligned16(scale) || !aligned16(zero) ||
@@ -648,6 +690,7 @@ tint4_status w4a16_gemv_gemm(const tint4_bf16* x, const uint8_t* w_q, const tint
     const auto* sb = reinterpret_cast<const __nv_bfloat16*>(scale);
     auto* yb = reinterpret_cast<__nv_bfloat16*>(y);
     cudaStream_t st = as_stream(stream);
+    if (!small) return launch_w4a16_gemm(xb, w_q, sb, zero, yb, M, N, K, st);
     // 16 tokens per launch: a 17..32-token batch streams the weights twice
     for (int m0 = 0; m0 < M; m0 += kW16MaxM) {
         const int mc = std::min(kW16MaxM, M - m0);

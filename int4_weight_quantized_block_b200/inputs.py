@@ -128,6 +128,8 @@ WORKLOADS = {
     "dit_mlp_down_w4a8": dict(M=4608, K=12288, N=3072, group=64, act_bits=8, x="gelu"),
     # small-M text-encoder decode
     "te_decode_w4a16": dict(Ms=(1, 4, 16), K=4096, N=12288, group=128),
+    # the same layer on a prefill batch: the tensor-core branch
+    "te_prefill_w4a16": dict(M=4096, K=4096, N=12288, group=128),
     "te_decode_w4a8": dict(Ms=(1, 4, 16), K=4096, N=12288, group=256, act_bits=8, x="attn"),
 }
 

@@ -114,7 +114,12 @@ def test_linear_workspace_rules(lib):
 
 def test_w4a16_rules(lib):
     assert lib.w4a16_gemv_gemm(16, 16, 16, 16, 64, 16, 1, 256, 256, NULL) == 2   # group
-    assert lib.w4a16_gemv_gemm(16, 16, 16, 16, 128, 16, 33, 256, 256, NULL) == 2  # M > 32
+    assert lib.w4a16_gemv_gemm(16, 16, 16, 16, 128, 16, 32, 256, 16512, NULL) == 2  # decode K
+    assert lib.w4a16_gemv_gemm(16, 16, 16, 16, 128, 16, 33, 256, 65664, NULL) == 2  # GEMM K
+    assert lib.w4a16_gemv_gemm(16, 16, 16, 16, 128, 16, 65535 * 128 + 1, 256, 256,
+                               NULL) == 2                                          # M
+    assert lib.w4a16_gemv_gemm(16, 16, 16, 16, 128, 16, 0, 256, 256, NULL) == 2    # M
+    assert lib.w4a16_gemv_gemm(16, 16, 16, 16, 128, 16, 33, 8, 256, NULL) == 2     # N % 16
     assert lib.w4a16_gemv_gemm(16, 16, 16, 16, 128, 16, 1, 256, 192, NULL) == 2  # K % 128
     assert lib.w4a16_gemv_gemm(NULL, 16, 16, 16, 128, 16, 1, 256, 256, NULL) == 1
     assert lib.w4a16_gemv_gemm(16, 24, 16, 16, 128, 16, 1, 256, 256, NULL) == 3

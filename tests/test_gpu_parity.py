@@ -349,6 +349,80 @@ def test_w4a16_full_size(M):
     assert c.ok, str(c)
 
 
+# W4A16 above 32 tokens: one tensor-core GEMM, weights widened to bf16 first
+# (the 16-bit unpack form); held to that form with the accumulation tolerance
+# and to the exact form with the layer's 1e-2 bar.
+def check_w4a16_large(y_bits, op, rows=None, cols=None):
+    x, q, sc, z = op.x, op.q, op.scale, op.zero
+    if rows is not None:
+        x = x[rows]
+        y_bits = y_bits[rows]
+    if cols is not None:
+        q, sc, z = q[cols], sc[cols], z[cols]
+        y_bits = y_bits[:, cols]
+    ref_dq = oracle.w4a16_dequant_f64(x, q, sc, z, 128)
+    c = check_bf16(y_bits, ref_dq, accumulation_error(ref_dq), TIE_FRAC_ACCUMULATED)
+    assert c.ok, "16-bit unpack form: " + str(c)
+    # against the exact form (q - z) * s: per element, the widening moves the
+    # value by at most 2^-8 sum_k |x_k| |w_k|, the output rounding by half an
+    # ulp (< 2^-8 |y|), the fp32 accumulation by the tolerance above
+    ref = oracle.w4a16_f64(x, q, sc, z, 128)
+    qk = np.empty((q.shape[0], 2 * q.shape[1]), np.float64)
+    qk[:, 0::2] = q & 0xF
+    qk[:, 1::2] = q >> 4
+    w = (qk - np.repeat(z.astype(np.float64), 128, axis=1)) * \
+        np.repeat(oracle.bf16_bits_to_f32(sc).astype(np.float64), 128, axis=1)
+    xa = np.abs(oracle.bf16_bits_to_f32(x).astype(np.float64))
+    bound = (xa @ np.abs(w).T + np.abs(ref_dq)) * 2.0 ** -8 + accumulation_error(ref_dq)
+    g = oracle.bf16_bits_to_f32(y_bits).astype(np.float64)
+    excess = np.abs(g - ref) - bound
+    assert np.all(excess <= 0), f"exact form: bound exceeded by {excess.max():.3e}"
+
+
+@pytest.mark.parametrize("M,N,K", [(33, 16, 128), (64, 272, 384), (192, 128, 1024),
+                                   (200, 1040, 256), (385, 512, 2048), (1000, 96, 640)])
+def test_w4a16_large_m(M, N, K):
+    op = inputs.w4a16_operands(M, N, K, 128, seed=900 + M)
+    y = t4.w4a16_gemv_gemm(bf16_to_gpu(op.x), to_gpu(op.q), bf16_to_gpu(op.scale),
+                           to_gpu(op.zero), 128)
+    torch.cuda.synchronize()
+    check_w4a16_large(bf16_from_gpu(y), op)
+
+
+def test_w4a16_large_m_extreme_token_values():
+    """Tiny and huge token values next to ordinary ones (bf16 range, not fp16's)."""
+    M, N, K = 96, 256, 1024
+    op = inputs.w4a16_operands(M, N, K, 128, seed=930)
+    x = oracle.bf16_bits_to_f32(op.x).reshape(M, K).astype(np.float64)
+    x[3, 17] = 1.0e-30
+    x[40, 600] = 3.0e-7
+    x[95, 1000] = 7.0e4
+    xb = inputs.f32_to_bf16_bits(x)
+    y = t4.w4a16_gemv_gemm(bf16_to_gpu(xb), to_gpu(op.q), bf16_to_gpu(op.scale),
+                           to_gpu(op.zero), 128)
+    torch.cuda.synchronize()
+    ref_dq = oracle.w4a16_dequant_f64(xb, op.q, op.scale, op.zero, 128)
+    c = check_bf16(bf16_from_gpu(y), ref_dq, accumulation_error(ref_dq), TIE_FRAC_ACCUMULATED)
+    assert c.ok, str(c)
+
+
+def test_w4a16_prefill_full_size():
+    """The prefill workload (weights of the decode layer, thousands of tokens),
+    checked on sampled token rows and weight rows."""
+    w = inputs.WORKLOADS["te_prefill_w4a16"]
+    M, N, K = w["M"], w["N"], w["K"]
+    op = inputs.w4a16_operands(M, N, K, w["group"])
+    y = t4.w4a16_gemv_gemm(bf16_to_gpu(op.x), to_gpu(op.q), bf16_to_gpu(op.scale),
+                           to_gpu(op.zero), w["group"])
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(7)
+    rows = np.sort(rng.choice(M, 48, replace=False))
+    rows[-1] = M - 1
+    cols = np.sort(rng.choice(N, 256, replace=False))
+    cols[-1] = N - 1
+    check_w4a16_large(bf16_from_gpu(y), op, rows, cols)
+
+
 # ------------------------------------------------------------------ edge cases
 
 def test_empty_m_is_a_no_op():
