@@ -136,7 +136,7 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
     uint8_t* sW = smem + kWgStages * kWgActBytes;
     uint8_t* sOut = sW + kWgStages * kWgWBytes;
     uint64_t* act_full = reinterpret_cast<uint64_t*>(sOut + kWgOutBytes);
-    uint64_t* a_full = act_full + kWgStages;       // TMEM A stage written (128 arrivals)
+    uint64_t* a_full = act_full + kWgStages;       // TMEM A stage written (one arrival per warp)
     uint64_t* empty = a_full + kWgStages;          // stage consumed by the MMAs (commit)
     uint64_t* acc_full = empty + kWgStages;        // [2] accumulator ready (commit)
     uint64_t* acc_empty = acc_full + 2;            // [2] accumulator drained (8 warp arrivals)
@@ -157,7 +157,7 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
     if (threadIdx.x == 0) {
         for (int s = 0; s < kWgStages; ++s) {
             mbar_init(&act_full[s], 1);
-            mbar_init(&a_full[s], 128);
+            mbar_init(&a_full[s], 4);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -232,9 +232,11 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                 for (int kt = 0; kt < KT; ++kt, ++c) {
                     const int s = c % kWgStages;
                     const uint32_t ph = (c / kWgStages) & 1;
-                    if (!mbar_wait_bounded(&act_full[s], ph, abort_flag, wait_ns,
-                                           kDevErrTimeoutConsumer) ||
-                        !mbar_wait_bounded(&a_full[s], ph, abort_flag, wait_ns,
+                    // a_full implies act_full: the unpack warps arrive on it only
+                    // after they have seen the stage land (one wait per stage:
+                    // the issuing thread's time per stage is the tensor pipe's
+                    // budget)
+                    if (!mbar_wait_bounded(&a_full[s], ph, abort_flag, wait_ns,
                                            kDevErrTimeoutConsumer)) {
                         ok = false;
                         break;
@@ -309,7 +311,8 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
             tmem_st_32x32b_x32(tmem_base + lane_base + kWgColA + 32 * s, a);
             tmem_st_wait();
             tcgen05_fence_before();
-            mbar_arrive(&a_full[s]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_full[s]);
         }
     } else if (warp < 18) {
         // ------------------------------------------------ epilogue (warps 10-17)
