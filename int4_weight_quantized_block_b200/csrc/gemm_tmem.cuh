@@ -194,7 +194,12 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = umma_idesc_i8(kTmBM, kTmBN);
-            uint32_t c = 0;
+            // B descriptors: stage s starts (s * bytes) / 16 units above stage 0,
+            // MMA kk of a stage 32 bytes = 2 units further (the address field
+            // cannot carry: shared addresses are below 2^18)
+            const uint64_t bdesc0 = umma_desc_sw128(smem_u32(sAct));
+            int s = 0;
+            uint32_t ph = 0u;
             bool ok = true;
             for (int i = 0; i < my_tiles && ok; ++i) {
                 const int buf = i & 1;
@@ -206,13 +211,10 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                 }
                 tcgen05_fence_after();
                 const uint32_t d_tmem = tmem_base + kTmColD + buf * kTmBN;
-                for (int kt = 0; kt < KT; ++kt, ++c) {
-                    const int s = c % kTmStages;
-                    const uint32_t ph = (c / kTmStages) & 1;
-                    // a_full implies act_full: the unpack warps arrive on it only
-                    // after they have seen the stage land (one wait per stage:
-                    // the issuing thread's time per stage is the tensor pipe's
-                    // budget)
+                for (int kt = 0; kt < KT; ++kt) {
+                    // a_full implies the stage has landed: the unpack warps arrive
+                    // on it only after they have seen it (one wait per stage: the
+                    // issuing thread's time per stage is the tensor pipe's budget)
                     if (!mbar_wait_bounded(&a_full[s], ph, abort_flag, wait_ns,
                                            kDevErrTimeoutConsumer)) {
                         ok = false;
@@ -220,12 +222,15 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                     }
                     tcgen05_fence_after();
                     const uint32_t a_tmem = tmem_base + kTmColA + 32 * s;
-                    const uint32_t b_addr = smem_u32(sAct + s * kTmActBytes);
+                    const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(s * (kTmActBytes >> 4));
 #pragma unroll
                     for (int kk = 0; kk < kTmBK / 32; ++kk)
-                        umma_i8_ts(d_tmem, a_tmem + 8 * kk, umma_desc_sw128(b_addr + 32 * kk),
-                                   idesc, (kt | kk) != 0);
+                        umma_i8_ts(d_tmem, a_tmem + 8 * kk, bdesc + 2 * kk, idesc, (kt | kk) != 0);
                     umma_commit(&empty[s]);
+                    if (++s == kTmStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 if (ok) umma_commit(&acc_full[buf]);
             }

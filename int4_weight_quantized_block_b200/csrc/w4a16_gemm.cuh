@@ -217,7 +217,12 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = umma_idesc_bf16(kWgBM, kWgBN);
-            uint32_t c = 0;
+            // B descriptors: stage s starts (s * bytes) / 16 units above stage 0,
+            // MMA kk of a stage 32 bytes = 2 units further (the address field
+            // cannot carry: shared addresses are below 2^18)
+            const uint64_t bdesc0 = umma_desc_sw128(smem_u32(sAct));
+            int s = 0;
+            uint32_t ph = 0u;
             bool ok = true;
             for (int i = 0; i < my_tiles && ok; ++i) {
                 const int buf = i & 1;
@@ -229,13 +234,10 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                 }
                 tcgen05_fence_after();
                 const uint32_t d_tmem = tmem_base + kWgColD + buf * kWgBN;
-                for (int kt = 0; kt < KT; ++kt, ++c) {
-                    const int s = c % kWgStages;
-                    const uint32_t ph = (c / kWgStages) & 1;
-                    // a_full implies act_full: the unpack warps arrive on it only
-                    // after they have seen the stage land (one wait per stage:
-                    // the issuing thread's time per stage is the tensor pipe's
-                    // budget)
+                for (int kt = 0; kt < KT; ++kt) {
+                    // a_full implies the stage has landed: the unpack warps arrive
+                    // on it only after they have seen it (one wait per stage: the
+                    // issuing thread's time per stage is the tensor pipe's budget)
                     if (!mbar_wait_bounded(&a_full[s], ph, abort_flag, wait_ns,
                                            kDevErrTimeoutConsumer)) {
                         ok = false;
@@ -243,12 +245,15 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                     }
                     tcgen05_fence_after();
                     const uint32_t a_tmem = tmem_base + kWgColA + 32 * s;
-                    const uint32_t b_addr = smem_u32(sAct + s * kWgActBytes);
+                    const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(s * (kWgActBytes >> 4));
 #pragma unroll
-                    for (int kk = 0; kk < kWgBK / 16; ++kk)   // K 16 = 32 bytes = 8 TMEM columns
-                        umma_bf16_ts(d_tmem, a_tmem + 8 * kk, umma_desc_sw128(b_addr + 32 * kk),
-                                     idesc, (kt | kk) != 0);
+                    for (int kk = 0; kk < kWgBK / 16; ++kk)
+                        umma_bf16_ts(d_tmem, a_tmem + 8 * kk, bdesc + 2 * kk, idesc, (kt | kk) != 0);
                     umma_commit(&empty[s]);
+                    if (++s == kWgStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 if (ok) umma_commit(&acc_full[buf]);
             }
