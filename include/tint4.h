@@ -176,6 +176,49 @@ tint4_status convrot_w4a8_linear_noalloc(const tint4_bf16* x, const uint8_t* w_p
                                          void* stream);
 
 /*
+ * Grouped GEMM: the same activation codes times up to TINT4_MAX_GROUPS
+ * weight matrices in one launch ("feat: packed int4 convrot model loading
+ * and dispatch", "Summary": the activation rotate + quantize is shared by the
+ * linears of one input; separate Q, K and V projections, say).  For each
+ * group g: y_g [M, N_g] = bf16(acc_g * s_tok * s_row_g (+ bias_g)), exactly
+ * what w4a8_gemm gives for that group alone.
+ *   - codes int8 [M, K], tok_scale fp32 [M] as for w4a8_gemm.
+ *   - groups: a HOST array of num_groups entries, read during the call only;
+ *     each entry holds device pointers (w_packed [N_g, K/2], row_scale [N_g],
+ *     bias [N_g] or NULL, y [M, N_g]) and N_g.
+ *   - 1 <= num_groups <= TINT4_MAX_GROUPS; every N_g obeys the w4a8_gemm
+ *     rules (N_g % 16 == 0), K too; all pointers 16-byte aligned.
+ *   - M <= 16 runs one small-M launch per group; above, one launch for all.
+ * Errors: TINT4_ERR_INVALID_ARG (null groups or pointers, num_groups < 1),
+ * TINT4_ERR_UNSUPPORTED_SHAPE (num_groups > TINT4_MAX_GROUPS, a bad N_g, M
+ * or K), TINT4_ERR_MISALIGNED; nothing is launched then.
+ */
+#define TINT4_MAX_GROUPS 4
+typedef struct {
+    const uint8_t* w_packed;
+    const float* row_scale;
+    const tint4_bf16* bias;
+    tint4_bf16* y;
+    int N;
+} tint4_weight_group;
+
+tint4_status w4a8_gemm_grouped(const int8_t* codes, const float* tok_scale,
+                               const tint4_weight_group* groups, int num_groups, int M, int K,
+                               void* stream);
+
+/*
+ * convrot_w4a8_linear over a group of weight matrices: x bf16 [M, K] is
+ * rotated (group `group`) and quantized to int8 once, into the workspace
+ * (convrot_linear_workspace_size(M, K, 8) bytes, 256-byte aligned), then
+ * w4a8_gemm_grouped runs.  Same rules and errors as convrot_w4a8_linear and
+ * w4a8_gemm_grouped.
+ */
+tint4_status convrot_w4a8_linear_grouped(const tint4_bf16* x, const tint4_weight_group* groups,
+                                         int num_groups, int M, int K, int group,
+                                         void* workspace, size_t workspace_bytes,
+                                         void* stream);
+
+/*
  * W4A16 group-wise asymmetric linear ("TINT4 v1.2", "v1.1 新特性 > 5"
  * _qdata/_scale/_zp, "参数选择指南" group 128; "ComfyUI-INT-Crush",
  * "Inference > INT4 > Triton backend" W4A16).  x bf16 [M, K]; w_q uint8

@@ -11,6 +11,8 @@ from __future__ import annotations
 
 from typing import Optional, Tuple
 
+import ctypes
+
 import torch
 
 from . import _native
@@ -183,6 +185,52 @@ def convrot_w4a8_linear_noalloc(x, w_packed, row_scale, group, bias=None, y=None
     _native.call("convrot_w4a8_linear_noalloc", _ptr(x), _ptr(w_packed), _ptr(row_scale),
                  _ptr(bias), _ptr(y), M, N, K, group, _stream(x.device))
     return y
+
+
+def _groups(M, K, device, groups):
+    """(w_packed, row_scale, bias or None, y or None) tuples -> ctypes array, ys."""
+    if not 1 <= len(groups) <= _native.MAX_GROUPS:
+        raise ValueError(f"1 to {_native.MAX_GROUPS} weight groups")
+    arr = (_native.WeightGroup * len(groups))()
+    ys = []
+    for i, (w, sr, bias, y) in enumerate(groups):
+        N = w.shape[0]
+        _need(w, "w_packed", torch.uint8, (N, K // 2))
+        _need(sr, "row_scale", torch.float32, (N,))
+        if bias is not None:
+            _need(bias, "bias", torch.bfloat16, (N,))
+        if y is None:
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        _need(y, "y", torch.bfloat16, (M, N))
+        arr[i] = _native.WeightGroup(_ptr(w), _ptr(sr), _ptr(bias), _ptr(y), N)
+        ys.append(y)
+    return arr, ys
+
+
+def w4a8_gemm_grouped(a, tok_scale, groups):
+    """int8 codes a [M, K] times each (w_packed [N_g, K/2], row_scale [N_g],
+    bias [N_g] or None, y [M, N_g] or None) of `groups`, one launch for all;
+    returns the list of bf16 outputs."""
+    _need(a, "a", torch.int8)
+    M, K = a.shape
+    _need(tok_scale, "tok_scale", torch.float32, (M,))
+    arr, ys = _groups(M, K, a.device, groups)
+    _native.call("w4a8_gemm_grouped", _ptr(a), _ptr(tok_scale), ctypes.addressof(arr),
+                 len(groups), M, K, _stream(a.device))
+    return ys
+
+
+def convrot_w4a8_linear_grouped(x, groups, group, workspace=None):
+    """Rotate + int8 quantize x once, then w4a8_gemm_grouped over `groups`."""
+    _need(x, "x", torch.bfloat16)
+    M, K = x.shape
+    arr, ys = _groups(M, K, x.device, groups)
+    need = convrot_linear_workspace_size(M, K, 8)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    _native.call("convrot_w4a8_linear_grouped", _ptr(x), ctypes.addressof(arr), len(groups),
+                 M, K, group, _ptr(workspace), workspace.numel(), _stream(x.device))
+    return ys
 
 
 def w4a16_gemv_gemm(x, w_q, scale, zero, group: int = 128, y=None) -> torch.Tensor:

@@ -28,6 +28,13 @@ I = ctypes.c_int
 U64 = ctypes.c_uint64
 SZ = ctypes.c_size_t
 
+MAX_GROUPS = 4   # TINT4_MAX_GROUPS
+
+
+class WeightGroup(ctypes.Structure):
+    """tint4_weight_group: one weight matrix of a grouped call (device pointers)."""
+    _fields_ = [("w_packed", P), ("row_scale", P), ("bias", P), ("y", P), ("N", I)]
+
 # name -> (restype, argtypes); mirrors include/tint4.h
 SIGNATURES = {
     "tint4_abi_version": (I, []),
@@ -41,6 +48,8 @@ SIGNATURES = {
     "convrot_w4a4_linear": (I, [P, P, P, P, P, I, I, I, I, P, SZ, P]),
     "convrot_w4a8_linear_noalloc": (I, [P, P, P, P, P, I, I, I, I, P]),
     "w4a16_gemv_gemm": (I, [P, P, P, P, I, P, I, I, I, P]),
+    "w4a8_gemm_grouped": (I, [P, P, P, I, I, I, P]),
+    "convrot_w4a8_linear_grouped": (I, [P, P, I, I, I, I, P, SZ, P]),
     "tint4_debug_int32_gemm": (I, [P, I, P, P, I, I, I, P]),
     "tint4_debug_bounded_wait": (I, [U64, P]),
     "tint4_get_device_error": (I, [P]),

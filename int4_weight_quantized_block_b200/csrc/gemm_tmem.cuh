@@ -73,6 +73,21 @@ constexpr uint32_t kTmColA = 2 * kTmBN;               // A stage s at kTmColA + 
 static_assert(kTmColA + 32 * kTmStages <= 512, "TMEM budget");
 static_assert(kTmActBytes % 1024 == 0 && kTmWBytes % 1024 == 0, "swizzled stage alignment");
 
+// The weight matrices one launch multiplies the same activation codes with:
+// one for a plain GEMM, up to kTmMaxGroups for a grouped one (separate Q, K,
+// V projections of one input, say).  The tile list runs group after group:
+// tiles [tile_end[g-1], tile_end[g]) belong to group g.
+constexpr int kTmMaxGroups = 4;
+struct TmGroups {
+    CUtensorMap w[kTmMaxGroups];              // packed weights [N_g, K/2]
+    const float* row_scale[kTmMaxGroups];     // [N_g]
+    const __nv_bfloat16* bias[kTmMaxGroups];  // [N_g] or null
+    void* out[kTmMaxGroups];                  // y_g [M, N_g] (bf16, or int32 sums)
+    int N[kTmMaxGroups];
+    int tile_end[kTmMaxGroups];
+    int count;
+};
+
 __device__ __forceinline__ void umma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                            uint32_t idesc, uint32_t accumulate) {
     asm volatile(
@@ -97,10 +112,8 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 template <bool OUT_I32, bool A_INT4>
 __global__ void __launch_bounds__(kTmThreads, 1)
 w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
-                      const __grid_constant__ CUtensorMap tmap_w,
-                      const float* __restrict__ tok_scale,
-                      const float* __restrict__ row_scale, const __nv_bfloat16* __restrict__ bias,
-                      void* __restrict__ out, int M, int N, int K, uint64_t wait_ns) {
+                      const __grid_constant__ TmGroups grp,
+                      const float* __restrict__ tok_scale, int M, int K, uint64_t wait_ns) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -121,10 +134,21 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int m_tiles = (M + kTmBN - 1) / kTmBN;
-    const int n_tiles = (N + kTmBM - 1) / kTmBM;
-    const int n_work = m_tiles * n_tiles;
+    const int n_work = grp.tile_end[grp.count - 1];
     const int KT = (K + kTmBK - 1) / kTmBK;
     const int my_tiles = (blockIdx.x < n_work) ? (n_work - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    // tile -> (group, first token, first weight row of the group)
+    struct TileAt {
+        int g, m0, n0;
+    };
+    auto tile_at = [&](int tile) -> TileAt {
+        int g = 0;
+#pragma unroll
+        for (int h = 0; h < kTmMaxGroups - 1; ++h)
+            if (h + 1 < grp.count && tile >= grp.tile_end[h]) g = h + 1;
+        const int t = tile - (g > 0 ? grp.tile_end[g - 1] : 0);
+        return TileAt{g, (t % m_tiles) * kTmBN, (t / m_tiles) * kTmBM};
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kTmStages; ++s) {
@@ -142,7 +166,7 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
     }
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tmap_act);
-        prefetch_tensormap(&tmap_w);
+        for (int g = 0; g < grp.count; ++g) prefetch_tensormap(&grp.w[g]);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
@@ -162,9 +186,9 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             uint32_t c = 0;
             int issued = 0;
             for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
-                const int tile = blockIdx.x + i * gridDim.x;
-                const int m0 = (tile % m_tiles) * kTmBN;
-                const int n0 = (tile / m_tiles) * kTmBM;
+                const TileAt ta = tile_at(blockIdx.x + i * gridDim.x);
+                const int m0 = ta.m0, n0 = ta.n0;
+                const CUtensorMap* tmap_w = &grp.w[ta.g];
                 for (int kt = 0; kt < KT; ++kt, ++c) {
                     const int s = c % kTmStages;
                     const uint32_t ph = (c / kTmStages) & 1;
@@ -178,7 +202,7 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                         mbar_arrive_expect_tx(&act_full[s], kTmActBytes + kTmWBytes);
                         tma_load_2d(&tmap_act, &act_full[s], sAct + s * kTmActBytes, kt * kTmBK, m0);
                     }
-                    tma_load_2d(&tmap_w, &act_full[s], sW + s * kTmWBytes, kt * (kTmBK / 2), n0);
+                    tma_load_2d(tmap_w, &act_full[s], sW + s * kTmWBytes, kt * (kTmBK / 2), n0);
                     ++issued;
                 }
             }
@@ -301,9 +325,12 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const bool leader = (e == 0 && lane == 0);
         for (int i = 0; i < my_tiles; ++i) {
-            const int tile = blockIdx.x + i * gridDim.x;
-            const int m0 = (tile % m_tiles) * kTmBN;
-            const int n0 = (tile / m_tiles) * kTmBM;
+            const TileAt ta = tile_at(blockIdx.x + i * gridDim.x);
+            const int m0 = ta.m0, n0 = ta.n0;
+            const int N = grp.N[ta.g];
+            const float* __restrict__ row_scale = grp.row_scale[ta.g];
+            const __nv_bfloat16* __restrict__ bias = grp.bias[ta.g];
+            void* __restrict__ out = grp.out[ta.g];
             const int n = n0 + r;
             const int buf = i & 1;
             // one thread waits for the accumulator; the named barrier hands the

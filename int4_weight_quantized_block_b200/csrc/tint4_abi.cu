@@ -211,17 +211,26 @@ cudaLaunchAttribute pdl_attr() {
 }
 
 // Weights widened into TMEM (gemm_tmem.cuh); activation codes int8, or
-// packed int4 widened in shared memory (A_INT4).
+// packed int4 widened in shared memory (A_INT4).  `grp` holds 1 to
+// kTmMaxGroups weight matrices sharing the activation codes (the tensor maps
+// and the tile list are filled in here).
 template <bool OUT_I32, bool A_INT4>
-tint4_status launch_gemm_tmem(const void* a, const uint8_t* w, const float* st, const float* sr,
-                              const __nv_bfloat16* bias, void* out, int M, int N, int K,
-                              cudaStream_t stream, bool pdl) {
+tint4_status launch_gemm_tmem(const void* a, const float* st, TmGroups& grp,
+                              const uint8_t* const* w, int M, int K, cudaStream_t stream,
+                              bool pdl) {
     auto kern = w4a8_tmem_gemm_kernel<OUT_I32, A_INT4>;
     constexpr int smem_bytes = A_INT4 ? kTmSmemBytesA4 : kTmSmemBytes;
-    CUtensorMap ta, tw;
+    CUtensorMap ta;
     bool ok = A_INT4 ? make_map_u8(&ta, a, K / 2, M, K / 2, kTmBK / 2, kTmBN, CU_TENSOR_MAP_SWIZZLE_NONE)
                      : make_map_u8(&ta, a, K, M, K, kTmBK, kTmBN, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && make_map_u8(&tw, w, K / 2, N, K / 2, kTmBK / 2, kTmBM, CU_TENSOR_MAP_SWIZZLE_64B);
+    const int m_tiles = (M + kTmBN - 1) / kTmBN;
+    int tiles = 0;
+    for (int g = 0; g < grp.count; ++g) {
+        ok = ok && make_map_u8(&grp.w[g], w[g], K / 2, grp.N[g], K / 2, kTmBK / 2, kTmBM,
+                               CU_TENSOR_MAP_SWIZZLE_64B);
+        tiles += m_tiles * ((grp.N[g] + kTmBM - 1) / kTmBM);
+        grp.tile_end[g] = tiles;
+    }
     if (!ok) return TINT4_ERR_CUDA;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -234,7 +243,6 @@ tint4_status launch_gemm_tmem(const void* a, const uint8_t* w, const float* st, 
         }
         attr_done[dev].store(true, std::memory_order_release);
     }
-    const int tiles = ((M + kTmBN - 1) / kTmBN) * ((N + kTmBM - 1) / kTmBM);
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(std::min(tiles, num_sms(dev)), 1, 1);
     cfg.blockDim = dim3(kTmThreads, 1, 1);
@@ -246,8 +254,7 @@ tint4_status launch_gemm_tmem(const void* a, const uint8_t* w, const float* st, 
         cfg.numAttrs = 1;
     }
     const uint64_t wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
-    if (cudaLaunchKernelEx(&cfg, kern, ta, tw, st, sr, bias, out, M, N, K, wait_ns) !=
-        cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, kern, ta, grp, st, M, K, wait_ns) != cudaSuccess) {
         cudaGetLastError();
         return TINT4_ERR_CUDA;
     }
@@ -365,7 +372,13 @@ tint4_status launch_gemm(const void* a, const uint8_t* w, const float* st, const
         return launch_gemm_small<1, A_INT4, OUT_I32>(a, w, st, sr, bias, out, M, N, K, stream, pdl);
     if (M <= kS8MaxM)
         return launch_gemm_small<2, A_INT4, OUT_I32>(a, w, st, sr, bias, out, M, N, K, stream, pdl);
-    return launch_gemm_tmem<OUT_I32, A_INT4>(a, w, st, sr, bias, out, M, N, K, stream, pdl);
+    TmGroups grp{};
+    grp.row_scale[0] = sr;
+    grp.bias[0] = bias;
+    grp.out[0] = out;
+    grp.N[0] = N;
+    grp.count = 1;
+    return launch_gemm_tmem<OUT_I32, A_INT4>(a, st, grp, &w, M, K, stream, pdl);
 }
 
 tint4_status gemm_entry(bool a_int4, const void* a, const float* tok_scale, const uint8_t* w,
@@ -558,6 +571,52 @@ void* static_scratch_address(int dev) {
     return g_static_scratch_ptr[dev];
 }
 
+static_assert(TINT4_MAX_GROUPS == kTmMaxGroups, "group limit of the ABI and the kernel");
+
+// Shape, pointer and alignment rules of a grouped call (nothing launched).
+tint4_status check_groups(const tint4_weight_group* groups, int num_groups, int M, int K) {
+    if (groups == nullptr || num_groups < 1) return TINT4_ERR_INVALID_ARG;
+    if (num_groups > TINT4_MAX_GROUPS) return TINT4_ERR_UNSUPPORTED_SHAPE;
+    for (int g = 0; g < num_groups; ++g) {
+        const tint4_weight_group& w = groups[g];
+        tint4_status s = check_mnk(M, w.N, K);
+        if (s != TINT4_OK) return s;
+        if (M > 0 && (!w.w_packed || !w.row_scale || !w.y)) return TINT4_ERR_INVALID_ARG;
+        if (!aligned16(w.w_packed) || !aligned16(w.row_scale) || !aligned16(w.bias) ||
+            !aligned16(w.y))
+            return TINT4_ERR_MISALIGNED;
+    }
+    return TINT4_OK;
+}
+
+tint4_status launch_gemm_grouped(const int8_t* codes, const float* tok_scale,
+                                 const tint4_weight_group* groups, int num_groups, int M, int K,
+                                 cudaStream_t st, bool pdl) {
+    if (M <= kS8MaxM) {
+        // every weight is read once per launch anyway: one small-M launch per group
+        for (int g = 0; g < num_groups; ++g) {
+            const tint4_weight_group& w = groups[g];
+            const tint4_status s = launch_gemm<false, false>(
+                codes, w.w_packed, tok_scale, w.row_scale,
+                reinterpret_cast<const __nv_bfloat16*>(w.bias), w.y, M, w.N, K, st,
+                pdl || g > 0);
+            if (s != TINT4_OK) return s;
+        }
+        return TINT4_OK;
+    }
+    TmGroups grp{};
+    const uint8_t* w[kTmMaxGroups] = {};
+    for (int g = 0; g < num_groups; ++g) {
+        w[g] = groups[g].w_packed;
+        grp.row_scale[g] = groups[g].row_scale;
+        grp.bias[g] = reinterpret_cast<const __nv_bfloat16*>(groups[g].bias);
+        grp.out[g] = groups[g].y;
+        grp.N[g] = groups[g].N;
+    }
+    grp.count = num_groups;
+    return launch_gemm_tmem<false, false>(codes, tok_scale, grp, w, M, K, st, pdl);
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -641,6 +700,44 @@ tint4_status convrot_w4a4_linear(const tint4_bf16* x, const uint8_t* w_packed,
                                  size_t workspace_bytes, void* stream) {
     return linear_entry(4, x, w_packed, row_scale, bias, y, M, N, K, group, workspace,
                         workspace_bytes, stream);
+}
+
+tint4_status w4a8_gemm_grouped(const int8_t* codes, const float* tok_scale,
+                                          const tint4_weight_group* groups, int num_groups, int M,
+                                          int K, void* stream) {
+    tint4_status s = check_groups(groups, num_groups, M, K);
+    if (s != TINT4_OK) return s;
+    if (M > 0 && (!codes || !tok_scale)) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(codes) || !aligned16(tok_scale)) return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (M == 0) return TINT4_OK;
+    return launch_gemm_grouped(codes, tok_scale, groups, num_groups, M, K, as_stream(stream),
+                               false);
+}
+
+tint4_status convrot_w4a8_linear_grouped(const tint4_bf16* x,
+                                                    const tint4_weight_group* groups,
+                                                    int num_groups, int M, int K, int group,
+                                                    void* workspace, size_t workspace_bytes,
+                                                    void* stream) {
+    tint4_status s = check_groups(groups, num_groups, M, K);
+    if (s != TINT4_OK) return s;
+    if ((s = check_rq_shape(M, K, group)) != TINT4_OK) return s;
+    if (M > 0 && !x) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(x)) return TINT4_ERR_MISALIGNED;
+    if (M > 0 && (!workspace || workspace_bytes < convrot_linear_workspace_size(M, K, 8)))
+        return TINT4_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (M == 0) return TINT4_OK;
+    int8_t* codes = static_cast<int8_t*>(workspace);
+    float* tok_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                                align_up(static_cast<size_t>(M) * K, 256));
+    cudaStream_t st = as_stream(stream);
+    launch_rq_g<__nv_bfloat16, 127, false>(reinterpret_cast<const __nv_bfloat16*>(x), M, K, group,
+                                           codes, tok_scale, st);
+    if ((s = last_launch_status()) != TINT4_OK) return s;
+    return launch_gemm_grouped(codes, tok_scale, groups, num_groups, M, K, st, true);
 }
 
 tint4_status convrot_w4a8_linear_noalloc(const tint4_bf16* x, const uint8_t* w_packed,

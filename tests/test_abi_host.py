@@ -125,6 +125,27 @@ def test_w4a16_rules(lib):
     assert lib.w4a16_gemv_gemm(16, 24, 16, 16, 128, 16, 1, 256, 256, NULL) == 3
 
 
+def test_grouped_rules(lib):
+    from int4_weight_quantized_block_b200._native import WeightGroup
+    G = WeightGroup * 5
+    ok = G(*[WeightGroup(16, 16, None, 16, 256) for _ in range(5)])
+    assert lib.w4a8_gemm_grouped(16, 16, NULL, 1, 4, 256, NULL) == 1                 # null groups
+    assert lib.w4a8_gemm_grouped(16, 16, ctypes.addressof(ok), 0, 4, 256, NULL) == 1  # none
+    assert lib.w4a8_gemm_grouped(16, 16, ctypes.addressof(ok), 5, 4, 256, NULL) == 2  # too many
+    bad_n = G(WeightGroup(16, 16, None, 16, 256), WeightGroup(16, 16, None, 16, 8))
+    assert lib.w4a8_gemm_grouped(16, 16, ctypes.addressof(bad_n), 2, 4, 256, NULL) == 2
+    bad_p = G(WeightGroup(16, 16, None, 16, 256), WeightGroup(None, 16, None, 16, 256))
+    assert lib.w4a8_gemm_grouped(16, 16, ctypes.addressof(bad_p), 2, 4, 256, NULL) == 1
+    mis = G(WeightGroup(16, 16, None, 24, 256))
+    assert lib.w4a8_gemm_grouped(16, 16, ctypes.addressof(mis), 1, 4, 256, NULL) == 3
+    assert lib.w4a8_gemm_grouped(NULL, 16, ctypes.addressof(ok), 1, 4, 256, NULL) == 1
+    need = lib.convrot_linear_workspace_size(4, 256, 8)
+    assert lib.convrot_w4a8_linear_grouped(16, ctypes.addressof(ok), 1, 4, 256, 16, NULL, need,
+                                           NULL) == 6
+    assert lib.convrot_w4a8_linear_grouped(16, ctypes.addressof(ok), 1, 4, 256, 32, 256, need,
+                                           NULL) == 1                                  # group value
+
+
 def test_debug_entries_rules(lib):
     assert lib.tint4_debug_int32_gemm(16, 6, 16, 16, 4, 256, 256, NULL) == 1
     assert lib.tint4_debug_bounded_wait(10, NULL) == 1

@@ -299,6 +299,70 @@ def test_full_size_workloads_sampled(name):
     assert np.array_equal(acc_gpu.cpu().numpy()[pairs[:, 0], pairs[:, 1]], acc)
 
 
+# ------------------------------------------------------------------ grouped GEMM
+
+@pytest.mark.parametrize("M", [8, 200])
+def test_gemm_grouped_matches_separate_calls(M):
+    """One grouped launch over three weight matrices (Q, K, V of different
+    widths) gives each group exactly the bits of its own w4a8_gemm, and those
+    match the oracle."""
+    K, g = 512, 64
+    Ns = (1024, 256, 272)
+    x = inputs.activations(M, K, seed=700 + M)
+    codes, st, _ = oracle.quantize_act(x, g, 8)
+    cg, sg = to_gpu(codes), to_gpu(st)
+    groups, ref = [], []
+    for i, N in enumerate(Ns):
+        wp, sr, _ = oracle.pack_weights(inputs.weights(N, K, seed=710 + i), g)
+        b = inputs.f32_to_bf16_bits(np.linspace(-0.5, 0.5, N, dtype=np.float32)) if i == 1 else None
+        groups.append((to_gpu(wp), to_gpu(sr), None if b is None else bf16_to_gpu(b), None))
+        ref.append((wp, sr, b))
+    ys = t4.w4a8_gemm_grouped(cg, sg, groups)
+    singles = [t4.w4a8_gemm(cg, sg, w, sr, b) for (w, sr, b, _) in groups]
+    torch.cuda.synchronize()
+    for y, y1, (wp, sr, b) in zip(ys, singles, ref):
+        assert np.array_equal(bf16_from_gpu(y), bf16_from_gpu(y1))
+        acc = oracle.gemm_i32(codes, oracle.unpack_int4(wp))
+        y64 = oracle.epilogue_f64(acc, st, sr, b)
+        assert_gemm_output(bf16_from_gpu(y), y64, b)
+
+
+@pytest.mark.parametrize("M", [1, 64, 333])
+def test_linear_grouped(M):
+    K, g = 768, 256
+    Ns = (512, 128)
+    x = inputs.activations(M, K, seed=720 + M)
+    groups, ref = [], []
+    for i, N in enumerate(Ns):
+        wp, sr, _ = oracle.pack_weights(inputs.weights(N, K, seed=730 + i), g)
+        groups.append((to_gpu(wp), to_gpu(sr), None, None))
+        ref.append((wp, sr))
+    ys = t4.convrot_w4a8_linear_grouped(bf16_to_gpu(x), groups, g)
+    torch.cuda.synchronize()
+    for y, (wp, sr) in zip(ys, ref):
+        assert_gemm_output(bf16_from_gpu(y), oracle.convrot_linear_f64(x, wp, sr, g, 8))
+
+
+def test_gemm_grouped_full_size_qkv_split():
+    """The DiT QKV layer with its 9216 weight rows split into separate Q, K
+    and V matrices: the grouped launch reproduces the concatenated GEMM's
+    columns bit for bit (that GEMM is itself held to the oracle)."""
+    w = inputs.WORKLOADS["dit_qkv_w4a8"]
+    M, N, K, g = w["M"], w["N"], w["K"], w["group"]
+    x_np, W_np = inputs.layer_inputs("dit_qkv_w4a8")
+    x = bf16_to_gpu(x_np)
+    wp, sr = t4.tint4_pack_weights(torch.from_numpy(W_np).to(dev()), g)
+    codes, st = t4.convrot_quantize_act(x, g, 8)
+    y = t4.w4a8_gemm(codes, st, wp, sr)
+    third = N // 3
+    parts = [(wp[i * third:(i + 1) * third].contiguous(), sr[i * third:(i + 1) * third].contiguous(),
+              None, None) for i in range(3)]
+    ys = t4.w4a8_gemm_grouped(codes, st, parts)
+    torch.cuda.synchronize()
+    for i, yg in enumerate(ys):
+        assert torch.equal(yg, y[:, i * third:(i + 1) * third])
+
+
 # ------------------------------------------------------------------ W4A16
 
 @pytest.mark.parametrize("M,N,K", [(1, 16, 128), (4, 272, 384), (16, 512, 1024),
