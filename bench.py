@@ -388,6 +388,41 @@ def bench_rows(args, t4, inputs, dev, flush, pk, int8_peak):
     rows["dit_mlp_up_w4a8"] = gemm_layer("dit_mlp_up_w4a8")
     rows["dit_mlp_down_w4a8"] = gemm_layer("dit_mlp_down_w4a8")
 
+    # the QKV layer as three separate 3072-row weight matrices (Q, K, V of one
+    # input): three GEMM launches against one grouped launch
+    w = inputs.WORKLOADS["dit_qkv_w4a8"]
+    M, N, K, g = w["M"], w["N"], w["K"], w["group"]
+    x_np, W_np = inputs.layer_inputs("dit_qkv_w4a8")
+    x = bf16_gpu(x_np, dev)
+    wp, sr = t4.tint4_pack_weights(torch.from_numpy(W_np).to(dev), g)
+    del W_np
+    codes, st = t4.convrot_quantize_act(x, g, 8)
+    third = N // 3
+    parts = [(wp[i * third:(i + 1) * third].contiguous(), sr[i * third:(i + 1) * third].contiguous(),
+              None, torch.empty((M, third), dtype=torch.bfloat16, device=dev)) for i in range(3)]
+    ws = torch.empty(t4.convrot_linear_workspace_size(M, K, 8), dtype=torch.uint8, device=dev)
+
+    def separate():
+        for (wq, srq, _, yq) in parts:
+            t4.w4a8_gemm(codes, st, wq, srq, None, yq)
+
+    separate()
+    t4.w4a8_gemm_grouped(codes, st, parts)
+    t4.convrot_w4a8_linear_grouped(x, parts, g, ws)
+    torch.cuda.synchronize(dev)
+    s_ms = statistics.median(time_steps(separate, reps, flush, dev))
+    g_ms = statistics.median(time_steps(lambda: t4.w4a8_gemm_grouped(codes, st, parts), reps, flush, dev))
+    l_ms = statistics.median(time_steps(lambda: t4.convrot_w4a8_linear_grouped(x, parts, g, ws),
+                                        reps, flush, dev))
+    ops = 2.0 * M * N * K
+    rows["dit_qkv_split_w4a8"] = {
+        "M": M, "N": f"3 x {third}", "K": K, "group": g,
+        "separate_gemms_us": round(s_ms * 1e3, 2), "separate_gemms_TOPS": round(ops / s_ms / 1e9, 2),
+        "grouped_gemm_us": round(g_ms * 1e3, 2), "grouped_gemm_TOPS": round(ops / g_ms / 1e9, 2),
+        "grouped_gemm_frac_int8": round(ops / g_ms / 1e9 / int8_peak, 4),
+        "grouped_linear_us": round(l_ms * 1e3, 2), "grouped_linear_TOPS": round(ops / l_ms / 1e9, 2)}
+    del parts, codes, st, wp, sr, x, ws
+
     # W4A16 decode: rotate over 8 weight copies (> L2) so bytes come from HBM
     w = inputs.WORKLOADS["te_decode_w4a16"]
     N, K, G = w["N"], w["K"], w["group"]
