@@ -73,6 +73,7 @@ def _load():
             "oracle_w4a16": [P, P, P, P, I, I, I, I, P],
             "oracle_w4a16_f64": [P, P, P, P, I, I, I, I, P],
             "oracle_w4a16_dequant_f64": [P, P, P, P, I, I, I, I, P],
+            "oracle_quantize_weights_int8": [P, I, I, I, P, P],
             "oracle_round_bf16": [P, L, P],
             "oracle_num_threads": [],
         }
@@ -202,6 +203,22 @@ def pack_weights(W: np.ndarray, g: int):
     _check(_load().oracle_pack_weights(_ptr(Wc), N, K, g, _ptr(packed), _ptr(scale),
                                        _ptr(codes)), "pack_weights")
     return packed, scale, codes
+
+
+def quantize_weights_int8(W: np.ndarray, g: int):
+    """Twin of ``tint4_quantize_weights_int8``: rotate W along K, per-row
+    symmetric int8 codes [N, K] in [-127, 127] and fp32 row scales [N].
+
+    "ComfyUI-INT-Crush", "Inference > INT8" (int8 weights x int8 activations,
+    int32 accumulation); the rotation and rounding are those of the int4
+    weights ("Weight Format", "Forward Pass")."""
+    Wc = _c(W, np.float32)
+    N, K = Wc.shape
+    codes = np.empty((N, K), dtype=np.int8)
+    scale = np.empty(N, dtype=np.float32)
+    _check(_load().oracle_quantize_weights_int8(_ptr(Wc), N, K, g, _ptr(codes), _ptr(scale)),
+           "quantize_weights_int8")
+    return codes, scale
 
 
 def quantize_act(x_bits: np.ndarray, g: int, bits: int):

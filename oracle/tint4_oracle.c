@@ -250,6 +250,34 @@ int oracle_pack_weights(const float* W, int N, int K, int g, uint8_t* packed,
     return bad ? ORACLE_BAD_ARG : ORACLE_OK;
 }
 
+/* W8A8 weights ("ComfyUI-INT-Crush", "Inference > INT8": the INT8 path
+ * multiplies int8 weights by int8 activations with int32 accumulation):
+ * W fp32 [N, K] -> rotate each g-block along K -> per-row symmetric int8
+ * codes in [-127, 127] [N, K] with an fp32 row scale absmax / 127. */
+int oracle_quantize_weights_int8(const float* W, int N, int K, int g, int8_t* codes,
+                                 float* row_scale) {
+    if (!W || !codes || !row_scale || N <= 0 || K <= 0) return ORACLE_BAD_ARG;
+    if (g != 0 && (!is_power_of_four(g) || K % g)) return ORACLE_BAD_ARG;
+    int bad = 0;
+#pragma omp parallel
+    {
+        float* v = (float*)malloc(sizeof(float) * (size_t)K);
+        if (!v) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(static)
+            for (int n = 0; n < N; ++n) {
+                memcpy(v, W + (long)n * K, sizeof(float) * (size_t)K);
+                if (g) for (int b = 0; b < K; b += g) fwht_f32_block(v + b, g);
+                quantize_row(v, K, 127, codes + (long)n * K, &row_scale[n]);
+            }
+        }
+        free(v);
+    }
+    return bad ? ORACLE_BAD_ARG : ORACLE_OK;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Dynamic per-token activation quantization (twin of convrot_quantize_act) */
 /* ------------------------------------------------------------------------ */

@@ -181,6 +181,37 @@ def test_weight_quant_error_bound(g):
     assert np.array_equal(oracle.unpack_int4(packed), codes)
 
 
+def test_int8_weight_codes_golden():
+    d = golden("w8a8_weight_codes.json")
+    codes, s = oracle.quantize_weights_int8(np.array(d["W"], np.float32), d["group"])
+    assert codes.tolist() == d["codes"]
+    assert s.tolist() == d["row_scale"]
+
+
+@pytest.mark.parametrize("g", (0,) + GROUPS)
+def test_int8_weight_quant_error_bound(g):
+    """Rotated rows (an independent fp64 rotation) within s/2 of q s, the
+    largest entry of every row at +-127; a one-hot row under group 16 becomes
+    16 equal values 1/4, all coded 127."""
+    K = 2 * (g or 32)
+    W = inputs.weights(6, K, seed=13)
+    codes, s = oracle.quantize_weights_int8(W, g)
+    if g:
+        H = oracle.hadamard(g)
+        v = (W.astype(np.float64).reshape(6, -1, g) @ H.T).reshape(6, -1)
+    else:
+        v = W.astype(np.float64)
+    for n in range(6):
+        err = np.abs(v[n] - codes[n] * np.float64(s[n]))
+        assert err.max() <= 0.5 * s[n] * (1 + 1e-5) + 1e-6 * np.abs(v[n]).max()
+        assert np.abs(codes[n]).max() == 127
+        assert abs(int(codes[n][np.argmax(np.abs(v[n]))])) == 127
+    e = np.zeros((1, 16), np.float32)
+    e[0, 0] = 1.0
+    c1, s1 = oracle.quantize_weights_int8(e, 16)
+    assert np.all(c1 == 127) and s1[0] == np.float32(np.float32(0.25) / np.float32(127))
+
+
 def test_zero_rows():
     """A zero row has scale 0 and codes 0 (no division by zero)."""
     x = np.zeros((2, 64), np.uint16)
