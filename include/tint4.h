@@ -176,6 +176,33 @@ tint4_status convrot_w4a8_linear_noalloc(const tint4_bf16* x, const uint8_t* w_p
                                          void* stream);
 
 /*
+ * W8A8 ("ComfyUI-INT-Crush", "Inference > INT8": int8 weights times int8
+ * activations with int32 accumulation; the rotation and per-row scales are
+ * those of the int4 path).
+ *   - tint4_quantize_weights_int8: W fp32 [N, K] -> rotated (group 0 / 16 /
+ *     64 / 256 along K) -> w_int8 [N, K] codes in [-127, 127], row_scale fp32
+ *     [N] = absmax / 127 (offline, like tint4_pack_weights; same rules).
+ *   - w8a8_gemm: codes int8 [M, K] (convrot_quantize_act, bits 8), tok_scale
+ *     fp32 [M], w_int8 [N, K], row_scale [N], bias bf16 [N] or NULL ->
+ *     y bf16 [M, N] = bf16(acc * s_tok * s_row (+ bias)), acc exact int32.
+ *     One tensor-core launch at every M (no streaming kernel for small M).
+ *   - convrot_w8a8_linear: rotate + quantize x bf16 [M, K] into the workspace
+ *     (convrot_linear_workspace_size(M, K, 8) bytes, 256-byte aligned), then
+ *     w8a8_gemm.
+ * Shape rules as w4a8_gemm / convrot_w4a8_linear (N % 16 == 0, K % 32 == 0,
+ * K % group == 0); errors as there.
+ */
+tint4_status tint4_quantize_weights_int8(const float* W, int N, int K, int group,
+                                         int8_t* w_int8, float* row_scale, void* stream);
+tint4_status w8a8_gemm(const int8_t* codes, const float* tok_scale, const int8_t* w_int8,
+                       const float* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
+                       int N, int K, void* stream);
+tint4_status convrot_w8a8_linear(const tint4_bf16* x, const int8_t* w_int8,
+                                 const float* row_scale, const tint4_bf16* bias, tint4_bf16* y,
+                                 int M, int N, int K, int group, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/*
  * Grouped GEMM: the same activation codes times up to TINT4_MAX_GROUPS
  * weight matrices in one launch ("feat: packed int4 convrot model loading
  * and dispatch", "Summary": the activation rotate + quantize is shared by the

@@ -187,6 +187,59 @@ def convrot_w4a8_linear_noalloc(x, w_packed, row_scale, group, bias=None, y=None
     return y
 
 
+def tint4_quantize_weights_int8(W, group: int, w_int8=None, row_scale=None):
+    """fp32 W [N, K] -> rotated int8 codes [N, K] and fp32 row scales [N] (W8A8)."""
+    _need(W, "W", torch.float32)
+    N, K = W.shape
+    if w_int8 is None:
+        w_int8 = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    if row_scale is None:
+        row_scale = torch.empty((N,), dtype=torch.float32, device=W.device)
+    _need(w_int8, "w_int8", torch.int8, (N, K))
+    _need(row_scale, "row_scale", torch.float32, (N,))
+    _native.call("tint4_quantize_weights_int8", _ptr(W), N, K, group, _ptr(w_int8),
+                 _ptr(row_scale), _stream(W.device))
+    return w_int8, row_scale
+
+
+def w8a8_gemm(a, tok_scale, w_int8, row_scale, bias=None, y=None) -> torch.Tensor:
+    """int8 codes a [M, K] x int8 W [N, K] -> bf16 y [M, N]."""
+    _need(a, "a", torch.int8)
+    M, K = a.shape
+    N = w_int8.shape[0]
+    _need(tok_scale, "tok_scale", torch.float32, (M,))
+    _need(w_int8, "w_int8", torch.int8, (N, K))
+    _need(row_scale, "row_scale", torch.float32, (N,))
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, (N,))
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    _need(y, "y", torch.bfloat16, (M, N))
+    _native.call("w8a8_gemm", _ptr(a), _ptr(tok_scale), _ptr(w_int8), _ptr(row_scale),
+                 _ptr(bias), _ptr(y), M, N, K, _stream(a.device))
+    return y
+
+
+def convrot_w8a8_linear(x, w_int8, row_scale, group, bias=None, y=None, workspace=None):
+    """Fused rotate + int8 quantize + W8A8 GEMM: bf16 x [M, K] -> bf16 y [M, N]."""
+    _need(x, "x", torch.bfloat16)
+    M, K = x.shape
+    N = w_int8.shape[0]
+    _need(w_int8, "w_int8", torch.int8, (N, K))
+    _need(row_scale, "row_scale", torch.float32, (N,))
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, (N,))
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(y, "y", torch.bfloat16, (M, N))
+    need = convrot_linear_workspace_size(M, K, 8)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    _native.call("convrot_w8a8_linear", _ptr(x), _ptr(w_int8), _ptr(row_scale), _ptr(bias),
+                 _ptr(y), M, N, K, group, _ptr(workspace), workspace.numel(), _stream(x.device))
+    return y
+
+
 def _groups(M, K, device, groups):
     """(w_packed, row_scale, bias or None, y or None) tuples -> ctypes array, ys."""
     if not 1 <= len(groups) <= _native.MAX_GROUPS:

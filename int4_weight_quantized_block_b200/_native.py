@@ -49,6 +49,9 @@ SIGNATURES = {
     "convrot_w4a8_linear_noalloc": (I, [P, P, P, P, P, I, I, I, I, P]),
     "w4a16_gemv_gemm": (I, [P, P, P, P, I, P, I, I, I, P]),
     "w4a8_gemm_grouped": (I, [P, P, P, I, I, I, P]),
+    "tint4_quantize_weights_int8": (I, [P, I, I, I, P, P, P]),
+    "w8a8_gemm": (I, [P, P, P, P, P, P, I, I, I, P]),
+    "convrot_w8a8_linear": (I, [P, P, P, P, P, I, I, I, I, P, SZ, P]),
     "convrot_w4a8_linear_grouped": (I, [P, P, I, I, I, I, P, SZ, P]),
     "tint4_debug_int32_gemm": (I, [P, I, P, P, I, I, I, P]),
     "tint4_debug_bounded_wait": (I, [U64, P]),

@@ -68,6 +68,9 @@ constexpr int kTmOutBytes = kTmBN * kTmBM * 2;        // 48 KB bf16 staging tile
 constexpr int kTmActPBytes = kTmBN * kTmBK / 2;       // 12 KB packed int4 activation codes per stage
 constexpr int kTmSmemBytes = kTmStages * (kTmActBytes + kTmWBytes) + kTmOutBytes + 256 + 1024;
 constexpr int kTmSmemBytesA4 = kTmSmemBytes + kTmStages * kTmActPBytes;
+constexpr int kTmW8Bytes = kTmBM * kTmBK;             // 16 KB int8 weights per stage (W8A8)
+constexpr int kTmSmemBytesW8 = kTmStages * (kTmActBytes + kTmW8Bytes) + kTmOutBytes + 256 + 1024;
+static_assert(kTmSmemBytesW8 <= 227 * 1024, "shared memory budget");
 constexpr uint32_t kTmColD = 0;                       // accumulator buffer b at b * kTmBN
 constexpr uint32_t kTmColA = 2 * kTmBN;               // A stage s at kTmColA + 32 s
 static_assert(kTmColA + 32 * kTmStages <= 512, "TMEM budget");
@@ -109,17 +112,22 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     return ok != 0;
 }
 
-template <bool OUT_I32, bool A_INT4>
+// W8: the weights are int8 codes already (W8A8): the TMA brings a 128 x 128
+// int8 tile (128-byte swizzle) and the MMA reads it from shared memory as its
+// A operand (kind::i8, both operands in shared memory); no unpack, no x16.
+template <bool OUT_I32, bool A_INT4, bool W8 = false>
 __global__ void __launch_bounds__(kTmThreads, 1)
 w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                       const __grid_constant__ TmGroups grp,
                       const float* __restrict__ tok_scale, int M, int K, uint64_t wait_ns) {
+    static_assert(!(W8 && A_INT4), "int8 weights run with int8 activation codes");
+    constexpr int kWB = W8 ? kTmW8Bytes : kTmWBytes;   // weight bytes per stage
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* sAct = smem;
     uint8_t* sW = smem + kTmStages * kTmActBytes;
-    uint8_t* sActP = sW + kTmStages * kTmWBytes;                       // A_INT4 only
+    uint8_t* sActP = sW + kTmStages * kWB;                             // A_INT4 only
     uint8_t* sOut = sActP + (A_INT4 ? kTmStages * kTmActPBytes : 0);
     uint64_t* act_full = reinterpret_cast<uint64_t*>(sOut + kTmOutBytes);
     uint64_t* a_full = act_full + kTmStages;       // TMEM A stage written (one arrival per warp)
@@ -199,10 +207,10 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                         mbar_arrive_expect_tx(&act_full[s], kTmActPBytes + kTmWBytes);
                         tma_load_2d(&tmap_act, &act_full[s], sActP + s * kTmActPBytes, kt * (kTmBK / 2), m0);
                     } else {
-                        mbar_arrive_expect_tx(&act_full[s], kTmActBytes + kTmWBytes);
+                        mbar_arrive_expect_tx(&act_full[s], kTmActBytes + kWB);
                         tma_load_2d(&tmap_act, &act_full[s], sAct + s * kTmActBytes, kt * kTmBK, m0);
                     }
-                    tma_load_2d(tmap_w, &act_full[s], sW + s * kTmWBytes, kt * (kTmBK / 2), n0);
+                    tma_load_2d(tmap_w, &act_full[s], sW + s * kWB, kt * (W8 ? kTmBK : kTmBK / 2), n0);
                     ++issued;
                 }
             }
@@ -222,6 +230,7 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             // MMA kk of a stage 32 bytes = 2 units further (the address field
             // cannot carry: shared addresses are below 2^18)
             const uint64_t bdesc0 = umma_desc_sw128(smem_u32(sAct));
+            const uint64_t adesc0 = umma_desc_sw128(smem_u32(sW));   // W8 only
             int s = 0;
             uint32_t ph = 0u;
             bool ok = true;
@@ -238,8 +247,9 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                 for (int kt = 0; kt < KT; ++kt) {
                     // a_full implies the stage has landed: the unpack warps arrive
                     // on it only after they have seen it (one wait per stage: the
-                    // issuing thread's time per stage is the tensor pipe's budget)
-                    if (!mbar_wait_bounded(&a_full[s], ph, abort_flag, wait_ns,
+                    // issuing thread's time per stage is the tensor pipe's budget);
+                    // int8 weights need no unpack: the landing itself
+                    if (!mbar_wait_bounded(W8 ? &act_full[s] : &a_full[s], ph, abort_flag, wait_ns,
                                            kDevErrTimeoutConsumer)) {
                         ok = false;
                         break;
@@ -247,9 +257,14 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                     tcgen05_fence_after();
                     const uint32_t a_tmem = tmem_base + kTmColA + 32 * s;
                     const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(s * (kTmActBytes >> 4));
+                    const uint64_t adesc = adesc0 + static_cast<uint64_t>(s * (kTmW8Bytes >> 4));
 #pragma unroll
-                    for (int kk = 0; kk < kTmBK / 32; ++kk)
-                        umma_i8_ts(d_tmem, a_tmem + 8 * kk, bdesc + 2 * kk, idesc, (kt | kk) != 0);
+                    for (int kk = 0; kk < kTmBK / 32; ++kk) {
+                        if constexpr (W8)
+                            umma_i8_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kt | kk) != 0);
+                        else
+                            umma_i8_ts(d_tmem, a_tmem + 8 * kk, bdesc + 2 * kk, idesc, (kt | kk) != 0);
+                    }
                     umma_commit(&empty[s]);
                     if (++s == kTmStages) {
                         s = 0;
@@ -266,55 +281,57 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
         __syncwarp();   // lanes 1-31 park here instead of polling a barrier
     } else if (warp < 10) {
         // ------------------------------------------------ weight unpack -> TMEM (warps 2-9)
-        const int q = warp & 3;                 // TMEM lane quarter
-        const int r = q * 32 + lane;            // weight row within the tile
-        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-        const int total = my_tiles * KT;        // K steps this CTA runs
-        // 64-byte swizzle of the TMA tile: chunk v of row r sits at chunk
-        // v ^ ((r >> 1) & 3); 8 consecutive rows then hit 8 distinct bank groups
-        const int sw = (r >> 1) & 3;
-        for (int j = (warp < 6 ? 0 : 1); j < total; j += 2) {
-            const int s = j % kTmStages;
-            const uint32_t ph = (j / kTmStages) & 1;
-            if (!warp_wait(&act_full[s], ph, abort_flag, wait_ns, kDevErrTimeoutConsumer)) break;
-            const uint8_t* row = sW + s * kTmWBytes + r * 64;
-            uint32_t a[32];
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const uint4 p = lds128(row + 16 * (v ^ sw));
-                const uint32_t w4[4] = {p.x, p.y, p.z, p.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) unpack8_natural(w4[u], a[8 * v + 2 * u], a[8 * v + 2 * u + 1]);
-            }
-            // the TMEM A stage is free: its previous MMAs completed before
-            // the producer refilled this stage (empty[s] -> act_full[s])
-            tcgen05_fence_after();
-            tmem_st_32x32b_x32(tmem_base + lane_base + kTmColA + 32 * s, a);
-            if (A_INT4) {
-                // widen the packed activation codes of this stage into the
-                // swizzled int8 B tile: 192 rows x 8 chunks of 16 codes, 12
-                // chunks per thread of this K-step parity (the B tile's last
-                // readers, the MMAs of 4 stages ago, completed before the
-                // producer refilled the stage)
-                const uint8_t* ap = sActP + s * kTmActPBytes;
-                uint8_t* ab = sAct + s * kTmActBytes;
-                const int tid = q * 32 + lane;
-#pragma unroll 4
-                for (int i = 0; i < kTmBN * 8 / 128; ++i) {
-                    const int c = tid + 128 * i;
-                    const int rr = c >> 3, k = c & 7;
-                    const uint2 pk = *reinterpret_cast<const uint2*>(ap + rr * 64 + 8 * k);
-                    uint4 o;
-                    unpack8_natural(pk.x, o.x, o.y);
-                    unpack8_natural(pk.y, o.z, o.w);
-                    sts128(ab + rr * 128 + ((k ^ (rr & 7)) << 4), o);
+        if constexpr (!W8) {   // int8 weights: nothing to widen
+            const int q = warp & 3;                 // TMEM lane quarter
+            const int r = q * 32 + lane;            // weight row within the tile
+            const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+            const int total = my_tiles * KT;        // K steps this CTA runs
+            // 64-byte swizzle of the TMA tile: chunk v of row r sits at chunk
+            // v ^ ((r >> 1) & 3); 8 consecutive rows then hit 8 distinct bank groups
+            const int sw = (r >> 1) & 3;
+            for (int j = (warp < 6 ? 0 : 1); j < total; j += 2) {
+                const int s = j % kTmStages;
+                const uint32_t ph = (j / kTmStages) & 1;
+                if (!warp_wait(&act_full[s], ph, abort_flag, wait_ns, kDevErrTimeoutConsumer)) break;
+                const uint8_t* row = sW + s * kTmWBytes + r * 64;
+                uint32_t a[32];
+    #pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const uint4 p = lds128(row + 16 * (v ^ sw));
+                    const uint32_t w4[4] = {p.x, p.y, p.z, p.w};
+    #pragma unroll
+                    for (int u = 0; u < 4; ++u) unpack8_natural(w4[u], a[8 * v + 2 * u], a[8 * v + 2 * u + 1]);
                 }
-                fence_proxy_async_smem();   // generic-proxy writes -> tensor-core reads
+                // the TMEM A stage is free: its previous MMAs completed before
+                // the producer refilled this stage (empty[s] -> act_full[s])
+                tcgen05_fence_after();
+                tmem_st_32x32b_x32(tmem_base + lane_base + kTmColA + 32 * s, a);
+                if (A_INT4) {
+                    // widen the packed activation codes of this stage into the
+                    // swizzled int8 B tile: 192 rows x 8 chunks of 16 codes, 12
+                    // chunks per thread of this K-step parity (the B tile's last
+                    // readers, the MMAs of 4 stages ago, completed before the
+                    // producer refilled the stage)
+                    const uint8_t* ap = sActP + s * kTmActPBytes;
+                    uint8_t* ab = sAct + s * kTmActBytes;
+                    const int tid = q * 32 + lane;
+    #pragma unroll 4
+                    for (int i = 0; i < kTmBN * 8 / 128; ++i) {
+                        const int c = tid + 128 * i;
+                        const int rr = c >> 3, k = c & 7;
+                        const uint2 pk = *reinterpret_cast<const uint2*>(ap + rr * 64 + 8 * k);
+                        uint4 o;
+                        unpack8_natural(pk.x, o.x, o.y);
+                        unpack8_natural(pk.y, o.z, o.w);
+                        sts128(ab + rr * 128 + ((k ^ (rr & 7)) << 4), o);
+                    }
+                    fence_proxy_async_smem();   // generic-proxy writes -> tensor-core reads
+                }
+                tmem_st_wait();
+                tcgen05_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&a_full[s]);
             }
-            tmem_st_wait();
-            tcgen05_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&a_full[s]);
         }
     } else if (warp < 18) {
         // ------------------------------------------------ epilogue (warps 10-17)
@@ -347,8 +364,8 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             const bool row_ok = n < N;
             // (16 acc) * s_tok * (s_row / 16) equals acc * s_tok * s_row in fp32:
             // scaling by a power of two commutes with the rounding (256 for A_INT4)
-            constexpr float kUnscale = A_INT4 ? 1.0f / 256.0f : 0.0625f;
-            constexpr int kShift = A_INT4 ? 8 : 4;
+            constexpr float kUnscale = A_INT4 ? 1.0f / 256.0f : (W8 ? 1.0f : 0.0625f);
+            constexpr int kShift = A_INT4 ? 8 : (W8 ? 0 : 4);
             const float sr16 = (row_ok && !OUT_I32) ? __ldg(row_scale + n) * kUnscale : 0.0f;
             const float b = (row_ok && !OUT_I32 && bias != nullptr) ? __bfloat162float(bias[n]) : 0.0f;
 #pragma unroll 1

@@ -214,20 +214,22 @@ cudaLaunchAttribute pdl_attr() {
 // packed int4 widened in shared memory (A_INT4).  `grp` holds 1 to
 // kTmMaxGroups weight matrices sharing the activation codes (the tensor maps
 // and the tile list are filled in here).
-template <bool OUT_I32, bool A_INT4>
+template <bool OUT_I32, bool A_INT4, bool W8 = false>
 tint4_status launch_gemm_tmem(const void* a, const float* st, TmGroups& grp,
                               const uint8_t* const* w, int M, int K, cudaStream_t stream,
                               bool pdl) {
-    auto kern = w4a8_tmem_gemm_kernel<OUT_I32, A_INT4>;
-    constexpr int smem_bytes = A_INT4 ? kTmSmemBytesA4 : kTmSmemBytes;
+    auto kern = w4a8_tmem_gemm_kernel<OUT_I32, A_INT4, W8>;
+    constexpr int smem_bytes = A_INT4 ? kTmSmemBytesA4 : (W8 ? kTmSmemBytesW8 : kTmSmemBytes);
     CUtensorMap ta;
     bool ok = A_INT4 ? make_map_u8(&ta, a, K / 2, M, K / 2, kTmBK / 2, kTmBN, CU_TENSOR_MAP_SWIZZLE_NONE)
                      : make_map_u8(&ta, a, K, M, K, kTmBK, kTmBN, CU_TENSOR_MAP_SWIZZLE_128B);
     const int m_tiles = (M + kTmBN - 1) / kTmBN;
     int tiles = 0;
     for (int g = 0; g < grp.count; ++g) {
-        ok = ok && make_map_u8(&grp.w[g], w[g], K / 2, grp.N[g], K / 2, kTmBK / 2, kTmBM,
-                               CU_TENSOR_MAP_SWIZZLE_64B);
+        ok = ok && (W8 ? make_map_u8(&grp.w[g], w[g], K, grp.N[g], K, kTmBK, kTmBM,
+                                     CU_TENSOR_MAP_SWIZZLE_128B)
+                       : make_map_u8(&grp.w[g], w[g], K / 2, grp.N[g], K / 2, kTmBK / 2, kTmBM,
+                                     CU_TENSOR_MAP_SWIZZLE_64B));
         tiles += m_tiles * ((grp.N[g] + kTmBM - 1) / kTmBM);
         grp.tile_end[g] = tiles;
     }
@@ -617,6 +619,20 @@ tint4_status launch_gemm_grouped(const int8_t* codes, const float* tok_scale,
     return launch_gemm_tmem<false, false>(codes, tok_scale, grp, w, M, K, st, pdl);
 }
 
+// W8A8: int8 codes x int8 weights, one tensor-core launch at every M.
+tint4_status launch_w8a8(const int8_t* codes, const float* st, const int8_t* w, const float* sr,
+                         const __nv_bfloat16* bias, __nv_bfloat16* y, int M, int N, int K,
+                         cudaStream_t stream, bool pdl) {
+    TmGroups grp{};
+    grp.row_scale[0] = sr;
+    grp.bias[0] = bias;
+    grp.out[0] = y;
+    grp.N[0] = N;
+    grp.count = 1;
+    const uint8_t* wp = reinterpret_cast<const uint8_t*>(w);
+    return launch_gemm_tmem<false, false, true>(codes, st, grp, &wp, M, K, stream, pdl);
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -738,6 +754,63 @@ tint4_status convrot_w4a8_linear_grouped(const tint4_bf16* x,
                                            codes, tok_scale, st);
     if ((s = last_launch_status()) != TINT4_OK) return s;
     return launch_gemm_grouped(codes, tok_scale, groups, num_groups, M, K, st, true);
+}
+
+tint4_status tint4_quantize_weights_int8(const float* W, int N, int K, int group,
+                                         int8_t* w_int8, float* row_scale, void* stream) {
+    tint4_status s = check_rq_shape(N, K, group);
+    if (s != TINT4_OK) return s;
+    if (N > 0 && (!W || !w_int8 || !row_scale)) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(w_int8) || !aligned16(row_scale)) return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (N == 0) return TINT4_OK;
+    launch_rq_g<float, 127, false>(W, N, K, group, w_int8, row_scale, as_stream(stream));
+    return last_launch_status();
+}
+
+tint4_status w8a8_gemm(const int8_t* codes, const float* tok_scale, const int8_t* w_int8,
+                       const float* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
+                       int N, int K, void* stream) {
+    tint4_status s = check_mnk(M, N, K);
+    if (s != TINT4_OK) return s;
+    if (M > 0 && (!codes || !tok_scale || !w_int8 || !row_scale || !y))
+        return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(codes) || !aligned16(tok_scale) || !aligned16(w_int8) ||
+        !aligned16(row_scale) || !aligned16(y) || !aligned16(bias))
+        return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (M == 0) return TINT4_OK;
+    return launch_w8a8(codes, tok_scale, w_int8, row_scale,
+                       reinterpret_cast<const __nv_bfloat16*>(bias),
+                       reinterpret_cast<__nv_bfloat16*>(y), M, N, K, as_stream(stream), false);
+}
+
+tint4_status convrot_w8a8_linear(const tint4_bf16* x, const int8_t* w_int8,
+                                 const float* row_scale, const tint4_bf16* bias, tint4_bf16* y,
+                                 int M, int N, int K, int group, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    tint4_status s = check_mnk(M, N, K);
+    if (s != TINT4_OK) return s;
+    if ((s = check_rq_shape(M, K, group)) != TINT4_OK) return s;
+    if (M > 0 && (!x || !w_int8 || !row_scale || !y)) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_int8) || !aligned16(row_scale) || !aligned16(y) ||
+        !aligned16(bias))
+        return TINT4_ERR_MISALIGNED;
+    if (M > 0 && (!workspace || workspace_bytes < convrot_linear_workspace_size(M, K, 8)))
+        return TINT4_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (M == 0) return TINT4_OK;
+    int8_t* codes = static_cast<int8_t*>(workspace);
+    float* tok_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                                align_up(static_cast<size_t>(M) * K, 256));
+    cudaStream_t st = as_stream(stream);
+    launch_rq_g<__nv_bfloat16, 127, false>(reinterpret_cast<const __nv_bfloat16*>(x), M, K, group,
+                                           codes, tok_scale, st);
+    if ((s = last_launch_status()) != TINT4_OK) return s;
+    return launch_w8a8(codes, tok_scale, w_int8, row_scale,
+                       reinterpret_cast<const __nv_bfloat16*>(bias),
+                       reinterpret_cast<__nv_bfloat16*>(y), M, N, K, st, true);
 }
 
 tint4_status convrot_w4a8_linear_noalloc(const tint4_bf16* x, const uint8_t* w_packed,

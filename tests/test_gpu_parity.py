@@ -299,6 +299,53 @@ def test_full_size_workloads_sampled(name):
     assert np.array_equal(acc_gpu.cpu().numpy()[pairs[:, 0], pairs[:, 1]], acc)
 
 
+# ------------------------------------------------------------------ W8A8
+
+@pytest.mark.parametrize("N,K,g", [(16, 32, 0), (272, 320, 64), (256, 4096, 256), (48, 352, 16)])
+def test_quantize_weights_int8_bit_exact(N, K, g):
+    W = inputs.weights(N, K, seed=150 + K)
+    W[2, :] = 0.0
+    c_ref, s_ref = oracle.quantize_weights_int8(W, g)
+    c, s = t4.tint4_quantize_weights_int8(to_gpu(W), g)
+    torch.cuda.synchronize()
+    assert np.array_equal(c.cpu().numpy(), c_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("M,N,K,g", [(1, 256, 256, 256), (17, 272, 320, 64), (200, 1040, 1024, 16),
+                                     (385, 128, 4096, 256)])
+def test_w8a8_gemm_and_linear(M, N, K, g):
+    x = inputs.activations(M, K, seed=160 + M)
+    wc, sr = oracle.quantize_weights_int8(inputs.weights(N, K, seed=161 + N), g)
+    codes, st, _ = oracle.quantize_act(x, g, 8)
+    b = inputs.f32_to_bf16_bits(np.linspace(-1, 1, N, dtype=np.float32))
+    y = t4.w8a8_gemm(to_gpu(codes), to_gpu(st), to_gpu(wc), to_gpu(sr), bf16_to_gpu(b))
+    yl = t4.convrot_w8a8_linear(bf16_to_gpu(x), to_gpu(wc), to_gpu(sr), g)
+    torch.cuda.synchronize()
+    acc = oracle.gemm_i32(codes, wc)
+    assert_gemm_output(bf16_from_gpu(y), oracle.epilogue_f64(acc, st, sr, b), b)
+    assert_gemm_output(bf16_from_gpu(yl), oracle.epilogue_f64(acc, st, sr))
+
+
+def test_w8a8_full_size_sampled():
+    """The DiT QKV layer as W8A8: all weight codes and scales bit-exact, the
+    output on sampled (m, n) pairs against the oracle."""
+    w = inputs.WORKLOADS["dit_qkv_w4a8"]
+    M, N, K, g = w["M"], w["N"], w["K"], w["group"]
+    x, W = inputs.layer_inputs("dit_qkv_w4a8")
+    wc_ref, sr_ref = oracle.quantize_weights_int8(W, g)
+    wc, sr = t4.tint4_quantize_weights_int8(to_gpu(W), g)
+    y = t4.convrot_w8a8_linear(bf16_to_gpu(x), wc, sr, g)
+    torch.cuda.synchronize()
+    assert np.array_equal(wc.cpu().numpy(), wc_ref)
+    assert np.array_equal(sr.cpu().numpy().view(np.uint32), sr_ref.view(np.uint32))
+    qa_ref, st_ref, _ = oracle.quantize_act(x, g, 8)
+    pairs = _sample_pairs(M, N, 4096, seed=19)
+    acc = oracle.gemm_i32_sampled(qa_ref, wc_ref, pairs)
+    y_ref = oracle.epilogue_sampled_f64(acc, st_ref, sr_ref, pairs)
+    assert_gemm_output(bf16_from_gpu(y)[pairs[:, 0], pairs[:, 1]], y_ref)
+
+
 # ------------------------------------------------------------------ grouped GEMM
 
 @pytest.mark.parametrize("M", [8, 200])
