@@ -60,17 +60,31 @@ namespace tint4 {
 constexpr int kTmBM = 128;       // weight rows per tile (UMMA M, TMEM lanes)
 constexpr int kTmBN = 192;       // tokens per tile (UMMA N)
 constexpr int kTmBK = 128;       // K values per stage
-constexpr int kTmStages = 4;     // activation smem stages = TMEM A stages
+constexpr int kTmStages = 4;     // TMEM A stages (and shared-memory stages of the A_INT4 / W8 forms)
+// Shared-memory stages: 5 for int8 codes x packed weights, so that the loads
+// run one stage further ahead of the unpack than the 4 TMEM A stages allow
+// (the unpack of step j also waits for the MMAs of step j - 4, which free its
+// TMEM stage); the packed-int4-code and int8-weight forms have no room for a
+// fifth stage.
+template <bool A_INT4, bool W8>
+struct TmRing {
+    static constexpr int S = (A_INT4 || W8) ? 4 : 5;
+};
 constexpr int kTmThreads = 576;  // 18 warps
 constexpr int kTmActBytes = kTmBN * kTmBK;            // 24 KB per stage
 constexpr int kTmWBytes = kTmBM * kTmBK / 2;          // 8 KB packed weights per stage
 constexpr int kTmOutBytes = kTmBN * kTmBM * 2;        // 48 KB bf16 staging tile
 constexpr int kTmActPBytes = kTmBN * kTmBK / 2;       // 12 KB packed int4 activation codes per stage
-constexpr int kTmSmemBytes = kTmStages * (kTmActBytes + kTmWBytes) + kTmOutBytes + 256 + 1024;
-constexpr int kTmSmemBytesA4 = kTmSmemBytes + kTmStages * kTmActPBytes;
+constexpr int kTmSmemBytes =
+    TmRing<false, false>::S * (kTmActBytes + kTmWBytes) + kTmOutBytes + 256 + 1024;
+constexpr int kTmSmemBytesA4 =
+    TmRing<true, false>::S * (kTmActBytes + kTmWBytes + kTmActPBytes) + kTmOutBytes + 256 + 1024;
 constexpr int kTmW8Bytes = kTmBM * kTmBK;             // 16 KB int8 weights per stage (W8A8)
-constexpr int kTmSmemBytesW8 = kTmStages * (kTmActBytes + kTmW8Bytes) + kTmOutBytes + 256 + 1024;
-static_assert(kTmSmemBytesW8 <= 227 * 1024, "shared memory budget");
+constexpr int kTmSmemBytesW8 =
+    TmRing<false, true>::S * (kTmActBytes + kTmW8Bytes) + kTmOutBytes + 256 + 1024;
+static_assert(kTmSmemBytes <= 227 * 1024 && kTmSmemBytesA4 <= 227 * 1024 &&
+                  kTmSmemBytesW8 <= 227 * 1024,
+              "shared memory budget");
 constexpr uint32_t kTmColD = 0;                       // accumulator buffer b at b * kTmBN
 constexpr uint32_t kTmColA = 2 * kTmBN;               // A stage s at kTmColA + 32 s
 static_assert(kTmColA + 32 * kTmStages <= 512, "TMEM budget");
@@ -101,6 +115,41 @@ __device__ __forceinline__ void umma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uin
         : "memory");
 }
 
+// The four K-32 MMAs of one 128-wide K step in one asm block: one predicate
+// for the step's first MMA (overwrite at the start of a tile), the others
+// accumulate; fewer instructions on the issuing thread, whose time per step
+// paces the tensor pipe.  TS: A from TMEM columns a, a+8, a+16, a+24.
+__device__ __forceinline__ void umma_i8_ts_step(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 q, %4, %4;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%5], %6, %3, q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%7], %8, %3, q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%9], %10, %3, q;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(a_tmem + 8), "l"(b_desc + 2),
+        "r"(a_tmem + 16), "l"(b_desc + 4), "r"(a_tmem + 24), "l"(b_desc + 6)
+        : "memory");
+}
+
+// SS: A from shared memory (descriptor advancing 32 bytes = 2 units per MMA)
+__device__ __forceinline__ void umma_i8_ss_step(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 q, %4, %4;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %5, %6, %3, q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %7, %8, %3, q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %9, %10, %3, q;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "l"(a_desc + 2), "l"(b_desc + 2),
+        "l"(a_desc + 4), "l"(b_desc + 4), "l"(a_desc + 6), "l"(b_desc + 6)
+        : "memory");
+}
+
 // Bounded wait by lane 0 of the warp, result broadcast: the warp leaves
 // together (tcgen05.st / tcgen05.ld are warp-collective).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
@@ -122,17 +171,19 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                       const float* __restrict__ tok_scale, int M, int K, uint64_t wait_ns) {
     static_assert(!(W8 && A_INT4), "int8 weights run with int8 activation codes");
     constexpr int kWB = W8 ? kTmW8Bytes : kTmWBytes;   // weight bytes per stage
+    constexpr int kS = TmRing<A_INT4, W8>::S;           // shared-memory stages
+    constexpr int kT = kTmStages;                       // TMEM A stages
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* sAct = smem;
-    uint8_t* sW = smem + kTmStages * kTmActBytes;
-    uint8_t* sActP = sW + kTmStages * kWB;                             // A_INT4 only
-    uint8_t* sOut = sActP + (A_INT4 ? kTmStages * kTmActPBytes : 0);
+    uint8_t* sW = smem + kS * kTmActBytes;
+    uint8_t* sActP = sW + kS * kWB;                                    // A_INT4 only
+    uint8_t* sOut = sActP + (A_INT4 ? kS * kTmActPBytes : 0);
     uint64_t* act_full = reinterpret_cast<uint64_t*>(sOut + kTmOutBytes);
-    uint64_t* a_full = act_full + kTmStages;       // TMEM A stage written (one arrival per warp)
-    uint64_t* empty = a_full + kTmStages;          // stage consumed by the MMAs (commit)
-    uint64_t* acc_full = empty + kTmStages;        // [2] accumulator ready (commit)
+    uint64_t* empty = act_full + kS;               // [kS] stage consumed by the MMAs (commit)
+    uint64_t* a_full = empty + kS;                 // [kT] TMEM A stage written (one arrival per warp)
+    uint64_t* acc_full = a_full + kT;              // [2] accumulator ready (commit)
     uint64_t* acc_empty = acc_full + 2;            // [2] accumulator drained (8 warp arrivals)
     uint64_t* final_bar = acc_empty + 2;           // all MMAs done (teardown)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
@@ -159,11 +210,11 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
     };
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kTmStages; ++s) {
+        for (int s = 0; s < kS; ++s) {
             mbar_init(&act_full[s], 1);
-            mbar_init(&a_full[s], 4);
             mbar_init(&empty[s], 1);
         }
+        for (int t = 0; t < kT; ++t) mbar_init(&a_full[t], 4);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
             mbar_init(&acc_empty[b], 8);
@@ -198,8 +249,8 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                 const int m0 = ta.m0, n0 = ta.n0;
                 const CUtensorMap* tmap_w = &grp.w[ta.g];
                 for (int kt = 0; kt < KT; ++kt, ++c) {
-                    const int s = c % kTmStages;
-                    const uint32_t ph = (c / kTmStages) & 1;
+                    const int s = c % kS;
+                    const uint32_t ph = (c / kS) & 1;
                     if (!mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, wait_ns,
                                            kDevErrTimeoutProducer))
                         break;
@@ -216,9 +267,9 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             }
             if (*abort_flag) {
                 uint32_t never = 0u;
-                const int first = issued > kTmStages ? issued - kTmStages : 0;
+                const int first = issued > kS ? issued - kS : 0;
                 for (int j = first; j < issued; ++j)
-                    (void)mbar_wait_bounded(&act_full[j % kTmStages], (j / kTmStages) & 1, &never,
+                    (void)mbar_wait_bounded(&act_full[j % kS], (j / kS) & 1, &never,
                                             wait_ns, 0u);
             }
         }
@@ -231,8 +282,11 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             // cannot carry: shared addresses are below 2^18)
             const uint64_t bdesc0 = umma_desc_sw128(smem_u32(sAct));
             const uint64_t adesc0 = umma_desc_sw128(smem_u32(sW));   // W8 only
-            int s = 0;
-            uint32_t ph = 0u;
+            static_assert(kTmBK == 4 * 32, "four MMAs per K step");
+            // ring positions, advanced per step: shared-memory stage s (phase
+            // sph) and TMEM stage t (phase tph)
+            int s = 0, t = 0;
+            uint32_t sph = 0u, tph = 0u;
             bool ok = true;
             for (int i = 0; i < my_tiles && ok; ++i) {
                 const int buf = i & 1;
@@ -249,26 +303,29 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                     // on it only after they have seen it (one wait per stage: the
                     // issuing thread's time per stage is the tensor pipe's budget);
                     // int8 weights need no unpack: the landing itself
-                    if (!mbar_wait_bounded(W8 ? &act_full[s] : &a_full[s], ph, abort_flag, wait_ns,
-                                           kDevErrTimeoutConsumer)) {
+                    const bool ready =
+                        W8 ? mbar_wait_bounded(&act_full[s], sph, abort_flag, wait_ns,
+                                               kDevErrTimeoutConsumer)
+                           : mbar_wait_bounded(&a_full[t], tph, abort_flag, wait_ns,
+                                               kDevErrTimeoutConsumer);
+                    if (!ready) {
                         ok = false;
                         break;
                     }
                     tcgen05_fence_after();
-                    const uint32_t a_tmem = tmem_base + kTmColA + 32 * s;
+                    const uint32_t a_tmem = tmem_base + kTmColA + 32 * t;
                     const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(s * (kTmActBytes >> 4));
                     const uint64_t adesc = adesc0 + static_cast<uint64_t>(s * (kTmW8Bytes >> 4));
-#pragma unroll
-                    for (int kk = 0; kk < kTmBK / 32; ++kk) {
-                        if constexpr (W8)
-                            umma_i8_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kt | kk) != 0);
-                        else
-                            umma_i8_ts(d_tmem, a_tmem + 8 * kk, bdesc + 2 * kk, idesc, (kt | kk) != 0);
-                    }
+                    if constexpr (W8) umma_i8_ss_step(d_tmem, adesc, bdesc, idesc, kt);
+                    else umma_i8_ts_step(d_tmem, a_tmem, bdesc, idesc, kt);
                     umma_commit(&empty[s]);
-                    if (++s == kTmStages) {
+                    if (++s == kS) {
                         s = 0;
-                        ph ^= 1u;
+                        sph ^= 1u;
+                    }
+                    if (++t == kT) {
+                        t = 0;
+                        tph ^= 1u;
                     }
                 }
                 if (ok) umma_commit(&acc_full[buf]);
@@ -290,9 +347,10 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             // v ^ ((r >> 1) & 3); 8 consecutive rows then hit 8 distinct bank groups
             const int sw = (r >> 1) & 3;
             for (int j = (warp < 6 ? 0 : 1); j < total; j += 2) {
-                const int s = j % kTmStages;
-                const uint32_t ph = (j / kTmStages) & 1;
-                if (!warp_wait(&act_full[s], ph, abort_flag, wait_ns, kDevErrTimeoutConsumer)) break;
+                const int s = j % kS, t = j % kT;
+                if (!warp_wait(&act_full[s], (j / kS) & 1, abort_flag, wait_ns,
+                               kDevErrTimeoutConsumer))
+                    break;
                 const uint8_t* row = sW + s * kTmWBytes + r * 64;
                 uint32_t a[32];
     #pragma unroll
@@ -302,10 +360,16 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
     #pragma unroll
                     for (int u = 0; u < 4; ++u) unpack8_natural(w4[u], a[8 * v + 2 * u], a[8 * v + 2 * u + 1]);
                 }
-                // the TMEM A stage is free: its previous MMAs completed before
-                // the producer refilled this stage (empty[s] -> act_full[s])
+                // the TMEM A stage t is free once the MMAs of step j - kT have
+                // completed; with as many shared-memory stages as TMEM stages the
+                // producer already waited for exactly that before this stage
+                // landed
+                if (kS != kT && j >= kT &&
+                    !warp_wait(&empty[(j - kT) % kS], ((j - kT) / kS) & 1, abort_flag, wait_ns,
+                               kDevErrTimeoutConsumer))
+                    break;
                 tcgen05_fence_after();
-                tmem_st_32x32b_x32(tmem_base + lane_base + kTmColA + 32 * s, a);
+                tmem_st_32x32b_x32(tmem_base + lane_base + kTmColA + 32 * t, a);
                 if (A_INT4) {
                     // widen the packed activation codes of this stage into the
                     // swizzled int8 B tile: 192 rows x 8 chunks of 16 codes, 12
@@ -330,7 +394,7 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                 tmem_st_wait();
                 tcgen05_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&a_full[s]);
+                if (lane == 0) mbar_arrive(&a_full[t]);
             }
         }
     } else if (warp < 18) {
