@@ -388,6 +388,30 @@ def bench_rows(args, t4, inputs, dev, flush, pk, int8_peak):
     rows["dit_mlp_up_w4a8"] = gemm_layer("dit_mlp_up_w4a8")
     rows["dit_mlp_down_w4a8"] = gemm_layer("dit_mlp_down_w4a8")
 
+    # the QKV layer with int8 weights (W8A8): the GEMM alone and the fused linear
+    w = inputs.WORKLOADS["dit_qkv_w4a8"]
+    M, N, K, g = w["M"], w["N"], w["K"], w["group"]
+    x_np, W_np = inputs.layer_inputs("dit_qkv_w4a8")
+    x = bf16_gpu(x_np, dev)
+    wc, sr = t4.tint4_quantize_weights_int8(torch.from_numpy(W_np).to(dev), g)
+    del W_np
+    codes, st = t4.convrot_quantize_act(x, g, 8)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(t4.convrot_linear_workspace_size(M, K, 8), dtype=torch.uint8, device=dev)
+    t4.w8a8_gemm(codes, st, wc, sr, None, y)
+    t4.convrot_w8a8_linear(x, wc, sr, g, None, y, ws)
+    torch.cuda.synchronize(dev)
+    g_ms = statistics.median(time_steps(lambda: t4.w8a8_gemm(codes, st, wc, sr, None, y), reps, flush, dev))
+    l_ms = statistics.median(time_steps(lambda: t4.convrot_w8a8_linear(x, wc, sr, g, None, y, ws),
+                                        reps, flush, dev))
+    ops = 2.0 * M * N * K
+    rows["dit_qkv_w8a8"] = {
+        "M": M, "N": N, "K": K, "group": g,
+        "gemm_us": round(g_ms * 1e3, 2), "gemm_TOPS": round(ops / g_ms / 1e9, 2),
+        "gemm_frac_int8": round(ops / g_ms / 1e9 / int8_peak, 4),
+        "linear_us": round(l_ms * 1e3, 2), "linear_TOPS": round(ops / l_ms / 1e9, 2)}
+    del wc, sr, codes, st, y, ws, x
+
     # the QKV layer as three separate 3072-row weight matrices (Q, K, V of one
     # input): three GEMM launches against one grouped launch
     w = inputs.WORKLOADS["dit_qkv_w4a8"]
