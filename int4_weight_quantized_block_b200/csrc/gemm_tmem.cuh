@@ -51,6 +51,16 @@
 // unpack warps also widen it (x16 again, natural K order) into the swizzled
 // int8 B tile before they signal the stage: the accumulators then hold
 // 256 * acc (|256 acc| < 2^31 for K <= 65536 with codes in [-7, 7]).
+//
+// Even/odd K order (EVOD, and always for A_INT4): a packed word holds 8 K
+// values, the even ones in its low nibbles and the odd ones in its high
+// nibbles.  Widened as (w << 4) & 0xF0F0F0F0 and w & 0xF0F0F0F0 it gives
+// the K order 0, 2, 4, 6, 1, 3, 5, 7 in every block of 8 at no extra cost,
+// where the natural order needs two byte permutes more per word.  A dot
+// product over K does not depend on the order as long as both operands use
+// the same one: the fused linears store their int8 activation codes in that
+// order (rotate_quantize_rows with EVOD), and the W4A4 form widens both
+// operands from packed nibbles in the kernel.
 #pragma once
 
 #include "ptx.cuh"
@@ -164,12 +174,15 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 // W8: the weights are int8 codes already (W8A8): the TMA brings a 128 x 128
 // int8 tile (128-byte swizzle) and the MMA reads it from shared memory as its
 // A operand (kind::i8, both operands in shared memory); no unpack, no x16.
-template <bool OUT_I32, bool A_INT4, bool W8 = false>
+// EVOD: the int8 activation codes are stored in the even/odd K order.
+template <bool OUT_I32, bool A_INT4, bool W8 = false, bool EVOD = false>
 __global__ void __launch_bounds__(kTmThreads, 1)
 w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                       const __grid_constant__ TmGroups grp,
                       const float* __restrict__ tok_scale, int M, int K, uint64_t wait_ns) {
     static_assert(!(W8 && A_INT4), "int8 weights run with int8 activation codes");
+    static_assert(!(W8 && EVOD), "int8 weights are stored in the natural K order");
+    constexpr bool kEvod = EVOD || A_INT4;   // widen in the even/odd K order
     constexpr int kWB = W8 ? kTmW8Bytes : kTmWBytes;   // weight bytes per stage
     constexpr int kS = TmRing<A_INT4, W8>::S;           // shared-memory stages
     constexpr int kT = kTmStages;                       // TMEM A stages
@@ -358,7 +371,12 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                     const uint4 p = lds128(row + 16 * (v ^ sw));
                     const uint32_t w4[4] = {p.x, p.y, p.z, p.w};
     #pragma unroll
-                    for (int u = 0; u < 4; ++u) unpack8_natural(w4[u], a[8 * v + 2 * u], a[8 * v + 2 * u + 1]);
+                    for (int u = 0; u < 4; ++u) {
+                        if constexpr (kEvod)
+                            unpack8_evod(w4[u], a[8 * v + 2 * u], a[8 * v + 2 * u + 1]);
+                        else
+                            unpack8_natural(w4[u], a[8 * v + 2 * u], a[8 * v + 2 * u + 1]);
+                    }
                 }
                 // the TMEM A stage t is free once the MMAs of step j - kT have
                 // completed; with as many shared-memory stages as TMEM stages the
@@ -371,8 +389,8 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                 tcgen05_fence_after();
                 tmem_st_32x32b_x32(tmem_base + lane_base + kTmColA + 32 * t, a);
                 if (A_INT4) {
-                    // widen the packed activation codes of this stage into the
-                    // swizzled int8 B tile: 192 rows x 8 chunks of 16 codes, 12
+                    // widen the packed activation codes of this stage (even/odd
+                    // K order, like the weights) into the swizzled int8 B tile: 192 rows x 8 chunks of 16 codes, 12
                     // chunks per thread of this K-step parity (the B tile's last
                     // readers, the MMAs of 4 stages ago, completed before the
                     // producer refilled the stage)
@@ -385,8 +403,8 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                         const int rr = c >> 3, k = c & 7;
                         const uint2 pk = *reinterpret_cast<const uint2*>(ap + rr * 64 + 8 * k);
                         uint4 o;
-                        unpack8_natural(pk.x, o.x, o.y);
-                        unpack8_natural(pk.y, o.z, o.w);
+                        unpack8_evod(pk.x, o.x, o.y);
+                        unpack8_evod(pk.y, o.z, o.w);
                         sts128(ab + rr * 128 + ((k ^ (rr & 7)) << 4), o);
                     }
                     fence_proxy_async_smem();   // generic-proxy writes -> tensor-core reads

@@ -259,6 +259,13 @@ __device__ __forceinline__ void unpack8_natural(uint32_t w, uint32_t& lo, uint32
     hi = __byte_perm(L, H, 0x7362);
 }
 
+// 8 packed nibbles -> 8 int8 values x16 in the even/odd K order
+// (0, 2, 4, 6 | 1, 3, 5, 7): the low nibbles moved up, then the high nibbles
+__device__ __forceinline__ void unpack8_evod(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    lo = (w << 4) & 0xF0F0F0F0u;
+    hi = w & 0xF0F0F0F0u;
+}
+
 // Shared-memory matrix descriptor for a K-major operand stored in the
 // 128-byte swizzled canonical layout: rows of 128 bytes, groups of 8 rows
 // 1024 bytes apart (stride byte offset), 16-byte chunks XOR-swizzled by

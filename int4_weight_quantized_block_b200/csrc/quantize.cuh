@@ -209,7 +209,11 @@ __device__ __forceinline__ void rotate_quantize_rows_to_smem(const __nv_bfloat16
 // flight while it rotates and quantizes the current one.
 // The rows of one CTA.  FULL: the CTA's warps hold exactly K values (every
 // chunk present and complete), so no per-chunk guard is needed.
-template <typename InT, int G, int Q, bool PACKED, int CH, bool FULL>
+// EVOD (int8 codes only): each block of 8 codes is stored with its even
+// positions first (codes 0, 2, 4, 6, 1, 3, 5, 7), the layout whose weights
+// the tensor-core GEMM unpacks without byte permutes; a private layout of the
+// fused linears' workspace (the sums over K are the same numbers).
+template <typename InT, int G, int Q, bool PACKED, int CH, bool FULL, bool EVOD = false>
 __device__ __forceinline__ void rotate_quantize_rows(const InT* __restrict__ in, int rows, int K,
                                                      void* __restrict__ codes,
                                                      float* __restrict__ scales,
@@ -276,7 +280,11 @@ __device__ __forceinline__ void rotate_quantize_rows(const InT* __restrict__ in,
             const uint32_t hi = __byte_perm(__byte_perm(m[4], m[5], 0x0040), __byte_perm(m[6], m[7], 0x0040), 0x5410);
             if (!PACKED) {
                 int8_t* dst = static_cast<int8_t*>(codes) + static_cast<size_t>(row) * K + base;
-                *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
+                if (EVOD)
+                    *reinterpret_cast<uint2*>(dst) =
+                        make_uint2(__byte_perm(lo, hi, 0x6420), __byte_perm(lo, hi, 0x7531));
+                else
+                    *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
             } else {
                 // low nibble = even index, high nibble = odd index: gather the
                 // even-index codes and the odd-index codes, then interleave nibbles
@@ -295,7 +303,7 @@ __device__ __forceinline__ void rotate_quantize_rows(const InT* __restrict__ in,
 // has blockDim.x / 32 warps (K <= warps * CH * 256).  Persistent: CTA b
 // handles rows b, b + gridDim.x, ..., and the loads of its next row are in
 // flight while it rotates and quantizes the current one.
-template <typename InT, int G, int Q, bool PACKED, int CH>
+template <typename InT, int G, int Q, bool PACKED, int CH, bool EVOD = false>
 __global__ void __launch_bounds__(CH == 1 ? 8 * 32 : kQuantMaxWarps * 32)   // one chunk per warp: K <= 2048
 rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K,
                             void* __restrict__ codes, float* __restrict__ scales) {
@@ -305,9 +313,9 @@ rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K,
     // reading the codes.
     grid_launch_dependents();
     if (K == static_cast<int>(blockDim.x / 32) * CH * kQuantChunk)
-        rotate_quantize_rows<InT, G, Q, PACKED, CH, true>(in, rows, K, codes, scales, red);
+        rotate_quantize_rows<InT, G, Q, PACKED, CH, true, EVOD>(in, rows, K, codes, scales, red);
     else
-        rotate_quantize_rows<InT, G, Q, PACKED, CH, false>(in, rows, K, codes, scales, red);
+        rotate_quantize_rows<InT, G, Q, PACKED, CH, false, EVOD>(in, rows, K, codes, scales, red);
 }
 
 }  // namespace tint4

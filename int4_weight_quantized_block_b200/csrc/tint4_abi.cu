@@ -136,10 +136,10 @@ int num_sms(int dev);
 
 // persistent grid: as many CTAs as fit on the GPU at once (per block size,
 // looked up once per device), at most one per row
-template <typename InT, int G, int Q, bool PACKED, int CH>
+template <typename InT, int G, int Q, bool PACKED, int CH, bool EVOD = false>
 void launch_rq_persistent(const InT* in, int rows, int K, void* codes, float* scales, int threads,
                           cudaStream_t st) {
-    auto kern = rotate_quantize_rows_kernel<InT, G, Q, PACKED, CH>;
+    auto kern = rotate_quantize_rows_kernel<InT, G, Q, PACKED, CH, EVOD>;
     int dev = 0;
     cudaGetDevice(&dev);
     static std::atomic<int> per_sm[kMaxDevices][kQuantMaxWarps + 1];
@@ -157,26 +157,26 @@ void launch_rq_persistent(const InT* in, int rows, int K, void* codes, float* sc
     kern<<<grid, threads, 0, st>>>(in, rows, K, codes, scales);
 }
 
-template <typename InT, int G, int Q, bool PACKED>
+template <typename InT, int G, int Q, bool PACKED, bool EVOD = false>
 void launch_rq_ch(const InT* in, int rows, int K, void* codes, float* scales, cudaStream_t st) {
     const int nchunks = (K + kQuantChunk - 1) / kQuantChunk;
     // two chunks per warp once a row has more than 8: the per-row work (the
     // absmax reduction, the scale's division) then spreads over more values
     if (nchunks <= 8)
-        launch_rq_persistent<InT, G, Q, PACKED, 1>(in, rows, K, codes, scales, nchunks * 32, st);
+        launch_rq_persistent<InT, G, Q, PACKED, 1, EVOD>(in, rows, K, codes, scales, nchunks * 32, st);
     else
-        launch_rq_persistent<InT, G, Q, PACKED, 2>(in, rows, K, codes, scales,
+        launch_rq_persistent<InT, G, Q, PACKED, 2, EVOD>(in, rows, K, codes, scales,
                                                    ((nchunks + 1) / 2) * 32, st);
 }
 
-template <typename InT, int Q, bool PACKED>
+template <typename InT, int Q, bool PACKED, bool EVOD = false>
 void launch_rq_g(const InT* in, int rows, int K, int g, void* codes, float* scales,
                  cudaStream_t st) {
     switch (g) {
-        case 0: launch_rq_ch<InT, 0, Q, PACKED>(in, rows, K, codes, scales, st); break;
-        case 16: launch_rq_ch<InT, 16, Q, PACKED>(in, rows, K, codes, scales, st); break;
-        case 64: launch_rq_ch<InT, 64, Q, PACKED>(in, rows, K, codes, scales, st); break;
-        default: launch_rq_ch<InT, 256, Q, PACKED>(in, rows, K, codes, scales, st); break;
+        case 0: launch_rq_ch<InT, 0, Q, PACKED, EVOD>(in, rows, K, codes, scales, st); break;
+        case 16: launch_rq_ch<InT, 16, Q, PACKED, EVOD>(in, rows, K, codes, scales, st); break;
+        case 64: launch_rq_ch<InT, 64, Q, PACKED, EVOD>(in, rows, K, codes, scales, st); break;
+        default: launch_rq_ch<InT, 256, Q, PACKED, EVOD>(in, rows, K, codes, scales, st); break;
     }
 }
 
@@ -214,11 +214,11 @@ cudaLaunchAttribute pdl_attr() {
 // packed int4 widened in shared memory (A_INT4).  `grp` holds 1 to
 // kTmMaxGroups weight matrices sharing the activation codes (the tensor maps
 // and the tile list are filled in here).
-template <bool OUT_I32, bool A_INT4, bool W8 = false>
+template <bool OUT_I32, bool A_INT4, bool W8 = false, bool EVOD = false>
 tint4_status launch_gemm_tmem(const void* a, const float* st, TmGroups& grp,
                               const uint8_t* const* w, int M, int K, cudaStream_t stream,
                               bool pdl) {
-    auto kern = w4a8_tmem_gemm_kernel<OUT_I32, A_INT4, W8>;
+    auto kern = w4a8_tmem_gemm_kernel<OUT_I32, A_INT4, W8, EVOD>;
     constexpr int smem_bytes = A_INT4 ? kTmSmemBytesA4 : (W8 ? kTmSmemBytesW8 : kTmSmemBytes);
     CUtensorMap ta;
     bool ok = A_INT4 ? make_map_u8(&ta, a, K / 2, M, K / 2, kTmBK / 2, kTmBN, CU_TENSOR_MAP_SWIZZLE_NONE)
@@ -365,11 +365,30 @@ tint4_status launch_linear_small_fused_g(const __nv_bfloat16* x, const uint8_t* 
     }
 }
 
+// The fused linears keep their int8 codes in the tensor-core GEMM's
+// even/odd K order whenever that GEMM runs them (past the small-M kernel).
+bool linear_codes_evod(int M) { return M > kS8MaxM; }
+
+// Rotation + int8 codes of x (codes in [-Q, Q]) for a fused linear, in the
+// order linear_codes_evod picks.
+template <int Q>
+void launch_linear_codes(const tint4_bf16* x, int M, int K, int group, void* codes,
+                         float* tok_scale, cudaStream_t st) {
+    const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    if (linear_codes_evod(M))
+        launch_rq_g<__nv_bfloat16, Q, false, true>(xb, M, K, group, codes, tok_scale, st);
+    else
+        launch_rq_g<__nv_bfloat16, Q, false>(xb, M, K, group, codes, tok_scale, st);
+}
+
 // A_INT4: activation codes packed two per byte (else int8, one per byte).
-template <bool A_INT4, bool OUT_I32>
+// EVOD: int8 codes in the even/odd K order (only where linear_codes_evod(M)).
+template <bool A_INT4, bool OUT_I32, bool EVOD = false>
 tint4_status launch_gemm(const void* a, const uint8_t* w, const float* st, const float* sr,
                          const __nv_bfloat16* bias, void* out, int M, int N, int K,
                          cudaStream_t stream, bool pdl) {
+    static_assert(!(EVOD && A_INT4), "packed codes are widened in the kernel");
+    if (EVOD && !linear_codes_evod(M)) return TINT4_ERR_INVALID_ARG;
     if (M <= 8)
         return launch_gemm_small<1, A_INT4, OUT_I32>(a, w, st, sr, bias, out, M, N, K, stream, pdl);
     if (M <= kS8MaxM)
@@ -380,7 +399,7 @@ tint4_status launch_gemm(const void* a, const uint8_t* w, const float* st, const
     grp.out[0] = out;
     grp.N[0] = N;
     grp.count = 1;
-    return launch_gemm_tmem<OUT_I32, A_INT4>(a, st, grp, &w, M, K, stream, pdl);
+    return launch_gemm_tmem<OUT_I32, A_INT4, false, EVOD>(a, st, grp, &w, M, K, stream, pdl);
 }
 
 tint4_status gemm_entry(bool a_int4, const void* a, const float* tok_scale, const uint8_t* w,
@@ -434,13 +453,15 @@ tint4_status linear_entry(int bits, const tint4_bf16* x, const uint8_t* w_packed
     uint8_t* codes = static_cast<uint8_t*>(workspace);
     float* tok_scale = reinterpret_cast<float*>(codes + align_up(code_bytes, 256));
     cudaStream_t st = as_stream(stream);
-    const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
     const auto* b = reinterpret_cast<const __nv_bfloat16*>(bias);
-    if (bits == 8) launch_rq_g<__nv_bfloat16, 127, false>(xb, M, K, group, codes, tok_scale, st);
-    else launch_rq_g<__nv_bfloat16, 7, false>(xb, M, K, group, codes, tok_scale, st);
+    if (bits == 8) launch_linear_codes<127>(x, M, K, group, codes, tok_scale, st);
+    else launch_linear_codes<7>(x, M, K, group, codes, tok_scale, st);
     if ((s = last_launch_status()) != TINT4_OK) return s;
-    return launch_gemm<false, false>(codes, w_packed, tok_scale, row_scale, b, y, M, N, K, st,
-                                     true);
+    return linear_codes_evod(M)
+               ? launch_gemm<false, false, true>(codes, w_packed, tok_scale, row_scale, b, y, M,
+                                                 N, K, st, true)
+               : launch_gemm<false, false>(codes, w_packed, tok_scale, row_scale, b, y, M, N, K,
+                                           st, true);
 }
 
 // ------------------------------------------------------------------ W4A16
@@ -591,9 +612,12 @@ tint4_status check_groups(const tint4_weight_group* groups, int num_groups, int 
     return TINT4_OK;
 }
 
+// EVOD: int8 codes in the even/odd K order (only where linear_codes_evod(M)).
+template <bool EVOD = false>
 tint4_status launch_gemm_grouped(const int8_t* codes, const float* tok_scale,
                                  const tint4_weight_group* groups, int num_groups, int M, int K,
                                  cudaStream_t st, bool pdl) {
+    if (EVOD && !linear_codes_evod(M)) return TINT4_ERR_INVALID_ARG;
     if (M <= kS8MaxM) {
         // every weight is read once per launch anyway: one small-M launch per group
         for (int g = 0; g < num_groups; ++g) {
@@ -616,7 +640,7 @@ tint4_status launch_gemm_grouped(const int8_t* codes, const float* tok_scale,
         grp.N[g] = groups[g].N;
     }
     grp.count = num_groups;
-    return launch_gemm_tmem<false, false>(codes, tok_scale, grp, w, M, K, st, pdl);
+    return launch_gemm_tmem<false, false, false, EVOD>(codes, tok_scale, grp, w, M, K, st, pdl);
 }
 
 // W8A8: int8 codes x int8 weights, one tensor-core launch at every M.
@@ -750,10 +774,11 @@ tint4_status convrot_w4a8_linear_grouped(const tint4_bf16* x,
     float* tok_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                                 align_up(static_cast<size_t>(M) * K, 256));
     cudaStream_t st = as_stream(stream);
-    launch_rq_g<__nv_bfloat16, 127, false>(reinterpret_cast<const __nv_bfloat16*>(x), M, K, group,
-                                           codes, tok_scale, st);
+    launch_linear_codes<127>(x, M, K, group, codes, tok_scale, st);
     if ((s = last_launch_status()) != TINT4_OK) return s;
-    return launch_gemm_grouped(codes, tok_scale, groups, num_groups, M, K, st, true);
+    return linear_codes_evod(M)
+               ? launch_gemm_grouped<true>(codes, tok_scale, groups, num_groups, M, K, st, true)
+               : launch_gemm_grouped(codes, tok_scale, groups, num_groups, M, K, st, true);
 }
 
 tint4_status tint4_quantize_weights_int8(const float* W, int N, int K, int group,
@@ -833,12 +858,14 @@ tint4_status convrot_w4a8_linear_noalloc(const tint4_bf16* x, const uint8_t* w_p
     float* tok_scale =
         reinterpret_cast<float*>(codes + align_up(static_cast<size_t>(M) * K, 256));
     cudaStream_t st = as_stream(stream);
-    launch_rq_g<__nv_bfloat16, 127, false>(reinterpret_cast<const __nv_bfloat16*>(x), M, K, group,
-                                           codes, tok_scale, st);
+    launch_linear_codes<127>(x, M, K, group, codes, tok_scale, st);
     if ((s = last_launch_status()) != TINT4_OK) return s;
-    return launch_gemm<false, false>(codes, w_packed, tok_scale, row_scale,
-                                     reinterpret_cast<const __nv_bfloat16*>(bias), y, M, N, K,
-                                     st, true);
+    const auto* b = reinterpret_cast<const __nv_bfloat16*>(bias);
+    return linear_codes_evod(M)
+               ? launch_gemm<false, false, true>(codes, w_packed, tok_scale, row_scale, b, y, M,
+                                                 N, K, st, true)
+               : launch_gemm<false, false>(codes, w_packed, tok_scale, row_scale, b, y, M, N, K,
+                                           st, true);
 }
 
 tint4_status w4a16_gemv_gemm(const tint4_bf16* x, const uint8_t* w_q, const tint4_bf16* scale,

@@ -243,6 +243,32 @@ def test_convrot_linear_small(M, N, K, g, act_bits):
     assert_gemm_output(bf16_from_gpu(y), y_ref)
 
 
+@pytest.mark.parametrize("act_bits", [8, 4])
+@pytest.mark.parametrize("M,N,K,g", [(17, 272, 320, 64), (200, 1040, 1024, 16),
+                                     (333, 256, 768, 256)])
+def test_fused_linear_even_odd_codes_match_gemm(M, N, K, g, act_bits):
+    """Past the small-M kernel the fused linears keep their workspace codes in
+    the tensor-core GEMM's even/odd K order; every fused entry gives, bit for
+    bit, the output of the quantize entry followed by the GEMM entry (natural
+    order codes), which the other tests hold to the oracle."""
+    x = bf16_to_gpu(inputs.activations(M, K, seed=540 + M))
+    wp, sr = t4.tint4_pack_weights(to_gpu(inputs.weights(N, K, seed=541 + N)), g)
+    b = bf16_to_gpu(inputs.f32_to_bf16_bits(np.linspace(-1, 1, N, dtype=np.float32)))
+    codes, st = t4.convrot_quantize_act(x, g, act_bits)
+    if act_bits == 8:
+        y0 = t4.w4a8_gemm(codes, st, wp, sr, b)
+        y1 = t4.convrot_w4a8_linear(x, wp, sr, g, b)
+        y2 = t4.convrot_w4a8_linear_noalloc(x, wp, sr, g, b)
+        y3 = t4.convrot_w4a8_linear_grouped(x, [(wp, sr, b, None)], g)[0]
+        ys = (y1, y2, y3)
+    else:
+        y0 = t4.w4a4_gemm(codes, st, wp, sr, b)
+        ys = (t4.convrot_w4a4_linear(x, wp, sr, g, b),)
+    torch.cuda.synchronize()
+    for y in ys:
+        assert torch.equal(y, y0)
+
+
 def test_quantized_linear_module_end_to_end():
     """Weights packed on the GPU, layer run on the GPU, both against the oracle."""
     M, N, K, g = 96, 320, 512, 64
