@@ -285,9 +285,17 @@ def run_ours(args, rank, world, dev):
     xs = [x] + [x.clone() for _ in range(7)]
     q_ms = graph_time(lambda i: t4.convrot_quantize_act(xs[i % 8], g, 8, codes, st), 32, dev)
     del xs
-    gemm_ms = statistics.median(time_steps(lambda: t4.w4a8_gemm(codes, st, wp, sr, None, y),
-                                           args.steps, flush, dev))
+    # the GEMM launch of the step: the fused linear's codes are in the even/odd
+    # K order, which the test entry takes as input (permuted here, untimed)
+    codes_eo = t4.even_odd_codes(codes)
+    gemm_ms = statistics.median(time_steps(
+        lambda: t4.tint4_debug_w4a8_gemm_even_odd(codes_eo, st, wp, sr, None, y),
+        args.steps, flush, dev))
     gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
+    # the public GEMM entry on natural-order codes (same kernel, two byte
+    # permutes more per packed weight word)
+    gemm_nat_ms = statistics.median(time_steps(lambda: t4.w4a8_gemm(codes, st, wp, sr, None, y),
+                                               max(3, args.steps // 4), flush, dev))
 
     # end to end through the same call, pinned host buffers, copies timed
     x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -336,13 +344,16 @@ def run_ours(args, rank, world, dev):
                    "M": M, "N": N, "K": K, "group": g, "act_bits": 8,
                    "per_gpu_tokens": M, "parallelism": f"independent batches x{world}",
                    "l2": "flushed (256 MiB write) before every timed step, outside the events"},
-        "roofline": {"bound": "tensor", "kernel": "w4a8_tmem_gemm_kernel (tcgen05 kind::i8)",
+        "roofline": {"bound": "tensor",
+                     "kernel": "w4a8_tmem_gemm_kernel<even/odd codes> (tcgen05 kind::i8), "
+                               "the GEMM launch of the fused linear",
                      "achieved": round(gemm_tops, 2), "peak": round(int8_peak, 1),
                      "unit": "TOPS", "frac": round(gemm_tops / int8_peak, 4),
                      "traffic": traffic,
                      "peak_source": f"{pk['source']}: 2 x bf16 cuBLAS burst "
                                     f"{pk['bf16']} TFLOP/s (nominal int8:bf16 = 2)",
-                     "kernel_us": round(gemm_ms * 1e3, 2)},
+                     "kernel_us": round(gemm_ms * 1e3, 2),
+                     "w4a8_gemm_natural_codes_us": round(gemm_nat_ms * 1e3, 2)},
         "e2e": {"value": round(world * ops / (e2e_ms_max * 1e-3) / 1e12, 3), "unit": "TOPS",
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
                 "ms_per_step": round(e2e_ms_max, 4)},
@@ -636,12 +647,17 @@ def run_profile_case(case: str, dev):
         wp, sr = t4.tint4_pack_weights(torch.from_numpy(W_np).to(dev), g)
         codes, st = t4.convrot_quantize_act(x, g, bits)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        gemm = t4.w4a8_gemm if bits == 8 else t4.w4a4_gemm
+        if bits == 8:
+            # the fused linear's GEMM launch (even/odd codes)
+            codes_eo = t4.even_odd_codes(codes)
+            gemm = lambda: t4.tint4_debug_w4a8_gemm_even_odd(codes_eo, st, wp, sr, None, y)
+        else:
+            gemm = lambda: t4.w4a4_gemm(codes, st, wp, sr, None, y)
         for _ in range(3):
             if case == "qkv_quantize":
                 t4.convrot_quantize_act(x, g, bits, codes, st)
             else:
-                gemm(codes, st, wp, sr, None, y)
+                gemm()
     elif case.startswith("decode_w4a8_M"):
         M = int(case[len("decode_w4a8_M"):])
         w = inputs.WORKLOADS["te_decode_w4a8"]

@@ -277,6 +277,19 @@ tint4_status tint4_debug_int32_gemm(const void* a, int act_bits, const uint8_t* 
                                     int32_t* acc, int M, int N, int K, void* stream);
 
 /*
+ * Test and timing entry: the GEMM launch the fused linears make for M > 16
+ * ("ComfyUI-INT-Crush", "Inference > INT4 > CUDA backend": INT8 GEMM with
+ * fused dequant), on int8 codes stored in the even/odd K order: within every
+ * block of 8 codes along K, the codes of positions 0, 2, 4, 6, 1, 3, 5, 7.
+ * Same arguments, rules and result as w4a8_gemm on the natural-order codes;
+ * M must be > 16 (TINT4_ERR_UNSUPPORTED_SHAPE otherwise, nothing launched).
+ */
+tint4_status tint4_debug_w4a8_gemm_even_odd(const int8_t* a_even_odd, const float* tok_scale,
+                                            const uint8_t* w_packed, const float* row_scale,
+                                            const tint4_bf16* bias, tint4_bf16* y, int M, int N,
+                                            int K, void* stream);
+
+/*
  * Test entry for the bounded waits: launches one CTA that waits on a barrier
  * nobody arrives at, for at most limit_ns nanoseconds, then records
  * TINT4_ERR_TIMEOUT in the device error word and returns.  The context stays

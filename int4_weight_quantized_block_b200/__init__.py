@@ -30,6 +30,8 @@ __all__ = [
     "convrot_w4a8_linear_noalloc",
     "w4a16_gemv_gemm",
     "tint4_debug_int32_gemm",
+    "tint4_debug_w4a8_gemm_even_odd",
+    "even_odd_codes",
     "tint4_debug_bounded_wait",
     "tint4_get_device_error",
     "tint4_set_wait_limit_ns",
@@ -317,6 +319,21 @@ def tint4_debug_int32_gemm(a, act_bits: int, w_packed, acc=None) -> torch.Tensor
     _native.call("tint4_debug_int32_gemm", _ptr(a), act_bits, _ptr(w_packed), _ptr(acc), M, N, K,
                  _stream(a.device))
     return acc
+
+
+def even_odd_codes(codes: torch.Tensor) -> torch.Tensor:
+    """int8 codes [M, K] in natural K order -> the even/odd K order of
+    tint4_debug_w4a8_gemm_even_odd (positions 0, 2, 4, 6, 1, 3, 5, 7 of every
+    block of 8).  A layout change only (torch ops, test and timing set-up)."""
+    M, K = codes.shape
+    return codes.view(M, K // 8, 4, 2).transpose(2, 3).contiguous().view(M, K)
+
+
+def tint4_debug_w4a8_gemm_even_odd(a_even_odd, tok_scale, w_packed, row_scale, bias=None,
+                                   y=None) -> torch.Tensor:
+    """The fused linears' GEMM launch (M > 16) on even/odd-order int8 codes."""
+    return _gemm("tint4_debug_w4a8_gemm_even_odd", a_even_odd, tok_scale, w_packed, row_scale,
+                 bias, y, torch.int8, lambda K: K)
 
 
 def tint4_debug_bounded_wait(limit_ns: int, device=None) -> None:

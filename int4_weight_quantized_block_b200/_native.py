@@ -54,6 +54,7 @@ SIGNATURES = {
     "convrot_w8a8_linear": (I, [P, P, P, P, P, I, I, I, I, P, SZ, P]),
     "convrot_w4a8_linear_grouped": (I, [P, P, I, I, I, I, P, SZ, P]),
     "tint4_debug_int32_gemm": (I, [P, I, P, P, I, I, I, P]),
+    "tint4_debug_w4a8_gemm_even_odd": (I, [P, P, P, P, P, P, I, I, I, P]),
     "tint4_debug_bounded_wait": (I, [U64, P]),
     "tint4_get_device_error": (I, [P]),
     "tint4_set_wait_limit_ns": (I, [U64]),

@@ -915,6 +915,23 @@ tint4_status tint4_debug_int32_gemm(const void* a, int act_bits, const uint8_t* 
                                                     M, N, K, as_stream(stream), false);
 }
 
+tint4_status tint4_debug_w4a8_gemm_even_odd(const int8_t* a_even_odd, const float* tok_scale,
+                                            const uint8_t* w_packed, const float* row_scale,
+                                            const tint4_bf16* bias, tint4_bf16* y, int M, int N,
+                                            int K, void* stream) {
+    tint4_status s = check_mnk(M, N, K);
+    if (s != TINT4_OK) return s;
+    if (!linear_codes_evod(M)) return TINT4_ERR_UNSUPPORTED_SHAPE;
+    if (!a_even_odd || !tok_scale || !w_packed || !row_scale || !y) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(a_even_odd) || !aligned16(tok_scale) || !aligned16(w_packed) ||
+        !aligned16(row_scale) || !aligned16(y) || !aligned16(bias))
+        return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    return launch_gemm<false, false, true>(a_even_odd, w_packed, tok_scale, row_scale,
+                                           reinterpret_cast<const __nv_bfloat16*>(bias), y, M, N,
+                                           K, as_stream(stream), false);
+}
+
 tint4_status tint4_debug_bounded_wait(uint64_t limit_ns, void* stream) {
     if (limit_ns < 1000ull || limit_ns > 10000000000ull) return TINT4_ERR_INVALID_ARG;
     tint4_status s = check_device();

@@ -149,6 +149,10 @@ def test_grouped_rules(lib):
 def test_debug_entries_rules(lib):
     assert lib.tint4_debug_int32_gemm(16, 6, 16, 16, 4, 256, 256, NULL) == 1
     assert lib.tint4_debug_bounded_wait(10, NULL) == 1
+    # the even/odd GEMM entry: M > 16 only, then the GEMM rules
+    assert lib.tint4_debug_w4a8_gemm_even_odd(16, 16, 16, 16, NULL, 16, 16, 256, 256, NULL) == 2
+    assert lib.tint4_debug_w4a8_gemm_even_odd(NULL, 16, 16, 16, NULL, 16, 17, 256, 256, NULL) == 1
+    assert lib.tint4_debug_w4a8_gemm_even_odd(16, 16, 16, 16, NULL, 16, 17, 256, 100, NULL) == 2
     assert lib.tint4_set_wait_limit_ns(10) == 1
     assert lib.tint4_set_wait_limit_ns(10 ** 11) == 1
     assert lib.tint4_set_wait_limit_ns(4 * 10 ** 9) == 0

@@ -264,6 +264,9 @@ def test_fused_linear_even_odd_codes_match_gemm(M, N, K, g, act_bits):
     else:
         y0 = t4.w4a4_gemm(codes, st, wp, sr, b)
         ys = (t4.convrot_w4a4_linear(x, wp, sr, g, b),)
+    if act_bits == 8:
+        # the test entry runs the same GEMM launch on codes permuted here
+        ys += (t4.tint4_debug_w4a8_gemm_even_odd(t4.even_odd_codes(codes), st, wp, sr, b),)
     torch.cuda.synchronize()
     for y in ys:
         assert torch.equal(y, y0)
