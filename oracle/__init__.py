@@ -74,6 +74,9 @@ def _load():
             "oracle_w4a16_f64": [P, P, P, P, I, I, I, I, P],
             "oracle_w4a16_dequant_f64": [P, P, P, P, I, I, I, I, P],
             "oracle_quantize_weights_int8": [P, I, I, I, P, P],
+            "oracle_pack_weights_groupwise": [P, I, I, I, I, I, P, P, P, P],
+            "oracle_gemm_groupwise_f64": [P, P, P, P, P, P, I, I, I, I, P, P],
+            "oracle_gemm_groupwise_sampled_f64": [P, P, P, P, P, P, I, I, I, I, P, L, P, P],
             "oracle_round_bf16": [P, L, P],
             "oracle_num_threads": [],
         }
@@ -343,6 +346,68 @@ def convrot_linear_f64(x_bits, w_packed, row_scale, g, act_bits, bias_bits=None)
     _check(_load().oracle_convrot_linear_f64(_ptr(x), _ptr(wp), _ptr(sr), _ptr(b), M, N, K, g,
                                              act_bits, _ptr(y)), "convrot_linear_f64")
     return y
+
+
+# --------------------------------------------------------------------------
+# Group-wise W4A8 (per row and K group weight scales; symmetric or asymmetric)
+# --------------------------------------------------------------------------
+
+def pack_weights_groupwise(W: np.ndarray, g: int, G: int = 128, asym: bool = False):
+    """Twin of ``tint4_pack_weights_groupwise``: rotate W along K, then int4
+    codes per (row, G-wide K group).
+
+    Returns (packed uint8 [N, K/2], scale fp32 [N, K/G], zero uint8 [N, K/G]
+    or None, codes int8 [N, K]).  "ComfyUI-INT-Crush", "Weight Format"
+    (scales [out, num_groups]); "feat: packed int4 convrot model loading and
+    dispatch", "Summary" (the asymmetric W4A8 format)."""
+    Wc = _c(W, np.float32)
+    N, K = Wc.shape
+    packed = np.empty((N, K // 2), dtype=np.uint8)
+    scale = np.empty((N, K // G), dtype=np.float32)
+    zero = np.empty((N, K // G), dtype=np.uint8) if asym else None
+    codes = np.empty((N, K), dtype=np.int8)
+    _check(_load().oracle_pack_weights_groupwise(_ptr(Wc), N, K, g, G, int(asym), _ptr(packed),
+                                                 _ptr(scale), _ptr(zero), _ptr(codes)),
+           "pack_weights_groupwise")
+    return packed, scale, zero, codes
+
+
+def gemm_groupwise_f64(a, tok_scale, w_packed, scale, zero=None, bias_bits=None, G: int = 128):
+    """y = s_tok * sum_j s[n, j] * sum_{k in j} a (q - z) (+ bias), unrounded
+    (fp64), and the magnitude of its terms (fp64), both [M, N]."""
+    ac = _c(a, np.int8)
+    st, sc = _c(tok_scale, np.float32), _c(scale, np.float32)
+    wp = _c(w_packed, np.uint8)
+    z = None if zero is None else _c(zero, np.uint8)
+    b = None if bias_bits is None else _c(bias_bits, np.uint16)
+    M, K = ac.shape
+    N = wp.shape[0]
+    y = np.empty((M, N), dtype=np.float64)
+    mag = np.empty((M, N), dtype=np.float64)
+    _check(_load().oracle_gemm_groupwise_f64(_ptr(ac), _ptr(st), _ptr(wp), _ptr(sc), _ptr(z),
+                                             _ptr(b), M, N, K, G, _ptr(y), _ptr(mag)),
+           "gemm_groupwise_f64")
+    return y, mag
+
+
+def gemm_groupwise_sampled_f64(a, tok_scale, w_packed, scale, pairs, zero=None, bias_bits=None,
+                               G: int = 128):
+    """The same for selected (m, n) pairs (pairs int64 [P, 2]): (y, mag) [P]."""
+    ac = _c(a, np.int8)
+    st, sc = _c(tok_scale, np.float32), _c(scale, np.float32)
+    wp = _c(w_packed, np.uint8)
+    z = None if zero is None else _c(zero, np.uint8)
+    b = None if bias_bits is None else _c(bias_bits, np.uint16)
+    pr = _c(pairs, np.int64)
+    M, K = ac.shape
+    N = wp.shape[0]
+    y = np.empty(pr.shape[0], dtype=np.float64)
+    mag = np.empty(pr.shape[0], dtype=np.float64)
+    _check(_load().oracle_gemm_groupwise_sampled_f64(_ptr(ac), _ptr(st), _ptr(wp), _ptr(sc),
+                                                     _ptr(z), _ptr(b), M, N, K, G, _ptr(pr),
+                                                     pr.shape[0], _ptr(y), _ptr(mag)),
+           "gemm_groupwise_sampled_f64")
+    return y, mag
 
 
 def w4a16_f64(x_bits, q_packed, scale_bits, zero, group) -> np.ndarray:

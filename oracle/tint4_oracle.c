@@ -525,6 +525,168 @@ int oracle_w4a16(const uint16_t* x, const uint8_t* q, const uint16_t* s, const u
     return rc;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Group-wise W4A8 weights and GEMM                                          */
+/* ------------------------------------------------------------------------ */
+
+/* "ComfyUI-INT-Crush", "Weight Format": the INT4 weight scales have one value
+ * per output row and K group ([out, num_groups]).  stable-diffusion.cpp
+ * "feat: packed int4 convrot model loading and dispatch", "Summary": an
+ * asymmetric W4A8 format (asym_w4a8_int8) next to the symmetric one.
+ * Readings (the pages fix none of this arithmetic):
+ *  - a weight group is G consecutive K values of one row, after the same
+ *    block rotation as the per-row format; its scale is fp32;
+ *  - symmetric: the per-row rule applied to the group: s = absmax / 7 and
+ *    q = clamp(rne(v / s), -7, 7), stored as two's complement nibbles;
+ *  - asymmetric: the group's range widened to contain 0, lo = min(0, min v),
+ *    hi = max(0, max v); s = (hi - lo) / 15; zero point z = rne(-lo / s),
+ *    clamped to [0, 15]; q = clamp(rne(v / s) + z, 0, 15), stored as plain
+ *    4-bit numbers; the weight the codes stand for is s * (q - z);
+ *  - an all-zero group has s = 0, z = 0 and q = 0;
+ *  - all of it in fp32 with IEEE division and round half to even (the codes
+ *    are decisions, taken in the kernel's precision). */
+static void quantize_group_asym(const float* v, int G, int8_t* q, float* scale, uint8_t* zero) {
+    float lo = 0.0f, hi = 0.0f;
+    for (int k = 0; k < G; ++k) {
+        if (v[k] < lo) lo = v[k];
+        if (v[k] > hi) hi = v[k];
+    }
+    float s = (hi - lo) / 15.0f;
+    int z = 0;
+    if (s > 0.0f) {
+        float t = rintf(-lo / s);
+        if (t < 0.0f) t = 0.0f;
+        if (t > 15.0f) t = 15.0f;
+        z = (int)t;
+    }
+    *scale = s;
+    *zero = (uint8_t)z;
+    for (int k = 0; k < G; ++k) {
+        int c = 0;
+        if (s > 0.0f) {
+            c = (int)rintf(v[k] / s) + z;
+            if (c < 0) c = 0;
+            if (c > 15) c = 15;
+        }
+        q[k] = (int8_t)c;
+    }
+}
+
+/* W fp32 [N, K] -> rotate each g-block along K -> group-wise int4 codes with
+ * scale fp32 [N, K/G] (and zero uint8 [N, K/G] when asym) -> packed uint8
+ * [N, K/2], byte j holding code 2j in its low nibble.  codes (optional)
+ * receives the codes as int8 [N, K]: signed for the symmetric form, 0..15 for
+ * the asymmetric one.  zero may be NULL when asym == 0. */
+int oracle_pack_weights_groupwise(const float* W, int N, int K, int g, int G, int asym,
+                                  uint8_t* packed, float* scale, uint8_t* zero, int8_t* codes) {
+    if (!W || !packed || !scale || (asym && !zero) || N <= 0 || K <= 0 || K % 2 || G <= 0 ||
+        G % 2 || K % G)
+        return ORACLE_BAD_ARG;
+    if (g != 0 && (!is_power_of_four(g) || K % g)) return ORACLE_BAD_ARG;
+    const int ng = K / G;
+    int bad = 0;
+#pragma omp parallel
+    {
+        float* v = (float*)malloc(sizeof(float) * (size_t)K);
+        int8_t* q = (int8_t*)malloc((size_t)K);
+        if (!v || !q) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(static)
+            for (int n = 0; n < N; ++n) {
+                memcpy(v, W + (long)n * K, sizeof(float) * (size_t)K);
+                if (g) for (int b = 0; b < K; b += g) fwht_f32_block(v + b, g);
+                for (int j = 0; j < ng; ++j) {
+                    if (asym)
+                        quantize_group_asym(v + (long)j * G, G, q + (long)j * G,
+                                            &scale[(long)n * ng + j], &zero[(long)n * ng + j]);
+                    else
+                        quantize_row(v + (long)j * G, G, 7, q + (long)j * G,
+                                     &scale[(long)n * ng + j]);
+                }
+                oracle_pack_int4(q, 1, K, packed + (long)n * (K / 2));
+                if (codes) memcpy(codes + (long)n * K, q, (size_t)K);
+            }
+        }
+        free(v);
+        free(q);
+    }
+    return bad ? ORACLE_BAD_ARG : ORACLE_OK;
+}
+
+/* Code of weight (n, k): the nibble read as two's complement (symmetric) or
+ * as a plain 4-bit number (asymmetric). */
+static int groupwise_code(const uint8_t* packed, int K, int n, int k, int asym) {
+    uint8_t b = packed[(long)n * (K / 2) + k / 2];
+    int c = (k % 2 == 0) ? (b & 0xF) : (b >> 4);
+    if (!asym && c >= 8) c -= 16;
+    return c;
+}
+
+/* One output of the group-wise W4A8 GEMM ("ComfyUI-INT-Crush", "Inference >
+ * INT4 > CUDA backend": integer GEMM, then dequant; "Weight Format": one
+ * scale per row and group): with the group's integer sum
+ *   p_j = sum_{k in group j} a[m, k] * (q[n, k] - z[n, j])     (exact),
+ *   y = s_tok[m] * sum_j s[n, j] * p_j (+ bias[n])              (fp64),
+ * and mag = |s_tok[m]| * sum_j |s[n, j] * p_j| + |bias[n]|, the size of the
+ * terms a floating-point evaluation adds up. */
+static void groupwise_one(const int8_t* a, const float* tok_scale, const uint8_t* packed,
+                          const float* scale, const uint8_t* zero, const uint16_t* bias, int N,
+                          int K, int G, int m, int n, double* y, double* mag) {
+    const int ng = K / G;
+    const int asym = zero != NULL;
+    double acc = 0.0, sum_abs = 0.0;
+    for (int j = 0; j < ng; ++j) {
+        const int z = asym ? zero[(long)n * ng + j] : 0;
+        long p = 0;
+        for (int k = j * G; k < (j + 1) * G; ++k)
+            p += (long)a[(long)m * K + k] * (groupwise_code(packed, K, n, k, asym) - z);
+        const double t = (double)scale[(long)n * ng + j] * (double)p;
+        acc += t;
+        sum_abs += fabs(t);
+    }
+    const double b = bias ? (double)bf16_bits_to_float(bias[n]) : 0.0;
+    *y = acc * (double)tok_scale[m] + b;
+    if (mag) *mag = fabs((double)tok_scale[m]) * sum_abs + fabs(b);
+    (void)N;
+}
+
+/* y fp64 [M, N] (unrounded) and, optionally, mag fp64 [M, N]; a int8 [M, K],
+ * zero NULL for the symmetric form. */
+int oracle_gemm_groupwise_f64(const int8_t* a, const float* tok_scale, const uint8_t* packed,
+                              const float* scale, const uint8_t* zero, const uint16_t* bias,
+                              int M, int N, int K, int G, double* y, double* mag) {
+    if (!a || !tok_scale || !packed || !scale || !y || M < 0 || N < 0 || K <= 0 || K % 2 ||
+        G <= 0 || K % G)
+        return ORACLE_BAD_ARG;
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n)
+        for (int m = 0; m < M; ++m)
+            groupwise_one(a, tok_scale, packed, scale, zero, bias, N, K, G, m, n,
+                          &y[(long)m * N + n], mag ? &mag[(long)m * N + n] : NULL);
+    return ORACLE_OK;
+}
+
+/* The same for a list of (m, n) pairs: pairs[2i] = m, pairs[2i + 1] = n. */
+int oracle_gemm_groupwise_sampled_f64(const int8_t* a, const float* tok_scale,
+                                      const uint8_t* packed, const float* scale,
+                                      const uint8_t* zero, const uint16_t* bias, int M, int N,
+                                      int K, int G, const int64_t* pairs, long npairs, double* y,
+                                      double* mag) {
+    if (!a || !tok_scale || !packed || !scale || !pairs || !y || npairs < 0 || K <= 0 ||
+        K % 2 || G <= 0 || K % G)
+        return ORACLE_BAD_ARG;
+    for (long i = 0; i < npairs; ++i)
+        if (pairs[2 * i] < 0 || pairs[2 * i] >= M || pairs[2 * i + 1] < 0 || pairs[2 * i + 1] >= N)
+            return ORACLE_BAD_ARG;
+#pragma omp parallel for schedule(static)
+    for (long i = 0; i < npairs; ++i)
+        groupwise_one(a, tok_scale, packed, scale, zero, bias, N, K, G, (int)pairs[2 * i],
+                      (int)pairs[2 * i + 1], &y[i], mag ? &mag[i] : NULL);
+    return ORACLE_OK;
+}
+
 /* Round an array of doubles to bf16 bits (nearest, ties to even). */
 int oracle_round_bf16(const double* v, long n, uint16_t* out) {
     if (!v || !out || n < 0) return ORACLE_BAD_ARG;

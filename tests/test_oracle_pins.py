@@ -530,3 +530,121 @@ def test_compare_accepts_2d_inputs_and_error_arrays():
     bias = np.broadcast_to(inputs.f32_to_bf16_bits(np.ones(32)), (8, 32))
     c = check_bf16(y, y64, gemm_eval_error(y64, oracle.bf16_bits_to_f32(bias)))
     assert c.ok
+
+
+# ------------------------------------------------------------------ group-wise W4A8
+
+def _unpack_nibbles(packed, signed):
+    """Independent nibble reader for the group-wise pins (numpy only)."""
+    p = np.asarray(packed, np.uint8)
+    q = np.empty((p.shape[0], 2 * p.shape[1]), np.int64)
+    q[:, 0::2] = p & 0xF
+    q[:, 1::2] = p >> 4
+    if signed:
+        q = np.where(q >= 8, q - 16, q)
+    return q
+
+
+def test_groupwise_weight_codes_golden():
+    d = golden("groupwise_weight_codes.json")
+    for mode in ("asym", "sym"):
+        W = np.array(d["W_" + mode], np.float32)
+        packed, s, z, codes = oracle.pack_weights_groupwise(W, d["group"], d["G"],
+                                                            asym=(mode == "asym"))
+        assert codes.tolist() == d["codes_" + mode]
+        assert s.tolist() == d["scale_" + mode]
+        if mode == "asym":
+            assert z.tolist() == d["zero_asym"]
+        else:
+            assert z is None
+        assert _unpack_nibbles(packed, mode == "sym").tolist() == d["codes_" + mode]
+
+
+@pytest.mark.parametrize("asym", [False, True])
+@pytest.mark.parametrize("g", (0,) + GROUPS)
+def test_groupwise_weight_quant_error_bound(g, asym):
+    """Rotated rows (an independent fp64 rotation) within s/2 of s (q - z) in
+    every group; the group extremes reach the end codes; every code and
+    zero point in range."""
+    G = 128
+    K = 2 * max(g, G)
+    W = inputs.weights(5, K, seed=14)
+    W[1, :G] = np.abs(W[1, :G])        # a group with no negative value
+    W[2, :G] = -np.abs(W[2, :G])       # and one with no positive value
+    packed, s, z, codes = oracle.pack_weights_groupwise(W, g, G, asym)
+    if g:
+        H = oracle.hadamard(g)
+        v = (W.astype(np.float64).reshape(5, -1, g) @ H.T).reshape(5, -1)
+    else:
+        v = W.astype(np.float64)
+    q = _unpack_nibbles(packed, not asym)
+    assert np.array_equal(q, codes)
+    for n in range(5):
+        for j in range(K // G):
+            vg = v[n, j * G:(j + 1) * G]
+            sg = np.float64(s[n, j])
+            zg = int(z[n, j]) if asym else 0
+            err = np.abs(vg - sg * (q[n, j * G:(j + 1) * G] - zg))
+            assert err.max() <= 0.5 * sg * (1 + 1e-5) + 1e-6 * np.abs(vg).max()
+            qg = q[n, j * G:(j + 1) * G]
+            if asym:
+                assert 0 <= qg.min() and qg.max() <= 15 and 0 <= zg <= 15
+                assert qg.max() == 15 or qg.min() == 0
+            else:
+                assert np.abs(qg).max() == 7
+    if asym and g == 0:
+        assert z[1, 0] == 0 and z[2, 0] == 15
+
+
+@pytest.mark.parametrize("asym", [False, True])
+def test_groupwise_gemm_brute_force(asym):
+    """The oracle's GEMM against the product written out with numpy: weights
+    dequantized as s (q - z) from an independent nibble reader, an fp64
+    matrix product, the token scale and the bias."""
+    M, N, K, G = 5, 7, 256, 64
+    rng = np.random.default_rng(21)
+    a = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    st = rng.uniform(0.01, 0.1, M).astype(np.float32)
+    W = inputs.weights(N, K, seed=22)
+    packed, s, z, _ = oracle.pack_weights_groupwise(W, 0, G, asym)
+    bias = inputs.f32_to_bf16_bits(np.linspace(-1, 1, N, dtype=np.float32))
+    y, mag = oracle.gemm_groupwise_f64(a, st, packed, s, z, bias, G)
+    q = _unpack_nibbles(packed, not asym).astype(np.float64)
+    zz = np.repeat(z.astype(np.float64), G, axis=1) if asym else 0.0
+    w = np.repeat(s.astype(np.float64), G, axis=1) * (q - zz)
+    b = oracle.bf16_bits_to_f32(bias).astype(np.float64)
+    ref = st.astype(np.float64)[:, None] * (a.astype(np.float64) @ w.T) + b
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    # the magnitude: |s_tok| sum_j |s_j p_j| + |bias|, never below |y|
+    p = np.einsum("mjk,njk->mnj", a.astype(np.float64).reshape(M, -1, G),
+                  (q - zz).reshape(N, -1, G))
+    mref = st.astype(np.float64)[:, None] * np.abs(p * s.astype(np.float64)[None]).sum(-1) + np.abs(b)
+    assert np.allclose(mag, mref, rtol=1e-12) and np.all(mag >= np.abs(y) * (1 - 1e-12))
+    pairs = np.array([[0, 0], [4, 6], [2, 3], [4, 0]], np.int64)
+    ys, ms = oracle.gemm_groupwise_sampled_f64(a, st, packed, s, pairs, z, bias, G)
+    assert np.array_equal(ys, y[pairs[:, 0], pairs[:, 1]])
+    assert np.array_equal(ms, mag[pairs[:, 0], pairs[:, 1]])
+
+
+def test_groupwise_gemm_reduces_to_per_row():
+    """Symmetric codes with every group scale equal to the row scale: the
+    group-wise GEMM is the per-row GEMM and epilogue."""
+    M, N, K, G = 4, 6, 512, 128
+    rng = np.random.default_rng(23)
+    a = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    st = rng.uniform(0.01, 0.1, M).astype(np.float32)
+    packed, sr, codes = oracle.pack_weights(inputs.weights(N, K, seed=24), 64)
+    s = np.repeat(sr[:, None], K // G, axis=1)
+    y, _ = oracle.gemm_groupwise_f64(a, st, packed, s, None, None, G)
+    ref = oracle.epilogue_f64(oracle.gemm_i32(a, codes), st, sr)
+    assert np.allclose(y, ref, rtol=1e-13, atol=0)
+
+
+def test_groupwise_rejects_bad_shapes():
+    W = np.zeros((2, 96), np.float32)
+    with pytest.raises(ValueError):
+        oracle.pack_weights_groupwise(W, 0, 64, False)     # K % G
+    with pytest.raises(ValueError):
+        oracle.gemm_groupwise_sampled_f64(np.zeros((2, 128), np.int8), np.ones(2, np.float32),
+                                          np.zeros((3, 64), np.uint8), np.ones((3, 1), np.float32),
+                                          np.array([[2, 0]], np.int64))
