@@ -73,6 +73,7 @@ KERNEL_SOURCES = {
     "w4a16_mma_kernel": ("w4a16.cuh", "ptx.cuh"),
     "w4a8_small_kernel": ("w4a8_small.cuh", "ptx.cuh"),
     "w4a16_tmem_gemm_kernel": ("w4a16_gemm.cuh", "ptx.cuh"),
+    "w4a8_gw_tmem_gemm_kernel": ("gemm_tmem_gw.cuh", "gemm_tmem.cuh", "ptx.cuh"),
 }
 
 
@@ -422,6 +423,41 @@ def bench_rows(args, t4, inputs, dev, flush, pk, int8_peak):
         "gemm_frac_int8": round(ops / g_ms / 1e9 / int8_peak, 4),
         "linear_us": round(l_ms * 1e3, 2), "linear_TOPS": round(ops / l_ms / 1e9, 2)}
     del wc, sr, codes, st, y, ws, x
+
+    # the QKV layer with group-wise weight scales (one per row and 128-wide K
+    # group), asymmetric (zero points) and symmetric: GEMM and fused linear
+    name = "dit_qkv_w4a8_asym_g128"
+    w = inputs.WORKLOADS[name]
+    M, N, K, g = w["M"], w["N"], w["K"], w["group"]
+    x_np, W_np = inputs.layer_inputs(name)
+    x = bf16_gpu(x_np, dev)
+    W_dev = torch.from_numpy(W_np).to(dev)
+    del W_np
+    codes, st = t4.convrot_quantize_act(x, g, 8)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(t4.convrot_linear_workspace_size(M, K, 8), dtype=torch.uint8, device=dev)
+    ops = 2.0 * M * N * K
+    row = {"M": M, "N": N, "K": K, "group": g, "weight_group": t4.WEIGHT_GROUP,
+           "kernel": "w4a8_gw_tmem_gemm_kernel"}
+    for asym in (True, False):
+        wp, s, z = t4.tint4_pack_weights_groupwise(W_dev, g, asym)
+        t4.w4a8_gemm_groupwise(codes, st, wp, s, z, None, y)
+        t4.convrot_w4a8_linear_groupwise(x, wp, s, g, z, None, y, ws)
+        torch.cuda.synchronize(dev)
+        g_ms = statistics.median(time_steps(
+            lambda: t4.w4a8_gemm_groupwise(codes, st, wp, s, z, None, y), reps, flush, dev))
+        l_ms = statistics.median(time_steps(
+            lambda: t4.convrot_w4a8_linear_groupwise(x, wp, s, g, z, None, y, ws), reps, flush,
+            dev))
+        tag = "asym" if asym else "sym"
+        row.update({f"{tag}_gemm_us": round(g_ms * 1e3, 2),
+                    f"{tag}_gemm_TOPS": round(ops / g_ms / 1e9, 2),
+                    f"{tag}_gemm_frac_int8": round(ops / g_ms / 1e9 / int8_peak, 4),
+                    f"{tag}_linear_us": round(l_ms * 1e3, 2),
+                    f"{tag}_linear_TOPS": round(ops / l_ms / 1e9, 2)})
+        del wp, s, z
+    rows[name] = row
+    del W_dev, codes, st, y, ws, x
 
     # the QKV layer as three separate 3072-row weight matrices (Q, K, V of one
     # input): three GEMM launches against one grouped launch

@@ -203,6 +203,51 @@ tint4_status convrot_w8a8_linear(const tint4_bf16* x, const int8_t* w_int8,
                                  size_t workspace_bytes, void* stream);
 
 /*
+ * Group-wise W4A8 ("ComfyUI-INT-Crush", "Weight Format": INT4 weight scales
+ * of shape [out, num_groups]; stable-diffusion.cpp "feat: packed int4
+ * convrot model loading and dispatch", "Summary": the asymmetric W4A8 format
+ * asym_w4a8_int8).  Weight groups are TINT4_WEIGHT_GROUP consecutive K
+ * values of a row; ng = K / TINT4_WEIGHT_GROUP.
+ *   - tint4_pack_weights_groupwise: W fp32 [N, K] -> rotated along K (group 0
+ *     / 16 / 64 / 256, as tint4_pack_weights) -> per weight group
+ *       asym == 0: w_scale = absmax / 7, codes clamp(rne(v / s), -7, 7) as
+ *                  two's complement nibbles; w_zero unused (may be NULL);
+ *       asym == 1: lo = min(0, min v), hi = max(0, max v), w_scale =
+ *                  (hi - lo) / 15, w_zero = clamp(rne(-lo / s), 0, 15),
+ *                  codes clamp(rne(v / s) + zero, 0, 15) as plain nibbles;
+ *       an all-zero group: scale 0, zero 0, codes 0 (fp32, IEEE division).
+ *     w_packed uint8 [N, K/2] (byte j: code 2j low nibble, 2j+1 high),
+ *     w_scale fp32 [N, ng], w_zero uint8 [N, ng].
+ *   - w4a8_gemm_groupwise: codes int8 [M, K] (convrot_quantize_act, bits 8),
+ *     tok_scale fp32 [M], w_packed, w_scale, w_zero (NULL: symmetric codes;
+ *     else asymmetric codes with these zero points), bias bf16 [N] or NULL ->
+ *     y bf16 [M, N] = bf16(s_tok[m] * sum_j s[n, j] * p_j (+ bias[n])), p_j the
+ *     exact integer sum over group j of a * (q - z); the sum over groups is
+ *     evaluated in fp32 in group order.  One tensor-core launch at every M.
+ *   - convrot_w4a8_linear_groupwise: rotate + quantize x bf16 [M, K] into the
+ *     workspace (convrot_linear_workspace_size(M, K, 8) bytes, 256-byte
+ *     aligned; the codes there are in a private K order), then the GEMM.
+ * Shape rules: those of w4a8_gemm (N % 16 == 0, 32 <= K <= 65536) plus
+ * K % TINT4_WEIGHT_GROUP == 0 (and, for the packing and the fused linear,
+ * K % group == 0, K <= 16384); all pointers 16-byte aligned.  Errors as
+ * w4a8_gemm / convrot_w4a8_linear; asym outside {0, 1} is
+ * TINT4_ERR_INVALID_ARG.  The caller owns every buffer.
+ */
+#define TINT4_WEIGHT_GROUP 128
+tint4_status tint4_pack_weights_groupwise(const float* W, int N, int K, int group, int asym,
+                                          uint8_t* w_packed, float* w_scale, uint8_t* w_zero,
+                                          void* stream);
+tint4_status w4a8_gemm_groupwise(const int8_t* a, const float* tok_scale,
+                                 const uint8_t* w_packed, const float* w_scale,
+                                 const uint8_t* w_zero, const tint4_bf16* bias, tint4_bf16* y,
+                                 int M, int N, int K, void* stream);
+tint4_status convrot_w4a8_linear_groupwise(const tint4_bf16* x, const uint8_t* w_packed,
+                                           const float* w_scale, const uint8_t* w_zero,
+                                           const tint4_bf16* bias, tint4_bf16* y, int M, int N,
+                                           int K, int group, void* workspace,
+                                           size_t workspace_bytes, void* stream);
+
+/*
  * Grouped GEMM: the same activation codes times up to TINT4_MAX_GROUPS
  * weight matrices in one launch ("feat: packed int4 convrot model loading
  * and dispatch", "Summary": the activation rotate + quantize is shared by the

@@ -29,6 +29,10 @@ __all__ = [
     "convrot_w4a4_linear",
     "convrot_w4a8_linear_noalloc",
     "w4a16_gemv_gemm",
+    "WEIGHT_GROUP",
+    "tint4_pack_weights_groupwise",
+    "w4a8_gemm_groupwise",
+    "convrot_w4a8_linear_groupwise",
     "tint4_debug_int32_gemm",
     "tint4_debug_w4a8_gemm_even_odd",
     "even_odd_codes",
@@ -319,6 +323,74 @@ def tint4_debug_int32_gemm(a, act_bits: int, w_packed, acc=None) -> torch.Tensor
     _native.call("tint4_debug_int32_gemm", _ptr(a), act_bits, _ptr(w_packed), _ptr(acc), M, N, K,
                  _stream(a.device))
     return acc
+
+
+WEIGHT_GROUP = 128   # K values per group-wise weight scale (TINT4_WEIGHT_GROUP)
+
+
+def tint4_pack_weights_groupwise(W: torch.Tensor, group: int, asym: bool = False,
+                                 w_packed=None, w_scale=None, w_zero=None):
+    """fp32 W [N, K] -> (packed uint8 [N, K/2], scale fp32 [N, K/128],
+    zero uint8 [N, K/128] or None): rotated, then int4 per 128-wide K group
+    (symmetric, or asymmetric with zero points)."""
+    _need(W, "W", torch.float32)
+    N, K = W.shape
+    ng = K // WEIGHT_GROUP
+    if w_packed is None:
+        w_packed = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    if w_scale is None:
+        w_scale = torch.empty((N, ng), dtype=torch.float32, device=W.device)
+    if asym and w_zero is None:
+        w_zero = torch.empty((N, ng), dtype=torch.uint8, device=W.device)
+    _need(w_packed, "w_packed", torch.uint8, (N, K // 2))
+    _need(w_scale, "w_scale", torch.float32, (N, ng))
+    if asym:
+        _need(w_zero, "w_zero", torch.uint8, (N, ng))
+    _native.call("tint4_pack_weights_groupwise", _ptr(W), N, K, group, int(bool(asym)),
+                 _ptr(w_packed), _ptr(w_scale), _ptr(w_zero if asym else None), _stream(W.device))
+    return w_packed, w_scale, (w_zero if asym else None)
+
+
+def _gw_operands(M, K, w_packed, w_scale, w_zero, bias, y, device):
+    N = w_packed.shape[0]
+    ng = K // WEIGHT_GROUP
+    _need(w_packed, "w_packed", torch.uint8, (N, K // 2))
+    _need(w_scale, "w_scale", torch.float32, (N, ng))
+    if w_zero is not None:
+        _need(w_zero, "w_zero", torch.uint8, (N, ng))
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, (N,))
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    _need(y, "y", torch.bfloat16, (M, N))
+    return N, y
+
+
+def w4a8_gemm_groupwise(a, tok_scale, w_packed, w_scale, w_zero=None, bias=None,
+                        y=None) -> torch.Tensor:
+    """int8 codes a [M, K] x group-wise packed int4 W [N, K/2] -> bf16 y [M, N]."""
+    _need(a, "a", torch.int8)
+    M, K = a.shape
+    _need(tok_scale, "tok_scale", torch.float32, (M,))
+    N, y = _gw_operands(M, K, w_packed, w_scale, w_zero, bias, y, a.device)
+    _native.call("w4a8_gemm_groupwise", _ptr(a), _ptr(tok_scale), _ptr(w_packed), _ptr(w_scale),
+                 _ptr(w_zero), _ptr(bias), _ptr(y), M, N, K, _stream(a.device))
+    return y
+
+
+def convrot_w4a8_linear_groupwise(x, w_packed, w_scale, group, w_zero=None, bias=None, y=None,
+                                  workspace=None) -> torch.Tensor:
+    """Fused rotate + int8 quantize + group-wise W4A8 GEMM: bf16 x [M, K] -> y."""
+    _need(x, "x", torch.bfloat16)
+    M, K = x.shape
+    N, y = _gw_operands(M, K, w_packed, w_scale, w_zero, bias, y, x.device)
+    need = convrot_linear_workspace_size(M, K, 8)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    _native.call("convrot_w4a8_linear_groupwise", _ptr(x), _ptr(w_packed), _ptr(w_scale),
+                 _ptr(w_zero), _ptr(bias), _ptr(y), M, N, K, group, _ptr(workspace),
+                 workspace.numel(), _stream(x.device))
+    return y
 
 
 def even_odd_codes(codes: torch.Tensor) -> torch.Tensor:

@@ -53,6 +53,9 @@ SIGNATURES = {
     "w8a8_gemm": (I, [P, P, P, P, P, P, I, I, I, P]),
     "convrot_w8a8_linear": (I, [P, P, P, P, P, I, I, I, I, P, SZ, P]),
     "convrot_w4a8_linear_grouped": (I, [P, P, I, I, I, I, P, SZ, P]),
+    "tint4_pack_weights_groupwise": (I, [P, I, I, I, I, P, P, P, P]),
+    "w4a8_gemm_groupwise": (I, [P, P, P, P, P, P, P, I, I, I, P]),
+    "convrot_w4a8_linear_groupwise": (I, [P, P, P, P, P, P, I, I, I, I, P, SZ, P]),
     "tint4_debug_int32_gemm": (I, [P, I, P, P, I, I, I, P]),
     "tint4_debug_w4a8_gemm_even_odd": (I, [P, P, P, P, P, P, I, I, I, P]),
     "tint4_debug_bounded_wait": (I, [U64, P]),

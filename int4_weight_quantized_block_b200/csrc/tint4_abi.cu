@@ -13,6 +13,8 @@
 
 #include "../../include/tint4.h"
 #include "gemm_tmem.cuh"
+#include "gemm_tmem_gw.cuh"
+#include "pack_groupwise.cuh"
 #include "ptx.cuh"
 #include "quantize.cuh"
 #include "w4a16.cuh"
@@ -657,6 +659,85 @@ tint4_status launch_w8a8(const int8_t* codes, const float* st, const int8_t* w, 
     return launch_gemm_tmem<false, false, true>(codes, st, grp, &wp, M, K, stream, pdl);
 }
 
+// ------------------------------------------------------------------ group-wise W4A8
+
+static_assert(TINT4_WEIGHT_GROUP == kWeightGroup, "weight group of the ABI and the kernels");
+
+// Shape rules of the group-wise GEMM: the W4A8 rules plus K a multiple of
+// the weight group.
+tint4_status check_gw_mnk(int M, int N, int K) {
+    tint4_status s = check_mnk(M, N, K);
+    if (s != TINT4_OK) return s;
+    if (K % kWeightGroup != 0) return TINT4_ERR_UNSUPPORTED_SHAPE;
+    return TINT4_OK;
+}
+
+template <int G>
+void launch_pack_gw(const float* W, int N, int K, int asym, uint8_t* packed, float* scale,
+                    uint8_t* zero, cudaStream_t st) {
+    const long warps = static_cast<long>(N) * ((K + kQuantChunk - 1) / kQuantChunk);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const long grid = std::min<long>((warps + 7) / 8, 8L * num_sms(dev));
+    pack_weights_groupwise_kernel<G><<<static_cast<int>(grid), 256, 0, st>>>(W, N, K, asym, packed,
+                                                                            scale, zero);
+}
+
+// The tensor-core GEMM with group-wise scales at every M (gemm_tmem_gw.cuh).
+template <bool ASYM, bool EVOD>
+tint4_status launch_gemm_gw(const int8_t* codes, const float* tok_scale, const uint8_t* w,
+                            const float* wscale, const uint8_t* wzero, const __nv_bfloat16* bias,
+                            __nv_bfloat16* y, int M, int N, int K, cudaStream_t stream, bool pdl) {
+    auto kern = w4a8_gw_tmem_gemm_kernel<ASYM, EVOD>;
+    CUtensorMap ta, tw, ty;
+    bool ok = make_map_u8(&ta, codes, K, M, K, kGwBK, kGwBN, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && make_map_u8(&tw, w, K / 2, N, K / 2, kGwBK / 2, kGwBM, CU_TENSOR_MAP_SWIZZLE_64B);
+    ok = ok && make_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M,
+                           static_cast<uint64_t>(N) * 2, kGwBM, kGwBN, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!ok) return TINT4_ERR_CUDA;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static std::atomic<bool> attr_done[kMaxDevices];
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGwSmemBytes) != cudaSuccess) {
+            cudaGetLastError();
+            return TINT4_ERR_CUDA;
+        }
+        attr_done[dev].store(true, std::memory_order_release);
+    }
+    const int tiles = ((M + kGwBN - 1) / kGwBN) * ((N + kGwBM - 1) / kGwBM);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(std::min(tiles, num_sms(dev)), 1, 1);
+    cfg.blockDim = dim3(kGwThreads, 1, 1);
+    cfg.dynamicSmemBytes = kGwSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    if (pdl) {
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    const uint64_t wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tw, ty, tok_scale, wscale, wzero, bias, M, N, K,
+                           wait_ns) != cudaSuccess) {
+        cudaGetLastError();
+        return TINT4_ERR_CUDA;
+    }
+    return TINT4_OK;
+}
+
+template <bool EVOD>
+tint4_status launch_gemm_gw_any(const int8_t* codes, const float* tok_scale, const uint8_t* w,
+                                const float* wscale, const uint8_t* wzero, const tint4_bf16* bias,
+                                tint4_bf16* y, int M, int N, int K, cudaStream_t st, bool pdl) {
+    const auto* b = reinterpret_cast<const __nv_bfloat16*>(bias);
+    auto* yb = reinterpret_cast<__nv_bfloat16*>(y);
+    return wzero ? launch_gemm_gw<true, EVOD>(codes, tok_scale, w, wscale, wzero, b, yb, M, N, K,
+                                              st, pdl)
+                 : launch_gemm_gw<false, EVOD>(codes, tok_scale, w, wscale, nullptr, b, yb, M, N,
+                                               K, st, pdl);
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -779,6 +860,73 @@ tint4_status convrot_w4a8_linear_grouped(const tint4_bf16* x,
     return linear_codes_evod(M)
                ? launch_gemm_grouped<true>(codes, tok_scale, groups, num_groups, M, K, st, true)
                : launch_gemm_grouped(codes, tok_scale, groups, num_groups, M, K, st, true);
+}
+
+tint4_status tint4_pack_weights_groupwise(const float* W, int N, int K, int group, int asym,
+                                          uint8_t* w_packed, float* w_scale, uint8_t* w_zero,
+                                          void* stream) {
+    if (asym != 0 && asym != 1) return TINT4_ERR_INVALID_ARG;
+    tint4_status s = check_rq_shape(N, K, group);
+    if (s != TINT4_OK) return s;
+    if (K % kWeightGroup != 0) return TINT4_ERR_UNSUPPORTED_SHAPE;
+    if (N > 0 && (!W || !w_packed || !w_scale || (asym && !w_zero))) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(w_packed) || !aligned16(w_scale) || !aligned16(w_zero))
+        return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (N == 0) return TINT4_OK;
+    cudaStream_t st = as_stream(stream);
+    switch (group) {
+        case 0: launch_pack_gw<0>(W, N, K, asym, w_packed, w_scale, w_zero, st); break;
+        case 16: launch_pack_gw<16>(W, N, K, asym, w_packed, w_scale, w_zero, st); break;
+        case 64: launch_pack_gw<64>(W, N, K, asym, w_packed, w_scale, w_zero, st); break;
+        default: launch_pack_gw<256>(W, N, K, asym, w_packed, w_scale, w_zero, st); break;
+    }
+    return last_launch_status();
+}
+
+tint4_status w4a8_gemm_groupwise(const int8_t* a, const float* tok_scale,
+                                 const uint8_t* w_packed, const float* w_scale,
+                                 const uint8_t* w_zero, const tint4_bf16* bias, tint4_bf16* y,
+                                 int M, int N, int K, void* stream) {
+    tint4_status s = check_gw_mnk(M, N, K);
+    if (s != TINT4_OK) return s;
+    if (M > 0 && (!a || !tok_scale || !w_packed || !w_scale || !y)) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(tok_scale) || !aligned16(w_packed) || !aligned16(w_scale) ||
+        !aligned16(w_zero) || !aligned16(bias) || !aligned16(y))
+        return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (M == 0) return TINT4_OK;
+    return launch_gemm_gw_any<false>(a, tok_scale, w_packed, w_scale, w_zero, bias, y, M, N, K,
+                                     as_stream(stream), false);
+}
+
+tint4_status convrot_w4a8_linear_groupwise(const tint4_bf16* x, const uint8_t* w_packed,
+                                           const float* w_scale, const uint8_t* w_zero,
+                                           const tint4_bf16* bias, tint4_bf16* y, int M, int N,
+                                           int K, int group, void* workspace,
+                                           size_t workspace_bytes, void* stream) {
+    tint4_status s = check_gw_mnk(M, N, K);
+    if (s != TINT4_OK) return s;
+    if ((s = check_rq_shape(M, K, group)) != TINT4_OK) return s;
+    if (M > 0 && (!x || !w_packed || !w_scale || !y)) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_packed) || !aligned16(w_scale) || !aligned16(w_zero) ||
+        !aligned16(bias) || !aligned16(y))
+        return TINT4_ERR_MISALIGNED;
+    if (M > 0 && (!workspace || workspace_bytes < convrot_linear_workspace_size(M, K, 8)))
+        return TINT4_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (M == 0) return TINT4_OK;
+    int8_t* codes = static_cast<int8_t*>(workspace);
+    float* tok_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                                align_up(static_cast<size_t>(M) * K, 256));
+    cudaStream_t st = as_stream(stream);
+    // every M runs the tensor-core kernel: the codes always go in its even/odd order
+    launch_rq_g<__nv_bfloat16, 127, false, true>(reinterpret_cast<const __nv_bfloat16*>(x), M, K,
+                                                 group, codes, tok_scale, st);
+    if ((s = last_launch_status()) != TINT4_OK) return s;
+    return launch_gemm_gw_any<true>(codes, tok_scale, w_packed, w_scale, w_zero, bias, y, M, N, K,
+                                    st, true);
 }
 
 tint4_status tint4_quantize_weights_int8(const float* W, int N, int K, int group,

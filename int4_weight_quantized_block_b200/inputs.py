@@ -123,6 +123,10 @@ WORKLOADS = {
     # fused-QKV attention projection: 64x64 latent patches + 512 text tokens
     "dit_qkv_w4a8": dict(M=4608, K=3072, N=9216, group=256, act_bits=8, x="attn"),
     "dit_qkv_w4a4": dict(M=4608, K=3072, N=9216, group=256, act_bits=4, x="attn"),
+    # the same layer with group-wise asymmetric weights (scale + zero point per
+    # row and 128-wide K group)
+    "dit_qkv_w4a8_asym_g128": dict(M=4608, K=3072, N=9216, group=256, act_bits=8, x="attn",
+                                   weight_group=128, asym=True),
     # MLP pair, group 64
     "dit_mlp_up_w4a8": dict(M=4608, K=3072, N=12288, group=64, act_bits=8, x="attn"),
     "dit_mlp_down_w4a8": dict(M=4608, K=12288, N=3072, group=64, act_bits=8, x="gelu"),

@@ -146,6 +146,22 @@ def test_grouped_rules(lib):
                                            NULL) == 1                                  # group value
 
 
+def test_groupwise_rules(lib):
+    assert lib.tint4_pack_weights_groupwise(16, 4, 256, 0, 2, 16, 16, 16, NULL) == 1   # asym
+    assert lib.tint4_pack_weights_groupwise(16, 4, 96, 0, 0, 16, 16, NULL, NULL) == 2  # K % 128
+    assert lib.tint4_pack_weights_groupwise(16, 4, 256, 0, 1, 16, 16, NULL, NULL) == 1  # no zero
+    assert lib.tint4_pack_weights_groupwise(16, 4, 256, 0, 0, 16, 17, NULL, NULL) == 3
+    assert lib.w4a8_gemm_groupwise(16, 16, 16, 16, NULL, NULL, 16, 4, 32, 160, NULL) == 2
+    assert lib.w4a8_gemm_groupwise(16, 16, 16, 16, NULL, NULL, 16, 4, 24, 256, NULL) == 2
+    assert lib.w4a8_gemm_groupwise(NULL, 16, 16, 16, NULL, NULL, 16, 4, 32, 256, NULL) == 1
+    assert lib.w4a8_gemm_groupwise(16, 16, 16, 16, 17, NULL, 16, 4, 32, 256, NULL) == 3
+    need = lib.convrot_linear_workspace_size(4, 256, 8)
+    assert lib.convrot_w4a8_linear_groupwise(16, 16, 16, NULL, NULL, 16, 4, 32, 256, 256, 256,
+                                             need - 1, NULL) == 6
+    assert lib.convrot_w4a8_linear_groupwise(16, 16, 16, NULL, NULL, 16, 4, 32, 256, 32, 256,
+                                             need, NULL) == 1                           # group value
+
+
 def test_debug_entries_rules(lib):
     assert lib.tint4_debug_int32_gemm(16, 6, 16, 16, 4, 256, 256, NULL) == 1
     assert lib.tint4_debug_bounded_wait(10, NULL) == 1

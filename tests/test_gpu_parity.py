@@ -439,6 +439,114 @@ def test_gemm_grouped_full_size_qkv_split():
         assert torch.equal(yg, y[:, i * third:(i + 1) * third])
 
 
+# ------------------------------------------------------------------ group-wise W4A8
+
+def assert_groupwise_output(y_gpu_bits, y64, mag, K):
+    """bf16 outputs against the oracle: the fp32 evaluation (one rounding per
+    weight group in the running sum, then the token scale and the bias) is
+    within (K / 128 + 3) 2^-24 of the size of the terms it adds up."""
+    err = (K // t4.WEIGHT_GROUP + 3) * 2.0 ** -24 * mag
+    c = check_bf16(y_gpu_bits, y64, err)
+    assert c.ok, str(c)
+
+
+@pytest.mark.parametrize("asym", [False, True])
+@pytest.mark.parametrize("N,K,g", [(16, 128, 0), (48, 384, 16), (272, 640, 64), (400, 1024, 256)])
+def test_pack_weights_groupwise_bit_exact(N, K, g, asym):
+    W = inputs.weights(N, K, seed=800 + K)
+    W[0, :128] = np.abs(W[0, :128])     # a group with no negative value
+    W[1, :128] = -np.abs(W[1, :128])    # and one with no positive value
+    W[2, 128:256 if K >= 256 else 128] = 0.0
+    wp_ref, s_ref, z_ref, _ = oracle.pack_weights_groupwise(W, g, 128, asym)
+    wp, s, z = t4.tint4_pack_weights_groupwise(to_gpu(W), g, asym)
+    torch.cuda.synchronize()
+    assert np.array_equal(wp.cpu().numpy(), wp_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    if asym:
+        assert np.array_equal(z.cpu().numpy(), z_ref)
+    else:
+        assert z is None
+
+
+@pytest.mark.parametrize("asym", [False, True])
+@pytest.mark.parametrize("M,N,K", [(1, 16, 128), (5, 272, 384), (130, 144, 256), (300, 400, 1024),
+                                   (129, 128, 2048)])
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_gemm_groupwise(M, N, K, asym, with_bias):
+    """Tiles, ragged M / N tails and 1 to 16 weight groups per row."""
+    x = inputs.activations(M, K, seed=810 + M)
+    codes, st, _ = oracle.quantize_act(x, 64, 8)
+    wp, s, z, _ = oracle.pack_weights_groupwise(inputs.weights(N, K, seed=811 + N), 64, 128, asym)
+    b = (inputs.f32_to_bf16_bits(np.linspace(-2, 2, N, dtype=np.float32)) if with_bias else None)
+    y = t4.w4a8_gemm_groupwise(to_gpu(codes), to_gpu(st), to_gpu(wp), to_gpu(s),
+                               to_gpu(z) if asym else None, bf16_to_gpu(b) if with_bias else None)
+    torch.cuda.synchronize()
+    y64, mag = oracle.gemm_groupwise_f64(codes, st, wp, s, z, b)
+    assert_groupwise_output(bf16_from_gpu(y), y64, mag, K)
+
+
+@pytest.mark.parametrize("asym", [False, True])
+@pytest.mark.parametrize("M,N,K,g", [(1, 256, 256, 256), (17, 272, 384, 64), (200, 528, 1024, 16)])
+def test_linear_groupwise(M, N, K, g, asym):
+    """The fused linear (codes in the private even/odd order) gives the bits
+    of quantize + GEMM (natural order), which match the oracle."""
+    x_np = inputs.activations(M, K, seed=820 + M)
+    x = bf16_to_gpu(x_np)
+    wp, s, z = t4.tint4_pack_weights_groupwise(to_gpu(inputs.weights(N, K, seed=821 + N)), g, asym)
+    b = bf16_to_gpu(inputs.f32_to_bf16_bits(np.linspace(-1, 1, N, dtype=np.float32)))
+    codes, st = t4.convrot_quantize_act(x, g, 8)
+    y0 = t4.w4a8_gemm_groupwise(codes, st, wp, s, z, b)
+    y1 = t4.convrot_w4a8_linear_groupwise(x, wp, s, g, z, b)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)
+    qa, st_ref, _ = oracle.quantize_act(x_np, g, 8)
+    frac, dmax = code_mismatch(codes.cpu().numpy(), qa)
+    assert frac <= CODE_MISMATCH_FRAC and dmax <= 1
+    y64, mag = oracle.gemm_groupwise_f64(codes.cpu().numpy(), st.cpu().numpy(), wp.cpu().numpy(),
+                                         s.cpu().numpy(), None if z is None else z.cpu().numpy(),
+                                         b.view(torch.int16).cpu().numpy().view(np.uint16))
+    assert_groupwise_output(bf16_from_gpu(y1), y64, mag, K)
+
+
+def test_groupwise_equal_scales_match_per_row_gemm():
+    """Symmetric group-wise weights whose group scales all equal the row
+    scale compute the per-row W4A8 layer (same codes): outputs within the
+    two kernels' evaluation bounds of each other."""
+    M, N, K, g = 256, 384, 1024, 64
+    x = bf16_to_gpu(inputs.activations(M, K, seed=830))
+    wp, sr = t4.tint4_pack_weights(to_gpu(inputs.weights(N, K, seed=831)), g)
+    s = sr[:, None].expand(N, K // 128).contiguous()
+    codes, st = t4.convrot_quantize_act(x, g, 8)
+    y_gw = t4.w4a8_gemm_groupwise(codes, st, wp, s)
+    y_row = t4.w4a8_gemm(codes, st, wp, sr)
+    torch.cuda.synchronize()
+    d = (y_gw.float() - y_row.float()).abs().max().item()
+    assert d <= 2 * 2.0 ** -8 * y_row.float().abs().max().item()
+
+
+def test_groupwise_full_size_sampled():
+    """The DiT QKV layer with asymmetric group-wise weights at full size:
+    packing bit-exact (all of it), the fused linear on sampled outputs the
+    oracle computes one by one."""
+    name = "dit_qkv_w4a8_asym_g128"
+    w = inputs.WORKLOADS[name]
+    M, N, K, g = w["M"], w["N"], w["K"], w["group"]
+    x_np, W = inputs.layer_inputs(name)
+    wp_ref, s_ref, z_ref, _ = oracle.pack_weights_groupwise(W, g, 128, True)
+    wp, s, z = t4.tint4_pack_weights_groupwise(to_gpu(W), g, True)
+    x = bf16_to_gpu(x_np)
+    y = t4.convrot_w4a8_linear_groupwise(x, wp, s, g, z)
+    codes, st = t4.convrot_quantize_act(x, g, 8)
+    torch.cuda.synchronize()
+    assert np.array_equal(wp.cpu().numpy(), wp_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(z.cpu().numpy(), z_ref)
+    pairs = _sample_pairs(M, N, 4096, seed=11)
+    y64, mag = oracle.gemm_groupwise_sampled_f64(codes.cpu().numpy(), st.cpu().numpy(), wp_ref,
+                                                 s_ref, pairs, z_ref)
+    assert_groupwise_output(bf16_from_gpu(y)[pairs[:, 0], pairs[:, 1]], y64, mag, K)
+
+
 # ------------------------------------------------------------------ W4A16
 
 @pytest.mark.parametrize("M,N,K", [(1, 16, 128), (4, 272, 384), (16, 512, 1024),
