@@ -694,6 +694,18 @@ def run_profile_case(case: str, dev):
                 t4.convrot_quantize_act(x, g, bits, codes, st)
             else:
                 gemm()
+    elif case == "qkv_gemm_gw":
+        # the group-wise GEMM (asymmetric weights) on the QKV layer
+        name = "dit_qkv_w4a8_asym_g128"
+        w = inputs.WORKLOADS[name]
+        M, N, K, g = w["M"], w["N"], w["K"], w["group"]
+        x_np, W_np = inputs.layer_inputs(name)
+        x = bf16_gpu(x_np, dev)
+        wp, s, z = t4.tint4_pack_weights_groupwise(torch.from_numpy(W_np).to(dev), g, True)
+        codes, st = t4.convrot_quantize_act(x, g, 8)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            t4.w4a8_gemm_groupwise(codes, st, wp, s, z, None, y)
     elif case.startswith("decode_w4a8_M"):
         M = int(case[len("decode_w4a8_M"):])
         w = inputs.WORKLOADS["te_decode_w4a8"]
@@ -729,7 +741,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--profile", default=None,
                     help="run only a few launches of one kernel for ncu: qkv_gemm, "
-                         "qkv_gemm_w4a4, qkv_quantize, w4a16_M<m>, decode_w4a8_M<m>")
+                         "qkv_gemm_w4a4, qkv_gemm_gw, qkv_quantize, w4a16_M<m>, "
+                         "decode_w4a8_M<m>")
     args = ap.parse_args()
     if args.profile:
         dev = torch.device("cuda", 0)

@@ -14,22 +14,23 @@
 // (producer warp, one MMA-issuing thread, 8 unpack warps widening the packed
 // weights into TMEM A stages, the activation codes as the MMA's B operand in
 // shared memory), with these differences:
-//  * tiles of 128 weight rows x 128 tokens; TMEM holds three int32 group-sum
-//    buffers (P0, P1, P2: K step j uses buffer j % 3, so the MMAs run up to
-//    two steps ahead of the fold) and the fp32 running sums (R): 4 x 128 =
-//    512 columns.  The widened weights therefore go to shared memory (a
-//    128-byte swizzled int8 tile per stage, the MMA's A operand, both
-//    operands from shared memory);
-//  * the group sums start from 1.5 * 2^23 (bits 0x4B400000, stored by the
-//    fold warps when they hand a buffer back), so every MMA accumulates and a
-//    finished sum p reads, as an fp32 bit pattern, exactly 1.5 * 2^23 + p
-//    (|p| < 2^22): the fold is one subtraction and one FMA per value
-//    (r = fma(s_j / 16, (bits - 1.5 * 2^23), r)), no integer conversion;
-//  * warps 10-17 fold: they wait for the MMAs of a step (the stage-empty
-//    commit), fold the step's group sums into R, refill the buffer with the
-//    start value and release it to the unpack warps of the step three ahead
-//    (which wait for it before they signal their A stage, so the MMA issuer
-//    still waits on one barrier per step).  After a tile's last step they
+//  * tiles of 128 weight rows x 128 tokens; TMEM holds three int32
+//    group-sum buffers (K step j uses buffer j % 3, so the MMAs run up to two
+//    steps ahead of the fold) and the 4 A stages: 3 x 128 + 4 x 32 = 512
+//    columns; the fp32 running sums live in the fold warps' registers (16
+//    warps, 32 of a row's 128 tokens each);
+//  * each step's first MMA overwrites its group-sum buffer; the fold turns a
+//    finished sum p into fp32 without the conversion unit: p + 0x4B400000
+//    (an integer add) is the bit pattern of the float 1.5 * 2^23 + p when
+//    |p| < 2^22, and subtracting 1.5 * 2^23 leaves p exactly; then one FMA
+//    per value, r = fma(s_j / 16, p, r), r starting at +0.  (Refilling the
+//    buffers with that
+//    start value from the fold warps, so that the MMAs add onto it, took
+//    TMEM store bandwidth and ran about 6 % slower);
+//  * warps 10-25 fold: they wait for the MMAs of a step (the stage-empty
+//    commit), fold the step's group sums into their running sums and release
+//    the buffer to the MMA issuer, which waits for it (and for the step's A
+//    stage) before the step's MMAs.  After a tile's last step they
 //    scale by the token scales, add the bias, round to bf16 into a staging
 //    tile and one thread stores it with a TMA tensor store (rows and columns
 //    outside y are clipped by the TMA unit);
@@ -41,7 +42,7 @@
 //    The fold scale is s_j / 8 (s_j / 16 for the symmetric x16 form).
 //
 // Ranges: |p| <= 128 * 127 * 7 * 16 (symmetric) or 128 * 127 * 15 * 8
-// (asymmetric), both below 2^22, so the start value trick is exact.
+// (asymmetric), both below 2^22, so the conversion above is exact.
 #pragma once
 
 #include "gemm_tmem.cuh"
@@ -53,19 +54,18 @@ constexpr int kGwBM = 128;                    // weight rows per tile (UMMA M)
 constexpr int kGwBN = 128;                    // tokens per tile (UMMA N)
 constexpr int kGwBK = kWeightGroup;           // K per step: one weight group
 constexpr int kGwStages = 4;                  // shared-memory stages = TMEM A stages
-constexpr int kGwThreads = 576;               // 18 warps
+constexpr int kGwFoldWarps = 16;
+constexpr int kGwThreads = (10 + kGwFoldWarps) * 32;   // 26 warps
 constexpr int kGwActBytes = kGwBN * kGwBK;    // 16 KB
 constexpr int kGwWBytes = kGwBM * kGwBK / 2;  // 8 KB packed weights
-constexpr int kGwUBytes = kGwBM * kGwBK;      // 16 KB widened weights (A operand)
 constexpr int kGwOutBytes = kGwBN * kGwBM * 2;   // 32 KB bf16 staging tile
-constexpr int kGwSmemBytes =
-    kGwStages * (kGwActBytes + kGwWBytes + kGwUBytes) + kGwOutBytes + 256 + 1024;
+constexpr int kGwSmemBytes = kGwStages * (kGwActBytes + kGwWBytes) + kGwOutBytes + 256 + 1024;
 static_assert(kGwSmemBytes <= 227 * 1024, "shared memory budget");
 constexpr int kGwPBufs = 3;                   // group-sum buffers
 constexpr uint32_t kGwColP = 0;               // group sums, buffer b at 128 b
-constexpr uint32_t kGwColR = kGwPBufs * kGwBN;   // fp32 running sums
-static_assert(kGwColR + kGwBN <= 512, "TMEM budget");
-constexpr uint32_t kGwStart = 0x4B400000u;    // 1.5 * 2^23 as fp32 bits
+constexpr uint32_t kGwColA = kGwPBufs * kGwBN;   // A stage s at kGwColA + 32 s
+static_assert(kGwColA + 32 * kGwStages <= 512, "TMEM budget");
+constexpr uint32_t kGwStart = 0x4B400000u;    // 1.5 * 2^23 as fp32 bits (the conversion)
 
 // 8 unsigned nibbles q (K order, low nibble first) with zero point z ->
 // 8 int8 values 8 (q - z), even/odd K order; zc = (128 - 8 z) * 0x01010101.
@@ -73,17 +73,6 @@ __device__ __forceinline__ void unpack8_asym_evod(uint32_t w, uint32_t zc, uint3
                                                   uint32_t& hi) {
     lo = (((w << 3) & 0x78787878u) + zc) ^ 0x80808080u;
     hi = (((w >> 1) & 0x78787878u) + zc) ^ 0x80808080u;
-}
-
-// warp_wait with the non-suspending poll
-__device__ __forceinline__ bool warp_wait_spin(uint64_t* bar, uint32_t parity,
-                                               volatile uint32_t* abort, uint64_t limit_ns,
-                                               unsigned err) {
-    const int lane = threadIdx.x & 31;
-    int ok = 0;
-    if (lane == 0) ok = mbar_wait_bounded_spin(bar, parity, abort, limit_ns, err) ? 1 : 0;
-    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-    return ok != 0;
 }
 
 // ASYM: unsigned nibbles with zero points (wzero [N, K/128]); else signed.
@@ -105,12 +94,11 @@ w4a8_gw_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* sAct = smem;
     uint8_t* sW = smem + kS * kGwActBytes;
-    uint8_t* sU = sW + kS * kGwWBytes;      // widened weights, 1024-byte aligned stages
-    uint8_t* sOut = sU + kS * kGwUBytes;
+    uint8_t* sOut = sW + kS * kGwWBytes;
     uint64_t* act_full = reinterpret_cast<uint64_t*>(sOut + kGwOutBytes);
     uint64_t* empty = act_full + kS;        // [kS] MMAs of the stage done (commit)
-    uint64_t* a_full = empty + kS;          // [kS] widened weights written (4 warp arrivals)
-    uint64_t* p_free = a_full + kS;         // [3] group-sum buffer folded + refilled (8 warps)
+    uint64_t* a_full = empty + kS;          // [kS] TMEM A stage written (4 warp arrivals)
+    uint64_t* p_free = a_full + kS;         // [3] group-sum buffer folded (16 warp arrivals)
     uint64_t* final_bar = p_free + kGwPBufs;   // all MMAs done (teardown)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
@@ -130,7 +118,7 @@ w4a8_gw_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             mbar_init(&empty[s], 1);
             mbar_init(&a_full[s], 4);
         }
-        for (int b = 0; b < kGwPBufs; ++b) mbar_init(&p_free[b], 8);
+        for (int b = 0; b < kGwPBufs; ++b) mbar_init(&p_free[b], kGwFoldWarps);
         mbar_init(final_bar, 1);
         *abort_flag = 0u;
         fence_mbarrier_init();
@@ -184,24 +172,28 @@ w4a8_gw_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
         if (lane == 0) {
             constexpr uint32_t idesc = umma_idesc_i8(kGwBM, kGwBN);
             const uint64_t bdesc0 = umma_desc_sw128(smem_u32(sAct));
-            const uint64_t adesc0 = umma_desc_sw128(smem_u32(sU));
             int j = 0;
             bool ok = true;
             for (int i = 0; i < my_tiles && ok; ++i) {
                 for (int kt = 0; kt < KT; ++kt, ++j) {
                     const int s = j % kS;
-                    // the unpack warps arrive only after the stage landed and
-                    // the step's group-sum buffer was handed back
+                    // the step's A stage (the unpack warps arrive only after the
+                    // stage landed), then its group-sum buffer, folded
                     if (!mbar_wait_bounded(&a_full[s], (j / kS) & 1, abort_flag, wait_ns,
                                            kDevErrTimeoutConsumer)) {
                         ok = false;
                         break;
                     }
+                    if (!mbar_wait_bounded(&p_free[j % kGwPBufs], (j / kGwPBufs) & 1, abort_flag,
+                                           wait_ns, kDevErrTimeoutConsumer)) {
+                        ok = false;
+                        break;
+                    }
                     tcgen05_fence_after();
                     const uint32_t d_tmem = tmem_base + kGwColP + (j % kGwPBufs) * kGwBN;
-                    const uint64_t adesc = adesc0 + static_cast<uint64_t>(s * (kGwUBytes >> 4));
+                    const uint32_t a_tmem = tmem_base + kGwColA + 32 * s;
                     const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(s * (kGwActBytes >> 4));
-                    umma_i8_ss_step(d_tmem, adesc, bdesc, idesc, 1u);   // onto the start value
+                    umma_i8_ts_step(d_tmem, a_tmem, bdesc, idesc, 0u);   // a fresh group sum
                     umma_commit(&empty[s]);
                 }
             }
@@ -211,7 +203,7 @@ w4a8_gw_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
         }
         __syncwarp();
     } else if (warp < 10) {
-        // ------------------------------------------------ weight unpack -> shared (warps 2-9)
+        // ------------------------------------------------ weight unpack -> TMEM (warps 2-9)
         const int q = warp & 3;
         const int r = q * 32 + lane;
         const int total = my_tiles * KT;
@@ -228,6 +220,9 @@ w4a8_gw_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             if (!warp_wait(&act_full[s], (j / kS) & 1, abort_flag, wait_ns, kDevErrTimeoutConsumer))
                 break;
             const uint8_t* row = sW + s * kGwWBytes + r * 64;
+            // 128 K values of row r into the TMEM A stage s (the MMAs of step
+            // j - 4, its last readers, completed before the producer refilled
+            // shared-memory stage s)
             uint32_t a[32];
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -247,52 +242,38 @@ w4a8_gw_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                     a[8 * v + 2 * u + 1] = hi;
                 }
             }
-            // row r of the 128-byte swizzled A tile: 16-byte chunk c at c ^ (r & 7)
-            // (the MMAs of step j - 4, the tile's last readers, completed before
-            // the producer refilled this stage)
-            uint8_t* urow = sU + s * kGwUBytes + r * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                sts128(urow + ((c ^ (r & 7)) << 4),
-                       make_uint4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]));
-            fence_proxy_async_smem();   // generic-proxy writes -> tensor-core reads
-            // the group-sum buffer of this step: its previous use (step j - 3)
-            // folded and refilled with the start value
-            if (!warp_wait(&p_free[j % kGwPBufs], (j / kGwPBufs) & 1, abort_flag, wait_ns,
-                           kDevErrTimeoutConsumer))
-                break;
+            tcgen05_fence_after();
+            tmem_st_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kGwColA + 32 * s,
+                               a);
+            tmem_st_wait();
+            tcgen05_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&a_full[s]);
         }
-    } else if (warp < 18) {
-        // ------------------------------------------------ fold + epilogue (warps 10-17)
-        const int e = warp - 10;
-        const int q = warp & 3;
-        const int half = e >> 2;                // tokens [64 half, 64 half + 64) of the tile
+    } else if (warp < 10 + kGwFoldWarps) {
+        // ------------------------------------------------ fold + epilogue (warps 10-25)
+        const int e = warp - 10;                // 0..15
+        const int q = warp & 3;                 // TMEM lane quarter
+        const int part = e >> 2;                // tokens [32 part, 32 part + 32) of the tile
         const int r = q * 32 + lane;            // weight row in the tile = output column
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const bool leader = (e == 0 && lane == 0);
+        constexpr uint32_t kFoldThreads = kGwFoldWarps * 32;
         constexpr float kUnscale = ASYM ? 0.125f : 0.0625f;
         constexpr float kStartF = 12582912.0f;   // 1.5 * 2^23
-        // every group-sum buffer starts at the start value
-#pragma unroll
-        for (int b = 0; b < kGwPBufs; ++b)
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-                tmem_st_32x32b_x32_fill(
-                    tmem_base + lane_base + kGwColP + b * kGwBN + half * 64 + c * 32, kGwStart);
-        tmem_st_wait();
-        tcgen05_fence_before();
-        __syncwarp();
+        // every group-sum buffer is free at the start
         if (lane == 0)
             for (int b = 0; b < kGwPBufs; ++b) mbar_arrive(&p_free[b]);
         int j = 0;
         // after a failed wait a fold warp goes on through every step without
         // waiting (its values are then meaningless and the call reports the
-        // error), so all 8 warps meet at the same named barriers
+        // error), so all fold warps meet at the same named barriers
         bool ok = true;
         bool stored = false;   // a TMA store of the staging tile is in flight (leader)
+        float acc[32];         // running sums: row r, tokens 32 part + x
         for (int i = 0; i < my_tiles; ++i) {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) acc[x] = 0.0f;
             const int tile = blockIdx.x + i * gridDim.x;
             const int m0 = (tile % m_tiles) * kGwBN, n0 = (tile / m_tiles) * kGwBM;
             const int n = n0 + r;
@@ -302,82 +283,63 @@ w4a8_gw_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             for (int kt = 0; kt < KT; ++kt, ++j) {
                 const float sg = sg_next;
                 if (kt + 1 < KT) sg_next = row_ok ? __ldg(srow + kt + 1) * kUnscale : 0.0f;
-                const bool first = kt == 0, last = kt == KT - 1;
-                if (ok && !warp_wait_spin(&empty[j % kS], (j / kS) & 1, abort_flag, wait_ns,
-                                          kDevErrTimeoutEpilogue))
+                if (ok && !warp_wait(&empty[j % kS], (j / kS) & 1, abort_flag, wait_ns,
+                                     kDevErrTimeoutEpilogue))
                     ok = false;
                 tcgen05_fence_after();
-                float b = 0.0f;
-                if (last) {
-                    // the staging tile is free once the previous tile's store read it
-                    if (leader && stored) bulk_wait_group_read0();
-                    named_barrier_sync(1, 256);
-                    b = (row_ok && bias != nullptr) ? __bfloat162float(bias[n]) : 0.0f;
-                }
                 const uint32_t pcol =
-                    tmem_base + lane_base + kGwColP + (j % kGwPBufs) * kGwBN + half * 64;
-                const uint32_t rcol = tmem_base + lane_base + kGwColR + half * 64;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {   // 16 columns at a time (registers)
+                    tmem_base + lane_base + kGwColP + (j % kGwPBufs) * kGwBN + part * 32;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {   // 16 columns at a time (registers)
                     uint32_t p[16];
-                    uint32_t acc[16];
                     tmem_ld_32x32b_x16(pcol + c * 16, p);
-                    if (!first) tmem_ld_32x32b_x16(rcol + c * 16, acc);
                     tmem_ld_wait();
-                    if (c % 2 == 1) tmem_st_32x32b_x32_fill(pcol + (c - 1) * 16, kGwStart);
 #pragma unroll
                     for (int x = 0; x < 16; ++x) {
-                        const float d = __fsub_rn(__uint_as_float(p[x]), kStartF);   // exact
-                        const float rr = first ? __fmul_rn(sg, d)
-                                               : __fmaf_rn(sg, d, __uint_as_float(acc[x]));
-                        acc[x] = __float_as_uint(rr);
-                    }
-                    if (!last) {
-                        tmem_st_32x32b_x16(rcol + c * 16, acc);
-                    } else {
-                        // y = r * s_tok + bias -> bf16 into the staging tile
-                        // (row = token, 256 bytes; column = this thread's row)
-                        const int t0 = half * 64 + c * 16;
-                        const int mb = m0 + t0;
-                        uint8_t* dst = sOut + t0 * (kGwBM * 2) + r * 2;
-#pragma unroll
-                        for (int x = 0; x < 16; x += 4) {
-                            float4 st4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                            if (mb + x + 3 < M) {
-                                st4 = __ldg(reinterpret_cast<const float4*>(tok_scale + mb + x));
-                            } else {
-                                if (mb + x < M) st4.x = __ldg(tok_scale + mb + x);
-                                if (mb + x + 1 < M) st4.y = __ldg(tok_scale + mb + x + 1);
-                                if (mb + x + 2 < M) st4.z = __ldg(tok_scale + mb + x + 2);
-                            }
-                            const float sv[4] = {st4.x, st4.y, st4.z, st4.w};
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                const float y = __fmaf_rn(__uint_as_float(acc[x + u]), sv[u], b);
-                                const __nv_bfloat16 h = __float2bfloat16_rn(y);
-                                asm volatile("st.shared.b16 [%0], %1;" ::"r"(
-                                                 smem_u32(dst + (x + u) * (kGwBM * 2))),
-                                             "h"(*reinterpret_cast<const unsigned short*>(&h))
-                                             : "memory");
-                            }
-                        }
+                        // = p, exactly; then acc += s_j p, one rounding
+                        const float d = __fsub_rn(__uint_as_float(p[x] + kGwStart), kStartF);
+                        acc[16 * c + x] = __fmaf_rn(sg, d, acc[16 * c + x]);
                     }
                 }
-                // the buffer holds the start value again: the unpack warps of
-                // step j + 3 may hand it to the MMAs
+                // hand the buffer back: the MMAs of step j + 3 may overwrite it
                 tmem_st_wait();
                 tcgen05_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_free[j % kGwPBufs]);
-                if (last) {
-                    fence_proxy_async_smem();   // staging writes -> the TMA unit
-                    named_barrier_sync(1, 256);
-                    if (leader) {
-                        tma_store_2d(&tmap_y, sOut, n0, m0);
-                        bulk_commit_group();
-                        stored = true;
-                    }
+            }
+            // ---- epilogue: y = r * s_tok + bias -> bf16 staging tile (row =
+            // token, 256 bytes; column = this thread's row) -> one TMA store
+            if (leader && stored) bulk_wait_group_read0();   // previous store read the tile
+            named_barrier_sync(1, kFoldThreads);
+            const float b = (row_ok && bias != nullptr) ? __bfloat162float(bias[n]) : 0.0f;
+            const int t0 = part * 32;
+            const int mb = m0 + t0;
+            uint8_t* dst = sOut + t0 * (kGwBM * 2) + r * 2;
+#pragma unroll
+            for (int x = 0; x < 32; x += 4) {
+                float4 st4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                if (mb + x + 3 < M) {
+                    st4 = __ldg(reinterpret_cast<const float4*>(tok_scale + mb + x));
+                } else {
+                    if (mb + x < M) st4.x = __ldg(tok_scale + mb + x);
+                    if (mb + x + 1 < M) st4.y = __ldg(tok_scale + mb + x + 1);
+                    if (mb + x + 2 < M) st4.z = __ldg(tok_scale + mb + x + 2);
                 }
+                const float sv[4] = {st4.x, st4.y, st4.z, st4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const __nv_bfloat16 h = __float2bfloat16_rn(__fmaf_rn(acc[x + u], sv[u], b));
+                    asm volatile("st.shared.b16 [%0], %1;" ::"r"(smem_u32(dst + (x + u) * (kGwBM * 2))),
+                                 "h"(*reinterpret_cast<const unsigned short*>(&h))
+                                 : "memory");
+                }
+            }
+            fence_proxy_async_smem();   // staging writes -> the TMA unit
+            named_barrier_sync(1, kFoldThreads);
+            if (leader) {
+                tma_store_2d(&tmap_y, sOut, n0, m0);
+                bulk_commit_group();
+                stored = true;
             }
         }
         if (leader && stored) bulk_wait_group0();
