@@ -590,6 +590,31 @@ def bench_rows(args, t4, inputs, dev, flush, pk, int8_peak):
             "gemm_frac_hbm_chained": round(g_bytes / g_ms_pf / 1e6 / pk["hbm"], 4),
             "timing": "64 calls in one CUDA graph, 8 weight copies rotated (201 MB > L2); "
                       "_chained: with tint4_set_decode_weight_prefetch(1)"}
+    del wcopies, wp0, sr0
+
+    # the same decode layer with group-wise asymmetric weights (scale + zero
+    # point per row and 128-wide K group): the streaming kernel's GEMM
+    W_dev = torch.from_numpy(inputs.layer_inputs("te_decode_w4a8", M=1)[1]).to(dev)
+    gw0 = t4.tint4_pack_weights_groupwise(W_dev, g, True)
+    del W_dev
+    gcopies = [tuple(t.clone() for t in gw0) for _ in range(8)]
+    for M in w["Ms"]:
+        x = bf16_gpu(inputs.activations(M, K, inputs.SEED), dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        codes, st = t4.convrot_quantize_act(x, g, 8)
+
+        def gwg(i):
+            wp, s, z = gcopies[i % len(gcopies)]
+            t4.w4a8_gemm_groupwise(codes, st, wp, s, z, None, y)
+
+        g_ms = graph_time(gwg, 64, dev)
+        g_bytes = N * K // 2 + N * (K // 128) * 5 + M * K + M * 4 + M * N * 2
+        rows[f"te_decode_w4a8_asym_g128_M{M}"] = {
+            "kernel": "w4a8_small_kernel<group-wise asymmetric>", "M": M, "N": N, "K": K,
+            "group": g, "weight_group": t4.WEIGHT_GROUP,
+            "gemm_us": round(g_ms * 1e3, 2), "gemm_GBps": round(g_bytes / g_ms / 1e6, 1),
+            "gemm_frac_hbm": round(g_bytes / g_ms / 1e6 / pk["hbm"], 4),
+            "timing": "64 calls in one CUDA graph, 8 weight copies rotated (>200 MB > L2)"}
     return rows
 
 

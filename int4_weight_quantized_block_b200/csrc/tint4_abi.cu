@@ -304,7 +304,8 @@ tint4_status launch_gemm_small(const void* a, const uint8_t* w, const float* st,
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, tw, static_cast<const uint8_t*>(a), st, sr, bias, out, M,
                            N, K, 0xF0F0F0F0u, g_decode_prefetch.load(std::memory_order_relaxed),
-                           g_wait_limit_ns.load(std::memory_order_relaxed)) != cudaSuccess) {
+                           g_wait_limit_ns.load(std::memory_order_relaxed),
+                           static_cast<const uint8_t*>(nullptr)) != cudaSuccess) {
         cudaGetLastError();
         return TINT4_ERR_CUDA;
     }
@@ -348,7 +349,8 @@ tint4_status launch_linear_small_fused(const __nv_bfloat16* x, const uint8_t* w,
     if (cudaLaunchKernelEx(&cfg, kern, tw, reinterpret_cast<const uint8_t*>(x),
                            static_cast<const float*>(nullptr), sr, bias, static_cast<void*>(y), M,
                            N, K, 0xF0F0F0F0u, g_decode_prefetch.load(std::memory_order_relaxed),
-                           g_wait_limit_ns.load(std::memory_order_relaxed)) != cudaSuccess) {
+                           g_wait_limit_ns.load(std::memory_order_relaxed),
+                           static_cast<const uint8_t*>(nullptr)) != cudaSuccess) {
         cudaGetLastError();
         return TINT4_ERR_CUDA;
     }
@@ -726,12 +728,68 @@ tint4_status launch_gemm_gw(const int8_t* codes, const float* tok_scale, const u
     return TINT4_OK;
 }
 
+// Small M (<= kS8MaxM tokens, natural-order codes): the streaming kernel
+// with group-wise scales (w4a8_small.cuh, GW = 1 symmetric / 2 asymmetric).
+template <int NB, int GW>
+tint4_status launch_gemm_small_gw(const int8_t* a, const uint8_t* w, const float* st,
+                                  const float* wscale, const uint8_t* wzero,
+                                  const __nv_bfloat16* bias, __nv_bfloat16* y, int M, int N, int K,
+                                  cudaStream_t stream, bool pdl) {
+    auto kern = w4a8_small_kernel<NB, false, false, 0, 0, GW>;
+    CUtensorMap tw;
+    if (!make_map_u8(&tw, w, K / 2, N, K / 2, 128, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+        return TINT4_ERR_CUDA;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static std::atomic<bool> attr_done[kMaxDevices];
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 S8Cfg<NB>::SMEM) != cudaSuccess) {
+            cudaGetLastError();
+            return TINT4_ERR_CUDA;
+        }
+        attr_done[dev].store(true, std::memory_order_release);
+    }
+    const int nblk = N / 16;
+    const int sms = num_sms(dev);
+    const int grid = nblk <= kS8MB * sms ? std::min(sms, nblk) : (nblk + kS8MB - 1) / kS8MB;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(S8Cfg<NB>::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = S8Cfg<NB>::SMEM;
+    cfg.stream = stream;
+    (void)pdl;   // always programmatic, as launch_gemm_small
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tw, reinterpret_cast<const uint8_t*>(a), st, wscale, bias,
+                           static_cast<void*>(y), M, N, K, 0xF0F0F0F0u,
+                           g_decode_prefetch.load(std::memory_order_relaxed),
+                           g_wait_limit_ns.load(std::memory_order_relaxed), wzero) != cudaSuccess) {
+        cudaGetLastError();
+        return TINT4_ERR_CUDA;
+    }
+    return last_launch_status();
+}
+
 template <bool EVOD>
 tint4_status launch_gemm_gw_any(const int8_t* codes, const float* tok_scale, const uint8_t* w,
                                 const float* wscale, const uint8_t* wzero, const tint4_bf16* bias,
                                 tint4_bf16* y, int M, int N, int K, cudaStream_t st, bool pdl) {
     const auto* b = reinterpret_cast<const __nv_bfloat16*>(bias);
     auto* yb = reinterpret_cast<__nv_bfloat16*>(y);
+    if (M <= kS8MaxM) {
+        if (EVOD) return TINT4_ERR_INVALID_ARG;   // the streaming kernel reads natural-order codes
+        if (M <= 8)
+            return wzero ? launch_gemm_small_gw<1, 2>(codes, w, tok_scale, wscale, wzero, b, yb, M,
+                                                      N, K, st, pdl)
+                         : launch_gemm_small_gw<1, 1>(codes, w, tok_scale, wscale, nullptr, b, yb,
+                                                      M, N, K, st, pdl);
+        return wzero ? launch_gemm_small_gw<2, 2>(codes, w, tok_scale, wscale, wzero, b, yb, M, N,
+                                                  K, st, pdl)
+                     : launch_gemm_small_gw<2, 1>(codes, w, tok_scale, wscale, nullptr, b, yb, M,
+                                                  N, K, st, pdl);
+    }
     return wzero ? launch_gemm_gw<true, EVOD>(codes, tok_scale, w, wscale, wzero, b, yb, M, N, K,
                                               st, pdl)
                  : launch_gemm_gw<false, EVOD>(codes, tok_scale, w, wscale, nullptr, b, yb, M, N,
@@ -921,12 +979,13 @@ tint4_status convrot_w4a8_linear_groupwise(const tint4_bf16* x, const uint8_t* w
     float* tok_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                                 align_up(static_cast<size_t>(M) * K, 256));
     cudaStream_t st = as_stream(stream);
-    // every M runs the tensor-core kernel: the codes always go in its even/odd order
-    launch_rq_g<__nv_bfloat16, 127, false, true>(reinterpret_cast<const __nv_bfloat16*>(x), M, K,
-                                                 group, codes, tok_scale, st);
+    launch_linear_codes<127>(x, M, K, group, codes, tok_scale, st);
     if ((s = last_launch_status()) != TINT4_OK) return s;
-    return launch_gemm_gw_any<true>(codes, tok_scale, w_packed, w_scale, w_zero, bias, y, M, N, K,
-                                    st, true);
+    return linear_codes_evod(M)
+               ? launch_gemm_gw_any<true>(codes, tok_scale, w_packed, w_scale, w_zero, bias, y, M,
+                                          N, K, st, true)
+               : launch_gemm_gw_any<false>(codes, tok_scale, w_packed, w_scale, w_zero, bias, y, M,
+                                           N, K, st, true);
 }
 
 tint4_status tint4_quantize_weights_int8(const float* W, int N, int K, int group,

@@ -31,7 +31,20 @@
 // fragments for the current K chunk and its int32 sums for every block of
 // the run in registers; the warps' sums meet in shared memory at the end
 // (integer adds: any order gives the same bits).
+//
+// Group-wise weight scales (GW = 1 symmetric, 2 asymmetric; "ComfyUI-INT-
+// Crush", "Weight Format": scales [out, num_groups]; stable-diffusion.cpp
+// "feat: packed int4 convrot model loading and dispatch": asym_w4a8_int8):
+// a half chunk (128 K) is exactly one weight group, so each half's four MMAs
+// sum into a fresh int32 fragment that is scaled by the group scale of its
+// row (an exact conversion: |sum| < 2^24) and added to fp32 sums; the warps'
+// fp32 sums meet in shared memory in warp order.  Asymmetric nibbles q with a
+// zero point z per row and group widen to the int8 value 8 (q - z): 8 q in
+// bits 3-6 of each byte, plus 128 - 8 z without a carry between bytes, then
+// bit 7 flipped.
 #pragma once
+
+#include <type_traits>
 
 #include "ptx.cuh"
 #include "quantize.cuh"
@@ -85,14 +98,21 @@ constexpr int kS8FuseBytes = kFuseMaxRows * kS8FuseMaxK + 64 + kFuseMaxRows * kQ
 // is x (bf16) and the CTA rotates (group FG, 0 = none) and quantizes it (to
 // [-FQ, FQ], one code per byte) into shared memory itself, while its first
 // weight boxes are in flight; tok_scale is then unused.  FQ = 0: not fused.
-template <int NB, bool A_INT4, bool OUT_I32, int FG = 0, int FQ = 0>
+// GW (group-wise weight scales): row_scale is then the scale matrix
+// [N, K/128] and wzero (GW = 2) the zero points [N, K/128].
+template <int NB, bool A_INT4, bool OUT_I32, int FG = 0, int FQ = 0, int GW = 0>
 __global__ void __launch_bounds__(S8Cfg<NB>::THREADS, 1)
 w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __restrict__ act,
                   const float* __restrict__ tok_scale, const float* __restrict__ row_scale,
                   const __nv_bfloat16* __restrict__ bias, void* __restrict__ out, int M, int N,
-                  int K, uint32_t hi_mask, int early_weights, uint64_t wait_ns) {
+                  int K, uint32_t hi_mask, int early_weights, uint64_t wait_ns,
+                  const uint8_t* __restrict__ wzero) {
     constexpr bool FUSED = FQ != 0;
     static_assert(!FUSED || (NB == 1 && !A_INT4 && !OUT_I32), "fused: int8 codes, bf16 out, <= 8 tokens");
+    static_assert(GW == 0 || (!FUSED && !A_INT4 && !OUT_I32), "group-wise: int8 codes, bf16 out");
+    using Acc = typename std::conditional<GW != 0, float, int32_t>::type;
+    constexpr float kGwUnscale = GW == 2 ? 0.125f : 0.0625f;   // the unpack's 8 x / 16 x
+    const int ngr = K / 128;                                    // weight groups per row
     using C = S8Cfg<NB>;
     constexpr int kS8Warps = C::WARPS, kS8Slots = C::SLOTS, kS8Threads = C::THREADS;
     extern __shared__ uint8_t s8_smem_raw[];
@@ -101,7 +121,7 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
     uint64_t* full_all = reinterpret_cast<uint64_t*>(sm + kS8Ring);
     volatile uint32_t* abort_flag =
         reinterpret_cast<volatile uint32_t*>(full_all + kS8Warps * kS8Slots);
-    int32_t* red = reinterpret_cast<int32_t*>(sm);   // reused after the main loop
+    Acc* red = reinterpret_cast<Acc*>(sm);   // reused after the main loop
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -159,7 +179,7 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
     float* sTok = reinterpret_cast<float*>(sm + C::EPI_OFF + kS8MB * 16 * 6);
     if constexpr (!OUT_I32) {
         const int tid = threadIdx.x;
-        if (tid < nb * 16) cp_async4(sRowScale + tid, row_scale + b0 * 16 + tid);
+        if (GW == 0 && tid < nb * 16) cp_async4(sRowScale + tid, row_scale + b0 * 16 + tid);
         if (bias != nullptr && tid < nb * 8) cp_async4(sBias + 2 * tid, bias + b0 * 16 + 2 * tid);
         if (!FUSED && tid < M) cp_async4(sTok + tid, tok_scale + tid);
     }
@@ -175,13 +195,13 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
             *reinterpret_cast<float(*)[kFuseMaxRows][kQuantMaxWarps]>(sfuse + kFuseMaxRows * kS8FuseMaxK + 64));
     }
 
-    int32_t total[kS8MB][NB][4];
+    Acc total[kS8MB][NB][4];
 #pragma unroll
     for (int j = 0; j < kS8MB; ++j)
 #pragma unroll
         for (int b = 0; b < NB; ++b)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) total[j][b][q] = 0;
+            for (int q = 0; q < 4; ++q) total[j][b][q] = Acc(0);
 
     int consumed = 0, cslot = 0;
     uint32_t cphase = 0u;
@@ -238,6 +258,29 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
         for (int bp = 0; bp < kS8MB / 2; ++bp) {
             if (bp >= bp_hi) break;   // warp-uniform
             if (bp < bp_lo) continue;
+            // group-wise: the scales (and zero points) of this unit's rows and
+            // two groups, requested before the wait for its box
+            float gsc[2][2][2] = {};         // [block of the pair][half][row A / B]
+            uint32_t gzc[2][2][2] = {};      // (128 - 8 z) in every byte
+            if constexpr (GW != 0) {
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+                    const int j = 2 * bp + hb;
+                    if (j >= nb) break;
+                    const size_t ra = static_cast<size_t>((b0 + j) * 16 + rA) * ngr + 2 * P;
+                    const size_t rb = static_cast<size_t>((b0 + j) * 16 + rB) * ngr + 2 * P;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (256 * P + 128 * h >= K) break;   // a half past K (its sums are 0)
+                        gsc[hb][h][0] = __ldg(row_scale + ra + h) * kGwUnscale;
+                        gsc[hb][h][1] = __ldg(row_scale + rb + h) * kGwUnscale;
+                        if constexpr (GW == 2) {
+                            gzc[hb][h][0] = (128u - 8u * __ldg(wzero + ra + h)) * 0x01010101u;
+                            gzc[hb][h][1] = (128u - 8u * __ldg(wzero + rb + h)) * 0x01010101u;
+                        }
+                    }
+                }
+            }
             const int slot = cslot;
             int ok = 0;
             if (lane == 0)
@@ -257,17 +300,55 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
                     const uint4 pb = *reinterpret_cast<const uint4*>(bbox + rB * 128 + coff);
                     const uint32_t wa[4] = {pa.x, pa.y, pa.z, pa.w};
                     const uint32_t wb[4] = {pb.x, pb.y, pb.z, pb.w};
+                    if constexpr (GW == 0) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        // word i: 8 consecutive weights; low nibbles = even positions
-                        uint32_t a[4];
-                        a[0] = (wa[i] << 4) & hi_mask;   // MMA row g,   first slot
-                        a[1] = (wb[i] << 4) & hi_mask;   // MMA row g+8, first slot
-                        a[2] = wa[i] & hi_mask;          // MMA row g,   second slot
-                        a[3] = wb[i] & hi_mask;          // MMA row g+8, second slot
+                        for (int i = 0; i < 4; ++i) {
+                            // word i: 8 consecutive weights; low nibbles = even positions
+                            uint32_t a[4];
+                            a[0] = (wa[i] << 4) & hi_mask;   // MMA row g,   first slot
+                            a[1] = (wb[i] << 4) & hi_mask;   // MMA row g+8, first slot
+                            a[2] = wa[i] & hi_mask;          // MMA row g,   second slot
+                            a[3] = wb[i] & hi_mask;          // MMA row g+8, second slot
+#pragma unroll
+                            for (int b = 0; b < NB; ++b)
+                                mma_s8_16832(total[j][b], a, bfr[h][b][i][0], bfr[h][b][i][1]);
+                        }
+                    } else {
+                        // half h is weight group 2 P + h: its own int32 sums, then
+                        // scaled into the fp32 totals
+                        int32_t part[NB][4];
 #pragma unroll
                         for (int b = 0; b < NB; ++b)
-                            mma_s8_16832(total[j][b], a, bfr[h][b][i][0], bfr[h][b][i][1]);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) part[b][q] = 0;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            uint32_t a[4];
+                            if constexpr (GW == 2) {
+                                const uint32_t za = gzc[hb][h][0], zb = gzc[hb][h][1];
+                                a[0] = (((wa[i] << 3) & 0x78787878u) + za) ^ 0x80808080u;
+                                a[1] = (((wb[i] << 3) & 0x78787878u) + zb) ^ 0x80808080u;
+                                a[2] = (((wa[i] >> 1) & 0x78787878u) + za) ^ 0x80808080u;
+                                a[3] = (((wb[i] >> 1) & 0x78787878u) + zb) ^ 0x80808080u;
+                            } else {
+                                a[0] = (wa[i] << 4) & hi_mask;
+                                a[1] = (wb[i] << 4) & hi_mask;
+                                a[2] = wa[i] & hi_mask;
+                                a[3] = wb[i] & hi_mask;
+                            }
+#pragma unroll
+                            for (int b = 0; b < NB; ++b)
+                                mma_s8_16832(part[b], a, bfr[h][b][i][0], bfr[h][b][i][1]);
+                        }
+                        // fragment: [0], [1] row g (A), [2], [3] row g + 8 (B); exact
+                        // conversions (|sum| < 2^24), one rounding per FMA
+#pragma unroll
+                        for (int b = 0; b < NB; ++b)
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                total[j][b][q] = __fmaf_rn(gsc[hb][h][q >> 1],
+                                                           static_cast<float>(part[b][q]),
+                                                           total[j][b][q]);
                     }
                 }
             }
@@ -297,8 +378,12 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
         if (j >= nb) break;
 #pragma unroll
         for (int b = 0; b < NB; ++b)
-            *reinterpret_cast<int4*>(red + (((warp * kS8MB + j) * NB + b) * 32 + lane) * 4) =
-                make_int4(total[j][b][0], total[j][b][1], total[j][b][2], total[j][b][3]);
+            if constexpr (GW != 0)
+                *reinterpret_cast<float4*>(red + (((warp * kS8MB + j) * NB + b) * 32 + lane) * 4) =
+                    make_float4(total[j][b][0], total[j][b][1], total[j][b][2], total[j][b][3]);
+            else
+                *reinterpret_cast<int4*>(red + (((warp * kS8MB + j) * NB + b) * 32 + lane) * 4) =
+                    make_int4(total[j][b][0], total[j][b][1], total[j][b][2], total[j][b][3]);
     }
     __syncthreads();
     if (*abort_flag) return;   // the device error word says why; the output is left as it was
@@ -308,11 +393,11 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
         const int ln = e & 31;
         const int b = (e >> 5) % NB;
         const int j = (e >> 5) / NB;
-        int32_t v[4] = {0, 0, 0, 0};
+        Acc v[4] = {Acc(0), Acc(0), Acc(0), Acc(0)};
 #pragma unroll
-        for (int w = 0; w < kS8Warps; ++w) {
-            const int4 p = *reinterpret_cast<const int4*>(red + (((w * kS8MB + j) * NB + b) * 32 + ln) * 4);
-            v[0] += p.x; v[1] += p.y; v[2] += p.z; v[3] += p.w;
+        for (int w = 0; w < kS8Warps; ++w) {   // in warp order (fp32 sums: a fixed order)
+            const Acc* p = red + (((w * kS8MB + j) * NB + b) * 32 + ln) * 4;
+            v[0] += p[0]; v[1] += p[1]; v[2] += p[2]; v[3] += p[3];
         }
         const int gg = ln >> 2, tt = ln & 3;
         const int tok0 = 8 * b + 2 * tt;
@@ -326,7 +411,12 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
             const int lrow = (q & 2) ? l1 : l0;
             if (tok >= M) continue;
             if constexpr (OUT_I32) {
-                reinterpret_cast<int32_t*>(out)[static_cast<size_t>(tok) * N + row] = v[q] >> kShift;
+                reinterpret_cast<int32_t*>(out)[static_cast<size_t>(tok) * N + row] =
+                    static_cast<int32_t>(v[q]) >> kShift;
+            } else if constexpr (GW != 0) {
+                const float bsv = bias ? __bfloat162float(sBias[lrow]) : 0.0f;
+                reinterpret_cast<__nv_bfloat16*>(out)[static_cast<size_t>(tok) * N + row] =
+                    __float2bfloat16_rn(__fmaf_rn(v[q], sTok[tok], bsv));
             } else {
                 const float bsv = bias ? __bfloat162float(sBias[lrow]) : 0.0f;
                 const float st = FUSED ? sTokScale[tok] : sTok[tok];
