@@ -223,7 +223,10 @@ tint4_status convrot_w8a8_linear(const tint4_bf16* x, const int8_t* w_int8,
  *     else asymmetric codes with these zero points), bias bf16 [N] or NULL ->
  *     y bf16 [M, N] = bf16(s_tok[m] * sum_j s[n, j] * p_j (+ bias[n])), p_j the
  *     exact integer sum over group j of a * (q - z); the sum over groups is
- *     evaluated in fp32 in group order.  One tensor-core launch at every M.
+ *     evaluated in fp32 in group order (at M <= 16 with K <= 8192, one
+ *     partial sum per warp of a streaming kernel, added in a fixed order).
+ *     One launch: the streaming kernel at M <= 16 and K <= 8192, else the
+ *     tensor-core GEMM.
  *   - convrot_w4a8_linear_groupwise: rotate + quantize x bf16 [M, K] into the
  *     workspace (convrot_linear_workspace_size(M, K, 8) bytes, 256-byte
  *     aligned; the codes there are in a private K order), then the GEMM.

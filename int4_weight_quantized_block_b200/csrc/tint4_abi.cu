@@ -728,14 +728,19 @@ tint4_status launch_gemm_gw(const int8_t* codes, const float* tok_scale, const u
     return TINT4_OK;
 }
 
-// Small M (<= kS8MaxM tokens, natural-order codes): the streaming kernel
-// with group-wise scales (w4a8_small.cuh, GW = 1 symmetric / 2 asymmetric).
+// Small M (<= kS8MaxM tokens, natural-order codes, K <= 128 kS8GwMaxGroups):
+// the streaming kernel with group-wise scales (w4a8_small.cuh, GW = 1
+// symmetric / 2 asymmetric); else the tensor-core kernel.
+bool gw_streaming(int M, int K) { return M <= kS8MaxM && K <= 128 * kS8GwMaxGroups; }
+
 template <int NB, int GW>
 tint4_status launch_gemm_small_gw(const int8_t* a, const uint8_t* w, const float* st,
                                   const float* wscale, const uint8_t* wzero,
                                   const __nv_bfloat16* bias, __nv_bfloat16* y, int M, int N, int K,
                                   cudaStream_t stream, bool pdl) {
     auto kern = w4a8_small_kernel<NB, false, false, 0, 0, GW>;
+    constexpr int smem = S8Cfg<NB>::FUSE_OFF + kS8GwBytes + 1024;
+    static_assert(smem <= 227 * 1024, "shared memory budget");
     CUtensorMap tw;
     if (!make_map_u8(&tw, w, K / 2, N, K / 2, 128, 32, CU_TENSOR_MAP_SWIZZLE_128B))
         return TINT4_ERR_CUDA;
@@ -743,8 +748,8 @@ tint4_status launch_gemm_small_gw(const int8_t* a, const uint8_t* w, const float
     cudaGetDevice(&dev);
     static std::atomic<bool> attr_done[kMaxDevices];
     if (!attr_done[dev].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 S8Cfg<NB>::SMEM) != cudaSuccess) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess) {
             cudaGetLastError();
             return TINT4_ERR_CUDA;
         }
@@ -756,7 +761,7 @@ tint4_status launch_gemm_small_gw(const int8_t* a, const uint8_t* w, const float
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(S8Cfg<NB>::THREADS, 1, 1);
-    cfg.dynamicSmemBytes = S8Cfg<NB>::SMEM;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     (void)pdl;   // always programmatic, as launch_gemm_small
     cudaLaunchAttribute attr[1] = {pdl_attr()};
@@ -778,7 +783,7 @@ tint4_status launch_gemm_gw_any(const int8_t* codes, const float* tok_scale, con
                                 tint4_bf16* y, int M, int N, int K, cudaStream_t st, bool pdl) {
     const auto* b = reinterpret_cast<const __nv_bfloat16*>(bias);
     auto* yb = reinterpret_cast<__nv_bfloat16*>(y);
-    if (M <= kS8MaxM) {
+    if (gw_streaming(M, K)) {
         if (EVOD) return TINT4_ERR_INVALID_ARG;   // the streaming kernel reads natural-order codes
         if (M <= 8)
             return wzero ? launch_gemm_small_gw<1, 2>(codes, w, tok_scale, wscale, wzero, b, yb, M,
@@ -979,9 +984,14 @@ tint4_status convrot_w4a8_linear_groupwise(const tint4_bf16* x, const uint8_t* w
     float* tok_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                                 align_up(static_cast<size_t>(M) * K, 256));
     cudaStream_t st = as_stream(stream);
-    launch_linear_codes<127>(x, M, K, group, codes, tok_scale, st);
+    // even/odd codes whenever the tensor-core kernel runs them
+    const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    if (gw_streaming(M, K))
+        launch_rq_g<__nv_bfloat16, 127, false>(xb, M, K, group, codes, tok_scale, st);
+    else
+        launch_rq_g<__nv_bfloat16, 127, false, true>(xb, M, K, group, codes, tok_scale, st);
     if ((s = last_launch_status()) != TINT4_OK) return s;
-    return linear_codes_evod(M)
+    return !gw_streaming(M, K)
                ? launch_gemm_gw_any<true>(codes, tok_scale, w_packed, w_scale, w_zero, bias, y, M,
                                           N, K, st, true)
                : launch_gemm_gw_any<false>(codes, tok_scale, w_packed, w_scale, w_zero, bias, y, M,

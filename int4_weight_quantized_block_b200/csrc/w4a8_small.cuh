@@ -87,6 +87,13 @@ __device__ __forceinline__ void mma_s8_16832(int32_t (&d)[4], const uint32_t (&a
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Group-wise weights: the scales and zero points of the CTA's whole run of
+// rows (at most kS8MB blocks x 16 rows x kS8GwMaxGroups groups), one bulk copy
+// each at the start, behind the ring and barriers where the fused linear
+// keeps its codes (the two are never combined).  K <= 128 kS8GwMaxGroups.
+constexpr int kS8GwMaxGroups = 64;
+constexpr int kS8GwBytes = 16 + kS8MB * 16 * kS8GwMaxGroups * 5;
+
 // Shared memory of the fused linear: the codes of up to kFuseMaxRows tokens
 // (one per byte) and their scales, behind the ring and barriers.
 constexpr int kS8FuseMaxK = 16 * kQuantChunk;   // one chunk per warp of the 16-warp CTA
@@ -171,6 +178,26 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
     grid_launch_dependents();
     if (lane == 0 && issued == 0 && nunits > 0) issue(issued++);
 
+    // group-wise: the run's scales (and zero points), contiguous in global
+    // memory, by two bulk copies completing on their own barrier
+    uint64_t* gw_bar = reinterpret_cast<uint64_t*>(sm + C::FUSE_OFF);
+    const float* sGwScale = reinterpret_cast<const float*>(sm + C::FUSE_OFF + 16);
+    const uint8_t* sGwZero = sm + C::FUSE_OFF + 16 + kS8MB * 16 * kS8GwMaxGroups * 4;
+    if constexpr (GW != 0) {
+        if (threadIdx.x == 0) {
+            mbar_init(gw_bar, 1);
+            fence_mbarrier_init();
+            const uint32_t nsc = static_cast<uint32_t>(nb * 16 * ngr);
+            mbar_arrive_expect_tx(gw_bar, nsc * 4 + (GW == 2 ? nsc : 0u));
+            bulk_load_1d(const_cast<float*>(sGwScale), row_scale + static_cast<size_t>(b0) * 16 * ngr,
+                         nsc * 4, gw_bar);
+            if (GW == 2)
+                bulk_load_1d(const_cast<uint8_t*>(sGwZero), wzero + static_cast<size_t>(b0) * 16 * ngr,
+                             nsc, gw_bar);
+        }
+        __syncthreads();   // the barrier is initialised before anyone waits on it
+    }
+
     // The epilogue's operands of this run go to shared memory now, by
     // asynchronous copies that land during the main loop: read from global
     // memory at the end they would add a memory round trip to every launch.
@@ -203,9 +230,15 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
 #pragma unroll
             for (int q = 0; q < 4; ++q) total[j][b][q] = Acc(0);
 
+    bool gw_failed = false;
+    if constexpr (GW != 0) {
+        int ok = 0;
+        if (lane == 0) ok = mbar_wait_bounded(gw_bar, 0, abort_flag, wait_ns, kDevErrTimeoutConsumer);
+        if (__shfl_sync(0xFFFFFFFFu, ok, 0) == 0) gw_failed = true;
+    }
     int consumed = 0, cslot = 0;
     uint32_t cphase = 0u;
-    bool aborted = false;
+    bool aborted = gw_failed;
     const int P0 = u0 / nbp, P1 = nunits > 0 ? (u1 - 1) / nbp : P0 - 1;
     for (int P = P0; P <= P1 && !aborted; ++P) {
         const int bp_lo = P == P0 ? u0 % nbp : 0;                 // this warp's block pairs of chunk P
@@ -259,7 +292,7 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
             if (bp >= bp_hi) break;   // warp-uniform
             if (bp < bp_lo) continue;
             // group-wise: the scales (and zero points) of this unit's rows and
-            // two groups, requested before the wait for its box
+            // two groups, from the run's copy in shared memory
             float gsc[2][2][2] = {};         // [block of the pair][half][row A / B]
             uint32_t gzc[2][2][2] = {};      // (128 - 8 z) in every byte
             if constexpr (GW != 0) {
@@ -267,16 +300,16 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
                 for (int hb = 0; hb < 2; ++hb) {
                     const int j = 2 * bp + hb;
                     if (j >= nb) break;
-                    const size_t ra = static_cast<size_t>((b0 + j) * 16 + rA) * ngr + 2 * P;
-                    const size_t rb = static_cast<size_t>((b0 + j) * 16 + rB) * ngr + 2 * P;
+                    const int ra = (j * 16 + rA) * ngr + 2 * P;
+                    const int rb = (j * 16 + rB) * ngr + 2 * P;
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         if (256 * P + 128 * h >= K) break;   // a half past K (its sums are 0)
-                        gsc[hb][h][0] = __ldg(row_scale + ra + h) * kGwUnscale;
-                        gsc[hb][h][1] = __ldg(row_scale + rb + h) * kGwUnscale;
+                        gsc[hb][h][0] = sGwScale[ra + h] * kGwUnscale;
+                        gsc[hb][h][1] = sGwScale[rb + h] * kGwUnscale;
                         if constexpr (GW == 2) {
-                            gzc[hb][h][0] = (128u - 8u * __ldg(wzero + ra + h)) * 0x01010101u;
-                            gzc[hb][h][1] = (128u - 8u * __ldg(wzero + rb + h)) * 0x01010101u;
+                            gzc[hb][h][0] = (128u - 8u * sGwZero[ra + h]) * 0x01010101u;
+                            gzc[hb][h][1] = (128u - 8u * sGwZero[rb + h]) * 0x01010101u;
                         }
                     }
                 }
@@ -371,6 +404,11 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
     }
 
     // ---- the warps' partial sums meet in shared memory
+    if constexpr (GW != 0) {
+        // the run's scale copy has landed before the CTA can finish
+        uint32_t never = 0u;
+        if (threadIdx.x == 0) (void)mbar_wait_bounded(gw_bar, 0, &never, wait_ns, 0u);
+    }
     cp_async_wait_all();
     __syncthreads();
 #pragma unroll
