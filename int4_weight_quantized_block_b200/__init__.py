@@ -42,6 +42,7 @@ __all__ = [
     "tint4_set_decode_weight_prefetch",
     "tint4_abi_version",
     "QuantizedLinear",
+    "GroupwiseQuantizedLinear",
 ]
 
 
@@ -467,3 +468,43 @@ class QuantizedLinear:
             self._workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=x.device)
         fn = convrot_w4a8_linear if self.act_bits == 8 else convrot_w4a4_linear
         return fn(x, self.w_packed, self.row_scale, self.group, self.bias, y, self._workspace)
+
+
+class GroupwiseQuantizedLinear:
+    """A W4A8 ConvRot linear layer with group-wise weight scales (one per row
+    and 128-wide K group; symmetric, or asymmetric with zero points).
+
+    "ComfyUI-INT-Crush", "Weight Format" (scales [out, num_groups]) and
+    "feat: packed int4 convrot model loading and dispatch", "Summary" (the
+    asymmetric W4A8 format): the weights are rotated and quantized once
+    (``from_float``); each call rotates + quantizes the activations to int8
+    and runs the group-wise GEMM."""
+
+    def __init__(self, w_packed, w_scale, w_zero, group: int, bias=None):
+        self.w_packed = w_packed
+        self.w_scale = w_scale
+        self.w_zero = w_zero
+        self.group = group
+        self.bias = bias
+        self._workspace = None
+
+    @classmethod
+    def from_float(cls, W: torch.Tensor, group: int, asym: bool = False, bias=None):
+        wp, s, z = tint4_pack_weights_groupwise(W.float().contiguous(), group, asym)
+        return cls(wp, s, z, group, bias)
+
+    @property
+    def out_features(self) -> int:
+        return self.w_packed.shape[0]
+
+    @property
+    def in_features(self) -> int:
+        return self.w_packed.shape[1] * 2
+
+    def __call__(self, x: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+        need = convrot_linear_workspace_size(x.shape[0], self.in_features, 8)
+        if self._workspace is None or self._workspace.numel() < need or \
+                self._workspace.device != x.device:
+            self._workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=x.device)
+        return convrot_w4a8_linear_groupwise(x, self.w_packed, self.w_scale, self.group,
+                                             self.w_zero, self.bias, y, self._workspace)

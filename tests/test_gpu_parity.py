@@ -533,6 +533,23 @@ def test_groupwise_decode_full_size(M, asym):
     assert torch.equal(y1, y2)
 
 
+@pytest.mark.parametrize("asym", [False, True])
+def test_groupwise_module_end_to_end(asym):
+    """Weights packed on the GPU by the module, layer run on the GPU, both
+    against the oracle (M spans a ragged tensor-core tile)."""
+    M, N, K, g = 150, 272, 640, 64
+    x = inputs.activations(M, K, seed=850)
+    W = inputs.weights(N, K, seed=851)
+    lin = t4.GroupwiseQuantizedLinear.from_float(to_gpu(W), g, asym=asym)
+    y = lin(bf16_to_gpu(x))
+    torch.cuda.synchronize()
+    wp, s, z, _ = oracle.pack_weights_groupwise(W, g, 128, asym)
+    assert np.array_equal(lin.w_packed.cpu().numpy(), wp)
+    qa, st, _ = oracle.quantize_act(x, g, 8)
+    y64, mag = oracle.gemm_groupwise_f64(qa, st, wp, s, z)
+    assert_groupwise_output(bf16_from_gpu(y), y64, mag, K)
+
+
 def test_groupwise_equal_scales_match_per_row_gemm():
     """Symmetric group-wise weights whose group scales all equal the row
     scale compute the per-row W4A8 layer (same codes): outputs within the
