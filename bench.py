@@ -731,6 +731,18 @@ def run_profile_case(case: str, dev):
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         for _ in range(3):
             t4.w4a8_gemm_groupwise(codes, st, wp, s, z, None, y)
+    elif case.startswith("decode_gw_M"):
+        # the decode layer with group-wise asymmetric weights (streaming kernel)
+        M = int(case[len("decode_gw_M"):])
+        w = inputs.WORKLOADS["te_decode_w4a8"]
+        N, K, g = w["N"], w["K"], w["group"]
+        _, W_np = inputs.layer_inputs("te_decode_w4a8", M=1)
+        wp, s, z = t4.tint4_pack_weights_groupwise(torch.from_numpy(W_np).to(dev), g, True)
+        x = bf16_gpu(inputs.activations(M, K, inputs.SEED), dev)
+        codes, st = t4.convrot_quantize_act(x, g, 8)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            t4.w4a8_gemm_groupwise(codes, st, wp, s, z, None, y)
     elif case.startswith("decode_w4a8_M"):
         M = int(case[len("decode_w4a8_M"):])
         w = inputs.WORKLOADS["te_decode_w4a8"]
@@ -767,7 +779,7 @@ def main():
     ap.add_argument("--profile", default=None,
                     help="run only a few launches of one kernel for ncu: qkv_gemm, "
                          "qkv_gemm_w4a4, qkv_gemm_gw, qkv_quantize, w4a16_M<m>, "
-                         "decode_w4a8_M<m>")
+                         "decode_w4a8_M<m>, decode_gw_M<m>")
     args = ap.parse_args()
     if args.profile:
         dev = torch.device("cuda", 0)
