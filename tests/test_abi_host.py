@@ -179,3 +179,20 @@ def test_decode_prefetch_switch_rules(lib):
     assert lib.tint4_set_decode_weight_prefetch(-1) == 1
     assert lib.tint4_set_decode_weight_prefetch(1) == 0
     assert lib.tint4_set_decode_weight_prefetch(0) == 0
+
+
+def test_even_odd_code_order():
+    """The test helper's permutation: within each block of 8 codes along K,
+    positions 0, 2, 4, 6 first, then 1, 3, 5, 7 (the order the fused linears
+    store and the tensor-core GEMM's weight unpack produces)."""
+    import torch
+    import int4_weight_quantized_block_b200 as t4
+    codes = torch.arange(2 * 16, dtype=torch.int8).view(2, 16)
+    eo = t4.even_odd_codes(codes)
+    assert eo[0].tolist() == [0, 2, 4, 6, 1, 3, 5, 7, 8, 10, 12, 14, 9, 11, 13, 15]
+    assert eo[1].tolist() == [v + 16 for v in eo[0].tolist()]
+    # a dot product over K does not depend on the order
+    w = torch.randint(-7, 8, (16,), dtype=torch.int32)
+    a = torch.randint(-127, 128, (16,), dtype=torch.int32)
+    perm = t4.even_odd_codes(torch.arange(16, dtype=torch.int8).view(1, 16))[0].long()
+    assert int((a * w).sum()) == int((a[perm] * w[perm]).sum())
