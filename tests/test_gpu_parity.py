@@ -550,6 +550,21 @@ def test_groupwise_module_end_to_end(asym):
     assert_groupwise_output(bf16_from_gpu(y), y64, mag, K)
 
 
+@pytest.mark.parametrize("M,N,K", [(4, 144, 12288), (40, 128, 128)])
+def test_groupwise_routing_edges(M, N, K):
+    """A small M with K past the streaming kernel's 8192 (the tensor-core
+    kernel then runs it), and a single weight group (K = 128) at M > 16."""
+    x = inputs.activations(M, K, seed=860 + K)
+    codes, st, _ = oracle.quantize_act(x, 0, 8)
+    wp, s, z, _ = oracle.pack_weights_groupwise(inputs.weights(N, K, seed=861), 0, 128, True)
+    y = t4.w4a8_gemm_groupwise(to_gpu(codes), to_gpu(st), to_gpu(wp), to_gpu(s), to_gpu(z))
+    y1 = t4.convrot_w4a8_linear_groupwise(bf16_to_gpu(x), to_gpu(wp), to_gpu(s), 0, to_gpu(z))
+    torch.cuda.synchronize()
+    y64, mag = oracle.gemm_groupwise_f64(codes, st, wp, s, z)
+    assert_groupwise_output(bf16_from_gpu(y), y64, mag, K)
+    assert_groupwise_output(bf16_from_gpu(y1), y64, mag, K)
+
+
 def test_groupwise_equal_scales_match_per_row_gemm():
     """Symmetric group-wise weights whose group scales all equal the row
     scale compute the per-row W4A8 layer (same codes): outputs within the
