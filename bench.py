@@ -390,10 +390,26 @@ def bench_rows(args, t4, inputs, dev, flush, pk, int8_peak):
         g_ms = statistics.median(time_steps(lambda: gemm(codes, st, wp, sr, None, y), reps, flush, dev))
         l_ms = statistics.median(time_steps(lambda: lin(x, wp, sr, g, None, y, ws), reps, flush, dev))
         ops = 2.0 * M * N * K
-        return {"M": M, "N": N, "K": K, "group": g, "act_bits": bits,
-                "gemm_us": round(g_ms * 1e3, 2), "gemm_TOPS": round(ops / g_ms / 1e9, 2),
-                "gemm_frac_int8": round(ops / g_ms / 1e9 / int8_peak, 4),
-                "linear_us": round(l_ms * 1e3, 2), "linear_TOPS": round(ops / l_ms / 1e9, 2)}
+        row = {"M": M, "N": N, "K": K, "group": g, "act_bits": bits,
+               "gemm_us": round(g_ms * 1e3, 2), "gemm_TOPS": round(ops / g_ms / 1e9, 2),
+               "gemm_frac_int8": round(ops / g_ms / 1e9 / int8_peak, 4),
+               "linear_us": round(l_ms * 1e3, 2), "linear_TOPS": round(ops / l_ms / 1e9, 2)}
+        if M > 16:
+            # the fused linear's own GEMM launch: int8 codes (W4A4 codes kept one
+            # per byte) in the even/odd K order, permuted here, untimed
+            if bits == 8:
+                c8 = codes
+            else:
+                pk = codes.view(torch.uint8).to(torch.int16)
+                q = torch.stack([pk & 0xF, pk >> 4], dim=-1).reshape(M, K)
+                c8 = torch.where(q >= 8, q - 16, q).to(torch.int8)
+            c8eo = t4.even_odd_codes(c8)
+            lg_ms = statistics.median(time_steps(
+                lambda: t4.tint4_debug_w4a8_gemm_even_odd(c8eo, st, wp, sr, None, y), reps, flush,
+                dev))
+            row.update({"linear_gemm_us": round(lg_ms * 1e3, 2),
+                        "linear_gemm_frac_int8": round(ops / lg_ms / 1e9 / int8_peak, 4)})
+        return row
 
     rows["tiny_w4a8"] = gemm_layer("tiny_w4a8")
     rows["dit_qkv_w4a4"] = gemm_layer("dit_qkv_w4a4")
