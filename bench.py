@@ -303,13 +303,42 @@ def run_ours(args, rank, world, dev):
     y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
     x_dev = torch.empty_like(x)
 
+    # token chunks pipelined over three streams: the copy in of chunk i + 1
+    # and the copy out of chunk i - 1 overlap the layer on chunk i (the
+    # per-token quantize makes any row split exact: the same bits as one call)
+    E2E_CHUNKS = 4
+    bounds = [M * i // E2E_CHUNKS for i in range(E2E_CHUNKS + 1)]
+    s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev_in = [torch.cuda.Event() for _ in range(E2E_CHUNKS)]
+    ev_run = [torch.cuda.Event() for _ in range(E2E_CHUNKS)]
+
     def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
-        t4.convrot_w4a8_linear(x_dev, wp, sr, g, None, y, ws)
-        y_host.copy_(y, non_blocking=True)
+        cur = torch.cuda.current_stream(dev)
+        for st_ in (s_in, s_run, s_out):
+            st_.wait_stream(cur)
+        for i in range(E2E_CHUNKS):
+            m0, m1 = bounds[i], bounds[i + 1]
+            with torch.cuda.stream(s_in):
+                x_dev[m0:m1].copy_(x_host[m0:m1], non_blocking=True)
+                ev_in[i].record(s_in)
+            with torch.cuda.stream(s_run):
+                s_run.wait_event(ev_in[i])
+                t4.convrot_w4a8_linear(x_dev[m0:m1], wp, sr, g, None, y[m0:m1], ws)
+                ev_run[i].record(s_run)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_run[i])
+                y_host[m0:m1].copy_(y[m0:m1], non_blocking=True)
+        cur.wait_stream(s_out)
 
     for _ in range(2):
         e2e_step()
+    torch.cuda.synchronize(dev)
+    # the pipelined layer gives the bits of the single call
+    y_ref = y.clone()
+    t4.convrot_w4a8_linear(x, wp, sr, g, None, y_ref, ws)
+    torch.cuda.synchronize(dev)
+    if not torch.equal(y_host.to(dev), y_ref):
+        raise SystemExit("end-to-end pipeline result differs from the single call")
     e2e_ms_max = max_over_ranks(statistics.mean(time_steps(e2e_step, max(3, args.steps // 4),
                                                            flush, dev)), dev)
 
