@@ -28,7 +28,9 @@
  *   scales        fp32, one per row of W (row_scale [N]) and one per token
  *                 (tok_scale [M]); scale = absmax / 7 (int4) or / 127 (int8),
  *                 code = clamp(round_half_even(v / scale)); an all-zero row
- *                 has scale 0 and codes 0.
+ *                 has scale 0 and codes 0.  The group-wise entry points
+ *                 (below) take one weight scale per row and 128-wide K
+ *                 group instead, optionally with zero points.
  *   output        y[m, n] = bf16( acc[m, n] * tok_scale[m] * row_scale[n]
  *                 (+ bias[n]) ), acc the exact int32 sum of code products.
  *
