@@ -40,7 +40,7 @@ def test_hadamard_orthonormal_exact(g):
     assert np.array_equal(H, H.T)
 
 
-@pytest.mark.parametrize("g", GROUPS)
+@pytest.mark.parametrize("g", GROUPS + (1024,))
 def test_hadamard_walsh_closed_form(g):
     """Sylvester order: H[i, j] = (-1)^popcount(i & j) / sqrt(g)."""
     H = oracle.hadamard(g)
@@ -61,7 +61,7 @@ def test_fwht_unit_vectors_are_hadamard_columns(g):
         assert np.array_equal(oracle.fwht_f32(e).astype(np.float64), H[:, j])
 
 
-@pytest.mark.parametrize("g", GROUPS)
+@pytest.mark.parametrize("g", GROUPS + (1024,))
 def test_fwht_matches_dense_fp64(g):
     """The fp32 FWHT equals the dense fp64 product H v up to fp32 rounding."""
     r = np.random.default_rng(1)
@@ -74,7 +74,7 @@ def test_fwht_matches_dense_fp64(g):
         assert np.abs(got - ref).max() <= tol
 
 
-@pytest.mark.parametrize("g", GROUPS)
+@pytest.mark.parametrize("g", GROUPS + (1024,))
 def test_rotation_is_an_involution(g):
     """H is symmetric and orthogonal, so rotating twice gives back the input."""
     r = np.random.default_rng(2)
@@ -83,7 +83,7 @@ def test_rotation_is_an_involution(g):
     assert np.allclose(back, x, rtol=0, atol=1e-5 * np.abs(x).max())
 
 
-@pytest.mark.parametrize("g", GROUPS)
+@pytest.mark.parametrize("g", GROUPS + (1024,))
 def test_rotation_leaves_product_unchanged(g):
     """(x R)(W R)^T = x W^T: rotating both operands by the same block rotation
     leaves the product unchanged (to 1e-5 relative in fp32)."""
