@@ -73,6 +73,7 @@ def _load():
             "oracle_w4a16": [P, P, P, P, I, I, I, I, P],
             "oracle_w4a16_f64": [P, P, P, P, I, I, I, I, P],
             "oracle_w4a16_dequant_f64": [P, P, P, P, I, I, I, I, P],
+            "oracle_w4a16_weights_f64": [P, P, P, I, I, I, I, P],
             "oracle_quantize_weights_int8": [P, I, I, I, P, P],
             "oracle_pack_weights_groupwise": [P, I, I, I, I, I, P, P, P, P],
             "oracle_gemm_groupwise_f64": [P, P, P, P, P, P, I, I, I, I, P, P],
@@ -442,6 +443,22 @@ def w4a16_dequant_f64(x_bits, q_packed, scale_bits, zero, group) -> np.ndarray:
     _check(_load().oracle_w4a16_dequant_f64(_ptr(x), _ptr(q), _ptr(s), _ptr(z), M, N, K, group,
                                             _ptr(y)), "w4a16_dequant_f64")
     return y
+
+
+def w4a16_weights_f64(q_packed, scale_bits, zero, group, widen: bool = False) -> np.ndarray:
+    """The W4A16 weights, fp64 [N, K]: (q - z) * s exactly, or (widen) that
+    product rounded once to bf16 (the 16-bit unpack form of
+    ``w4a16_dequant_f64``).  For shapes where the per-output loops are slow,
+    ``bf16_bits_to_f32(x) @ w.T`` (a library matrix product) gives the same
+    layer values up to fp64 rounding."""
+    q = _c(q_packed, np.uint8)
+    s = _c(scale_bits, np.uint16)
+    z = _c(zero, np.uint8)
+    N, K = q.shape[0], 2 * q.shape[1]
+    w = np.empty((N, K), dtype=np.float64)
+    _check(_load().oracle_w4a16_weights_f64(_ptr(q), _ptr(s), _ptr(z), N, K, group, int(widen),
+                                            _ptr(w)), "w4a16_weights_f64")
+    return w
 
 
 def w4a16(x_bits, q_packed, scale_bits, zero, group) -> np.ndarray:

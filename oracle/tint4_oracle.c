@@ -513,6 +513,27 @@ int oracle_w4a16_dequant_f64(const uint16_t* x, const uint8_t* q, const uint16_t
     return bad ? ORACLE_BAD_ARG : ORACLE_OK;
 }
 
+/* The W4A16 weights themselves, fp64 [N, K]: w = (q - z) * s exactly
+ * (widen = 0), or that product rounded once to the nearest bf16 (widen = 1,
+ * the 16-bit unpack form above).  A dense matrix product of x with these
+ * gives the two forms of the layer for large shapes. */
+int oracle_w4a16_weights_f64(const uint8_t* q, const uint16_t* s, const uint8_t* z, int N, int K,
+                             int G, int widen, double* w) {
+    if (!q || !s || !z || !w || N < 0 || K <= 0 || G <= 0 || K % G || K % 2) return ORACLE_BAD_ARG;
+    int ng = K / G;
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n)
+        for (int k = 0; k < K; ++k) {
+            uint8_t b = q[(long)n * (K / 2) + k / 2];
+            int code = (k % 2 == 0) ? (b & 0xF) : (b >> 4);
+            double exact = ((double)code - (double)z[(long)n * ng + k / G]) *
+                           (double)bf16_bits_to_float(s[(long)n * ng + k / G]);
+            w[(long)n * K + k] =
+                widen ? (double)bf16_bits_to_float(double_to_bf16_bits(exact)) : exact;
+        }
+    return ORACLE_OK;
+}
+
 /* The same, rounded once to bf16: the layer's output. */
 int oracle_w4a16(const uint16_t* x, const uint8_t* q, const uint16_t* s, const uint8_t* z,
                  int M, int N, int K, int G, uint16_t* y) {
