@@ -8,8 +8,9 @@ Every test feeds the same seeded inputs to both sides.  Bars:
     difference counts as a rounding tie (not an error) when the oracle's fp64
     value lies within the kernel's fp32 evaluation error of the bf16 rounding
     midpoint; ties must stay below 1e-3 of the outputs (oracle/compare.py).
-Small cases span several tiles and ragged tails in M, N and K; the full-size
-workloads are checked on sampled outputs the oracle computes one by one.
+Small cases span several tiles and ragged tails in M, N and K; a mid-size
+case runs several tiles per persistent CTA; the full-size workloads are
+checked on every output.
 """
 import numpy as np
 import pytest
@@ -18,17 +19,36 @@ import torch
 import oracle
 import int4_weight_quantized_block_b200 as t4
 from int4_weight_quantized_block_b200 import inputs
-from oracle.compare import TIE_FRAC_ACCUMULATED, accumulation_error, check_bf16, gemm_eval_error
+from oracle.compare import (check_bf16, gemm_eval_error, tie_capacity, w4a16_stream_error,
+                            w4a16_tc_error)
 from gpu_util import CODE_MISMATCH_FRAC, bf16_from_gpu, bf16_to_gpu, code_mismatch, dev, to_gpu
 
 
 def assert_gemm_output(y_gpu_bits, ref64, bias_bits=None):
     b64 = None if bias_bits is None else oracle.bf16_bits_to_f32(bias_bits).astype(np.float64)
-    c = check_bf16(y_gpu_bits, ref64, gemm_eval_error(ref64, b64))
+    flat = np.asarray(ref64, np.float64).ravel()
+    bflat = None if b64 is None else np.broadcast_to(b64, np.shape(ref64)).ravel()
+
+    def err(i):   # the bound where the roundings differ (full-size outputs are large)
+        return gemm_eval_error(flat[i], None if bflat is None else bflat[i])
+
+    c = check_bf16(y_gpu_bits, ref64, err)
     assert c.ok, str(c)
 
 
 pytestmark = pytest.mark.gpu
+
+
+def assert_w4a16_stream(y_bits, x_bits, q, scale, zero, ref64=None):
+    """The streaming W4A16 kernel against the exact layer: per element within
+    the bound of its fp32 evaluation order (w4a16_stream_error); a one-ulp
+    difference only where the exact value lies within that bound of a bf16
+    rounding midpoint."""
+    if ref64 is None:
+        ref64 = oracle.w4a16_f64(x_bits, q, scale, zero, 128)
+    err = w4a16_stream_error(x_bits, q, scale, zero, 128)
+    c = check_bf16(y_bits, ref64, err, tie_capacity(ref64, err))
+    assert c.ok, str(c)
 
 
 # ------------------------------------------------------------------ weights
@@ -221,10 +241,7 @@ def test_decode_weight_prefetch_switch(prefetch):
         assert np.array_equal(bf16_from_gpu(o[2]), y16)
     assert_gemm_output(y8, oracle.convrot_linear_f64(x, wp, sr, g, 8))
     assert_gemm_output(y4, oracle.convrot_linear_f64(x, wp, sr, g, 4))
-    c = check_bf16(y16, oracle.w4a16_f64(op.x, op.q, op.scale, op.zero, 128),
-                   accumulation_error(oracle.w4a16_f64(op.x, op.q, op.scale, op.zero, 128)),
-                   TIE_FRAC_ACCUMULATED)
-    assert c.ok, str(c)
+    assert_w4a16_stream(y16, op.x, op.q, op.scale, op.zero)
 
 
 # ------------------------------------------------------------------ fused linear
@@ -285,21 +302,14 @@ def test_quantized_linear_module_end_to_end():
     assert_gemm_output(bf16_from_gpu(y), oracle.convrot_linear_f64(x, wp, sr, g, 8))
 
 
-def _sample_pairs(M, N, n, seed):
-    r = np.random.default_rng(seed)
-    pairs = np.stack([r.integers(0, M, n), r.integers(0, N, n)], axis=1)
-    corners = np.array([[0, 0], [M - 1, N - 1], [0, N - 1], [M - 1, 0],
-                        [M // 2, N // 2], [127, 255], [128, 256]])
-    corners = corners[(corners[:, 0] < M) & (corners[:, 1] < N)]
-    return np.concatenate([pairs, corners]).astype(np.int64)
-
-
 @pytest.mark.parametrize("name", ["dit_qkv_w4a8", "dit_qkv_w4a4", "dit_mlp_up_w4a8",
                                   "dit_mlp_down_w4a8"])
-def test_full_size_workloads_sampled(name):
-    """The full-size layers: weights packed on the GPU (bit-exact against the
-    oracle, all of them), activation codes (all of them), and the layer output
-    on sampled (m, n) pairs that the oracle computes one by one."""
+def test_full_size_workloads(name):
+    """The full-size layers, every element: weights packed on the GPU
+    (bit-exact against the oracle), activation codes and token scales, the
+    fused linear's output against the oracle's epilogue of its exact int32
+    sums, and those int32 sums themselves (bit-exact) from the GEMM that the
+    persistent kernel runs over many tiles per CTA."""
     w = inputs.WORKLOADS[name]
     M, N, K, g, bits = w["M"], w["N"], w["K"], w["group"], w["act_bits"]
     x, W = inputs.layer_inputs(name)
@@ -316,16 +326,39 @@ def test_full_size_workloads_sampled(name):
     frac, dmax = code_mismatch(qa_gpu, qa_ref)
     assert frac <= CODE_MISMATCH_FRAC and dmax <= 1
     assert np.array_equal(st.cpu().numpy().view(np.uint32), st_ref.view(np.uint32))
-    pairs = _sample_pairs(M, N, 4096, seed=9)
-    acc = oracle.gemm_i32_sampled(qa_ref, qw_ref, pairs)
-    y_ref = oracle.epilogue_sampled_f64(acc, st_ref, sr_ref, pairs)
-    y_gpu = bf16_from_gpu(y)[pairs[:, 0], pairs[:, 1]]
-    assert_gemm_output(y_gpu, y_ref)
-    # int32 accumulators of the same codes, bit-exact on the samples
+    acc = oracle.gemm_i32(qa_ref, qw_ref)
+    assert_gemm_output(bf16_from_gpu(y), oracle.epilogue_f64(acc, st_ref, sr_ref))
+    # int32 accumulators of the same codes, bit-exact everywhere
     a = to_gpu(qa_ref) if bits == 8 else to_gpu(oracle.pack_int4(qa_ref))
     acc_gpu = t4.tint4_debug_int32_gemm(a, bits, to_gpu(wp_ref))
     torch.cuda.synchronize()
-    assert np.array_equal(acc_gpu.cpu().numpy()[pairs[:, 0], pairs[:, 1]], acc)
+    assert np.array_equal(acc_gpu.cpu().numpy(), acc)
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_many_tiles_per_cta(bits):
+    """A mid-size layer (2048 tokens, 8192 weight rows, K 1024: 704 tiles of
+    128 x 192, between 4 and 5 per persistent CTA), every element: each CTA
+    reuses both accumulator buffers and crosses tile boundaries in its rings
+    several times.  int32 sums bit-exact (packed and int8 codes), the fused
+    linear and the GEMM entries against the oracle."""
+    M, N, K, g = 2048, 8192, 1024, 256
+    x = inputs.activations(M, K, seed=1300 + bits)
+    W = inputs.weights(N, K, seed=1310)
+    wp, sr, qw = oracle.pack_weights(W, g)
+    qa, st, packed = oracle.quantize_act(x, g, bits)
+    acc = oracle.gemm_i32(qa, qw)
+    a = to_gpu(qa) if bits == 8 else to_gpu(packed)
+    acc_gpu = t4.tint4_debug_int32_gemm(a, bits, to_gpu(wp))
+    fn = t4.convrot_w4a8_linear if bits == 8 else t4.convrot_w4a4_linear
+    y = fn(bf16_to_gpu(x), to_gpu(wp), to_gpu(sr), g)
+    gemm = t4.w4a8_gemm if bits == 8 else t4.w4a4_gemm
+    y2 = gemm(a, to_gpu(st), to_gpu(wp), to_gpu(sr))
+    torch.cuda.synchronize()
+    assert np.array_equal(acc_gpu.cpu().numpy(), acc)
+    ref = oracle.epilogue_f64(acc, st, sr)
+    assert_gemm_output(bf16_from_gpu(y), ref)
+    assert np.array_equal(bf16_from_gpu(y), bf16_from_gpu(y2))
 
 
 # ------------------------------------------------------------------ W8A8
@@ -356,9 +389,9 @@ def test_w8a8_gemm_and_linear(M, N, K, g):
     assert_gemm_output(bf16_from_gpu(yl), oracle.epilogue_f64(acc, st, sr))
 
 
-def test_w8a8_full_size_sampled():
-    """The DiT QKV layer as W8A8: all weight codes and scales bit-exact, the
-    output on sampled (m, n) pairs against the oracle."""
+def test_w8a8_full_size():
+    """The DiT QKV layer as W8A8: all weight codes and scales bit-exact, every
+    output against the oracle."""
     w = inputs.WORKLOADS["dit_qkv_w4a8"]
     M, N, K, g = w["M"], w["N"], w["K"], w["group"]
     x, W = inputs.layer_inputs("dit_qkv_w4a8")
@@ -369,10 +402,8 @@ def test_w8a8_full_size_sampled():
     assert np.array_equal(wc.cpu().numpy(), wc_ref)
     assert np.array_equal(sr.cpu().numpy().view(np.uint32), sr_ref.view(np.uint32))
     qa_ref, st_ref, _ = oracle.quantize_act(x, g, 8)
-    pairs = _sample_pairs(M, N, 4096, seed=19)
-    acc = oracle.gemm_i32_sampled(qa_ref, wc_ref, pairs)
-    y_ref = oracle.epilogue_sampled_f64(acc, st_ref, sr_ref, pairs)
-    assert_gemm_output(bf16_from_gpu(y)[pairs[:, 0], pairs[:, 1]], y_ref)
+    acc = oracle.gemm_i32(qa_ref, wc_ref)
+    assert_gemm_output(bf16_from_gpu(y), oracle.epilogue_f64(acc, st_ref, sr_ref))
 
 
 # ------------------------------------------------------------------ grouped GEMM
@@ -581,10 +612,9 @@ def test_groupwise_equal_scales_match_per_row_gemm():
     assert d <= 2 * 2.0 ** -8 * y_row.float().abs().max().item()
 
 
-def test_groupwise_full_size_sampled():
+def test_groupwise_full_size():
     """The DiT QKV layer with asymmetric group-wise weights at full size:
-    packing bit-exact (all of it), the fused linear on sampled outputs the
-    oracle computes one by one."""
+    packing bit-exact, every output of the fused linear against the oracle."""
     name = "dit_qkv_w4a8_asym_g128"
     w = inputs.WORKLOADS[name]
     M, N, K, g = w["M"], w["N"], w["K"], w["group"]
@@ -598,10 +628,9 @@ def test_groupwise_full_size_sampled():
     assert np.array_equal(wp.cpu().numpy(), wp_ref)
     assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
     assert np.array_equal(z.cpu().numpy(), z_ref)
-    pairs = _sample_pairs(M, N, 4096, seed=11)
-    y64, mag = oracle.gemm_groupwise_sampled_f64(codes.cpu().numpy(), st.cpu().numpy(), wp_ref,
-                                                 s_ref, pairs, z_ref)
-    assert_groupwise_output(bf16_from_gpu(y)[pairs[:, 0], pairs[:, 1]], y64, mag, K)
+    y64, mag = oracle.gemm_groupwise_f64(codes.cpu().numpy(), st.cpu().numpy(), wp_ref, s_ref,
+                                         z_ref)
+    assert_groupwise_output(bf16_from_gpu(y), y64, mag, K)
 
 
 # ------------------------------------------------------------------ W4A16
@@ -611,12 +640,10 @@ def test_groupwise_full_size_sampled():
                                    (16, 2400, 1024), (3, 12288, 256)])
 def test_w4a16(M, N, K):
     op = inputs.w4a16_operands(M, N, K, 128, seed=600 + M)
-    y_ref = oracle.w4a16_f64(op.x, op.q, op.scale, op.zero, 128)
     y = t4.w4a16_gemv_gemm(bf16_to_gpu(op.x), to_gpu(op.q), bf16_to_gpu(op.scale),
                            to_gpu(op.zero), 128)
     torch.cuda.synchronize()
-    c = check_bf16(bf16_from_gpu(y), y_ref, accumulation_error(y_ref), TIE_FRAC_ACCUMULATED)
-    assert c.ok, str(c)
+    assert_w4a16_stream(bf16_from_gpu(y), op.x, op.q, op.scale, op.zero)
 
 
 @pytest.mark.parametrize("M", [1, 9])
@@ -634,51 +661,41 @@ def test_w4a16_extreme_token_values(M):
         # bf16 rounding midpoint: a tie the other token rows dilute)
         x[M - 1, 1100] = 7.0e4
     xb = inputs.f32_to_bf16_bits(x)
-    y_ref = oracle.w4a16_f64(xb, op.q, op.scale, op.zero, 128)
     y = t4.w4a16_gemv_gemm(bf16_to_gpu(xb), to_gpu(op.q), bf16_to_gpu(op.scale),
                            to_gpu(op.zero), 128)
     torch.cuda.synchronize()
-    c = check_bf16(bf16_from_gpu(y), y_ref, accumulation_error(y_ref), TIE_FRAC_ACCUMULATED)
-    assert c.ok, str(c)
+    assert_w4a16_stream(bf16_from_gpu(y), xb, op.q, op.scale, op.zero)
 
 
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_w4a16_full_size(M):
     w = inputs.WORKLOADS["te_decode_w4a16"]
     op = inputs.w4a16_operands(M, w["N"], w["K"], w["group"])
-    y_ref = oracle.w4a16_f64(op.x, op.q, op.scale, op.zero, w["group"])
     y = t4.w4a16_gemv_gemm(bf16_to_gpu(op.x), to_gpu(op.q), bf16_to_gpu(op.scale),
                            to_gpu(op.zero), w["group"])
     torch.cuda.synchronize()
-    c = check_bf16(bf16_from_gpu(y), y_ref, accumulation_error(y_ref), TIE_FRAC_ACCUMULATED)
-    assert c.ok, str(c)
+    assert_w4a16_stream(bf16_from_gpu(y), op.x, op.q, op.scale, op.zero)
 
 
 # W4A16 above 32 tokens: one tensor-core GEMM, weights widened to bf16 first
-# (the 16-bit unpack form); held to that form with the accumulation tolerance
-# and to the exact form with the layer's 1e-2 bar.
-def check_w4a16_large(y_bits, op, rows=None, cols=None):
-    x, q, sc, z = op.x, op.q, op.scale, op.zero
-    if rows is not None:
-        x = x[rows]
-        y_bits = y_bits[rows]
-    if cols is not None:
-        q, sc, z = q[cols], sc[cols], z[cols]
-        y_bits = y_bits[:, cols]
-    ref_dq = oracle.w4a16_dequant_f64(x, q, sc, z, 128)
-    c = check_bf16(y_bits, ref_dq, accumulation_error(ref_dq), TIE_FRAC_ACCUMULATED)
+# (the 16-bit unpack form); held to that form within the bound of its fp32
+# accumulation, and to the exact form with the widening's and the output
+# rounding's error added.  The reference is a library matrix product of x
+# with the oracle's weights (every output).
+def check_w4a16_large(y_bits, op):
+    x64 = oracle.bf16_bits_to_f32(op.x).astype(np.float64)
+    xa = np.abs(x64)
+    w_dq = oracle.w4a16_weights_f64(op.q, op.scale, op.zero, 128, widen=True)
+    ref_dq = x64 @ w_dq.T
+    err = w4a16_tc_error(op.x, w_dq)
+    c = check_bf16(y_bits, ref_dq, err, tie_capacity(ref_dq, err))
     assert c.ok, "16-bit unpack form: " + str(c)
     # against the exact form (q - z) * s: per element, the widening moves the
     # value by at most 2^-8 sum_k |x_k| |w_k|, the output rounding by half an
-    # ulp (< 2^-8 |y|), the fp32 accumulation by the tolerance above
-    ref = oracle.w4a16_f64(x, q, sc, z, 128)
-    qk = np.empty((q.shape[0], 2 * q.shape[1]), np.float64)
-    qk[:, 0::2] = q & 0xF
-    qk[:, 1::2] = q >> 4
-    w = (qk - np.repeat(z.astype(np.float64), 128, axis=1)) * \
-        np.repeat(oracle.bf16_bits_to_f32(sc).astype(np.float64), 128, axis=1)
-    xa = np.abs(oracle.bf16_bits_to_f32(x).astype(np.float64))
-    bound = (xa @ np.abs(w).T + np.abs(ref_dq)) * 2.0 ** -8 + accumulation_error(ref_dq)
+    # ulp (< 2^-8 |y|), the fp32 accumulation by the bound above
+    w = oracle.w4a16_weights_f64(op.q, op.scale, op.zero, 128)
+    ref = x64 @ w.T
+    bound = (xa @ np.abs(w).T + np.abs(ref_dq)) * 2.0 ** -8 + err
     g = oracle.bf16_bits_to_f32(y_bits).astype(np.float64)
     excess = np.abs(g - ref) - bound
     assert np.all(excess <= 0), f"exact form: bound exceeded by {excess.max():.3e}"
@@ -707,25 +724,21 @@ def test_w4a16_large_m_extreme_token_values():
                            to_gpu(op.zero), 128)
     torch.cuda.synchronize()
     ref_dq = oracle.w4a16_dequant_f64(xb, op.q, op.scale, op.zero, 128)
-    c = check_bf16(bf16_from_gpu(y), ref_dq, accumulation_error(ref_dq), TIE_FRAC_ACCUMULATED)
+    err = w4a16_tc_error(xb, oracle.w4a16_weights_f64(op.q, op.scale, op.zero, 128, widen=True))
+    c = check_bf16(bf16_from_gpu(y), ref_dq, err, tie_capacity(ref_dq, err))
     assert c.ok, str(c)
 
 
 def test_w4a16_prefill_full_size():
     """The prefill workload (weights of the decode layer, thousands of tokens),
-    checked on sampled token rows and weight rows."""
+    every output checked."""
     w = inputs.WORKLOADS["te_prefill_w4a16"]
     M, N, K = w["M"], w["N"], w["K"]
     op = inputs.w4a16_operands(M, N, K, w["group"])
     y = t4.w4a16_gemv_gemm(bf16_to_gpu(op.x), to_gpu(op.q), bf16_to_gpu(op.scale),
                            to_gpu(op.zero), w["group"])
     torch.cuda.synchronize()
-    rng = np.random.default_rng(7)
-    rows = np.sort(rng.choice(M, 48, replace=False))
-    rows[-1] = M - 1
-    cols = np.sort(rng.choice(N, 256, replace=False))
-    cols[-1] = N - 1
-    check_w4a16_large(bf16_from_gpu(y), op, rows, cols)
+    check_w4a16_large(bf16_from_gpu(y), op)
 
 
 # ------------------------------------------------------------------ edge cases
