@@ -122,19 +122,29 @@ tint4_status w4a4_gemm(const uint8_t* a_packed, const float* tok_scale, const ui
                        const float* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
                        int N, int K, void* stream);
 
-/* Bytes of workspace convrot_w4a8_linear (bits 8) / convrot_w4a4_linear
- * (bits 4) need: the activation codes, one byte per code for both widths
- * (M * K), plus the token scales (4 * M), each rounded up to 256. */
+/* Bytes of workspace the fused linears need (convrot_w4a8_linear: bits 8,
+ * convrot_w4a4_linear: bits 4; the grouped, group-wise and W8A8 linears: bits
+ * 8): the activation codes, one byte per code for both widths (M * K), plus
+ * the token scales (4 * M), each rounded up to 256.  0 for invalid
+ * arguments. */
 size_t convrot_linear_workspace_size(int M, int K, int bits);
+
+/* The W4A8 workspace size under the name of the boundary's specification:
+ * convrot_linear_workspace_size(M, K, 8). */
+size_t convrot_w4a8_linear_workspace(int M, int K);
 
 /*
  * Fused ConvRot linear ("ComfyUI-INT-Crush", "Inference > INT4 > CUDA
  * backend": Hadamard rotation + activation quantization + INT8 GEMM as one
  * call; "Forward Pass" last note).  x bf16 [M, K] -> y bf16 [M, N].  The
- * rotate+quantize grid and the GEMM grid run back to back on `stream` with
- * programmatic dependent launch; the codes pass through `workspace`
- * (device memory of at least convrot_linear_workspace_size(M, K, 8) bytes,
- * 256-byte aligned, owned by the caller; its contents are scratch).
+ * codes pass through `workspace` (device memory of at least
+ * convrot_linear_workspace_size(M, K, 8) bytes, 256-byte aligned, owned by
+ * the caller; its contents are scratch).
+ *   - M = 1 (K <= 4096): one launch that rotates and quantizes x inside the
+ *     GEMM's CTAs.
+ *   - otherwise: the rotate + quantize grid, then the GEMM grid (the
+ *     streaming kernel up to 16 tokens, the tensor-core kernel above), back to
+ *     back on `stream` with programmatic dependent launch.
  */
 tint4_status convrot_w4a8_linear(const tint4_bf16* x, const uint8_t* w_packed,
                                  const float* row_scale, const tint4_bf16* bias, tint4_bf16* y,
@@ -157,20 +167,25 @@ tint4_status convrot_w4a4_linear(const tint4_bf16* x, const uint8_t* w_packed,
  * inside a fixed memory budget, a host program without a device allocator
  * of its own, or a plug-in whose host application owns every allocation.
  * (The pages have no counterpart: it is a packaging of the same layer.)
- * The activation codes and token scales go to one fixed 16 MiB device array
- * inside this library, which every GPU that loads the library holds until
- * the process exits.  Inputs and outputs are as convrot_w4a8_linear; the
- * caller still owns x, w_packed, row_scale, bias and y.
- *   - Sizes: M * K + 4 * M bytes (each rounded up to 256) must fit in
- *     16 MiB, else TINT4_ERR_WORKSPACE is returned and nothing is launched.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ * The workspace (activation codes and token scales) is one fixed 16 MiB
+ * device array inside this library.  A GPU
+ * reserves it when the library's device code is first loaded there (its
+ * first kernel launch or its first call of this entry), whether or not this
+ * entry is used, and holds it until the process exits.  Inputs and outputs
+ * are as convrot_w4a8_linear; the caller still owns x, w_packed, row_scale,
+ * bias and y.
+ *   - Sizes: convrot_linear_workspace_size(M, K, 8) must fit in 16 MiB, else
+ *     TINT4_ERR_WORKSPACE is returned and nothing is launched.
+ *   - The first call on a device (and the first after the device's context
+ *     has been rebuilt, e.g. by cudaDeviceReset) looks up the array's device
+ *     address (cudaGetSymbolAddress); make that call before any stream
+ *     capture.
  *   - No allocation: the call makes no cudaMalloc / cudaFree and calls no
  *     allocating routine.
  *   - Every call on a device shares the one array, and it keeps whatever the
  *     last call left in it (nothing in it needs to start at zero).  Calls
- *     whose work overlaps on the GPU (two streams, or two host threads)
- *     race on it and corrupt each other's results: serialize them.
+ *     whose work overlaps on the GPU (two streams, or two host threads) race
+ *     on it and corrupt each other's results: serialize them.
  */
 tint4_status convrot_w4a8_linear_noalloc(const tint4_bf16* x, const uint8_t* w_packed,
                                          const float* row_scale, const tint4_bf16* bias,

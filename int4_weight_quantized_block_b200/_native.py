@@ -44,6 +44,7 @@ SIGNATURES = {
     "w4a8_gemm": (I, [P, P, P, P, P, P, I, I, I, P]),
     "w4a4_gemm": (I, [P, P, P, P, P, P, I, I, I, P]),
     "convrot_linear_workspace_size": (SZ, [I, I, I]),
+    "convrot_w4a8_linear_workspace": (SZ, [I, I]),
     "convrot_w4a8_linear": (I, [P, P, P, P, P, I, I, I, I, P, SZ, P]),
     "convrot_w4a4_linear": (I, [P, P, P, P, P, I, I, I, I, P, SZ, P]),
     "convrot_w4a8_linear_noalloc": (I, [P, P, P, P, P, I, I, I, I, P]),

@@ -202,57 +202,307 @@ __device__ __forceinline__ void rotate_quantize_rows_to_smem(const __nv_bfloat16
     __syncthreads();
 }
 
-// Q = 127 (int8 codes) or 7 (int4 codes); PACKED: int4 codes two per byte,
-// else one code per int8.  CH = chunks per warp held in registers; the CTA
-// has blockDim.x / 32 warps (K <= warps * CH * 256).  Persistent: CTA b
-// handles rows b, b + gridDim.x, ..., and the loads of its next row are in
-// flight while it rotates and quantizes the current one.
-// The rows of one CTA.  FULL: the CTA's warps hold exactly K values (every
-// chunk present and complete), so no per-chunk guard is needed.
-// EVOD (int8 codes only): each block of 8 codes is stored with its even
-// positions first (codes 0, 2, 4, 6, 1, 3, 5, 7), the layout whose weights
-// the tensor-core GEMM unpacks without byte permutes; a private layout of the
-// fused linears' workspace (the sums over K are the same numbers).
-template <typename InT, int G, int Q, bool PACKED, int CH, bool FULL, bool EVOD = false>
-__device__ __forceinline__ void rotate_quantize_rows(const InT* __restrict__ in, int rows, int K,
-                                                     void* __restrict__ codes,
-                                                     float* __restrict__ scales,
-                                                     float (&red)[2][kQuantMaxWarps]) {
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int nwarps = blockDim.x >> 5;
-    const int nchunks = (K + kQuantChunk - 1) / kQuantChunk;
-    auto present = [&](int c) { return FULL || warp + c * nwarps < nchunks; };   // warp-uniform
-    auto base_of = [&](int c) { return (warp + c * nwarps) * kQuantChunk + lane * 8; };
+// ================================================================ row kernels
+//
+// Rotate + quantize whole rows with a team of W warps per row (the CTA).
+// Each lane holds CPL chunks of 8 consecutive values (CPL = 1, 2 or 4; one
+// 16-byte bf16 load per chunk), so a lane keeps up to 32 values of its row in
+// registers and the team covers K = 256 W CPL values.  The chunks of a lane
+// are placed so that as many butterfly spans as possible fall inside the
+// lane (RqLayout): a rotation block of G values is CB = G/8 chunks; a lane
+// holds min(CB, CPL) of them, spaced LPB = CB/CPL chunks apart, so the spans
+// of the chunk index's low bits cross lanes (lane distance 1 .. LPB/2) and
+// those of its high bits stay in registers.  With G = 256 and CPL = 4 that is
+// three in-register spans (1, 2, 4), three shuffle spans (8, 16, 32) and two
+// in-register spans (64, 128), in that order: the order every butterfly of
+// the transform is taken in, so the rotated values are bit-identical to a
+// sequential transform whichever lane computes them.
+//
+// Arithmetic runs on packed fp32 pairs (add / sub / fma .f32x2, one rounding
+// per element as the scalar forms): a pair holds the same element of two
+// neighbouring chunks, so every butterfly span except the one between those
+// two chunks is one packed add and one packed subtract per two butterflies.
+//
+// The transform is left unnormalised: with u the unnormalised value and k =
+// log2(sqrt(G)), the rotated value is v = u 2^-k, the token scale s = fl(
+// absmax(v) / Q) = fl(absmax(u) / Q) 2^-k and v / s = u / (s 2^k) exactly,
+// so the codes and the stored scale are those of the normalised transform as
+// long as nothing is subnormal (rows whose absmax(u) is below 2^-100 take the
+// normalised path value by value).
 
-    RawChunk<InT> raw[CH];
+// 64-bit register holding two fp32 values: lo in the low word
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t p, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// a * b + c, each element rounded once
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// (a, b) -> (a + b, a - b) for two element pairs at once
+__device__ __forceinline__ void f2_bfly(uint64_t& a, uint64_t& b) {
+    const uint64_t s = f2_add(a, b);
+    b = f2_sub(a, b);
+    a = s;
+}
+
+// (lo, hi) -> (lo + hi, lo - hi) inside one pair
+__device__ __forceinline__ uint64_t f2_bfly_inner(uint64_t p) {
+    float lo, hi;
+    f2_unpack(p, lo, hi);
+    return f2_pack(lo + hi, lo - hi);
+}
+
+template <int G, int CPL>
+struct RqLayout {
+    static_assert(CPL == 1 || CPL == 2 || CPL == 4, "chunks per lane");
+    static constexpr int CB = G == 0 ? CPL : G / 8;          // chunks per rotation block
+    static constexpr int LPB = CB >= CPL ? CB / CPL : 1;     // lanes sharing a block
+    static constexpr int CPBL = CB >= CPL ? CPL : CB;        // chunks of one block in a lane
+    static constexpr int BPL = CPL / CPBL;                   // blocks per lane
+    static_assert(LPB <= 32, "a rotation block stays inside one warp");
+    // chunk (8 values) of the row held as register chunk i by team lane L of
+    // TL; without rotation consecutive lanes take consecutive chunks
+    __device__ __forceinline__ static int chunk(int i, int L, int TL) {
+        if (G == 0) return i * TL + L;
+        const int bi = i / CPBL, ji = i % CPBL;
+        return ((L / LPB) * BPL + bi) * CB + ji * LPB + (L % LPB);
+    }
+};
+
+// Pairs: CPL >= 2: p[8k + e] = (element e of chunk 2k, element e of chunk
+// 2k + 1); CPL = 1: p[e] = (element e, element e + 4), e < 4.
+template <int CPL>
+struct RqPairs {
+    static constexpr int N = CPL * 4;
+};
+
+// Unnormalised FWHT of the lane's values (see above for the span order).
+template <int G, int CPL>
+__device__ __forceinline__ void fwht_team(uint64_t (&p)[RqPairs<CPL>::N], int lane) {
+    if constexpr (G != 0) {
+        using Lt = RqLayout<G, CPL>;
+        // spans 1, 2, 4: inside each chunk
+        if constexpr (CPL >= 2) {
+#pragma unroll
+            for (int h = 1; h < 8; h *= 2)
+#pragma unroll
+                for (int k = 0; k < CPL / 2; ++k)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if ((e & h) == 0) f2_bfly(p[8 * k + e], p[8 * k + e + h]);
+        } else {
+#pragma unroll
+            for (int h = 1; h < 4; h *= 2)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if ((e & h) == 0) f2_bfly(p[e], p[e + h]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) p[e] = f2_bfly_inner(p[e]);
+        }
+        // spans 8 .. 8 (LPB / 2): across lanes; the lower lane holds a, the
+        // upper b: fma(+-1, own, other) is a + b or a - b, rounded once
+#pragma unroll
+        for (int d = 1; d < Lt::LPB; d *= 2) {
+            const float sg = (lane & d) ? -1.0f : 1.0f;
+            const uint64_t s2 = f2_pack(sg, sg);
+#pragma unroll
+            for (int q = 0; q < RqPairs<CPL>::N; ++q) {
+                float lo, hi;
+                f2_unpack(p[q], lo, hi);
+                const float olo = __shfl_xor_sync(0xFFFFFFFFu, lo, d);
+                const float ohi = __shfl_xor_sync(0xFFFFFFFFu, hi, d);
+                p[q] = f2_fma(s2, p[q], f2_pack(olo, ohi));
+            }
+        }
+        // the spans of the lane's chunk index: bit 0 inside each pair, bit 1
+        // between the two pairs of chunks
+        if constexpr (CPL >= 2 && Lt::CPBL >= 2) {
+#pragma unroll
+            for (int q = 0; q < RqPairs<CPL>::N; ++q) p[q] = f2_bfly_inner(p[q]);
+        }
+        if constexpr (CPL == 4 && Lt::CPBL == 4) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f2_bfly(p[e], p[8 + e]);
+        }
+    }
+}
+
+// The 8 codes of a chunk from the bit patterns of their rounding sums (the
+// code of a value is the low byte, two's complement), in the natural K order
+// or with the even positions first (EVOD).
+template <bool EVOD>
+__device__ __forceinline__ uint2 rq_bytes8(const uint32_t (&w)[8]) {
+    if (EVOD)
+        return make_uint2(__byte_perm(__byte_perm(w[0], w[2], 0x0040), __byte_perm(w[4], w[6], 0x0040), 0x5410),
+                          __byte_perm(__byte_perm(w[1], w[3], 0x0040), __byte_perm(w[5], w[7], 0x0040), 0x5410));
+    return make_uint2(__byte_perm(__byte_perm(w[0], w[1], 0x0040), __byte_perm(w[2], w[3], 0x0040), 0x5410),
+                      __byte_perm(__byte_perm(w[4], w[5], 0x0040), __byte_perm(w[6], w[7], 0x0040), 0x5410));
+}
+
+// The sums of the pairs -> the code words of every register chunk
+template <int CPL, bool EVOD>
+__device__ __forceinline__ void rq_pairs_to_chunks(const uint64_t* m, int k, uint2 (&cw)[CPL]) {
+    uint32_t lo[8], hi[8];
+    if constexpr (CPL >= 2) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            float a, b;
+            f2_unpack(m[e], a, b);
+            lo[e] = __float_as_uint(a);
+            hi[e] = __float_as_uint(b);
+        }
+        cw[2 * k] = rq_bytes8<EVOD>(lo);
+        cw[2 * k + 1] = rq_bytes8<EVOD>(hi);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float a, b;
+            f2_unpack(m[e], a, b);
+            lo[e] = __float_as_uint(a);
+            lo[e + 4] = __float_as_uint(b);
+        }
+        cw[0] = rq_bytes8<EVOD>(lo);
+    }
+}
+
+// The codes of a lane's values.  Fast path (rs = fl(1/s), s the scale of the
+// unnormalised values): r = fma(u, rs, 1.5 2^23) rounds the exact product
+// u rs to the nearest integer n and leaves n in the low byte of r's bits; d =
+// fma(u, rs, -n) is u rs - n rounded once.  u rs is within 1.6e-5 of
+// fl(u / s) (|u / s| <= Q + 1/2, two roundings of 2^-24), so whenever |d| <=
+// 1/2 - 2^-15, n = rint(fl(u / s)), the oracle's code.  Returns whether some
+// value of the lane came closer to a half-integer than that (the warp then
+// recomputes with the IEEE division).  No clamp is needed: |u rs| <= Q (1 +
+// 2^-23) < Q + 1/2.
+template <int Q, int CPL, bool EVOD>
+__device__ __forceinline__ bool rq_codes_fast(const uint64_t (&p)[RqPairs<CPL>::N], float rs,
+                                              uint2 (&cw)[CPL]) {
+    constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+    const uint64_t rs2 = f2_pack(rs, rs);
+    const uint64_t mg2 = f2_pack(kMagic, kMagic);
+    float dmax = 0.0f;
+    constexpr int G8 = CPL >= 2 ? 8 : 4;   // pairs per group of chunks
+#pragma unroll
+    for (int k = 0; k < RqPairs<CPL>::N / G8; ++k) {
+        uint64_t m[G8];
+#pragma unroll
+        for (int e = 0; e < G8; ++e) {
+            m[e] = f2_fma(p[G8 * k + e], rs2, mg2);
+            const uint64_t nn = f2_sub(mg2, m[e]);   // -n, exact
+            float dlo, dhi;
+            f2_unpack(f2_fma(p[G8 * k + e], rs2, nn), dlo, dhi);
+            dmax = fmaxf(dmax, fmaxf(fabsf(dlo), fabsf(dhi)));
+        }
+        rq_pairs_to_chunks<CPL, EVOD>(m, k, cw);
+    }
+    return dmax > 0.5f - 3.0517578125e-5f;
+}
+
+// The oracle's steps value by value: v = fl(u norm), q = clamp(rint(fl(v /
+// s)), -Q, Q); all codes 0 for s = 0.  The fallback of the fast path (norm =
+// 1, s unnormalised: fl(u / s) is then the same quotient) and the path of
+// rows whose normalised scale would be subnormal.
+template <int Q, int CPL, bool EVOD>
+__device__ __forceinline__ void rq_codes_div(const uint64_t (&p)[RqPairs<CPL>::N], float norm, float s,
+                                             uint2 (&cw)[CPL]) {
+    constexpr float kMagic = 12582912.0f;
+    constexpr int G8 = CPL >= 2 ? 8 : 4;
+#pragma unroll
+    for (int k = 0; k < RqPairs<CPL>::N / G8; ++k) {
+        uint64_t m[G8];
+#pragma unroll
+        for (int e = 0; e < G8; ++e) {
+            float lo, hi;
+            f2_unpack(p[G8 * k + e], lo, hi);
+            float tlo = 0.0f, thi = 0.0f;
+            if (s > 0.0f) {
+                tlo = fminf(fmaxf(__fdiv_rn(lo * norm, s), static_cast<float>(-Q)), static_cast<float>(Q));
+                thi = fminf(fmaxf(__fdiv_rn(hi * norm, s), static_cast<float>(-Q)), static_cast<float>(Q));
+            }
+            m[e] = f2_pack(tlo + kMagic, thi + kMagic);
+        }
+        rq_pairs_to_chunks<CPL, EVOD>(m, k, cw);
+    }
+}
+
+// Rows blockIdx.x, blockIdx.x + gridDim.x, ... of [0, rows), one row per
+// pass of the CTA (blockDim.x / 32 warps, CPL chunks per lane, K <= 8 CPL
+// blockDim.x); the next row's loads are in flight while the current one is
+// transformed.  Q = 127 (int8 codes) or 7 (int4 codes); PACKED: int4 codes
+// two per byte (low nibble = even K index), else one code per byte.  EVOD
+// (one code per byte only): each block of 8 codes stored with its even
+// positions first (0, 2, 4, 6, 1, 3, 5, 7), the order the tensor-core GEMM
+// widens its weights in.
+template <typename InT, int G, int Q, bool PACKED, bool EVOD, int CPL>
+__device__ __forceinline__ void rq_team_rows(const InT* __restrict__ in, int rows, int K,
+                                             void* __restrict__ codes, float* __restrict__ scales,
+                                             float (&red)[2][kQuantMaxWarps]) {
+    static_assert(!(PACKED && EVOD), "even/odd order is for one code per byte");
+    using Lt = RqLayout<G, CPL>;
+    constexpr int NP = RqPairs<CPL>::N;
+    const int TL = blockDim.x;
+    const int L = threadIdx.x;
+    const int lane = L & 31, warp = L >> 5, nwarps = TL >> 5;
+    const int nC = K >> 3;
+    // chunk of register chunk i (recomputed where used: registers are scarce)
+    auto cidx = [&](int i) { return Lt::chunk(i, L, TL); };
+    RawChunk<InT> raw[CPL];
     auto fetch = [&](int r) {
 #pragma unroll
-        for (int c = 0; c < CH; ++c) {
-            const int base = base_of(c);
-            if (r < rows && present(c) && (FULL || base < K))
-                raw[c].load(in + static_cast<size_t>(r) * K + base);
-            else
-                raw[c].zero();
+        for (int i = 0; i < CPL; ++i) {
+            if (r < rows && cidx(i) < nC) raw[i].load(in + static_cast<size_t>(r) * K + cidx(i) * 8);
+            else raw[i].zero();
         }
     };
-    fetch(blockIdx.x);
+    // 2^-k: the normalisation of the transform (exact for G = 4^j)
+    constexpr float kNorm = (G == 16) ? 0.25f : (G == 64) ? 0.125f : (G == 256) ? 0.0625f : 1.0f;
 
-    int it = 0;
-    for (int row = blockIdx.x; row < rows; row += gridDim.x, ++it) {
-        float v[CH][8];
+    int row = static_cast<int>(blockIdx.x);
+    fetch(row);
+    for (int it = 0; row < rows; ++it) {
+        const int nrow = row + static_cast<int>(gridDim.x);
+        uint64_t p[NP];
+        {
+            float v[CPL][8];
 #pragma unroll
-        for (int c = 0; c < CH; ++c) raw[c].to_f32(v[c]);
-        fetch(row + gridDim.x);
+            for (int i = 0; i < CPL; ++i) raw[i].to_f32(v[i]);
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+                if constexpr (CPL >= 2) p[q] = f2_pack(v[2 * (q / 8)][q % 8], v[2 * (q / 8) + 1][q % 8]);
+                else p[q] = f2_pack(v[0][q], v[0][q + 4]);
+            }
+        }
+        fetch(nrow);
+        fwht_team<G, CPL>(p, lane);
 
         float amax = 0.0f;
 #pragma unroll
-        for (int c = 0; c < CH; ++c) {
-            if (present(c)) {
-                if (G > 0) fwht_lane8<(G > 0 ? G : 16)>(v[c], lane);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[c][j]));
-            }
+        for (int q = 0; q < NP; ++q) {
+            float lo, hi;
+            f2_unpack(p[q], lo, hi);
+            amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
         }
 #pragma unroll
         for (int d = 16; d >= 1; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, d));
@@ -262,60 +512,50 @@ __device__ __forceinline__ void rotate_quantize_rows(const InT* __restrict__ in,
         amax = rb[0];
         for (int w = 1; w < nwarps; ++w) amax = fmaxf(amax, rb[w]);
 
-        const float scale = __fdiv_rn(amax, static_cast<float>(Q));
-        const float rscale = scale > 0.0f ? __frcp_rn(scale) : 0.0f;
-        const bool tiny = scale < 1e-30f;   // row-uniform: take the clamped path
-        if (threadIdx.x == 0) scales[row] = scale;
+        uint2 cw[CPL];
+        float scale;
+        if (amax >= 0x1p-100f) {
+            const float su = __fdiv_rn(amax, static_cast<float>(Q));
+            scale = su * kNorm;
+            const bool near = rq_codes_fast<Q, CPL, EVOD>(p, __frcp_rn(su), cw);
+            if (__any_sync(0xFFFFFFFFu, near)) rq_codes_div<Q, CPL, EVOD>(p, 1.0f, su, cw);
+        } else {
+            // tiny or zero row: normalise first, as the oracle does
+            scale = __fdiv_rn(amax * kNorm, static_cast<float>(Q));
+            rq_codes_div<Q, CPL, EVOD>(p, kNorm, scale, cw);
+        }
+        if (L == 0) scales[row] = scale;
 
 #pragma unroll
-        for (int c = 0; c < CH; ++c) {
-            if (!present(c)) continue;   // warp-uniform (quant8 votes across the warp)
-            const int base = base_of(c);
-            uint32_t m[8];
-            if (tiny) quant8<Q, true>(v[c], scale, rscale, m);
-            else quant8<Q, false>(v[c], scale, rscale, m);
-            if (!FULL && base >= K) continue;
-            // the code of value j is the low byte of m[j] (two's complement)
-            const uint32_t lo = __byte_perm(__byte_perm(m[0], m[1], 0x0040), __byte_perm(m[2], m[3], 0x0040), 0x5410);
-            const uint32_t hi = __byte_perm(__byte_perm(m[4], m[5], 0x0040), __byte_perm(m[6], m[7], 0x0040), 0x5410);
-            if (!PACKED) {
-                int8_t* dst = static_cast<int8_t*>(codes) + static_cast<size_t>(row) * K + base;
-                if (EVOD)
-                    *reinterpret_cast<uint2*>(dst) =
-                        make_uint2(__byte_perm(lo, hi, 0x6420), __byte_perm(lo, hi, 0x7531));
-                else
-                    *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
+        for (int i = 0; i < CPL; ++i) {
+            if (cidx(i) >= nC) continue;
+            if constexpr (!PACKED) {
+                *reinterpret_cast<uint2*>(static_cast<int8_t*>(codes) + static_cast<size_t>(row) * K +
+                                          cidx(i) * 8) = cw[i];
             } else {
-                // low nibble = even index, high nibble = odd index: gather the
-                // even-index codes and the odd-index codes, then interleave nibbles
-                const uint32_t ev = __byte_perm(lo, hi, 0x6420);   // codes 0, 2, 4, 6
-                const uint32_t od = __byte_perm(lo, hi, 0x7531);   // codes 1, 3, 5, 7
-                const uint32_t out = (ev & 0x0F0F0F0Fu) | ((od & 0x0F0F0F0Fu) << 4);
-                uint8_t* dst = static_cast<uint8_t*>(codes) + static_cast<size_t>(row) * (K / 2) + base / 2;
-                *reinterpret_cast<uint32_t*>(dst) = out;
+                // low nibble = even index, high nibble = odd index
+                const uint32_t ev = __byte_perm(cw[i].x, cw[i].y, 0x6420);
+                const uint32_t od = __byte_perm(cw[i].x, cw[i].y, 0x7531);
+                *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(codes) + static_cast<size_t>(row) * (K / 2) +
+                                             cidx(i) * 4) =
+                    (ev & 0x0F0F0F0Fu) | ((od & 0x0F0F0F0Fu) << 4);
             }
         }
+        row = nrow;
     }
 }
 
-// Q = 127 (int8 codes) or 7 (int4 codes); PACKED: int4 codes two per byte,
-// else one code per int8.  CH = chunks per warp held in registers; the CTA
-// has blockDim.x / 32 warps (K <= warps * CH * 256).  Persistent: CTA b
-// handles rows b, b + gridDim.x, ..., and the loads of its next row are in
-// flight while it rotates and quantizes the current one.
-template <typename InT, int G, int Q, bool PACKED, int CH, bool EVOD = false>
-__global__ void __launch_bounds__(CH == 1 ? 8 * 32 : kQuantMaxWarps * 32)   // one chunk per warp: K <= 2048
-rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K,
-                            void* __restrict__ codes, float* __restrict__ scales) {
-    __shared__ float red[2][kQuantMaxWarps];   // per-warp maxima, alternate rows
-    // Under programmatic dependent launch, let the consumer grid start its
-    // prologue while this grid runs; it waits for our completion before
-    // reading the codes.
+// Persistent grid over all rows (convrot_quantize_act, tint4_pack_weights,
+// tint4_quantize_weights_int8, the fused linears).  Under programmatic
+// dependent launch the consumer grid may start its prologue while this grid
+// runs; it waits for this grid's completion before reading the codes.
+template <typename InT, int G, int Q, bool PACKED, bool EVOD, int CPL>
+__global__ void __launch_bounds__(512)
+rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K, void* __restrict__ codes,
+                            float* __restrict__ scales) {
+    __shared__ float red[2][kQuantMaxWarps];
     grid_launch_dependents();
-    if (K == static_cast<int>(blockDim.x / 32) * CH * kQuantChunk)
-        rotate_quantize_rows<InT, G, Q, PACKED, CH, true, EVOD>(in, rows, K, codes, scales, red);
-    else
-        rotate_quantize_rows<InT, G, Q, PACKED, CH, false, EVOD>(in, rows, K, codes, scales, red);
+    rq_team_rows<InT, G, Q, PACKED, EVOD, CPL>(in, rows, K, codes, scales, red);
 }
 
 }  // namespace tint4

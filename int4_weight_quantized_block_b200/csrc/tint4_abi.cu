@@ -133,15 +133,26 @@ bool valid_group(int g) { return g == 0 || g == 16 || g == 64 || g == 256; }
 // ------------------------------------------------------------------ rotate + quantize
 
 // Q = 127 or 7; PACKED: int4 codes two per byte, else one code per int8.
-// One CTA per row, one warp per 256-value chunk (two per warp above 32).
+// One row per pass of a CTA (rq_team_rows): CPL chunks of 8 values per lane
+// and as many warps as cover K.
 int num_sms(int dev);
+
+struct RqShape {
+    int cpl, warps;
+};
+
+RqShape rq_shape(int K) {
+    const int nc = K / 8;
+    const int cpl = nc <= 32 ? 1 : (nc <= 64 ? 2 : 4);
+    return RqShape{cpl, (nc + 32 * cpl - 1) / (32 * cpl)};
+}
 
 // persistent grid: as many CTAs as fit on the GPU at once (per block size,
 // looked up once per device), at most one per row
-template <typename InT, int G, int Q, bool PACKED, int CH, bool EVOD = false>
+template <typename InT, int G, int Q, bool PACKED, bool EVOD, int CPL>
 void launch_rq_persistent(const InT* in, int rows, int K, void* codes, float* scales, int threads,
                           cudaStream_t st) {
-    auto kern = rotate_quantize_rows_kernel<InT, G, Q, PACKED, CH, EVOD>;
+    auto kern = rotate_quantize_rows_kernel<InT, G, Q, PACKED, EVOD, CPL>;
     int dev = 0;
     cudaGetDevice(&dev);
     static std::atomic<int> per_sm[kMaxDevices][kQuantMaxWarps + 1];
@@ -161,14 +172,14 @@ void launch_rq_persistent(const InT* in, int rows, int K, void* codes, float* sc
 
 template <typename InT, int G, int Q, bool PACKED, bool EVOD = false>
 void launch_rq_ch(const InT* in, int rows, int K, void* codes, float* scales, cudaStream_t st) {
-    const int nchunks = (K + kQuantChunk - 1) / kQuantChunk;
-    // two chunks per warp once a row has more than 8: the per-row work (the
-    // absmax reduction, the scale's division) then spreads over more values
-    if (nchunks <= 8)
-        launch_rq_persistent<InT, G, Q, PACKED, 1, EVOD>(in, rows, K, codes, scales, nchunks * 32, st);
+    const RqShape sh = rq_shape(K);
+    const int threads = sh.warps * 32;
+    if (sh.cpl == 1)
+        launch_rq_persistent<InT, G, Q, PACKED, EVOD, 1>(in, rows, K, codes, scales, threads, st);
+    else if (sh.cpl == 2)
+        launch_rq_persistent<InT, G, Q, PACKED, EVOD, 2>(in, rows, K, codes, scales, threads, st);
     else
-        launch_rq_persistent<InT, G, Q, PACKED, 2, EVOD>(in, rows, K, codes, scales,
-                                                   ((nchunks + 1) / 2) * 32, st);
+        launch_rq_persistent<InT, G, Q, PACKED, EVOD, 4>(in, rows, K, codes, scales, threads, st);
 }
 
 template <typename InT, int Q, bool PACKED, bool EVOD = false>
@@ -406,6 +417,18 @@ tint4_status launch_gemm(const void* a, const uint8_t* w, const float* st, const
     return launch_gemm_tmem<OUT_I32, A_INT4, false, EVOD>(a, st, grp, &w, M, K, stream, pdl);
 }
 
+// The fused linears' workspace: the activation codes (one byte per code) and
+// the token scales, each part 256-byte aligned.
+struct LinearWs {
+    uint8_t* codes;
+    float* tok_scale;
+};
+
+LinearWs linear_ws(void* ws, int M, int K) {
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    return LinearWs{b, reinterpret_cast<float*>(b + align_up(static_cast<size_t>(M) * K, 256))};
+}
+
 tint4_status gemm_entry(bool a_int4, const void* a, const float* tok_scale, const uint8_t* w,
                         const float* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
                         int N, int K, void* stream) {
@@ -424,6 +447,36 @@ tint4_status gemm_entry(bool a_int4, const void* a, const float* tok_scale, cons
                                               as_stream(stream), false);
 }
 
+// The fused linear after its checks (M > 0; ws: a workspace of at least
+// convrot_linear_workspace_size bytes, 256-byte aligned).
+tint4_status linear_run(int bits, const tint4_bf16* x, const uint8_t* w_packed,
+                        const float* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
+                        int N, int K, int group, void* ws, cudaStream_t st) {
+    const auto* b = reinterpret_cast<const __nv_bfloat16*>(bias);
+    if (M <= kFuseMaxRows && K <= kS8FuseMaxK) {
+        // decode: one launch, the codes never leave the CTA
+        const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+        auto* yb = reinterpret_cast<__nv_bfloat16*>(y);
+        return bits == 8 ? launch_linear_small_fused_g<127>(xb, w_packed, row_scale, b, yb, M, N, K,
+                                                            group, st)
+                         : launch_linear_small_fused_g<7>(xb, w_packed, row_scale, b, yb, M, N, K,
+                                                          group, st);
+    }
+    // one int8 per code for both widths: the W4A4 codes (in [-7, 7]) are kept
+    // one per byte in the workspace and run through the W4A8 kernel, whose
+    // int32 sums are the same numbers
+    const LinearWs w = linear_ws(ws, M, K);
+    if (bits == 8) launch_linear_codes<127>(x, M, K, group, w.codes, w.tok_scale, st);
+    else launch_linear_codes<7>(x, M, K, group, w.codes, w.tok_scale, st);
+    tint4_status s = last_launch_status();
+    if (s != TINT4_OK) return s;
+    return linear_codes_evod(M)
+               ? launch_gemm<false, false, true>(w.codes, w_packed, w.tok_scale, row_scale, b, y, M,
+                                                 N, K, st, true)
+               : launch_gemm<false, false>(w.codes, w_packed, w.tok_scale, row_scale, b, y, M, N, K,
+                                           st, true);
+}
+
 tint4_status linear_entry(int bits, const tint4_bf16* x, const uint8_t* w_packed,
                           const float* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
                           int N, int K, int group, void* workspace, size_t workspace_bytes,
@@ -440,32 +493,8 @@ tint4_status linear_entry(int bits, const tint4_bf16* x, const uint8_t* w_packed
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TINT4_ERR_MISALIGNED;
     if ((s = check_device()) != TINT4_OK) return s;
     if (M == 0) return TINT4_OK;
-    if (M <= kFuseMaxRows && K <= kS8FuseMaxK) {
-        // decode: one launch, the codes never leave the CTA
-        const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
-        const auto* b = reinterpret_cast<const __nv_bfloat16*>(bias);
-        auto* yb = reinterpret_cast<__nv_bfloat16*>(y);
-        return bits == 8 ? launch_linear_small_fused_g<127>(xb, w_packed, row_scale, b, yb, M, N, K,
-                                                            group, as_stream(stream))
-                         : launch_linear_small_fused_g<7>(xb, w_packed, row_scale, b, yb, M, N, K,
-                                                          group, as_stream(stream));
-    }
-    // one int8 per code for both widths: the W4A4 codes (in [-7, 7]) are kept
-    // one per byte in the workspace and run through the W4A8 kernel, whose
-    // int32 sums are the same numbers
-    const size_t code_bytes = static_cast<size_t>(M) * K;
-    uint8_t* codes = static_cast<uint8_t*>(workspace);
-    float* tok_scale = reinterpret_cast<float*>(codes + align_up(code_bytes, 256));
-    cudaStream_t st = as_stream(stream);
-    const auto* b = reinterpret_cast<const __nv_bfloat16*>(bias);
-    if (bits == 8) launch_linear_codes<127>(x, M, K, group, codes, tok_scale, st);
-    else launch_linear_codes<7>(x, M, K, group, codes, tok_scale, st);
-    if ((s = last_launch_status()) != TINT4_OK) return s;
-    return linear_codes_evod(M)
-               ? launch_gemm<false, false, true>(codes, w_packed, tok_scale, row_scale, b, y, M,
-                                                 N, K, st, true)
-               : launch_gemm<false, false>(codes, w_packed, tok_scale, row_scale, b, y, M, N, K,
-                                           st, true);
+    return linear_run(bits, x, w_packed, row_scale, bias, y, M, N, K, group, workspace,
+                      as_stream(stream));
 }
 
 // ------------------------------------------------------------------ W4A16
@@ -582,18 +611,45 @@ static __device__ __align__(256) uint8_t g_static_linear_scratch[kStaticScratchB
 
 std::mutex g_static_scratch_mu;
 void* g_static_scratch_ptr[kMaxDevices];
+void* g_static_scratch_ctx[kMaxDevices];   // the context the address belongs to
 
-// Device address of the scratch array on `dev` (the current device); the
-// first call on a device resolves it.  nullptr on failure.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// Device address of the scratch array on `dev` (the current device), looked
+// up on the first call and again whenever the device's context has changed
+// since (a context rebuilt after cudaDeviceReset loads the module anew, and
+// the array may move).  nullptr on failure.
 void* static_scratch_address(int dev) {
     std::lock_guard<std::mutex> lock(g_static_scratch_mu);
-    if (g_static_scratch_ptr[dev] == nullptr) {
+    CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    if (get_ctx == nullptr) return nullptr;
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+    if (ctx == nullptr || g_static_scratch_ptr[dev] == nullptr || g_static_scratch_ctx[dev] != ctx) {
+        // (the lookup also makes the device's primary context current)
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_static_linear_scratch) != cudaSuccess) {
+        if (cudaGetSymbolAddress(&p, g_static_linear_scratch) != cudaSuccess ||
+            get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) {
             cudaGetLastError();
             return nullptr;
         }
         g_static_scratch_ptr[dev] = p;
+        g_static_scratch_ctx[dev] = ctx;
     }
     return g_static_scratch_ptr[dev];
 }
@@ -864,6 +920,10 @@ tint4_status w4a4_gemm(const uint8_t* a_packed, const float* tok_scale, const ui
     return gemm_entry(true, a_packed, tok_scale, w_packed, row_scale, bias, y, M, N, K, stream);
 }
 
+size_t convrot_w4a8_linear_workspace(int M, int K) {
+    return convrot_linear_workspace_size(M, K, 8);
+}
+
 size_t convrot_linear_workspace_size(int M, int K, int bits) {
     if (M < 0 || K < 0 || (bits != 8 && bits != 4)) return 0;
     const size_t code_bytes = static_cast<size_t>(M) * K;   // one byte per code, both widths
@@ -914,15 +974,14 @@ tint4_status convrot_w4a8_linear_grouped(const tint4_bf16* x,
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TINT4_ERR_MISALIGNED;
     if ((s = check_device()) != TINT4_OK) return s;
     if (M == 0) return TINT4_OK;
-    int8_t* codes = static_cast<int8_t*>(workspace);
-    float* tok_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                                align_up(static_cast<size_t>(M) * K, 256));
+    const LinearWs w = linear_ws(workspace, M, K);
+    int8_t* codes = reinterpret_cast<int8_t*>(w.codes);
     cudaStream_t st = as_stream(stream);
-    launch_linear_codes<127>(x, M, K, group, codes, tok_scale, st);
+    launch_linear_codes<127>(x, M, K, group, codes, w.tok_scale, st);
     if ((s = last_launch_status()) != TINT4_OK) return s;
     return linear_codes_evod(M)
-               ? launch_gemm_grouped<true>(codes, tok_scale, groups, num_groups, M, K, st, true)
-               : launch_gemm_grouped(codes, tok_scale, groups, num_groups, M, K, st, true);
+               ? launch_gemm_grouped<true>(codes, w.tok_scale, groups, num_groups, M, K, st, true)
+               : launch_gemm_grouped(codes, w.tok_scale, groups, num_groups, M, K, st, true);
 }
 
 tint4_status tint4_pack_weights_groupwise(const float* W, int N, int K, int group, int asym,
@@ -1070,19 +1129,10 @@ tint4_status convrot_w4a8_linear_noalloc(const tint4_bf16* x, const uint8_t* w_p
     int dev = 0;
     if ((s = check_device(&dev)) != TINT4_OK) return s;
     if (M == 0) return TINT4_OK;
-    uint8_t* codes = static_cast<uint8_t*>(static_scratch_address(dev));
-    if (codes == nullptr) return TINT4_ERR_CUDA;
-    float* tok_scale =
-        reinterpret_cast<float*>(codes + align_up(static_cast<size_t>(M) * K, 256));
-    cudaStream_t st = as_stream(stream);
-    launch_linear_codes<127>(x, M, K, group, codes, tok_scale, st);
-    if ((s = last_launch_status()) != TINT4_OK) return s;
-    const auto* b = reinterpret_cast<const __nv_bfloat16*>(bias);
-    return linear_codes_evod(M)
-               ? launch_gemm<false, false, true>(codes, w_packed, tok_scale, row_scale, b, y, M,
-                                                 N, K, st, true)
-               : launch_gemm<false, false>(codes, w_packed, tok_scale, row_scale, b, y, M, N, K,
-                                           st, true);
+    void* scratch = static_scratch_address(dev);
+    if (scratch == nullptr) return TINT4_ERR_CUDA;
+    return linear_run(8, x, w_packed, row_scale, bias, y, M, N, K, group, scratch,
+                      as_stream(stream));
 }
 
 tint4_status w4a16_gemv_gemm(const tint4_bf16* x, const uint8_t* w_q, const tint4_bf16* scale,

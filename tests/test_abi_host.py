@@ -62,11 +62,15 @@ def test_version_and_status_strings(lib):
 
 
 def test_workspace_size(lib):
-    assert lib.convrot_linear_workspace_size(4608, 3072, 8) == 4608 * 3072 + 4608 * 4 + 0
+    # codes | token scales, each part 256-aligned
+    assert lib.convrot_linear_workspace_size(4608, 3072, 8) == 4608 * 3072 + 4608 * 4
     assert lib.convrot_linear_workspace_size(4608, 3072, 4) == 4608 * 3072 + 4608 * 4
     assert lib.convrot_linear_workspace_size(3, 64, 8) == 256 + 256
     assert lib.convrot_linear_workspace_size(3, 64, 5) == 0
     assert lib.convrot_linear_workspace_size(-1, 64, 8) == 0
+    # the boundary specification's name for the W4A8 size
+    for M, K in ((4608, 3072), (3, 64), (1, 4096)):
+        assert lib.convrot_w4a8_linear_workspace(M, K) == lib.convrot_linear_workspace_size(M, K, 8)
 
 
 NULL = None
