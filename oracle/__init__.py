@@ -75,7 +75,10 @@ def _load():
             "oracle_w4a16_dequant_f64": [P, P, P, P, I, I, I, I, P],
             "oracle_w4a16_weights_f64": [P, P, P, I, I, I, I, P],
             "oracle_quantize_weights_int8": [P, I, I, I, P, P],
+            "oracle_quantize_weights_int8_ex": [P, I, I, I, I, P, P],
             "oracle_pack_weights_groupwise": [P, I, I, I, I, I, P, P, P, P],
+            "oracle_pack_weights_groupwise_ex": [P, I, I, I, I, I, I, P, P, P, P],
+            "oracle_round_f16": [P, L, P],
             "oracle_gemm_groupwise_f64": [P, P, P, P, P, P, I, I, I, I, P, P],
             "oracle_gemm_groupwise_sampled_f64": [P, P, P, P, P, P, I, I, I, I, P, L, P, P],
             "oracle_round_bf16": [P, L, P],
@@ -209,20 +212,54 @@ def pack_weights(W: np.ndarray, g: int):
     return packed, scale, codes
 
 
-def quantize_weights_int8(W: np.ndarray, g: int):
+def quantize_weights_int8(W: np.ndarray, g: int, scale_f16: bool = False):
     """Twin of ``tint4_quantize_weights_int8``: rotate W along K, per-row
     symmetric int8 codes [N, K] in [-127, 127] and fp32 row scales [N].
 
     "ComfyUI-INT-Crush", "Inference > INT8" (int8 weights x int8 activations,
     int32 accumulation); the rotation and rounding are those of the int4
-    weights ("Weight Format", "Forward Pass")."""
+    weights ("Weight Format", "Forward Pass").  scale_f16 (twin of
+    ``tint4_quantize_weights_int8_f16``; "Weight Format": INT8 scales fp16
+    [out, 1]): each scale is rounded to fp16 and the codes are taken against
+    that stored scale; the scales come back as float32 values on the fp16
+    grid (``f16_bits`` gives their bit patterns)."""
     Wc = _c(W, np.float32)
     N, K = Wc.shape
     codes = np.empty((N, K), dtype=np.int8)
     scale = np.empty(N, dtype=np.float32)
-    _check(_load().oracle_quantize_weights_int8(_ptr(Wc), N, K, g, _ptr(codes), _ptr(scale)),
-           "quantize_weights_int8")
+    _check(_load().oracle_quantize_weights_int8_ex(_ptr(Wc), N, K, g, int(scale_f16), _ptr(codes),
+                                                   _ptr(scale)), "quantize_weights_int8")
     return codes, scale
+
+
+def round_f16(v: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest fp16 number (ties to even; from
+    65520 on infinity), returned as float32."""
+    a = _c(v, np.float32)
+    out = np.empty(a.shape, dtype=np.float32)
+    _check(_load().oracle_round_f16(_ptr(a), a.size, _ptr(out)), "round_f16")
+    return out
+
+
+def f16_bits(v: np.ndarray) -> np.ndarray:
+    """IEEE fp16 bit patterns (uint16) of float32 values that lie on the fp16
+    grid (the oracle's fp16 scales): sign bit, 5-bit biased exponent, 10-bit
+    fraction; subnormals are multiples of 2^-24."""
+    a = np.asarray(v, np.float32)
+    mag = np.abs(a.astype(np.float64))
+    finite = np.isfinite(mag)
+    m = np.where(finite, mag, 1.0)
+    e = np.floor(np.log2(np.where(m > 0, m, 1.0)))
+    normal = finite & (m >= 2.0 ** -14)
+    frac_n = np.where(normal, m / 2.0 ** e - 1.0, 0.0) * 1024.0
+    sub_n = np.where(finite & ~normal, m * 2.0 ** 24, 0.0)
+    if np.any(np.isnan(a)) or np.any(finite & (mag > 65504.0)) or \
+            np.any(frac_n != np.rint(frac_n)) or np.any(sub_n != np.rint(sub_n)):
+        raise ValueError("values not on the fp16 grid")
+    out = np.where(normal, ((e.astype(np.int64) + 15) << 10) | frac_n.astype(np.int64),
+                   sub_n.astype(np.int64))
+    out = np.where(finite, out, 0x7C00)
+    return (out | np.where(np.signbit(a), 0x8000, 0)).astype(np.uint16)
 
 
 def quantize_act(x_bits: np.ndarray, g: int, bits: int):
@@ -353,22 +390,28 @@ def convrot_linear_f64(x_bits, w_packed, row_scale, g, act_bits, bias_bits=None)
 # Group-wise W4A8 (per row and K group weight scales; symmetric or asymmetric)
 # --------------------------------------------------------------------------
 
-def pack_weights_groupwise(W: np.ndarray, g: int, G: int = 128, asym: bool = False):
+def pack_weights_groupwise(W: np.ndarray, g: int, G: int = 128, asym: bool = False,
+                           scale_f16: bool = False):
     """Twin of ``tint4_pack_weights_groupwise``: rotate W along K, then int4
     codes per (row, G-wide K group).
 
     Returns (packed uint8 [N, K/2], scale fp32 [N, K/G], zero uint8 [N, K/G]
     or None, codes int8 [N, K]).  "ComfyUI-INT-Crush", "Weight Format"
     (scales [out, num_groups]); "feat: packed int4 convrot model loading and
-    dispatch", "Summary" (the asymmetric W4A8 format)."""
+    dispatch", "Summary" (the asymmetric W4A8 format).  scale_f16 (twin of
+    ``tint4_pack_weights_groupwise_f16``; "Weight Format": the scales are
+    stored as fp16): each group scale is rounded to fp16 first and the zero
+    point and codes are taken against that stored scale; the scales come back
+    as float32 values on the fp16 grid."""
     Wc = _c(W, np.float32)
     N, K = Wc.shape
     packed = np.empty((N, K // 2), dtype=np.uint8)
     scale = np.empty((N, K // G), dtype=np.float32)
     zero = np.empty((N, K // G), dtype=np.uint8) if asym else None
     codes = np.empty((N, K), dtype=np.int8)
-    _check(_load().oracle_pack_weights_groupwise(_ptr(Wc), N, K, g, G, int(asym), _ptr(packed),
-                                                 _ptr(scale), _ptr(zero), _ptr(codes)),
+    _check(_load().oracle_pack_weights_groupwise_ex(_ptr(Wc), N, K, g, G, int(asym),
+                                                    int(scale_f16), _ptr(packed), _ptr(scale),
+                                                    _ptr(zero), _ptr(codes)),
            "pack_weights_groupwise")
     return packed, scale, zero, codes
 

@@ -88,6 +88,35 @@ static uint16_t double_to_bf16_bits(double v) {
     return (uint16_t)(u >> 16);
 }
 
+/* Round a float to the nearest IEEE fp16 number (ties to even), returned as
+ * the float of the same value (every fp16 value is exact in fp32).  fp16 has
+ * 11 significant bits and exponents -14..15; below 2^-14 the grid is the
+ * subnormal spacing 2^-24; a result above the largest finite value 65504
+ * (that is, from 65520 on) is infinity.  "ComfyUI-INT-Crush", "Weight
+ * Format": the stored weight scales are fp16. */
+static float round_to_f16(float v) {
+    if (isnan(v)) return v;
+    double a = fabs((double)v);
+    double r;
+    if (a == 0.0) {
+        r = 0.0;
+    } else if (a < ldexp(1.0, -14)) {
+        r = nearbyint(a * ldexp(1.0, 24)) * ldexp(1.0, -24);
+    } else {
+        int e;
+        double m = frexp(a, &e);              /* a = m * 2^e, m in [0.5, 1) */
+        r = ldexp(nearbyint(ldexp(m, 11)), e - 11);
+    }
+    if (r > 65504.0) r = INFINITY;
+    return (float)copysign(r, (double)v);
+}
+
+int oracle_round_f16(const float* v, long n, float* out) {
+    if ((!v || !out) && n > 0) return ORACLE_BAD_ARG;
+    for (long i = 0; i < n; ++i) out[i] = round_to_f16(v[i]);
+    return ORACLE_OK;
+}
+
 static int is_power_of_four(int g) {
     if (g < 4) return 0;
     while (g > 1) {
@@ -164,13 +193,15 @@ int oracle_rotate_rows_f32(float* rows, long nrows, int K, int g) {
 /* One row of K fp32 values -> codes in [-qmax, qmax] and one fp32 scale.
  * scale = absmax / qmax; code = clamp(rne(v / scale)); zero row -> scale 0,
  * codes 0. */
-static void quantize_row(const float* v, int K, int qmax, int8_t* q, float* scale) {
+static void quantize_row_s(const float* v, int K, int qmax, int s16, int8_t* q, float* scale) {
     float amax = 0.0f;
     for (int k = 0; k < K; ++k) {
         float a = fabsf(v[k]);
         if (a > amax) amax = a;
     }
     float s = amax / (float)qmax;
+    /* fp16 storage: the codes are taken against the stored scale */
+    if (s16) s = round_to_f16(s);
     *scale = s;
     for (int k = 0; k < K; ++k) {
         int c = 0;
@@ -182,6 +213,10 @@ static void quantize_row(const float* v, int K, int qmax, int8_t* q, float* scal
         }
         q[k] = (int8_t)c;
     }
+}
+
+static void quantize_row(const float* v, int K, int qmax, int8_t* q, float* scale) {
+    quantize_row_s(v, K, qmax, 0, q, scale);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -254,8 +289,18 @@ int oracle_pack_weights(const float* W, int N, int K, int g, uint8_t* packed,
  * multiplies int8 weights by int8 activations with int32 accumulation):
  * W fp32 [N, K] -> rotate each g-block along K -> per-row symmetric int8
  * codes in [-127, 127] [N, K] with an fp32 row scale absmax / 127. */
+/* As oracle_quantize_weights_int8, with the row scale rounded to fp16 (and
+ * the codes taken against that stored scale) when s16 != 0. */
+int oracle_quantize_weights_int8_ex(const float* W, int N, int K, int g, int s16, int8_t* codes,
+                                    float* row_scale);
+
 int oracle_quantize_weights_int8(const float* W, int N, int K, int g, int8_t* codes,
                                  float* row_scale) {
+    return oracle_quantize_weights_int8_ex(W, N, K, g, 0, codes, row_scale);
+}
+
+int oracle_quantize_weights_int8_ex(const float* W, int N, int K, int g, int s16, int8_t* codes,
+                                    float* row_scale) {
     if (!W || !codes || !row_scale || N <= 0 || K <= 0) return ORACLE_BAD_ARG;
     if (g != 0 && (!is_power_of_four(g) || K % g)) return ORACLE_BAD_ARG;
     int bad = 0;
@@ -270,7 +315,7 @@ int oracle_quantize_weights_int8(const float* W, int N, int K, int g, int8_t* co
             for (int n = 0; n < N; ++n) {
                 memcpy(v, W + (long)n * K, sizeof(float) * (size_t)K);
                 if (g) for (int b = 0; b < K; b += g) fwht_f32_block(v + b, g);
-                quantize_row(v, K, 127, codes + (long)n * K, &row_scale[n]);
+                quantize_row_s(v, K, 127, s16, codes + (long)n * K, &row_scale[n]);
             }
         }
         free(v);
@@ -566,13 +611,15 @@ int oracle_w4a16(const uint16_t* x, const uint8_t* q, const uint16_t* s, const u
  *  - an all-zero group has s = 0, z = 0 and q = 0;
  *  - all of it in fp32 with IEEE division and round half to even (the codes
  *    are decisions, taken in the kernel's precision). */
-static void quantize_group_asym(const float* v, int G, int8_t* q, float* scale, uint8_t* zero) {
+static void quantize_group_asym(const float* v, int G, int s16, int8_t* q, float* scale,
+                                uint8_t* zero) {
     float lo = 0.0f, hi = 0.0f;
     for (int k = 0; k < G; ++k) {
         if (v[k] < lo) lo = v[k];
         if (v[k] > hi) hi = v[k];
     }
     float s = (hi - lo) / 15.0f;
+    if (s16) s = round_to_f16(s);   /* the zero point and codes use the stored scale */
     int z = 0;
     if (s > 0.0f) {
         float t = rintf(-lo / s);
@@ -598,8 +645,19 @@ static void quantize_group_asym(const float* v, int G, int8_t* q, float* scale, 
  * [N, K/2], byte j holding code 2j in its low nibble.  codes (optional)
  * receives the codes as int8 [N, K]: signed for the symmetric form, 0..15 for
  * the asymmetric one.  zero may be NULL when asym == 0. */
+/* As oracle_pack_weights_groupwise, with every group scale rounded to fp16
+ * (and the zero points and codes taken against that stored scale) when
+ * s16 != 0; scale then holds the fp16 values as floats. */
+int oracle_pack_weights_groupwise_ex(const float* W, int N, int K, int g, int G, int asym, int s16,
+                                     uint8_t* packed, float* scale, uint8_t* zero, int8_t* codes);
+
 int oracle_pack_weights_groupwise(const float* W, int N, int K, int g, int G, int asym,
                                   uint8_t* packed, float* scale, uint8_t* zero, int8_t* codes) {
+    return oracle_pack_weights_groupwise_ex(W, N, K, g, G, asym, 0, packed, scale, zero, codes);
+}
+
+int oracle_pack_weights_groupwise_ex(const float* W, int N, int K, int g, int G, int asym, int s16,
+                                     uint8_t* packed, float* scale, uint8_t* zero, int8_t* codes) {
     if (!W || !packed || !scale || (asym && !zero) || N <= 0 || K <= 0 || K % 2 || G <= 0 ||
         G % 2 || K % G)
         return ORACLE_BAD_ARG;
@@ -620,11 +678,11 @@ int oracle_pack_weights_groupwise(const float* W, int N, int K, int g, int G, in
                 if (g) for (int b = 0; b < K; b += g) fwht_f32_block(v + b, g);
                 for (int j = 0; j < ng; ++j) {
                     if (asym)
-                        quantize_group_asym(v + (long)j * G, G, q + (long)j * G,
+                        quantize_group_asym(v + (long)j * G, G, s16, q + (long)j * G,
                                             &scale[(long)n * ng + j], &zero[(long)n * ng + j]);
                     else
-                        quantize_row(v + (long)j * G, G, 7, q + (long)j * G,
-                                     &scale[(long)n * ng + j]);
+                        quantize_row_s(v + (long)j * G, G, 7, s16, q + (long)j * G,
+                                       &scale[(long)n * ng + j]);
                 }
                 oracle_pack_int4(q, 1, K, packed + (long)n * (K / 2));
                 if (codes) memcpy(codes + (long)n * K, q, (size_t)K);

@@ -580,6 +580,78 @@ def test_w4a16_tensor_core_bound_holds_for_an_fp32_evaluation():
     assert np.all(np.abs(acc - ref) <= w4a16_tc_error(op.x, wd))
 
 
+# ---------------------------------------------------------------- fp16 scales
+
+def test_round_f16_matches_ieee_half():
+    """The oracle's fp16 rounding against numpy's IEEE half conversion (an
+    independent implementation): random magnitudes over and past the whole
+    fp16 range, subnormals, ties, and the overflow boundary (65504 stays,
+    65520 becomes infinity)."""
+    rng = np.random.default_rng(40)
+    v = (rng.standard_normal(200000) * np.exp2(rng.uniform(-30, 18, 200000))).astype(np.float32)
+    edges = np.array([0.0, -0.0, 65504.0, 65519.0, 65520.0, 1e9, 2.0 ** -24, 2.0 ** -25,
+                      3 * 2.0 ** -25, 2.0 ** -14, 1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11,
+                      -(1 + 2.0 ** -11)], np.float32)
+    v = np.concatenate([v, edges])
+    with np.errstate(over="ignore"):
+        ref = v.astype(np.float16)
+    got = oracle.round_f16(v)
+    assert np.array_equal(got.view(np.uint32), ref.astype(np.float32).view(np.uint32))
+    assert np.array_equal(oracle.f16_bits(got), ref.view(np.uint16))
+
+
+def test_fp16_scale_golden():
+    """Hand-derived rows where rounding the stored scale to fp16 changes a
+    code (tests/golden/fp16_scale_codes.json): group-wise symmetric and
+    asymmetric int4, and int8 (W8A8) weights."""
+    d = golden("fp16_scale_codes.json")
+    K, G = d["K"], d["group"]
+
+    def row(head):
+        W = np.zeros((1, K), np.float32)
+        W[0, :2] = head
+        return W
+
+    for asym, key in ((False, "sym"), (True, "asym")):
+        wp, sc, z, codes = oracle.pack_weights_groupwise(row(d["row_" + key]), 0, G, asym,
+                                                         scale_f16=True)
+        assert codes[0, :2].tolist() == d["codes_" + key] and not codes[0, 2:].any()
+        assert sc[0, 0] == d["scale"] and oracle.f16_bits(sc)[0, 0] == d["scale_f16_bits"]
+        assert wp[0, 0] == d["byte0_" + key]
+        if asym:
+            assert z[0, 0] == d["zero_asym"]
+        _, sc32, _, codes32 = oracle.pack_weights_groupwise(row(d["row_" + key]), 0, G, asym)
+        assert codes32[0, :2].tolist() == d["codes_" + key + "_f32_scale"]
+        assert sc32[0, 0] == d["scale_f32"]
+    codes, sc = oracle.quantize_weights_int8(row(d["row_int8"]), 0, scale_f16=True)
+    assert codes[0, :2].tolist() == d["codes_int8"] and sc[0] == d["scale"]
+    codes32, sc32 = oracle.quantize_weights_int8(row(d["row_int8"]), 0)
+    assert codes32[0, :2].tolist() == d["codes_int8_f32_scale"] and sc32[0] == d["scale_f32"]
+
+
+@pytest.mark.parametrize("g", [0, 64, 256])
+def test_fp16_scale_quantization_error_bound(g):
+    """With the stored fp16 scale s, every weight is within s / 2 of s (q - z)
+    (s q for the symmetric forms), the scales lie on the fp16 grid, and the
+    extremes still reach the end codes (the fp16 rounding moves a scale by at
+    most 2^-11 of itself, far less than half a step of the codes)."""
+    N, K = 24, 512
+    W = inputs.weights(N, K, seed=41)
+    v = oracle.rotate_rows_f32(W.copy(), g).astype(np.float64) if g else W.astype(np.float64)
+    for asym in (False, True):
+        _, sc, z, codes = oracle.pack_weights_groupwise(W, g, 128, asym, scale_f16=True)
+        assert np.array_equal(oracle.round_f16(sc), sc)
+        s = np.repeat(sc.astype(np.float64), 128, axis=1)
+        zz = np.repeat(z.astype(np.float64), 128, axis=1) if asym else 0.0
+        assert np.all(np.abs(v - s * (codes - zz)) <= s / 2 * (1 + 1e-6))
+        if not asym:
+            assert np.all(np.abs(codes).reshape(N, -1, 128).max(axis=2) == 7)
+    codes, sc = oracle.quantize_weights_int8(W, g, scale_f16=True)
+    assert np.array_equal(oracle.round_f16(sc), sc)
+    assert np.all(np.abs(v - sc[:, None].astype(np.float64) * codes) <= sc[:, None] / 2 * (1 + 1e-6))
+    assert np.all(np.abs(codes).max(axis=1) == 127)
+
+
 # ---------------------------------------------------------------- fp64 outputs and the comparison
 
 def test_unrounded_outputs_round_to_the_bf16_outputs():

@@ -61,6 +61,33 @@ def test_noalloc_matches_workspace_entry_two_calls(case):
     assert t4.tint4_get_device_error() == 0
 
 
+@pytest.mark.parametrize("M", [1, 9])
+def test_noalloc_small_m_against_oracle(M):
+    """Decode-sized calls: one token runs the one-launch small-M path of
+    convrot_w4a8_linear (the GEMM's CTAs rotate and quantize x themselves),
+    nine tokens the quantize grid and the streaming GEMM with natural-order
+    codes in the fixed array.  Both are checked against the oracle, on two
+    calls in a row, and against the workspace entry."""
+    N, K, g = 256, 4096, 256
+    xb = inputs.activations(M, K, seed=90 + M)
+    W = inputs.weights(N, K, seed=91 + M)
+    wp_ref, sr_ref, _ = oracle.pack_weights(W, g)
+    x = _bf16(xb)
+    wp = torch.from_numpy(wp_ref).cuda()
+    sr = torch.from_numpy(sr_ref).cuda()
+    ref64 = oracle.convrot_linear_f64(xb, wp_ref, sr_ref, g, 8)
+    y_ws = t4.convrot_w4a8_linear(x, wp, sr, g)
+    for _ in range(2):
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        assert _noalloc(x, wp, sr, g, y) == 0
+        torch.cuda.synchronize()
+        got = y.view(torch.int16).cpu().numpy().view(np.uint16)
+        c = check_bf16(got, ref64, gemm_eval_error(ref64))
+        assert c.ok, str(c)
+        assert np.array_equal(got, y_ws.view(torch.int16).cpu().numpy().view(np.uint16))
+    assert t4.tint4_get_device_error() == 0
+
+
 def test_noalloc_against_oracle_and_size_limit():
     M, N, K, g = 96, 320, 512, 64
     xb = inputs.activations(M, K, seed=77)
