@@ -74,6 +74,9 @@ typedef enum {
 } tint4_status;
 
 typedef uint16_t tint4_bf16;
+/* IEEE binary16 bit patterns: the stored weight-scale format of
+ * "ComfyUI-INT-Crush", "Weight Format". */
+typedef uint16_t tint4_f16;
 
 /* ABI version, bumped on any signature change. */
 int tint4_abi_version(void);
@@ -220,6 +223,24 @@ tint4_status convrot_w8a8_linear(const tint4_bf16* x, const int8_t* w_int8,
                                  size_t workspace_bytes, void* stream);
 
 /*
+ * W8A8 with the row scales in the pages' stored INT8 format, fp16 [out, 1]
+ * ("ComfyUI-INT-Crush", "Weight Format"): tint4_quantize_weights_int8_f16
+ * rounds each row scale absmax / 127 to the nearest fp16 (ties to even) and
+ * takes the codes against that stored value (a scale that rounds to 0 or to
+ * infinity gives codes 0); the GEMM and the fused linear widen it exactly.
+ * Otherwise as the fp32 forms above.
+ */
+tint4_status tint4_quantize_weights_int8_f16(const float* W, int N, int K, int group,
+                                             int8_t* w_int8, tint4_f16* row_scale, void* stream);
+tint4_status w8a8_gemm_f16(const int8_t* codes, const float* tok_scale, const int8_t* w_int8,
+                           const tint4_f16* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
+                           int N, int K, void* stream);
+tint4_status convrot_w8a8_linear_f16(const tint4_bf16* x, const int8_t* w_int8,
+                                     const tint4_f16* row_scale, const tint4_bf16* bias,
+                                     tint4_bf16* y, int M, int N, int K, int group, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/*
  * Group-wise W4A8 ("ComfyUI-INT-Crush", "Weight Format": INT4 weight scales
  * of shape [out, num_groups]; stable-diffusion.cpp "feat: packed int4
  * convrot model loading and dispatch", "Summary": the asymmetric W4A8 format
@@ -266,6 +287,29 @@ tint4_status convrot_w4a8_linear_groupwise(const tint4_bf16* x, const uint8_t* w
                                            const tint4_bf16* bias, tint4_bf16* y, int M, int N,
                                            int K, int group, void* workspace,
                                            size_t workspace_bytes, void* stream);
+
+/*
+ * The same three calls with the scales in the pages' stored format: fp16
+ * [out, num_groups] ("ComfyUI-INT-Crush", "Weight Format").  The packing
+ * computes each group scale as above in fp32, rounds it to the nearest fp16
+ * (ties to even; 65520 and above becomes infinity), and takes the zero point
+ * and the codes against that stored value; a scale that rounds to 0 (or to
+ * infinity) gives codes 0 (and zero point 0).  The GEMM and the fused linear
+ * widen each fp16 scale exactly and otherwise compute as the fp32 forms.
+ * Arguments, rules and errors as above.
+ */
+tint4_status tint4_pack_weights_groupwise_f16(const float* W, int N, int K, int group, int asym,
+                                              uint8_t* w_packed, tint4_f16* w_scale,
+                                              uint8_t* w_zero, void* stream);
+tint4_status w4a8_gemm_groupwise_f16(const int8_t* a, const float* tok_scale,
+                                     const uint8_t* w_packed, const tint4_f16* w_scale,
+                                     const uint8_t* w_zero, const tint4_bf16* bias, tint4_bf16* y,
+                                     int M, int N, int K, void* stream);
+tint4_status convrot_w4a8_linear_groupwise_f16(const tint4_bf16* x, const uint8_t* w_packed,
+                                               const tint4_f16* w_scale, const uint8_t* w_zero,
+                                               const tint4_bf16* bias, tint4_bf16* y, int M, int N,
+                                               int K, int group, void* workspace,
+                                               size_t workspace_bytes, void* stream);
 
 /*
  * Grouped GEMM: the same activation codes times up to TINT4_MAX_GROUPS

@@ -194,18 +194,30 @@ def convrot_w4a8_linear_noalloc(x, w_packed, row_scale, group, bias=None, y=None
     return y
 
 
-def tint4_quantize_weights_int8(W, group: int, w_int8=None, row_scale=None):
-    """fp32 W [N, K] -> rotated int8 codes [N, K] and fp32 row scales [N] (W8A8)."""
+def _scale_dtype(t, name):
+    """fp32 scales, or fp16 ones (the pages' stored format): the entry-point
+    suffix for that dtype."""
+    if t.dtype == torch.float32:
+        return ""
+    if t.dtype == torch.float16:
+        return "_f16"
+    raise TypeError(f"{name}: float32 or float16 scales, got {t.dtype}")
+
+
+def tint4_quantize_weights_int8(W, group: int, w_int8=None, row_scale=None,
+                                scale_dtype=torch.float32):
+    """fp32 W [N, K] -> rotated int8 codes [N, K] and row scales [N] (W8A8);
+    scale_dtype torch.float16 stores the scales in the pages' fp16 format."""
     _need(W, "W", torch.float32)
     N, K = W.shape
     if w_int8 is None:
         w_int8 = torch.empty((N, K), dtype=torch.int8, device=W.device)
     if row_scale is None:
-        row_scale = torch.empty((N,), dtype=torch.float32, device=W.device)
+        row_scale = torch.empty((N,), dtype=scale_dtype, device=W.device)
     _need(w_int8, "w_int8", torch.int8, (N, K))
-    _need(row_scale, "row_scale", torch.float32, (N,))
-    _native.call("tint4_quantize_weights_int8", _ptr(W), N, K, group, _ptr(w_int8),
-                 _ptr(row_scale), _stream(W.device))
+    _need(row_scale, "row_scale", row_scale.dtype, (N,))
+    _native.call("tint4_quantize_weights_int8" + _scale_dtype(row_scale, "row_scale"), _ptr(W), N,
+                 K, group, _ptr(w_int8), _ptr(row_scale), _stream(W.device))
     return w_int8, row_scale
 
 
@@ -216,14 +228,14 @@ def w8a8_gemm(a, tok_scale, w_int8, row_scale, bias=None, y=None) -> torch.Tenso
     N = w_int8.shape[0]
     _need(tok_scale, "tok_scale", torch.float32, (M,))
     _need(w_int8, "w_int8", torch.int8, (N, K))
-    _need(row_scale, "row_scale", torch.float32, (N,))
+    _need(row_scale, "row_scale", row_scale.dtype, (N,))
     if bias is not None:
         _need(bias, "bias", torch.bfloat16, (N,))
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
     _need(y, "y", torch.bfloat16, (M, N))
-    _native.call("w8a8_gemm", _ptr(a), _ptr(tok_scale), _ptr(w_int8), _ptr(row_scale),
-                 _ptr(bias), _ptr(y), M, N, K, _stream(a.device))
+    _native.call("w8a8_gemm" + _scale_dtype(row_scale, "row_scale"), _ptr(a), _ptr(tok_scale),
+                 _ptr(w_int8), _ptr(row_scale), _ptr(bias), _ptr(y), M, N, K, _stream(a.device))
     return y
 
 
@@ -233,7 +245,7 @@ def convrot_w8a8_linear(x, w_int8, row_scale, group, bias=None, y=None, workspac
     M, K = x.shape
     N = w_int8.shape[0]
     _need(w_int8, "w_int8", torch.int8, (N, K))
-    _need(row_scale, "row_scale", torch.float32, (N,))
+    _need(row_scale, "row_scale", row_scale.dtype, (N,))
     if bias is not None:
         _need(bias, "bias", torch.bfloat16, (N,))
     if y is None:
@@ -242,8 +254,9 @@ def convrot_w8a8_linear(x, w_int8, row_scale, group, bias=None, y=None, workspac
     need = convrot_linear_workspace_size(M, K, 8)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
-    _native.call("convrot_w8a8_linear", _ptr(x), _ptr(w_int8), _ptr(row_scale), _ptr(bias),
-                 _ptr(y), M, N, K, group, _ptr(workspace), workspace.numel(), _stream(x.device))
+    _native.call("convrot_w8a8_linear" + _scale_dtype(row_scale, "row_scale"), _ptr(x),
+                 _ptr(w_int8), _ptr(row_scale), _ptr(bias), _ptr(y), M, N, K, group,
+                 _ptr(workspace), workspace.numel(), _stream(x.device))
     return y
 
 
@@ -330,25 +343,28 @@ WEIGHT_GROUP = 128   # K values per group-wise weight scale (TINT4_WEIGHT_GROUP)
 
 
 def tint4_pack_weights_groupwise(W: torch.Tensor, group: int, asym: bool = False,
-                                 w_packed=None, w_scale=None, w_zero=None):
-    """fp32 W [N, K] -> (packed uint8 [N, K/2], scale fp32 [N, K/128],
-    zero uint8 [N, K/128] or None): rotated, then int4 per 128-wide K group
-    (symmetric, or asymmetric with zero points)."""
+                                 w_packed=None, w_scale=None, w_zero=None,
+                                 scale_dtype=torch.float32):
+    """fp32 W [N, K] -> (packed uint8 [N, K/2], scale [N, K/128], zero uint8
+    [N, K/128] or None): rotated, then int4 per 128-wide K group (symmetric,
+    or asymmetric with zero points).  scale_dtype torch.float16 stores the
+    scales in the pages' fp16 format (codes taken against the fp16 scale)."""
     _need(W, "W", torch.float32)
     N, K = W.shape
     ng = K // WEIGHT_GROUP
     if w_packed is None:
         w_packed = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
     if w_scale is None:
-        w_scale = torch.empty((N, ng), dtype=torch.float32, device=W.device)
+        w_scale = torch.empty((N, ng), dtype=scale_dtype, device=W.device)
     if asym and w_zero is None:
         w_zero = torch.empty((N, ng), dtype=torch.uint8, device=W.device)
     _need(w_packed, "w_packed", torch.uint8, (N, K // 2))
-    _need(w_scale, "w_scale", torch.float32, (N, ng))
+    _need(w_scale, "w_scale", w_scale.dtype, (N, ng))
     if asym:
         _need(w_zero, "w_zero", torch.uint8, (N, ng))
-    _native.call("tint4_pack_weights_groupwise", _ptr(W), N, K, group, int(bool(asym)),
-                 _ptr(w_packed), _ptr(w_scale), _ptr(w_zero if asym else None), _stream(W.device))
+    _native.call("tint4_pack_weights_groupwise" + _scale_dtype(w_scale, "w_scale"), _ptr(W), N, K,
+                 group, int(bool(asym)), _ptr(w_packed), _ptr(w_scale),
+                 _ptr(w_zero if asym else None), _stream(W.device))
     return w_packed, w_scale, (w_zero if asym else None)
 
 
@@ -356,7 +372,8 @@ def _gw_operands(M, K, w_packed, w_scale, w_zero, bias, y, device):
     N = w_packed.shape[0]
     ng = K // WEIGHT_GROUP
     _need(w_packed, "w_packed", torch.uint8, (N, K // 2))
-    _need(w_scale, "w_scale", torch.float32, (N, ng))
+    _need(w_scale, "w_scale", w_scale.dtype, (N, ng))
+    _scale_dtype(w_scale, "w_scale")
     if w_zero is not None:
         _need(w_zero, "w_zero", torch.uint8, (N, ng))
     if bias is not None:
@@ -374,8 +391,9 @@ def w4a8_gemm_groupwise(a, tok_scale, w_packed, w_scale, w_zero=None, bias=None,
     M, K = a.shape
     _need(tok_scale, "tok_scale", torch.float32, (M,))
     N, y = _gw_operands(M, K, w_packed, w_scale, w_zero, bias, y, a.device)
-    _native.call("w4a8_gemm_groupwise", _ptr(a), _ptr(tok_scale), _ptr(w_packed), _ptr(w_scale),
-                 _ptr(w_zero), _ptr(bias), _ptr(y), M, N, K, _stream(a.device))
+    _native.call("w4a8_gemm_groupwise" + _scale_dtype(w_scale, "w_scale"), _ptr(a),
+                 _ptr(tok_scale), _ptr(w_packed), _ptr(w_scale), _ptr(w_zero), _ptr(bias), _ptr(y),
+                 M, N, K, _stream(a.device))
     return y
 
 
@@ -388,9 +406,9 @@ def convrot_w4a8_linear_groupwise(x, w_packed, w_scale, group, w_zero=None, bias
     need = convrot_linear_workspace_size(M, K, 8)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
-    _native.call("convrot_w4a8_linear_groupwise", _ptr(x), _ptr(w_packed), _ptr(w_scale),
-                 _ptr(w_zero), _ptr(bias), _ptr(y), M, N, K, group, _ptr(workspace),
-                 workspace.numel(), _stream(x.device))
+    _native.call("convrot_w4a8_linear_groupwise" + _scale_dtype(w_scale, "w_scale"), _ptr(x),
+                 _ptr(w_packed), _ptr(w_scale), _ptr(w_zero), _ptr(bias), _ptr(y), M, N, K, group,
+                 _ptr(workspace), workspace.numel(), _stream(x.device))
     return y
 
 
@@ -489,8 +507,10 @@ class GroupwiseQuantizedLinear:
         self._workspace = None
 
     @classmethod
-    def from_float(cls, W: torch.Tensor, group: int, asym: bool = False, bias=None):
-        wp, s, z = tint4_pack_weights_groupwise(W.float().contiguous(), group, asym)
+    def from_float(cls, W: torch.Tensor, group: int, asym: bool = False, bias=None,
+                   scale_dtype=torch.float32):
+        wp, s, z = tint4_pack_weights_groupwise(W.float().contiguous(), group, asym,
+                                                scale_dtype=scale_dtype)
         return cls(wp, s, z, group, bias)
 
     @property

@@ -57,6 +57,12 @@ SIGNATURES = {
     "tint4_pack_weights_groupwise": (I, [P, I, I, I, I, P, P, P, P]),
     "w4a8_gemm_groupwise": (I, [P, P, P, P, P, P, P, I, I, I, P]),
     "convrot_w4a8_linear_groupwise": (I, [P, P, P, P, P, P, I, I, I, I, P, SZ, P]),
+    "tint4_pack_weights_groupwise_f16": (I, [P, I, I, I, I, P, P, P, P]),
+    "w4a8_gemm_groupwise_f16": (I, [P, P, P, P, P, P, P, I, I, I, P]),
+    "convrot_w4a8_linear_groupwise_f16": (I, [P, P, P, P, P, P, I, I, I, I, P, SZ, P]),
+    "tint4_quantize_weights_int8_f16": (I, [P, I, I, I, P, P, P]),
+    "w8a8_gemm_f16": (I, [P, P, P, P, P, P, I, I, I, P]),
+    "convrot_w8a8_linear_f16": (I, [P, P, P, P, P, I, I, I, I, P, SZ, P]),
     "tint4_debug_int32_gemm": (I, [P, I, P, P, I, I, I, P]),
     "tint4_debug_w4a8_gemm_even_odd": (I, [P, P, P, P, P, P, I, I, I, P]),
     "tint4_debug_bounded_wait": (I, [U64, P]),

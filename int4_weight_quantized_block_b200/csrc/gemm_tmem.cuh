@@ -175,7 +175,9 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 // int8 tile (128-byte swizzle) and the MMA reads it from shared memory as its
 // A operand (kind::i8, both operands in shared memory); no unpack, no x16.
 // EVOD: the int8 activation codes are stored in the even/odd K order.
-template <bool OUT_I32, bool A_INT4, bool W8 = false, bool EVOD = false>
+// S16: the row scales are IEEE fp16 (the stored format of "ComfyUI-INT-
+// Crush", "Weight Format"), widened exactly in the epilogue.
+template <bool OUT_I32, bool A_INT4, bool W8 = false, bool EVOD = false, bool S16 = false>
 __global__ void __launch_bounds__(kTmThreads, 1)
 w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                       const __grid_constant__ TmGroups grp,
@@ -448,7 +450,7 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             // scaling by a power of two commutes with the rounding (256 for A_INT4)
             constexpr float kUnscale = A_INT4 ? 1.0f / 256.0f : (W8 ? 1.0f : 0.0625f);
             constexpr int kShift = A_INT4 ? 8 : (W8 ? 0 : 4);
-            const float sr16 = (row_ok && !OUT_I32) ? __ldg(row_scale + n) * kUnscale : 0.0f;
+            const float sr16 = (row_ok && !OUT_I32) ? ld_scale<S16>(row_scale, n) * kUnscale : 0.0f;
             const float b = (row_ok && !OUT_I32 && bias != nullptr) ? __bfloat162float(bias[n]) : 0.0f;
 #pragma unroll 1
             for (int c0 = half * (kTmBN / 2); c0 < (half + 1) * (kTmBN / 2); c0 += 32) {

@@ -79,12 +79,14 @@ __device__ __forceinline__ void unpack8_asym_evod(uint32_t w, uint32_t zc, uint3
 // EVOD: the int8 activation codes are stored in the even/odd K order
 // (0, 2, 4, 6, 1, 3, 5, 7 in every block of 8), the order the unpack
 // produces without byte permutes.
-template <bool ASYM, bool EVOD>
+// S16: the group scales are IEEE fp16 ("ComfyUI-INT-Crush", "Weight
+// Format": the stored format), widened exactly where they are read.
+template <bool ASYM, bool EVOD, bool S16 = false>
 __global__ void __launch_bounds__(kGwThreads, 1)
 w4a8_gw_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                          const __grid_constant__ CUtensorMap tmap_w,
                          const __grid_constant__ CUtensorMap tmap_y,
-                         const float* __restrict__ tok_scale, const float* __restrict__ wscale,
+                         const float* __restrict__ tok_scale, const void* __restrict__ wscale,
                          const uint8_t* __restrict__ wzero,
                          const __nv_bfloat16* __restrict__ bias, int M, int N, int K,
                          uint64_t wait_ns) {
@@ -278,11 +280,11 @@ w4a8_gw_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             const int m0 = (tile % m_tiles) * kGwBN, n0 = (tile / m_tiles) * kGwBM;
             const int n = n0 + r;
             const bool row_ok = n < N;
-            const float* srow = wscale + static_cast<size_t>(row_ok ? n : 0) * ng;
-            float sg_next = row_ok ? __ldg(srow) * kUnscale : 0.0f;
+            const size_t srow = static_cast<size_t>(row_ok ? n : 0) * ng;
+            float sg_next = row_ok ? ld_scale<S16>(wscale, srow) * kUnscale : 0.0f;
             for (int kt = 0; kt < KT; ++kt, ++j) {
                 const float sg = sg_next;
-                if (kt + 1 < KT) sg_next = row_ok ? __ldg(srow + kt + 1) * kUnscale : 0.0f;
+                if (kt + 1 < KT) sg_next = row_ok ? ld_scale<S16>(wscale, srow + kt + 1) * kUnscale : 0.0f;
                 if (ok && !warp_wait(&empty[j % kS], (j / kS) & 1, abort_flag, wait_ns,
                                      kDevErrTimeoutEpilogue))
                     ok = false;

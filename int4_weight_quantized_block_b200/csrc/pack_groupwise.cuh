@@ -26,10 +26,13 @@ namespace tint4 {
 
 constexpr int kWeightGroup = 128;   // K values per weight group (one GEMM K step)
 
-template <int G>
+// S16: the scales are stored as IEEE fp16 ("Weight Format": the pages'
+// stored format): each is rounded to the nearest fp16 (ties to even) and the
+// zero point and codes are taken against that stored value.
+template <int G, bool S16 = false>
 __global__ void __launch_bounds__(256)
 pack_weights_groupwise_kernel(const float* __restrict__ W, int N, int K, int asym,
-                              uint8_t* __restrict__ packed, float* __restrict__ scale,
+                              uint8_t* __restrict__ packed, void* __restrict__ scale,
                               uint8_t* __restrict__ zero) {
     static_assert(kWeightGroup == 16 * 8, "a weight group is 16 lanes of 8 values");
     const int lane = threadIdx.x & 31;
@@ -61,7 +64,9 @@ pack_weights_groupwise_kernel(const float* __restrict__ W, int N, int K, int asy
             hi = fmaxf(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, d));
         }
         // lo <= 0 <= hi, so the absolute maximum is max(-lo, hi)
-        const float s = asym ? __fdiv_rn(__fsub_rn(hi, lo), 15.0f) : __fdiv_rn(fmaxf(-lo, hi), 7.0f);
+        const float s32 = asym ? __fdiv_rn(__fsub_rn(hi, lo), 15.0f) : __fdiv_rn(fmaxf(-lo, hi), 7.0f);
+        const __half s16 = __float2half_rn(s32);
+        const float s = S16 ? __half2float(s16) : s32;
         int z = 0;
         if (asym && s > 0.0f) z = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.0f), 15.0f));
         uint32_t word = 0u;
@@ -78,7 +83,8 @@ pack_weights_groupwise_kernel(const float* __restrict__ W, int N, int K, int asy
         *reinterpret_cast<uint32_t*>(packed + static_cast<size_t>(n) * (K / 2) + base / 2) = word;
         if ((lane & 15) == 0) {
             const size_t gi = static_cast<size_t>(n) * ng + base / kWeightGroup;
-            scale[gi] = s;
+            if (S16) static_cast<__half*>(scale)[gi] = s16;
+            else static_cast<float*>(scale)[gi] = s;
             if (asym) zero[gi] = static_cast<uint8_t>(z);
         }
     }

@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace tint4 {
 
@@ -88,6 +89,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
             return false;
         }
     }
+}
+
+// Weight scale i of an array of fp32 scales, or (S16) of IEEE fp16 scales
+// widened to fp32 (exact).
+template <bool S16>
+__device__ __forceinline__ float ld_scale(const void* p, size_t i) {
+    if constexpr (S16) return __half2float(__ldg(reinterpret_cast<const __half*>(p) + i));
+    else return __ldg(reinterpret_cast<const float*>(p) + i);
 }
 
 // [lo, hi) of part i when n items are split into p contiguous parts of

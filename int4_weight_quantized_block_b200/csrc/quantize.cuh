@@ -455,9 +455,12 @@ __device__ __forceinline__ void rq_codes_div(const uint64_t (&p)[RqPairs<CPL>::N
 // (one code per byte only): each block of 8 codes stored with its even
 // positions first (0, 2, 4, 6, 1, 3, 5, 7), the order the tensor-core GEMM
 // widens its weights in.
-template <typename InT, int G, int Q, bool PACKED, bool EVOD, int CPL>
+// S16: the scales are stored as IEEE fp16 (the int8 weights of the W8A8
+// path in the pages' stored format, "Weight Format"): each is rounded to the
+// nearest fp16 and the codes are taken against that stored scale.
+template <typename InT, int G, int Q, bool PACKED, bool EVOD, int CPL, bool S16 = false>
 __device__ __forceinline__ void rq_team_rows(const InT* __restrict__ in, int rows, int K,
-                                             void* __restrict__ codes, float* __restrict__ scales,
+                                             void* __restrict__ codes, void* __restrict__ scales,
                                              float (&red)[2][kQuantMaxWarps]) {
     static_assert(!(PACKED && EVOD), "even/odd order is for one code per byte");
     using Lt = RqLayout<G, CPL>;
@@ -513,18 +516,37 @@ __device__ __forceinline__ void rq_team_rows(const InT* __restrict__ in, int row
         for (int w = 1; w < nwarps; ++w) amax = fmaxf(amax, rb[w]);
 
         uint2 cw[CPL];
-        float scale;
-        if (amax >= 0x1p-100f) {
-            const float su = __fdiv_rn(amax, static_cast<float>(Q));
-            scale = su * kNorm;
-            const bool near = rq_codes_fast<Q, CPL, EVOD>(p, __frcp_rn(su), cw);
-            if (__any_sync(0xFFFFFFFFu, near)) rq_codes_div<Q, CPL, EVOD>(p, 1.0f, su, cw);
+        if constexpr (!S16) {
+            float scale;
+            if (amax >= 0x1p-100f) {
+                const float su = __fdiv_rn(amax, static_cast<float>(Q));
+                scale = su * kNorm;
+                const bool near = rq_codes_fast<Q, CPL, EVOD>(p, __frcp_rn(su), cw);
+                if (__any_sync(0xFFFFFFFFu, near)) rq_codes_div<Q, CPL, EVOD>(p, 1.0f, su, cw);
+            } else {
+                // tiny or zero row: normalise first, as the oracle does
+                scale = __fdiv_rn(amax * kNorm, static_cast<float>(Q));
+                rq_codes_div<Q, CPL, EVOD>(p, kNorm, scale, cw);
+            }
+            if (L == 0) static_cast<float*>(scales)[row] = scale;
         } else {
-            // tiny or zero row: normalise first, as the oracle does
-            scale = __fdiv_rn(amax * kNorm, static_cast<float>(Q));
-            rq_codes_div<Q, CPL, EVOD>(p, kNorm, scale, cw);
+            // the fp32 scale as above, rounded to fp16; the codes against it
+            const float s32 = amax >= 0x1p-100f ? __fdiv_rn(amax, static_cast<float>(Q)) * kNorm
+                                                : __fdiv_rn(amax * kNorm, static_cast<float>(Q));
+            const __half h = __float2half_rn(s32);
+            const float sf = __half2float(h);
+            if (L == 0) static_cast<__half*>(scales)[row] = h;
+            if (sf >= 0x1p-14f && sf <= 65504.0f) {
+                // a normal fp16 scale: the fast path on the unnormalised values
+                // (|u / su| <= Q (1 + 2^-11) < Q + 1/2: still no clamp)
+                const float su = sf / kNorm;
+                const bool near = rq_codes_fast<Q, CPL, EVOD>(p, __frcp_rn(su), cw);
+                if (__any_sync(0xFFFFFFFFu, near)) rq_codes_div<Q, CPL, EVOD>(p, 1.0f, su, cw);
+            } else {
+                // subnormal, zero or infinite: value by value, clamped
+                rq_codes_div<Q, CPL, EVOD>(p, kNorm, sf, cw);
+            }
         }
-        if (L == 0) scales[row] = scale;
 
 #pragma unroll
         for (int i = 0; i < CPL; ++i) {
@@ -549,13 +571,13 @@ __device__ __forceinline__ void rq_team_rows(const InT* __restrict__ in, int row
 // tint4_quantize_weights_int8, the fused linears).  Under programmatic
 // dependent launch the consumer grid may start its prologue while this grid
 // runs; it waits for this grid's completion before reading the codes.
-template <typename InT, int G, int Q, bool PACKED, bool EVOD, int CPL>
+template <typename InT, int G, int Q, bool PACKED, bool EVOD, int CPL, bool S16 = false>
 __global__ void __launch_bounds__(512)
 rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K, void* __restrict__ codes,
-                            float* __restrict__ scales) {
+                            void* __restrict__ scales) {
     __shared__ float red[2][kQuantMaxWarps];
     grid_launch_dependents();
-    rq_team_rows<InT, G, Q, PACKED, EVOD, CPL>(in, rows, K, codes, scales, red);
+    rq_team_rows<InT, G, Q, PACKED, EVOD, CPL, S16>(in, rows, K, codes, scales, red);
 }
 
 }  // namespace tint4

@@ -149,10 +149,10 @@ RqShape rq_shape(int K) {
 
 // persistent grid: as many CTAs as fit on the GPU at once (per block size,
 // looked up once per device), at most one per row
-template <typename InT, int G, int Q, bool PACKED, bool EVOD, int CPL>
-void launch_rq_persistent(const InT* in, int rows, int K, void* codes, float* scales, int threads,
+template <typename InT, int G, int Q, bool PACKED, bool EVOD, int CPL, bool S16 = false>
+void launch_rq_persistent(const InT* in, int rows, int K, void* codes, void* scales, int threads,
                           cudaStream_t st) {
-    auto kern = rotate_quantize_rows_kernel<InT, G, Q, PACKED, EVOD, CPL>;
+    auto kern = rotate_quantize_rows_kernel<InT, G, Q, PACKED, EVOD, CPL, S16>;
     int dev = 0;
     cudaGetDevice(&dev);
     static std::atomic<int> per_sm[kMaxDevices][kQuantMaxWarps + 1];
@@ -170,26 +170,26 @@ void launch_rq_persistent(const InT* in, int rows, int K, void* codes, float* sc
     kern<<<grid, threads, 0, st>>>(in, rows, K, codes, scales);
 }
 
-template <typename InT, int G, int Q, bool PACKED, bool EVOD = false>
-void launch_rq_ch(const InT* in, int rows, int K, void* codes, float* scales, cudaStream_t st) {
+template <typename InT, int G, int Q, bool PACKED, bool EVOD = false, bool S16 = false>
+void launch_rq_ch(const InT* in, int rows, int K, void* codes, void* scales, cudaStream_t st) {
     const RqShape sh = rq_shape(K);
     const int threads = sh.warps * 32;
     if (sh.cpl == 1)
-        launch_rq_persistent<InT, G, Q, PACKED, EVOD, 1>(in, rows, K, codes, scales, threads, st);
+        launch_rq_persistent<InT, G, Q, PACKED, EVOD, 1, S16>(in, rows, K, codes, scales, threads, st);
     else if (sh.cpl == 2)
-        launch_rq_persistent<InT, G, Q, PACKED, EVOD, 2>(in, rows, K, codes, scales, threads, st);
+        launch_rq_persistent<InT, G, Q, PACKED, EVOD, 2, S16>(in, rows, K, codes, scales, threads, st);
     else
-        launch_rq_persistent<InT, G, Q, PACKED, EVOD, 4>(in, rows, K, codes, scales, threads, st);
+        launch_rq_persistent<InT, G, Q, PACKED, EVOD, 4, S16>(in, rows, K, codes, scales, threads, st);
 }
 
-template <typename InT, int Q, bool PACKED, bool EVOD = false>
-void launch_rq_g(const InT* in, int rows, int K, int g, void* codes, float* scales,
+template <typename InT, int Q, bool PACKED, bool EVOD = false, bool S16 = false>
+void launch_rq_g(const InT* in, int rows, int K, int g, void* codes, void* scales,
                  cudaStream_t st) {
     switch (g) {
-        case 0: launch_rq_ch<InT, 0, Q, PACKED, EVOD>(in, rows, K, codes, scales, st); break;
-        case 16: launch_rq_ch<InT, 16, Q, PACKED, EVOD>(in, rows, K, codes, scales, st); break;
-        case 64: launch_rq_ch<InT, 64, Q, PACKED, EVOD>(in, rows, K, codes, scales, st); break;
-        default: launch_rq_ch<InT, 256, Q, PACKED, EVOD>(in, rows, K, codes, scales, st); break;
+        case 0: launch_rq_ch<InT, 0, Q, PACKED, EVOD, S16>(in, rows, K, codes, scales, st); break;
+        case 16: launch_rq_ch<InT, 16, Q, PACKED, EVOD, S16>(in, rows, K, codes, scales, st); break;
+        case 64: launch_rq_ch<InT, 64, Q, PACKED, EVOD, S16>(in, rows, K, codes, scales, st); break;
+        default: launch_rq_ch<InT, 256, Q, PACKED, EVOD, S16>(in, rows, K, codes, scales, st); break;
     }
 }
 
@@ -227,11 +227,11 @@ cudaLaunchAttribute pdl_attr() {
 // packed int4 widened in shared memory (A_INT4).  `grp` holds 1 to
 // kTmMaxGroups weight matrices sharing the activation codes (the tensor maps
 // and the tile list are filled in here).
-template <bool OUT_I32, bool A_INT4, bool W8 = false, bool EVOD = false>
+template <bool OUT_I32, bool A_INT4, bool W8 = false, bool EVOD = false, bool S16 = false>
 tint4_status launch_gemm_tmem(const void* a, const float* st, TmGroups& grp,
                               const uint8_t* const* w, int M, int K, cudaStream_t stream,
                               bool pdl) {
-    auto kern = w4a8_tmem_gemm_kernel<OUT_I32, A_INT4, W8, EVOD>;
+    auto kern = w4a8_tmem_gemm_kernel<OUT_I32, A_INT4, W8, EVOD, S16>;
     constexpr int smem_bytes = A_INT4 ? kTmSmemBytesA4 : (W8 ? kTmSmemBytesW8 : kTmSmemBytes);
     CUtensorMap ta;
     bool ok = A_INT4 ? make_map_u8(&ta, a, K / 2, M, K / 2, kTmBK / 2, kTmBN, CU_TENSOR_MAP_SWIZZLE_NONE)
@@ -703,18 +703,20 @@ tint4_status launch_gemm_grouped(const int8_t* codes, const float* tok_scale,
     return launch_gemm_tmem<false, false, false, EVOD>(codes, tok_scale, grp, w, M, K, st, pdl);
 }
 
-// W8A8: int8 codes x int8 weights, one tensor-core launch at every M.
-tint4_status launch_w8a8(const int8_t* codes, const float* st, const int8_t* w, const float* sr,
+// W8A8: int8 codes x int8 weights, one tensor-core launch at every M; S16:
+// fp16 row scales.
+template <bool S16 = false>
+tint4_status launch_w8a8(const int8_t* codes, const float* st, const int8_t* w, const void* sr,
                          const __nv_bfloat16* bias, __nv_bfloat16* y, int M, int N, int K,
                          cudaStream_t stream, bool pdl) {
     TmGroups grp{};
-    grp.row_scale[0] = sr;
+    grp.row_scale[0] = static_cast<const float*>(sr);   // fp16 bits when S16
     grp.bias[0] = bias;
     grp.out[0] = y;
     grp.N[0] = N;
     grp.count = 1;
     const uint8_t* wp = reinterpret_cast<const uint8_t*>(w);
-    return launch_gemm_tmem<false, false, true>(codes, st, grp, &wp, M, K, stream, pdl);
+    return launch_gemm_tmem<false, false, true, false, S16>(codes, st, grp, &wp, M, K, stream, pdl);
 }
 
 // ------------------------------------------------------------------ group-wise W4A8
@@ -730,23 +732,23 @@ tint4_status check_gw_mnk(int M, int N, int K) {
     return TINT4_OK;
 }
 
-template <int G>
-void launch_pack_gw(const float* W, int N, int K, int asym, uint8_t* packed, float* scale,
+template <int G, bool S16 = false>
+void launch_pack_gw(const float* W, int N, int K, int asym, uint8_t* packed, void* scale,
                     uint8_t* zero, cudaStream_t st) {
     const long warps = static_cast<long>(N) * ((K + kQuantChunk - 1) / kQuantChunk);
     int dev = 0;
     cudaGetDevice(&dev);
     const long grid = std::min<long>((warps + 7) / 8, 8L * num_sms(dev));
-    pack_weights_groupwise_kernel<G><<<static_cast<int>(grid), 256, 0, st>>>(W, N, K, asym, packed,
-                                                                            scale, zero);
+    pack_weights_groupwise_kernel<G, S16><<<static_cast<int>(grid), 256, 0, st>>>(W, N, K, asym,
+                                                                                 packed, scale, zero);
 }
 
 // The tensor-core GEMM with group-wise scales at every M (gemm_tmem_gw.cuh).
-template <bool ASYM, bool EVOD>
+template <bool ASYM, bool EVOD, bool S16 = false>
 tint4_status launch_gemm_gw(const int8_t* codes, const float* tok_scale, const uint8_t* w,
-                            const float* wscale, const uint8_t* wzero, const __nv_bfloat16* bias,
+                            const void* wscale, const uint8_t* wzero, const __nv_bfloat16* bias,
                             __nv_bfloat16* y, int M, int N, int K, cudaStream_t stream, bool pdl) {
-    auto kern = w4a8_gw_tmem_gemm_kernel<ASYM, EVOD>;
+    auto kern = w4a8_gw_tmem_gemm_kernel<ASYM, EVOD, S16>;
     CUtensorMap ta, tw, ty;
     bool ok = make_map_u8(&ta, codes, K, M, K, kGwBK, kGwBN, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && make_map_u8(&tw, w, K / 2, N, K / 2, kGwBK / 2, kGwBM, CU_TENSOR_MAP_SWIZZLE_64B);
@@ -789,12 +791,12 @@ tint4_status launch_gemm_gw(const int8_t* codes, const float* tok_scale, const u
 // symmetric / 2 asymmetric); else the tensor-core kernel.
 bool gw_streaming(int M, int K) { return M <= kS8MaxM && K <= 128 * kS8GwMaxGroups; }
 
-template <int NB, int GW>
+template <int NB, int GW, bool S16 = false>
 tint4_status launch_gemm_small_gw(const int8_t* a, const uint8_t* w, const float* st,
-                                  const float* wscale, const uint8_t* wzero,
+                                  const void* wscale, const uint8_t* wzero,
                                   const __nv_bfloat16* bias, __nv_bfloat16* y, int M, int N, int K,
                                   cudaStream_t stream, bool pdl) {
-    auto kern = w4a8_small_kernel<NB, false, false, 0, 0, GW>;
+    auto kern = w4a8_small_kernel<NB, false, false, 0, 0, GW, S16>;
     constexpr int smem = S8Cfg<NB>::FUSE_OFF + kS8GwBytes + 1024;
     static_assert(smem <= 227 * 1024, "shared memory budget");
     CUtensorMap tw;
@@ -823,8 +825,9 @@ tint4_status launch_gemm_small_gw(const int8_t* a, const uint8_t* w, const float
     cudaLaunchAttribute attr[1] = {pdl_attr()};
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, tw, reinterpret_cast<const uint8_t*>(a), st, wscale, bias,
-                           static_cast<void*>(y), M, N, K, 0xF0F0F0F0u,
+    if (cudaLaunchKernelEx(&cfg, kern, tw, reinterpret_cast<const uint8_t*>(a), st,
+                           static_cast<const float*>(wscale), bias, static_cast<void*>(y), M, N, K,
+                           0xF0F0F0F0u,
                            g_decode_prefetch.load(std::memory_order_relaxed),
                            g_wait_limit_ns.load(std::memory_order_relaxed), wzero) != cudaSuccess) {
         cudaGetLastError();
@@ -833,28 +836,167 @@ tint4_status launch_gemm_small_gw(const int8_t* a, const uint8_t* w, const float
     return last_launch_status();
 }
 
-template <bool EVOD>
+template <bool EVOD, bool S16 = false>
 tint4_status launch_gemm_gw_any(const int8_t* codes, const float* tok_scale, const uint8_t* w,
-                                const float* wscale, const uint8_t* wzero, const tint4_bf16* bias,
+                                const void* wscale, const uint8_t* wzero, const tint4_bf16* bias,
                                 tint4_bf16* y, int M, int N, int K, cudaStream_t st, bool pdl) {
     const auto* b = reinterpret_cast<const __nv_bfloat16*>(bias);
     auto* yb = reinterpret_cast<__nv_bfloat16*>(y);
     if (gw_streaming(M, K)) {
         if (EVOD) return TINT4_ERR_INVALID_ARG;   // the streaming kernel reads natural-order codes
         if (M <= 8)
-            return wzero ? launch_gemm_small_gw<1, 2>(codes, w, tok_scale, wscale, wzero, b, yb, M,
-                                                      N, K, st, pdl)
-                         : launch_gemm_small_gw<1, 1>(codes, w, tok_scale, wscale, nullptr, b, yb,
-                                                      M, N, K, st, pdl);
-        return wzero ? launch_gemm_small_gw<2, 2>(codes, w, tok_scale, wscale, wzero, b, yb, M, N,
-                                                  K, st, pdl)
-                     : launch_gemm_small_gw<2, 1>(codes, w, tok_scale, wscale, nullptr, b, yb, M,
-                                                  N, K, st, pdl);
+            return wzero ? launch_gemm_small_gw<1, 2, S16>(codes, w, tok_scale, wscale, wzero, b, yb,
+                                                           M, N, K, st, pdl)
+                         : launch_gemm_small_gw<1, 1, S16>(codes, w, tok_scale, wscale, nullptr, b,
+                                                           yb, M, N, K, st, pdl);
+        return wzero ? launch_gemm_small_gw<2, 2, S16>(codes, w, tok_scale, wscale, wzero, b, yb, M,
+                                                       N, K, st, pdl)
+                     : launch_gemm_small_gw<2, 1, S16>(codes, w, tok_scale, wscale, nullptr, b, yb,
+                                                       M, N, K, st, pdl);
     }
-    return wzero ? launch_gemm_gw<true, EVOD>(codes, tok_scale, w, wscale, wzero, b, yb, M, N, K,
-                                              st, pdl)
-                 : launch_gemm_gw<false, EVOD>(codes, tok_scale, w, wscale, nullptr, b, yb, M, N,
-                                               K, st, pdl);
+    return wzero ? launch_gemm_gw<true, EVOD, S16>(codes, tok_scale, w, wscale, wzero, b, yb, M, N,
+                                                   K, st, pdl)
+                 : launch_gemm_gw<false, EVOD, S16>(codes, tok_scale, w, wscale, nullptr, b, yb, M,
+                                                    N, K, st, pdl);
+}
+
+// ------------------------------------------------------------------ fp32 / fp16 weight scales
+//
+// The group-wise and W8A8 entry points with S16 = false take fp32 scales,
+// with S16 = true IEEE fp16 scales (the stored format of "ComfyUI-INT-Crush",
+// "Weight Format").
+
+template <bool S16>
+tint4_status pack_weights_groupwise_impl(const float* W, int N, int K, int group, int asym,
+                                         uint8_t* w_packed, void* w_scale, uint8_t* w_zero,
+                                         void* stream) {
+    if (asym != 0 && asym != 1) return TINT4_ERR_INVALID_ARG;
+    tint4_status s = check_rq_shape(N, K, group);
+    if (s != TINT4_OK) return s;
+    if (K % kWeightGroup != 0) return TINT4_ERR_UNSUPPORTED_SHAPE;
+    if (N > 0 && (!W || !w_packed || !w_scale || (asym && !w_zero))) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(w_packed) || !aligned16(w_scale) || !aligned16(w_zero))
+        return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (N == 0) return TINT4_OK;
+    cudaStream_t st = as_stream(stream);
+    switch (group) {
+        case 0: launch_pack_gw<0, S16>(W, N, K, asym, w_packed, w_scale, w_zero, st); break;
+        case 16: launch_pack_gw<16, S16>(W, N, K, asym, w_packed, w_scale, w_zero, st); break;
+        case 64: launch_pack_gw<64, S16>(W, N, K, asym, w_packed, w_scale, w_zero, st); break;
+        default: launch_pack_gw<256, S16>(W, N, K, asym, w_packed, w_scale, w_zero, st); break;
+    }
+    return last_launch_status();
+}
+
+template <bool S16>
+tint4_status gemm_groupwise_impl(const int8_t* a, const float* tok_scale, const uint8_t* w_packed,
+                                 const void* w_scale, const uint8_t* w_zero, const tint4_bf16* bias,
+                                 tint4_bf16* y, int M, int N, int K, void* stream) {
+    tint4_status s = check_gw_mnk(M, N, K);
+    if (s != TINT4_OK) return s;
+    if (M > 0 && (!a || !tok_scale || !w_packed || !w_scale || !y)) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(tok_scale) || !aligned16(w_packed) || !aligned16(w_scale) ||
+        !aligned16(w_zero) || !aligned16(bias) || !aligned16(y))
+        return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (M == 0) return TINT4_OK;
+    return launch_gemm_gw_any<false, S16>(a, tok_scale, w_packed, w_scale, w_zero, bias, y, M, N, K,
+                                          as_stream(stream), false);
+}
+
+template <bool S16>
+tint4_status linear_groupwise_impl(const tint4_bf16* x, const uint8_t* w_packed, const void* w_scale,
+                                   const uint8_t* w_zero, const tint4_bf16* bias, tint4_bf16* y,
+                                   int M, int N, int K, int group, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+    tint4_status s = check_gw_mnk(M, N, K);
+    if (s != TINT4_OK) return s;
+    if ((s = check_rq_shape(M, K, group)) != TINT4_OK) return s;
+    if (M > 0 && (!x || !w_packed || !w_scale || !y)) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_packed) || !aligned16(w_scale) || !aligned16(w_zero) ||
+        !aligned16(bias) || !aligned16(y))
+        return TINT4_ERR_MISALIGNED;
+    if (M > 0 && (!workspace || workspace_bytes < convrot_linear_workspace_size(M, K, 8)))
+        return TINT4_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (M == 0) return TINT4_OK;
+    int8_t* codes = static_cast<int8_t*>(workspace);
+    float* tok_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                                align_up(static_cast<size_t>(M) * K, 256));
+    cudaStream_t st = as_stream(stream);
+    // even/odd codes whenever the tensor-core kernel runs them
+    const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    if (gw_streaming(M, K))
+        launch_rq_g<__nv_bfloat16, 127, false>(xb, M, K, group, codes, tok_scale, st);
+    else
+        launch_rq_g<__nv_bfloat16, 127, false, true>(xb, M, K, group, codes, tok_scale, st);
+    if ((s = last_launch_status()) != TINT4_OK) return s;
+    return !gw_streaming(M, K)
+               ? launch_gemm_gw_any<true, S16>(codes, tok_scale, w_packed, w_scale, w_zero, bias, y,
+                                               M, N, K, st, true)
+               : launch_gemm_gw_any<false, S16>(codes, tok_scale, w_packed, w_scale, w_zero, bias,
+                                                y, M, N, K, st, true);
+}
+
+template <bool S16>
+tint4_status quantize_weights_int8_impl(const float* W, int N, int K, int group, int8_t* w_int8,
+                                        void* row_scale, void* stream) {
+    tint4_status s = check_rq_shape(N, K, group);
+    if (s != TINT4_OK) return s;
+    if (N > 0 && (!W || !w_int8 || !row_scale)) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(w_int8) || !aligned16(row_scale)) return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (N == 0) return TINT4_OK;
+    launch_rq_g<float, 127, false, false, S16>(W, N, K, group, w_int8, row_scale, as_stream(stream));
+    return last_launch_status();
+}
+
+template <bool S16>
+tint4_status w8a8_gemm_impl(const int8_t* codes, const float* tok_scale, const int8_t* w_int8,
+                            const void* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
+                            int N, int K, void* stream) {
+    tint4_status s = check_mnk(M, N, K);
+    if (s != TINT4_OK) return s;
+    if (M > 0 && (!codes || !tok_scale || !w_int8 || !row_scale || !y))
+        return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(codes) || !aligned16(tok_scale) || !aligned16(w_int8) ||
+        !aligned16(row_scale) || !aligned16(y) || !aligned16(bias))
+        return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (M == 0) return TINT4_OK;
+    return launch_w8a8<S16>(codes, tok_scale, w_int8, row_scale,
+                            reinterpret_cast<const __nv_bfloat16*>(bias),
+                            reinterpret_cast<__nv_bfloat16*>(y), M, N, K, as_stream(stream), false);
+}
+
+template <bool S16>
+tint4_status w8a8_linear_impl(const tint4_bf16* x, const int8_t* w_int8, const void* row_scale,
+                              const tint4_bf16* bias, tint4_bf16* y, int M, int N, int K, int group,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    tint4_status s = check_mnk(M, N, K);
+    if (s != TINT4_OK) return s;
+    if ((s = check_rq_shape(M, K, group)) != TINT4_OK) return s;
+    if (M > 0 && (!x || !w_int8 || !row_scale || !y)) return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_int8) || !aligned16(row_scale) || !aligned16(y) ||
+        !aligned16(bias))
+        return TINT4_ERR_MISALIGNED;
+    if (M > 0 && (!workspace || workspace_bytes < convrot_linear_workspace_size(M, K, 8)))
+        return TINT4_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TINT4_ERR_MISALIGNED;
+    if ((s = check_device()) != TINT4_OK) return s;
+    if (M == 0) return TINT4_OK;
+    int8_t* codes = static_cast<int8_t*>(workspace);
+    float* tok_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                                align_up(static_cast<size_t>(M) * K, 256));
+    cudaStream_t st = as_stream(stream);
+    launch_rq_g<__nv_bfloat16, 127, false>(reinterpret_cast<const __nv_bfloat16*>(x), M, K, group,
+                                           codes, tok_scale, st);
+    if ((s = last_launch_status()) != TINT4_OK) return s;
+    return launch_w8a8<S16>(codes, tok_scale, w_int8, row_scale,
+                            reinterpret_cast<const __nv_bfloat16*>(bias),
+                            reinterpret_cast<__nv_bfloat16*>(y), M, N, K, st, true);
 }
 
 }  // namespace
@@ -987,39 +1129,29 @@ tint4_status convrot_w4a8_linear_grouped(const tint4_bf16* x,
 tint4_status tint4_pack_weights_groupwise(const float* W, int N, int K, int group, int asym,
                                           uint8_t* w_packed, float* w_scale, uint8_t* w_zero,
                                           void* stream) {
-    if (asym != 0 && asym != 1) return TINT4_ERR_INVALID_ARG;
-    tint4_status s = check_rq_shape(N, K, group);
-    if (s != TINT4_OK) return s;
-    if (K % kWeightGroup != 0) return TINT4_ERR_UNSUPPORTED_SHAPE;
-    if (N > 0 && (!W || !w_packed || !w_scale || (asym && !w_zero))) return TINT4_ERR_INVALID_ARG;
-    if (!aligned16(W) || !aligned16(w_packed) || !aligned16(w_scale) || !aligned16(w_zero))
-        return TINT4_ERR_MISALIGNED;
-    if ((s = check_device()) != TINT4_OK) return s;
-    if (N == 0) return TINT4_OK;
-    cudaStream_t st = as_stream(stream);
-    switch (group) {
-        case 0: launch_pack_gw<0>(W, N, K, asym, w_packed, w_scale, w_zero, st); break;
-        case 16: launch_pack_gw<16>(W, N, K, asym, w_packed, w_scale, w_zero, st); break;
-        case 64: launch_pack_gw<64>(W, N, K, asym, w_packed, w_scale, w_zero, st); break;
-        default: launch_pack_gw<256>(W, N, K, asym, w_packed, w_scale, w_zero, st); break;
-    }
-    return last_launch_status();
+    return pack_weights_groupwise_impl<false>(W, N, K, group, asym, w_packed, w_scale, w_zero, stream);
+}
+
+tint4_status tint4_pack_weights_groupwise_f16(const float* W, int N, int K, int group, int asym,
+                                              uint8_t* w_packed, tint4_f16* w_scale,
+                                              uint8_t* w_zero, void* stream) {
+    return pack_weights_groupwise_impl<true>(W, N, K, group, asym, w_packed, w_scale, w_zero, stream);
 }
 
 tint4_status w4a8_gemm_groupwise(const int8_t* a, const float* tok_scale,
                                  const uint8_t* w_packed, const float* w_scale,
                                  const uint8_t* w_zero, const tint4_bf16* bias, tint4_bf16* y,
                                  int M, int N, int K, void* stream) {
-    tint4_status s = check_gw_mnk(M, N, K);
-    if (s != TINT4_OK) return s;
-    if (M > 0 && (!a || !tok_scale || !w_packed || !w_scale || !y)) return TINT4_ERR_INVALID_ARG;
-    if (!aligned16(a) || !aligned16(tok_scale) || !aligned16(w_packed) || !aligned16(w_scale) ||
-        !aligned16(w_zero) || !aligned16(bias) || !aligned16(y))
-        return TINT4_ERR_MISALIGNED;
-    if ((s = check_device()) != TINT4_OK) return s;
-    if (M == 0) return TINT4_OK;
-    return launch_gemm_gw_any<false>(a, tok_scale, w_packed, w_scale, w_zero, bias, y, M, N, K,
-                                     as_stream(stream), false);
+    return gemm_groupwise_impl<false>(a, tok_scale, w_packed, w_scale, w_zero, bias, y, M, N, K,
+                                      stream);
+}
+
+tint4_status w4a8_gemm_groupwise_f16(const int8_t* a, const float* tok_scale,
+                                     const uint8_t* w_packed, const tint4_f16* w_scale,
+                                     const uint8_t* w_zero, const tint4_bf16* bias, tint4_bf16* y,
+                                     int M, int N, int K, void* stream) {
+    return gemm_groupwise_impl<true>(a, tok_scale, w_packed, w_scale, w_zero, bias, y, M, N, K,
+                                     stream);
 }
 
 tint4_status convrot_w4a8_linear_groupwise(const tint4_bf16* x, const uint8_t* w_packed,
@@ -1027,91 +1159,55 @@ tint4_status convrot_w4a8_linear_groupwise(const tint4_bf16* x, const uint8_t* w
                                            const tint4_bf16* bias, tint4_bf16* y, int M, int N,
                                            int K, int group, void* workspace,
                                            size_t workspace_bytes, void* stream) {
-    tint4_status s = check_gw_mnk(M, N, K);
-    if (s != TINT4_OK) return s;
-    if ((s = check_rq_shape(M, K, group)) != TINT4_OK) return s;
-    if (M > 0 && (!x || !w_packed || !w_scale || !y)) return TINT4_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(w_packed) || !aligned16(w_scale) || !aligned16(w_zero) ||
-        !aligned16(bias) || !aligned16(y))
-        return TINT4_ERR_MISALIGNED;
-    if (M > 0 && (!workspace || workspace_bytes < convrot_linear_workspace_size(M, K, 8)))
-        return TINT4_ERR_WORKSPACE;
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TINT4_ERR_MISALIGNED;
-    if ((s = check_device()) != TINT4_OK) return s;
-    if (M == 0) return TINT4_OK;
-    int8_t* codes = static_cast<int8_t*>(workspace);
-    float* tok_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                                align_up(static_cast<size_t>(M) * K, 256));
-    cudaStream_t st = as_stream(stream);
-    // even/odd codes whenever the tensor-core kernel runs them
-    const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
-    if (gw_streaming(M, K))
-        launch_rq_g<__nv_bfloat16, 127, false>(xb, M, K, group, codes, tok_scale, st);
-    else
-        launch_rq_g<__nv_bfloat16, 127, false, true>(xb, M, K, group, codes, tok_scale, st);
-    if ((s = last_launch_status()) != TINT4_OK) return s;
-    return !gw_streaming(M, K)
-               ? launch_gemm_gw_any<true>(codes, tok_scale, w_packed, w_scale, w_zero, bias, y, M,
-                                          N, K, st, true)
-               : launch_gemm_gw_any<false>(codes, tok_scale, w_packed, w_scale, w_zero, bias, y, M,
-                                           N, K, st, true);
+    return linear_groupwise_impl<false>(x, w_packed, w_scale, w_zero, bias, y, M, N, K, group,
+                                        workspace, workspace_bytes, stream);
+}
+
+tint4_status convrot_w4a8_linear_groupwise_f16(const tint4_bf16* x, const uint8_t* w_packed,
+                                               const tint4_f16* w_scale, const uint8_t* w_zero,
+                                               const tint4_bf16* bias, tint4_bf16* y, int M, int N,
+                                               int K, int group, void* workspace,
+                                               size_t workspace_bytes, void* stream) {
+    return linear_groupwise_impl<true>(x, w_packed, w_scale, w_zero, bias, y, M, N, K, group,
+                                       workspace, workspace_bytes, stream);
 }
 
 tint4_status tint4_quantize_weights_int8(const float* W, int N, int K, int group,
                                          int8_t* w_int8, float* row_scale, void* stream) {
-    tint4_status s = check_rq_shape(N, K, group);
-    if (s != TINT4_OK) return s;
-    if (N > 0 && (!W || !w_int8 || !row_scale)) return TINT4_ERR_INVALID_ARG;
-    if (!aligned16(W) || !aligned16(w_int8) || !aligned16(row_scale)) return TINT4_ERR_MISALIGNED;
-    if ((s = check_device()) != TINT4_OK) return s;
-    if (N == 0) return TINT4_OK;
-    launch_rq_g<float, 127, false>(W, N, K, group, w_int8, row_scale, as_stream(stream));
-    return last_launch_status();
+    return quantize_weights_int8_impl<false>(W, N, K, group, w_int8, row_scale, stream);
+}
+
+tint4_status tint4_quantize_weights_int8_f16(const float* W, int N, int K, int group,
+                                             int8_t* w_int8, tint4_f16* row_scale, void* stream) {
+    return quantize_weights_int8_impl<true>(W, N, K, group, w_int8, row_scale, stream);
 }
 
 tint4_status w8a8_gemm(const int8_t* codes, const float* tok_scale, const int8_t* w_int8,
                        const float* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
                        int N, int K, void* stream) {
-    tint4_status s = check_mnk(M, N, K);
-    if (s != TINT4_OK) return s;
-    if (M > 0 && (!codes || !tok_scale || !w_int8 || !row_scale || !y))
-        return TINT4_ERR_INVALID_ARG;
-    if (!aligned16(codes) || !aligned16(tok_scale) || !aligned16(w_int8) ||
-        !aligned16(row_scale) || !aligned16(y) || !aligned16(bias))
-        return TINT4_ERR_MISALIGNED;
-    if ((s = check_device()) != TINT4_OK) return s;
-    if (M == 0) return TINT4_OK;
-    return launch_w8a8(codes, tok_scale, w_int8, row_scale,
-                       reinterpret_cast<const __nv_bfloat16*>(bias),
-                       reinterpret_cast<__nv_bfloat16*>(y), M, N, K, as_stream(stream), false);
+    return w8a8_gemm_impl<false>(codes, tok_scale, w_int8, row_scale, bias, y, M, N, K, stream);
+}
+
+tint4_status w8a8_gemm_f16(const int8_t* codes, const float* tok_scale, const int8_t* w_int8,
+                           const tint4_f16* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
+                           int N, int K, void* stream) {
+    return w8a8_gemm_impl<true>(codes, tok_scale, w_int8, row_scale, bias, y, M, N, K, stream);
 }
 
 tint4_status convrot_w8a8_linear(const tint4_bf16* x, const int8_t* w_int8,
                                  const float* row_scale, const tint4_bf16* bias, tint4_bf16* y,
                                  int M, int N, int K, int group, void* workspace,
                                  size_t workspace_bytes, void* stream) {
-    tint4_status s = check_mnk(M, N, K);
-    if (s != TINT4_OK) return s;
-    if ((s = check_rq_shape(M, K, group)) != TINT4_OK) return s;
-    if (M > 0 && (!x || !w_int8 || !row_scale || !y)) return TINT4_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(w_int8) || !aligned16(row_scale) || !aligned16(y) ||
-        !aligned16(bias))
-        return TINT4_ERR_MISALIGNED;
-    if (M > 0 && (!workspace || workspace_bytes < convrot_linear_workspace_size(M, K, 8)))
-        return TINT4_ERR_WORKSPACE;
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TINT4_ERR_MISALIGNED;
-    if ((s = check_device()) != TINT4_OK) return s;
-    if (M == 0) return TINT4_OK;
-    int8_t* codes = static_cast<int8_t*>(workspace);
-    float* tok_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                                align_up(static_cast<size_t>(M) * K, 256));
-    cudaStream_t st = as_stream(stream);
-    launch_rq_g<__nv_bfloat16, 127, false>(reinterpret_cast<const __nv_bfloat16*>(x), M, K, group,
-                                           codes, tok_scale, st);
-    if ((s = last_launch_status()) != TINT4_OK) return s;
-    return launch_w8a8(codes, tok_scale, w_int8, row_scale,
-                       reinterpret_cast<const __nv_bfloat16*>(bias),
-                       reinterpret_cast<__nv_bfloat16*>(y), M, N, K, st, true);
+    return w8a8_linear_impl<false>(x, w_int8, row_scale, bias, y, M, N, K, group, workspace,
+                                   workspace_bytes, stream);
+}
+
+tint4_status convrot_w8a8_linear_f16(const tint4_bf16* x, const int8_t* w_int8,
+                                     const tint4_f16* row_scale, const tint4_bf16* bias,
+                                     tint4_bf16* y, int M, int N, int K, int group, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+    return w8a8_linear_impl<true>(x, w_int8, row_scale, bias, y, M, N, K, group, workspace,
+                                  workspace_bytes, stream);
 }
 
 tint4_status convrot_w4a8_linear_noalloc(const tint4_bf16* x, const uint8_t* w_packed,

@@ -107,7 +107,9 @@ constexpr int kS8FuseBytes = kFuseMaxRows * kS8FuseMaxK + 64 + kFuseMaxRows * kQ
 // weight boxes are in flight; tok_scale is then unused.  FQ = 0: not fused.
 // GW (group-wise weight scales): row_scale is then the scale matrix
 // [N, K/128] and wzero (GW = 2) the zero points [N, K/128].
-template <int NB, bool A_INT4, bool OUT_I32, int FG = 0, int FQ = 0, int GW = 0>
+// S16 (group-wise only): the scales are IEEE fp16 ("ComfyUI-INT-Crush",
+// "Weight Format": the stored format), copied as such and widened exactly.
+template <int NB, bool A_INT4, bool OUT_I32, int FG = 0, int FQ = 0, int GW = 0, bool S16 = false>
 __global__ void __launch_bounds__(S8Cfg<NB>::THREADS, 1)
 w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __restrict__ act,
                   const float* __restrict__ tok_scale, const float* __restrict__ row_scale,
@@ -188,9 +190,11 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
             mbar_init(gw_bar, 1);
             fence_mbarrier_init();
             const uint32_t nsc = static_cast<uint32_t>(nb * 16 * ngr);
-            mbar_arrive_expect_tx(gw_bar, nsc * 4 + (GW == 2 ? nsc : 0u));
-            bulk_load_1d(const_cast<float*>(sGwScale), row_scale + static_cast<size_t>(b0) * 16 * ngr,
-                         nsc * 4, gw_bar);
+            constexpr uint32_t kSB = S16 ? 2u : 4u;   // bytes per scale
+            mbar_arrive_expect_tx(gw_bar, nsc * kSB + (GW == 2 ? nsc : 0u));
+            bulk_load_1d(const_cast<float*>(sGwScale),
+                         reinterpret_cast<const uint8_t*>(row_scale) + static_cast<size_t>(b0) * 16 * ngr * kSB,
+                         nsc * kSB, gw_bar);
             if (GW == 2)
                 bulk_load_1d(const_cast<uint8_t*>(sGwZero), wzero + static_cast<size_t>(b0) * 16 * ngr,
                              nsc, gw_bar);
@@ -305,8 +309,14 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         if (256 * P + 128 * h >= K) break;   // a half past K (its sums are 0)
-                        gsc[hb][h][0] = sGwScale[ra + h] * kGwUnscale;
-                        gsc[hb][h][1] = sGwScale[rb + h] * kGwUnscale;
+                        if constexpr (S16) {
+                            const __half* s16 = reinterpret_cast<const __half*>(sGwScale);
+                            gsc[hb][h][0] = __half2float(s16[ra + h]) * kGwUnscale;
+                            gsc[hb][h][1] = __half2float(s16[rb + h]) * kGwUnscale;
+                        } else {
+                            gsc[hb][h][0] = sGwScale[ra + h] * kGwUnscale;
+                            gsc[hb][h][1] = sGwScale[rb + h] * kGwUnscale;
+                        }
                         if constexpr (GW == 2) {
                             gzc[hb][h][0] = (128u - 8u * sGwZero[ra + h]) * 0x01010101u;
                             gzc[hb][h][1] = (128u - 8u * sGwZero[rb + h]) * 0x01010101u;

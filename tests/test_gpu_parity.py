@@ -633,6 +633,107 @@ def test_groupwise_full_size():
     assert_groupwise_output(bf16_from_gpu(y), y64, mag, K)
 
 
+# ------------------------------------------------------------------ fp16 weight scales
+# ("ComfyUI-INT-Crush", "Weight Format": the stored scales are fp16)
+
+def _f16_to_gpu(scale_f32):
+    """Oracle scales (float32 on the fp16 grid) -> a float16 device tensor."""
+    return torch.from_numpy(np.ascontiguousarray(scale_f32).astype(np.float16)).to(dev())
+
+
+def _fixture_rows(N, K):
+    """Weights whose first rows hold the hand-derived cases where the fp16
+    rounding of a scale changes a code (tests/golden/fp16_scale_codes.json)."""
+    import json
+    import os
+    d = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "fp16_scale_codes.json")))
+    W = inputs.weights(N, K, seed=840 + K)
+    for r, key in enumerate(("row_sym", "row_asym", "row_int8")):
+        W[r, :] = 0.0
+        W[r, :2] = d[key]
+    W[3, :] = 1e-9           # scales below fp16's smallest subnormal: 0
+    return W
+
+
+@pytest.mark.parametrize("asym", [False, True])
+@pytest.mark.parametrize("N,K,g", [(16, 128, 0), (48, 384, 16), (272, 640, 64), (400, 1024, 256)])
+def test_pack_weights_groupwise_f16_bit_exact(N, K, g, asym):
+    W = _fixture_rows(N, K)
+    wp_ref, s_ref, z_ref, _ = oracle.pack_weights_groupwise(W, g, 128, asym, scale_f16=True)
+    wp, s, z = t4.tint4_pack_weights_groupwise(to_gpu(W), g, asym, scale_dtype=torch.float16)
+    torch.cuda.synchronize()
+    assert s.dtype == torch.float16
+    assert np.array_equal(wp.cpu().numpy(), wp_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint16), oracle.f16_bits(s_ref))
+    if asym:
+        assert np.array_equal(z.cpu().numpy(), z_ref)
+
+
+@pytest.mark.parametrize("asym", [False, True])
+@pytest.mark.parametrize("M,N,K", [(1, 16, 128), (9, 272, 384), (130, 144, 256), (300, 400, 1024)])
+def test_gemm_and_linear_groupwise_f16(M, N, K, asym):
+    """GEMM (streaming and tensor-core kernels) and fused linear with fp16
+    group scales against the oracle on the same fp16 scales."""
+    g = 64
+    x = inputs.activations(M, K, seed=850 + M)
+    codes, st, _ = oracle.quantize_act(x, g, 8)
+    wp, s, z, _ = oracle.pack_weights_groupwise(_fixture_rows(N, K), g, 128, asym, scale_f16=True)
+    zg = to_gpu(z) if asym else None
+    y = t4.w4a8_gemm_groupwise(to_gpu(codes), to_gpu(st), to_gpu(wp), _f16_to_gpu(s), zg)
+    yl = t4.convrot_w4a8_linear_groupwise(bf16_to_gpu(x), to_gpu(wp), _f16_to_gpu(s), g, zg)
+    torch.cuda.synchronize()
+    y64, mag = oracle.gemm_groupwise_f64(codes, st, wp, s, z)
+    assert_groupwise_output(bf16_from_gpu(y), y64, mag, K)
+    assert_groupwise_output(bf16_from_gpu(yl), y64, mag, K)
+
+
+@pytest.mark.parametrize("N,K,g", [(16, 128, 0), (272, 320, 64), (256, 4096, 256), (48, 352, 16)])
+def test_quantize_weights_int8_f16_bit_exact(N, K, g):
+    W = _fixture_rows(N, K)
+    c_ref, s_ref = oracle.quantize_weights_int8(W, g, scale_f16=True)
+    c, s = t4.tint4_quantize_weights_int8(to_gpu(W), g, scale_dtype=torch.float16)
+    torch.cuda.synchronize()
+    assert s.dtype == torch.float16
+    assert np.array_equal(c.cpu().numpy(), c_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint16), oracle.f16_bits(s_ref))
+
+
+@pytest.mark.parametrize("M,N,K,g", [(1, 256, 256, 256), (17, 272, 320, 64), (385, 128, 4096, 256)])
+def test_w8a8_f16_gemm_and_linear(M, N, K, g):
+    x = inputs.activations(M, K, seed=860 + M)
+    wc, sr = oracle.quantize_weights_int8(inputs.weights(N, K, seed=861 + N), g, scale_f16=True)
+    codes, st, _ = oracle.quantize_act(x, g, 8)
+    b = inputs.f32_to_bf16_bits(np.linspace(-1, 1, N, dtype=np.float32))
+    y = t4.w8a8_gemm(to_gpu(codes), to_gpu(st), to_gpu(wc), _f16_to_gpu(sr), bf16_to_gpu(b))
+    yl = t4.convrot_w8a8_linear(bf16_to_gpu(x), to_gpu(wc), _f16_to_gpu(sr), g)
+    torch.cuda.synchronize()
+    acc = oracle.gemm_i32(codes, wc)
+    assert_gemm_output(bf16_from_gpu(y), oracle.epilogue_f64(acc, st, sr, b), b)
+    assert_gemm_output(bf16_from_gpu(yl), oracle.epilogue_f64(acc, st, sr))
+
+
+def test_groupwise_f16_full_size():
+    """The DiT QKV layer with asymmetric group-wise weights in the pages'
+    stored format (fp16 scales): packing bit-exact, every output of the fused
+    linear against the oracle."""
+    name = "dit_qkv_w4a8_asym_g128"
+    w = inputs.WORKLOADS[name]
+    M, N, K, g = w["M"], w["N"], w["K"], w["group"]
+    x_np, W = inputs.layer_inputs(name)
+    wp_ref, s_ref, z_ref, _ = oracle.pack_weights_groupwise(W, g, 128, True, scale_f16=True)
+    wp, s, z = t4.tint4_pack_weights_groupwise(to_gpu(W), g, True, scale_dtype=torch.float16)
+    x = bf16_to_gpu(x_np)
+    y = t4.convrot_w4a8_linear_groupwise(x, wp, s, g, z)
+    codes, st = t4.convrot_quantize_act(x, g, 8)
+    torch.cuda.synchronize()
+    assert np.array_equal(wp.cpu().numpy(), wp_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint16), oracle.f16_bits(s_ref))
+    assert np.array_equal(z.cpu().numpy(), z_ref)
+    y64, mag = oracle.gemm_groupwise_f64(codes.cpu().numpy(), st.cpu().numpy(), wp_ref, s_ref,
+                                         z_ref)
+    assert_groupwise_output(bf16_from_gpu(y), y64, mag, K)
+
+
 # ------------------------------------------------------------------ W4A16
 
 @pytest.mark.parametrize("M,N,K", [(1, 16, 128), (4, 272, 384), (16, 512, 1024),
