@@ -20,10 +20,15 @@ region) and, under "rows", the other workloads' kernels: the tiny layer, the
 W4A4 variant, the MLP pair (group 64), the small-M W4A16 decode GEMM, and the
 rotate+quantize kernel alone.
 
-Multi-GPU (torchrun): every rank runs the same per-GPU workload on its own
-tokens (independent batches, no exchange: weak scaling); the step time is the
-max over ranks.  ``--impl reference`` times the CPU oracle on the host cores
-instead (rank 0 only).
+Multi-GPU: one process per GPU (``--gpus N`` starts them through torch's
+launcher when no launcher has; under torchrun the environment gives the
+ranks).  Default (``--parallel replicas``): every rank runs the same per-GPU
+workload on its own tokens (independent batches, no exchange: weak scaling).
+``--parallel nsplit``: the layer's weight rows are split over the ranks
+(column-parallel, the same tokens on every rank; ``--gather`` all-gathers
+the column shards into the full y over NCCL): strong scaling.  The step
+time is the max over ranks.  ``--impl reference`` times the CPU oracle on
+the host cores instead (rank 0 only).
 """
 from __future__ import annotations
 
@@ -394,6 +399,112 @@ def run_ours(args, rank, world, dev):
         line["cpu_baseline"] = cpu
     if rows:
         line["rows"] = rows
+    return line
+
+
+def run_nsplit(args, rank, world, dev):
+    """The same layer split along N over the ranks (column-parallel): every
+    rank holds its N / world weight rows, receives the whole x (the same
+    tokens on every rank) and computes its columns of y; with --gather the
+    shards are all-gathered into the full y on every rank (NCCL).  Total work
+    is fixed as the ranks grow: strong scaling."""
+    import int4_weight_quantized_block_b200 as t4
+    from int4_weight_quantized_block_b200 import inputs, build as _build
+    from int4_weight_quantized_block_b200.column_parallel import ColumnParallelLinear
+
+    _build.build()
+    pk = peaks()
+    int8_peak = INT8_OVER_BF16 * pk["bf16"]
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.zero_()
+
+    w = inputs.WORKLOADS[MAIN]
+    M, N, K, g = w["M"], w["N"], w["K"], w["group"]
+    x_np, W_np = inputs.layer_inputs(MAIN)          # replicated: the same x and W everywhere
+    x = bf16_gpu(x_np, dev)
+    wp, sr = t4.tint4_pack_weights(torch.from_numpy(W_np).to(dev), g)
+    wps, srs, _ = ColumnParallelLinear.shard(wp, sr, rank, world)
+    del wp, sr
+    layer = ColumnParallelLinear(wps, srs, g, N, rank, world, gather=args.gather)
+    ws = torch.empty(t4.convrot_linear_workspace_size(M, K, 8), dtype=torch.uint8, device=dev)
+    n_r = layer.hi - layer.lo
+    ops = 2.0 * M * N * K
+
+    def step():
+        return layer(x, ws)
+
+    for _ in range(args.warmup):
+        flush()
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev) as clk:
+        times = time_steps(step, args.steps, flush, dev)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    ms = max_over_ranks(sum(times) / len(times), dev)
+
+    # the shard's GEMM launch (even/odd codes, as inside the fused linear)
+    codes, st = t4.convrot_quantize_act(x, g, 8)
+    codes_eo = t4.even_odd_codes(codes)
+    y_r = torch.empty((M, n_r), dtype=torch.bfloat16, device=dev)
+    gemm_ms = statistics.median(time_steps(
+        lambda: t4.tint4_debug_w4a8_gemm_even_odd(codes_eo, st, wps, srs, None, y_r),
+        args.steps, flush, dev))
+    gemm_tops = 2.0 * M * n_r * K / (gemm_ms * 1e-3) / 1e12
+
+    # end to end: x from pinned host memory on every rank, the rank's columns
+    # (or, gathered, the full y) back to pinned host memory
+    x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_cols = N if args.gather else n_r
+    y_host = torch.empty((M, out_cols), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        y_host.copy_(layer(x_dev, ws), non_blocking=True)
+
+    e2e_ms = max_over_ranks(statistics.mean(time_steps(e2e_step, max(3, args.steps // 4),
+                                                       flush, dev)), dev)
+    line = {
+        "metric": METRIC,
+        "value": round(ops / (ms * 1e-3) / 1e12, 3),
+        "unit": "TOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 5),
+        "higher_is_better": True,
+        "scaling": "strong",
+        "vs_baseline": None,
+        "dtype": "int8",
+        "data": "synthetic (seeded; x ~ N(0,1) with 1% channels x50, W ~ N(0,0.02) packed offline)",
+        "config": {"workload": f"{MAIN}: ConvRot W4A8 fused-QKV projection, M={M} tokens, "
+                               f"K={K}, N={N}, Hadamard group {g}, split along N over {world} GPUs",
+                   "M": M, "N": N, "K": K, "group": g, "act_bits": 8,
+                   "parallelism": f"nsplit{world}" + (" + all-gather of y" if args.gather else ""),
+                   "rows_per_gpu": n_r,
+                   "l2": "flushed (256 MiB write) before every timed step, outside the events"},
+        "roofline": {"bound": "tensor",
+                     "kernel": "w4a8_tmem_gemm_kernel<even/odd codes> on the rank's weight rows",
+                     "achieved": round(gemm_tops, 2), "peak": round(int8_peak, 1),
+                     "unit": "TOPS", "frac": round(gemm_tops / int8_peak, 4), "traffic": None,
+                     "peak_source": f"{pk['source']}: 2 x bf16 cuBLAS burst "
+                                    f"{pk['bf16']} TFLOP/s (nominal int8:bf16 = 2)",
+                     "kernel_us": round(gemm_ms * 1e3, 2)},
+        "e2e": {"value": round(ops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TOPS",
+                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * out_cols * 2,
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(w, target_s=args.cpu_seconds)
     return line
 
 
@@ -821,6 +932,11 @@ def main():
     ap.add_argument("--no-rows", action="store_true", help="skip the per-workload rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--parallel", choices=["replicas", "nsplit"], default="replicas",
+                    help="replicas: every GPU runs the layer on its own tokens (weak scaling); "
+                         "nsplit: the layer's weight rows split over the GPUs (strong scaling)")
+    ap.add_argument("--gather", action="store_true",
+                    help="nsplit: all-gather the column shards into the full y on every GPU")
     ap.add_argument("--profile", default=None,
                     help="run only a few launches of one kernel for ncu: qkv_gemm, "
                          "qkv_gemm_w4a4, qkv_gemm_gw, qkv_quantize, w4a16_M<m>, "
@@ -834,9 +950,23 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # one process per GPU: start the ranks ourselves (torchrun on this node)
+        import socket
+        sock = socket.socket()
+        sock.bind(("127.0.0.1", 0))
+        port = sock.getsockname()[1]
+        sock.close()
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+               f"--nproc-per-node={args.gpus}", "--master-addr", "127.0.0.1",
+               "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+        sys.exit(subprocess.call(cmd))
+
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if "WORLD_SIZE" in os.environ and args.gpus not in (1, world):
+        ap.error(f"--gpus {args.gpus} under a launcher of {world} ranks")
 
     if args.impl == "reference":
         if rank == 0:
@@ -853,7 +983,7 @@ def main():
         torch.distributed.init_process_group("nccl", device_id=dev,
                                              timeout=datetime.timedelta(seconds=120))
     try:
-        line = run_ours(args, rank, world, dev)
+        line = (run_nsplit if args.parallel == "nsplit" else run_ours)(args, rank, world, dev)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

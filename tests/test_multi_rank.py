@@ -84,3 +84,19 @@ def test_reference_arm_prints_on_rank0_only(rank):
         assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
     else:
         assert lines == []
+
+
+def test_gpus_flag_launches_the_ranks_itself():
+    """bench.py --gpus 2 outside a launcher starts two ranks itself (torch's
+    launcher on this node); the reference arm then prints one line, from rank
+    0, and both ranks exit 0."""
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl",
+                        "reference", "--steps", "1", "--warmup", "3", "--cpu-seconds", "0.2"],
+                       capture_output=True, text=True, env=env, timeout=900)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0
