@@ -549,6 +549,16 @@ def bench_rows(args, t4, inputs, dev, flush, pk, int8_peak):
                 dev))
             row.update({"linear_gemm_us": round(lg_ms * 1e3, 2),
                         "linear_gemm_frac_int8": round(ops / lg_ms / 1e9 / int8_peak, 4)})
+            if bits == 4:
+                # packed codes widened once into a workspace, then the int8 GEMM
+                # (w4a4_gemm_widened: both launches inside the timed region)
+                wsw = torch.empty(t4.convrot_linear_workspace_size(M, K, 4), dtype=torch.uint8,
+                                  device=dev)
+                gw_ms = statistics.median(time_steps(
+                    lambda: t4.w4a4_gemm_widened(codes, st, wp, sr, None, y, wsw), reps, flush,
+                    dev))
+                row.update({"gemm_widened_us": round(gw_ms * 1e3, 2),
+                            "gemm_widened_frac_int8": round(ops / gw_ms / 1e9 / int8_peak, 4)})
         return row
 
     rows["tiny_w4a8"] = gemm_layer("tiny_w4a8")

@@ -125,6 +125,21 @@ tint4_status w4a4_gemm(const uint8_t* a_packed, const float* tok_scale, const ui
                        const float* row_scale, const tint4_bf16* bias, tint4_bf16* y, int M,
                        int N, int K, void* stream);
 
+/*
+ * w4a4_gemm with a caller workspace (at least convrot_linear_workspace_size(M,
+ * K, 4) bytes, 256-byte aligned; its contents are scratch): above 16 tokens
+ * the packed activation codes are widened once, to one int8 per code in the
+ * workspace, and the int8 tensor-core GEMM runs on them, instead of being
+ * widened in shared memory for every weight-row tile.  Same int32 sums and
+ * the same output bits as w4a4_gemm; at most 16 tokens it is w4a4_gemm (the
+ * workspace is unused and may be NULL).  Errors as w4a4_gemm, plus
+ * TINT4_ERR_WORKSPACE.
+ */
+tint4_status w4a4_gemm_widened(const uint8_t* a_packed, const float* tok_scale,
+                               const uint8_t* w_packed, const float* row_scale,
+                               const tint4_bf16* bias, tint4_bf16* y, int M, int N, int K,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of workspace the fused linears need (convrot_w4a8_linear: bits 8,
  * convrot_w4a4_linear: bits 4; the grouped, group-wise and W8A8 linears: bits
  * 8): the activation codes, one byte per code for both widths (M * K), plus

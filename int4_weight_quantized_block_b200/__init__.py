@@ -25,6 +25,7 @@ __all__ = [
     "w4a8_gemm",
     "w4a4_gemm",
     "convrot_linear_workspace_size",
+    "w4a4_gemm_widened",
     "convrot_w4a8_linear",
     "convrot_w4a4_linear",
     "convrot_w4a8_linear_noalloc",
@@ -139,6 +140,32 @@ def w4a4_gemm(a_packed, tok_scale, w_packed, row_scale, bias=None, y=None) -> to
     """packed int4 codes a [M, K/2] x packed int4 W [N, K/2] -> bf16 y [M, N]."""
     return _gemm("w4a4_gemm", a_packed, tok_scale, w_packed, row_scale, bias, y, torch.uint8,
                  lambda K: K // 2)
+
+
+def w4a4_gemm_widened(a_packed, tok_scale, w_packed, row_scale, bias=None, y=None,
+                      workspace=None) -> torch.Tensor:
+    """w4a4_gemm whose packed activation codes are widened once into a
+    workspace (above 16 tokens) before the int8 tensor-core GEMM: the same
+    output bits."""
+    _need(a_packed, "a_packed", torch.uint8)
+    M = a_packed.shape[0]
+    K = 2 * a_packed.shape[1]
+    N = w_packed.shape[0]
+    _need(tok_scale, "tok_scale", torch.float32, (M,))
+    _need(w_packed, "w_packed", torch.uint8, (N, K // 2))
+    _need(row_scale, "row_scale", torch.float32, (N,))
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, (N,))
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=a_packed.device)
+    _need(y, "y", torch.bfloat16, (M, N))
+    need = convrot_linear_workspace_size(M, K, 4)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=a_packed.device)
+    _native.call("w4a4_gemm_widened", _ptr(a_packed), _ptr(tok_scale), _ptr(w_packed),
+                 _ptr(row_scale), _ptr(bias), _ptr(y), M, N, K, _ptr(workspace), workspace.numel(),
+                 _stream(a_packed.device))
+    return y
 
 
 def convrot_linear_workspace_size(M: int, K: int, bits: int) -> int:

@@ -43,6 +43,7 @@ SIGNATURES = {
     "convrot_quantize_act": (I, [P, I, I, I, I, P, P, P]),
     "w4a8_gemm": (I, [P, P, P, P, P, P, I, I, I, P]),
     "w4a4_gemm": (I, [P, P, P, P, P, P, I, I, I, P]),
+    "w4a4_gemm_widened": (I, [P, P, P, P, P, P, I, I, I, P, SZ, P]),
     "convrot_linear_workspace_size": (SZ, [I, I, I]),
     "convrot_w4a8_linear_workspace": (SZ, [I, I]),
     "convrot_w4a8_linear": (I, [P, P, P, P, P, I, I, I, I, P, SZ, P]),

@@ -580,4 +580,31 @@ rotate_quantize_rows_kernel(const InT* __restrict__ in, int rows, int K, void* _
     rq_team_rows<InT, G, Q, PACKED, EVOD, CPL, S16>(in, rows, K, codes, scales, red);
 }
 
+// Packed int4 activation codes [rows, K/2] (two's complement nibbles, low
+// nibble = even K index) -> one int8 code per byte [rows, K] in the even/odd
+// K order of the tensor-core GEMM (0, 2, 4, 6, 1, 3, 5, 7 in every block of
+// 8): per packed word, the low nibbles sign-extended into the first four
+// bytes, the high nibbles into the last four.  Grid-stride over 16-byte
+// pieces of the packed rows (K % 32 == 0: a row is whole pieces).
+__global__ void __launch_bounds__(256)
+widen_int4_codes_kernel(const uint8_t* __restrict__ packed, int8_t* __restrict__ codes, long pieces) {
+    grid_dependency_wait();   // the codes may come from the grid just before
+    for (long i = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; i < pieces;
+         i += static_cast<long>(gridDim.x) * blockDim.x) {
+        const uint4 p = __ldg(reinterpret_cast<const uint4*>(packed) + i);
+        const uint32_t w[4] = {p.x, p.y, p.z, p.w};
+        uint32_t o[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            // (n ^ 8) - 8 sign-extends a nibble; byte-wise, no borrow between bytes
+            o[2 * j] = __vsub4((w[j] & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);
+            o[2 * j + 1] = __vsub4(((w[j] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(codes) + 2 * i;
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+    grid_launch_dependents();
+}
+
 }  // namespace tint4

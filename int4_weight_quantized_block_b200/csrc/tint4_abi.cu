@@ -1062,6 +1062,44 @@ tint4_status w4a4_gemm(const uint8_t* a_packed, const float* tok_scale, const ui
     return gemm_entry(true, a_packed, tok_scale, w_packed, row_scale, bias, y, M, N, K, stream);
 }
 
+tint4_status w4a4_gemm_widened(const uint8_t* a_packed, const float* tok_scale,
+                               const uint8_t* w_packed, const float* row_scale,
+                               const tint4_bf16* bias, tint4_bf16* y, int M, int N, int K,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+    tint4_status s = check_mnk(M, N, K);
+    if (s != TINT4_OK) return s;
+    if (M > 0 && (!a_packed || !tok_scale || !w_packed || !row_scale || !y))
+        return TINT4_ERR_INVALID_ARG;
+    if (!aligned16(a_packed) || !aligned16(tok_scale) || !aligned16(w_packed) ||
+        !aligned16(row_scale) || !aligned16(y) || !aligned16(bias))
+        return TINT4_ERR_MISALIGNED;
+    if (!linear_codes_evod(M))   // the streaming kernel reads packed codes itself
+        return gemm_entry(true, a_packed, tok_scale, w_packed, row_scale, bias, y, M, N, K, stream);
+    if (!workspace || workspace_bytes < convrot_linear_workspace_size(M, K, 4))
+        return TINT4_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TINT4_ERR_MISALIGNED;
+    int dev = 0;
+    if ((s = check_device(&dev)) != TINT4_OK) return s;
+    cudaStream_t st = as_stream(stream);
+    int8_t* codes = static_cast<int8_t*>(workspace);
+    const long pieces = static_cast<long>(M) * K / 32;
+    const int grid = static_cast<int>(std::min<long>((pieces + 255) / 256, 8L * num_sms(dev)));
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, widen_int4_codes_kernel, a_packed, codes, pieces) != cudaSuccess) {
+        cudaGetLastError();
+        return TINT4_ERR_CUDA;
+    }
+    return launch_gemm<false, false, true>(codes, w_packed, tok_scale, row_scale,
+                                           reinterpret_cast<const __nv_bfloat16*>(bias), y, M, N,
+                                           K, st, true);
+}
+
 size_t convrot_w4a8_linear_workspace(int M, int K) {
     return convrot_linear_workspace_size(M, K, 8);
 }

@@ -333,6 +333,35 @@ def test_full_size_workloads(name):
     acc_gpu = t4.tint4_debug_int32_gemm(a, bits, to_gpu(wp_ref))
     torch.cuda.synchronize()
     assert np.array_equal(acc_gpu.cpu().numpy(), acc)
+    if bits == 4:
+        # the packed-code GEMM entries on the same codes: every output
+        y4 = t4.w4a4_gemm(a, to_gpu(st_ref), to_gpu(wp_ref), to_gpu(sr_ref))
+        y4w = t4.w4a4_gemm_widened(a, to_gpu(st_ref), to_gpu(wp_ref), to_gpu(sr_ref))
+        torch.cuda.synchronize()
+        ref = oracle.epilogue_f64(acc, st_ref, sr_ref)
+        assert_gemm_output(bf16_from_gpu(y4), ref)
+        assert np.array_equal(bf16_from_gpu(y4w), bf16_from_gpu(y4))
+
+
+@pytest.mark.parametrize("M,N,K", [(9, 272, 512), (17, 144, 256), (300, 768, 3072),
+                                   (2048, 8192, 1024)])
+def test_w4a4_gemm_widened(M, N, K):
+    """Packed int4 codes widened once into a workspace, then the int8
+    tensor-core GEMM: the bits of w4a4_gemm, which the oracle holds."""
+    g = 256
+    x = inputs.activations(M, K, seed=1400 + M)
+    W = inputs.weights(N, K, seed=1401)
+    wp, sr, qw = oracle.pack_weights(W, g)
+    qa, st, packed = oracle.quantize_act(x, g, 4)
+    b = inputs.f32_to_bf16_bits(np.linspace(-1, 1, N, dtype=np.float32))
+    a, stg, wpg, srg, bg = to_gpu(packed), to_gpu(st), to_gpu(wp), to_gpu(sr), bf16_to_gpu(b)
+    y = t4.w4a4_gemm(a, stg, wpg, srg, bg)
+    yw = t4.w4a4_gemm_widened(a, stg, wpg, srg, bg)
+    yw2 = t4.w4a4_gemm_widened(a, stg, wpg, srg, bg)   # the workspace holds the last call's codes
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_from_gpu(yw), bf16_from_gpu(y))
+    assert np.array_equal(bf16_from_gpu(yw2), bf16_from_gpu(y))
+    assert_gemm_output(bf16_from_gpu(yw), oracle.epilogue_f64(oracle.gemm_i32(qa, qw), st, sr, b), b)
 
 
 @pytest.mark.parametrize("bits", [8, 4])
