@@ -11,36 +11,47 @@
 // byte per weight).
 //
 // Shape of the product on the tensor core: the weights are the MMA's M side
-// (128 rows = the 128 TMEM lanes) and the tokens its N side (192 per tile).
-// Per 128-wide K step the TMA brings one activation tile (192 tokens x 128
-// int8 codes, 128-byte swizzle: the MMA's B operand) and one packed weight
-// tile (128 rows x 64 bytes, 64-byte swizzle) into shared memory.  Each of
-// 128 unpack threads owns one weight row: it reads its 64 packed bytes
-// (bank-conflict-free thanks to the swizzle), widens every nibble to an int8
-// (x16, see below) and writes the 128 K values with one tcgen05.st into a
-// TMEM A-operand stage.  The widened weights never go back to shared memory.
+// (128 rows = the 128 TMEM lanes) and the tokens its N side (BN per tile:
+// 256 for int8 activation codes, 192 for the packed-int4-code and int8-weight
+// forms, see TmCfg).  Per 128-wide K step the TMA brings one activation tile
+// (BN tokens x 128 int8 codes, 128-byte swizzle: the MMA's B operand) and one
+// packed weight tile (128 rows x 64 bytes, 64-byte swizzle) into shared
+// memory.  Each of 128 unpack threads owns one weight row: it reads its 64
+// packed bytes (bank-conflict-free thanks to the swizzle), widens every
+// nibble to an int8 (x16, see below) and writes the 128 K values with one
+// tcgen05.st into a TMEM A-operand stage.  The widened weights never go back
+// to shared memory.
 //
-// The CTA is persistent (one per SM) and walks a static list of 128 x 192
+// The CTA is persistent (one per SM) and walks a static list of 128 x BN
 // tiles.  Warp roles (18 warps):
-//   warp 0      TMA producer (4-deep ring of 24 KB activation + 8 KB weight
-//               stages)
+//   warp 0      TMA producer (ring of 4 or 5 activation + weight stages)
 //   warp 1      TMEM owner; one thread issues tcgen05.mma.cta_group::1.kind::i8
-//               (A from TMEM, B from shared memory, M 128, N 192, K 32)
+//               (A from TMEM, B from shared memory, M 128, N BN, K 32)
 //   warps 2-9   weight unpack into the 4 TMEM A stages (32 columns each);
 //               warps 2-5 take the even K steps and warps 6-9 the odd ones,
 //               so two unpack chains run side by side on every SM
 //               sub-partition (each warp may only reach its quarter of the
 //               TMEM lanes, warp % 4)
-//   warps 10-17 epilogue: tcgen05.ld of one accumulator buffer while the MMAs
-//               fill the other (two 192-column int32 buffers); two warps per
-//               TMEM lane quarter, each on half of the tokens.  A thread holds
-//               one weight row (= one output column), so it scales its values,
+//   warps 10-17 epilogue: tcgen05.ld of the accumulator; two warps per TMEM
+//               lane quarter, each on half of the tokens.  A thread holds one
+//               weight row (= one output column), so it scales its values,
 //               rounds them to bf16 and writes them with 2-byte shared-memory
-//               stores into a [192 tokens][128 columns] staging tile, which the
+//               stores into a [BN tokens][128 columns] staging tile, which the
 //               8 warps then copy to y (row-major [M, N]) in 16-byte row pieces
 //               (a TMA tensor store of the tile shared the copy engine with the
-//               mainloop's loads and cost about 15 %).
-// TMEM columns: accumulators at 0 and 192, A stages at 384 + 32 s.
+//               mainloop's loads and cost about 15 %).  The tile's token
+//               scales are copied to shared memory while its MMAs run.
+// TMEM columns: BN = 256: one accumulator at 0, A stages at 256 + 32 s; the
+// epilogue reads it two 32-token chunks at a time and hands it back after
+// its last read, before the math on those chunks.  BN = 192: two
+// accumulators at 0 and 192 (the epilogue drains one while the MMAs fill the
+// other), A stages at 384 + 32 s.
+//
+// Why 256 tokens: the step time follows the bytes the TMA brings per step
+// (about 40 B per cycle and SM), of which the weight tile is a fixed 8 KB;
+// a 256-token tile moves 40 KB for 4/3 of the work of a 192-token one (32
+// KB).  On the DiT layers it took QKV 127 -> 123 us, MLP up 164 -> 156, MLP
+// down 162 -> 145 (K = 12288: 96 steps per tile share one drain).
 //
 // A nibble moved into the high half of its byte, low half cleared, is the
 // int8 value 16 * code; the accumulators hold 16 * acc and the epilogue
@@ -68,37 +79,40 @@
 namespace tint4 {
 
 constexpr int kTmBM = 128;       // weight rows per tile (UMMA M, TMEM lanes)
-constexpr int kTmBN = 192;       // tokens per tile (UMMA N)
 constexpr int kTmBK = 128;       // K values per stage
-constexpr int kTmStages = 4;     // TMEM A stages (and shared-memory stages of the A_INT4 / W8 forms)
-// Shared-memory stages: 5 for int8 codes x packed weights, so that the loads
-// run one stage further ahead of the unpack than the 4 TMEM A stages allow
-// (the unpack of step j also waits for the MMAs of step j - 4, which free its
-// TMEM stage); the packed-int4-code and int8-weight forms have no room for a
-// fifth stage.
-template <bool A_INT4, bool W8>
-struct TmRing {
-    static constexpr int S = (A_INT4 || W8) ? 4 : 5;
-};
+constexpr int kTmStages = 4;     // TMEM A stages
 constexpr int kTmThreads = 576;  // 18 warps
-constexpr int kTmActBytes = kTmBN * kTmBK;            // 24 KB per stage
 constexpr int kTmWBytes = kTmBM * kTmBK / 2;          // 8 KB packed weights per stage
-constexpr int kTmOutBytes = kTmBN * kTmBM * 2;        // 48 KB bf16 staging tile
-constexpr int kTmActPBytes = kTmBN * kTmBK / 2;       // 12 KB packed int4 activation codes per stage
-constexpr int kTmSmemBytes =
-    TmRing<false, false>::S * (kTmActBytes + kTmWBytes) + kTmOutBytes + 256 + 1024;
-constexpr int kTmSmemBytesA4 =
-    TmRing<true, false>::S * (kTmActBytes + kTmWBytes + kTmActPBytes) + kTmOutBytes + 256 + 1024;
 constexpr int kTmW8Bytes = kTmBM * kTmBK;             // 16 KB int8 weights per stage (W8A8)
-constexpr int kTmSmemBytesW8 =
-    TmRing<false, true>::S * (kTmActBytes + kTmW8Bytes) + kTmOutBytes + 256 + 1024;
-static_assert(kTmSmemBytes <= 227 * 1024 && kTmSmemBytesA4 <= 227 * 1024 &&
-                  kTmSmemBytesW8 <= 227 * 1024,
-              "shared memory budget");
-constexpr uint32_t kTmColD = 0;                       // accumulator buffer b at b * kTmBN
-constexpr uint32_t kTmColA = 2 * kTmBN;               // A stage s at kTmColA + 32 s
-static_assert(kTmColA + 32 * kTmStages <= 512, "TMEM budget");
-static_assert(kTmActBytes % 1024 == 0 && kTmWBytes % 1024 == 0, "swizzled stage alignment");
+
+// Tile shape and rings of the three forms.  Int8 codes x packed int4
+// weights (the fused linears' form): 256 tokens per tile (N = 256, 128-cycle
+// MMAs: a third more work per issued MMA than N = 192) with one accumulator
+// buffer (256 TMEM columns + 4 A stages of 32); the epilogue hands the
+// buffer back as soon as it has read it.  Packed int4 codes (A_INT4) and
+// int8 weights (W8): 192 tokens, two accumulator buffers (the larger stages
+// leave no room for 256-token tiles).
+template <bool A_INT4, bool W8>
+struct TmCfg {
+    static constexpr bool WIDE = !A_INT4 && !W8;
+    static constexpr int BN = WIDE ? 256 : 192;            // tokens per tile (UMMA N)
+    static constexpr int NBUF = WIDE ? 1 : 2;              // accumulator buffers
+    // shared-memory stages: 5 for int8 codes x packed weights at N = 192, so
+    // that the loads run one stage further ahead of the unpack than the 4 TMEM
+    // A stages allow (the unpack of step j also waits for the MMAs of step
+    // j - 4, which free its TMEM stage); no room for a fifth otherwise
+    static constexpr int S = (A_INT4 || W8 || WIDE) ? 4 : 5;
+    static constexpr int ACT = BN * kTmBK;                 // int8 codes per stage
+    static constexpr int ACTP = A_INT4 ? BN * kTmBK / 2 : 0;   // packed int4 codes per stage
+    static constexpr int WB = W8 ? kTmW8Bytes : kTmWBytes;
+    static constexpr int OUT = BN * kTmBM * 2;             // bf16 staging tile
+    static constexpr int SMEM = S * (ACT + WB + ACTP) + OUT + 256 + BN * 4 + 1024;
+    static constexpr uint32_t COL_A = NBUF * BN;           // A stage s at COL_A + 32 s
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
+    static_assert(COL_A + 32 * kTmStages <= 512, "TMEM budget");
+    static_assert(ACT % 1024 == 0 && kTmWBytes % 1024 == 0, "swizzled stage alignment");
+};
+constexpr uint32_t kTmColD = 0;                       // accumulator buffer b at b * BN
 
 // The weight matrices one launch multiplies the same activation codes with:
 // one for a plain GEMM, up to kTmMaxGroups for a grouped one (separate Q, K,
@@ -186,16 +200,18 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
     static_assert(!(W8 && EVOD), "int8 weights are stored in the natural K order");
     constexpr bool kEvod = EVOD || A_INT4;   // widen in the even/odd K order
     constexpr int kWB = W8 ? kTmW8Bytes : kTmWBytes;   // weight bytes per stage
-    constexpr int kS = TmRing<A_INT4, W8>::S;           // shared-memory stages
+    using C = TmCfg<A_INT4, W8>;
+    constexpr int kBN = C::BN;                          // tokens per tile
+    constexpr int kS = C::S;                            // shared-memory stages
     constexpr int kT = kTmStages;                       // TMEM A stages
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* sAct = smem;
-    uint8_t* sW = smem + kS * kTmActBytes;
+    uint8_t* sW = smem + kS * C::ACT;
     uint8_t* sActP = sW + kS * kWB;                                    // A_INT4 only
-    uint8_t* sOut = sActP + (A_INT4 ? kS * kTmActPBytes : 0);
-    uint64_t* act_full = reinterpret_cast<uint64_t*>(sOut + kTmOutBytes);
+    uint8_t* sOut = sActP + kS * C::ACTP;
+    uint64_t* act_full = reinterpret_cast<uint64_t*>(sOut + C::OUT);
     uint64_t* empty = act_full + kS;               // [kS] stage consumed by the MMAs (commit)
     uint64_t* a_full = empty + kS;                 // [kT] TMEM A stage written (one arrival per warp)
     uint64_t* acc_full = a_full + kT;              // [2] accumulator ready (commit)
@@ -204,10 +220,11 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
     volatile uint32_t* epi_go = tmem_slot + 2;     // epilogue: proceed with this tile
+    float* sTok = reinterpret_cast<float*>(sOut + C::OUT + 256);   // the tile's token scales
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int m_tiles = (M + kTmBN - 1) / kTmBN;
+    const int m_tiles = (M + kBN - 1) / kBN;
     const int n_work = grp.tile_end[grp.count - 1];
     const int KT = (K + kTmBK - 1) / kTmBK;
     const int my_tiles = (blockIdx.x < n_work) ? (n_work - 1 - blockIdx.x) / gridDim.x + 1 : 0;
@@ -221,7 +238,7 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
         for (int h = 0; h < kTmMaxGroups - 1; ++h)
             if (h + 1 < grp.count && tile >= grp.tile_end[h]) g = h + 1;
         const int t = tile - (g > 0 ? grp.tile_end[g - 1] : 0);
-        return TileAt{g, (t % m_tiles) * kTmBN, (t / m_tiles) * kTmBM};
+        return TileAt{g, (t % m_tiles) * kBN, (t / m_tiles) * kTmBM};
     };
 
     if (threadIdx.x == 0) {
@@ -270,11 +287,11 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                                            kDevErrTimeoutProducer))
                         break;
                     if (A_INT4) {
-                        mbar_arrive_expect_tx(&act_full[s], kTmActPBytes + kTmWBytes);
-                        tma_load_2d(&tmap_act, &act_full[s], sActP + s * kTmActPBytes, kt * (kTmBK / 2), m0);
+                        mbar_arrive_expect_tx(&act_full[s], C::ACTP + kTmWBytes);
+                        tma_load_2d(&tmap_act, &act_full[s], sActP + s * C::ACTP, kt * (kTmBK / 2), m0);
                     } else {
-                        mbar_arrive_expect_tx(&act_full[s], kTmActBytes + kWB);
-                        tma_load_2d(&tmap_act, &act_full[s], sAct + s * kTmActBytes, kt * kTmBK, m0);
+                        mbar_arrive_expect_tx(&act_full[s], C::ACT + kWB);
+                        tma_load_2d(&tmap_act, &act_full[s], sAct + s * C::ACT, kt * kTmBK, m0);
                     }
                     tma_load_2d(tmap_w, &act_full[s], sW + s * kWB, kt * (W8 ? kTmBK : kTmBK / 2), n0);
                     ++issued;
@@ -291,7 +308,7 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = umma_idesc_i8(kTmBM, kTmBN);
+            constexpr uint32_t idesc = umma_idesc_i8(kTmBM, kBN);
             // B descriptors: stage s starts (s * bytes) / 16 units above stage 0,
             // MMA kk of a stage 32 bytes = 2 units further (the address field
             // cannot carry: shared addresses are below 2^18)
@@ -304,15 +321,15 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             uint32_t sph = 0u, tph = 0u;
             bool ok = true;
             for (int i = 0; i < my_tiles && ok; ++i) {
-                const int buf = i & 1;
-                const uint32_t aph = (i >> 1) & 1;
+                const int buf = C::NBUF == 2 ? (i & 1) : 0;
+                const uint32_t aph = C::NBUF == 2 ? ((i >> 1) & 1) : (i & 1);
                 if (!mbar_wait_bounded(&acc_empty[buf], aph ^ 1, abort_flag, wait_ns,
                                        kDevErrTimeoutConsumer)) {
                     ok = false;
                     break;
                 }
                 tcgen05_fence_after();
-                const uint32_t d_tmem = tmem_base + kTmColD + buf * kTmBN;
+                const uint32_t d_tmem = tmem_base + kTmColD + buf * kBN;
                 for (int kt = 0; kt < KT; ++kt) {
                     // a_full implies the stage has landed: the unpack warps arrive
                     // on it only after they have seen it (one wait per stage: the
@@ -328,8 +345,8 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                         break;
                     }
                     tcgen05_fence_after();
-                    const uint32_t a_tmem = tmem_base + kTmColA + 32 * t;
-                    const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(s * (kTmActBytes >> 4));
+                    const uint32_t a_tmem = tmem_base + C::COL_A + 32 * t;
+                    const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(s * (C::ACT >> 4));
                     const uint64_t adesc = adesc0 + static_cast<uint64_t>(s * (kTmW8Bytes >> 4));
                     if constexpr (W8) umma_i8_ss_step(d_tmem, adesc, bdesc, idesc, kt);
                     else umma_i8_ts_step(d_tmem, a_tmem, bdesc, idesc, kt);
@@ -389,18 +406,18 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                                kDevErrTimeoutConsumer))
                     break;
                 tcgen05_fence_after();
-                tmem_st_32x32b_x32(tmem_base + lane_base + kTmColA + 32 * t, a);
+                tmem_st_32x32b_x32(tmem_base + lane_base + C::COL_A + 32 * t, a);
                 if (A_INT4) {
                     // widen the packed activation codes of this stage (even/odd
                     // K order, like the weights) into the swizzled int8 B tile: 192 rows x 8 chunks of 16 codes, 12
                     // chunks per thread of this K-step parity (the B tile's last
                     // readers, the MMAs of 4 stages ago, completed before the
                     // producer refilled the stage)
-                    const uint8_t* ap = sActP + s * kTmActPBytes;
-                    uint8_t* ab = sAct + s * kTmActBytes;
+                    const uint8_t* ap = sActP + s * C::ACTP;
+                    uint8_t* ab = sAct + s * C::ACT;
                     const int tid = q * 32 + lane;
     #pragma unroll 4
-                    for (int i = 0; i < kTmBN * 8 / 128; ++i) {
+                    for (int i = 0; i < kBN * 8 / 128; ++i) {
                         const int c = tid + 128 * i;
                         const int rr = c >> 3, k = c & 7;
                         const uint2 pk = *reinterpret_cast<const uint2*>(ap + rr * 64 + 8 * k);
@@ -421,7 +438,7 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
         // ------------------------------------------------ epilogue (warps 10-17)
         const int e = warp - 10;                // 0..7
         const int q = warp & 3;                 // TMEM lane quarter
-        const int half = e >> 2;                // tokens [96 half, 96 half + 96)
+        const int half = e >> 2;                // tokens [BN/2 half, BN/2 (half + 1))
         const int r = q * 32 + lane;            // weight row in the tile = output column
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const bool leader = (e == 0 && lane == 0);
@@ -433,12 +450,20 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             const __nv_bfloat16* __restrict__ bias = grp.bias[ta.g];
             void* __restrict__ out = grp.out[ta.g];
             const int n = n0 + r;
-            const int buf = i & 1;
+            const int buf = C::NBUF == 2 ? (i & 1) : 0;
+            const uint32_t fph = C::NBUF == 2 ? ((i >> 1) & 1) : (i & 1);
+            // the tile's token scales into shared memory (0 beyond M), read
+            // while the MMAs run: the accumulator is then drained without global
+            // loads (the previous tile's readers passed the copy-out barrier)
+            if (!OUT_I32)
+                for (int t = e * 32 + lane; t < kBN; t += 256)
+                    sTok[t] = (m0 + t < M) ? __ldg(tok_scale + m0 + t) : 0.0f;
             // one thread waits for the accumulator; the named barrier hands the
             // decision to all 8 warps at once (and orders the previous tile's
-            // copy-out before this tile's staging writes)
+            // copy-out before this tile's staging writes, the token scales
+            // before their reads)
             if (leader) {
-                const bool ok = mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1, abort_flag,
+                const bool ok = mbar_wait_bounded(&acc_full[buf], fph, abort_flag,
                                                   wait_ns, kDevErrTimeoutEpilogue);
                 *epi_go = ok ? 1u : 0u;
             }
@@ -452,49 +477,69 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             constexpr int kShift = A_INT4 ? 8 : (W8 ? 0 : 4);
             const float sr16 = (row_ok && !OUT_I32) ? ld_scale<S16>(row_scale, n) * kUnscale : 0.0f;
             const float b = (row_ok && !OUT_I32 && bias != nullptr) ? __bfloat162float(bias[n]) : 0.0f;
-#pragma unroll 1
-            for (int c0 = half * (kTmBN / 2); c0 < (half + 1) * (kTmBN / 2); c0 += 32) {
-                if (m0 + c0 >= M) break;   // warp-uniform
-                uint32_t acc[32];
-                tmem_ld_32x32b_x32(tmem_base + lane_base + kTmColD + buf * kTmBN + c0, acc);
-                tmem_ld_wait();
+            // the accumulator buffer is handed back (acc_empty) once this warp has
+            // read its last chunk: with one buffer the next tile's MMAs wait for it
+            bool released = false;
+            // one chunk of 32 tokens from registers: int32 sums, or scaled to
+            // bf16 into the staging tile (row = token, 256 bytes; column = this
+            // thread's row), two tokens at a time on packed fp32 pairs: (acc
+            // s_tok) s_row + b, each element rounded as the scalar multiply and
+            // fma would (rows beyond M are written, never copied out)
+            auto emit = [&](int c0, const uint32_t (&acc)[32]) {
                 const int mb = m0 + c0;
-                const int mcount = min(32, M - mb);
                 if (OUT_I32) {
-                    if (!row_ok) continue;
+                    if (!row_ok) return;
+                    const int mcount = min(32, M - mb);
                     int32_t* o = static_cast<int32_t*>(out) + static_cast<size_t>(mb) * N + n;
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
                         if (j < mcount) o[static_cast<size_t>(j) * N] = static_cast<int32_t>(acc[j]) >> kShift;
                 } else {
-                    float st[32];
-                    if (mcount == 32) {
+                    const float2* st2 = reinterpret_cast<const float2*>(sTok + c0);
+                    const uint32_t dst = smem_u32(sOut + c0 * (kTmBM * 2) + r * 2);
+                    const uint64_t sr2 = f2_pack(sr16, sr16), b2 = f2_pack(b, b);
 #pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            const float4 v = __ldg(reinterpret_cast<const float4*>(tok_scale + mb + j));
-                            st[j] = v.x; st[j + 1] = v.y; st[j + 2] = v.z; st[j + 3] = v.w;
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) st[j] = (j < mcount) ? __ldg(tok_scale + mb + j) : 0.0f;
-                    }
-                    // staging tile row = token (256 bytes), column = this thread's row
-                    uint8_t* dst = sOut + c0 * (kTmBM * 2) + r * 2;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float v =
-                            static_cast<float>(static_cast<int32_t>(acc[j])) * st[j] * sr16 + b;
-                        const __nv_bfloat16 h = __float2bfloat16_rn(v);
-                        asm volatile("st.shared.b16 [%0], %1;" ::"r"(smem_u32(dst + j * (kTmBM * 2))),
-                                     "h"(*reinterpret_cast<const unsigned short*>(&h))
-                                     : "memory");
+                    for (int j = 0; j < 32; j += 2) {
+                        const uint64_t a2 = f2_pack(static_cast<float>(static_cast<int32_t>(acc[j])),
+                                                    static_cast<float>(static_cast<int32_t>(acc[j + 1])));
+                        const float2 tj = st2[j / 2];
+                        const uint32_t h2 = f2_to_bf16x2(f2_fma(f2_mul(a2, f2_pack(tj.x, tj.y)), sr2, b2));
+                        asm volatile(
+                            "{\n\t.reg .b16 l, h;\n\t"
+                            "mov.b32 {l, h}, %2;\n\t"
+                            "st.shared.b16 [%0], l;\n\t"
+                            "st.shared.b16 [%1], h;\n\t}" ::"r"(dst + j * (kTmBM * 2)),
+                            "r"(dst + (j + 1) * (kTmBM * 2)), "r"(h2)
+                            : "memory");
                     }
                 }
+            };
+            // with one accumulator buffer two chunks per TMEM read: the next
+            // tile's MMAs wait for this warp's last read, not for its math
+            constexpr int kStep = C::NBUF == 1 ? 64 : 32;
+            const int cend = (half + 1) * (kBN / 2);
+#pragma unroll 1
+            for (int c0 = half * (kBN / 2); c0 < cend; c0 += kStep) {
+                if (m0 + c0 >= M) break;   // warp-uniform
+                const bool two = kStep == 64 && c0 + 32 < cend && m0 + c0 + 32 < M;   // warp-uniform
+                uint32_t acc0[32], acc1[32];
+                tmem_ld_32x32b_x32(tmem_base + lane_base + kTmColD + buf * kBN + c0, acc0);
+                if (two) tmem_ld_32x32b_x32(tmem_base + lane_base + kTmColD + buf * kBN + c0 + 32, acc1);
+                tmem_ld_wait();
+                if (c0 + kStep >= cend || m0 + c0 + kStep >= M) {   // this warp's last read (warp-uniform)
+                    tcgen05_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&acc_empty[buf]);
+                    released = true;
+                }
+                emit(c0, acc0);
+                if (two) emit(c0 + 32, acc1);
             }
-            // the accumulator buffer is drained: the MMAs may refill it
-            tcgen05_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            if (!released) {   // no chunk of this warp's half lies below M
+                tcgen05_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            }
             if (!OUT_I32) {
                 // the staging tile is complete: the 8 warps copy it out, one
                 // 16-byte piece of a token row per thread and step (coalesced
@@ -503,7 +548,7 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                 const int et = e * 32 + lane;
                 __nv_bfloat16* yb = static_cast<__nv_bfloat16*>(out);
 #pragma unroll 4
-                for (int c = et; c < kTmBN * (kTmBM / 8); c += 256) {
+                for (int c = et; c < kBN * (kTmBM / 8); c += 256) {
                     const int tok = c >> 4, piece = c & 15;
                     if (m0 + tok < M && n0 + piece * 8 < N)
                         *reinterpret_cast<uint4*>(yb + static_cast<size_t>(m0 + tok) * N + n0 + piece * 8) =

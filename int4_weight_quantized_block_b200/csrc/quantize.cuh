@@ -230,36 +230,6 @@ __device__ __forceinline__ void rotate_quantize_rows_to_smem(const __nv_bfloat16
 // long as nothing is subnormal (rows whose absmax(u) is below 2^-100 take the
 // normalised path value by value).
 
-// 64-bit register holding two fp32 values: lo in the low word
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-
-__device__ __forceinline__ void f2_unpack(uint64_t p, float& lo, float& hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
-}
-
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-
-// a * b + c, each element rounded once
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-
 // (a, b) -> (a + b, a - b) for two element pairs at once
 __device__ __forceinline__ void f2_bfly(uint64_t& a, uint64_t& b) {
     const uint64_t s = f2_add(a, b);

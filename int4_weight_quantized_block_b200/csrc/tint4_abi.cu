@@ -232,11 +232,12 @@ tint4_status launch_gemm_tmem(const void* a, const float* st, TmGroups& grp,
                               const uint8_t* const* w, int M, int K, cudaStream_t stream,
                               bool pdl) {
     auto kern = w4a8_tmem_gemm_kernel<OUT_I32, A_INT4, W8, EVOD, S16>;
-    constexpr int smem_bytes = A_INT4 ? kTmSmemBytesA4 : (W8 ? kTmSmemBytesW8 : kTmSmemBytes);
+    using C = TmCfg<A_INT4, W8>;
+    constexpr int smem_bytes = C::SMEM;
     CUtensorMap ta;
-    bool ok = A_INT4 ? make_map_u8(&ta, a, K / 2, M, K / 2, kTmBK / 2, kTmBN, CU_TENSOR_MAP_SWIZZLE_NONE)
-                     : make_map_u8(&ta, a, K, M, K, kTmBK, kTmBN, CU_TENSOR_MAP_SWIZZLE_128B);
-    const int m_tiles = (M + kTmBN - 1) / kTmBN;
+    bool ok = A_INT4 ? make_map_u8(&ta, a, K / 2, M, K / 2, kTmBK / 2, C::BN, CU_TENSOR_MAP_SWIZZLE_NONE)
+                     : make_map_u8(&ta, a, K, M, K, kTmBK, C::BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    const int m_tiles = (M + C::BN - 1) / C::BN;
     int tiles = 0;
     for (int g = 0; g < grp.count; ++g) {
         ok = ok && (W8 ? make_map_u8(&grp.w[g], w[g], K, grp.N[g], K, kTmBK, kTmBM,

@@ -366,12 +366,14 @@ def test_w4a4_gemm_widened(M, N, K):
 
 @pytest.mark.parametrize("bits", [8, 4])
 def test_many_tiles_per_cta(bits):
-    """A mid-size layer (2048 tokens, 8192 weight rows, K 1024: 704 tiles of
-    128 x 192, between 4 and 5 per persistent CTA), every element: each CTA
-    reuses both accumulator buffers and crosses tile boundaries in its rings
-    several times.  int32 sums bit-exact (packed and int8 codes), the fused
-    linear and the GEMM entries against the oracle."""
-    M, N, K, g = 2048, 8192, 1024, 256
+    """A mid-size layer (2000 tokens, 12288 weight rows, K 1024), every
+    element: 768 tiles of 128 x 256 for int8 codes (5 or 6 per persistent CTA,
+    the single accumulator handed back and forth each tile, the last token
+    tile ragged) and 1056 tiles of 128 x 192 for packed codes (7 or 8 per CTA,
+    both accumulator buffers reused); each CTA crosses tile boundaries in its
+    rings several times.  int32 sums bit-exact (packed and int8 codes), the
+    fused linear and the GEMM entries against the oracle."""
+    M, N, K, g = 2000, 12288, 1024, 256
     x = inputs.activations(M, K, seed=1300 + bits)
     W = inputs.weights(N, K, seed=1310)
     wp, sr, qw = oracle.pack_weights(W, g)
