@@ -13,8 +13,8 @@
 // accumulate in fp32.
 //
 // Shape on the tensor core: the weights are the MMA's M side (128 rows = the
-// 128 TMEM lanes), the tokens its N side (192 per tile), as in the int8 GEMM
-// (gemm_tmem.cuh).  Per 64-wide K step the TMA brings one token tile (192
+// 128 TMEM lanes), the tokens its N side (256 per tile), as in the int8 GEMM
+// (gemm_tmem.cuh).  Per 64-wide K step the TMA brings one token tile (256
 // tokens x 64 bf16 = 128-byte rows, 128-byte swizzle: the MMA's B operand) and
 // one packed weight tile (128 rows x 32 bytes).  Each of 128 dequant threads
 // owns one weight row: it reads its 32 packed bytes, forms bf16(128 + q) for
@@ -30,14 +30,18 @@
 // while it works on the current one.
 //
 // Warp roles (18 warps, one persistent CTA per SM, static tile list):
-//   warp 0      TMA producer (4-deep ring of 24 KB token + 4 KB weight stages)
+//   warp 0      TMA producer (4-deep ring of 32 KB token + 4 KB weight stages)
 //   warp 1      TMEM owner; one thread issues tcgen05.mma.kind::f16 (A bf16
-//               from TMEM, B bf16 from shared memory, fp32 D; M 128, N 192, K 16)
+//               from TMEM, B bf16 from shared memory, fp32 D; M 128, N 256, K 16)
 //   warps 2-9   dequant into the 4 TMEM A stages (32 columns each)
-//   warps 10-17 epilogue: tcgen05.ld of one accumulator buffer while the MMAs
-//               fill the other, rounding to bf16 into a [192 tokens][128
-//               columns] staging tile, copied to y in 16-byte row pieces.
-// TMEM columns: accumulators at 0 and 192, A stages at 384 + 32 s.
+//   warps 10-17 epilogue: tcgen05.ld of the accumulator two 32-token chunks
+//               at a time, handed back to the MMAs after the last read,
+//               rounding to bf16 into a [256 tokens][128 columns] staging
+//               tile, copied to y in 16-byte row pieces.
+// TMEM columns: one accumulator at 0 (256 columns), A stages at 256 + 32 s.
+// (256 tokens per tile rather than 192 with two accumulators: the dequant
+// work of a step, the kernel's critical path, then serves a third more
+// tokens.)
 #pragma once
 
 #include "ptx.cuh"
@@ -45,18 +49,19 @@
 namespace tint4 {
 
 constexpr int kWgBM = 128;       // weight rows per tile (UMMA M, TMEM lanes)
-constexpr int kWgBN = 192;       // tokens per tile (UMMA N)
+constexpr int kWgBN = 256;       // tokens per tile (UMMA N)
 constexpr int kWgBK = 64;        // K values per stage (bf16: 128-byte rows)
 constexpr int kWgStages = 4;     // shared-memory stages = TMEM A stages
 constexpr int kWgThreads = 576;  // 18 warps
 constexpr int kWgGroup = 128;    // quantization group along K
-constexpr int kWgActBytes = kWgBN * kWgBK * 2;        // 24 KB token tile per stage
+constexpr int kWgActBytes = kWgBN * kWgBK * 2;        // 32 KB token tile per stage
 constexpr int kWgWBytes = kWgBM * kWgBK / 2;          // 4 KB packed weights per stage
-constexpr int kWgOutBytes = kWgBN * kWgBM * 2;        // 48 KB bf16 staging tile
+constexpr int kWgOutBytes = kWgBN * kWgBM * 2;        // 64 KB bf16 staging tile
 constexpr int kWgSmemBytes = kWgStages * (kWgActBytes + kWgWBytes) + kWgOutBytes + 256 + 1024;
-constexpr uint32_t kWgColD = 0;                       // accumulator buffer b at b * kWgBN
-constexpr uint32_t kWgColA = 2 * kWgBN;               // A stage s at kWgColA + 32 s
+constexpr uint32_t kWgColD = 0;                       // the accumulator
+constexpr uint32_t kWgColA = kWgBN;                   // A stage s at kWgColA + 32 s
 static_assert(kWgColA + 32 * kWgStages <= 512, "TMEM budget");
+static_assert(kWgSmemBytes <= 227 * 1024, "shared memory budget");
 static_assert(kWgActBytes % 1024 == 0 && kWgWBytes % 1024 == 0, "stage alignment");
 static_assert(kWgGroup == 2 * kWgBK, "a group is two K steps");
 
@@ -138,8 +143,8 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
     uint64_t* act_full = reinterpret_cast<uint64_t*>(sOut + kWgOutBytes);
     uint64_t* a_full = act_full + kWgStages;       // TMEM A stage written (one arrival per warp)
     uint64_t* empty = a_full + kWgStages;          // stage consumed by the MMAs (commit)
-    uint64_t* acc_full = empty + kWgStages;        // [2] accumulator ready (commit)
-    uint64_t* acc_empty = acc_full + 2;            // [2] accumulator drained (8 warp arrivals)
+    uint64_t* acc_full = empty + kWgStages;        // accumulator ready (commit)
+    uint64_t* acc_empty = acc_full + 2;            // accumulator read (8 warp arrivals)
     uint64_t* final_bar = acc_empty + 2;           // all MMAs done (teardown)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
@@ -225,8 +230,8 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
             uint32_t ph = 0u;
             bool ok = true;
             for (int i = 0; i < my_tiles && ok; ++i) {
-                const int buf = i & 1;
-                const uint32_t aph = (i >> 1) & 1;
+                const int buf = 0;
+                const uint32_t aph = i & 1;
                 if (!mbar_wait_bounded(&acc_empty[buf], aph ^ 1, abort_flag, wait_ns,
                                        kDevErrTimeoutConsumer)) {
                     ok = false;
@@ -331,34 +336,58 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
             const int tile = blockIdx.x + i * gridDim.x;
             const int m0 = (tile % m_tiles) * kWgBN;
             const int n0 = (tile / m_tiles) * kWgBM;
-            const int buf = i & 1;
             if (leader) {
-                const bool ok = mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1, abort_flag,
+                const bool ok = mbar_wait_bounded(&acc_full[0], i & 1, abort_flag,
                                                   wait_ns, kDevErrTimeoutEpilogue);
                 *epi_go = ok ? 1u : 0u;
             }
             named_barrier_sync(1, 256);
             if (*epi_go == 0u) break;
             tcgen05_fence_after();
-#pragma unroll 1
-            for (int cc = half * (kWgBN / 2); cc < (half + 1) * (kWgBN / 2); cc += 32) {
-                if (m0 + cc >= M) break;   // warp-uniform
-                uint32_t acc[32];
-                tmem_ld_32x32b_x32(tmem_base + lane_base + kWgColD + buf * kWgBN + cc, acc);
-                tmem_ld_wait();
-                // staging tile row = token (256 bytes), column = this thread's row
-                uint8_t* dst = sOut + cc * (kWgBM * 2) + r * 2;
+            // 32 tokens from registers: fp32 sums rounded to bf16 (two at a time)
+            // into the staging tile (row = token, 256 bytes; column = this
+            // thread's row)
+            auto emit = [&](int cc, const uint32_t (&acc)[32]) {
+                const uint32_t dst = smem_u32(sOut + cc * (kWgBM * 2) + r * 2);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(acc[j]));
-                    asm volatile("st.shared.b16 [%0], %1;" ::"r"(smem_u32(dst + j * (kWgBM * 2))),
-                                 "h"(*reinterpret_cast<const unsigned short*>(&h))
-                                 : "memory");
+                for (int j = 0; j < 32; j += 2) {
+                    const uint32_t h2 =
+                        f2_to_bf16x2(f2_pack(__uint_as_float(acc[j]), __uint_as_float(acc[j + 1])));
+                    asm volatile(
+                        "{\n\t.reg .b16 l, h;\n\t"
+                        "mov.b32 {l, h}, %2;\n\t"
+                        "st.shared.b16 [%0], l;\n\t"
+                        "st.shared.b16 [%1], h;\n\t}" ::"r"(dst + j * (kWgBM * 2)),
+                        "r"(dst + (j + 1) * (kWgBM * 2)), "r"(h2)
+                        : "memory");
                 }
+            };
+            // two chunks per TMEM read; the accumulator goes back to the MMAs
+            // after this warp's last read, before the math on it
+            bool released = false;
+            const int cend = (half + 1) * (kWgBN / 2);
+#pragma unroll 1
+            for (int cc = half * (kWgBN / 2); cc < cend; cc += 64) {
+                if (m0 + cc >= M) break;   // warp-uniform
+                const bool two = cc + 32 < cend && m0 + cc + 32 < M;   // warp-uniform
+                uint32_t acc0[32], acc1[32];
+                tmem_ld_32x32b_x32(tmem_base + lane_base + kWgColD + cc, acc0);
+                if (two) tmem_ld_32x32b_x32(tmem_base + lane_base + kWgColD + cc + 32, acc1);
+                tmem_ld_wait();
+                if (cc + 64 >= cend || m0 + cc + 64 >= M) {   // warp-uniform
+                    tcgen05_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&acc_empty[0]);
+                    released = true;
+                }
+                emit(cc, acc0);
+                if (two) emit(cc + 32, acc1);
             }
-            tcgen05_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            if (!released) {   // no token of this warp's half below M
+                tcgen05_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[0]);
+            }
             named_barrier_sync(1, 256);
             const int et = e * 32 + lane;
 #pragma unroll 4
