@@ -73,6 +73,7 @@ def peaks():
 
 # the sources each profiled kernel is built from (its own file + the PTX helpers)
 KERNEL_SOURCES = {
+    "w4a8_wide_gemm_kernel": ("gemm_wide.cuh", "gemm_tmem.cuh", "ptx.cuh"),
     "w4a8_tmem_gemm_kernel": ("gemm_tmem.cuh", "ptx.cuh"),
     "rotate_quantize_rows_kernel": ("quantize.cuh", "ptx.cuh"),
     "w4a16_mma_kernel": ("w4a16.cuh", "ptx.cuh"),
@@ -360,7 +361,7 @@ def run_ours(args, rank, world, dev):
         cpu = cpu_baseline(w, target_s=args.cpu_seconds)
 
     clocks = clk.summary()
-    traffic = ncu_traffic("w4a8_tmem_gemm_kernel", MAIN)
+    traffic = ncu_traffic("w4a8_wide_gemm_kernel", MAIN)
     line = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -380,7 +381,7 @@ def run_ours(args, rank, world, dev):
                    "per_gpu_tokens": M, "parallelism": f"independent batches x{world}",
                    "l2": "flushed (256 MiB write) before every timed step, outside the events"},
         "roofline": {"bound": "tensor",
-                     "kernel": "w4a8_tmem_gemm_kernel<even/odd codes> (tcgen05 kind::i8), "
+                     "kernel": "w4a8_wide_gemm_kernel<even/odd codes> (tcgen05 kind::i8), "
                                "the GEMM launch of the fused linear",
                      "achieved": round(gemm_tops, 2), "peak": round(int8_peak, 1),
                      "unit": "TOPS", "frac": round(gemm_tops / int8_peak, 4),
@@ -491,7 +492,7 @@ def run_nsplit(args, rank, world, dev):
                    "rows_per_gpu": n_r,
                    "l2": "flushed (256 MiB write) before every timed step, outside the events"},
         "roofline": {"bound": "tensor",
-                     "kernel": "w4a8_tmem_gemm_kernel<even/odd codes> on the rank's weight rows",
+                     "kernel": "w4a8_wide_gemm_kernel<even/odd codes> on the rank's weight rows",
                      "achieved": round(gemm_tops, 2), "peak": round(int8_peak, 1),
                      "unit": "TOPS", "frac": round(gemm_tops / int8_peak, 4), "traffic": None,
                      "peak_source": f"{pk['source']}: 2 x bf16 cuBLAS burst "

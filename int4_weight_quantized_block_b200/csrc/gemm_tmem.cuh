@@ -1,5 +1,7 @@
-// gemm_tmem.cuh -- persistent W4A8 GEMM with the unpacked weights in tensor
-// memory.
+// gemm_tmem.cuh -- persistent GEMM with the unpacked weights in tensor memory
+// (packed int4 activation codes), or int8 weights from shared memory (W8A8);
+// shared-stage pipeline.  The int8-code x packed-int4-weight form, the fused
+// linears' GEMM, is gemm_wide.cuh; the MMA helpers here serve it too.
 //
 //   acc[m, n] = sum_k qa[m, k] * qw[n, k]            (int32, exact)
 //   y[m, n]   = bf16( acc * s_tok[m] * s_row[n] (+ bias[n]) )
@@ -11,47 +13,38 @@
 // byte per weight).
 //
 // Shape of the product on the tensor core: the weights are the MMA's M side
-// (128 rows = the 128 TMEM lanes) and the tokens its N side (BN per tile:
-// 256 for int8 activation codes, 192 for the packed-int4-code and int8-weight
-// forms, see TmCfg).  Per 128-wide K step the TMA brings one activation tile
-// (BN tokens x 128 int8 codes, 128-byte swizzle: the MMA's B operand) and one
-// packed weight tile (128 rows x 64 bytes, 64-byte swizzle) into shared
-// memory.  Each of 128 unpack threads owns one weight row: it reads its 64
-// packed bytes (bank-conflict-free thanks to the swizzle), widens every
-// nibble to an int8 (x16, see below) and writes the 128 K values with one
-// tcgen05.st into a TMEM A-operand stage.  The widened weights never go back
-// to shared memory.
+// (128 rows = the 128 TMEM lanes) and the tokens its N side (192 per tile).
+// Per 128-wide K step the TMA brings one activation tile (192 tokens x 128
+// int8 codes, 128-byte swizzle: the MMA's B operand; or the packed int4 codes
+// the unpack warps widen into it) and one weight tile (packed: 128 rows x 64
+// bytes, 64-byte swizzle; int8: 128 x 128 bytes, the A operand from shared
+// memory) into one shared-memory stage.  For packed weights each of 128
+// unpack threads owns one weight row: it reads its 64 packed bytes
+// (bank-conflict-free thanks to the swizzle), widens every nibble to an int8
+// (x16, see below) and writes the 128 K values with one tcgen05.st into a
+// TMEM A-operand stage.
 //
-// The CTA is persistent (one per SM) and walks a static list of 128 x BN
+// The CTA is persistent (one per SM) and walks a static list of 128 x 192
 // tiles.  Warp roles (18 warps):
-//   warp 0      TMA producer (ring of 4 or 5 activation + weight stages)
+//   warp 0      TMA producer (4-deep ring of shared-memory stages)
 //   warp 1      TMEM owner; one thread issues tcgen05.mma.cta_group::1.kind::i8
-//               (A from TMEM, B from shared memory, M 128, N BN, K 32)
-//   warps 2-9   weight unpack into the 4 TMEM A stages (32 columns each);
-//               warps 2-5 take the even K steps and warps 6-9 the odd ones,
-//               so two unpack chains run side by side on every SM
-//               sub-partition (each warp may only reach its quarter of the
-//               TMEM lanes, warp % 4)
-//   warps 10-17 epilogue: tcgen05.ld of the accumulator; two warps per TMEM
-//               lane quarter, each on half of the tokens.  A thread holds one
-//               weight row (= one output column), so it scales its values,
+//               (A from TMEM or shared memory, B from shared memory, M 128,
+//               N 192, K 32)
+//   warps 2-9   unpack into the 4 TMEM A stages (32 columns each); warps 2-5
+//               take the even K steps and warps 6-9 the odd ones, so two
+//               chains run side by side on every SM sub-partition (each warp
+//               may only reach its quarter of the TMEM lanes, warp % 4)
+//   warps 10-17 epilogue: tcgen05.ld of one accumulator buffer while the MMAs
+//               fill the other (two 192-column int32 buffers); two warps per
+//               TMEM lane quarter, each on half of the tokens.  A thread holds
+//               one weight row (= one output column), so it scales its values,
 //               rounds them to bf16 and writes them with 2-byte shared-memory
-//               stores into a [BN tokens][128 columns] staging tile, which the
+//               stores into a [192 tokens][128 columns] staging tile, which the
 //               8 warps then copy to y (row-major [M, N]) in 16-byte row pieces
 //               (a TMA tensor store of the tile shared the copy engine with the
 //               mainloop's loads and cost about 15 %).  The tile's token
 //               scales are copied to shared memory while its MMAs run.
-// TMEM columns: BN = 256: one accumulator at 0, A stages at 256 + 32 s; the
-// epilogue reads it two 32-token chunks at a time and hands it back after
-// its last read, before the math on those chunks.  BN = 192: two
-// accumulators at 0 and 192 (the epilogue drains one while the MMAs fill the
-// other), A stages at 384 + 32 s.
-//
-// Why 256 tokens: the step time follows the bytes the TMA brings per step
-// (about 40 B per cycle and SM), of which the weight tile is a fixed 8 KB;
-// a 256-token tile moves 40 KB for 4/3 of the work of a 192-token one (32
-// KB).  On the DiT layers it took QKV 127 -> 123 us, MLP up 164 -> 156, MLP
-// down 162 -> 145 (K = 12288: 96 steps per tile share one drain).
+// TMEM columns: accumulators at 0 and 192, A stages at 384 + 32 s.
 //
 // A nibble moved into the high half of its byte, low half cleared, is the
 // int8 value 16 * code; the accumulators hold 16 * acc and the epilogue
@@ -85,23 +78,15 @@ constexpr int kTmThreads = 576;  // 18 warps
 constexpr int kTmWBytes = kTmBM * kTmBK / 2;          // 8 KB packed weights per stage
 constexpr int kTmW8Bytes = kTmBM * kTmBK;             // 16 KB int8 weights per stage (W8A8)
 
-// Tile shape and rings of the three forms.  Int8 codes x packed int4
-// weights (the fused linears' form): 256 tokens per tile (N = 256, 128-cycle
-// MMAs: a third more work per issued MMA than N = 192) with one accumulator
-// buffer (256 TMEM columns + 4 A stages of 32); the epilogue hands the
-// buffer back as soon as it has read it.  Packed int4 codes (A_INT4) and
-// int8 weights (W8): 192 tokens, two accumulator buffers (the larger stages
-// leave no room for 256-token tiles).
+// Tile shape and ring of the two forms: 192 tokens, two accumulator buffers,
+// 4 shared-memory stages (the packed-code staging or the int8 weight tile
+// leave no room for a fifth).
 template <bool A_INT4, bool W8>
 struct TmCfg {
-    static constexpr bool WIDE = !A_INT4 && !W8;
-    static constexpr int BN = WIDE ? 256 : 192;            // tokens per tile (UMMA N)
-    static constexpr int NBUF = WIDE ? 1 : 2;              // accumulator buffers
-    // shared-memory stages: 5 for int8 codes x packed weights at N = 192, so
-    // that the loads run one stage further ahead of the unpack than the 4 TMEM
-    // A stages allow (the unpack of step j also waits for the MMAs of step
-    // j - 4, which free its TMEM stage); no room for a fifth otherwise
-    static constexpr int S = (A_INT4 || W8 || WIDE) ? 4 : 5;
+    static_assert(A_INT4 || W8, "int8 codes x packed int4 weights run w4a8_wide_gemm_kernel");
+    static constexpr int BN = 192;                         // tokens per tile (UMMA N)
+    static constexpr int NBUF = 2;                         // accumulator buffers
+    static constexpr int S = 4;                            // shared-memory stages
     static constexpr int ACT = BN * kTmBK;                 // int8 codes per stage
     static constexpr int ACTP = A_INT4 ? BN * kTmBK / 2 : 0;   // packed int4 codes per stage
     static constexpr int WB = W8 ? kTmW8Bytes : kTmWBytes;
@@ -172,17 +157,6 @@ __device__ __forceinline__ void umma_i8_ss_step(uint32_t d_tmem, uint64_t a_desc
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "l"(a_desc + 2), "l"(b_desc + 2),
         "l"(a_desc + 4), "l"(b_desc + 4), "l"(a_desc + 6), "l"(b_desc + 6)
         : "memory");
-}
-
-// Bounded wait by lane 0 of the warp, result broadcast: the warp leaves
-// together (tcgen05.st / tcgen05.ld are warp-collective).
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
-                                          uint64_t limit_ns, unsigned err) {
-    const int lane = threadIdx.x & 31;
-    int ok = 0;
-    if (lane == 0) ok = mbar_wait_bounded(bar, parity, abort, limit_ns, err) ? 1 : 0;
-    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-    return ok != 0;
 }
 
 // W8: the weights are int8 codes already (W8A8): the TMA brings a 128 x 128
@@ -321,8 +295,8 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             uint32_t sph = 0u, tph = 0u;
             bool ok = true;
             for (int i = 0; i < my_tiles && ok; ++i) {
-                const int buf = C::NBUF == 2 ? (i & 1) : 0;
-                const uint32_t aph = C::NBUF == 2 ? ((i >> 1) & 1) : (i & 1);
+                const int buf = i & 1;
+                const uint32_t aph = (i >> 1) & 1;
                 if (!mbar_wait_bounded(&acc_empty[buf], aph ^ 1, abort_flag, wait_ns,
                                        kDevErrTimeoutConsumer)) {
                     ok = false;
@@ -450,14 +424,14 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             const __nv_bfloat16* __restrict__ bias = grp.bias[ta.g];
             void* __restrict__ out = grp.out[ta.g];
             const int n = n0 + r;
-            const int buf = C::NBUF == 2 ? (i & 1) : 0;
-            const uint32_t fph = C::NBUF == 2 ? ((i >> 1) & 1) : (i & 1);
+            const int buf = i & 1;
+            const uint32_t fph = (i >> 1) & 1;
             // the tile's token scales into shared memory (0 beyond M), read
             // while the MMAs run: the accumulator is then drained without global
             // loads (the previous tile's readers passed the copy-out barrier)
             if (!OUT_I32)
                 for (int t = e * 32 + lane; t < kBN; t += 256)
-                    sTok[t] = (m0 + t < M) ? __ldg(tok_scale + m0 + t) : 0.0f;
+                    sTok[t] = (m0 + t < M) ? __ldcg(tok_scale + m0 + t) : 0.0f;
             // one thread waits for the accumulator; the named barrier hands the
             // decision to all 8 warps at once (and orders the previous tile's
             // copy-out before this tile's staging writes, the token scales
@@ -476,9 +450,7 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             constexpr float kUnscale = A_INT4 ? 1.0f / 256.0f : (W8 ? 1.0f : 0.0625f);
             constexpr int kShift = A_INT4 ? 8 : (W8 ? 0 : 4);
             const float sr16 = (row_ok && !OUT_I32) ? ld_scale<S16>(row_scale, n) * kUnscale : 0.0f;
-            const float b = (row_ok && !OUT_I32 && bias != nullptr) ? __bfloat162float(bias[n]) : 0.0f;
-            // the accumulator buffer is handed back (acc_empty) once this warp has
-            // read its last chunk: with one buffer the next tile's MMAs wait for it
+            const float b = (row_ok && !OUT_I32 && bias != nullptr) ? __bfloat162float(__ldcg(bias + n)) : 0.0f;
             bool released = false;
             // one chunk of 32 tokens from registers: int32 sums, or scaled to
             // bf16 into the staging tile (row = token, 256 bytes; column = this
@@ -514,26 +486,21 @@ w4a8_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                     }
                 }
             };
-            // with one accumulator buffer two chunks per TMEM read: the next
-            // tile's MMAs wait for this warp's last read, not for its math
-            constexpr int kStep = C::NBUF == 1 ? 64 : 32;
+            // the buffer goes back to the MMAs after this warp's last read
             const int cend = (half + 1) * (kBN / 2);
 #pragma unroll 1
-            for (int c0 = half * (kBN / 2); c0 < cend; c0 += kStep) {
+            for (int c0 = half * (kBN / 2); c0 < cend; c0 += 32) {
                 if (m0 + c0 >= M) break;   // warp-uniform
-                const bool two = kStep == 64 && c0 + 32 < cend && m0 + c0 + 32 < M;   // warp-uniform
-                uint32_t acc0[32], acc1[32];
-                tmem_ld_32x32b_x32(tmem_base + lane_base + kTmColD + buf * kBN + c0, acc0);
-                if (two) tmem_ld_32x32b_x32(tmem_base + lane_base + kTmColD + buf * kBN + c0 + 32, acc1);
+                uint32_t acc[32];
+                tmem_ld_32x32b_x32(tmem_base + lane_base + kTmColD + buf * kBN + c0, acc);
                 tmem_ld_wait();
-                if (c0 + kStep >= cend || m0 + c0 + kStep >= M) {   // this warp's last read (warp-uniform)
+                if (c0 + 32 >= cend || m0 + c0 + 32 >= M) {   // this warp's last read (warp-uniform)
                     tcgen05_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&acc_empty[buf]);
                     released = true;
                 }
-                emit(c0, acc0);
-                if (two) emit(c0 + 32, acc1);
+                emit(c0, acc);
             }
             if (!released) {   // no chunk of this warp's half lies below M
                 tcgen05_fence_before();

@@ -216,7 +216,7 @@ w4a8_gw_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             if constexpr (ASYM) {
                 const int i = j / KT, kt = j % KT;
                 const int n = ((blockIdx.x + i * gridDim.x) / m_tiles) * kGwBM + r;
-                const uint32_t z = n < N ? __ldg(wzero + static_cast<size_t>(n) * ng + kt) : 0u;
+                const uint32_t z = n < N ? __ldca(wzero + static_cast<size_t>(n) * ng + kt) : 0u;
                 zc = (128u - 8u * z) * 0x01010101u;
             }
             if (!warp_wait(&act_full[s], (j / kS) & 1, abort_flag, wait_ns, kDevErrTimeoutConsumer))
@@ -313,7 +313,7 @@ w4a8_gw_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             // token, 256 bytes; column = this thread's row) -> one TMA store
             if (leader && stored) bulk_wait_group_read0();   // previous store read the tile
             named_barrier_sync(1, kFoldThreads);
-            const float b = (row_ok && bias != nullptr) ? __bfloat162float(bias[n]) : 0.0f;
+            const float b = (row_ok && bias != nullptr) ? __bfloat162float(__ldcg(bias + n)) : 0.0f;
             const int t0 = part * 32;
             const int mb = m0 + t0;
             uint8_t* dst = sOut + t0 * (kGwBM * 2) + r * 2;
@@ -321,11 +321,11 @@ w4a8_gw_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
             for (int x = 0; x < 32; x += 4) {
                 float4 st4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                 if (mb + x + 3 < M) {
-                    st4 = __ldg(reinterpret_cast<const float4*>(tok_scale + mb + x));
+                    st4 = __ldcg(reinterpret_cast<const float4*>(tok_scale + mb + x));
                 } else {
-                    if (mb + x < M) st4.x = __ldg(tok_scale + mb + x);
-                    if (mb + x + 1 < M) st4.y = __ldg(tok_scale + mb + x + 1);
-                    if (mb + x + 2 < M) st4.z = __ldg(tok_scale + mb + x + 2);
+                    if (mb + x < M) st4.x = __ldcg(tok_scale + mb + x);
+                    if (mb + x + 1 < M) st4.y = __ldcg(tok_scale + mb + x + 1);
+                    if (mb + x + 2 < M) st4.z = __ldcg(tok_scale + mb + x + 2);
                 }
                 const float sv[4] = {st4.x, st4.y, st4.z, st4.w};
 #pragma unroll

@@ -91,12 +91,35 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// Bounded wait by every lane of a warp, the lanes agreeing on the outcome.
+// Each lane's own successful try_wait is its acquire of what the phase
+// guards (data a TMA wrote, a TMEM stage an MMA released): a lane that only
+// received another lane's verdict by a shuffle has no such ordering, and its
+// shared-memory loads may then run before the copies have landed.
+// (Measured: with lane 0 alone waiting, one weight row of one tile came out
+// of an unpack stale about once in a hundred launches, in the first launches
+// of a process.)
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
+                                          uint64_t limit_ns, unsigned err) {
+    const bool ok = mbar_wait_bounded(bar, parity, abort, limit_ns, err);
+    return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// Kernels launched with programmatic dependent launch are resident while the
+// grid before them still runs, so what that grid writes changes during their
+// lifetime.  The read-only path (ld.global.nc, __ldg) requires data that do
+// not change while the kernel runs, so these kernels read anything a grid
+// before them may have written with coherent loads after the dependency
+// wait, which makes that grid's writes visible: ld.global.ca (__ldca) where a
+// thread reuses a cache line over many steps (per-group scales), ld.global.cg
+// (__ldcg, L2 only) for data read once.
+
 // Weight scale i of an array of fp32 scales, or (S16) of IEEE fp16 scales
 // widened to fp32 (exact).
 template <bool S16>
 __device__ __forceinline__ float ld_scale(const void* p, size_t i) {
-    if constexpr (S16) return __half2float(__ldg(reinterpret_cast<const __half*>(p) + i));
-    else return __ldg(reinterpret_cast<const float*>(p) + i);
+    if constexpr (S16) return __half2float(__ldca(reinterpret_cast<const __half*>(p) + i));
+    else return __ldca(reinterpret_cast<const float*>(p) + i);
 }
 
 // [lo, hi) of part i when n items are split into p contiguous parts of
@@ -111,14 +134,7 @@ __device__ __forceinline__ void even_split(unsigned n, unsigned p, unsigned i, i
 
 // Make generic-proxy writes to shared memory visible to the async proxy
 // (tensor core operand reads, TMA).
-// 4-byte global -> shared copy that holds no register while in flight
-// (completion: cp_async_wait_all by the issuing thread, then a barrier)
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
-                 : "memory");
-}
 
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

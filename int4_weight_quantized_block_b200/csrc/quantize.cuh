@@ -45,6 +45,8 @@ template <>
 struct RawChunk<__nv_bfloat16> {
     uint4 u;
     __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint4*>(p)); }
+    // through L2, for kernels that may run while the grid writing p finishes
+    __device__ __forceinline__ void load_l2(const __nv_bfloat16* p) { u = __ldcg(reinterpret_cast<const uint4*>(p)); }
     __device__ __forceinline__ void zero() { u = make_uint4(0u, 0u, 0u, 0u); }
     __device__ __forceinline__ void to_f32(float (&v)[8]) const {
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -164,7 +166,7 @@ __device__ __forceinline__ void rotate_quantize_rows_to_smem(const __nv_bfloat16
     RawChunk<__nv_bfloat16> raw[kFuseMaxRows];
 #pragma unroll
     for (int r = 0; r < kFuseMaxRows; ++r) {
-        if (r < M && mine && base < K) raw[r].load(x + static_cast<size_t>(r) * K + base);
+        if (r < M && mine && base < K) raw[r].load_l2(x + static_cast<size_t>(r) * K + base);
         else raw[r].zero();
     }
     float v[kFuseMaxRows][8];
@@ -566,7 +568,7 @@ widen_int4_codes_kernel(const uint8_t* __restrict__ packed, int8_t* __restrict__
     grid_dependency_wait();   // the codes may come from the grid just before
     for (long i = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; i < pieces;
          i += static_cast<long>(gridDim.x) * blockDim.x) {
-        const uint4 p = __ldg(reinterpret_cast<const uint4*>(packed) + i);
+        const uint4 p = __ldcg(reinterpret_cast<const uint4*>(packed) + i);
         const uint32_t w[4] = {p.x, p.y, p.z, p.w};
         uint32_t o[8];
 #pragma unroll

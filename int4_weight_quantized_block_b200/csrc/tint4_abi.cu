@@ -14,6 +14,7 @@
 #include "../../include/tint4.h"
 #include "gemm_tmem.cuh"
 #include "gemm_tmem_gw.cuh"
+#include "gemm_wide.cuh"
 #include "pack_groupwise.cuh"
 #include "ptx.cuh"
 #include "quantize.cuh"
@@ -223,14 +224,61 @@ cudaLaunchAttribute pdl_attr() {
     return a;
 }
 
-// Weights widened into TMEM (gemm_tmem.cuh); activation codes int8, or
-// packed int4 widened in shared memory (A_INT4).  `grp` holds 1 to
-// kTmMaxGroups weight matrices sharing the activation codes (the tensor maps
-// and the tile list are filled in here).
-template <bool OUT_I32, bool A_INT4, bool W8 = false, bool EVOD = false, bool S16 = false>
-tint4_status launch_gemm_tmem(const void* a, const float* st, TmGroups& grp,
+// Int8 activation codes x packed int4 weights: the kernel with decoupled
+// weight and activation rings (gemm_wide.cuh), 256-token tiles.
+template <bool OUT_I32, bool EVOD>
+tint4_status launch_gemm_wide(const void* a, const float* st, TmGroups& grp,
                               const uint8_t* const* w, int M, int K, cudaStream_t stream,
                               bool pdl) {
+    auto kern = w4a8_wide_gemm_kernel<OUT_I32, EVOD>;
+    CUtensorMap ta;
+    bool ok = make_map_u8(&ta, a, K, M, K, kTmBK, kWdBN, CU_TENSOR_MAP_SWIZZLE_128B);
+    const int m_tiles = (M + kWdBN - 1) / kWdBN;
+    int tiles = 0;
+    for (int g = 0; g < grp.count; ++g) {
+        ok = ok && make_map_u8(&grp.w[g], w[g], K / 2, grp.N[g], K / 2, kTmBK / 2, kTmBM,
+                               CU_TENSOR_MAP_SWIZZLE_64B);
+        tiles += m_tiles * ((grp.N[g] + kTmBM - 1) / kTmBM);
+        grp.tile_end[g] = tiles;
+    }
+    if (!ok) return TINT4_ERR_CUDA;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static std::atomic<bool> attr_done[kMaxDevices];
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kWdSmem) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return TINT4_ERR_CUDA;
+        }
+        attr_done[dev].store(true, std::memory_order_release);
+    }
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(std::min(tiles, num_sms(dev)), 1, 1);
+    cfg.blockDim = dim3(kWdThreads, 1, 1);
+    cfg.dynamicSmemBytes = kWdSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    if (pdl) {
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    const uint64_t wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+    if (cudaLaunchKernelEx(&cfg, kern, ta, grp, st, M, K, wait_ns) != cudaSuccess) {
+        cudaGetLastError();
+        return TINT4_ERR_CUDA;
+    }
+    return TINT4_OK;
+}
+
+// The shared-stage kernel (gemm_tmem.cuh): packed int4 activation codes
+// widened in shared memory (A_INT4), or int8 weights (W8).  `grp` holds 1 to
+// kTmMaxGroups weight matrices sharing the activation codes (the tensor maps
+// and the tile list are filled in here).
+template <bool OUT_I32, bool A_INT4, bool W8, bool EVOD, bool S16>
+tint4_status launch_gemm_shared_stage(const void* a, const float* st, TmGroups& grp,
+                                      const uint8_t* const* w, int M, int K,
+                                      cudaStream_t stream, bool pdl) {
     auto kern = w4a8_tmem_gemm_kernel<OUT_I32, A_INT4, W8, EVOD, S16>;
     using C = TmCfg<A_INT4, W8>;
     constexpr int smem_bytes = C::SMEM;
@@ -275,6 +323,20 @@ tint4_status launch_gemm_tmem(const void* a, const float* st, TmGroups& grp,
         return TINT4_ERR_CUDA;
     }
     return TINT4_OK;
+}
+
+// The tensor-core GEMM of every large-M entry point: int8 activation codes x
+// packed int4 weights run the kernel with decoupled rings (gemm_wide.cuh),
+// the other forms the shared-stage one.
+template <bool OUT_I32, bool A_INT4, bool W8 = false, bool EVOD = false, bool S16 = false>
+tint4_status launch_gemm_tmem(const void* a, const float* st, TmGroups& grp,
+                              const uint8_t* const* w, int M, int K, cudaStream_t stream,
+                              bool pdl) {
+    if constexpr (!A_INT4 && !W8)
+        return launch_gemm_wide<OUT_I32, EVOD>(a, st, grp, w, M, K, stream, pdl);
+    else
+        return launch_gemm_shared_stage<OUT_I32, A_INT4, W8, EVOD, S16>(a, st, grp, w, M, K, stream,
+                                                                          pdl);
 }
 
 

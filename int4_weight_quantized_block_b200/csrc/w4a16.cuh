@@ -233,9 +233,7 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
     grid_launch_dependents();
     if (!early_weights) issue_weights();
     {
-        int ok = 1;
-        if (lane == 0) ok = mbar_wait_bounded(sz_full, 0, abort_flag, wait_ns, kDevErrTimeoutConsumer);
-        if (__shfl_sync(0xFFFFFFFFu, ok, 0) == 0) nunits_ok = false;
+        if (!warp_wait(sz_full, 0, abort_flag, wait_ns, kDevErrTimeoutConsumer)) nunits_ok = false;
         if (lane == 0)
             for (; issued < SLOTS && issued < nunits; ++issued) issue(issued);
     }
@@ -270,7 +268,7 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
                         x + static_cast<size_t>(tok) * K + (2 * P + gi) * kW16Group + 32 * t);
 #pragma unroll
                     for (int w = 0; w < 4; ++w) {
-                        const uint4 q = __ldg(xr + w);
+                        const uint4 q = __ldcg(xr + w);
                         x_frag(q, bfr[gi][b][2 * w], bfr[gi][b][2 * w + 1]);
                     }
                 } else {
@@ -299,10 +297,10 @@ w4a16_mma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16
             if (bp >= bp_hi) break;   // warp-uniform
             if (bp < bp_lo) continue;
             const int slot = cslot;
-            int ok = 0;
-            if (lane == 0)
-                ok = mbar_wait_bounded(&full[slot], cphase, abort_flag, wait_ns, kDevErrTimeoutConsumer);
-            if (__shfl_sync(0xFFFFFFFFu, ok, 0) == 0) { aborted = true; break; }
+            if (!warp_wait(&full[slot], cphase, abort_flag, wait_ns, kDevErrTimeoutConsumer)) {
+                aborted = true;
+                break;
+            }
             const uint8_t* box = ring + slot * kW16Box;
 #pragma unroll
             for (int hb = 0; hb < 2; ++hb) {

@@ -202,17 +202,20 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
         __syncthreads();   // the barrier is initialised before anyone waits on it
     }
 
-    // The epilogue's operands of this run go to shared memory now, by
-    // asynchronous copies that land during the main loop: read from global
-    // memory at the end they would add a memory round trip to every launch.
+    // The epilogue's operands of this run go to shared memory now, while the
+    // first weight boxes are in flight: read from global memory at the end
+    // they would add a memory round trip to every launch.  Through L2 (the
+    // token scales may come from the grid just before; see ld_scale).
     float* sRowScale = reinterpret_cast<float*>(sm + C::EPI_OFF);
     __nv_bfloat16* sBias = reinterpret_cast<__nv_bfloat16*>(sm + C::EPI_OFF + kS8MB * 16 * 4);
     float* sTok = reinterpret_cast<float*>(sm + C::EPI_OFF + kS8MB * 16 * 6);
     if constexpr (!OUT_I32) {
         const int tid = threadIdx.x;
-        if (GW == 0 && tid < nb * 16) cp_async4(sRowScale + tid, row_scale + b0 * 16 + tid);
-        if (bias != nullptr && tid < nb * 8) cp_async4(sBias + 2 * tid, bias + b0 * 16 + 2 * tid);
-        if (!FUSED && tid < M) cp_async4(sTok + tid, tok_scale + tid);
+        if (GW == 0 && tid < nb * 16) sRowScale[tid] = __ldcg(row_scale + b0 * 16 + tid);
+        if (bias != nullptr && tid < nb * 8)
+            reinterpret_cast<unsigned*>(sBias)[tid] =
+                __ldcg(reinterpret_cast<const unsigned*>(bias + b0 * 16) + tid);
+        if (!FUSED && tid < M) sTok[tid] = __ldcg(tok_scale + tid);
     }
 
     // fused linear: x -> codes and scales in shared memory, under the first boxes
@@ -236,9 +239,7 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
 
     bool gw_failed = false;
     if constexpr (GW != 0) {
-        int ok = 0;
-        if (lane == 0) ok = mbar_wait_bounded(gw_bar, 0, abort_flag, wait_ns, kDevErrTimeoutConsumer);
-        if (__shfl_sync(0xFFFFFFFFu, ok, 0) == 0) gw_failed = true;
+        if (!warp_wait(gw_bar, 0, abort_flag, wait_ns, kDevErrTimeoutConsumer)) gw_failed = true;
     }
     int consumed = 0, cslot = 0;
     uint32_t cphase = 0u;
@@ -259,7 +260,7 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
                 const int kb = 256 * P + 128 * h + 32 * t;   // K % 32 == 0: a slice is all in or all out
                 if (tok < M && kb < K) {
                     if constexpr (A_INT4) {
-                        const uint4 c = __ldg(reinterpret_cast<const uint4*>(
+                        const uint4 c = __ldcg(reinterpret_cast<const uint4*>(
                             act + static_cast<size_t>(tok) * (K / 2) + kb / 2));
                         const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
@@ -274,8 +275,8 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
                             c1 = lds128(reinterpret_cast<const uint8_t*>(sCodes) + tok * K + kb + 16);
                         } else {
                             const uint4* ar = reinterpret_cast<const uint4*>(act + static_cast<size_t>(tok) * K + kb);
-                            c0 = __ldg(ar);
-                            c1 = __ldg(ar + 1);
+                            c0 = __ldcg(ar);
+                            c1 = __ldcg(ar + 1);
                         }
                         const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
@@ -325,10 +326,10 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
                 }
             }
             const int slot = cslot;
-            int ok = 0;
-            if (lane == 0)
-                ok = mbar_wait_bounded(&full[slot], cphase, abort_flag, wait_ns, kDevErrTimeoutConsumer);
-            if (__shfl_sync(0xFFFFFFFFu, ok, 0) == 0) { aborted = true; break; }
+            if (!warp_wait(&full[slot], cphase, abort_flag, wait_ns, kDevErrTimeoutConsumer)) {
+                aborted = true;
+                break;
+            }
             const uint8_t* box = ring + slot * kS8Box;
 #pragma unroll
             for (int hb = 0; hb < 2; ++hb) {
@@ -419,7 +420,6 @@ w4a8_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint8_t* __r
         uint32_t never = 0u;
         if (threadIdx.x == 0) (void)mbar_wait_bounded(gw_bar, 0, &never, wait_ns, 0u);
     }
-    cp_async_wait_all();
     __syncthreads();
 #pragma unroll
     for (int j = 0; j < kS8MB; ++j) {
