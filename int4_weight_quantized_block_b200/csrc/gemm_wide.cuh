@@ -59,6 +59,11 @@ constexpr int kWdSmem = kWdActStages * kWdAct + kWdWStages * kTmWBytes + kWdOut 
                         kWdBN * 4 + 1024;
 constexpr uint32_t kWdColA = kWdBN;        // A stage s at kWdColA + 32 s
 static_assert(kWdColA + 32 * kWdAStages <= 512, "TMEM budget");
+// each unpack chain takes every other K step, so a weight or A stage must
+// belong to one chain (even stage counts): a chain then waits on its stages'
+// phases in order and a parity wait cannot pass on a phase it skipped
+static_assert(kWdWStages % 2 == 0 && kWdAStages % 2 == 0, "stages of one chain");
+static_assert(kWdActStages <= kWdAStages, "the A-stage barriers also free the activation stages");
 static_assert(kWdSmem <= 227 * 1024, "shared memory budget");
 static_assert(kWdAct % 1024 == 0 && kTmWBytes % 1024 == 0, "swizzled stage alignment");
 

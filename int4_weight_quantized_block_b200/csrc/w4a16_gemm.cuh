@@ -71,6 +71,11 @@ constexpr int kWgSmemBytes =
 constexpr uint32_t kWgColD = 0;                       // the accumulator
 constexpr uint32_t kWgColA = kWgBN;                   // A stage s at kWgColA + 32 s
 static_assert(kWgColA + 32 * kWgAStages <= 512, "TMEM budget");
+// each unpack chain takes every other K step, so a weight or A stage must
+// belong to one chain (even stage counts): a chain then waits on its stages'
+// phases in order and a parity wait cannot pass on a phase it skipped
+static_assert(kWgWStages % 2 == 0 && kWgAStages % 2 == 0, "stages of one chain");
+static_assert(kWgActStages <= kWgAStages, "the A-stage barriers also free the activation stages");
 static_assert(kWgSmemBytes <= 227 * 1024, "shared memory budget");
 static_assert(kWgActBytes % 1024 == 0 && kWgWBytes % 1024 == 0, "stage alignment");
 static_assert(kWgGroup == 2 * kWgBK, "a group is two K steps");
