@@ -29,25 +29,19 @@
 // loads the scale and zero point of its row for the group of its next step
 // while it works on the current one.
 //
-// The pipeline is that of gemm_wide.cuh: the token tiles and the packed
-// weights have rings of their own, and the dequantized weights a ring of 8
-// TMEM stages, so the dequant (the kernel's critical path) runs up to 8 steps
-// ahead of the MMAs and a token stage's round trip is TMA latency and MMAs.
-// Warp roles (19 warps, one persistent CTA per SM, static tile list):
-//   warp 0      token-tile producer (4 stages of 32 KB, refilled when the
-//               MMAs of the step 4 back have completed)
+// Warp roles (18 warps, one persistent CTA per SM, static tile list):
+//   warp 0      TMA producer (4-deep ring of 32 KB token + 4 KB weight stages)
 //   warp 1      TMEM owner; one thread issues tcgen05.mma.kind::f16 (A bf16
-//               from TMEM, B bf16 from shared memory, fp32 D; M 128, N 256,
-//               K 16) and commits each step to its A stage's barrier
-//   warps 2-9   dequant into the 8 TMEM A stages (32 columns each)
+//               from TMEM, B bf16 from shared memory, fp32 D; M 128, N 256, K 16)
+//   warps 2-9   dequant into the 4 TMEM A stages (32 columns each)
 //   warps 10-17 epilogue: tcgen05.ld of the accumulator two 32-token chunks
 //               at a time, handed back to the MMAs after the last read,
 //               rounding to bf16 into a [256 tokens][128 columns] staging
 //               tile, copied to y in 16-byte row pieces.
-//   warp 18     packed-weight producer (4 stages of 4 KB, refilled once read)
 // TMEM columns: one accumulator at 0 (256 columns), A stages at 256 + 32 s.
 // (256 tokens per tile rather than 192 with two accumulators: the dequant
-// work of a step then serves a third more tokens.)
+// work of a step, the kernel's critical path, then serves a third more
+// tokens.)
 #pragma once
 
 #include "ptx.cuh"
@@ -57,25 +51,20 @@ namespace tint4 {
 constexpr int kWgBM = 128;       // weight rows per tile (UMMA M, TMEM lanes)
 constexpr int kWgBN = 256;       // tokens per tile (UMMA N)
 constexpr int kWgBK = 64;        // K values per stage (bf16: 128-byte rows)
-constexpr int kWgActStages = 4;  // token-tile stages in shared memory
-constexpr int kWgWStages = 4;    // packed-weight stages in shared memory
-constexpr int kWgAStages = 8;    // dequantized-weight stages in TMEM
-constexpr int kWgThreads = 608;  // 19 warps
+constexpr int kWgStages = 4;     // shared-memory stages = TMEM A stages
+constexpr int kWgThreads = 576;  // 18 warps
 constexpr int kWgGroup = 128;    // quantization group along K
 constexpr int kWgActBytes = kWgBN * kWgBK * 2;        // 32 KB token tile per stage
 constexpr int kWgWBytes = kWgBM * kWgBK / 2;          // 4 KB packed weights per stage
 constexpr int kWgOutBytes = kWgBN * kWgBM * 2;        // 64 KB bf16 staging tile
-constexpr int kWgBarBytes = 512;
-constexpr int kWgSmemBytes =
-    kWgActStages * kWgActBytes + kWgWStages * kWgWBytes + kWgOutBytes + kWgBarBytes + 1024;
+constexpr int kWgSmemBytes = kWgStages * (kWgActBytes + kWgWBytes) + kWgOutBytes + 256 + 1024;
 constexpr uint32_t kWgColD = 0;                       // the accumulator
 constexpr uint32_t kWgColA = kWgBN;                   // A stage s at kWgColA + 32 s
-static_assert(kWgColA + 32 * kWgAStages <= 512, "TMEM budget");
-// each unpack chain takes every other K step, so a weight or A stage must
-// belong to one chain (even stage counts): a chain then waits on its stages'
-// phases in order and a parity wait cannot pass on a phase it skipped
-static_assert(kWgWStages % 2 == 0 && kWgAStages % 2 == 0, "stages of one chain");
-static_assert(kWgActStages <= kWgAStages, "the A-stage barriers also free the activation stages");
+static_assert(kWgColA + 32 * kWgStages <= 512, "TMEM budget");
+// warps 2-5 take the even K steps and 6-9 the odd ones, so a stage must belong
+// to one chain (an even count): a chain then waits on its stages' phases in
+// order and a parity wait cannot pass on a phase it skipped
+static_assert(kWgStages % 2 == 0, "stages of one chain");
 static_assert(kWgSmemBytes <= 227 * 1024, "shared memory budget");
 static_assert(kWgActBytes % 1024 == 0 && kWgWBytes % 1024 == 0, "stage alignment");
 static_assert(kWgGroup == 2 * kWgBK, "a group is two K steps");
@@ -142,21 +131,17 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* sAct = smem;
-    uint8_t* sW = sAct + kWgActStages * kWgActBytes;
-    uint8_t* sOut = sW + kWgWStages * kWgWBytes;
-    uint64_t* act_full = reinterpret_cast<uint64_t*>(sOut + kWgOutBytes);   // [4] landed (TMA)
-    uint64_t* w_full = act_full + kWgActStages;    // [4] landed (TMA)
-    uint64_t* w_empty = w_full + kWgWStages;       // [4] read by the 4 warps of a chain
-    uint64_t* a_full = w_empty + kWgWStages;       // [8] TMEM A stage written (4 warps)
-    uint64_t* a_empty = a_full + kWgAStages;       // [8] the step's MMAs completed (commit)
-    uint64_t* acc_full = a_empty + kWgAStages;     // accumulator ready (commit)
-    uint64_t* acc_empty = acc_full + 1;            // accumulator read (8 warps)
-    uint64_t* final_bar = acc_empty + 1;           // all MMAs done (teardown)
+    uint8_t* sW = smem + kWgStages * kWgActBytes;
+    uint8_t* sOut = sW + kWgStages * kWgWBytes;
+    uint64_t* act_full = reinterpret_cast<uint64_t*>(sOut + kWgOutBytes);
+    uint64_t* a_full = act_full + kWgStages;       // TMEM A stage written (one arrival per warp)
+    uint64_t* empty = a_full + kWgStages;          // stage consumed by the MMAs (commit)
+    uint64_t* acc_full = empty + kWgStages;        // accumulator ready (commit)
+    uint64_t* acc_empty = acc_full + 2;            // accumulator read (8 warp arrivals)
+    uint64_t* final_bar = acc_empty + 2;           // all MMAs done (teardown)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
     volatile uint32_t* epi_go = tmem_slot + 2;
-    static_assert((2 * kWgActStages + 2 * kWgWStages + 2 * kWgAStages + 3) * 8 + 12 <= kWgBarBytes,
-                  "barrier area");
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -166,20 +151,17 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
     const int KT = K / kWgBK;                      // even: K % 128 == 0
     const int ngroups = K / kWgGroup;
     const int my_tiles = (blockIdx.x < n_work) ? (n_work - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const int total = my_tiles * KT;               // K steps this CTA runs
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kWgActStages; ++s) mbar_init(&act_full[s], 1);
-        for (int s = 0; s < kWgWStages; ++s) {
-            mbar_init(&w_full[s], 1);
-            mbar_init(&w_empty[s], 4);
-        }
-        for (int s = 0; s < kWgAStages; ++s) {
+        for (int s = 0; s < kWgStages; ++s) {
+            mbar_init(&act_full[s], 1);
             mbar_init(&a_full[s], 4);
-            mbar_init(&a_empty[s], 1);
+            mbar_init(&empty[s], 1);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 8);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 8);
+        }
         mbar_init(final_bar, 1);
         *abort_flag = 0u;
         fence_mbarrier_init();
@@ -197,64 +179,35 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
     tcgen05_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    // x (and the weights) may come from the grid launched just before
+    // x may come from the grid launched just before
     grid_dependency_wait();
 
     if (warp == 0) {
-        // ------------------------------------------------ token-tile producer
+        // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            int j = 0, issued = 0;
+            uint32_t c = 0;
+            int issued = 0;
             for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
-                const int m0 = ((blockIdx.x + i * gridDim.x) % m_tiles) * kWgBN;
-                bool ok = true;
-                for (int kt = 0; kt < KT; ++kt, ++j) {
-                    // stage j % 4 is free once the MMAs of step j - 4 have completed
-                    if (j >= kWgActStages &&
-                        !mbar_wait_bounded(&a_empty[(j - kWgActStages) % kWgAStages],
-                                           ((j - kWgActStages) / kWgAStages) & 1, abort_flag,
-                                           wait_ns, kDevErrTimeoutProducer)) {
-                        ok = false;
+                const int tile = blockIdx.x + i * gridDim.x;
+                const int m0 = (tile % m_tiles) * kWgBN;
+                const int n0 = (tile / m_tiles) * kWgBM;
+                for (int kt = 0; kt < KT; ++kt, ++c) {
+                    const int s = c % kWgStages;
+                    const uint32_t ph = (c / kWgStages) & 1;
+                    if (!mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, wait_ns,
+                                           kDevErrTimeoutProducer))
                         break;
-                    }
-                    const int s = j % kWgActStages;
-                    mbar_arrive_expect_tx(&act_full[s], kWgActBytes);
+                    mbar_arrive_expect_tx(&act_full[s], kWgActBytes + kWgWBytes);
                     tma_load_2d(&tmap_x, &act_full[s], sAct + s * kWgActBytes, kt * kWgBK, m0);
+                    tma_load_2d(&tmap_q, &act_full[s], sW + s * kWgWBytes, kt * (kWgBK / 2), n0);
                     ++issued;
                 }
-                if (!ok) break;
             }
             if (*abort_flag) {
                 uint32_t never = 0u;
-                for (int q = issued > kWgActStages ? issued - kWgActStages : 0; q < issued; ++q)
-                    (void)mbar_wait_bounded(&act_full[q % kWgActStages], (q / kWgActStages) & 1,
-                                            &never, wait_ns, 0u);
-            }
-        }
-    } else if (warp == 18) {
-        // ------------------------------------------------ packed-weight producer
-        if (lane == 0) {
-            int j = 0, issued = 0;
-            for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
-                const int n0 = ((blockIdx.x + i * gridDim.x) / m_tiles) * kWgBM;
-                bool ok = true;
-                for (int kt = 0; kt < KT; ++kt, ++j) {
-                    const int s = j % kWgWStages;
-                    // stage s is free once the dequant of step j - 4 has read it
-                    if (!mbar_wait_bounded(&w_empty[s], ((j / kWgWStages) & 1) ^ 1, abort_flag,
-                                           wait_ns, kDevErrTimeoutProducer)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&w_full[s], kWgWBytes);
-                    tma_load_2d(&tmap_q, &w_full[s], sW + s * kWgWBytes, kt * (kWgBK / 2), n0);
-                    ++issued;
-                }
-                if (!ok) break;
-            }
-            if (*abort_flag) {
-                uint32_t never = 0u;
-                for (int q = issued > kWgWStages ? issued - kWgWStages : 0; q < issued; ++q)
-                    (void)mbar_wait_bounded(&w_full[q % kWgWStages], (q / kWgWStages) & 1, &never,
+                const int first = issued > kWgStages ? issued - kWgStages : 0;
+                for (int j = first; j < issued; ++j)
+                    (void)mbar_wait_bounded(&act_full[j % kWgStages], (j / kWgStages) & 1, &never,
                                             wait_ns, 0u);
             }
         }
@@ -266,35 +219,41 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
             // MMA kk of a stage 32 bytes = 2 units further (the address field
             // cannot carry: shared addresses are below 2^18)
             const uint64_t bdesc0 = umma_desc_sw128(smem_u32(sAct));
-            int j = 0;
+            int s = 0;
+            uint32_t ph = 0u;
             bool ok = true;
             for (int i = 0; i < my_tiles && ok; ++i) {
-                if (!mbar_wait_bounded(acc_empty, (i & 1) ^ 1, abort_flag, wait_ns,
+                const int buf = 0;
+                const uint32_t aph = i & 1;
+                if (!mbar_wait_bounded(&acc_empty[buf], aph ^ 1, abort_flag, wait_ns,
                                        kDevErrTimeoutConsumer)) {
                     ok = false;
                     break;
                 }
                 tcgen05_fence_after();
-                for (int kt = 0; kt < KT; ++kt, ++j) {
-                    const int as = j % kWgAStages, s = j % kWgActStages;
-                    // the dequantized weights (usually ready well ahead), then the tokens
-                    if (!mbar_wait_bounded(&a_full[as], (j / kWgAStages) & 1, abort_flag, wait_ns,
-                                           kDevErrTimeoutConsumer) ||
-                        !mbar_wait_bounded(&act_full[s], (j / kWgActStages) & 1, abort_flag,
-                                           wait_ns, kDevErrTimeoutConsumer)) {
+                const uint32_t d_tmem = tmem_base + kWgColD + buf * kWgBN;
+                for (int kt = 0; kt < KT; ++kt) {
+                    // a_full implies the stage has landed: the unpack warps arrive
+                    // on it only after they have seen it (one wait per stage: the
+                    // issuing thread's time per stage is the tensor pipe's budget)
+                    if (!mbar_wait_bounded(&a_full[s], ph, abort_flag, wait_ns,
+                                           kDevErrTimeoutConsumer)) {
                         ok = false;
                         break;
                     }
                     tcgen05_fence_after();
-                    const uint32_t a_tmem = tmem_base + kWgColA + 32 * as;
+                    const uint32_t a_tmem = tmem_base + kWgColA + 32 * s;
                     const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(s * (kWgActBytes >> 4));
 #pragma unroll
                     for (int kk = 0; kk < kWgBK / 16; ++kk)
-                        umma_bf16_ts(tmem_base + kWgColD, a_tmem + 8 * kk, bdesc + 2 * kk, idesc,
-                                     (kt | kk) != 0);
-                    umma_commit(&a_empty[as]);
+                        umma_bf16_ts(d_tmem, a_tmem + 8 * kk, bdesc + 2 * kk, idesc, (kt | kk) != 0);
+                    umma_commit(&empty[s]);
+                    if (++s == kWgStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
-                if (ok) umma_commit(acc_full);
+                if (ok) umma_commit(&acc_full[buf]);
             }
             umma_commit(final_bar);
             uint32_t never = 0u;
@@ -306,6 +265,7 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
         const int q = warp & 3;                 // TMEM lane quarter
         const int r = q * 32 + lane;            // weight row within the tile
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        const int total = my_tiles * KT;
         // a row is 32 bytes (two 16-byte chunks), rows 32 bytes apart: lanes r
         // and r + 4 of a load phase take different chunks first, so the 8
         // lanes of a phase cover the 32 banks once
@@ -319,7 +279,7 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
             uint16_t sb = 0, zb = 0;
             if (n < N) {
                 sb = __ldca(reinterpret_cast<const unsigned short*>(wscale) +
-                            static_cast<size_t>(n) * ngroups + g);
+                           static_cast<size_t>(n) * ngroups + g);
                 zb = __ldca(wzero + static_cast<size_t>(n) * ngroups + g);
             }
             const uint32_t zh = 0x4300u | zb;   // bf16(128 + z)
@@ -332,11 +292,10 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
             zc = zc_next;
             s2 = s2_next;
             if (j + 2 < total) load_sz(j + 2, zc_next, s2_next);   // lands while this step runs
-            const int ws = j % kWgWStages, as = j % kWgAStages;
-            if (!warp_wait(&w_full[ws], (j / kWgWStages) & 1, abort_flag, wait_ns,
-                              kDevErrTimeoutConsumer))
-                break;
-            const uint8_t* row = sW + ws * kWgWBytes + r * 32;
+            const int s = j % kWgStages;
+            const uint32_t ph = (j / kWgStages) & 1;
+            if (!warp_wait(&act_full[s], ph, abort_flag, wait_ns, kDevErrTimeoutConsumer)) break;
+            const uint8_t* row = sW + s * kWgWBytes + r * 32;
             const uint4 p0 = lds128(row + 16 * c0);
             const uint4 p1 = lds128(row + 16 * (c0 ^ 1));
             const uint4 lo = c0 ? p1 : p0, hi = c0 ? p0 : p1;   // K 0..31 / 32..63 of the step
@@ -349,21 +308,14 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
 #pragma unroll
                 for (int p = 0; p < 4; ++p) a[4 * v + p] = o[p];
             }
-            // the packed stage is in registers (the values above depend on every
-            // load): the weight producer may refill it
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&w_empty[ws]);
-            // TMEM stage as is free once the MMAs of step j - 8 have completed
-            if (j >= kWgAStages &&
-                !warp_wait(&a_empty[as], ((j - kWgAStages) / kWgAStages) & 1, abort_flag,
-                              wait_ns, kDevErrTimeoutConsumer))
-                break;
+            // the TMEM A stage is free: its previous MMAs completed before the
+            // producer refilled this stage (empty[s] -> act_full[s])
             tcgen05_fence_after();
-            tmem_st_32x32b_x32(tmem_base + lane_base + kWgColA + 32 * as, a);
+            tmem_st_32x32b_x32(tmem_base + lane_base + kWgColA + 32 * s, a);
             tmem_st_wait();
             tcgen05_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&a_full[as]);
+            if (lane == 0) mbar_arrive(&a_full[s]);
         }
     } else if (warp < 18) {
         // ------------------------------------------------ epilogue (warps 10-17)
@@ -378,7 +330,7 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
             const int m0 = (tile % m_tiles) * kWgBN;
             const int n0 = (tile / m_tiles) * kWgBM;
             if (leader) {
-                const bool ok = mbar_wait_bounded(acc_full, i & 1, abort_flag,
+                const bool ok = mbar_wait_bounded(&acc_full[0], i & 1, abort_flag,
                                                   wait_ns, kDevErrTimeoutEpilogue);
                 *epi_go = ok ? 1u : 0u;
             }
@@ -391,15 +343,15 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
             auto emit = [&](int cc, const uint32_t (&acc)[32]) {
                 const uint32_t dst = smem_u32(sOut + cc * (kWgBM * 2) + r * 2);
 #pragma unroll
-                for (int jj = 0; jj < 32; jj += 2) {
+                for (int j = 0; j < 32; j += 2) {
                     const uint32_t h2 =
-                        f2_to_bf16x2(f2_pack(__uint_as_float(acc[jj]), __uint_as_float(acc[jj + 1])));
+                        f2_to_bf16x2(f2_pack(__uint_as_float(acc[j]), __uint_as_float(acc[j + 1])));
                     asm volatile(
                         "{\n\t.reg .b16 l, h;\n\t"
                         "mov.b32 {l, h}, %2;\n\t"
                         "st.shared.b16 [%0], l;\n\t"
-                        "st.shared.b16 [%1], h;\n\t}" ::"r"(dst + jj * (kWgBM * 2)),
-                        "r"(dst + (jj + 1) * (kWgBM * 2)), "r"(h2)
+                        "st.shared.b16 [%1], h;\n\t}" ::"r"(dst + j * (kWgBM * 2)),
+                        "r"(dst + (j + 1) * (kWgBM * 2)), "r"(h2)
                         : "memory");
                 }
             };
@@ -418,7 +370,7 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                 if (cc + 64 >= cend || m0 + cc + 64 >= M) {   // warp-uniform
                     tcgen05_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(acc_empty);
+                    if (lane == 0) mbar_arrive(&acc_empty[0]);
                     released = true;
                 }
                 emit(cc, acc0);
@@ -427,7 +379,7 @@ w4a16_tmem_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
             if (!released) {   // no token of this warp's half below M
                 tcgen05_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(acc_empty);
+                if (lane == 0) mbar_arrive(&acc_empty[0]);
             }
             named_barrier_sync(1, 256);
             const int et = e * 32 + lane;
